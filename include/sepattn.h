@@ -1,0 +1,202 @@
+/*
+ * sepattn.h -- C ABI of the Sep-Attention / SepCache library (B200, sm_100a).
+ *
+ * Sep-Attention is causal softmax attention in which query i attends to key
+ * j only when j <= i and (j < a, or token j is a separator, or i - j < n).
+ * Definition: "HKUDS047: SepLLM ..." study, section "SepAttention"
+ * (build_prefill_mask: separator columns, initial columns, local triangular
+ * window, AND the lower-triangular causal mask) and the jieyibu.net SepLLM
+ * explainer, section 1.2 (binary mask M; masked scores are -inf before the
+ * softmax).  The four-block KV cache (initial / separator cache capped at s
+ * evicting the oldest / past window that keeps only separators when flushed
+ * / local window w) follows the xugj520 SepLLM article, section 3.3 table,
+ * and the KV-manager steps of the HKUDS047 study, section "KV Cache Manager".
+ *
+ * Conventions shared by every call:
+ *  - All pointers are DEVICE pointers unless a parameter says "host".
+ *    All memory is owned by the caller; no call allocates or frees memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *    Calls only enqueue work on it; none synchronises, except
+ *    sep_device_status() and sepcache_status(), which say so.
+ *  - Return value: SEP_OK (0) or a negative SEP_E* code.  On an error
+ *    return nothing was enqueued.
+ *  - dtype codes: SEP_F32 (fp32) and SEP_BF16 (bfloat16).
+ *  - Layouts are row-major with the last dimension contiguous:
+ *      q, out [B, Hq, S, D];  k, v [B, Hkv, S, D];  lse [B, Hq, S] fp32;
+ *      is_sep [B, S] uint8 in {0,1};  query head h reads kv head
+ *      h / (Hq / Hkv) (contiguous groups).
+ *  - a counts the initial tokens kept (positions 0..a-1); n counts the
+ *    window including the query itself (keys with 0 <= i - j < n).
+ *  - scale <= 0 selects 1/sqrt(D).  lse is the natural log of the softmax
+ *    denominator over the scaled scores.
+ */
+#ifndef SEPATTN_H
+#define SEPATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define SEP_OK 0
+#define SEP_EINVAL (-1)  /* bad size / parameter (also the budget rules below) */
+#define SEP_EDTYPE (-2)  /* unsupported dtype or head_dim for this call */
+#define SEP_EALIGN (-3)  /* a pointer is not 16-byte aligned */
+#define SEP_ECUDA (-4)   /* a CUDA launch or runtime call failed */
+#define SEP_EDEVICE (-5) /* a kernel reported an error in a status word */
+#define SEP_ENULL (-6)   /* a required pointer is NULL */
+
+#define SEP_F32 0
+#define SEP_BF16 1
+
+/* Human-readable name of a status code (static string). */
+const char* sep_strerror(int status);
+
+/* Library ABI version (major * 100 + minor). */
+int sep_version(void);
+
+/* ---------------------------------------------------------------------- */
+/* Separator flags and index lists                                          */
+/* ---------------------------------------------------------------------- */
+
+/* is_sep[t] = 1 iff ids[t] is one of sep_ids[0..n_sep_ids) (HKUDS047 study,
+ * sections "Separator Tokens" and "SepAttention": token_id in
+ * separator_token_ids).  ids: int32 [n_tok]; sep_ids: HOST int32 array,
+ * 1 <= n_sep_ids <= 32; is_sep: uint8 [n_tok].  n_tok = 0 is a no-op. */
+int sep_flags_from_ids(const int32_t* ids, int64_t n_tok, const int32_t* sep_ids, int n_sep_ids,
+                       uint8_t* is_sep, void* stream);
+
+/* Per-sequence prefix-scan compaction of the separator flags (the
+ * separator index lists used to gather separator rows).
+ *   prefix [B, S+1]: prefix[b][j] = number of separators among positions < j
+ *   idx    [B, S]  : positions of the separators of sequence b in increasing
+ *                    order, then -1 up to S
+ *   count  [B]     : prefix[b][S]
+ * B >= 1, S >= 1.  Results are exact integers. */
+int sep_build_index(const uint8_t* is_sep, int B, int S, int32_t* prefix, int32_t* idx,
+                    int32_t* count, void* stream);
+
+/* Kept (query, key) pairs of one head of each sequence (the retention
+ * statistics of the HKUDS047 study, section "Forward Input Wrapper").
+ * prefix: from sep_build_index; kept_pairs: int64 [B]. a >= 0, n >= 1. */
+int sep_count_pairs(const int32_t* prefix, int B, int S, int a, int n, int64_t* kept_pairs,
+                    void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Prefill / training forward                                               */
+/* ---------------------------------------------------------------------- */
+
+/* Workspace bytes sep_attn_prefill needs for these sizes (bf16: room for the
+ * compacted initial+separator K and V rows of every (b, kv head), i.e. two
+ * buffers of k's size, plus 256 bytes; fp32: 256 bytes). */
+size_t sep_attn_prefill_workspace(int B, int Hq, int Hkv, int S, int D, int dtype);
+
+/* Sep-Attention over whole sequences:
+ *   out[b,h,i,:] = sum_{j in K_i} softmax_j(scale * q_i . k_j) v_j,
+ *   K_i = { j <= i : j < a or is_sep[b,j] or i - j < n },
+ *   lse[b,h,i]  = ln sum_{j in K_i} exp(scale * q_i . k_j).
+ * q, k, v, out: dtype elements in the layouts above; lse: fp32 (may be NULL).
+ * is_sep, prefix, idx: the flags and their sep_build_index results.
+ * dtype SEP_BF16 requires D in {64, 128} and runs on tcgen05 tensor cores
+ * (fp32 accumulation); dtype SEP_F32 requires D in {32, 64, 128} and runs
+ * in exact fp32 FMA arithmetic.  Constraints: B, Hq, Hkv, S >= 1,
+ * Hq % Hkv == 0, a >= 0, n >= 1; pointers 16-byte aligned; workspace of at
+ * least sep_attn_prefill_workspace() bytes, 256-byte aligned, contents
+ * arbitrary.  Calls that share a workspace must not overlap on the GPU. */
+int sep_attn_prefill(const void* q, const void* k, const void* v, int dtype, const uint8_t* is_sep,
+                     const int32_t* prefix, const int32_t* idx, int B, int Hq, int Hkv, int S, int D,
+                     int a, int n, float scale, void* out, float* lse, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- */
+/* Streaming decode over the four-block SepCache                            */
+/* ---------------------------------------------------------------------- */
+
+/* Block sizes: a initial tokens, s separator-cache entries, `past` past-
+ * window entries, w local-window entries; capacity c = a + s + past + w
+ * (the KV-manager budget rules of the HKUDS047 study, section "Streaming
+ * parameter constraints": init >= 0, local > 0; SepLLM needs s > 0, and s =
+ * 0 with past = 0 is the StreamingLLM special case). */
+typedef struct {
+  int32_t a, s, past, w;
+} sep_cache_cfg;
+
+/* Cache state.  Every pointer is device memory inside one caller-owned
+ * buffer laid out by sepcache_carve().  Rows of each (layer, b, kv head)
+ * are stored in increasing position order: initial | separator | past |
+ * local, cap = c + 1 rows (one spare row holds the newest token between
+ * sepcache_append and sepcache_compact). */
+typedef struct {
+  void* k;           /* [layers][B][Hkv][cap][D] dtype */
+  void* v;           /* [layers][B][Hkv][cap][D] dtype */
+  int32_t* pos;      /* [B][cap]  token position of each row, -1 when empty */
+  uint8_t* flag;     /* [B][cap]  separator flag of each row */
+  int32_t* counts;   /* [B][4]    rows in blocks I, S, P, L */
+  int32_t* plan;     /* [B][cap+4] this step's slot / flush / move list */
+  int64_t* step;     /* [B]       tokens appended so far */
+  int32_t* status;   /* [1]       0, or SEP_CACHE_E* bits set by a kernel */
+  int32_t layers, B, Hkv, D, dtype, cap;
+  sep_cache_cfg cfg;
+} sepcache;
+
+#define SEP_CACHE_EOVERFLOW 1 /* a step found more rows than the capacity */
+#define SEP_CACHE_ESTATE 2    /* corrupt block counts */
+
+/* Bytes of the single buffer holding a cache (256-byte aligned pieces). */
+size_t sepcache_bytes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype);
+
+/* Fill *cache with pointers into `buffer` (device, >= sepcache_bytes(),
+ * 256-byte aligned) and the sizes.  Host-only; enqueues nothing.
+ * Validation: a >= 0, s >= 0, past >= 0, w >= 1, D in {64, 128},
+ * dtype in {SEP_F32, SEP_BF16}, layers, B, Hkv >= 1. */
+int sepcache_carve(sepcache* cache, void* buffer, size_t bytes, sep_cache_cfg cfg, int layers,
+                   int B, int Hkv, int D, int dtype);
+
+/* Reset to the empty state (no tokens; status 0). */
+int sepcache_init(const sepcache* cache, void* stream);
+
+/* Append one token to every sequence at `layer`: k_new, v_new [B, Hkv, D].
+ * At layer 0 this also advances the shared block bookkeeping by one token
+ * using is_sep_new [B] (uint8): the token joins the initial block while it
+ * holds fewer than a tokens, else the local window, whose oldest token
+ * moves to the past window when it holds more than w; when the past window
+ * then holds more than `past` tokens this step is a flush step (xugj520
+ * article, section 3.3).  is_sep_new is ignored at layers > 0.  Per step:
+ * append(layer 0) must come first, then for every layer append -> compact
+ * -> decode; the next step starts after all layers have been compacted. */
+int sepcache_append(const sepcache* cache, int layer, const void* k_new, const void* v_new,
+                    const uint8_t* is_sep_new, void* stream);
+
+/* Apply this step's flush to `layer` in place: the separators of the past
+ * window join the separator cache, which keeps its newest s entries, the
+ * past window empties and the local window slides down (order-preserving
+ * warp-ballot stream compaction).  A no-op on steps without a flush. */
+int sepcache_compact(const sepcache* cache, int layer, void* stream);
+
+/* Workspace bytes sep_attn_decode needs (split-K partials and counters). */
+size_t sep_attn_decode_workspace(const sepcache* cache, int Hq);
+
+/* Attention of the newest token over the retained rows of `layer`:
+ * q [B, Hq, D] (cache dtype), out [B, Hq, D] (cache dtype), lse [B, Hq]
+ * fp32 (may be NULL).  Hq % Hkv == 0 and Hq / Hkv <= 8.  workspace: at least
+ * sep_attn_decode_workspace() bytes, zero-filled before its first use (the
+ * kernel leaves its counters at zero); calls sharing a workspace must not
+ * overlap on the GPU. */
+int sep_attn_decode(const sepcache* cache, int layer, const void* q, int Hq, float scale, void* out,
+                    float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronise `stream`, copy the cache status word to *host_status (host)
+ * and return SEP_EDEVICE if it is nonzero, SEP_OK otherwise. */
+int sepcache_status(const sepcache* cache, int32_t* host_status, void* stream);
+
+/* Synchronise `stream` and report the library's device-side error bits
+ * (a bounded wait inside a kernel that timed out sets them); clear them when
+ * `clear` is nonzero.  Returns SEP_EDEVICE when any bit was set. */
+int sep_device_status(int32_t* host_bits, int clear, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SEPATTN_H */

@@ -1,0 +1,294 @@
+"""Sep-Attention and the four-block SepCache on B200 (sm_100a).
+
+Thin Python binding of the C ABI in include/sepattn.h (libsepattn.so, built
+in-tree by `python -m streaming_kv_cache_sep_b200.build`).  It only
+marshals arguments: every step of the path runs in the CUDA library.
+PyTorch supplies device memory and the current CUDA stream.  There is no
+CPU fallback: if the library is missing, importing this package fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsepattn.so")
+
+SEP_OK = 0
+SEP_F32 = 0
+SEP_BF16 = 1
+
+# every symbol include/sepattn.h declares
+ABI_SYMBOLS = (
+    "sep_strerror", "sep_version", "sep_flags_from_ids", "sep_build_index", "sep_count_pairs",
+    "sep_attn_prefill_workspace", "sep_attn_prefill", "sepcache_bytes", "sepcache_carve",
+    "sepcache_init", "sepcache_append", "sepcache_compact", "sep_attn_decode_workspace",
+    "sep_attn_decode", "sepcache_status", "sep_device_status",
+)
+
+
+class SepError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        msg = _lib.sep_strerror(status).decode() if _lib is not None else str(status)
+        super().__init__("%s failed: %s (%d)" % (fn, msg, status))
+        self.status = status
+
+
+class SepCacheCfg(ctypes.Structure):
+    _fields_ = [("a", ctypes.c_int32), ("s", ctypes.c_int32), ("past", ctypes.c_int32),
+                ("w", ctypes.c_int32)]
+
+
+class _SepCacheC(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("pos", ctypes.c_void_p),
+                ("flag", ctypes.c_void_p), ("counts", ctypes.c_void_p), ("plan", ctypes.c_void_p),
+                ("step", ctypes.c_void_p), ("status", ctypes.c_void_p), ("layers", ctypes.c_int32),
+                ("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("cap", ctypes.c_int32), ("cfg", SepCacheCfg)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libsepattn.so is not built; run `python -m streaming_kv_cache_sep_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    L.sep_strerror.argtypes = [i32]
+    L.sep_strerror.restype = ctypes.c_char_p
+    L.sep_version.argtypes = []
+    L.sep_flags_from_ids.argtypes = [P, i64, P, i32, P, P]
+    L.sep_build_index.argtypes = [P, i32, i32, P, P, P, P]
+    L.sep_count_pairs.argtypes = [P, i32, i32, i32, i32, P, P]
+    L.sep_attn_prefill_workspace.argtypes = [i32, i32, i32, i32, i32, i32]
+    L.sep_attn_prefill_workspace.restype = sz
+    L.sep_attn_prefill.argtypes = [P, P, P, i32, P, P, P, i32, i32, i32, i32, i32, i32, i32, f32,
+                                   P, P, P, sz, P]
+    L.sepcache_bytes.argtypes = [SepCacheCfg, i32, i32, i32, i32, i32]
+    L.sepcache_bytes.restype = sz
+    L.sepcache_carve.argtypes = [ctypes.POINTER(_SepCacheC), P, sz, SepCacheCfg, i32, i32, i32,
+                                 i32, i32]
+    L.sepcache_init.argtypes = [ctypes.POINTER(_SepCacheC), P]
+    L.sepcache_append.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, P, P, P]
+    L.sepcache_compact.argtypes = [ctypes.POINTER(_SepCacheC), i32, P]
+    L.sep_attn_decode_workspace.argtypes = [ctypes.POINTER(_SepCacheC), i32]
+    L.sep_attn_decode_workspace.restype = sz
+    L.sep_attn_decode.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, i32, f32, P, P, P, sz, P]
+    L.sepcache_status.argtypes = [ctypes.POINTER(_SepCacheC), ctypes.POINTER(ctypes.c_int32), P]
+    L.sep_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32), i32, P]
+    for name in ABI_SYMBOLS:
+        fn = getattr(L, name)
+        if name not in ("sep_strerror", "sep_attn_prefill_workspace", "sepcache_bytes",
+                        "sep_attn_decode_workspace"):
+            fn.restype = ctypes.c_int
+    return L
+
+
+_lib = _load()
+
+
+def lib():
+    """The loaded ctypes handle of libsepattn.so."""
+    return _lib
+
+
+def _check(fn: str, rc: int):
+    if rc != SEP_OK:
+        raise SepError(fn, rc)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return SEP_BF16
+    if t.dtype == torch.float32:
+        return SEP_F32
+    raise TypeError("unsupported dtype %s" % t.dtype)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("expected contiguous CUDA tensors")
+
+
+# ------------------------------------------------------------------ index
+
+
+def flags_from_ids(ids: torch.Tensor, sep_ids, stream=None) -> torch.Tensor:
+    """uint8 flags: 1 where ids is one of sep_ids (a host list, <= 32 ids)."""
+    _need_cuda(ids)
+    assert ids.dtype == torch.int32
+    out = torch.empty(ids.shape, dtype=torch.uint8, device=ids.device)
+    arr = (ctypes.c_int32 * len(sep_ids))(*[int(x) for x in sep_ids])
+    _check("sep_flags_from_ids", _lib.sep_flags_from_ids(
+        _ptr(ids), ids.numel(), ctypes.cast(arr, ctypes.c_void_p), len(sep_ids), _ptr(out),
+        _stream(stream)))
+    return out
+
+
+def build_index(is_sep: torch.Tensor, out=None, stream=None):
+    """(prefix [B,S+1], idx [B,S] (-1 padded), count [B]) int32 on the device."""
+    _need_cuda(is_sep)
+    B, S = is_sep.shape
+    dev = is_sep.device
+    if out is None:
+        out = (torch.empty((B, S + 1), dtype=torch.int32, device=dev),
+               torch.empty((B, S), dtype=torch.int32, device=dev),
+               torch.empty((B,), dtype=torch.int32, device=dev))
+    prefix, idx, count = out
+    _check("sep_build_index", _lib.sep_build_index(_ptr(is_sep), B, S, _ptr(prefix), _ptr(idx),
+                                                   _ptr(count), _stream(stream)))
+    return prefix, idx, count
+
+
+def count_pairs(prefix: torch.Tensor, a: int, n: int, out=None, stream=None) -> torch.Tensor:
+    """Kept (query, key) pairs per sequence for one head, int64 [B]."""
+    _need_cuda(prefix)
+    B, S1 = prefix.shape
+    out = out if out is not None else torch.empty((B,), dtype=torch.int64, device=prefix.device)
+    _check("sep_count_pairs", _lib.sep_count_pairs(_ptr(prefix), B, S1 - 1, a, n, _ptr(out),
+                                                   _stream(stream)))
+    return out
+
+
+# ------------------------------------------------------------------ prefill
+
+
+def prefill_workspace_bytes(B, Hq, Hkv, S, D, dtype) -> int:
+    return int(_lib.sep_attn_prefill_workspace(B, Hq, Hkv, S, D, dtype))
+
+
+def prefill(q, k, v, is_sep, prefix, idx, a: int, n: int, scale: float = 0.0, out=None,
+            lse=None, workspace=None, want_lse: bool = True, stream=None):
+    """Sep-Attention over whole sequences.  q [B,Hq,S,D], k/v [B,Hkv,S,D]
+    (bf16 -> tcgen05 path, fp32 -> exact FMA path).  Returns (out, lse)."""
+    _need_cuda(q, k, v, is_sep, prefix, idx, out, lse, workspace)
+    B, Hq, S, D = q.shape
+    Hkv = k.shape[1]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    need = prefill_workspace_bytes(B, Hq, Hkv, S, D, dt)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    _check("sep_attn_prefill", _lib.sep_attn_prefill(
+        _ptr(q), _ptr(k), _ptr(v), dt, _ptr(is_sep), _ptr(prefix), _ptr(idx), B, Hq, Hkv, S, D,
+        a, n, float(scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+    return out, lse
+
+
+def device_status(clear: bool = True, stream=None) -> int:
+    """Synchronise and return the library's device error bits (0 = none)."""
+    bits = ctypes.c_int32(0)
+    _lib.sep_device_status(ctypes.byref(bits), 1 if clear else 0, _stream(stream))
+    return bits.value
+
+
+# ------------------------------------------------------------------ SepCache
+
+
+class SepCache:
+    """The four-block KV cache of `layers` layers for B sequences, in one
+    device buffer.  Sizes: a initial, s separator, past window, w local."""
+
+    def __init__(self, a: int, s: int, past: int, w: int, layers: int, B: int, Hkv: int, D: int,
+                 dtype=torch.bfloat16, device="cuda", stream=None):
+        self.cfg = SepCacheCfg(a, s, past, w)
+        self.dt = SEP_BF16 if dtype == torch.bfloat16 else SEP_F32
+        nbytes = int(_lib.sepcache_bytes(self.cfg, layers, B, Hkv, D, self.dt))
+        if nbytes == 0:
+            raise SepError("sepcache_bytes", -1)
+        self.buffer = torch.empty((nbytes,), dtype=torch.uint8, device=device)
+        self.c = _SepCacheC()
+        _check("sepcache_carve", _lib.sepcache_carve(ctypes.byref(self.c), _ptr(self.buffer),
+                                                     nbytes, self.cfg, layers, B, Hkv, D, self.dt))
+        self.layers, self.B, self.Hkv, self.D, self.cap = layers, B, Hkv, D, self.c.cap
+        self.dtype = dtype
+        self._ws = {}
+        self.init(stream)
+
+    def _view(self, addr, shape, dtype):
+        base = self.buffer.data_ptr()
+        off = addr - base
+        esz = torch.tensor([], dtype=dtype).element_size()
+        n = 1
+        for d in shape:
+            n *= d
+        return self.buffer[off: off + n * esz].view(dtype).view(*shape)
+
+    # device views of the cache state
+    @property
+    def k(self):
+        return self._view(self.c.k, (self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
+
+    @property
+    def v(self):
+        return self._view(self.c.v, (self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
+
+    @property
+    def pos(self):
+        return self._view(self.c.pos, (self.B, self.cap), torch.int32)
+
+    @property
+    def flag(self):
+        return self._view(self.c.flag, (self.B, self.cap), torch.uint8)
+
+    @property
+    def counts(self):
+        return self._view(self.c.counts, (self.B, 4), torch.int32)
+
+    @property
+    def step(self):
+        return self._view(self.c.step, (self.B,), torch.int64)
+
+    def init(self, stream=None):
+        _check("sepcache_init", _lib.sepcache_init(ctypes.byref(self.c), _stream(stream)))
+
+    def append(self, layer: int, k_new, v_new, is_sep_new=None, stream=None):
+        _need_cuda(k_new, v_new, is_sep_new)
+        _check("sepcache_append", _lib.sepcache_append(
+            ctypes.byref(self.c), layer, _ptr(k_new), _ptr(v_new), _ptr(is_sep_new),
+            _stream(stream)))
+
+    def compact(self, layer: int, stream=None):
+        _check("sepcache_compact", _lib.sepcache_compact(ctypes.byref(self.c), layer,
+                                                         _stream(stream)))
+
+    def workspace(self, Hq: int):
+        ws = self._ws.get(Hq)
+        if ws is None:
+            nbytes = int(_lib.sep_attn_decode_workspace(ctypes.byref(self.c), Hq))
+            ws = torch.zeros((nbytes,), dtype=torch.uint8, device=self.buffer.device)
+            self._ws[Hq] = ws
+        return ws
+
+    def decode(self, layer: int, q, scale: float = 0.0, out=None, lse=None, want_lse=True,
+               stream=None):
+        _need_cuda(q, out, lse)
+        B, Hq, D = q.shape
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        ws = self.workspace(Hq)
+        _check("sep_attn_decode", _lib.sep_attn_decode(
+            ctypes.byref(self.c), layer, _ptr(q), Hq, float(scale), _ptr(out), _ptr(lse),
+            _ptr(ws), ws.numel(), _stream(stream)))
+        return out, lse
+
+    def status(self, stream=None) -> int:
+        v = ctypes.c_int32(0)
+        _lib.sepcache_status(ctypes.byref(self.c), ctypes.byref(v), _stream(stream))
+        return v.value

@@ -1,0 +1,189 @@
+// Separator flags, per-sequence separator index lists, and kept-pair counts.
+//
+// The separator set and the kept rule follow the "HKUDS047: SepLLM ..." study,
+// sections "Separator Tokens" and "SepAttention" (token_id in
+// separator_token_ids; initial + separator + local-window columns AND the
+// causal mask).  The index list is the prefix-scan compaction of the flags
+// that lets the attention kernel fetch separator rows by position.
+#include <string.h>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int kMaxSepIds = 32;
+struct SepIdSet {
+  int32_t id[kMaxSepIds];
+  int n;
+};
+
+__global__ void k_flags_from_ids(const int32_t* __restrict__ ids, int64_t n_tok, SepIdSet set,
+                                 uint8_t* __restrict__ is_sep) {
+  int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (; t < n_tok; t += stride) {
+    int32_t v = ids[t];
+    uint8_t f = 0;
+#pragma unroll 4
+    for (int k = 0; k < set.n; ++k) f |= (v == set.id[k]);
+    is_sep[t] = f;
+  }
+}
+
+// One CTA per (chunk of kChunk positions, sequence).  Each CTA counts the
+// separators before its chunk and in the whole sequence (the flags of a
+// sequence are at most a few hundred KB, read from L2), then scans its own
+// chunk: thread t owns kPer consecutive positions.  No CTA waits on another.
+constexpr int kScanThreads = 1024;
+constexpr int kPer = 16;
+constexpr int kChunk = kScanThreads * kPer;
+
+__device__ __forceinline__ int block_sum_1024(int v, int* red) {
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  int s = 0;
+  if (w == 0) {
+    s = red[l];
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (l == 0) red[32] = s;
+  }
+  __syncthreads();
+  return red[32];
+}
+
+__global__ void __launch_bounds__(kScanThreads) k_build_index(const uint8_t* __restrict__ is_sep,
+                                                              int S, int32_t* __restrict__ prefix,
+                                                              int32_t* __restrict__ idx,
+                                                              int32_t* __restrict__ count) {
+  __shared__ int red[33];
+  __shared__ int wsum[32];
+  const int b = blockIdx.y;
+  const int64_t chunk0 = static_cast<int64_t>(blockIdx.x) * kChunk;
+  const uint8_t* f = is_sep + static_cast<int64_t>(b) * S;
+
+  // separators before the chunk, and in the whole sequence
+  int before = 0, total = 0;
+  for (int64_t p = threadIdx.x; p < S; p += kScanThreads) {
+    int v = f[p];
+    total += v;
+    before += (p < chunk0) ? v : 0;
+  }
+  before = block_sum_1024(before, red);
+  total = block_sum_1024(total, red);
+
+  // local counts of this thread's kPer positions
+  const int64_t p0 = chunk0 + static_cast<int64_t>(threadIdx.x) * kPer;
+  uint32_t bits = 0;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    int64_t p = p0 + e;
+    if (p < S && f[p]) bits |= 1u << e;
+  }
+  int mine = __popc(bits);
+  // exclusive scan of `mine` over the block
+  int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int incl = mine;
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int x = wsum[lane];
+    int xi = x;
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, xi, o);
+      if (lane >= o) xi += y;
+    }
+    wsum[lane] = xi - x;  // exclusive over warps
+  }
+  __syncthreads();
+  int run = before + wsum[warp] + (incl - mine);
+
+  int32_t* pre = prefix + static_cast<int64_t>(b) * (S + 1);
+  int32_t* ix = idx + static_cast<int64_t>(b) * S;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    pre[0] = 0;
+    count[b] = total;
+  }
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) {
+    int64_t p = p0 + e;
+    if (p < S) {
+      if (bits & (1u << e)) {
+        ix[run] = static_cast<int32_t>(p);
+        ++run;
+      }
+      pre[p + 1] = run;
+      // idx slots at or after the total count are padding
+      if (p >= total) ix[p] = -1;
+    }
+  }
+}
+
+// Closed form of one row's kept count: window [lo, i] + initial tokens left
+// of it + separators in [a, lo), lo = max(0, i - n + 1).
+__global__ void k_count_pairs(const int32_t* __restrict__ prefix, int S, int a, int n,
+                              int64_t* __restrict__ kept) {
+  __shared__ long long red[32];
+  const int b = blockIdx.x;
+  const int32_t* pre = prefix + static_cast<int64_t>(b) * (S + 1);
+  const int aa = a < S ? a : S;
+  long long acc = 0;
+  for (int i = threadIdx.x; i < S; i += blockDim.x) {
+    int lo = i - n + 1;
+    if (lo < 0) lo = 0;
+    long long c = static_cast<long long>(i - lo + 1) + (a < lo ? a : lo);
+    if (lo > aa) c += pre[lo] - pre[aa];
+    acc += c;
+  }
+  for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    long long s = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0;
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (threadIdx.x == 0) kept[b] = s;
+  }
+}
+
+}  // namespace
+
+extern "C" int sep_flags_from_ids(const int32_t* ids, int64_t n_tok, const int32_t* sep_ids,
+                                  int n_sep_ids, uint8_t* is_sep, void* stream) {
+  if (n_tok < 0 || n_sep_ids < 1 || n_sep_ids > kMaxSepIds) return SEP_EINVAL;
+  if (!sep_ids) return SEP_ENULL;
+  if (n_tok == 0) return SEP_OK;
+  if (!ids || !is_sep) return SEP_ENULL;
+  SepIdSet set;
+  memset(&set, 0, sizeof set);
+  set.n = n_sep_ids;
+  for (int k = 0; k < n_sep_ids; ++k) set.id[k] = sep_ids[k];
+  int64_t blocks = (n_tok + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k_flags_from_ids<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      ids, n_tok, set, is_sep);
+  return sep::launch_status();
+}
+
+extern "C" int sep_build_index(const uint8_t* is_sep, int B, int S, int32_t* prefix, int32_t* idx,
+                               int32_t* count, void* stream) {
+  if (B < 1 || S < 1 || B > 65535) return SEP_EINVAL;
+  if (!is_sep || !prefix || !idx || !count) return SEP_ENULL;
+  dim3 grid((S + kChunk - 1) / kChunk, B);
+  k_build_index<<<grid, kScanThreads, 0, static_cast<cudaStream_t>(stream)>>>(is_sep, S, prefix,
+                                                                              idx, count);
+  return sep::launch_status();
+}
+
+extern "C" int sep_count_pairs(const int32_t* prefix, int B, int S, int a, int n,
+                               int64_t* kept_pairs, void* stream) {
+  if (B < 1 || S < 1 || a < 0 || n < 1) return SEP_EINVAL;
+  if (!prefix || !kept_pairs) return SEP_ENULL;
+  k_count_pairs<<<B, 1024, 0, static_cast<cudaStream_t>(stream)>>>(prefix, S, a, n, kept_pairs);
+  return sep::launch_status();
+}

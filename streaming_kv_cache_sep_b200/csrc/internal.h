@@ -1,0 +1,15 @@
+// Entry points shared between the library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sep {
+int prefill_f32(const float* q, const float* k, const float* v, const int32_t* prefix,
+                const int32_t* idx, int B, int Hq, int Hkv, int S, int D, int a, int n,
+                float scale, float* out, float* lse, cudaStream_t st);
+size_t prefill_tc_workspace(int B, int Hkv, int S, int D);
+int prefill_tc(const void* q, const void* k, const void* v, const uint8_t* is_sep,
+               const int32_t* prefix, const int32_t* idx, int B, int Hq, int Hkv, int S, int D,
+               int a, int n, float scale, void* out, float* lse, void* workspace, cudaStream_t st);
+}  // namespace sep

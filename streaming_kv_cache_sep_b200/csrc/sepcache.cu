@@ -1,0 +1,328 @@
+// The four-block SepCache: bookkeeping, token append and in-place compaction.
+//
+// Blocks (xugj520 SepLLM article, section 3.3 table; KV-manager steps of the
+// "HKUDS047: SepLLM ..." study, section "KV Cache Manager"):
+//   I  initial cache: the first a tokens, never evicted;
+//   S  separator cache: at most s separator tokens, oldest evicted first;
+//   P  past window: tokens that slid out of the local window; when it holds
+//      more than `past` tokens it is flushed -- its separators join S (which
+//      then keeps its newest s entries) and it empties;
+//   L  local window: the newest w tokens.
+// Rows of each (layer, b, kv head) are stored I | S | P | L in increasing
+// position order.  P and L are one contiguous run of recent positions, so a
+// token sliding from L to P moves no data; only a flush moves rows, and it
+// does so in place with an order-preserving stream compaction (every row
+// moves down or stays, and rows are processed in ascending order).
+//
+// Bookkeeping is shared by all layers: sepcache_append at layer 0 runs the
+// state machine for the new token and records this step's plan (the row the
+// token is written to and, on a flush, the source row of every destination
+// row); every layer's append/compact then applies that plan to its K/V.
+#include <string.h>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int kPlanHdr = 4;  // plan[b] = {flush, slot, new_len, first_moved_row, src[cap]...}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+  uint32_t m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+// One warp per sequence.
+__global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__ flag,
+                                int32_t* __restrict__ counts, int32_t* __restrict__ plan,
+                                int64_t* __restrict__ step, int32_t* __restrict__ status,
+                                const uint8_t* __restrict__ is_sep_new, int B, int cap, int a,
+                                int s, int past, int w) {
+  const int b = blockIdx.x;
+  const int lane = threadIdx.x;
+  if (b >= B) return;
+  int32_t* cnt = counts + 4 * b;
+  int32_t* pl = plan + static_cast<int64_t>(b) * (cap + kPlanHdr);
+  int32_t* ps = pos + static_cast<int64_t>(b) * cap;
+  uint8_t* fl = flag + static_cast<int64_t>(b) * cap;
+  int nI = cnt[0], nS = cnt[1], nP = cnt[2], nL = cnt[3];
+  const int64_t t = step[b];
+  const uint8_t f = is_sep_new[b] ? 1 : 0;
+  int len = nI + nS + nP + nL;
+  const bool bad = nI < 0 || nS < 0 || nP < 0 || nL < 0 || nI > a || nS > s || nP > past ||
+                   nL > w || len > cap - 1 || (nI < a && len != nI);
+  __syncwarp();
+  if (bad) {
+    if (lane == 0) {
+      atomicOr(status, SEP_CACHE_ESTATE);
+      pl[0] = 0;
+      pl[1] = -1;
+      pl[2] = len > cap ? cap : (len < 0 ? 0 : len);
+      pl[3] = 0;
+    }
+    return;
+  }
+  // 1. place the token: initial block while it has room, else local window
+  const int slot = len;
+  if (nI < a) {
+    ++nI;
+  } else {
+    ++nL;
+    if (nL > w) {  // the oldest local token now belongs to the past window
+      --nL;
+      ++nP;
+    }
+  }
+  if (lane == 0) {
+    ps[slot] = static_cast<int32_t>(t);
+    fl[slot] = f;
+  }
+  ++len;
+  __syncwarp();
+  // 2. flush the past window when it overflows
+  const bool flush = nP > past;
+  int new_len = len;
+  if (flush) {
+    const int eS = nI + nS, eP = eS + nP;
+    int ncand = nS;
+    for (int base = eS; base < eP; base += 32) {
+      const int r = base + lane;
+      ncand += __popc(__ballot_sync(0xffffffffu, r < eP && fl[r] != 0));
+    }
+    const int drop = ncand > s ? ncand - s : 0;
+    int rank = 0, dst = nI;
+    for (int base = nI; base < len; base += 32) {
+      const int r = base + lane;
+      const bool valid = r < len;
+      const int32_t my_pos = valid ? ps[r] : -1;
+      const uint8_t my_flag = valid ? fl[r] : 0;
+      const bool is_cand = valid && r < eP && (r < eS || my_flag != 0);
+      const bool is_local = valid && r >= eP;
+      const uint32_t cb = __ballot_sync(0xffffffffu, is_cand);
+      const int my_rank = rank + __popc(cb & lanemask_lt());
+      const bool keep = is_local || (is_cand && my_rank >= drop);
+      const uint32_t kb = __ballot_sync(0xffffffffu, keep);
+      const int d = dst + __popc(kb & lanemask_lt());
+      __syncwarp();  // every read of this chunk happens before any write
+      if (keep) {
+        ps[d] = my_pos;
+        fl[d] = my_flag;
+        pl[kPlanHdr + d] = r;
+      }
+      __syncwarp();
+      rank += __popc(cb);
+      dst += __popc(kb);
+    }
+    new_len = dst;
+    for (int r = new_len + lane; r < len; r += 32) {
+      ps[r] = -1;
+      fl[r] = 0;
+    }
+    nS = ncand < s ? ncand : s;
+    nP = 0;
+    if (new_len != nI + nS + nL && lane == 0) atomicOr(status, SEP_CACHE_ESTATE);
+  }
+  if (lane == 0) {
+    pl[0] = flush ? 1 : 0;
+    pl[1] = slot;
+    pl[2] = new_len;
+    pl[3] = nI;
+    cnt[0] = nI;
+    cnt[1] = nS;
+    cnt[2] = nP;
+    cnt[3] = nL;
+    step[b] = t + 1;
+  }
+}
+
+// Write the new token's K and V rows of one layer at this step's slot.
+__global__ void k_cache_write(uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
+                              const uint8_t* __restrict__ k_new, const uint8_t* __restrict__ v_new,
+                              const int32_t* __restrict__ plan, int layer, int B, int Hkv, int cap,
+                              int row_bytes) {
+  const int b = blockIdx.x;
+  const int slot = plan[static_cast<int64_t>(b) * (cap + kPlanHdr) + 1];
+  if (slot < 0 || slot >= cap) return;
+  const int ch = row_bytes / 16;
+  const int per = Hkv * ch;
+  for (int e = threadIdx.x; e < 2 * per; e += blockDim.x) {
+    const int which = e / per, g = (e % per) / ch, c = e % ch;
+    const int64_t dst = ((static_cast<int64_t>(layer) * B + b) * Hkv + g) * cap + slot;
+    const int64_t src = static_cast<int64_t>(b) * Hkv + g;
+    const uint4 val =
+        reinterpret_cast<const uint4*>((which ? v_new : k_new) + src * row_bytes)[c];
+    reinterpret_cast<uint4*>((which ? vc : kc) + dst * row_bytes)[c] = val;
+  }
+}
+
+// Apply this step's flush to one layer: one CTA per (b, kv head, K|V).
+// Destination row r takes source row plan.src[r] >= r; rows are handled in
+// ascending chunks and each chunk is read completely before it is written,
+// so no source row is overwritten before it is read.
+__global__ void __launch_bounds__(256) k_cache_compact(uint8_t* __restrict__ kc,
+                                                       uint8_t* __restrict__ vc,
+                                                       const int32_t* __restrict__ plan, int layer,
+                                                       int B, int Hkv, int cap, int row_bytes) {
+  const int b = blockIdx.x / (2 * Hkv);
+  const int g = (blockIdx.x / 2) % Hkv;
+  const int which = blockIdx.x & 1;
+  const int32_t* pl = plan + static_cast<int64_t>(b) * (cap + kPlanHdr);
+  if (pl[0] == 0) return;
+  const int new_len = pl[2], first = pl[3];
+  const int ch = row_bytes / 16;
+  const int rows_per = 256 / ch;
+  uint8_t* base = (which ? vc : kc) +
+                  ((static_cast<int64_t>(layer) * B + b) * Hkv + g) * cap * row_bytes;
+  const int rr = threadIdx.x / ch, c = threadIdx.x % ch;
+  for (int r0 = first; r0 < new_len; r0 += rows_per) {
+    const int r = r0 + rr;
+    const bool act = rr < rows_per && r < new_len;
+    int src = r;
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (act) {
+      src = pl[kPlanHdr + r];
+      if (src != r && src > r && src < cap) val = reinterpret_cast<const uint4*>(base + static_cast<int64_t>(src) * row_bytes)[c];
+    }
+    __syncthreads();
+    if (act && src != r && src > r && src < cap)
+      reinterpret_cast<uint4*>(base + static_cast<int64_t>(r) * row_bytes)[c] = val;
+    __syncthreads();
+  }
+}
+
+size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+struct Sizes {
+  size_t k, v, pos, flag, counts, plan, step, status;
+  size_t total() const { return k + v + pos + flag + counts + plan + step + status; }
+};
+
+Sizes sizes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
+  const int64_t cap = static_cast<int64_t>(cfg.a) + cfg.s + cfg.past + cfg.w + 1;
+  Sizes z;
+  z.k = round256(static_cast<size_t>(layers) * B * Hkv * cap * D * sep::elem_bytes(dtype));
+  z.v = z.k;
+  z.pos = round256(static_cast<size_t>(B) * cap * 4);
+  z.flag = round256(static_cast<size_t>(B) * cap);
+  z.counts = round256(static_cast<size_t>(B) * 16);
+  z.plan = round256(static_cast<size_t>(B) * (cap + kPlanHdr) * 4);
+  z.step = round256(static_cast<size_t>(B) * 8);
+  z.status = 256;
+  return z;
+}
+
+bool cfg_ok(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
+  if (cfg.a < 0 || cfg.s < 0 || cfg.past < 0 || cfg.w < 1) return false;
+  if (layers < 1 || B < 1 || Hkv < 1 || B > 65535) return false;
+  if (dtype != SEP_F32 && dtype != SEP_BF16) return false;
+  if (D != 64 && D != 128) return false;
+  const int64_t cap = static_cast<int64_t>(cfg.a) + cfg.s + cfg.past + cfg.w + 1;
+  return cap < (1 << 20);
+}
+
+bool cache_ok(const sepcache* c) {
+  return c && c->k && c->v && c->pos && c->flag && c->counts && c->plan && c->step && c->status &&
+         cfg_ok(c->cfg, c->layers, c->B, c->Hkv, c->D, c->dtype) &&
+         c->cap == c->cfg.a + c->cfg.s + c->cfg.past + c->cfg.w + 1;
+}
+
+}  // namespace
+
+extern "C" size_t sepcache_bytes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
+  if (!cfg_ok(cfg, layers, B, Hkv, D, dtype)) return 0;
+  return sizes(cfg, layers, B, Hkv, D, dtype).total();
+}
+
+extern "C" int sepcache_carve(sepcache* cache, void* buffer, size_t bytes, sep_cache_cfg cfg,
+                              int layers, int B, int Hkv, int D, int dtype) {
+  if (!cache || !buffer) return SEP_ENULL;
+  if (!cfg_ok(cfg, layers, B, Hkv, D, dtype)) {
+    if (dtype != SEP_F32 && dtype != SEP_BF16) return SEP_EDTYPE;
+    if (D != 64 && D != 128) return SEP_EDTYPE;
+    return SEP_EINVAL;
+  }
+  if ((reinterpret_cast<uintptr_t>(buffer) & 255u) != 0) return SEP_EALIGN;
+  const Sizes z = sizes(cfg, layers, B, Hkv, D, dtype);
+  if (bytes < z.total()) return SEP_EINVAL;
+  uint8_t* p = static_cast<uint8_t*>(buffer);
+  memset(cache, 0, sizeof *cache);
+  cache->k = p;
+  p += z.k;
+  cache->v = p;
+  p += z.v;
+  cache->pos = reinterpret_cast<int32_t*>(p);
+  p += z.pos;
+  cache->flag = p;
+  p += z.flag;
+  cache->counts = reinterpret_cast<int32_t*>(p);
+  p += z.counts;
+  cache->plan = reinterpret_cast<int32_t*>(p);
+  p += z.plan;
+  cache->step = reinterpret_cast<int64_t*>(p);
+  p += z.step;
+  cache->status = reinterpret_cast<int32_t*>(p);
+  cache->layers = layers;
+  cache->B = B;
+  cache->Hkv = Hkv;
+  cache->D = D;
+  cache->dtype = dtype;
+  cache->cap = cfg.a + cfg.s + cfg.past + cfg.w + 1;
+  cache->cfg = cfg;
+  return SEP_OK;
+}
+
+extern "C" int sepcache_init(const sepcache* c, void* stream) {
+  if (!cache_ok(c)) return c ? SEP_EINVAL : SEP_ENULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t cap = static_cast<size_t>(c->cap);
+  bool ok = cudaMemsetAsync(c->pos, 0xff, c->B * cap * 4, st) == cudaSuccess &&
+            cudaMemsetAsync(c->flag, 0, c->B * cap, st) == cudaSuccess &&
+            cudaMemsetAsync(c->counts, 0, c->B * 16, st) == cudaSuccess &&
+            cudaMemsetAsync(c->plan, 0, c->B * (cap + kPlanHdr) * 4, st) == cudaSuccess &&
+            cudaMemsetAsync(c->step, 0, c->B * 8, st) == cudaSuccess &&
+            cudaMemsetAsync(c->status, 0, 4, st) == cudaSuccess;
+  return ok ? SEP_OK : SEP_ECUDA;
+}
+
+extern "C" int sepcache_append(const sepcache* c, int layer, const void* k_new, const void* v_new,
+                               const uint8_t* is_sep_new, void* stream) {
+  if (!cache_ok(c)) return c ? SEP_EINVAL : SEP_ENULL;
+  if (layer < 0 || layer >= c->layers) return SEP_EINVAL;
+  if (!k_new || !v_new || (layer == 0 && !is_sep_new)) return SEP_ENULL;
+  if (!sep::aligned16(k_new) || !sep::aligned16(v_new)) return SEP_EALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (layer == 0) {
+    k_cache_advance<<<c->B, 32, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step, c->status,
+                                          is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
+                                          c->cfg.past, c->cfg.w);
+    if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  }
+  const int row_bytes = c->D * sep::elem_bytes(c->dtype);
+  const int threads = 2 * c->Hkv * row_bytes / 16 < 512 ? 2 * c->Hkv * row_bytes / 16 : 512;
+  k_cache_write<<<c->B, (threads + 31) / 32 * 32, 0, st>>>(
+      static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v),
+      static_cast<const uint8_t*>(k_new), static_cast<const uint8_t*>(v_new), c->plan, layer, c->B,
+      c->Hkv, c->cap, row_bytes);
+  return sep::launch_status();
+}
+
+extern "C" int sepcache_compact(const sepcache* c, int layer, void* stream) {
+  if (!cache_ok(c)) return c ? SEP_EINVAL : SEP_ENULL;
+  if (layer < 0 || layer >= c->layers) return SEP_EINVAL;
+  const int row_bytes = c->D * sep::elem_bytes(c->dtype);
+  k_cache_compact<<<c->B * c->Hkv * 2, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), c->plan, layer, c->B, c->Hkv,
+      c->cap, row_bytes);
+  return sep::launch_status();
+}
+
+extern "C" int sepcache_status(const sepcache* c, int32_t* host_status, void* stream) {
+  if (!c || !c->status) return SEP_ENULL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, c->status, 4, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return SEP_ECUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return SEP_ECUDA;
+  if (host_status) *host_status = v;
+  return v ? SEP_EDEVICE : SEP_OK;
+}
