@@ -1,0 +1,627 @@
+#!/usr/bin/env python
+"""Benchmark of the Sep-Attention hot path; prints ONE JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Workloads (synthetic, seeded; see synth.WORKLOADS):
+  prefill_* : one step = separator flags from token ids (when the workload has
+              ids) -> separator index lists -> Sep-Attention prefill over the
+              whole batch.  Metric: TFLOP/s on kept pairs (4*D FLOP per kept
+              (query, key) pair and head).  L2 is flushed (256 MiB write)
+              between timed steps; the flush is outside the timed events.
+  decode_*  : one step = one token for every sequence through all layers:
+              append (layer 0 also advances the block bookkeeping) ->
+              compact -> decode, per layer, replayed as a CUDA graph.
+              Metric: decode tokens/s.  The cache (~1 GB) is far larger than L2.
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (weak
+scaling, no data-path collective); the timing is the max over ranks.
+--impl reference times the CPU oracle on this host's cores instead (the
+reference arm), on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+DEFAULT_WORKLOAD = "prefill_pythia160m_b8h12_s2048_d64_bf16"
+PREFILL_METRIC = "Sep-Attn prefill TFLOP/s on kept pairs"
+DECODE_METRIC = "Sep-Attn decode tokens/s over the four-block SepCache"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            d = json.load(fh)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sust=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed
+
+
+def _dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- prefill
+
+
+class PrefillWorkload:
+    def __init__(self, sl, name, seed):
+        self.sl = sl
+        self.name = name
+        self.cfg = cfg = synth.WORKLOADS[name]
+        inp = synth.prefill_inputs(cfg, seed)
+        self.host = inp
+        self.q, self.k, self.v = inp["q"].cuda(), inp["k"].cuda(), inp["v"].cuda()
+        self.has_ids = "ids" in inp
+        if self.has_ids:
+            self.ids = torch.from_numpy(inp["ids"]).cuda()
+            self.sep_ids = [int(x) for x in inp["sep_ids"]]
+            self.is_sep = torch.empty(self.ids.shape, dtype=torch.uint8, device="cuda")
+        else:
+            self.is_sep = torch.from_numpy(inp["is_sep"]).cuda()
+        B, S = self.is_sep.shape
+        self.B, self.S = B, S
+        self.prefix = torch.empty((B, S + 1), dtype=torch.int32, device="cuda")
+        self.idx = torch.empty((B, S), dtype=torch.int32, device="cuda")
+        self.count = torch.empty((B,), dtype=torch.int32, device="cuda")
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(self.q.shape[:3], dtype=torch.float32, device="cuda")
+        dt = 1 if self.q.dtype == torch.bfloat16 else 0
+        self.ws = torch.empty((sl.prefill_workspace_bytes(B, cfg["Hq"], cfg["Hkv"], S, cfg["D"], dt),),
+                              dtype=torch.uint8, device="cuda")
+        # algorithmic work: 4*D FLOP per kept pair and head
+        flags = torch.from_numpy(inp["is_sep"]).cuda()
+        prefix, _, _ = sl.build_index(flags)
+        kept = int(sl.count_pairs(prefix, cfg["a"], cfg["n"]).sum().item()) * cfg["Hq"]
+        self.kept_pairs = kept
+        self.flops = 4.0 * cfg["D"] * kept
+        self.launches_per_step = (1 if self.has_ids else 0) + 1 + (2 if dt == 1 else 1)
+
+    def front(self):
+        if self.has_ids:
+            self._flags_into()
+        self.sl.build_index(self.is_sep, out=(self.prefix, self.idx, self.count))
+
+    def _flags_into(self):
+        import ctypes
+        arr = (ctypes.c_int32 * len(self.sep_ids))(*self.sep_ids)
+        rc = self.sl.lib().sep_flags_from_ids(
+            ctypes.c_void_p(self.ids.data_ptr()), self.ids.numel(), ctypes.cast(arr, ctypes.c_void_p),
+            len(self.sep_ids), ctypes.c_void_p(self.is_sep.data_ptr()),
+            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        if rc != 0:
+            raise RuntimeError("sep_flags_from_ids failed %d" % rc)
+
+    def attn(self):
+        c = self.cfg
+        self.sl.prefill(self.q, self.k, self.v, self.is_sep, self.prefix, self.idx, c["a"], c["n"],
+                        out=self.out, lse=self.lse, workspace=self.ws)
+
+    def step(self):
+        self.front()
+        self.attn()
+
+
+def bench_prefill(sl, args, world, rank):
+    name = args.workload
+    wl = PrefillWorkload(sl, name, synth.WORKLOAD_SEED[name] + 7919 * rank)
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        flush.zero_()
+        wl.step()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    _barrier(world)
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()  # untimed: evict L2 between steps
+        ev[i][0].record()
+        wl.front()
+        ev[i][1].record()
+        wl.attn()
+        ev[i][2].record()
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(c) for a, b, c in ev]
+    attn_ms = [b.elapsed_time(c) for a, b, c in ev]
+    t_local = sum(step_ms) / 1e3
+    t = _max_over_ranks(t_local, world)
+    value = wl.flops * K * world / t / 1e12
+
+    # end to end through the public API with host buffers: pinned host inputs
+    # -> device, the whole step, output -> pinned host, all inside the events
+    e2e = None
+    if not args.skip_e2e:
+        h = wl.host
+        hq, hk, hv = (x.pin_memory() for x in (h["q"], h["k"], h["v"]))
+        hin = torch.from_numpy(h["ids"]).pin_memory() if wl.has_ids else \
+            torch.from_numpy(h["is_sep"]).pin_memory()
+        hout = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+        hlse = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
+        dq, dk, dv = torch.empty_like(wl.q), torch.empty_like(wl.k), torch.empty_like(wl.v)
+        din = wl.ids if wl.has_ids else wl.is_sep
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            din.copy_(hin, non_blocking=True)
+            wl.front()
+            c = wl.cfg
+            sl.prefill(dq, dk, dv, wl.is_sep, wl.prefix, wl.idx, c["a"], c["n"], out=wl.out,
+                       lse=wl.lse, workspace=wl.ws)
+            hout.copy_(wl.out, non_blocking=True)
+            hlse.copy_(wl.lse, non_blocking=True)
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        Ke = max(3, K // 2)
+        _barrier(world)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(Ke):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        te = _max_over_ranks(s0.elapsed_time(s1) / 1e3, world)
+        bi = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hin))
+        bo = hout.numel() * hout.element_size() + hlse.numel() * 4
+        e2e = {"value": wl.flops * Ke * world / te / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo)}
+
+    pk = _peaks()
+    attn_s = statistics.mean(attn_ms) / 1e3
+    achieved = wl.flops / attn_s / 1e12
+    c = wl.cfg
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16"],
+                "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4), "traffic": None,
+                "kernel": "sep_attn_prefill (separator-row gather + tcgen05 attention)",
+                "peak_source": pk["src"] + " bf16 dense burst"}
+    line = {
+        "metric": PREFILL_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(t / K * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if wl.q.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+        "config": {"workload": name, "B": c["B"], "Hq": c["Hq"], "Hkv": c["Hkv"], "S": c["S"],
+                   "D": c["D"], "a": c["a"], "n": c["n"], "kept_pairs": wl.kept_pairs,
+                   "gflop_per_step": round(wl.flops / 1e9, 4),
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)",
+                   "parallelism": "replica per GPU (weak)"},
+        "roofline": roofline, "e2e": e2e, "clocks": clk,
+        "gpu_launches": wl.launches_per_step * K,
+    }
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        line["cpu_baseline"] = cpu_baseline_prefill(wl, budget_s=args.cpu_seconds)
+    return line
+
+
+def cpu_baseline_prefill(wl, budget_s=10.0):
+    import oracle
+    h, c = wl.host, wl.cfg
+    rows, frac = _sample_rows(c, budget_hint=budget_s)
+    kept = _kept_pairs_rows(h["is_sep"], c, rows)
+    t0 = time.time()
+    reps = 0
+    while True:
+        oracle.prefill_rows(h["q"], h["k"], h["v"], h["is_sep"], c["a"], c["n"], rows=rows)
+        reps += 1
+        if time.time() - t0 >= budget_s:
+            break
+    dt = time.time() - t0
+    return {"value": round(4.0 * c["D"] * kept * reps / dt / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.nthreads(), "kind": "oracle",
+            "sample": "%d of %d query rows (%.3g of the workload), repeated %d times, %.1f s" % (
+                rows.size, c["B"] * c["Hq"] * c["S"], frac, reps, dt)}
+
+
+def _sample_rows(c, budget_hint=10.0):
+    """A deterministic bounded sample of query rows: every row for workloads
+    the oracle finishes in about a second, else an evenly strided subset."""
+    total = c["B"] * c["Hq"] * c["S"]
+    est = 4.0 * c["D"] * total * min(c["S"], c["n"] + 0.1 * c["S"] / 2 + c["a"]) / 1e10  # s, 8 cores
+    stride = 1
+    while est / stride > budget_hint / 4 and stride < total:
+        stride *= 2
+    rows = np.arange(0, total, stride, dtype=np.int64)
+    return rows, rows.size / total
+
+
+def _kept_pairs_rows(flags, c, rows):
+    a, n, S = c["a"], c["n"], c["S"]
+    C = np.concatenate([np.zeros((flags.shape[0], 1), np.int64), np.cumsum(flags, 1)], 1)
+    i = rows % S
+    b = rows // (S * c["Hq"])
+    lo = np.maximum(0, i - n + 1)
+    aa = min(a, S)
+    kept = (i - lo + 1) + np.minimum(a, lo) + np.where(lo > aa, C[b, lo] - C[b, aa], 0)
+    return int(kept.sum())
+
+
+# ---------------------------------------------------------------- decode
+
+
+class DecodeWorkload:
+    RING = 4
+
+    def __init__(self, sl, name, seed):
+        self.sl = sl
+        self.cfg = c = synth.WORKLOADS[name]
+        self.B, self.Hq, self.Hkv, self.D, self.L = c["B"], c["Hq"], c["Hkv"], c["D"], c["layers"]
+        self.cache = sl.SepCache(c["a"], c["s"], c["past"], c["w"], self.L, self.B, self.Hkv, self.D,
+                                 dtype=torch.bfloat16)
+        g = torch.Generator(device="cuda")
+        g.manual_seed(seed)
+        R = self.RING
+        self.q = torch.randn((R, self.L, self.B, self.Hq, self.D), generator=g, device="cuda").bfloat16()
+        self.k = torch.randn((R, self.L, self.B, self.Hkv, self.D), generator=g, device="cuda").bfloat16()
+        self.v = torch.randn((R, self.L, self.B, self.Hkv, self.D), generator=g, device="cuda").bfloat16()
+        self.flags_host = synth.decode_flags(c, seed)
+        self.flags = torch.from_numpy(self.flags_host).cuda()
+        self.flag_buf = torch.zeros((self.B,), dtype=torch.uint8, device="cuda")
+        self.out = torch.empty((self.L, self.B, self.Hq, self.D), dtype=torch.bfloat16, device="cuda")
+        self.lse = torch.empty((self.L, self.B, self.Hq), dtype=torch.float32, device="cuda")
+        self.cache.workspace(self.Hq)
+        self.t = 0
+        self.graphs = None
+
+    def layer_ops(self, r, l):
+        self.cache.append(l, self.k[r, l], self.v[r, l], self.flag_buf if l == 0 else None)
+        self.cache.compact(l)
+        self.cache.decode(l, self.q[r, l], out=self.out[l], lse=self.lse[l])
+
+    def eager_step(self):
+        self.flag_buf.copy_(self.flags[self.t])
+        r = self.t % self.RING
+        for l in range(self.L):
+            self.layer_ops(r, l)
+        self.t += 1
+
+    def capture(self):
+        self.graphs = []
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            for r in range(self.RING):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=s):
+                    for l in range(self.L):
+                        self.layer_ops(r, l)
+                self.graphs.append(g)
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+
+    def graph_step(self):
+        self.flag_buf.copy_(self.flags[self.t])
+        self.graphs[self.t % self.RING].replay()
+        self.t += 1
+
+
+def bench_decode(sl, args, world, rank):
+    name = args.workload
+    c = synth.WORKLOADS[name]
+    wl = DecodeWorkload(sl, name, synth.WORKLOAD_SEED[name] + 7919 * rank)
+    fill = min(1000, c["T"] - args.steps - args.warmup)
+    for _ in range(fill):  # reach the steady-state block sizes (untimed set-up)
+        wl.eager_step()
+    wl.capture()
+    for _ in range(args.warmup):
+        wl.graph_step()
+    torch.cuda.synchronize()
+    K = args.steps
+    assert wl.t + K <= c["T"], "stream too short for the requested steps"
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    _barrier(world)
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(K):
+        wl.graph_step()
+    s1.record()
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk = clocks.stop()
+    t = _max_over_ranks(s0.elapsed_time(s1) / 1e3, world)
+    value = c["B"] * K * world / t
+    # dominant kernel: decode, timed alone over every layer of the current state
+    counts = wl.cache.counts.cpu().numpy()
+    rows = int(counts.sum())
+    kv_bytes = rows * wl.Hkv * wl.D * 2 * 2  # K and V, bf16, every sequence, one layer
+    r = wl.t % wl.RING
+    reps = 20
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        for l in range(wl.L):
+            wl.cache.decode(l, wl.q[r, l], out=wl.out[l], lse=wl.lse[l])
+    torch.cuda.synchronize()
+    d0.record()
+    for _ in range(reps):
+        for l in range(wl.L):
+            wl.cache.decode(l, wl.q[r, l], out=wl.out[l], lse=wl.lse[l])
+    d1.record()
+    torch.cuda.synchronize()
+    dec_s = d0.elapsed_time(d1) / 1e3 / (reps * wl.L)
+    achieved = kv_bytes / dec_s / 1e9
+    pk = _peaks()
+    # e2e: the step with its per-step inputs copied from pinned host memory
+    # (q, k_new, v_new of every layer and the flags) and the outputs read back
+    e2e = None
+    if not args.skip_e2e:
+        hq = wl.q[0].cpu().pin_memory()
+        hk = wl.k[0].cpu().pin_memory()
+        hv = wl.v[0].cpu().pin_memory()
+        hf = torch.from_numpy(wl.flags_host).pin_memory()
+        hout = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+        hlse = torch.empty(wl.lse.shape, dtype=torch.float32).pin_memory()
+        Ke = min(200, c["T"] - wl.t)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(Ke):
+            r = wl.t % wl.RING
+            wl.q[r].copy_(hq, non_blocking=True)
+            wl.k[r].copy_(hk, non_blocking=True)
+            wl.v[r].copy_(hv, non_blocking=True)
+            wl.flag_buf.copy_(hf[wl.t], non_blocking=True)
+            wl.graphs[r].replay()
+            wl.t += 1
+            hout.copy_(wl.out, non_blocking=True)
+            hlse.copy_(wl.lse, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        te = _max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+        bi = (hq.numel() + hk.numel() + hv.numel()) * 2 + wl.B
+        bo = hout.numel() * 2 + hlse.numel() * 4
+        e2e = {"value": round(c["B"] * Ke * world / te, 2), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo)}
+    line = {
+        "metric": DECODE_METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(t / K * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": name, "B": c["B"], "Hq": c["Hq"], "Hkv": c["Hkv"], "D": c["D"],
+                   "layers": c["layers"], "a": c["a"], "s": c["s"], "past": c["past"], "w": c["w"],
+                   "timed_tokens": [wl.t - K, wl.t] if e2e is None else None,
+                   "mean_retained_rows": round(rows / wl.B, 2),
+                   "l2": "working set (~1 GB of cache) far above L2",
+                   "parallelism": "replica per GPU (weak)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": None,
+                     "kernel": "sep_attn_decode", "peak_source": pk["src"] + " HBM copy"},
+        "e2e": e2e, "clocks": clk,
+        "gpu_launches": (3 * wl.L) * K,
+    }
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        line["cpu_baseline"] = cpu_baseline_decode(wl, budget_s=args.cpu_seconds)
+    return line
+
+
+def cpu_baseline_decode(wl, budget_s=10.0):
+    """The oracle's decode path on host cores: the four-block state machine
+    over the token stream (per-token cost) plus fp64 attention of every
+    query head over the retained rows (per-layer cost), combined into
+    tokens/s for all layers."""
+    import oracle
+    c = wl.cfg
+    T0 = 1000
+    flags = wl.flags_host
+    t0 = time.time()
+    sim = oracle.sepcache_simulate(flags[: T0 + 1], c["a"], c["s"], c["past"], c["w"], [T0])
+    state_s = (time.time() - t0) / ((T0 + 1) * wl.B)  # per token and sequence
+    q = wl.q[0, 0].float().cpu()
+    k = wl.k[0, 0].float().cpu()
+    v = wl.v[0, 0].float().cpu()
+    t0 = time.time()
+    reps = 0
+    while True:
+        for b in range(wl.B):
+            n = int(sim["counts"][0, b].sum())
+            kk = k[b].unsqueeze(1).expand(wl.Hkv, n, wl.D).contiguous()
+            vv = v[b].unsqueeze(1).expand(wl.Hkv, n, wl.D).contiguous()
+            oracle.attend(q[b], kk, vv)
+        reps += 1
+        if time.time() - t0 >= budget_s:
+            break
+    attn_s = (time.time() - t0) / (reps * wl.B)  # per layer, token and sequence
+    tok_s = 1.0 / (state_s + wl.L * attn_s)
+    return {"value": round(tok_s, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": "state machine over %d tokens x %d sequences; fp64 attention of all %d heads "
+                      "at token %d, %d repetitions of %d sequences, scaled to %d layers" % (
+                          T0 + 1, wl.B, wl.Hq, T0, reps, wl.B, wl.L)}
+
+
+# ---------------------------------------------------------------- reference arm
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle
+    name = args.workload
+    c = synth.WORKLOADS[name]
+    if c["kind"] != "prefill":
+        wl_cores = oracle.nthreads()
+        return {"impl": "reference", "metric": DECODE_METRIC,
+                "unavailable": "reference arm implemented for prefill workloads only",
+                "cores": wl_cores}
+    inp = synth.prefill_inputs(c, synth.WORKLOAD_SEED[name])
+    rows, frac = _sample_rows(c, budget_hint=4.0)
+    kept = _kept_pairs_rows(inp["is_sep"], c, rows)
+    flops = 4.0 * c["D"] * kept
+    for _ in range(args.warmup):
+        oracle.prefill_rows(inp["q"], inp["k"], inp["v"], inp["is_sep"], c["a"], c["n"], rows=rows)
+    t0 = time.time()
+    for _ in range(args.steps):
+        oracle.prefill_rows(inp["q"], inp["k"], inp["v"], inp["is_sep"], c["a"], c["n"], rows=rows)
+    dt = time.time() - t0
+    value = flops * args.steps / dt / 1e12
+    sample = "%d of %d query rows (%.3g of the workload) per step" % (
+        rows.size, c["B"] * c["Hq"] * c["S"], frac)
+    return {"impl": "reference", "metric": PREFILL_METRIC, "value": round(value, 6),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name, "B": c["B"], "Hq": c["Hq"], "Hkv": c["Hkv"], "S": c["S"],
+                       "D": c["D"], "a": c["a"], "n": c["n"]},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                             "cores": oracle.nthreads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--skip-cpu", action="store_true", help="omit the cpu_baseline leg")
+    ap.add_argument("--skip-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    kind = synth.WORKLOADS[args.workload]["kind"]
+    if args.steps is None:
+        args.steps = 50 if kind == "prefill" else 2000
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        line = run_reference(args, world, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    world, rank, _ = _dist_setup(args.gpus)
+    import streaming_kv_cache_sep_b200 as sl
+    if kind == "prefill":
+        line = bench_prefill(sl, args, world, rank)
+    else:
+        line = bench_decode(sl, args, world, rank)
+    status = sl.device_status()
+    if status != 0:
+        raise RuntimeError("device error bits set: %d" % status)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
