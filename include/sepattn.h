@@ -47,6 +47,7 @@ extern "C" {
 #define SEP_ECUDA (-4)   /* a CUDA launch or runtime call failed */
 #define SEP_EDEVICE (-5) /* a kernel reported an error in a status word */
 #define SEP_ENULL (-6)   /* a required pointer is NULL */
+#define SEP_ETOOBIG (-7) /* sizes exceed the fixed scratch of sep_attn_decode_noalloc */
 
 #define SEP_F32 0
 #define SEP_BF16 1
@@ -186,6 +187,25 @@ size_t sep_attn_decode_workspace(const sepcache* cache, int Hq);
  * overlap on the GPU. */
 int sep_attn_decode(const sepcache* cache, int layer, const void* q, int Hq, float scale, void* out,
                     float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Decode for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is a library convenience.  Some callers cannot pass a
+ * workspace -- a plug-in that a host framework calls with only the tensors
+ * of the call (the framework owns every device allocation), or a serving
+ * loop whose device memory is fully reserved for its KV pool, where a new
+ * cudaMalloc would fail or stall the device.  Same arguments and result as
+ * sep_attn_decode, without the workspace: the split-K partials and tickets
+ * live in a fixed scratch array inside the library (about 4.1 MiB, held by
+ * every GPU that loads the library until the process exits).
+ * Limits: B * Hq * ceil((a+s+past+w+1) / 64) <= 8192 and B * Hkv <= 4096;
+ * larger sizes return SEP_ETOOBIG before anything is enqueued.
+ * The first call on a device looks up the array's device address (with
+ * that device current); make that first call before any stream capture.
+ * Each call clears the tickets on `stream` before its kernel and calls no
+ * allocating routine.  All calls share the array, so calls that overlap on
+ * the GPU (other streams, other threads) race on it. */
+int sep_attn_decode_noalloc(const sepcache* cache, int layer, const void* q, int Hq, float scale,
+                            void* out, float* lse, void* stream);
 
 /* Synchronise `stream`, copy the cache status word to *host_status (host)
  * and return SEP_EDEVICE if it is nonzero, SEP_OK otherwise. */

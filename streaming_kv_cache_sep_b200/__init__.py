@@ -1,7 +1,7 @@
 """Sep-Attention and the four-block SepCache on B200 (sm_100a).
 
 Thin Python binding of the C ABI in include/sepattn.h (libsepattn.so, built
-in-tree by `python -m streaming_kv_cache_sep_b200.build`).  It only
+in-tree by `python streaming_kv_cache_sep_b200/build.py`).  It only
 marshals arguments: every step of the path runs in the CUDA library.
 PyTorch supplies device memory and the current CUDA stream.  There is no
 CPU fallback: if the library is missing, importing this package fails.
@@ -25,7 +25,7 @@ ABI_SYMBOLS = (
     "sep_strerror", "sep_version", "sep_flags_from_ids", "sep_build_index", "sep_count_pairs",
     "sep_attn_prefill_workspace", "sep_attn_prefill", "sepcache_bytes", "sepcache_carve",
     "sepcache_init", "sepcache_append", "sepcache_compact", "sep_attn_decode_workspace",
-    "sep_attn_decode", "sepcache_status", "sep_device_status",
+    "sep_attn_decode", "sepcache_status", "sep_device_status", "sep_attn_decode_noalloc",
 )
 
 
@@ -51,7 +51,7 @@ class _SepCacheC(ctypes.Structure):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libsepattn.so is not built; run `python -m streaming_kv_cache_sep_b200.build`")
+        raise ImportError("libsepattn.so is not built; run `python streaming_kv_cache_sep_b200/build.py`")
     L = ctypes.CDLL(LIB_PATH)
     P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
     L.sep_strerror.argtypes = [i32]
@@ -74,6 +74,7 @@ def _load():
     L.sep_attn_decode_workspace.argtypes = [ctypes.POINTER(_SepCacheC), i32]
     L.sep_attn_decode_workspace.restype = sz
     L.sep_attn_decode.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, i32, f32, P, P, P, sz, P]
+    L.sep_attn_decode_noalloc.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, i32, f32, P, P, P]
     L.sepcache_status.argtypes = [ctypes.POINTER(_SepCacheC), ctypes.POINTER(ctypes.c_int32), P]
     L.sep_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32), i32, P]
     for name in ABI_SYMBOLS:
@@ -286,6 +287,21 @@ class SepCache:
         _check("sep_attn_decode", _lib.sep_attn_decode(
             ctypes.byref(self.c), layer, _ptr(q), Hq, float(scale), _ptr(out), _ptr(lse),
             _ptr(ws), ws.numel(), _stream(stream)))
+        return out, lse
+
+    def decode_noalloc(self, layer: int, q, scale: float = 0.0, out=None, lse=None,
+                       want_lse=True, stream=None):
+        """decode() for callers that cannot allocate: no workspace; the
+        library's fixed scratch holds the partials (see the header)."""
+        _need_cuda(q, out, lse)
+        B, Hq, D = q.shape
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        _check("sep_attn_decode_noalloc", _lib.sep_attn_decode_noalloc(
+            ctypes.byref(self.c), layer, _ptr(q), Hq, float(scale), _ptr(out), _ptr(lse),
+            _stream(stream)))
         return out, lse
 
     def status(self, stream=None) -> int:

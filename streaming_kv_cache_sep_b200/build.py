@@ -1,6 +1,6 @@
 """Build the CUDA library libsepattn.so in-tree (sm_100a only).
 
-    python -m streaming_kv_cache_sep_b200.build [--verbose-ptxas]
+    python streaming_kv_cache_sep_b200/build.py [--verbose-ptxas]
 
 Every .cu file under csrc/ is compiled with nvcc for sm_100a (objects are
 cached under _build/ by source timestamp) and linked into

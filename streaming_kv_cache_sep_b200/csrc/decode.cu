@@ -323,3 +323,83 @@ extern "C" int sep_attn_decode(const sepcache* c, int layer, const void* q, int 
     return c->D == 64 ? launch_g<__nv_bfloat16, 64>(p, G, st) : launch_g<__nv_bfloat16, 128>(p, G, st);
   return c->D == 64 ? launch_g<float, 64>(p, G, st) : launch_g<float, 128>(p, G, st);
 }
+
+// ---------------------------------------------------------------------------
+// Decode for callers that cannot allocate device memory.
+//
+// Some callers cannot hand this library a workspace: a plug-in that a host
+// framework calls with only the tensors of the call (the framework owns
+// every device allocation), or a serving loop whose device memory is fully
+// reserved for its KV pool, where a new cudaMalloc would fail or stall the
+// device.  This entry point keeps the split-K partials and tickets in a
+// fixed scratch array inside the library instead.  Every GPU that loads the
+// library holds the array (about 4.1 MiB) until the process exits; every
+// call shares it, so calls that overlap on the GPU race on it.
+namespace {
+
+constexpr int kNoAllocMaxPartials = 8192;  // B * Hq * splits, splits = ceil(cap / 64)
+constexpr int kNoAllocMaxTickets = 4096;   // B * Hkv
+constexpr size_t kNoAllocMlBytes = static_cast<size_t>(kNoAllocMaxPartials) * 2 * 4;
+constexpr size_t kNoAllocOBytes = static_cast<size_t>(kNoAllocMaxPartials) * 128 * 4;
+constexpr size_t kNoAllocTicketBytes = static_cast<size_t>(kNoAllocMaxTickets) * 4;
+constexpr size_t kNoAllocBytes = kNoAllocMlBytes + kNoAllocOBytes + kNoAllocTicketBytes;
+
+__device__ __align__(256) uint8_t g_decode_scratch[kNoAllocBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+uint8_t* g_decode_scratch_addr[kNoAllocMaxDevices];  // device address, per device
+
+}  // namespace
+
+extern "C" int sep_attn_decode_noalloc(const sepcache* c, int layer, const void* q, int Hq,
+                                       float scale, void* out, float* lse, void* stream) {
+  if (!c) return SEP_ENULL;
+  if (!cache_ok(c)) return SEP_EINVAL;
+  if (layer < 0 || layer >= c->layers) return SEP_EINVAL;
+  if (Hq < 1 || Hq % c->Hkv != 0) return SEP_EINVAL;
+  const int G = Hq / c->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SEP_EINVAL;
+  if (!q || !out) return SEP_ENULL;
+  if (!sep::aligned16(q) || !sep::aligned16(out)) return SEP_EALIGN;
+  const int nsplit = (c->cap + ROWS - 1) / ROWS;
+  if (static_cast<int64_t>(c->B) * Hq * nsplit > kNoAllocMaxPartials ||
+      static_cast<int64_t>(c->B) * c->Hkv > kNoAllocMaxTickets)
+    return SEP_ETOOBIG;
+  // set-up, once per device with that device current: the device address of
+  // the scratch array (the host-side symbol itself is not a device address)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return SEP_ECUDA;
+  if (!g_decode_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return SEP_ECUDA;
+    g_decode_scratch_addr[dev] = static_cast<uint8_t*>(p);
+  }
+  uint8_t* scratch = g_decode_scratch_addr[dev];
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int32_t* tickets = reinterpret_cast<int32_t*>(scratch + kNoAllocMlBytes + kNoAllocOBytes);
+  // the tickets must start at zero (the array keeps the previous call's contents)
+  if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(c->B) * c->Hkv * 4, st) != cudaSuccess)
+    return SEP_ECUDA;
+  DecodeParams p;
+  p.q = q;
+  p.kc = c->k;
+  p.vc = c->v;
+  p.counts = c->counts;
+  p.out = out;
+  p.lse = lse;
+  p.part_ml = reinterpret_cast<float*>(scratch);
+  p.part_o = reinterpret_cast<float*>(scratch + kNoAllocMlBytes);
+  p.ticket = tickets;
+  p.err = sep::device_error_word();
+  p.layer = layer;
+  p.B = c->B;
+  p.Hq = Hq;
+  p.Hkv = c->Hkv;
+  p.cap = c->cap;
+  p.nsplit = nsplit;
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(c->D));
+  p.scale_log2 = sc * 1.44269504088896340736f;
+  if (c->dtype == SEP_BF16)
+    return c->D == 64 ? launch_g<__nv_bfloat16, 64>(p, G, st) : launch_g<__nv_bfloat16, 128>(p, G, st);
+  return c->D == 64 ? launch_g<float, 64>(p, G, st) : launch_g<float, 128>(p, G, st);
+}

@@ -33,6 +33,7 @@ extern "C" const char* sep_strerror(int status) {
     case SEP_ECUDA: return "CUDA launch or runtime error";
     case SEP_EDEVICE: return "a kernel reported an error";
     case SEP_ENULL: return "required pointer is NULL";
+    case SEP_ETOOBIG: return "sizes exceed the no-allocation decode scratch";
     default: return "unknown status";
   }
 }
