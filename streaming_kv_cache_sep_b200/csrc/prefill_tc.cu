@@ -5,27 +5,32 @@
 //   out_i = sum_{j in K_i} softmax(scale * q_i . k_j) v_j,
 //   K_i = { j <= i : j < a  or  is_sep[j]  or  i - j < n }.
 //
-// How.  A CTA owns one (batch b, query head h, tile of 128 query rows
-// [q0, q0+128)).  With lo = max(0, q0 - n + 1) every kept key of every row
-// of the tile lies in one of two sets:
-//   * the gathered set: initial tokens [0, min(a, lo)) and the separators in
-//     [a, lo).  These are kept by every row of the tile, so their blocks need
+// Key sets of a 128-row tile [q0, q0+128), with lo = max(0, q0 - n + 1):
+//   * the gathered set -- initial tokens [0, min(a, lo)) and separators in
+//     [a, lo).  Every row of the tile keeps all of them, so their blocks need
 //     no element mask.  A small kernel first copies, per (b, kv head), the
-//     K/V rows of the initial tokens followed by all separators at positions
-//     >= a into a contiguous workspace buffer; the gathered set of any tile is
-//     then a prefix of that buffer, and is loaded with plain TMA tiles.
-//   * the window range [lo, q0 + 128), loaded contiguously from K/V.  Its
-//     blocks carry the element mask  j <= i and (i - j < n or is_sep[j] or
-//     j < a), which handles separators that sit inside some rows' windows.
-// Each key of K_i is therefore scored exactly once.
+//     K/V rows of the initial tokens followed by every separator at a
+//     position >= a into a contiguous workspace buffer; the gathered set of
+//     any tile is then a prefix of that list, loaded with plain TMA tiles.
+//   * the window range [lo, q0 + 128), loaded contiguously from K/V, with the
+//     element mask  j >= lo, j <= i and (i - j < n or is_sep[j] or j < a).
+// Each key of K_i is scored exactly once.
 //
-// Warp roles (192 threads): warps 0-3 run the softmax, one thread per query
-// row (TMEM lane = row); warp 4 issues TMA loads; warp 5 owns TMEM and issues
-// the tcgen05.mma instructions.  S = Q K^T goes to one of two 128-column TMEM
-// buffers, so the MMA for block j+1 overlaps the softmax of block j.  P is
-// rounded to bf16 into a 128-byte-swizzled shared tile and O += P V
-// accumulates in TMEM.  The running maximum is only moved (and O rescaled)
-// when it grows by more than 2^8, so P stays <= 256.
+// Work item = two 128-row tiles that share one key stream:
+//   * GQA (an even number of query heads per kv head): the same rows of two
+//     query heads of one group -- identical key sets;
+//   * otherwise: rows [q0, q0+128) and [q0+128, q0+256) of one head -- the
+//     stream is the union (the larger gathered prefix and the window range
+//     from the first tile's lo); per-tile masks keep each tile's own set.
+// The kernel is persistent (one CTA per SM, items heaviest first, strided
+// over the grid).  Warps 0-3 and 4-7 are the softmax warpgroups of tiles A
+// and B (thread = query row = TMEM lane), warp 8 issues TMA loads, warp 9
+// owns TMEM and issues tcgen05.mma.  TMEM: S_A | S_B | O_A | O_B; each tile's
+// P (bf16) is written over the first 64 columns of its S and feeds the PV
+// MMA from TMEM.  While one warpgroup runs its softmax the tensor core works
+// on the other tile, and the next item's Q/K/V loads overlap the current
+// item's tail.  The running maximum moves (and O is rescaled) only when it
+// grows by more than 2^8, so P stays <= 256.
 #include <string.h>
 
 #include "common.cuh"
@@ -34,33 +39,34 @@ namespace {
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per block
-constexpr int NST = 2;   // K/V shared-memory stages
-constexpr int kThreads = 192;
-constexpr int kTmaWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr uint32_t kTmemCols = 512;  // S0 | S1 | O
+constexpr int kThreads = 320;
+constexpr int kTmaWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
-struct Layout {
+struct Cfg {
+  static constexpr int NST = D == 64 ? 4 : 2;  // K/V shared-memory stages
   static constexpr int REG = 128 * 128;        // one 64-column region of a 128-row tile
   static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;  // one K (or V) stage
-  static constexpr int P_BYTES = BM * BN * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int KV_BYTES = BN * D * 2;
+  static constexpr int OFF_QA = 0;
+  static constexpr int OFF_QB = OFF_QA + Q_BYTES;
+  static constexpr int OFF_K = OFF_QB + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int BYTES = OFF_BAR + 256;
-  // +1024 slack for 1024-byte alignment; at least 120 KB so that one CTA
-  // (which owns all 512 TMEM columns) runs per SM
-  static constexpr int ALLOC = BYTES + 1024 > 120 * 1024 ? BYTES + 1024 : 120 * 1024;
+  static constexpr int OFF_BAR = OFF_V + NST * KV_BYTES;
+  static constexpr int BYTES = OFF_BAR + 512;
+  static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
+  static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
 };
 
+template <int NST>
 struct Bars {
+  uint64_t q_full, q_empty;
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
-  uint64_t s_full[2], p_full, o_done, drain;
+  uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -68,20 +74,66 @@ struct Bars {
 struct Params {
   const uint8_t* is_sep;
   const int32_t* prefix;
-  int B, Hq, Hkv, S, a, n, G, ntiles;
+  int B, Hq, Hkv, S, a, n, G;
+  int pair_heads;  // 1: the two tiles are two heads of a group; 0: two row tiles of one head
+  int npairs, ntiles_item, n_items;
   float scale_log2;
   __nv_bfloat16* out;
   float* lse;
   int32_t* err;
 };
 
+// Geometry of one work item, computed identically by every role.
+struct Item {
+  int b, g;
+  int h[2];    // query head of tile A / B
+  int q0[2];   // first row of tile A / B
+  int lo[2];   // window start of tile A / B
+  int nG[2];   // gathered keys of tile A / B (a prefix of the compact list)
+  int win_lo;  // window range streamed: [win_lo, win_hi)
+  int win_hi;
+  int nblk_g, nblk;
+};
+
+__device__ __forceinline__ Item make_item(const Params& p, int item) {
+  Item it;
+  const int per_tile = p.B * p.npairs;
+  const int qt = p.ntiles_item - 1 - item / per_tile;  // heaviest (last) tiles first
+  const int rem = item % per_tile;
+  it.b = rem / p.npairs;
+  const int pr = rem % p.npairs;
+  if (p.pair_heads) {
+    it.h[0] = 2 * pr;
+    it.h[1] = 2 * pr + 1;
+    it.q0[0] = it.q0[1] = qt * BM;
+  } else {
+    it.h[0] = it.h[1] = pr;
+    it.q0[0] = qt * 2 * BM;
+    it.q0[1] = qt * 2 * BM + BM;
+  }
+  it.g = it.h[0] / p.G;
+  const int32_t* pre = p.prefix + static_cast<int64_t>(it.b) * (p.S + 1);
+  const int aa = p.a < p.S ? p.a : p.S;
+  for (int t = 0; t < 2; ++t) {
+    const int q0 = it.q0[t] < p.S ? it.q0[t] : p.S - 1;
+    const int lo = q0 - p.n + 1 > 0 ? q0 - p.n + 1 : 0;
+    it.lo[t] = lo;
+    it.nG[t] = (p.a < lo ? p.a : lo) + (lo > aa ? pre[lo] - pre[aa] : 0);
+  }
+  const int nG_all = it.nG[0] > it.nG[1] ? it.nG[0] : it.nG[1];
+  it.win_lo = it.lo[0] < it.lo[1] ? it.lo[0] : it.lo[1];
+  const int hi = (it.q0[0] > it.q0[1] ? it.q0[0] : it.q0[1]) + BM;
+  it.win_hi = hi < p.S ? hi : p.S;
+  it.nblk_g = (nG_all + BN - 1) / BN;
+  it.nblk = it.nblk_g + (it.win_hi - it.win_lo + BN - 1) / BN;
+  return it;
+}
+
 // mask of bit positions c in [0, 32) with c <= x
 __device__ __forceinline__ uint32_t bits_le(int x) {
   return x < 0 ? 0u : (x >= 31 ? 0xffffffffu : (0xffffffffu >> (31 - x)));
 }
 
-// Wait without the abort short-cut (used only to drain in-flight copies or
-// MMAs before the CTA exits after an abort).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   int dummy = 0;
   sep::mbar_wait(bar, parity, &dummy, nullptr);
@@ -92,42 +144,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_prefill_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
                  const __grid_constant__ CUtensorMap tm_vc, const Params p) {
-  using L = Layout<D>;
+  using C = Cfg<D>;
+  constexpr int NST = C::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  Bars* bars = reinterpret_cast<Bars*>(smem + L::OFF_BAR);
+  Bars<NST>* bars = reinterpret_cast<Bars<NST>*>(smem + C::OFF_BAR);
   volatile int* abort = &bars->abort;
-
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = p.ntiles - 1 - static_cast<int>(blockIdx.x);  // heaviest tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int g = h / p.G;
-  const int S = p.S;
-  const int q0 = qt * BM;
-  const int q1 = q0 + BM < S ? q0 + BM : S;
-  const int lo = q0 - p.n + 1 > 0 ? q0 - p.n + 1 : 0;
-  const int32_t* pre = p.prefix + static_cast<int64_t>(b) * (S + 1);
-  const int aa = p.a < S ? p.a : S;
-  const int n_init = p.a < lo ? p.a : lo;
-  const int n_sep = lo > aa ? pre[lo] - pre[aa] : 0;
-  const int nG = n_init + n_sep;                 // gathered keys (prefix of the compact buffer)
-  const int nblk_g = (nG + BN - 1) / BN;
-  const int nblk_w = (q1 - lo + BN - 1) / BN;
-  const int nblk = nblk_g + nblk_w;
-  const int64_t kv_row0 = static_cast<int64_t>(b * p.Hkv + g) * S;  // row of key 0 in K/V/Kc/Vc
 
   if (threadIdx.x == 0) {
+    sep::mbar_init(&bars->q_full, 1);
+    sep::mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < NST; ++s) {
       sep::mbar_init(&bars->k_full[s], 1);
       sep::mbar_init(&bars->k_empty[s], 1);
       sep::mbar_init(&bars->v_full[s], 1);
       sep::mbar_init(&bars->v_empty[s], 1);
     }
-    sep::mbar_init(&bars->s_full[0], 1);
-    sep::mbar_init(&bars->s_full[1], 1);
-    sep::mbar_init(&bars->p_full, 128);
-    sep::mbar_init(&bars->o_done, 1);
+    for (int t = 0; t < 2; ++t) {
+      sep::mbar_init(&bars->s_full[t], 1);
+      sep::mbar_init(&bars->p_full[t], 128);
+      sep::mbar_init(&bars->o_full[t], 1);
+      sep::mbar_init(&bars->o_empty[t], 128);
+    }
     sep::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     sep::mbar_fence_init();
@@ -149,44 +189,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       sep::tma_prefetch_desc(&tm_v);
       sep::tma_prefetch_desc(&tm_kc);
       sep::tma_prefetch_desc(&tm_vc);
-      int last_k[NST], last_v[NST];  // last block loaded into each stage
+      uint32_t gblk = 0, nitem = 0;
+      int last_k[NST], last_v[NST];
       for (int s2 = 0; s2 < NST; ++s2) last_k[s2] = last_v[s2] = -1;
-      for (int j = 0; j < nblk; ++j) {
-        const int st = j % NST;
-        const uint32_t use = j / NST;
-        const bool gathered = j < nblk_g;
-        const CUtensorMap* mk = gathered ? &tm_kc : &tm_k;
-        const CUtensorMap* mv = gathered ? &tm_vc : &tm_v;
-        const int64_t row = kv_row0 + (gathered ? static_cast<int64_t>(j) * BN
-                                                : lo + static_cast<int64_t>(j - nblk_g) * BN);
-        if (j >= NST && !sep::mbar_wait(&bars->k_empty[st], (use - 1) & 1, abort, p.err)) break;
-        uint8_t* sk = smem + L::OFF_K + st * L::KV_BYTES;
-        if (j == 0) {
-          sep::mbar_arrive_expect_tx(&bars->k_full[0], L::KV_BYTES + L::Q_BYTES);
-          const int64_t qrow = static_cast<int64_t>(b * p.Hq + h) * S + q0;
+      int last_q = -1;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
+        const Item it = make_item(p, item);
+        const int64_t kv_row0 = static_cast<int64_t>(it.b * p.Hkv + it.g) * p.S;
+        if (nitem > 0 && !sep::mbar_wait(&bars->q_empty, (nitem - 1) & 1, abort, p.err)) break;
+        sep::mbar_arrive_expect_tx(&bars->q_full, 2 * C::Q_BYTES);
+        for (int t = 0; t < 2; ++t) {
+          const int64_t qrow = static_cast<int64_t>(it.b * p.Hq + it.h[t]) * p.S + it.q0[t];
+          uint8_t* dst = smem + (t ? C::OFF_QB : C::OFF_QA);
 #pragma unroll
           for (int r = 0; r < D / 64; ++r)
-            sep::tma_load_2d(smem + L::OFF_Q + r * L::REG, &tm_q, r * 64, static_cast<int32_t>(qrow),
-                             &bars->k_full[0]);
-        } else {
-          sep::mbar_arrive_expect_tx(&bars->k_full[st], L::KV_BYTES);
+            sep::tma_load_2d(dst + r * C::REG, &tm_q, r * 64, static_cast<int32_t>(qrow),
+                             &bars->q_full);
         }
+        last_q = static_cast<int>(nitem);
+        for (int j = 0; j < it.nblk; ++j, ++gblk) {
+          const int st = gblk % NST;
+          const uint32_t use = gblk / NST;
+          const bool gathered = j < it.nblk_g;
+          const int64_t row = kv_row0 + (gathered ? static_cast<int64_t>(j) * BN
+                                                  : it.win_lo + static_cast<int64_t>(j - it.nblk_g) * BN);
+          if (gblk >= static_cast<uint32_t>(NST) &&
+              !sep::mbar_wait(&bars->k_empty[st], (use - 1) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          sep::mbar_arrive_expect_tx(&bars->k_full[st], C::KV_BYTES);
 #pragma unroll
-        for (int r = 0; r < D / 64; ++r)
-          sep::tma_load_2d(sk + r * L::REG, mk, r * 64, static_cast<int32_t>(row), &bars->k_full[st]);
-        last_k[st] = j;
-        if (j >= NST && !sep::mbar_wait(&bars->v_empty[st], (use - 1) & 1, abort, p.err)) break;
-        uint8_t* sv = smem + L::OFF_V + st * L::KV_BYTES;
-        sep::mbar_arrive_expect_tx(&bars->v_full[st], L::KV_BYTES);
+          for (int r = 0; r < D / 64; ++r)
+            sep::tma_load_2d(smem + C::OFF_K + st * C::KV_BYTES + r * C::REG, gathered ? &tm_kc : &tm_k,
+                             r * 64, static_cast<int32_t>(row), &bars->k_full[st]);
+          last_k[st] = static_cast<int>(gblk);
+          if (gblk >= static_cast<uint32_t>(NST) &&
+              !sep::mbar_wait(&bars->v_empty[st], (use - 1) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          sep::mbar_arrive_expect_tx(&bars->v_full[st], C::KV_BYTES);
 #pragma unroll
-        for (int r = 0; r < D / 64; ++r)
-          sep::tma_load_2d(sv + r * L::REG, mv, r * 64, static_cast<int32_t>(row), &bars->v_full[st]);
-        last_v[st] = j;
+          for (int r = 0; r < D / 64; ++r)
+            sep::tma_load_2d(smem + C::OFF_V + st * C::KV_BYTES + r * C::REG, gathered ? &tm_vc : &tm_v,
+                             r * 64, static_cast<int32_t>(row), &bars->v_full[st]);
+          last_v[st] = static_cast<int>(gblk);
+        }
       }
       if (*abort) {
-        // Only the last load of each stage can still be in flight (a stage is
-        // reloaded only after its previous contents were consumed): let those
-        // land before the CTA's shared memory goes away.
+        // only the most recent load of each buffer can still be in flight
+        if (last_q >= 0) drain_wait(&bars->q_full, last_q & 1);
         for (int s2 = 0; s2 < NST; ++s2) {
           if (last_k[s2] >= 0) drain_wait(&bars->k_full[s2], (last_k[s2] / NST) & 1);
           if (last_v[s2] >= 0) drain_wait(&bars->v_full[s2], (last_v[s2] / NST) & 1);
@@ -198,160 +252,206 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = sep::idesc_bf16_f32(BM, BN, false);
       constexpr uint32_t idesc_o = sep::idesc_bf16_f32(BM, D, true);
-      const uint32_t sq = sep::smem_u32(smem + L::OFF_Q);
-      const uint32_t sp = sep::smem_u32(smem + L::OFF_P);
-      auto issue_pv = [&](int jj) -> bool {
-        const int st = jj % NST;
-        if (!sep::mbar_wait(&bars->p_full, jj & 1, abort, p.err)) return false;
-        if (!sep::mbar_wait(&bars->v_full[st], (jj / NST) & 1, abort, p.err)) return false;
+      const uint32_t sq0 = sep::smem_u32(smem + C::OFF_QA), sq1 = sep::smem_u32(smem + C::OFF_QB);
+      uint32_t gblk = 0, nitem = 0, pphase = 0;  // bit t: phase of p_full[t]
+      bool ok = true;
+      // O_t += P_t V (block `vblk` of the global stream); the first PV of an
+      // item overwrites O_t, so it waits until the previous item's epilogue
+      // of tile t has read O_t.
+      auto issue_pv = [&](int t, uint32_t vblk, bool first) -> bool {
+        if (!sep::mbar_wait(&bars->p_full[t], (pphase >> t) & 1u, abort, p.err)) return false;
+        pphase ^= 1u << t;
+        if (t == 0 && !sep::mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err))
+          return false;
+        if (first && nitem > 0 && !sep::mbar_wait(&bars->o_empty[t], (nitem - 1) & 1, abort, p.err))
+          return false;
         sep::tc_fence_after();
-        const uint32_t sv = sep::smem_u32(smem + L::OFF_V + st * L::KV_BYTES);
+        const uint32_t sv = sep::smem_u32(smem + C::OFF_V + (vblk % NST) * C::KV_BYTES);
+        const uint32_t ptm = tmem + (t ? C::COL_S1 : C::COL_S0);
+        const uint32_t otm = tmem + (t ? C::COL_O1 : C::COL_O0);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t ad = sep::smem_desc_sw128(sp + (kk / 4) * L::REG + (kk % 4) * 32, 16);
-          const uint64_t bd = sep::smem_desc_sw128(sv + kk * 2048, L::REG);
-          sep::mma_bf16_ss(tmem + 256, ad, bd, idesc_o, (jj > 0 || kk > 0) ? 1u : 0u);
+          const uint64_t bd = sep::smem_desc_sw128(sv + kk * 2048, C::REG);
+          sep::mma_bf16_ts(otm, ptm + kk * 8, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
         }
-        sep::mma_commit(&bars->o_done);
-        sep::mma_commit(&bars->v_empty[st]);
         return true;
       };
-      bool ok = true;
-      for (int j = 0; j < nblk && ok; ++j) {
-        const int st = j % NST;
-        if (!sep::mbar_wait(&bars->k_full[st], (j / NST) & 1, abort, p.err)) {
-          ok = false;
-          break;
-        }
-        sep::tc_fence_after();
-        const uint32_t sk = sep::smem_u32(smem + L::OFF_K + st * L::KV_BYTES);
-        const uint32_t s_tmem = tmem + (j & 1) * 128;
+      auto issue_s = [&](int t, uint32_t kblk) {
+        const uint32_t sk = sep::smem_u32(smem + C::OFF_K + (kblk % NST) * C::KV_BYTES);
+        const uint32_t sq = t ? sq1 : sq0;
+        const uint32_t stm = tmem + (t ? C::COL_S1 : C::COL_S0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sep::smem_desc_sw128(sq + (kk / 4) * L::REG + (kk % 4) * 32, 16);
-          const uint64_t bd = sep::smem_desc_sw128(sk + (kk / 4) * L::REG + (kk % 4) * 32, 16);
-          sep::mma_bf16_ss(s_tmem, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t ad = sep::smem_desc_sw128(sq + (kk / 4) * C::REG + (kk % 4) * 32, 16);
+          const uint64_t bd = sep::smem_desc_sw128(sk + (kk / 4) * C::REG + (kk % 4) * 32, 16);
+          sep::mma_bf16_ss(stm, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
         }
-        sep::mma_commit(&bars->s_full[j & 1]);
-        sep::mma_commit(&bars->k_empty[st]);
-        if (j >= 1) ok = issue_pv(j - 1);
+        sep::mma_commit(&bars->s_full[t]);
+      };
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
+        const Item it = make_item(p, item);
+        if (!sep::mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
+        for (int j = 0; j < it.nblk; ++j, ++gblk) {
+          if (!sep::mbar_wait(&bars->k_full[gblk % NST], (gblk / NST) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          sep::tc_fence_after();
+          // tile A: finish the previous block's PV, then this block's S
+          if (j > 0 && !(ok = issue_pv(0, gblk - 1, j == 1))) break;
+          issue_s(0, gblk);
+          if (j > 0) {
+            if (!(ok = issue_pv(1, gblk - 1, j == 1))) break;
+            sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
+          }
+          issue_s(1, gblk);
+          sep::mma_commit(&bars->k_empty[gblk % NST]);
+          if (j == it.nblk - 1) sep::mma_commit(&bars->q_empty);
+        }
+        if (!ok) break;
+        // last block's PV of both tiles, then hand O to the epilogues
+        if (!(ok = issue_pv(0, gblk - 1, it.nblk == 1))) break;
+        sep::mma_commit(&bars->o_full[0]);
+        if (!(ok = issue_pv(1, gblk - 1, it.nblk == 1))) break;
+        sep::mma_commit(&bars->o_full[1]);
+        sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
       }
-      if (ok) issue_pv(nblk - 1);
-      // every MMA issued above has completed once `drain` fires
       sep::mma_commit(&bars->drain);
       drain_wait(&bars->drain, 0);
     }
   } else {
-    // ------------------------------------------------------------ softmax
-    const int t = threadIdx.x;  // tile row == TMEM lane
-    const int i = q0 + t;
-    const int ie = i < S ? i : S - 1;  // rows past the end mask like the last row
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const uint8_t* flags = p.is_sep + static_cast<int64_t>(b) * S;
-    float m_ref = -INFINITY, l = 0.f;
-    uint8_t* sp_row = smem + L::OFF_P + (t >> 3) * 1024 + (t & 7) * 128;
+    // ------------------------------------------------------------ softmax (tile t)
+    const int t = warp >> 2;            // 0: tile A, 1: tile B
+    const int row = threadIdx.x & 127;  // tile row == TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = tmem + lane_base + (t ? C::COL_S1 : C::COL_S0);
+    const uint32_t o_col = tmem + lane_base + (t ? C::COL_O1 : C::COL_O0);
+    uint32_t sphase = 0, nitem = 0;
     bool ok = true;
-    for (int j = 0; j < nblk; ++j) {
-      // keep-bits of this row for the block's 128 columns
-      uint32_t keep[4];
-      if (j < nblk_g) {
-        const int valid = nG - j * BN;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
+      const Item it = make_item(p, item);
+      const int i = (t ? it.q0[1] : it.q0[0]) + row;
+      const int ie = i < p.S ? i : p.S - 1;  // rows past the end mask like the last row
+      const uint8_t* flags = p.is_sep + static_cast<int64_t>(it.b) * p.S;
+      const int my_lo = t ? it.lo[1] : it.lo[0];
+      const int my_nG = t ? it.nG[1] : it.nG[0];
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < it.nblk; ++j) {
+        uint32_t keep[4];
+        if (j < it.nblk_g) {
+          const int valid = my_nG - j * BN;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) keep[c] = bits_le(valid - 1 - 32 * c);
-      } else {
-        const int base = lo + (j - nblk_g) * BN;
-        const int ihi = ie - base, ilo = ie - p.n - base;
+          for (int c = 0; c < 4; ++c) keep[c] = bits_le(valid - 1 - 32 * c);
+        } else {
+          const int base = it.win_lo + (j - it.nblk_g) * BN;
+          const int ihi = ie - base, ilo = ie - p.n - base, jlo = my_lo - base;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int pos = base + 32 * c + lane;
-          const bool f = pos < S && (flags[pos] != 0 || pos < p.a);
-          const uint32_t sepbits = __ballot_sync(0xffffffffu, f);
-          keep[c] = bits_le(ihi - 32 * c) & (~bits_le(ilo - 32 * c) | sepbits);
+          for (int c = 0; c < 4; ++c) {
+            const int pos = base + 32 * c + lane;
+            const bool f = pos < p.S && (flags[pos] != 0 || pos < p.a);
+            const uint32_t sepbits = __ballot_sync(0xffffffffu, f);
+            keep[c] = bits_le(ihi - 32 * c) & (~bits_le(ilo - 32 * c) | sepbits) &
+                      ~bits_le(jlo - 1 - 32 * c);
+          }
         }
+        if (!__all_sync(0xffffffffu, sep::mbar_wait(&bars->s_full[t], sphase, abort, p.err))) {
+          ok = false;
+          break;
+        }
+        sphase ^= 1;
+        sep::tc_fence_after();
+        // pass 1: masked row maximum of the raw scores (8 independent chains)
+        float mx[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+        // (loops over the 4 column groups stay rolled: one group of scores in
+        // registers at a time; the keep words rotate instead of being indexed)
+        uint32_t k0 = keep[0], k1 = keep[1], k2 = keep[2], k3 = keep[3];
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          sep::tmem_ld32(s_col + 32 * c, r);
+          sep::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            mx[e & 7] = fmaxf(mx[e & 7], (k0 >> e) & 1u ? __uint_as_float(r[e]) : -INFINITY);
+          k0 = k1;
+          k1 = k2;
+          k2 = k3;
+        }
+        const float mblk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                           p.scale_log2;
+        float alpha = 1.f;
+        const bool grow = mblk > m_ref + kRescaleLog2;
+        if (grow) {
+          alpha = sep::ex2_approx(m_ref - mblk);  // 0 while m_ref is -inf
+          m_ref = mblk;
+        }
+        // S_t of this block was issued after this tile's previous P*V, and
+        // MMAs complete in order, so that P*V is done: O_t may be rescaled.
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            sep::tmem_ld32(o_col + 32 * c, o);
+            sep::tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            sep::tmem_st32(o_col + 32 * c, o);
+          }
+        }
+        const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+        float sm[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) sm[u] = 0.f;
+        // pass 2: P = 2^(s*scale - m) as bf16 pairs written over S_t: keys
+        // [32c, 32c+32) go to columns [16c, 16c+16), which hold scores of
+        // keys already read back
+        k0 = keep[0];
+        k1 = keep[1];
+        k2 = keep[2];
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t r[32];
+          sep::tmem_ld32(s_col + 32 * c, r);
+          sep::tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float x0 = (k0 >> e) & 1u ? __uint_as_float(r[e]) : -INFINITY;
+            const float x1 = (k0 >> (e + 1)) & 1u ? __uint_as_float(r[e + 1]) : -INFINITY;
+            const float p0 = sep::ex2_approx(fmaf(x0, p.scale_log2, -mr));
+            const float p1 = sep::ex2_approx(fmaf(x1, p.scale_log2, -mr));
+            sm[e & 7] += p0;
+            sm[(e + 1) & 7] += p1;
+            r[e >> 1] = sep::pack_bf16x2(p0, p1);
+          }
+          sep::tmem_st16(s_col + 16 * c, r);
+          k0 = k1;
+          k1 = k2;
+          k2 = keep[3];
+        }
+        l = l * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+        sep::tmem_wait_st();
+        sep::tc_fence_before();
+        sep::mbar_arrive(&bars->p_full[t]);
       }
-      if (!__all_sync(0xffffffffu, sep::mbar_wait(&bars->s_full[j & 1], (j >> 1) & 1, abort, p.err))) {
+      if (!ok) break;
+      // epilogue: O_t / l -> out (bf16), lse
+      if (!__all_sync(0xffffffffu, sep::mbar_wait(&bars->o_full[t], nitem & 1, abort, p.err))) {
         ok = false;
         break;
       }
       sep::tc_fence_after();
-      uint32_t r[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) sep::tmem_ld32(tmem + lane_base + (j & 1) * 128 + 32 * c, r[c]);
-      sep::tmem_wait_ld();
-      float mblk = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float x = (keep[c] >> e) & 1u ? __uint_as_float(r[c][e]) * p.scale_log2 : -INFINITY;
-          r[c][e] = __float_as_uint(x);
-          mblk = fmaxf(mblk, x);
-        }
-      float alpha = 1.f;
-      const bool grow = mblk > m_ref + kRescaleLog2;
-      if (grow) {
-        alpha = sep::ex2_approx(m_ref - mblk);  // 0 while m_ref is -inf
-        m_ref = mblk;
-      }
-      const float mr = m_ref == -INFINITY ? 0.f : m_ref;
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float pe = sep::ex2_approx(__uint_as_float(r[c][e]) - mr);
-          r[c][e] = __float_as_uint(pe);
-          sum += pe;
-        }
-      l = l * alpha + sum;
-      // the previous P*V must be done before P is overwritten or O rescaled
-      if (j >= 1) {
-        if (!__all_sync(0xffffffffu, sep::mbar_wait(&bars->o_done, (j - 1) & 1, abort, p.err))) {
-          ok = false;
-          break;
-        }
-        sep::tc_fence_after();
-        if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            const uint32_t ta = tmem + lane_base + 256 + 32 * c;
-            sep::tmem_ld32(ta, o);
-            sep::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            sep::tmem_st32(ta, o);
-          }
-          sep::tmem_wait_st();
-        }
-      }
-      // P row -> shared memory, bf16, 128-byte swizzle (two 64-key regions)
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int c = ch >> 2, e0 = (ch & 3) * 8;
-        uint4 w;
-        w.x = sep::pack_bf16x2(__uint_as_float(r[c][e0 + 0]), __uint_as_float(r[c][e0 + 1]));
-        w.y = sep::pack_bf16x2(__uint_as_float(r[c][e0 + 2]), __uint_as_float(r[c][e0 + 3]));
-        w.z = sep::pack_bf16x2(__uint_as_float(r[c][e0 + 4]), __uint_as_float(r[c][e0 + 5]));
-        w.w = sep::pack_bf16x2(__uint_as_float(r[c][e0 + 6]), __uint_as_float(r[c][e0 + 7]));
-        const int region = ch >> 3, cc = ch & 7;
-        *reinterpret_cast<uint4*>(sp_row + region * L::REG + ((cc ^ (t & 7)) << 4)) = w;
-      }
-      sep::fence_proxy_async_smem();
-      sep::tc_fence_before();
-      sep::mbar_arrive(&bars->p_full);
-    }
-    // epilogue: O / l -> out (bf16), lse
-    if (ok && __all_sync(0xffffffffu, sep::mbar_wait(&bars->o_done, (nblk - 1) & 1, abort, p.err))) {
-      sep::tc_fence_after();
       const float inv = 1.f / l;
-      __nv_bfloat16* orow = p.out + (static_cast<int64_t>(b * p.Hq + h) * S + i) * D;
+      const int h = t ? it.h[1] : it.h[0];
+      __nv_bfloat16* orow = p.out + (static_cast<int64_t>(it.b * p.Hq + h) * p.S + i) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
-        sep::tmem_ld32(tmem + lane_base + 256 + 32 * c, o);
+        sep::tmem_ld32(o_col + 32 * c, o);
         sep::tmem_wait_ld();
-        if (i < S) {
+        if (i < p.S) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             uint4 w;
@@ -363,9 +463,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (p.lse && i < S)
-        p.lse[static_cast<int64_t>(b * p.Hq + h) * S + i] =
+      if (p.lse && i < p.S)
+        p.lse[static_cast<int64_t>(it.b * p.Hq + h) * p.S + i] =
             (m_ref + __log2f(l)) * 0.69314718055994530942f;
+      sep::tc_fence_before();
+      sep::mbar_arrive(&bars->o_empty[t]);
     }
   }
   sep::tc_fence_before();
@@ -451,17 +553,30 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int D) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+int num_sms() {
+  static int sms[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!sms[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    sms[dev] = v > 0 ? v : 148;
+  }
+  return sms[dev];
+}
+
 template <int D>
 int launch(const void* q, const void* k, const void* v, const uint8_t* is_sep,
            const int32_t* prefix, const int32_t* idx, int B, int Hq, int Hkv, int S, int a, int n,
            float scale, void* out, float* lse, void* kc, void* vc, cudaStream_t st) {
-  using L = Layout<D>;
+  using C = Cfg<D>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     if (cudaFuncSetAttribute(k_prefill_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             L::ALLOC) != cudaSuccess)
+                             C::ALLOC) != cudaSuccess)
       return SEP_ECUDA;
     attr_set[dev] = true;
   }
@@ -490,13 +605,23 @@ int launch(const void* q, const void* k, const void* v, const uint8_t* is_sep,
   p.a = a;
   p.n = n;
   p.G = Hq / Hkv;
-  p.ntiles = (S + BM - 1) / BM;
+  p.pair_heads = (p.G % 2 == 0) ? 1 : 0;
+  if (p.pair_heads) {
+    p.npairs = Hq / 2;
+    p.ntiles_item = (S + BM - 1) / BM;
+  } else {
+    p.npairs = Hq;
+    p.ntiles_item = (S + 2 * BM - 1) / (2 * BM);
+  }
+  const int64_t items = static_cast<int64_t>(p.ntiles_item) * B * p.npairs;
+  if (items >= (1ll << 31)) return SEP_EINVAL;
+  p.n_items = static_cast<int>(items);
   p.scale_log2 = scale * 1.44269504088896340736f;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.err = sep::device_error_word();
-  dim3 grid(p.ntiles, Hq, B);
-  k_prefill_tc<D><<<grid, kThreads, L::ALLOC, st>>>(mq, mk, mv, mkc, mvc, p);
+  const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
+  k_prefill_tc<D><<<grid, kThreads, C::ALLOC, st>>>(mq, mk, mv, mkc, mvc, p);
   return sep::launch_status();
 }
 
