@@ -26,6 +26,7 @@ ABI_SYMBOLS = (
     "sep_attn_prefill_workspace", "sep_attn_prefill", "sepcache_bytes", "sepcache_carve",
     "sepcache_init", "sepcache_append", "sepcache_compact", "sep_attn_decode_workspace",
     "sep_attn_decode", "sepcache_status", "sep_device_status", "sep_attn_decode_noalloc",
+    "sep_attn_decode_step",
 )
 
 
@@ -44,7 +45,8 @@ class SepCacheCfg(ctypes.Structure):
 class _SepCacheC(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("pos", ctypes.c_void_p),
                 ("flag", ctypes.c_void_p), ("counts", ctypes.c_void_p), ("plan", ctypes.c_void_p),
-                ("step", ctypes.c_void_p), ("status", ctypes.c_void_p), ("layers", ctypes.c_int32),
+                ("step", ctypes.c_void_p), ("status", ctypes.c_void_p), ("cur", ctypes.c_void_p),
+                ("layers", ctypes.c_int32),
                 ("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("cap", ctypes.c_int32), ("cfg", SepCacheCfg)]
 
@@ -74,6 +76,8 @@ def _load():
     L.sep_attn_decode_workspace.argtypes = [ctypes.POINTER(_SepCacheC), i32]
     L.sep_attn_decode_workspace.restype = sz
     L.sep_attn_decode.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, i32, f32, P, P, P, sz, P]
+    L.sep_attn_decode_step.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, P, P, P, i32, f32, P, P,
+                                       P, sz, P]
     L.sep_attn_decode_noalloc.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, i32, f32, P, P, P]
     L.sepcache_status.argtypes = [ctypes.POINTER(_SepCacheC), ctypes.POINTER(ctypes.c_int32), P]
     L.sep_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32), i32, P]
@@ -229,14 +233,19 @@ class SepCache:
             n *= d
         return self.buffer[off: off + n * esz].view(dtype).view(*shape)
 
-    # device views of the cache state
+    # device views of the cache state; K/V have two buffers per sequence and
+    # cur[b] names the current one
     @property
     def k(self):
-        return self._view(self.c.k, (self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
+        return self._view(self.c.k, (2, self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
 
     @property
     def v(self):
-        return self._view(self.c.v, (self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
+        return self._view(self.c.v, (2, self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
+
+    @property
+    def cur(self):
+        return self._view(self.c.cur, (self.B,), torch.int32)
 
     @property
     def pos(self):
@@ -287,6 +296,22 @@ class SepCache:
         _check("sep_attn_decode", _lib.sep_attn_decode(
             ctypes.byref(self.c), layer, _ptr(q), Hq, float(scale), _ptr(out), _ptr(lse),
             _ptr(ws), ws.numel(), _stream(stream)))
+        return out, lse
+
+    def decode_step(self, layer: int, q, k_new, v_new, is_sep_new=None, scale: float = 0.0,
+                    out=None, lse=None, want_lse=True, stream=None):
+        """append + compact + decode of one layer in one launch (plus the
+        layer-0 bookkeeping launch)."""
+        _need_cuda(q, k_new, v_new, is_sep_new, out, lse)
+        B, Hq, D = q.shape
+        if out is None:
+            out = torch.empty_like(q)
+        if lse is None and want_lse:
+            lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        ws = self.workspace(Hq)
+        _check("sep_attn_decode_step", _lib.sep_attn_decode_step(
+            ctypes.byref(self.c), layer, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(is_sep_new), Hq,
+            float(scale), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)))
         return out, lse
 
     def decode_noalloc(self, layer: int, q, scale: float = 0.0, out=None, lse=None,

@@ -3,27 +3,33 @@
 // The cache keeps only the initial, separator, past-window and local-window
 // rows, so a decode step reads len[b] <= a + s + past + w K/V rows per
 // (sequence, kv head) (jieyibu.net explainer, section 1.3: fewer KV pairs to
-// load).  The kernel is bound by HBM bandwidth:
+// load).  The kernel is bound by HBM bandwidth and by its latency chain:
 //   * grid (split, kv head, sequence); a CTA takes 64 consecutive rows of one
 //     (b, kv head) and pulls them into shared memory with two bulk copies
 //     (K and V, one mbarrier), so each byte is read from HBM once per step;
-//   * the G = Hq/Hkv query heads of the group share every K/V row;
-//   * each CTA writes an unnormalised partial (max, sum, G x D output); the
-//     last CTA of a (b, kv head) to finish (an atomic ticket, no waiting)
-//     merges the partials and writes out and lse.
+//   * the G = Hq/Hkv query heads of the group share every K/V row; a warp
+//     scores four rows at a time (eight lanes per row, each lane 8 or 16
+//     dims), so a row costs three shuffle levels instead of five;
+//   * each CTA produces an unnormalised partial (max, sum, G x D output).
+//     With at most 8 splits the splits of a (b, kv head) form one
+//     thread-block cluster and merge the partials through distributed shared
+//     memory; otherwise they go through the workspace and the last CTA to
+//     finish (an atomic ticket, no waiting) merges them;
+//   * launched as a programmatic dependent launch: the grid may start while
+//     the previous kernel on the stream drains, and waits for it before its
+//     first global read.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
+#include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace {
 
 constexpr int ROWS = 64;  // rows per split
 constexpr int kThreads = 128;
-
-template <typename T>
-__device__ __forceinline__ float to_f(T x);
-template <>
-__device__ __forceinline__ float to_f<float>(float x) { return x; }
-template <>
-__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+constexpr int kMaxClusterSplits = 8;
 
 template <typename T>
 __device__ __forceinline__ T from_f(float x);
@@ -32,107 +38,312 @@ __device__ __forceinline__ float from_f<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
-// DPL consecutive elements of a row starting at element d0, as floats.
-template <typename T, int DPL>
-__device__ __forceinline__ void load_row_slice(const T* row, int d0, float (&x)[DPL]) {
+// 8 consecutive elements (16-byte aligned) as floats.
+__device__ __forceinline__ void ld8(const __nv_bfloat16* p, float* x) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) x[e] = to_f(row[d0 + e]);
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
 }
+__device__ __forceinline__ void ld8(const float* p, float* x) {
+  const float4 a = reinterpret_cast<const float4*>(p)[0];
+  const float4 b = reinterpret_cast<const float4*>(p)[1];
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+  x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 struct DecodeParams {
   const void* q;
   const void* kc;
   const void* vc;
   const int32_t* counts;
+  const int32_t* cur;   // [B] current K/V buffer
+  const int32_t* plan;  // [B][cap + header] this step's plan (fused step only)
+  const void* k_new;    // [B][Hkv][D] (fused step only)
+  const void* v_new;
   void* out;
   float* lse;
   float* part_ml;  // [B][Hq][nsplit][2]
   float* part_o;   // [B][Hq][nsplit][D]
   int32_t* ticket; // [B][Hkv]
   int32_t* err;
-  int layer, B, Hq, Hkv, cap, nsplit;
+  int layer, layers, B, Hq, Hkv, cap, nsplit;
   float scale_log2;
 };
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) k_decode(const DecodeParams p) {
-  constexpr int DPL = D / 32;
+// The last part of a split: its unnormalised partial (po, sm = max, sl = sum,
+// in this CTA's shared memory, rows with no keys at -inf / 0) is merged with
+// the other splits of the (b, kv head) and written out.
+template <typename T, int D, int G, bool CLUSTER, int NCL = kMaxClusterSplits>
+__device__ __forceinline__ void decode_finish(const DecodeParams& p, float (*po)[D], float* sm,
+                                              float* sl, int nsplit_b, int split, int b, int g) {
+  __shared__ int is_last;
+  __shared__ float Ms[G], Ls[G];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  T* out = static_cast<T*>(p.out);
+  const int hq0 = g * G;
+  if (nsplit_b == 1) {
+    if (split == 0) {
+      for (int e = threadIdx.x; e < G * D; e += kThreads) {
+        const int h = e / D, d = e % D;
+        out[(static_cast<int64_t>(b) * p.Hq + hq0 + h) * D + d] = from_f<T>(po[h][d] / sl[h]);
+      }
+      if (p.lse && threadIdx.x < G)
+        p.lse[static_cast<int64_t>(b) * p.Hq + hq0 + threadIdx.x] =
+            (sm[threadIdx.x] + log2f(sl[threadIdx.x])) * 0.69314718055994530942f;
+    }
+    if (CLUSTER) {
+      cg::this_cluster().sync();
+      cg::this_cluster().sync();
+    }
+    return;
+  }
+  if (CLUSTER) {
+    // after the cluster barrier CTA `split` merges outputs
+    // [split*G*D/NCL, (split+1)*G*D/NCL) from the shared memory of all splits
+    cg::cluster_group cl = cg::this_cluster();
+    cl.sync();
+    constexpr int PER = G * D / NCL;
+    for (int e = threadIdx.x; e < PER; e += blockDim.x) {
+      const int idx = split * PER + e;
+      const int h = idx / D, d = idx % D;
+      float M = -INFINITY;
+      float mk[NCL], lk[NCL], ok[NCL];
+#pragma unroll
+      for (int k = 0; k < NCL; ++k) {
+        const bool in = k < nsplit_b;
+        mk[k] = in ? *cl.map_shared_rank(&sm[h], k) : -INFINITY;
+        lk[k] = in ? *cl.map_shared_rank(&sl[h], k) : 0.f;
+        ok[k] = in ? *cl.map_shared_rank(&po[h][d], k) : 0.f;
+        M = fmaxf(M, mk[k]);
+      }
+      float L = 0.f, acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < NCL; ++k) {
+        const float w = k < nsplit_b ? exp2f(mk[k] - M) : 0.f;
+        L += lk[k] * w;
+        acc += ok[k] * w;
+      }
+      out[(static_cast<int64_t>(b) * p.Hq + hq0 + h) * D + d] = from_f<T>(acc / L);
+      if (p.lse && d == 0)
+        p.lse[static_cast<int64_t>(b) * p.Hq + hq0 + h] = (M + log2f(L)) * 0.69314718055994530942f;
+    }
+    cl.sync();  // keep this CTA's partial alive until every reader is done
+    return;
+  }
+  if (split >= nsplit_b) return;
+  // write this split's partial to the workspace
+  for (int e = threadIdx.x; e < G * D; e += kThreads) {
+    const int h = e / D, d = e % D;
+    p.part_o[((static_cast<int64_t>(b) * p.Hq + hq0 + h) * p.nsplit + split) * D + d] = po[h][d];
+  }
+  if (threadIdx.x < G) {
+    float* ml = p.part_ml + ((static_cast<int64_t>(b) * p.Hq + hq0 + threadIdx.x) * p.nsplit + split) * 2;
+    ml[0] = sm[threadIdx.x];
+    ml[1] = sl[threadIdx.x];
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t* tk = p.ticket + static_cast<int64_t>(b) * p.Hkv + g;
+    const int prev = atomicAdd(tk, 1);
+    is_last = prev == nsplit_b - 1;
+    if (is_last) atomicExch(tk, 0);  // ready for the next call
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  // merge the partials of every split of this (b, kv head).  Loads that do
+  // not depend on each other are issued together: one lane per split for the
+  // (max, sum) pairs, then eight splits at a time for the output rows.
+  for (int h = warp; h < G; h += 4) {
+    const float* ml = p.part_ml + (static_cast<int64_t>(b) * p.Hq + hq0 + h) * p.nsplit * 2;
+    float M = -INFINITY;
+    for (int s = lane; s < nsplit_b; s += 32) M = fmaxf(M, __ldcg(ml + 2 * s));
+    for (int o2 = 16; o2; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o2));
+    float Lsum = 0.f;
+    for (int s = lane; s < nsplit_b; s += 32) Lsum += __ldcg(ml + 2 * s + 1) * exp2f(__ldcg(ml + 2 * s) - M);
+    for (int o2 = 16; o2; o2 >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o2);
+    if (lane == 0) {
+      Ms[h] = M;
+      Ls[h] = Lsum;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * D; e += kThreads) {
+    const int h = e / D, d = e % D;
+    const float* ml = p.part_ml + (static_cast<int64_t>(b) * p.Hq + hq0 + h) * p.nsplit * 2;
+    const float* pp = p.part_o + (static_cast<int64_t>(b) * p.Hq + hq0 + h) * p.nsplit * D;
+    const float M = Ms[h];
+    float acc = 0.f;
+    for (int s0 = 0; s0 < nsplit_b; s0 += 8) {
+      float ov[8], mv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int s = s0 + u;
+        const bool in = s < nsplit_b;
+        ov[u] = in ? __ldcg(pp + s * D + d) : 0.f;
+        mv[u] = in ? __ldcg(ml + 2 * s) : -INFINITY;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) acc += ov[u] * exp2f(mv[u] - M);
+    }
+    out[(static_cast<int64_t>(b) * p.Hq + hq0 + h) * D + d] = from_f<T>(acc / Ls[h]);
+  }
+  if (p.lse && threadIdx.x < G)
+    p.lse[static_cast<int64_t>(b) * p.Hq + hq0 + threadIdx.x] =
+        (Ms[threadIdx.x] + log2f(Ls[threadIdx.x])) * 0.69314718055994530942f;
+}
+
+// FUSED: one decode step of the layer -- the CTA also writes the new token's
+// K/V row and, on a flush step, copies its share of the surviving rows into
+// the sequence's other buffer while loading them (see sepcache.cu).
+// CLUSTER: the grid's x dimension (the splits) is one cluster.
+template <typename T, int D, int G, bool FUSED, bool CLUSTER>
+__global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const DecodeParams p) {
+  constexpr int NI = D / 64;   // 8-element slices per lane: dims 8*c8 + 64*i + e
+  constexpr int DPL = 8 * NI;  // dims per lane
   // dynamic: K rows | V rows; the cross-warp reduction reuses the K rows
   extern __shared__ __align__(128) uint8_t dsm[];
   T* sk = reinterpret_cast<T*>(dsm);
   T* sv = sk + ROWS * D;
   float(*red)[G][D] = reinterpret_cast<float(*)[G][D]>(dsm);
   static_assert(sizeof(T) * ROWS * D >= sizeof(float) * 4 * G * D, "reduction must fit in K rows");
-  __shared__ float sq[G][D];
   __shared__ float ss[G][ROWS];
+  __shared__ float po[G][D];  // this CTA's partial output (cluster merge)
   __shared__ float sm[G], sl[G];
   __shared__ __align__(8) uint64_t bar;
-  __shared__ int is_last;
   __shared__ int abort_flag;
 
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int32_t* cnt = p.counts + 4 * b;
-  const int len = cnt[0] + cnt[1] + cnt[2] + cnt[3];
-  const int r0 = split * ROWS;
-  if (len <= 0 || len > p.cap || r0 >= len) return;
-  const int nrows = len - r0 < ROWS ? len - r0 : ROWS;
-  const int nsplit_b = (len + ROWS - 1) / ROWS;
+  const int rr = lane >> 3, c8 = lane & 7;  // row of the 4-row group, 8-dim slice
 
-  const int64_t kv_base =
-      ((static_cast<int64_t>(p.layer) * p.B + b) * p.Hkv + g) * p.cap * D + static_cast<int64_t>(r0) * D;
+  // wait for the previous kernel on the stream (programmatic dependent launch)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
+  // metadata: independent loads issued together
+  const int32_t* cnt = p.counts + 4 * b;
+  const int32_t* pl = p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr);
+  const int c0 = cnt[0], c1 = cnt[1], c2 = cnt[2], c3 = cnt[3];
+  const int buf = p.cur[b] & 1;  // current after this step's bookkeeping
+  const int flush = FUSED ? pl[0] : 0;
+  const int slot = FUSED ? pl[1] : -1;
+  const int sbuf = FUSED ? (pl[4] & 1) : buf;
+  int len = c0 + c1 + c2 + c3;
+  if (len < 0 || len > p.cap) len = 0;
+  const int r0 = split * ROWS;
+  const int nrows = len - r0 < 0 ? 0 : (len - r0 < ROWS ? len - r0 : ROWS);
+  if (!CLUSTER && nrows == 0) return;
+  const int nsplit_b = (len + ROWS - 1) / ROWS;
+  // element offset of row 0 of (buffer, layer, b, g)
+  auto base_of = [&](int bb) -> int64_t {
+    return ((((static_cast<int64_t>(bb) * p.layers + p.layer) * p.B + b) * p.Hkv + g) * p.cap) * D;
+  };
+  const int64_t kv_base = base_of(buf) + static_cast<int64_t>(r0) * D;
   if (threadIdx.x == 0) {
     abort_flag = 0;
     sep::mbar_init(&bar, 1);
     sep::mbar_fence_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  const bool bulk = nrows > 0 && !flush;
+  if (threadIdx.x == 0 && bulk) {
     const uint32_t bytes = static_cast<uint32_t>(nrows * D * sizeof(T));
     sep::mbar_arrive_expect_tx(&bar, 2 * bytes);
     sep::bulk_load(sk, static_cast<const T*>(p.kc) + kv_base, bytes, &bar);
     sep::bulk_load(sv, static_cast<const T*>(p.vc) + kv_base, bytes, &bar);
   }
-  // query rows of the group's heads, pre-scaled into the log2 domain
+  // let the next kernel on the stream begin launching
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // this lane's query slices of the group's heads, pre-scaled (log2 domain)
   const T* qg = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
-  for (int e = threadIdx.x; e < G * D; e += kThreads) sq[e / D][e % D] = to_f(qg[e]) * p.scale_log2;
-  __syncthreads();
-  const bool landed = sep::mbar_wait(&bar, 0, &abort_flag, p.err);
-  if (!landed) {  // the copies must land before this CTA's shared memory is reused
-    int keep_waiting = 0;
-    sep::mbar_wait(&bar, 0, &keep_waiting, nullptr);
-  }
-
-  // scores: warp w takes rows w, w+4, ...; lane owns DPL consecutive dims
-  const int d0 = lane * DPL;
   float qv[G][DPL];
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) qv[h][e] = sq[h][d0 + e];
-  if (landed) {
-    for (int r = warp; r < nrows; r += 4) {
-      float x[DPL];
-      load_row_slice<T, DPL>(sk + r * D, d0, x);
-      float acc[G];
+    for (int i = 0; i < NI; ++i) {
+      ld8(qg + h * D + 64 * i + 8 * c8, &qv[h][8 * i]);
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) a = fmaf(qv[h][e], x[e], a);
-        acc[h] = a;
+      for (int e = 0; e < 8; ++e) qv[h][8 * i + e] *= p.scale_log2;
+    }
+  constexpr int CH = D * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per row
+  if (FUSED && flush && nrows > 0) {
+    // rows of the post-flush layout come from their source rows in the old
+    // buffer (the new token from k_new/v_new); each is also stored at its
+    // destination in the new buffer
+    const int64_t sbase = base_of(sbuf);
+    const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+    const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+    for (int e = threadIdx.x; e < 2 * nrows * CH; e += kThreads) {
+      const int which = e / (nrows * CH), r = (e / CH) % nrows, c = e % CH;
+      const int src = pl[sep::kCachePlanHdr + r0 + r];
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (src == slot) {
+        val = (which ? vn : kn)[c];
+      } else if (src >= 0 && src < p.cap) {
+        val = reinterpret_cast<const uint4*>(static_cast<const T*>(which ? p.vc : p.kc) + sbase +
+                                             static_cast<int64_t>(src) * D)[c];
       }
+      reinterpret_cast<uint4*>((which ? sv : sk) + r * D)[c] = val;
+      reinterpret_cast<uint4*>(const_cast<T*>(static_cast<const T*>(which ? p.vc : p.kc)) + kv_base +
+                               static_cast<int64_t>(r) * D)[c] = val;
+    }
+    __syncthreads();
+  } else if (bulk) {
+    const bool landed = sep::mbar_wait(&bar, 0, &abort_flag, p.err);
+    if (!landed) {  // the copies must land before this CTA's shared memory is reused
+      int keep_waiting = 0;
+      sep::mbar_wait(&bar, 0, &keep_waiting, nullptr);
+    }
+    if (FUSED && slot >= r0 && slot < r0 + nrows) {
+      // the new token is the last row (no flush): take it from k_new/v_new
+      // and store it into the cache
+      const int r = slot - r0;
+      const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+      const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+      for (int e = threadIdx.x; e < 2 * CH; e += kThreads) {
+        const int which = e / CH, c = e % CH;
+        const uint4 val = (which ? vn : kn)[c];
+        reinterpret_cast<uint4*>((which ? sv : sk) + r * D)[c] = val;
+        reinterpret_cast<uint4*>(const_cast<T*>(static_cast<const T*>(which ? p.vc : p.kc)) + kv_base +
+                                 static_cast<int64_t>(r) * D)[c] = val;
+      }
+      __syncthreads();
+    }
+  }
+
+  // scores: warp w takes 4-row groups w, w+4, ...; lane (rr, c8) covers dims
+  // 8*c8 + 64*i + [0, 8) of row 4*group + rr
+  for (int r4 = 4 * warp; r4 < nrows; r4 += 16) {
+    const int r = r4 + rr;
+    float acc[G];
+#pragma unroll
+    for (int h = 0; h < G; ++h) acc[h] = 0.f;
+    if (r < nrows) {
+#pragma unroll
+      for (int i = 0; i < NI; ++i) {
+        float x[8];
+        ld8(sk + r * D + 64 * i + 8 * c8, x);
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[h] = fmaf(qv[h][8 * i + e], x[e], acc[h]);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
+    if (r < nrows) {
 #pragma unroll
       for (int h = 0; h < G; ++h)
-#pragma unroll
-        for (int o = 16; o; o >>= 1) acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], o);
-      if (lane < G) {
-        float v = acc[0];
-#pragma unroll
-        for (int h = 1; h < G; ++h)
-          if (lane == h) v = acc[h];
-        ss[lane][r] = v;
-      }
+        if (c8 == (h & 7)) ss[h][r] = acc[h];
     }
   }
   __syncthreads();
@@ -154,116 +365,392 @@ __global__ void __launch_bounds__(kThreads) k_decode(const DecodeParams p) {
     }
   }
   __syncthreads();
-  // P V: warp-private accumulators, then a cross-warp sum
+  // P V: lane (rr, c8) accumulates its dims over rows rr, rr+4, ... of the
+  // warp's groups; then rows of a lane slice and warps are summed
   float o[G][DPL];
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int e = 0; e < DPL; ++e) o[h][e] = 0.f;
-  if (landed) {
-    for (int r = warp; r < nrows; r += 4) {
-      float x[DPL];
-      load_row_slice<T, DPL>(sv + r * D, d0, x);
+  for (int r4 = 4 * warp; r4 < nrows; r4 += 16) {
+    const int r = r4 + rr;
+    if (r < nrows) {
+      float pr[G];
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float pr = ss[h][r];
+      for (int h = 0; h < G; ++h) pr[h] = ss[h][r];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) o[h][e] = fmaf(pr, x[e], o[h][e]);
+      for (int i = 0; i < NI; ++i) {
+        float x[8];
+        ld8(sv + r * D + 64 * i + 8 * c8, x);
+#pragma unroll
+        for (int h = 0; h < G; ++h)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[h][8 * i + e] = fmaf(pr[h], x[e], o[h][8 * i + e]);
       }
     }
   }
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) red[warp][h][d0 + e] = o[h][e];  // K rows are no longer read
+    for (int e = 0; e < DPL; ++e) {
+      o[h][e] += __shfl_xor_sync(0xffffffffu, o[h][e], 8);
+      o[h][e] += __shfl_xor_sync(0xffffffffu, o[h][e], 16);
+    }
+  __syncthreads();  // K rows are no longer read: reuse them for the reduction
+  if (rr == 0) {
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int i = 0; i < NI; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[warp][h][64 * i + 8 * c8 + e] = o[h][8 * i + e];
+  }
   __syncthreads();
 
-  T* out = static_cast<T*>(p.out);
-  const int hq0 = g * G;
-  if (nsplit_b == 1) {
-    for (int e = threadIdx.x; e < G * D; e += kThreads) {
-      const int h = e / D, d = e % D;
-      const float s = red[0][h][d] + red[1][h][d] + red[2][h][d] + red[3][h][d];
-      out[(static_cast<int64_t>(b) * p.Hq + hq0 + h) * D + d] = from_f<T>(s / sl[h]);
-    }
-    if (p.lse && threadIdx.x < G)
-      p.lse[static_cast<int64_t>(b) * p.Hq + hq0 + threadIdx.x] =
-          (sm[threadIdx.x] + log2f(sl[threadIdx.x])) * 0.69314718055994530942f;
-    return;
-  }
-  // write this split's partial
   for (int e = threadIdx.x; e < G * D; e += kThreads) {
     const int h = e / D, d = e % D;
-    const float s = red[0][h][d] + red[1][h][d] + red[2][h][d] + red[3][h][d];
-    p.part_o[((static_cast<int64_t>(b) * p.Hq + hq0 + h) * p.nsplit + split) * D + d] = s;
+    po[h][d] = nrows > 0 ? red[0][h][d] + red[1][h][d] + red[2][h][d] + red[3][h][d] : 0.f;
   }
-  if (threadIdx.x < G) {
-    float* ml = p.part_ml + ((static_cast<int64_t>(b) * p.Hq + hq0 + threadIdx.x) * p.nsplit + split) * 2;
-    ml[0] = sm[threadIdx.x];
-    ml[1] = sl[threadIdx.x];
-  }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int32_t* tk = p.ticket + static_cast<int64_t>(b) * p.Hkv + g;
-    const int prev = atomicAdd(tk, 1);
-    is_last = prev == nsplit_b - 1;
-    if (is_last) atomicExch(tk, 0);  // ready for the next call
+  if (threadIdx.x < G && nrows == 0) {
+    sm[threadIdx.x] = -INFINITY;
+    sl[threadIdx.x] = 0.f;
   }
   __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  // merge the partials of every split of this (b, kv head)
-  for (int h = warp; h < G; h += 4) {
-    const float* ml = p.part_ml + (static_cast<int64_t>(b) * p.Hq + hq0 + h) * p.nsplit * 2;
-    float M = -INFINITY;
-    for (int s = 0; s < nsplit_b; ++s) M = fmaxf(M, __ldcg(ml + 2 * s));
-    float Lsum = 0.f;
-    for (int s = 0; s < nsplit_b; ++s) Lsum += __ldcg(ml + 2 * s + 1) * exp2f(__ldcg(ml + 2 * s) - M);
-    const float* po = p.part_o + (static_cast<int64_t>(b) * p.Hq + hq0 + h) * p.nsplit * D;
-    for (int d = lane; d < D; d += 32) {
-      float acc = 0.f;
-      for (int s = 0; s < nsplit_b; ++s) acc += __ldcg(po + s * D + d) * exp2f(__ldcg(ml + 2 * s) - M);
-      out[(static_cast<int64_t>(b) * p.Hq + hq0 + h) * D + d] = from_f<T>(acc / Lsum);
-    }
-    if (p.lse && lane == 0)
-      p.lse[static_cast<int64_t>(b) * p.Hq + hq0 + h] = (M + log2f(Lsum)) * 0.69314718055994530942f;
-  }
+  decode_finish<T, D, G, CLUSTER>(p, po, sm, sl, nsplit_b, split, b, g);
 }
 
-template <typename T, int D, int G>
+// ---- warp-level tensor-core helpers (bf16 in, fp32 accumulate)
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// c (16x8 fp32) += a (16x16 bf16, row-major fragment) * b (16x8 bf16, col fragment)
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// bf16 decode on warp-level tensor cores, streamed.  The rows of a (b, kv
+// head) are split between the two CTAs of a cluster.  A producer warp streams
+// each CTA's rows in 64-row chunks through a 3-stage shared-memory ring (one
+// bulk copy per row and tensor; a stage is refilled once all consumers have
+// released it).  Each of the four consumer warps owns 16 rows of every chunk
+// and keeps its own online softmax in registers:
+//   S = Q K^T with the G query heads as the rows of a 16-row A operand (rows
+//     >= G are zero) and its 16 keys as two n-tiles;
+//   the S accumulator fragments become the P operand directly (bf16), and
+//   O += P V with V as B (ldmatrix.trans) over all head dims.
+// No CTA-wide barrier inside the loop.  At the end the warps' partials are
+// combined in shared memory and the two CTAs merge through distributed
+// shared memory.  K/V rows sit at a padded stride (D + 8 elements) so that
+// ldmatrix reads are conflict-free.
+constexpr int kPipeStages = 3;
+constexpr int kPipeCluster = 2;
+constexpr int kPipeThreads = 160;  // 4 consumer warps + 1 producer warp
+
+template <int D>
+constexpr int pipe_smem_bytes() {
+  return kPipeStages * 2 * ROWS * (D + 8) * 2;
+}
+
+template <int D, int G, bool FUSED>
+__global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodeParams p) {
+  static_assert(G <= 8, "at most 8 query heads per kv head");
+  using T = __nv_bfloat16;
+  constexpr int RS = D + 8;  // K/V row stride in shared memory (elements)
+  constexpr int CH = D * 2 / 16;
+  constexpr int NT = D / 8;  // n-tiles of the output
+  extern __shared__ __align__(128) uint8_t dsm[];
+  T* const stages = reinterpret_cast<T*>(dsm);  // [stage][K rows | V rows]
+  float* const wpart = reinterpret_cast<float*>(dsm);  // after the loop: [4][G][D]
+  static_assert(kPipeStages * 2 * ROWS * RS * 2 >= 4 * G * D * 4, "warp partials fit in the ring");
+  __shared__ float po[G][D];
+  __shared__ float sm[G], sl[G];
+  __shared__ float wm[4][G], wl[4][G];
+  __shared__ __align__(8) uint64_t full[kPipeStages], empty[kPipeStages];
+  __shared__ int abort_flag;
+
+  const int half = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int32_t* cnt = p.counts + 4 * b;
+  const int32_t* pl = p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr);
+  const int c0 = cnt[0], c1 = cnt[1], c2 = cnt[2], c3 = cnt[3];
+  const int buf = p.cur[b] & 1;
+  const int flush = FUSED ? pl[0] : 0;
+  const int slot = FUSED ? pl[1] : -1;
+  const int sbuf = FUSED ? (pl[4] & 1) : buf;
+  int len = c0 + c1 + c2 + c3;
+  if (len < 0 || len > p.cap) len = 0;
+  int mid = ((len + 1) / 2 + 15) / 16 * 16;
+  if (mid > len) mid = len;
+  const int rs = half ? mid : 0, re = half ? len : mid;
+  const int nchunks = (re - rs + ROWS - 1) / ROWS;
+  const int nsplit_b = mid < len ? 2 : (len > 0 ? 1 : 0);
+  auto base_of = [&](int bb) -> int64_t {
+    return ((((static_cast<int64_t>(bb) * p.layers + p.layer) * p.B + b) * p.Hkv + g) * p.cap) * D;
+  };
+  const int64_t kv_base = base_of(buf);
+  const T* kc = static_cast<const T*>(p.kc);
+  const T* vc = static_cast<const T*>(p.vc);
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    for (int st = 0; st < kPipeStages; ++st) {
+      sep::mbar_init(&full[st], 1);
+      sep::mbar_init(&empty[st], 4);
+    }
+    sep::mbar_fence_init();
+  }
+  __syncthreads();
+  float o[NT][4];                        // consumer warps: O rows of head gq
+  float m_run = -INFINITY, l_run = 0.f;  // head gq (lanes gq < G)
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+
+  if (warp == 4) {
+    // ---------------------------------------------------------- producer
+    for (int c = 0; c < nchunks; ++c) {
+      const int st = c % kPipeStages;
+      const int r0 = rs + c * ROWS;
+      const int nr = re - r0 < ROWS ? re - r0 : ROWS;
+      T* sk = stages + st * 2 * ROWS * RS;
+      T* sv = sk + ROWS * RS;
+      if (c >= kPipeStages &&
+          !__all_sync(0xffffffffu, sep::mbar_wait(&empty[st], ((c / kPipeStages) - 1) & 1, &abort_flag, p.err)))
+        break;
+      if (FUSED && flush) {
+        // rows of the post-flush layout come from their source rows in the
+        // old buffer (the new token from k_new/v_new); each is also stored
+        // at its destination in the new buffer
+        const int64_t sbase = base_of(sbuf);
+        const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+        const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+        for (int e = lane; e < 2 * nr * CH; e += 32) {
+          const int which = e / (nr * CH), r = (e / CH) % nr, cc = e % CH;
+          const int src = pl[sep::kCachePlanHdr + r0 + r];
+          uint4 val = make_uint4(0, 0, 0, 0);
+          if (src == slot) {
+            val = (which ? vn : kn)[cc];
+          } else if (src >= 0 && src < p.cap) {
+            val = reinterpret_cast<const uint4*>((which ? vc : kc) + sbase + static_cast<int64_t>(src) * D)[cc];
+          }
+          reinterpret_cast<uint4*>((which ? sv : sk) + r * RS)[cc] = val;
+          reinterpret_cast<uint4*>(const_cast<T*>(which ? vc : kc) + kv_base + static_cast<int64_t>(r0 + r) * D)[cc] = val;
+        }
+        __syncwarp();
+        if (lane == 0) sep::mbar_arrive(&full[st]);  // plain stores, released by the arrive
+      } else {
+        if (lane == 0) sep::mbar_arrive_expect_tx(&full[st], 2u * nr * D * 2);
+        __syncwarp();
+        for (int e = lane; e < 2 * nr; e += 32) {
+          const int which = e / nr, r = e % nr;
+          sep::bulk_load((which ? sv : sk) + r * RS, (which ? vc : kc) + kv_base + static_cast<int64_t>(r0 + r) * D,
+                         D * 2, &full[st]);
+        }
+      }
+    }
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  } else {
+    // ---------------------------------------------------------- consumers
+    uint32_t qa[D / 16][4];  // Q fragments (rows = heads; heads >= G are zero)
+    {
+      const T* qg = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const bool in = gq < G;
+        qa[kk][0] = in ? *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * kk + 2 * tq) : 0u;
+        qa[kk][2] = in ? *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * kk + 8 + 2 * tq) : 0u;
+        qa[kk][1] = 0u;
+        qa[kk][3] = 0u;
+      }
+    }
+    for (int c = 0; c < nchunks; ++c) {
+      const int st = c % kPipeStages;
+      const int r0 = rs + c * ROWS;
+      const int nr = re - r0 < ROWS ? re - r0 : ROWS;
+      T* sk = stages + st * 2 * ROWS * RS;
+      T* sv = sk + ROWS * RS;
+      if (!__all_sync(0xffffffffu, sep::mbar_wait(&full[st], (c / kPipeStages) & 1, &abort_flag, p.err)))
+        break;
+      const int kr = 16 * warp;  // this warp's rows of the chunk
+      if (kr < nr) {
+        if (FUSED && !flush && slot >= r0 + kr && slot < r0 + kr + 16 && slot < r0 + nr) {
+          // the new token (the last row without a flush): from k_new/v_new,
+          // also stored into the cache
+          const int r = slot - r0;
+          const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+          const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+          for (int e = lane; e < 2 * CH; e += 32) {
+            const int which = e / CH, cc = e % CH;
+            const uint4 val = (which ? vn : kn)[cc];
+            reinterpret_cast<uint4*>((which ? sv : sk) + r * RS)[cc] = val;
+            reinterpret_cast<uint4*>(const_cast<T*>(which ? vc : kc) + kv_base + static_cast<int64_t>(r0 + r) * D)[cc] = val;
+          }
+        }
+        // V rows of this warp past the chunk's end: P is 0 there, and
+        // 0 * garbage may be NaN
+        const int vr = nr - kr < 16 ? nr - kr : 16;
+        for (int e = lane; e < (16 - vr) * CH; e += 32)
+          reinterpret_cast<uint4*>(sv + (kr + vr + e / CH) * RS)[e % CH] = make_uint4(0, 0, 0, 0);
+        __syncwarp();
+        // S for the warp's 16 keys: two n-tiles
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int kk = 0; kk < D / 16; kk += 2) {
+          uint32_t f0[4], f1[4];
+          ldsm_x4(sep::smem_u32(sk + (kr + (lane & 7)) * RS + 16 * kk + (lane >> 3) * 8), f0);
+          ldsm_x4(sep::smem_u32(sk + (kr + 8 + (lane & 7)) * RS + 16 * kk + (lane >> 3) * 8), f1);
+          mma16816(sa, qa[kk], f0[0], f0[1]);
+          mma16816(sb, qa[kk], f1[0], f1[1]);
+          mma16816(sa, qa[kk + 1], f0[2], f0[3]);
+          mma16816(sb, qa[kk + 1], f1[2], f1[3]);
+        }
+        // keys kr + {2tq, 2tq+1} (sa) and kr + 8 + {2tq, 2tq+1} (sb)
+        float x[4] = {sa[0] * p.scale_log2, sa[1] * p.scale_log2, sb[0] * p.scale_log2, sb[1] * p.scale_log2};
+        const int kk0 = kr + 2 * tq, kk1 = kr + 8 + 2 * tq;
+        if (kk0 >= nr) x[0] = -INFINITY;
+        if (kk0 + 1 >= nr) x[1] = -INFINITY;
+        if (kk1 >= nr) x[2] = -INFINITY;
+        if (kk1 + 1 >= nr) x[3] = -INFINITY;
+        float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+        const float m_new = fmaxf(m_run, mb);
+        const float alpha = exp2f(m_run - m_new);  // 0 on the warp's first keys
+        float pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) pr[e] = exp2f(x[e] - m_new);
+        float ls = (pr[0] + pr[1]) + (pr[2] + pr[3]);
+        ls += __shfl_xor_sync(0xffffffffu, ls, 1);
+        ls += __shfl_xor_sync(0xffffffffu, ls, 2);
+        l_run = l_run * alpha + ls;
+        m_run = m_new;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          o[nt][0] *= alpha;
+          o[nt][1] *= alpha;
+        }
+        // P as the A operand (rows = heads, the 16 keys as k)
+        uint32_t pa[4];
+        pa[0] = sep::pack_bf16x2(pr[0], pr[1]);
+        pa[1] = 0u;
+        pa[2] = sep::pack_bf16x2(pr[2], pr[3]);
+        pa[3] = 0u;
+#pragma unroll
+        for (int np = 0; np < NT / 2; ++np) {
+          uint32_t vb[4];
+          ldsm_x4_t(sep::smem_u32(sv + (kr + ((lane >> 3) & 1) * 8 + (lane & 7)) * RS + 16 * np + (lane >> 4) * 8), vb);
+          mma16816(o[2 * np], pa, vb[0], vb[1]);
+          mma16816(o[2 * np + 1], pa, vb[2], vb[3]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) sep::mbar_arrive(&empty[st]);
+    }
+    // this warp's partial (lanes gq < G hold head gq)
+    if (gq < G && tq == 0) {
+      wm[warp][gq] = m_run;
+      wl[warp][gq] = l_run;
+    }
+  }
+  __syncthreads();  // the ring is idle: reuse it for the warps' outputs
+  if (warp < 4 && gq < G) {
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      wpart[(warp * G + gq) * D + 8 * nt + 2 * tq] = o[nt][0];
+      wpart[(warp * G + gq) * D + 8 * nt + 2 * tq + 1] = o[nt][1];
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G; e += blockDim.x) {
+    float M = -INFINITY;
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w][e]);
+    float L = 0.f;
+    for (int w = 0; w < 4; ++w) L += wm[w][e] == -INFINITY ? 0.f : wl[w][e] * exp2f(wm[w][e] - M);
+    sm[e] = M;
+    sl[e] = L;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+    const int h = e / D, d = e % D;
+    const float M = sm[h];
+    float acc = 0.f;
+    for (int w = 0; w < 4; ++w)
+      if (wm[w][h] != -INFINITY) acc += wpart[(w * G + h) * D + d] * exp2f(wm[w][h] - M);
+    po[h][d] = acc;
+  }
+  __syncthreads();
+  decode_finish<T, D, G, true, kPipeCluster>(p, po, sm, sl, nsplit_b, half, b, g);
+}
+
+template <typename T, int D, int G, bool FUSED, bool CLUSTER>
 int launch_one(const DecodeParams& p, cudaStream_t st) {
-  constexpr int smem = 2 * ROWS * D * static_cast<int>(sizeof(T));
+  constexpr bool TC = sizeof(T) == 2;  // bf16: streamed tensor-core kernel; fp32: exact FMA kernel
+  constexpr int smem = TC ? pipe_smem_bytes<D>() : 2 * ROWS * D * static_cast<int>(sizeof(T));
+  void (*kern)(const DecodeParams);
+  if constexpr (TC)
+    kern = k_decode_pipe<D, G, FUSED>;
+  else
+    kern = k_decode<T, D, G, FUSED, CLUSTER>;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (smem > 48 * 1024 && dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(k_decode<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return SEP_ECUDA;
     attr_set[dev] = true;
   }
-  dim3 grid(p.nsplit, p.Hkv, p.B);
-  k_decode<T, D, G><<<grid, kThreads, smem, st>>>(p);
+  const int ncl = TC ? kPipeCluster : (CLUSTER ? kMaxClusterSplits : 1);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(TC ? kPipeCluster : (CLUSTER ? kMaxClusterSplits : p.nsplit), p.Hkv, p.B);
+  cfg.blockDim = dim3(TC ? kPipeThreads : kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (ncl > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = ncl;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return SEP_ECUDA;
   return sep::launch_status();
 }
 
-template <typename T, int D>
+template <typename T, int D, bool FUSED = false>
 int launch_g(const DecodeParams& p, int G, cudaStream_t st) {
+  const bool cl = p.nsplit <= kMaxClusterSplits;
   switch (G) {
-    case 1: return launch_one<T, D, 1>(p, st);
-    case 2: return launch_one<T, D, 2>(p, st);
-    case 4: return launch_one<T, D, 4>(p, st);
-    case 8: return launch_one<T, D, 8>(p, st);
+    case 1: return cl ? launch_one<T, D, 1, FUSED, true>(p, st) : launch_one<T, D, 1, FUSED, false>(p, st);
+    case 2: return cl ? launch_one<T, D, 2, FUSED, true>(p, st) : launch_one<T, D, 2, FUSED, false>(p, st);
+    case 4: return cl ? launch_one<T, D, 4, FUSED, true>(p, st) : launch_one<T, D, 4, FUSED, false>(p, st);
+    case 8: return cl ? launch_one<T, D, 8, FUSED, true>(p, st) : launch_one<T, D, 8, FUSED, false>(p, st);
     default: return SEP_EINVAL;
   }
 }
 
-bool cache_ok(const sepcache* c) {
-  return c && c->k && c->v && c->counts && c->cap == c->cfg.a + c->cfg.s + c->cfg.past + c->cfg.w + 1 &&
-         c->layers >= 1 && c->B >= 1 && c->Hkv >= 1 && (c->D == 64 || c->D == 128) &&
-         (c->dtype == SEP_F32 || c->dtype == SEP_BF16);
-}
+bool cache_ok(const sepcache* c) { return sep::cache_valid(c); }
 
 struct WsLayout {
   size_t ml, o, ticket;
@@ -303,6 +790,11 @@ extern "C" int sep_attn_decode(const sepcache* c, int layer, const void* q, int 
   p.kc = c->k;
   p.vc = c->v;
   p.counts = c->counts;
+  p.cur = c->cur;
+  p.plan = c->plan;
+  p.k_new = nullptr;
+  p.v_new = nullptr;
+  p.layers = c->layers;
   p.out = out;
   p.lse = lse;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -322,6 +814,59 @@ extern "C" int sep_attn_decode(const sepcache* c, int layer, const void* q, int 
   if (c->dtype == SEP_BF16)
     return c->D == 64 ? launch_g<__nv_bfloat16, 64>(p, G, st) : launch_g<__nv_bfloat16, 128>(p, G, st);
   return c->D == 64 ? launch_g<float, 64>(p, G, st) : launch_g<float, 128>(p, G, st);
+}
+
+extern "C" int sep_attn_decode_step(const sepcache* c, int layer, const void* q,
+                                    const void* k_new, const void* v_new,
+                                    const uint8_t* is_sep_new, int Hq, float scale, void* out,
+                                    float* lse, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  if (!c) return SEP_ENULL;
+  if (!cache_ok(c)) return SEP_EINVAL;
+  if (layer < 0 || layer >= c->layers) return SEP_EINVAL;
+  if (Hq < 1 || Hq % c->Hkv != 0) return SEP_EINVAL;
+  const int G = Hq / c->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return SEP_EINVAL;
+  if (!q || !out || !workspace || !k_new || !v_new || (layer == 0 && !is_sep_new)) return SEP_ENULL;
+  if (!sep::aligned16(q) || !sep::aligned16(out) || !sep::aligned16(workspace) ||
+      !sep::aligned16(k_new) || !sep::aligned16(v_new))
+    return SEP_EALIGN;
+  const WsLayout w = ws_layout(c, Hq);
+  if (workspace_bytes < w.ml + w.o + w.ticket) return SEP_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (layer == 0) {
+    const int rc = sep::cache_advance(c, is_sep_new, st);
+    if (rc != SEP_OK) return rc;
+  }
+  DecodeParams p;
+  p.q = q;
+  p.kc = c->k;
+  p.vc = c->v;
+  p.counts = c->counts;
+  p.cur = c->cur;
+  p.plan = c->plan;
+  p.k_new = k_new;
+  p.v_new = v_new;
+  p.layers = c->layers;
+  p.out = out;
+  p.lse = lse;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  p.part_ml = reinterpret_cast<float*>(ws);
+  p.part_o = reinterpret_cast<float*>(ws + w.ml);
+  p.ticket = reinterpret_cast<int32_t*>(ws + w.ml + w.o);
+  p.err = sep::device_error_word();
+  p.layer = layer;
+  p.B = c->B;
+  p.Hq = Hq;
+  p.Hkv = c->Hkv;
+  p.cap = c->cap;
+  p.nsplit = (c->cap + ROWS - 1) / ROWS;
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(c->D));
+  p.scale_log2 = sc * 1.44269504088896340736f;
+  if (c->dtype == SEP_BF16)
+    return c->D == 64 ? launch_g<__nv_bfloat16, 64, true>(p, G, st)
+                      : launch_g<__nv_bfloat16, 128, true>(p, G, st);
+  return c->D == 64 ? launch_g<float, 64, true>(p, G, st) : launch_g<float, 128, true>(p, G, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -385,6 +930,11 @@ extern "C" int sep_attn_decode_noalloc(const sepcache* c, int layer, const void*
   p.kc = c->k;
   p.vc = c->v;
   p.counts = c->counts;
+  p.cur = c->cur;
+  p.plan = c->plan;
+  p.k_new = nullptr;
+  p.v_new = nullptr;
+  p.layers = c->layers;
   p.out = out;
   p.lse = lse;
   p.part_ml = reinterpret_cast<float*>(scratch);

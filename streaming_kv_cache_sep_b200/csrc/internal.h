@@ -4,6 +4,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "sepattn.h"
+
 namespace sep {
 int prefill_f32(const float* q, const float* k, const float* v, const int32_t* prefix,
                 const int32_t* idx, int B, int Hq, int Hkv, int S, int D, int a, int n,
@@ -12,4 +14,9 @@ size_t prefill_tc_workspace(int B, int Hkv, int S, int D);
 int prefill_tc(const void* q, const void* k, const void* v, const uint8_t* is_sep,
                const int32_t* prefix, const int32_t* idx, int B, int Hq, int Hkv, int S, int D,
                int a, int n, float scale, void* out, float* lse, void* workspace, cudaStream_t st);
+// Run the cache state machine for one token of every sequence (layer-0 part
+// of sepcache_append); defined in sepcache.cu.
+int cache_advance(const sepcache* c, const uint8_t* is_sep_new, cudaStream_t st);
+bool cache_valid(const sepcache* c);
+constexpr int kCachePlanHdr = 8;  // plan header words per sequence (see sepcache.cu)
 }  // namespace sep

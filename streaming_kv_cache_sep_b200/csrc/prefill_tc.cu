@@ -129,6 +129,20 @@ __device__ __forceinline__ Item make_item(const Params& p, int item) {
   return it;
 }
 
+// Does tile t keep any key of block j of its item's stream?  Gathered block
+// j: j*128 < nG_t.  Window block at `base`: [base, base+128) meets
+// [lo_t, last row of the tile] (keys below lo_t are the tile's gathered
+// keys; keys above its last row are causal-masked).  Blocks no tile keeps
+// are not streamed, and a tile skips the blocks it does not keep.
+__device__ __forceinline__ bool block_active(const Item& it, int t, int j, int S) {
+  if (j < it.nblk_g) return j * BN < (t ? it.nG[1] : it.nG[0]);
+  const int base = it.win_lo + (j - it.nblk_g) * BN;
+  const int q0 = t ? it.q0[1] : it.q0[0];
+  const int last = q0 + BM - 1 < S - 1 ? q0 + BM - 1 : S - 1;
+  const int lo = t ? it.lo[1] : it.lo[0];
+  return base <= last && base + BN - 1 >= lo;
+}
+
 // mask of bit positions c in [0, 32) with c <= x
 __device__ __forceinline__ uint32_t bits_le(int x) {
   return x < 0 ? 0u : (x >= 31 ? 0xffffffffu : (0xffffffffu >> (31 - x)));
@@ -258,11 +272,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // O_t += P_t V (block `vblk` of the global stream); the first PV of an
       // item overwrites O_t, so it waits until the previous item's epilogue
       // of tile t has read O_t.
+      bool v_ready = false;  // V of the block whose PVs are being issued has landed
       auto issue_pv = [&](int t, uint32_t vblk, bool first) -> bool {
         if (!sep::mbar_wait(&bars->p_full[t], (pphase >> t) & 1u, abort, p.err)) return false;
         pphase ^= 1u << t;
-        if (t == 0 && !sep::mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err))
+        if (!v_ready && !sep::mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err))
           return false;
+        v_ready = true;
         if (first && nitem > 0 && !sep::mbar_wait(&bars->o_empty[t], (nitem - 1) & 1, abort, p.err))
           return false;
         sep::tc_fence_after();
@@ -291,28 +307,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
         const Item it = make_item(p, item);
         if (!sep::mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
+        bool prev_a = false, prev_b = false;  // tile kept the previous block
+        bool pv_a = false, pv_b = false;      // tile already accumulated into O this item
         for (int j = 0; j < it.nblk; ++j, ++gblk) {
           if (!sep::mbar_wait(&bars->k_full[gblk % NST], (gblk / NST) & 1, abort, p.err)) {
             ok = false;
             break;
           }
           sep::tc_fence_after();
+          const bool act_a = block_active(it, 0, j, p.S), act_b = block_active(it, 1, j, p.S);
+          v_ready = false;
           // tile A: finish the previous block's PV, then this block's S
-          if (j > 0 && !(ok = issue_pv(0, gblk - 1, j == 1))) break;
-          issue_s(0, gblk);
-          if (j > 0) {
-            if (!(ok = issue_pv(1, gblk - 1, j == 1))) break;
-            sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
+          if (prev_a) {
+            if (!(ok = issue_pv(0, gblk - 1, !pv_a))) break;
+            pv_a = true;
           }
-          issue_s(1, gblk);
+          if (act_a) issue_s(0, gblk);
+          if (prev_b) {
+            if (!(ok = issue_pv(1, gblk - 1, !pv_b))) break;
+            pv_b = true;
+          }
+          if (j > 0) sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
+          if (act_b) issue_s(1, gblk);
           sep::mma_commit(&bars->k_empty[gblk % NST]);
           if (j == it.nblk - 1) sep::mma_commit(&bars->q_empty);
+          prev_a = act_a;
+          prev_b = act_b;
         }
         if (!ok) break;
         // last block's PV of both tiles, then hand O to the epilogues
-        if (!(ok = issue_pv(0, gblk - 1, it.nblk == 1))) break;
+        v_ready = false;
+        if (prev_a && !(ok = issue_pv(0, gblk - 1, !pv_a))) break;
         sep::mma_commit(&bars->o_full[0]);
-        if (!(ok = issue_pv(1, gblk - 1, it.nblk == 1))) break;
+        if (prev_b && !(ok = issue_pv(1, gblk - 1, !pv_b))) break;
         sep::mma_commit(&bars->o_full[1]);
         sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
       }
@@ -330,26 +357,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
       const Item it = make_item(p, item);
-      const int i = (t ? it.q0[1] : it.q0[0]) + row;
-      const int ie = i < p.S ? i : p.S - 1;  // rows past the end mask like the last row
-      const uint8_t* flags = p.is_sep + static_cast<int64_t>(it.b) * p.S;
+      // this tile's scalars (the rest of the item is not needed here)
+      const int my_q0 = t ? it.q0[1] : it.q0[0];
       const int my_lo = t ? it.lo[1] : it.lo[0];
       const int my_nG = t ? it.nG[1] : it.nG[0];
+      const int my_last = my_q0 + BM - 1 < p.S - 1 ? my_q0 + BM - 1 : p.S - 1;
+      const int nblk_g = it.nblk_g, nblk = it.nblk, win_lo = it.win_lo;
+      const int h = t ? it.h[1] : it.h[0];
+      const int b = it.b;
+      const int i = my_q0 + row;
+      const int ie = i < p.S ? i : p.S - 1;  // rows past the end mask like the last row
+      const uint8_t* flags = p.is_sep + static_cast<int64_t>(b) * p.S;
       float m_ref = -INFINITY, l = 0.f;
-      for (int j = 0; j < it.nblk; ++j) {
+      // separator-or-initial flags of 4 positions (base + 32c + lane) per lane,
+      // loaded one window block ahead of their use
+      auto load_flags = [&](int base) -> uint32_t {
+        uint32_t f = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int pos = base + 32 * c + lane;
+          if (pos < p.S && (flags[pos] != 0 || pos < p.a)) f |= 1u << c;
+        }
+        return f;
+      };
+      uint32_t fl_next = load_flags(win_lo), fl_cur = 0;
+      for (int j = 0; j < nblk; ++j) {
+        if (j >= nblk_g) {
+          fl_cur = fl_next;
+          if (j + 1 < nblk) fl_next = load_flags(win_lo + (j + 1 - nblk_g) * BN);
+        }
+        // skip blocks this tile keeps nothing of (see block_active)
+        if (j < nblk_g ? j * BN >= my_nG
+                       : (win_lo + (j - nblk_g) * BN > my_last ||
+                          win_lo + (j - nblk_g) * BN + BN - 1 < my_lo))
+          continue;
         uint32_t keep[4];
-        if (j < it.nblk_g) {
+        if (j < nblk_g) {
           const int valid = my_nG - j * BN;
 #pragma unroll
           for (int c = 0; c < 4; ++c) keep[c] = bits_le(valid - 1 - 32 * c);
         } else {
-          const int base = it.win_lo + (j - it.nblk_g) * BN;
+          const int base = win_lo + (j - nblk_g) * BN;
           const int ihi = ie - base, ilo = ie - p.n - base, jlo = my_lo - base;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const int pos = base + 32 * c + lane;
-            const bool f = pos < p.S && (flags[pos] != 0 || pos < p.a);
-            const uint32_t sepbits = __ballot_sync(0xffffffffu, f);
+            const uint32_t sepbits = __ballot_sync(0xffffffffu, (fl_cur >> c) & 1u);
             keep[c] = bits_le(ihi - 32 * c) & (~bits_le(ilo - 32 * c) | sepbits) &
                       ~bits_le(jlo - 1 - 32 * c);
           }
@@ -360,78 +412,151 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         sphase ^= 1;
         sep::tc_fence_after();
-        // pass 1: masked row maximum of the raw scores (8 independent chains)
-        float mx[8];
+        // Fast path (after the block where a row first saw a key): one pass
+        // over S against the running reference m_ref, P kept in registers
+        // until every score of the row is known to be within 2^8 of m_ref.
+        // Otherwise (first block, or a score that grew past 2^8): the exact
+        // two-pass path that moves the reference and rescales O.
+        bool fast_done = false;
+        if (__all_sync(0xffffffffu, m_ref != -INFINITY)) {
+          uint32_t pk[64];
+          uint32_t ra[32], rb[32];
+          float sm[8], pm[2];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
-        // (loops over the 4 column groups stay rolled: one group of scores in
-        // registers at a time; the keep words rotate instead of being indexed)
-        uint32_t k0 = keep[0], k1 = keep[1], k2 = keep[2], k3 = keep[3];
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          sep::tmem_ld32(s_col + 32 * c, r);
-          sep::tmem_wait_ld();
+          for (int u = 0; u < 8; ++u) sm[u] = 0.f;
+          pm[0] = pm[1] = 0.f;
+          sep::tmem_ld32(s_col, ra);
+          sep::tmem_wait_ld_r32(ra);
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            mx[e & 7] = fmaxf(mx[e & 7], (k0 >> e) & 1u ? __uint_as_float(r[e]) : -INFINITY);
-          k0 = k1;
-          k1 = k2;
-          k2 = k3;
-        }
-        const float mblk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
-                           p.scale_log2;
-        float alpha = 1.f;
-        const bool grow = mblk > m_ref + kRescaleLog2;
-        if (grow) {
-          alpha = sep::ex2_approx(m_ref - mblk);  // 0 while m_ref is -inf
-          m_ref = mblk;
-        }
-        // S_t of this block was issued after this tile's previous P*V, and
-        // MMAs complete in order, so that P*V is done: O_t may be rescaled.
-        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          for (int c = 0; c < 4; ++c) {
+            uint32_t* cur = (c & 1) ? rb : ra;
+            uint32_t* nxt = (c & 1) ? ra : rb;
+            if (c < 3) sep::tmem_ld32(s_col + 32 * (c + 1), nxt);  // overlaps this group's math
+            const uint32_t kc = keep[c];
+            if (__all_sync(0xffffffffu, kc == 0u)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            sep::tmem_ld32(o_col + 32 * c, o);
-            sep::tmem_wait_ld();
+              for (int e = 0; e < 16; ++e) pk[16 * c + e] = 0u;
+            } else if (__all_sync(0xffffffffu, kc == 0xffffffffu)) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            sep::tmem_st32(o_col + 32 * c, o);
+              for (int e = 0; e < 32; e += 2) {
+                const float p0 = sep::ex2_approx(fmaf(__uint_as_float(cur[e]), p.scale_log2, -m_ref));
+                const float p1 = sep::ex2_approx(fmaf(__uint_as_float(cur[e + 1]), p.scale_log2, -m_ref));
+                sm[e & 7] += p0;
+                sm[(e + 1) & 7] += p1;
+                pm[0] = fmaxf(pm[0], p0);
+                pm[1] = fmaxf(pm[1], p1);
+                pk[16 * c + (e >> 1)] = sep::pack_bf16x2(p0, p1);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; e += 2) {
+                const float x0 = (kc >> e) & 1u ? __uint_as_float(cur[e]) : -INFINITY;
+                const float x1 = (kc >> (e + 1)) & 1u ? __uint_as_float(cur[e + 1]) : -INFINITY;
+                const float p0 = sep::ex2_approx(fmaf(x0, p.scale_log2, -m_ref));
+                const float p1 = sep::ex2_approx(fmaf(x1, p.scale_log2, -m_ref));
+                sm[e & 7] += p0;
+                sm[(e + 1) & 7] += p1;
+                pm[0] = fmaxf(pm[0], p0);
+                pm[1] = fmaxf(pm[1], p1);
+                pk[16 * c + (e >> 1)] = sep::pack_bf16x2(p0, p1);
+              }
+            }
+            if (c < 3) sep::tmem_wait_ld_r32(nxt);
+          }
+          const float pmax = fmaxf(pm[0], pm[1]);
+          // 2^8 bound on P (the lazy-rescale rule); a NaN here also falls back
+          if (!__any_sync(0xffffffffu, !(pmax <= 256.f))) {
+            l += ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
+            sep::tmem_st32(s_col, pk);
+            sep::tmem_st32(s_col + 32, pk + 32);
+            fast_done = true;
           }
         }
-        const float mr = m_ref == -INFINITY ? 0.f : m_ref;
-        float sm[8];
+        if (!fast_done) {
+          // pass 1: masked row maximum of the raw scores (8 independent chains)
+          float mx[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) sm[u] = 0.f;
-        // pass 2: P = 2^(s*scale - m) as bf16 pairs written over S_t: keys
-        // [32c, 32c+32) go to columns [16c, 16c+16), which hold scores of
-        // keys already read back
-        k0 = keep[0];
-        k1 = keep[1];
-        k2 = keep[2];
+          for (int u = 0; u < 8; ++u) mx[u] = -INFINITY;
+          // (loops over the 4 column groups stay rolled: one group of scores in
+          // registers at a time; the keep words rotate instead of being indexed)
+          uint32_t k0 = keep[0], k1 = keep[1], k2 = keep[2], k3 = keep[3];
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          sep::tmem_ld32(s_col + 32 * c, r);
-          sep::tmem_wait_ld();
+          for (int c = 0; c < 4; ++c) {
+            if (__any_sync(0xffffffffu, k0 != 0u)) {
+              uint32_t r[32];
+              sep::tmem_ld32(s_col + 32 * c, r);
+              sep::tmem_wait_ld_r32(r);
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const float x0 = (k0 >> e) & 1u ? __uint_as_float(r[e]) : -INFINITY;
-            const float x1 = (k0 >> (e + 1)) & 1u ? __uint_as_float(r[e + 1]) : -INFINITY;
-            const float p0 = sep::ex2_approx(fmaf(x0, p.scale_log2, -mr));
-            const float p1 = sep::ex2_approx(fmaf(x1, p.scale_log2, -mr));
-            sm[e & 7] += p0;
-            sm[(e + 1) & 7] += p1;
-            r[e >> 1] = sep::pack_bf16x2(p0, p1);
+              for (int e = 0; e < 32; ++e)
+                mx[e & 7] = fmaxf(mx[e & 7], (k0 >> e) & 1u ? __uint_as_float(r[e]) : -INFINITY);
+            }
+            k0 = k1;
+            k1 = k2;
+            k2 = k3;
           }
-          sep::tmem_st16(s_col + 16 * c, r);
-          k0 = k1;
-          k1 = k2;
-          k2 = keep[3];
+          const float mblk = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+                             p.scale_log2;
+          float alpha = 1.f;
+          const bool grow = mblk > m_ref + kRescaleLog2;
+          if (grow) {
+            alpha = sep::ex2_approx(m_ref - mblk);  // 0 while m_ref is -inf
+            m_ref = mblk;
+          }
+          // S_t of this block was issued after this tile's previous P*V, and
+          // MMAs complete in order, so that P*V is done: O_t may be rescaled.
+          if (j > 0 && __any_sync(0xffffffffu, grow)) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t o[32];
+              sep::tmem_ld32(o_col + 32 * c, o);
+              sep::tmem_wait_ld_r32(o);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              sep::tmem_st32(o_col + 32 * c, o);
+            }
+          }
+          const float mr = m_ref == -INFINITY ? 0.f : m_ref;
+          float sm[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) sm[u] = 0.f;
+          // pass 2: P = 2^(s*scale - m) as bf16 pairs written over S_t: keys
+          // [32c, 32c+32) go to columns [16c, 16c+16), which hold scores of
+          // keys already read back
+          k0 = keep[0];
+          k1 = keep[1];
+          k2 = keep[2];
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            if (!__any_sync(0xffffffffu, k0 != 0u)) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) r[e] = 0u;
+              sep::tmem_st16(s_col + 16 * c, r);
+              k0 = k1;
+              k1 = k2;
+              k2 = keep[3];
+              continue;
+            }
+            sep::tmem_ld32(s_col + 32 * c, r);
+            sep::tmem_wait_ld_r32(r);
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+              const float x0 = (k0 >> e) & 1u ? __uint_as_float(r[e]) : -INFINITY;
+              const float x1 = (k0 >> (e + 1)) & 1u ? __uint_as_float(r[e + 1]) : -INFINITY;
+              const float p0 = sep::ex2_approx(fmaf(x0, p.scale_log2, -mr));
+              const float p1 = sep::ex2_approx(fmaf(x1, p.scale_log2, -mr));
+              sm[e & 7] += p0;
+              sm[(e + 1) & 7] += p1;
+              r[e >> 1] = sep::pack_bf16x2(p0, p1);
+            }
+            sep::tmem_st16(s_col + 16 * c, r);
+            k0 = k1;
+            k1 = k2;
+            k2 = keep[3];
+          }
+          l = l * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
         }
-        l = l * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
         sep::tmem_wait_st();
         sep::tc_fence_before();
         sep::mbar_arrive(&bars->p_full[t]);
@@ -444,13 +569,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       sep::tc_fence_after();
       const float inv = 1.f / l;
-      const int h = t ? it.h[1] : it.h[0];
-      __nv_bfloat16* orow = p.out + (static_cast<int64_t>(it.b * p.Hq + h) * p.S + i) * D;
+      __nv_bfloat16* orow = p.out + (static_cast<int64_t>(b * p.Hq + h) * p.S + i) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         sep::tmem_ld32(o_col + 32 * c, o);
-        sep::tmem_wait_ld();
+        sep::tmem_wait_ld_r32(o);
         if (i < p.S) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -464,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (p.lse && i < p.S)
-        p.lse[static_cast<int64_t>(it.b * p.Hq + h) * p.S + i] =
+        p.lse[static_cast<int64_t>(b * p.Hq + h) * p.S + i] =
             (m_ref + __log2f(l)) * 0.69314718055994530942f;
       sep::tc_fence_before();
       sep::mbar_arrive(&bars->o_empty[t]);

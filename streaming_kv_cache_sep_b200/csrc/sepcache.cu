@@ -1,4 +1,4 @@
-// The four-block SepCache: bookkeeping, token append and in-place compaction.
+// The four-block SepCache: bookkeeping, token append and flush compaction.
 //
 // Blocks (xugj520 SepLLM article, section 3.3 table; KV-manager steps of the
 // "HKUDS047: SepLLM ..." study, section "KV Cache Manager"):
@@ -10,21 +10,28 @@
 //   L  local window: the newest w tokens.
 // Rows of each (layer, b, kv head) are stored I | S | P | L in increasing
 // position order.  P and L are one contiguous run of recent positions, so a
-// token sliding from L to P moves no data; only a flush moves rows, and it
-// does so in place with an order-preserving stream compaction (every row
-// moves down or stays, and rows are processed in ascending order).
+// token sliding from L to P moves no data; only a flush moves rows.  The
+// K/V rows live in two buffers per sequence: a flush copies the surviving
+// rows, in order, from the current buffer into the other one (out of place,
+// so every row can be copied in parallel and the decode of the same step can
+// fetch its rows from either side without hazards), and that buffer becomes
+// current.  The surviving rows are found with an order-preserving
+// warp-ballot stream compaction of the I | S | P | L rows.
 //
 // Bookkeeping is shared by all layers: sepcache_append at layer 0 runs the
 // state machine for the new token and records this step's plan (the row the
-// token is written to and, on a flush, the source row of every destination
-// row); every layer's append/compact then applies that plan to its K/V.
+// token is written to, the source and destination buffers and, on a flush,
+// the source row of every destination row); every layer's append/compact
+// (or the fused decode step) then applies that plan to its K/V.
 #include <string.h>
 
 #include "common.cuh"
 
 namespace {
 
-constexpr int kPlanHdr = 4;  // plan[b] = {flush, slot, new_len, first_moved_row, src[cap]...}
+// plan[b] = {flush, slot, new_len, nI, src_buf, dst_buf, -, -, src row of each
+// destination row (flush steps)...}
+constexpr int kPlanHdr = 8;
 
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
@@ -36,8 +43,8 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__ flag,
                                 int32_t* __restrict__ counts, int32_t* __restrict__ plan,
                                 int64_t* __restrict__ step, int32_t* __restrict__ status,
-                                const uint8_t* __restrict__ is_sep_new, int B, int cap, int a,
-                                int s, int past, int w) {
+                                int32_t* __restrict__ cur, const uint8_t* __restrict__ is_sep_new,
+                                int B, int cap, int a, int s, int past, int w) {
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
   if (b >= B) return;
@@ -47,6 +54,7 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
   uint8_t* fl = flag + static_cast<int64_t>(b) * cap;
   int nI = cnt[0], nS = cnt[1], nP = cnt[2], nL = cnt[3];
   const int64_t t = step[b];
+  const int cb = cur[b] & 1;
   const uint8_t f = is_sep_new[b] ? 1 : 0;
   int len = nI + nS + nP + nL;
   const bool bad = nI < 0 || nS < 0 || nP < 0 || nL < 0 || nI > a || nS > s || nP > past ||
@@ -59,6 +67,7 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
       pl[1] = -1;
       pl[2] = len > cap ? cap : (len < 0 ? 0 : len);
       pl[3] = 0;
+      pl[4] = pl[5] = cb;
     }
     return;
   }
@@ -90,6 +99,7 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
       ncand += __popc(__ballot_sync(0xffffffffu, r < eP && fl[r] != 0));
     }
     const int drop = ncand > s ? ncand - s : 0;
+    for (int r = lane; r < nI; r += 32) pl[kPlanHdr + r] = r;  // initial rows keep their place
     int rank = 0, dst = nI;
     for (int base = nI; base < len; base += 32) {
       const int r = base + lane;
@@ -98,8 +108,8 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
       const uint8_t my_flag = valid ? fl[r] : 0;
       const bool is_cand = valid && r < eP && (r < eS || my_flag != 0);
       const bool is_local = valid && r >= eP;
-      const uint32_t cb = __ballot_sync(0xffffffffu, is_cand);
-      const int my_rank = rank + __popc(cb & lanemask_lt());
+      const uint32_t candb = __ballot_sync(0xffffffffu, is_cand);
+      const int my_rank = rank + __popc(candb & lanemask_lt());
       const bool keep = is_local || (is_cand && my_rank >= drop);
       const uint32_t kb = __ballot_sync(0xffffffffu, keep);
       const int d = dst + __popc(kb & lanemask_lt());
@@ -110,7 +120,7 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
         pl[kPlanHdr + d] = r;
       }
       __syncwarp();
-      rank += __popc(cb);
+      rank += __popc(candb);
       dst += __popc(kb);
     }
     new_len = dst;
@@ -127,6 +137,9 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
     pl[1] = slot;
     pl[2] = new_len;
     pl[3] = nI;
+    pl[4] = cb;                   // rows are read from (and the token written to)
+    pl[5] = flush ? 1 - cb : cb;  // rows are current in after this step
+    cur[b] = pl[5];
     cnt[0] = nI;
     cnt[1] = nS;
     cnt[2] = nP;
@@ -135,72 +148,72 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
   }
 }
 
-// Write the new token's K and V rows of one layer at this step's slot.
+// Byte offset of row 0 of (buffer, layer, b, kv head).
+__device__ __forceinline__ int64_t row0(int buf, int layer, int b, int g, int layers, int B,
+                                        int Hkv, int cap, int row_bytes) {
+  return ((((static_cast<int64_t>(buf) * layers + layer) * B + b) * Hkv + g) * cap) * row_bytes;
+}
+
+// Write the new token's K and V rows of one layer at this step's slot of the
+// buffer the step reads from.
 __global__ void k_cache_write(uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
                               const uint8_t* __restrict__ k_new, const uint8_t* __restrict__ v_new,
-                              const int32_t* __restrict__ plan, int layer, int B, int Hkv, int cap,
-                              int row_bytes) {
+                              const int32_t* __restrict__ plan, int layer, int layers, int B,
+                              int Hkv, int cap, int row_bytes) {
   const int b = blockIdx.x;
-  const int slot = plan[static_cast<int64_t>(b) * (cap + kPlanHdr) + 1];
+  const int32_t* pl = plan + static_cast<int64_t>(b) * (cap + kPlanHdr);
+  const int slot = pl[1], sb = pl[4] & 1;
   if (slot < 0 || slot >= cap) return;
   const int ch = row_bytes / 16;
   const int per = Hkv * ch;
   for (int e = threadIdx.x; e < 2 * per; e += blockDim.x) {
     const int which = e / per, g = (e % per) / ch, c = e % ch;
-    const int64_t dst = ((static_cast<int64_t>(layer) * B + b) * Hkv + g) * cap + slot;
-    const int64_t src = static_cast<int64_t>(b) * Hkv + g;
-    const uint4 val =
-        reinterpret_cast<const uint4*>((which ? v_new : k_new) + src * row_bytes)[c];
-    reinterpret_cast<uint4*>((which ? vc : kc) + dst * row_bytes)[c] = val;
+    const int64_t dst = row0(sb, layer, b, g, layers, B, Hkv, cap, row_bytes) +
+                        static_cast<int64_t>(slot) * row_bytes;
+    const int64_t src = (static_cast<int64_t>(b) * Hkv + g) * row_bytes;
+    const uint4 val = reinterpret_cast<const uint4*>((which ? v_new : k_new) + src)[c];
+    reinterpret_cast<uint4*>((which ? vc : kc) + dst)[c] = val;
   }
 }
 
-// Apply this step's flush to one layer: one CTA per (b, kv head, K|V).
-// Destination row r takes source row plan.src[r] >= r; rows are handled in
-// ascending chunks and each chunk is read completely before it is written,
-// so no source row is overwritten before it is read.
+// Apply this step's flush to one layer: destination row r of the other
+// buffer takes source row plan.src[r] of the current one.  Out of place, so
+// every 16-byte chunk is copied independently.  Grid: (chunks, kv head, b).
 __global__ void __launch_bounds__(256) k_cache_compact(uint8_t* __restrict__ kc,
                                                        uint8_t* __restrict__ vc,
                                                        const int32_t* __restrict__ plan, int layer,
-                                                       int B, int Hkv, int cap, int row_bytes) {
-  const int b = blockIdx.x / (2 * Hkv);
-  const int g = (blockIdx.x / 2) % Hkv;
-  const int which = blockIdx.x & 1;
+                                                       int layers, int B, int Hkv, int cap,
+                                                       int row_bytes) {
+  const int g = blockIdx.y, b = blockIdx.z;
   const int32_t* pl = plan + static_cast<int64_t>(b) * (cap + kPlanHdr);
   if (pl[0] == 0) return;
-  const int new_len = pl[2], first = pl[3];
+  const int new_len = pl[2], sb = pl[4] & 1, db = pl[5] & 1;
   const int ch = row_bytes / 16;
-  const int rows_per = 256 / ch;
-  uint8_t* base = (which ? vc : kc) +
-                  ((static_cast<int64_t>(layer) * B + b) * Hkv + g) * cap * row_bytes;
-  const int rr = threadIdx.x / ch, c = threadIdx.x % ch;
-  for (int r0 = first; r0 < new_len; r0 += rows_per) {
-    const int r = r0 + rr;
-    const bool act = rr < rows_per && r < new_len;
-    int src = r;
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (act) {
-      src = pl[kPlanHdr + r];
-      if (src != r && src > r && src < cap) val = reinterpret_cast<const uint4*>(base + static_cast<int64_t>(src) * row_bytes)[c];
-    }
-    __syncthreads();
-    if (act && src != r && src > r && src < cap)
-      reinterpret_cast<uint4*>(base + static_cast<int64_t>(r) * row_bytes)[c] = val;
-    __syncthreads();
+  const int64_t sbase = row0(sb, layer, b, g, layers, B, Hkv, cap, row_bytes);
+  const int64_t dbase = row0(db, layer, b, g, layers, B, Hkv, cap, row_bytes);
+  const int total = 2 * new_len * ch;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+    const int which = e / (new_len * ch);
+    const int r = (e / ch) % new_len, c = e % ch;
+    const int src = pl[kPlanHdr + r];
+    if (src < 0 || src >= cap) continue;
+    uint8_t* base = which ? vc : kc;
+    const uint4 val = reinterpret_cast<const uint4*>(base + sbase + static_cast<int64_t>(src) * row_bytes)[c];
+    reinterpret_cast<uint4*>(base + dbase + static_cast<int64_t>(r) * row_bytes)[c] = val;
   }
 }
 
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct Sizes {
-  size_t k, v, pos, flag, counts, plan, step, status;
-  size_t total() const { return k + v + pos + flag + counts + plan + step + status; }
+  size_t k, v, pos, flag, counts, plan, step, status, cur;
+  size_t total() const { return k + v + pos + flag + counts + plan + step + status + cur; }
 };
 
 Sizes sizes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
   const int64_t cap = static_cast<int64_t>(cfg.a) + cfg.s + cfg.past + cfg.w + 1;
   Sizes z;
-  z.k = round256(static_cast<size_t>(layers) * B * Hkv * cap * D * sep::elem_bytes(dtype));
+  z.k = round256(2 * static_cast<size_t>(layers) * B * Hkv * cap * D * sep::elem_bytes(dtype));
   z.v = z.k;
   z.pos = round256(static_cast<size_t>(B) * cap * 4);
   z.flag = round256(static_cast<size_t>(B) * cap);
@@ -208,6 +221,7 @@ Sizes sizes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
   z.plan = round256(static_cast<size_t>(B) * (cap + kPlanHdr) * 4);
   z.step = round256(static_cast<size_t>(B) * 8);
   z.status = 256;
+  z.cur = round256(static_cast<size_t>(B) * 4);
   return z;
 }
 
@@ -222,6 +236,7 @@ bool cfg_ok(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
 
 bool cache_ok(const sepcache* c) {
   return c && c->k && c->v && c->pos && c->flag && c->counts && c->plan && c->step && c->status &&
+         c->cur &&
          cfg_ok(c->cfg, c->layers, c->B, c->Hkv, c->D, c->dtype) &&
          c->cap == c->cfg.a + c->cfg.s + c->cfg.past + c->cfg.w + 1;
 }
@@ -261,6 +276,8 @@ extern "C" int sepcache_carve(sepcache* cache, void* buffer, size_t bytes, sep_c
   cache->step = reinterpret_cast<int64_t*>(p);
   p += z.step;
   cache->status = reinterpret_cast<int32_t*>(p);
+  p += z.status;
+  cache->cur = reinterpret_cast<int32_t*>(p);
   cache->layers = layers;
   cache->B = B;
   cache->Hkv = Hkv;
@@ -280,9 +297,20 @@ extern "C" int sepcache_init(const sepcache* c, void* stream) {
             cudaMemsetAsync(c->counts, 0, c->B * 16, st) == cudaSuccess &&
             cudaMemsetAsync(c->plan, 0, c->B * (cap + kPlanHdr) * 4, st) == cudaSuccess &&
             cudaMemsetAsync(c->step, 0, c->B * 8, st) == cudaSuccess &&
-            cudaMemsetAsync(c->status, 0, 4, st) == cudaSuccess;
+            cudaMemsetAsync(c->status, 0, 4, st) == cudaSuccess &&
+            cudaMemsetAsync(c->cur, 0, c->B * 4, st) == cudaSuccess;
   return ok ? SEP_OK : SEP_ECUDA;
 }
+
+namespace sep {
+int cache_advance(const sepcache* c, const uint8_t* is_sep_new, cudaStream_t st) {
+  k_cache_advance<<<c->B, 32, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step, c->status,
+                                        c->cur, is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
+                                        c->cfg.past, c->cfg.w);
+  return launch_status();
+}
+bool cache_valid(const sepcache* c) { return cache_ok(c); }
+}  // namespace sep
 
 extern "C" int sepcache_append(const sepcache* c, int layer, const void* k_new, const void* v_new,
                                const uint8_t* is_sep_new, void* stream) {
@@ -293,7 +321,7 @@ extern "C" int sepcache_append(const sepcache* c, int layer, const void* k_new, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (layer == 0) {
     k_cache_advance<<<c->B, 32, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step, c->status,
-                                          is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
+                                          c->cur, is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
                                           c->cfg.past, c->cfg.w);
     if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   }
@@ -301,8 +329,8 @@ extern "C" int sepcache_append(const sepcache* c, int layer, const void* k_new, 
   const int threads = 2 * c->Hkv * row_bytes / 16 < 512 ? 2 * c->Hkv * row_bytes / 16 : 512;
   k_cache_write<<<c->B, (threads + 31) / 32 * 32, 0, st>>>(
       static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v),
-      static_cast<const uint8_t*>(k_new), static_cast<const uint8_t*>(v_new), c->plan, layer, c->B,
-      c->Hkv, c->cap, row_bytes);
+      static_cast<const uint8_t*>(k_new), static_cast<const uint8_t*>(v_new), c->plan, layer,
+      c->layers, c->B, c->Hkv, c->cap, row_bytes);
   return sep::launch_status();
 }
 
@@ -310,9 +338,10 @@ extern "C" int sepcache_compact(const sepcache* c, int layer, void* stream) {
   if (!cache_ok(c)) return c ? SEP_EINVAL : SEP_ENULL;
   if (layer < 0 || layer >= c->layers) return SEP_EINVAL;
   const int row_bytes = c->D * sep::elem_bytes(c->dtype);
-  k_cache_compact<<<c->B * c->Hkv * 2, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), c->plan, layer, c->B, c->Hkv,
-      c->cap, row_bytes);
+  dim3 grid(2, c->Hkv, c->B);
+  k_cache_compact<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), c->plan, layer, c->layers, c->B,
+      c->Hkv, c->cap, row_bytes);
   return sep::launch_status();
 }
 

@@ -83,15 +83,16 @@ def test_cache_layout_and_validation(sl):
     nb = L.sepcache_bytes(cfg, 32, 16, 8, 128, 1)
     cap = 4 + 64 + 128 + 256 + 1
     kv = 32 * 16 * 8 * cap * 128 * 2
-    assert nb >= 2 * kv and nb < 2 * kv + 256 * 1024
+    assert nb >= 4 * kv and nb < 4 * kv + 256 * 1024  # K and V, two buffers each
     assert L.sepcache_bytes(sl.SepCacheCfg(4, 64, 128, 0), 1, 1, 1, 128, 1) == 0  # w >= 1
     assert L.sepcache_bytes(sl.SepCacheCfg(-1, 64, 128, 4), 1, 1, 1, 128, 1) == 0
     assert L.sepcache_bytes(cfg, 1, 1, 1, 96, 1) == 0
     c = sl._SepCacheC()
     base = ctypes.c_void_p(1 << 20)
     assert L.sepcache_carve(ctypes.byref(c), base, nb, cfg, 32, 16, 8, 128, 1) == 0
-    assert c.cap == cap and c.k == (1 << 20) and c.v - c.k >= kv
-    assert all(getattr(c, f) % 256 == 0 for f in ("pos", "flag", "counts", "plan", "step", "status"))
+    assert c.cap == cap and c.k == (1 << 20) and c.v - c.k >= 2 * kv
+    assert all(getattr(c, f) % 256 == 0
+               for f in ("pos", "flag", "counts", "plan", "step", "status", "cur"))
     assert L.sepcache_carve(ctypes.byref(c), ctypes.c_void_p((1 << 20) + 16), nb, cfg, 32, 16, 8,
                             128, 1) == -3
     assert L.sepcache_carve(ctypes.byref(c), base, nb - 1, cfg, 32, 16, 8, 128, 1) == -1

@@ -30,7 +30,8 @@ def sl():
 class Stream:
     """Drive a SepCache through the C ABI with ring-cycled synthetic inputs."""
 
-    def __init__(self, sl, a, s, past, w, B, Hkv, Hq, D, layers, dtype, seed, T):
+    def __init__(self, sl, a, s, past, w, B, Hkv, Hq, D, layers, dtype, seed, T, fused=False):
+        self.fused = fused
         self.sl = sl
         self.cfg = dict(a=a, s=s, past=past, w=w)
         self.B, self.Hkv, self.Hq, self.D, self.layers = B, Hkv, Hq, D, layers
@@ -54,7 +55,13 @@ class Stream:
         t, r = self.t, self.t % RING
         outs = {}
         for l in range(self.layers):
-            self.cache.append(l, self.dk[l][r], self.dv[l][r], self.dflags[t] if l == 0 else None)
+            f = self.dflags[t] if l == 0 else None
+            if self.fused:  # one launch per layer: append + compact + decode
+                o = self.cache.decode_step(l, self.dq[l][r], self.dk[l][r], self.dv[l][r], f)
+                if l in decode_layers:
+                    outs[l] = o
+                continue
+            self.cache.append(l, self.dk[l][r], self.dv[l][r], f)
             self.cache.compact(l)
             if l in decode_layers:
                 outs[l] = self.cache.decode(l, self.dq[l][r])
@@ -80,14 +87,15 @@ def _check_meta(st, snap, k):
 
 def _check_kv(st, snap, k):
     c = st.cache
-    K, V = c.k.cpu(), c.v.cpu()
+    K, V, cur = c.k.cpu(), c.v.cpu(), c.cur.cpu()
     for b in range(st.B):
         n = int(snap["counts"][k, b].sum())
         pos = snap["pos"][k, b, :n]
+        cb = int(cur[b])
         for l in range(st.layers):
             kr, vr = st.kv_rows(l, pos, b)
-            assert torch.equal(K[l, b, :, :n], kr), (k, b, l)
-            assert torch.equal(V[l, b, :, :n], vr), (k, b, l)
+            assert torch.equal(K[cb, l, b, :, :n], kr), (k, b, l)
+            assert torch.equal(V[cb, l, b, :, :n], vr), (k, b, l)
 
 
 def _check_decode(st, snap, k, outs, t):
@@ -119,11 +127,13 @@ SMALL = [
 ]
 
 
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
 @pytest.mark.parametrize("shape", SMALL, ids=lambda s: "_".join(map(str, s[:8])))
-def test_small_caches_every_step(sl, shape):
+def test_small_caches_every_step(sl, shape, fused):
     a, s, past, w, B, Hkv, Hq, D, dtype = shape
     T = 400
-    st = Stream(sl, a, s, past, w, B, Hkv, Hq, D, 2, dtype, seed=a * 100 + s + past + w, T=T)
+    st = Stream(sl, a, s, past, w, B, Hkv, Hq, D, 2, dtype, seed=a * 100 + s + past + w, T=T,
+                fused=fused)
     snap = oracle.sepcache_simulate(st.flags, a, s, past, w, np.arange(T))
     for t in range(T):
         outs = st.step(decode_layers=(0, 1))
@@ -135,12 +145,14 @@ def test_small_caches_every_step(sl, shape):
     assert sl.device_status() == 0
 
 
-def test_llama3_8b_shape_first_2000_steps(sl):
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_llama3_8b_shape_first_2000_steps(sl, fused):
     cfg = synth.WORKLOADS["decode_llama3_8b_b16_l32_t65536_d128_bf16"]
     a, s, past, w = cfg["a"], cfg["s"], cfg["past"], cfg["w"]
     T = 2000
     st = Stream(sl, a, s, past, w, cfg["B"], cfg["Hkv"], cfg["Hq"], cfg["D"], 2, torch.bfloat16,
-                seed=synth.WORKLOAD_SEED["decode_llama3_8b_b16_l32_t65536_d128_bf16"], T=T)
+                seed=synth.WORKLOAD_SEED["decode_llama3_8b_b16_l32_t65536_d128_bf16"], T=T,
+                fused=fused)
     snap = oracle.sepcache_simulate(st.flags, a, s, past, w, np.arange(T))
     flushes = {a + w + k * (past + 1) - 1 for k in range(1, 20)}
     near_flush = {t + d for t in flushes for d in (-2, -1, 0, 1, 2)}
@@ -159,7 +171,8 @@ def test_llama3_8b_shape_full_stream_checkpoints(sl):
     cfg = synth.WORKLOADS["decode_llama3_8b_b16_l32_t65536_d128_bf16"]
     a, s, past, w, T = cfg["a"], cfg["s"], cfg["past"], cfg["w"], cfg["T"]
     st = Stream(sl, a, s, past, w, cfg["B"], cfg["Hkv"], cfg["Hq"], cfg["D"], 2, torch.bfloat16,
-                seed=synth.WORKLOAD_SEED["decode_llama3_8b_b16_l32_t65536_d128_bf16"] + 1, T=T)
+                seed=synth.WORKLOAD_SEED["decode_llama3_8b_b16_l32_t65536_d128_bf16"] + 1, T=T,
+                fused=True)
     checks = sorted(set([1000, 4095, 4096, 10000, 32767, 40000, 65534, T - 1] +
                         [a + w + k * (past + 1) - 1 for k in (100, 300, 505)]))
     snap = oracle.sepcache_simulate(st.flags, a, s, past, w, checks)
