@@ -440,43 +440,61 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// bf16 decode on warp-level tensor cores, streamed.  The rows of a (b, kv
-// head) are split between the two CTAs of a cluster.  A producer warp streams
-// each CTA's rows in 64-row chunks through a 3-stage shared-memory ring (one
-// bulk copy per row and tensor; a stage is refilled once all consumers have
-// released it).  Each of the four consumer warps owns 16 rows of every chunk
-// and keeps its own online softmax in registers:
+// bf16 decode on warp-level tensor cores, streamed by the tensor-copy
+// engine.  The rows of a (b, kv head) are split between the two CTAs of a
+// cluster.  One producer thread streams each CTA's rows in 64-row chunks
+// through a 3-stage shared-memory ring: per chunk and tensor, D/64
+// tensor-map tiles of 64 rows x 128 bytes, written 128-byte swizzled
+// (16-byte unit u of row r lands at unit u ^ (r & 7)).  A chunk is
+// 2 * D/64 copy requests of 8 KB, and the ldmatrix reads below hit eight
+// different bank groups.  Each of the four consumer warps owns 16 rows of
+// every chunk and keeps its own online softmax in registers:
 //   S = Q K^T with the G query heads as the rows of a 16-row A operand (rows
 //     >= G are zero) and its 16 keys as two n-tiles;
 //   the S accumulator fragments become the P operand directly (bf16), and
 //   O += P V with V as B (ldmatrix.trans) over all head dims.
-// No CTA-wide barrier inside the loop.  At the end the warps' partials are
-// combined in shared memory and the two CTAs merge through distributed
-// shared memory.  K/V rows sit at a padded stride (D + 8 elements) so that
-// ldmatrix reads are conflict-free.
+// No CTA-wide barrier inside the loop.  At the end the partials of the
+// 4 warps x 2 CTAs meet in one pass over distributed shared memory.
 constexpr int kPipeStages = 3;
 constexpr int kPipeCluster = 2;
 constexpr int kPipeThreads = 160;  // 4 consumer warps + 1 producer warp
+constexpr int kTileBytes = ROWS * 128;
 
 template <int D>
+constexpr int pipe_stage_bytes() {
+  return 2 * (D / 64) * kTileBytes;
+}
+template <int D>
 constexpr int pipe_smem_bytes() {
-  return kPipeStages * 2 * ROWS * (D + 8) * 2;
+  return kPipeStages * pipe_stage_bytes<D>() + 1024;  // + alignment slack
+}
+
+// Byte offset of (row r, element d) in one tensor's D/64 swizzled tiles.
+__device__ __forceinline__ uint32_t swz(int r, int d) {
+  return static_cast<uint32_t>((d >> 6) * kTileBytes + r * 128 +
+                               ((((d >> 3) & 7) ^ (r & 7)) << 4) + (d & 7) * 2);
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 template <int D, int G, bool FUSED>
-__global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodeParams p) {
+__global__ void __launch_bounds__(kPipeThreads, 2)
+    k_decode_pipe(const DecodeParams p, const __grid_constant__ CUtensorMap map_k,
+                  const __grid_constant__ CUtensorMap map_v) {
   static_assert(G <= 8, "at most 8 query heads per kv head");
   using T = __nv_bfloat16;
-  constexpr int RS = D + 8;  // K/V row stride in shared memory (elements)
-  constexpr int CH = D * 2 / 16;
-  constexpr int NT = D / 8;  // n-tiles of the output
-  extern __shared__ __align__(128) uint8_t dsm[];
-  T* const stages = reinterpret_cast<T*>(dsm);  // [stage][K rows | V rows]
-  float* const wpart = reinterpret_cast<float*>(dsm);  // after the loop: [4][G][D]
-  static_assert(kPipeStages * 2 * ROWS * RS * 2 >= 4 * G * D * 4, "warp partials fit in the ring");
-  __shared__ float po[G][D];
-  __shared__ float sm[G], sl[G];
-  __shared__ float wm[4][G], wl[4][G];
+  constexpr int CH = D / 8;   // 16-byte units per row
+  constexpr int NT = D / 8;   // n-tiles of the output
+  constexpr int NB = D / 64;  // tiles per chunk and tensor
+  constexpr int SB = pipe_stage_bytes<D>();
+  static_assert(4 * G * D * 4 <= kPipeStages * SB, "warp partials fit in the ring");
+  extern __shared__ uint8_t dsm_raw[];
+  // the swizzle pattern repeats every 1024 bytes: tiles start on that boundary
+  uint8_t* const ring = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ float wm[4][G], wl[4][G];  // the warps' running max (log2 units) and sum
   __shared__ __align__(8) uint64_t full[kPipeStages], empty[kPipeStages];
   __shared__ int abort_flag;
 
@@ -484,27 +502,6 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodePar
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
 
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int32_t* cnt = p.counts + 4 * b;
-  const int32_t* pl = p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr);
-  const int c0 = cnt[0], c1 = cnt[1], c2 = cnt[2], c3 = cnt[3];
-  const int buf = p.cur[b] & 1;
-  const int flush = FUSED ? pl[0] : 0;
-  const int slot = FUSED ? pl[1] : -1;
-  const int sbuf = FUSED ? (pl[4] & 1) : buf;
-  int len = c0 + c1 + c2 + c3;
-  if (len < 0 || len > p.cap) len = 0;
-  int mid = ((len + 1) / 2 + 15) / 16 * 16;
-  if (mid > len) mid = len;
-  const int rs = half ? mid : 0, re = half ? len : mid;
-  const int nchunks = (re - rs + ROWS - 1) / ROWS;
-  const int nsplit_b = mid < len ? 2 : (len > 0 ? 1 : 0);
-  auto base_of = [&](int bb) -> int64_t {
-    return ((((static_cast<int64_t>(bb) * p.layers + p.layer) * p.B + b) * p.Hkv + g) * p.cap) * D;
-  };
-  const int64_t kv_base = base_of(buf);
-  const T* kc = static_cast<const T*>(p.kc);
-  const T* vc = static_cast<const T*>(p.vc);
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int st = 0; st < kPipeStages; ++st) {
@@ -512,9 +509,33 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodePar
       sep::mbar_init(&empty[st], 4);
     }
     sep::mbar_fence_init();
+    sep::tma_prefetch_desc(&map_k);
+    sep::tma_prefetch_desc(&map_v);
   }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int32_t* cnt = p.counts + 4 * b;
+  const int32_t* pl = p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr);
+  int len = cnt[0] + cnt[1] + cnt[2] + cnt[3];
+  const int buf = p.cur[b] & 1;
+  const int flush = FUSED ? pl[0] : 0;
+  const int slot = FUSED ? pl[1] : -1;
+  const int sbuf = FUSED ? (pl[4] & 1) : buf;
+  if (len < 0 || len > p.cap) len = 0;
+  int mid = ((len + 1) / 2 + 15) / 16 * 16;
+  if (mid > len) mid = len;
+  const int rs = half ? mid : 0, re = half ? len : mid;
+  const int nchunks = (re - rs + ROWS - 1) / ROWS;
+  // first row of this (buffer, layer, b, kv head) in the [rows, D] view
+  auto row_of = [&](int bb) -> int64_t {
+    return (((static_cast<int64_t>(bb) * p.layers + p.layer) * p.B + b) * p.Hkv + g) * p.cap;
+  };
+  const int64_t row0 = row_of(buf);
+  T* const kc = static_cast<T*>(const_cast<void*>(p.kc));
+  T* const vc = static_cast<T*>(const_cast<void*>(p.vc));
   __syncthreads();
-  float o[NT][4];                        // consumer warps: O rows of head gq
+
+  int issued = 0;  // producer: chunks whose copies were started
+  float o[NT][4];
   float m_run = -INFINITY, l_run = 0.f;  // head gq (lanes gq < G)
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -527,8 +548,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodePar
       const int st = c % kPipeStages;
       const int r0 = rs + c * ROWS;
       const int nr = re - r0 < ROWS ? re - r0 : ROWS;
-      T* sk = stages + st * 2 * ROWS * RS;
-      T* sv = sk + ROWS * RS;
+      uint8_t* const kt = ring + st * SB;
+      uint8_t* const vt = kt + NB * kTileBytes;
       if (c >= kPipeStages &&
           !__all_sync(0xffffffffu, sep::mbar_wait(&empty[st], ((c / kPipeStages) - 1) & 1, &abort_flag, p.err)))
         break;
@@ -536,7 +557,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodePar
         // rows of the post-flush layout come from their source rows in the
         // old buffer (the new token from k_new/v_new); each is also stored
         // at its destination in the new buffer
-        const int64_t sbase = base_of(sbuf);
+        const int64_t srow = row_of(sbuf);
         const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
         const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
         for (int e = lane; e < 2 * nr * CH; e += 32) {
@@ -546,24 +567,25 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodePar
           if (src == slot) {
             val = (which ? vn : kn)[cc];
           } else if (src >= 0 && src < p.cap) {
-            val = reinterpret_cast<const uint4*>((which ? vc : kc) + sbase + static_cast<int64_t>(src) * D)[cc];
+            val = reinterpret_cast<const uint4*>((which ? vc : kc) + (srow + src) * D)[cc];
           }
-          reinterpret_cast<uint4*>((which ? sv : sk) + r * RS)[cc] = val;
-          reinterpret_cast<uint4*>(const_cast<T*>(which ? vc : kc) + kv_base + static_cast<int64_t>(r0 + r) * D)[cc] = val;
+          *reinterpret_cast<uint4*>((which ? vt : kt) + swz(r, 8 * cc)) = val;
+          reinterpret_cast<uint4*>((which ? vc : kc) + (row0 + r0 + r) * D)[cc] = val;
         }
+        sep::fence_proxy_async_smem();  // later tensor copies refill these bytes
         __syncwarp();
         if (lane == 0) sep::mbar_arrive(&full[st]);  // plain stores, released by the arrive
-      } else {
-        if (lane == 0) sep::mbar_arrive_expect_tx(&full[st], 2u * nr * D * 2);
-        __syncwarp();
-        for (int e = lane; e < 2 * nr; e += 32) {
-          const int which = e / nr, r = e % nr;
-          sep::bulk_load((which ? sv : sk) + r * RS, (which ? vc : kc) + kv_base + static_cast<int64_t>(r0 + r) * D,
-                         D * 2, &full[st]);
+      } else if (lane == 0) {
+        sep::mbar_arrive_expect_tx(&full[st], SB);
+#pragma unroll
+        for (int j = 0; j < NB; ++j) {
+          sep::tma_load_2d(kt + j * kTileBytes, &map_k, 64 * j, static_cast<int32_t>(row0 + r0), &full[st]);
+          sep::tma_load_2d(vt + j * kTileBytes, &map_v, 64 * j, static_cast<int32_t>(row0 + r0), &full[st]);
         }
       }
+      issued = c + 1;
     }
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (lane == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   } else {
     // ---------------------------------------------------------- consumers
     uint32_t qa[D / 16][4];  // Q fragments (rows = heads; heads >= G are zero)
@@ -578,16 +600,17 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodePar
         qa[kk][3] = 0u;
       }
     }
+    const int kr = 16 * warp;  // this warp's rows of each chunk
     for (int c = 0; c < nchunks; ++c) {
       const int st = c % kPipeStages;
       const int r0 = rs + c * ROWS;
       const int nr = re - r0 < ROWS ? re - r0 : ROWS;
-      T* sk = stages + st * 2 * ROWS * RS;
-      T* sv = sk + ROWS * RS;
+      uint8_t* const kt = ring + st * SB;
+      uint8_t* const vt = kt + NB * kTileBytes;
       if (!__all_sync(0xffffffffu, sep::mbar_wait(&full[st], (c / kPipeStages) & 1, &abort_flag, p.err)))
         break;
-      const int kr = 16 * warp;  // this warp's rows of the chunk
       if (kr < nr) {
+        bool wrote = false;
         if (FUSED && !flush && slot >= r0 + kr && slot < r0 + kr + 16 && slot < r0 + nr) {
           // the new token (the last row without a flush): from k_new/v_new,
           // also stored into the cache
@@ -597,30 +620,36 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodePar
           for (int e = lane; e < 2 * CH; e += 32) {
             const int which = e / CH, cc = e % CH;
             const uint4 val = (which ? vn : kn)[cc];
-            reinterpret_cast<uint4*>((which ? sv : sk) + r * RS)[cc] = val;
-            reinterpret_cast<uint4*>(const_cast<T*>(which ? vc : kc) + kv_base + static_cast<int64_t>(r0 + r) * D)[cc] = val;
+            *reinterpret_cast<uint4*>((which ? vt : kt) + swz(r, 8 * cc)) = val;
+            reinterpret_cast<uint4*>((which ? vc : kc) + (row0 + r0 + r) * D)[cc] = val;
           }
+          wrote = true;
         }
-        // V rows of this warp past the chunk's end: P is 0 there, and
-        // 0 * garbage may be NaN
+        // V rows of this warp past the chunk's end (whatever the copy
+        // brought in): P is 0 there, and 0 * garbage may be NaN
         const int vr = nr - kr < 16 ? nr - kr : 16;
         for (int e = lane; e < (16 - vr) * CH; e += 32)
-          reinterpret_cast<uint4*>(sv + (kr + vr + e / CH) * RS)[e % CH] = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(vt + swz(kr + vr + e / CH, 8 * (e % CH))) = make_uint4(0, 0, 0, 0);
+        if (wrote || vr < 16) sep::fence_proxy_async_smem();  // refilled by tensor copies later
         __syncwarp();
-        // S for the warp's 16 keys: two n-tiles
-        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        // S for the warp's 16 keys: two n-tiles, two accumulators each
+        float sa0[4] = {0.f, 0.f, 0.f, 0.f}, sa1[4] = {0.f, 0.f, 0.f, 0.f};
+        float sb0[4] = {0.f, 0.f, 0.f, 0.f}, sb1[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint32_t kb = sep::smem_u32(kt), vb0 = sep::smem_u32(vt);
 #pragma unroll
         for (int kk = 0; kk < D / 16; kk += 2) {
           uint32_t f0[4], f1[4];
-          ldsm_x4(sep::smem_u32(sk + (kr + (lane & 7)) * RS + 16 * kk + (lane >> 3) * 8), f0);
-          ldsm_x4(sep::smem_u32(sk + (kr + 8 + (lane & 7)) * RS + 16 * kk + (lane >> 3) * 8), f1);
-          mma16816(sa, qa[kk], f0[0], f0[1]);
-          mma16816(sb, qa[kk], f1[0], f1[1]);
-          mma16816(sa, qa[kk + 1], f0[2], f0[3]);
-          mma16816(sb, qa[kk + 1], f1[2], f1[3]);
+          const int d0 = 16 * kk + 8 * (lane >> 3);
+          ldsm_x4(kb + swz(kr + (lane & 7), d0), f0);
+          ldsm_x4(kb + swz(kr + 8 + (lane & 7), d0), f1);
+          mma16816(sa0, qa[kk], f0[0], f0[1]);
+          mma16816(sb0, qa[kk], f1[0], f1[1]);
+          mma16816(sa1, qa[kk + 1], f0[2], f0[3]);
+          mma16816(sb1, qa[kk + 1], f1[2], f1[3]);
         }
         // keys kr + {2tq, 2tq+1} (sa) and kr + 8 + {2tq, 2tq+1} (sb)
-        float x[4] = {sa[0] * p.scale_log2, sa[1] * p.scale_log2, sb[0] * p.scale_log2, sb[1] * p.scale_log2};
+        float x[4] = {(sa0[0] + sa1[0]) * p.scale_log2, (sa0[1] + sa1[1]) * p.scale_log2,
+                      (sb0[0] + sb1[0]) * p.scale_log2, (sb0[1] + sb1[1]) * p.scale_log2};
         const int kk0 = kr + 2 * tq, kk1 = kr + 8 + 2 * tq;
         if (kk0 >= nr) x[0] = -INFINITY;
         if (kk0 + 1 >= nr) x[1] = -INFINITY;
@@ -652,68 +681,95 @@ __global__ void __launch_bounds__(kPipeThreads, 2) k_decode_pipe(const DecodePar
         pa[3] = 0u;
 #pragma unroll
         for (int np = 0; np < NT / 2; ++np) {
-          uint32_t vb[4];
-          ldsm_x4_t(sep::smem_u32(sv + (kr + ((lane >> 3) & 1) * 8 + (lane & 7)) * RS + 16 * np + (lane >> 4) * 8), vb);
-          mma16816(o[2 * np], pa, vb[0], vb[1]);
-          mma16816(o[2 * np + 1], pa, vb[2], vb[3]);
+          uint32_t vf[4];
+          ldsm_x4_t(vb0 + swz(kr + ((lane >> 3) & 1) * 8 + (lane & 7), 16 * np + 8 * (lane >> 4)), vf);
+          mma16816(o[2 * np], pa, vf[0], vf[1]);
+          mma16816(o[2 * np + 1], pa, vf[2], vf[3]);
         }
       }
       __syncwarp();
       if (lane == 0) sep::mbar_arrive(&empty[st]);
     }
-    // this warp's partial (lanes gq < G hold head gq)
     if (gq < G && tq == 0) {
       wm[warp][gq] = m_run;
       wl[warp][gq] = l_run;
     }
   }
-  __syncthreads();  // the ring is idle: reuse it for the warps' outputs
+  __syncthreads();
+  if (abort_flag) {
+    // a wait gave up: let this CTA's copies land before the ring is reused
+    if (threadIdx.x == 4 * 32) {
+      int dummy = 0;
+      for (int c = issued - kPipeStages < 0 ? 0 : issued - kPipeStages; c < issued; ++c)
+        sep::mbar_wait(&full[c % kPipeStages], (c / kPipeStages) & 1, &dummy, nullptr);
+    }
+    __syncthreads();
+  }
+  // the ring is idle: it now holds the warps' unnormalised outputs [4][G][D]
+  float* const wo = reinterpret_cast<float*>(ring);
   if (warp < 4 && gq < G) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      wpart[(warp * G + gq) * D + 8 * nt + 2 * tq] = o[nt][0];
-      wpart[(warp * G + gq) * D + 8 * nt + 2 * tq + 1] = o[nt][1];
+    for (int nt = 0; nt < NT; ++nt)
+      *reinterpret_cast<float2*>(wo + (warp * G + gq) * D + 8 * nt + 2 * tq) = make_float2(o[nt][0], o[nt][1]);
+  }
+  cluster_sync_all();  // both CTAs' partials are visible cluster-wide
+  cg::cluster_group cl = cg::this_cluster();
+  const float* const wo_r = cl.map_shared_rank(wo, half ^ 1);
+  const float* const wm_r = cl.map_shared_rank(&wm[0][0], half ^ 1);
+  const float* const wl_r = cl.map_shared_rank(&wl[0][0], half ^ 1);
+  T* const out = static_cast<T*>(p.out);
+  constexpr int PAIRS = G * D / 2 / kPipeCluster;  // output pairs merged by each CTA
+  for (int e = threadIdx.x; e < PAIRS; e += kPipeThreads) {
+    const int idx = 2 * (half * PAIRS + e);
+    const int h = idx / D, d = idx % D;
+    float mk[8], lk[8];
+    float2 ok[8];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      mk[w] = wm[w][h];
+      lk[w] = wl[w][h];
+      ok[w] = *reinterpret_cast<const float2*>(wo + (w * G + h) * D + d);
+      mk[4 + w] = wm_r[w * G + h];
+      lk[4 + w] = wl_r[w * G + h];
+      ok[4 + w] = *reinterpret_cast<const float2*>(wo_r + (w * G + h) * D + d);
     }
+    float M = mk[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) M = fmaxf(M, mk[k]);
+    float L = 0.f, ax = 0.f, ay = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float wgt = mk[k] == -INFINITY ? 0.f : exp2f(mk[k] - M);
+      L += lk[k] * wgt;
+      ax += ok[k].x * wgt;
+      ay += ok[k].y * wgt;
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    *reinterpret_cast<__nv_bfloat162*>(out + (static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d) =
+        __floats2bfloat162_rn(ax * inv, ay * inv);
+    if (p.lse && d == 0)
+      p.lse[static_cast<int64_t>(b) * p.Hq + g * G + h] =
+          L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < G; e += blockDim.x) {
-    float M = -INFINITY;
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, wm[w][e]);
-    float L = 0.f;
-    for (int w = 0; w < 4; ++w) L += wm[w][e] == -INFINITY ? 0.f : wl[w][e] * exp2f(wm[w][e] - M);
-    sm[e] = M;
-    sl[e] = L;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-    const int h = e / D, d = e % D;
-    const float M = sm[h];
-    float acc = 0.f;
-    for (int w = 0; w < 4; ++w)
-      if (wm[w][h] != -INFINITY) acc += wpart[(w * G + h) * D + d] * exp2f(wm[w][h] - M);
-    po[h][d] = acc;
-  }
-  __syncthreads();
-  decode_finish<T, D, G, true, kPipeCluster>(p, po, sm, sl, nsplit_b, half, b, g);
+  cluster_sync_all();  // keep this CTA's partials alive until the partner has read them
+}
+
+// Maximum dynamic shared memory for `kern` on the current device, set once.
+template <typename K>
+bool allow_smem(K kern, int smem, bool* done) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (smem <= 48 * 1024 || dev < 0 || dev >= 64 || done[dev]) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return false;
+  done[dev] = true;
+  return true;
 }
 
 template <typename T, int D, int G, bool FUSED, bool CLUSTER>
 int launch_one(const DecodeParams& p, cudaStream_t st) {
   constexpr bool TC = sizeof(T) == 2;  // bf16: streamed tensor-core kernel; fp32: exact FMA kernel
   constexpr int smem = TC ? pipe_smem_bytes<D>() : 2 * ROWS * D * static_cast<int>(sizeof(T));
-  void (*kern)(const DecodeParams);
-  if constexpr (TC)
-    kern = k_decode_pipe<D, G, FUSED>;
-  else
-    kern = k_decode<T, D, G, FUSED, CLUSTER>;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (smem > 48 * 1024 && dev >= 0 && dev < 64 && !attr_set[dev]) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return SEP_ECUDA;
-    attr_set[dev] = true;
-  }
   const int ncl = TC ? kPipeCluster : (CLUSTER ? kMaxClusterSplits : 1);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(TC ? kPipeCluster : (CLUSTER ? kMaxClusterSplits : p.nsplit), p.Hkv, p.B);
@@ -734,7 +790,22 @@ int launch_one(const DecodeParams& p, cudaStream_t st) {
   }
   cfg.attrs = attr;
   cfg.numAttrs = na;
-  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return SEP_ECUDA;
+  static bool attr_set[64] = {false};
+  if constexpr (TC) {
+    // the K and V arrays as [2 * layers * B * Hkv * cap, D] rows
+    const int64_t rows = 2LL * p.layers * p.B * p.Hkv * p.cap;
+    if (rows > 0x7fffffffLL) return SEP_ETOOBIG;
+    CUtensorMap mk, mv;
+    if (!sep::make_rows_map(&mk, p.kc, rows, D, ROWS) || !sep::make_rows_map(&mv, p.vc, rows, D, ROWS))
+      return SEP_ECUDA;
+    auto kern = k_decode_pipe<D, G, FUSED>;
+    if (!allow_smem(kern, smem, attr_set)) return SEP_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, p, mk, mv) != cudaSuccess) return SEP_ECUDA;
+  } else {
+    auto kern = k_decode<T, D, G, FUSED, CLUSTER>;
+    if (!allow_smem(kern, smem, attr_set)) return SEP_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) return SEP_ECUDA;
+  }
   return sep::launch_status();
 }
 

@@ -1,5 +1,6 @@
 // Entry points shared between the library's translation units.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -19,4 +20,7 @@ int prefill_tc(const void* q, const void* k, const void* v, const uint8_t* is_se
 int cache_advance(const sepcache* c, const uint8_t* is_sep_new, cudaStream_t st);
 bool cache_valid(const sepcache* c);
 constexpr int kCachePlanHdr = 8;  // plan header words per sequence (see sepcache.cu)
+// Tensor map of a bf16 [rows, D] row-major array (D = 64 or 128): tiles of
+// 64 columns x box_rows rows, 128-byte swizzled.  Defined in prefill_tc.cu.
+bool make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int D, int box_rows);  // plan header words per sequence (see sepcache.cu)
 }  // namespace sep

@@ -34,6 +34,7 @@
 #include <string.h>
 
 #include "common.cuh"
+#include "internal.h"
 
 namespace {
 
@@ -664,17 +665,8 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D bf16 view [rows, D] with 128-byte swizzled boxes of 64 columns x 128 rows.
 bool make_map(CUtensorMap* m, const void* base, int64_t rows, int D) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  cuuint32_t box[2] = {64, 128};
-  cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return sep::make_rows_map(m, base, rows, D, 128);
 }
 
 int num_sms() {
@@ -769,5 +761,19 @@ int prefill_tc(const void* q, const void* k, const void* v, const uint8_t* is_se
     return launch<128>(q, k, v, is_sep, prefix, idx, B, Hq, Hkv, S, a, n, scale, out, lse, kc, vc,
                        st);
   return SEP_EDTYPE;
+}
+}  // namespace sep
+
+namespace sep {
+bool make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int D, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows < 1 || box_rows < 1 || box_rows > 256) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 }  // namespace sep
