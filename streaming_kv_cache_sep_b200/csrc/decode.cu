@@ -73,6 +73,7 @@ struct DecodeParams {
   int32_t* ticket; // [B][Hkv]
   int32_t* err;
   int layer, layers, B, Hq, Hkv, cap, nsplit;
+  int early;  // fused step of layer >= 1: cache reads may precede the grid-dependency wait
   float scale_log2;
 };
 
@@ -430,10 +431,17 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(addr));
 }
+// Transpose of an 8x8 b16 matrix held one 32-bit pair per lane (lane t:
+// row t/4, columns 2(t%4), 2(t%4)+1), returned in the same layout.
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t y;
+  asm("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
 // c (16x8 fp32) += a (16x16 bf16, row-major fragment) * b (16x8 bf16, col fragment)
 __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
                                          uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
@@ -441,32 +449,42 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
 }
 
 // bf16 decode on warp-level tensor cores, streamed by the tensor-copy
-// engine.  The rows of a (b, kv head) are split between the two CTAs of a
-// cluster.  One producer thread streams each CTA's rows in 64-row chunks
-// through a 3-stage shared-memory ring: per chunk and tensor, D/64
-// tensor-map tiles of 64 rows x 128 bytes, written 128-byte swizzled
-// (16-byte unit u of row r lands at unit u ^ (r & 7)).  A chunk is
-// 2 * D/64 copy requests of 8 KB, and the ldmatrix reads below hit eight
-// different bank groups.  Each of the four consumer warps owns 16 rows of
-// every chunk and keeps its own online softmax in registers:
-//   S = Q K^T with the G query heads as the rows of a 16-row A operand (rows
-//     >= G are zero) and its 16 keys as two n-tiles;
-//   the S accumulator fragments become the P operand directly (bf16), and
-//   O += P V with V as B (ldmatrix.trans) over all head dims.
-// No CTA-wide barrier inside the loop.  At the end the partials of the
-// 4 warps x 2 CTAs meet in one pass over distributed shared memory.
-constexpr int kPipeStages = 3;
+// engine.  The rows of a (b, kv head) are split between the NCL CTAs of a
+// cluster (about len/NCL rows each).  One producer thread streams a CTA's
+// rows in 64-row chunks through a shared-memory ring: per chunk and tensor,
+// D/64 tensor-map tiles of 64 rows x 128 bytes, written 128-byte swizzled
+// (16-byte unit u of row r lands at unit u ^ (r & 7)), so a chunk is
+// 2 * D/64 copy requests of 8 KB and the ldmatrix reads hit eight different
+// bank groups.  When a CTA's rows fit the ring (len <= NCL * stages * 64)
+// all its copies start at once.  Each of the four consumer warps owns 16
+// rows of every chunk and keeps its own online softmax in registers, with
+// the keys as the 16 rows of the tensor-core tile:
+//   S^T = K Q^T (A = K rows, B = Q^T: the G query heads as the 8 columns);
+//   a head's reference max moves only when a score exceeds it by 2^8;
+//   P^T reaches the B operand by an in-register 8x8 transpose (movmatrix);
+//   O^T += V^T P^T (A = V^T by ldmatrix.trans).
+// No CTA-wide barrier inside the loop.  At the end each CTA merges 1/NCL of
+// the D x G outputs: every warp sends its partial for each slice to the CTA
+// that merges it with asynchronous remote stores that complete on that
+// CTA's mbarrier by byte count, so no sender waits for an acknowledgement.
 constexpr int kPipeCluster = 2;
 constexpr int kPipeThreads = 160;  // 4 consumer warps + 1 producer warp
 constexpr int kTileBytes = ROWS * 128;
+constexpr float kLazyLog2 = 8.f;  // reference-max slack (log2 units) before a rescale
 
 template <int D>
-constexpr int pipe_stage_bytes() {
+__host__ __device__ constexpr int pipe_stage_bytes() {
   return 2 * (D / 64) * kTileBytes;
 }
-template <int D>
-constexpr int pipe_smem_bytes() {
-  return kPipeStages * pipe_stage_bytes<D>() + 1024;  // + alignment slack
+// ring stages: three, except where two CTAs per SM would not fit
+template <int D, int G>
+__host__ __device__ constexpr int pipe_stages() {
+  return D * G >= 1024 ? 2 : 3;
+}
+// the ring, then the partials this CTA merges ([NCL][4 warps][D/NCL x G] fp32)
+template <int D, int G>
+__host__ __device__ constexpr int pipe_smem_bytes() {
+  return pipe_stages<D, G>() * pipe_stage_bytes<D>() + 4 * G * D * 4 + 1024;  // + alignment slack
 }
 
 // Byte offset of (row r, element d) in one tensor's D/64 swizzled tiles.
@@ -475,30 +493,33 @@ __device__ __forceinline__ uint32_t swz(int r, int d) {
                                ((((d >> 3) & 7) ^ (r & 7)) << 4) + (d & 7) * 2);
 }
 
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-
 template <int D, int G, bool FUSED>
 __global__ void __launch_bounds__(kPipeThreads, 2)
     k_decode_pipe(const DecodeParams p, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v) {
   static_assert(G <= 8, "at most 8 query heads per kv head");
   using T = __nv_bfloat16;
+  constexpr int NCL = kPipeCluster;
+  constexpr int kPipeStages = pipe_stages<D, G>();
   constexpr int CH = D / 8;   // 16-byte units per row
-  constexpr int NT = D / 8;   // n-tiles of the output
+  constexpr int DT = D / 16;  // 16-dim tiles of the output
   constexpr int NB = D / 64;  // tiles per chunk and tensor
   constexpr int SB = pipe_stage_bytes<D>();
-  static_assert(4 * G * D * 4 <= kPipeStages * SB, "warp partials fit in the ring");
+  constexpr int DQ = D / NCL;   // dims merged by each CTA
+  constexpr int PART = DQ * G;  // one warp's partial for one CTA's slice, [DQ][G]
+  // bytes that reach each CTA's merge barrier: NCL ranks x 4 warps x
+  // (partial + max and sum per head)
+  constexpr uint32_t kMergeBytes = NCL * 4 * (PART + 2 * G) * 4;
   extern __shared__ uint8_t dsm_raw[];
   // the swizzle pattern repeats every 1024 bytes: tiles start on that boundary
   uint8_t* const ring = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ float wm[4][G], wl[4][G];  // the warps' running max (log2 units) and sum
-  __shared__ __align__(8) uint64_t full[kPipeStages], empty[kPipeStages];
+  float* const recv_o = reinterpret_cast<float*>(ring + kPipeStages * SB);  // [NCL][4][PART]
+  __shared__ float rm[NCL][4][G], rl[NCL][4][G];  // every warp's running max (log2) and sum
+  __shared__ __align__(8) uint64_t full[kPipeStages], empty[kPipeStages], mrg;
   __shared__ int abort_flag;
 
-  const int half = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int rank = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
 
@@ -508,11 +529,23 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
       sep::mbar_init(&full[st], 1);
       sep::mbar_init(&empty[st], 4);
     }
+    sep::mbar_init(&mrg, 1);
     sep::mbar_fence_init();
+    sep::mbar_arrive_expect_tx(&mrg, kMergeBytes);  // completes once every partial is here
     sep::tma_prefetch_desc(&map_k);
     sep::tma_prefetch_desc(&map_v);
+    // let the next grid on the stream launch now: its CTAs take SM slots as
+    // soon as ours retire and start their copies while ours drain (its own
+    // grid-dependency wait still orders it after this grid)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   }
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // completes long before the first remote store (after the chunk loop):
+  // every CTA's barriers are initialised by then
+  sep::cluster_arrive_relaxed();
+  // With p.early the cache metadata and this layer's rows were last written
+  // at least two launches back, so they are read before waiting on the
+  // previous grid; q, k_new, v_new and every store still come after the wait.
+  if (!p.early) asm volatile("griddepcontrol.wait;" ::: "memory");
   const int32_t* cnt = p.counts + 4 * b;
   const int32_t* pl = p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr);
   int len = cnt[0] + cnt[1] + cnt[2] + cnt[3];
@@ -521,9 +554,9 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   const int slot = FUSED ? pl[1] : -1;
   const int sbuf = FUSED ? (pl[4] & 1) : buf;
   if (len < 0 || len > p.cap) len = 0;
-  int mid = ((len + 1) / 2 + 15) / 16 * 16;
-  if (mid > len) mid = len;
-  const int rs = half ? mid : 0, re = half ? len : mid;
+  const int per = ((len + NCL - 1) / NCL + 15) / 16 * 16;  // rows per CTA (multiple of 16)
+  const int rs = rank * per < len ? rank * per : len;
+  const int re = rs + per < len ? rs + per : len;
   const int nchunks = (re - rs + ROWS - 1) / ROWS;
   // first row of this (buffer, layer, b, kv head) in the [rows, D] view
   auto row_of = [&](int bb) -> int64_t {
@@ -535,12 +568,15 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   __syncthreads();
 
   int issued = 0;  // producer: chunks whose copies were started
-  float o[NT][4];
-  float m_run = -INFINITY, l_run = 0.f;  // head gq (lanes gq < G)
+  // consumer state.  O^T tiles: o[dt] holds dims 16dt + gq (+8) x heads
+  // 2tq, 2tq + 1; the reference max of those two heads (equal across the
+  // lanes of a column) and this lane's share of their sums.
+  float o[DT][4];
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
+  for (int dt = 0; dt < DT; ++dt)
 #pragma unroll
-    for (int e = 0; e < 4; ++e) o[nt][e] = 0.f;
+    for (int e = 0; e < 4; ++e) o[dt][e] = 0.f;
 
   if (warp == 4) {
     // ---------------------------------------------------------- producer
@@ -557,6 +593,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         // rows of the post-flush layout come from their source rows in the
         // old buffer (the new token from k_new/v_new); each is also stored
         // at its destination in the new buffer
+        asm volatile("griddepcontrol.wait;" ::: "memory");
         const int64_t srow = row_of(sbuf);
         const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
         const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
@@ -576,28 +613,30 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         __syncwarp();
         if (lane == 0) sep::mbar_arrive(&full[st]);  // plain stores, released by the arrive
       } else if (lane == 0) {
+        // K/V rows are read once per step: evict them from L2 before the
+        // metadata, q and outputs that the next launches need
+        const uint64_t pol = sep::l2_evict_first_policy();
         sep::mbar_arrive_expect_tx(&full[st], SB);
 #pragma unroll
         for (int j = 0; j < NB; ++j) {
-          sep::tma_load_2d(kt + j * kTileBytes, &map_k, 64 * j, static_cast<int32_t>(row0 + r0), &full[st]);
-          sep::tma_load_2d(vt + j * kTileBytes, &map_v, 64 * j, static_cast<int32_t>(row0 + r0), &full[st]);
+          sep::tma_load_2d_hint(kt + j * kTileBytes, &map_k, 64 * j, static_cast<int32_t>(row0 + r0), &full[st], pol);
+          sep::tma_load_2d_hint(vt + j * kTileBytes, &map_v, 64 * j, static_cast<int32_t>(row0 + r0), &full[st], pol);
         }
       }
       issued = c + 1;
     }
-    if (lane == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // before this warp's stores in the merge
   } else {
     // ---------------------------------------------------------- consumers
-    uint32_t qa[D / 16][4];  // Q fragments (rows = heads; heads >= G are zero)
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // q, k_new, v_new
+    uint32_t qb[DT][2];  // Q^T as the B operand: dims x heads (heads >= G are zero)
     {
       const T* qg = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
+      for (int kk = 0; kk < DT; ++kk) {
         const bool in = gq < G;
-        qa[kk][0] = in ? *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * kk + 2 * tq) : 0u;
-        qa[kk][2] = in ? *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * kk + 8 + 2 * tq) : 0u;
-        qa[kk][1] = 0u;
-        qa[kk][3] = 0u;
+        qb[kk][0] = in ? *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * kk + 2 * tq) : 0u;
+        qb[kk][1] = in ? *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * kk + 8 + 2 * tq) : 0u;
       }
     }
     const int kr = 16 * warp;  // this warp's rows of each chunk
@@ -632,72 +671,76 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
           *reinterpret_cast<uint4*>(vt + swz(kr + vr + e / CH, 8 * (e % CH))) = make_uint4(0, 0, 0, 0);
         if (wrote || vr < 16) sep::fence_proxy_async_smem();  // refilled by tensor copies later
         __syncwarp();
-        // S for the warp's 16 keys: two n-tiles, two accumulators each
-        float sa0[4] = {0.f, 0.f, 0.f, 0.f}, sa1[4] = {0.f, 0.f, 0.f, 0.f};
-        float sb0[4] = {0.f, 0.f, 0.f, 0.f}, sb1[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint32_t kb = sep::smem_u32(kt), vb0 = sep::smem_u32(vt);
+        // all K and V fragments of the warp's 16 rows first: each ldmatrix
+        // waits ~100 cycles, back to back they overlap
+        const uint32_t kb = sep::smem_u32(kt), vb = sep::smem_u32(vt);
+        uint32_t ka[DT][4], va[DT][4];
 #pragma unroll
-        for (int kk = 0; kk < D / 16; kk += 2) {
-          uint32_t f0[4], f1[4];
-          const int d0 = 16 * kk + 8 * (lane >> 3);
-          ldsm_x4(kb + swz(kr + (lane & 7), d0), f0);
-          ldsm_x4(kb + swz(kr + 8 + (lane & 7), d0), f1);
-          mma16816(sa0, qa[kk], f0[0], f0[1]);
-          mma16816(sb0, qa[kk], f1[0], f1[1]);
-          mma16816(sa1, qa[kk + 1], f0[2], f0[3]);
-          mma16816(sb1, qa[kk + 1], f1[2], f1[3]);
+        for (int kk = 0; kk < DT; ++kk)
+          ldsm_x4(kb + swz(kr + (lane & 7) + ((lane >> 3) & 1) * 8, 16 * kk + (lane >> 4) * 8), ka[kk]);
+#pragma unroll
+        for (int dt = 0; dt < DT; ++dt)
+          ldsm_x4_t(vb + swz(kr + (lane & 7) + (lane >> 4) * 8, 16 * dt + ((lane >> 3) & 1) * 8), va[dt]);
+        // S^T = K Q^T for the warp's 16 keys (rows) x 8 heads, four chains
+        float sacc[4][4] = {};
+#pragma unroll
+        for (int kk = 0; kk < DT; ++kk) mma16816(sacc[kk & 3], ka[kk], qb[kk][0], qb[kk][1]);
+        // x0/x1: key kr + gq, heads 2tq / 2tq + 1; x2/x3: key kr + gq + 8
+        float x[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          x[e] = ((sacc[0][e] + sacc[1][e]) + (sacc[2][e] + sacc[3][e])) * p.scale_log2;
+        if (kr + gq >= nr) x[0] = x[1] = -INFINITY;
+        if (kr + gq + 8 >= nr) x[2] = x[3] = -INFINITY;
+        // the reference maxima move only when a score exceeds them by more
+        // than 2^8 (always on the warp's first keys); otherwise P <= 256
+        const bool up = x[0] > m0 + kLazyLog2 || x[2] > m0 + kLazyLog2 ||
+                        x[1] > m1 + kLazyLog2 || x[3] > m1 + kLazyLog2;
+        if (__any_sync(0xffffffffu, up)) {
+          float c0 = fmaxf(x[0], x[2]), c1 = fmaxf(x[1], x[3]);  // column maxima
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            c0 = fmaxf(c0, __shfl_xor_sync(0xffffffffu, c0, off));
+            c1 = fmaxf(c1, __shfl_xor_sync(0xffffffffu, c1, off));
+          }
+          const float n0 = fmaxf(m0, c0), n1 = fmaxf(m1, c1);
+          const float al0 = exp2f(m0 - n0), al1 = exp2f(m1 - n1);  // 0 on the first keys
+          l0 *= al0;
+          l1 *= al1;
+#pragma unroll
+          for (int dt = 0; dt < DT; ++dt) {
+            o[dt][0] *= al0;
+            o[dt][1] *= al1;
+            o[dt][2] *= al0;
+            o[dt][3] *= al1;
+          }
+          m0 = n0;
+          m1 = n1;
         }
-        // keys kr + {2tq, 2tq+1} (sa) and kr + 8 + {2tq, 2tq+1} (sb)
-        float x[4] = {(sa0[0] + sa1[0]) * p.scale_log2, (sa0[1] + sa1[1]) * p.scale_log2,
-                      (sb0[0] + sb1[0]) * p.scale_log2, (sb0[1] + sb1[1]) * p.scale_log2};
-        const int kk0 = kr + 2 * tq, kk1 = kr + 8 + 2 * tq;
-        if (kk0 >= nr) x[0] = -INFINITY;
-        if (kk0 + 1 >= nr) x[1] = -INFINITY;
-        if (kk1 >= nr) x[2] = -INFINITY;
-        if (kk1 + 1 >= nr) x[3] = -INFINITY;
-        float mb = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
-        mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-        const float m_new = fmaxf(m_run, mb);
-        const float alpha = exp2f(m_run - m_new);  // 0 on the warp's first keys
-        float pr[4];
+        const float p0 = exp2f(x[0] - m0), p1 = exp2f(x[1] - m1);
+        const float p2 = exp2f(x[2] - m0), p3 = exp2f(x[3] - m1);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
+        // P^T (keys x heads) as the B operand: transpose the 8x8 blocks
+        const uint32_t pb0 = movmatrix_t(sep::pack_bf16x2(p0, p1));
+        const uint32_t pb1 = movmatrix_t(sep::pack_bf16x2(p2, p3));
+        // O^T += V^T P^T, V^T as the A operand (ldmatrix.trans of V rows)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) pr[e] = exp2f(x[e] - m_new);
-        float ls = (pr[0] + pr[1]) + (pr[2] + pr[3]);
-        ls += __shfl_xor_sync(0xffffffffu, ls, 1);
-        ls += __shfl_xor_sync(0xffffffffu, ls, 2);
-        l_run = l_run * alpha + ls;
-        m_run = m_new;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          o[nt][0] *= alpha;
-          o[nt][1] *= alpha;
-        }
-        // P as the A operand (rows = heads, the 16 keys as k)
-        uint32_t pa[4];
-        pa[0] = sep::pack_bf16x2(pr[0], pr[1]);
-        pa[1] = 0u;
-        pa[2] = sep::pack_bf16x2(pr[2], pr[3]);
-        pa[3] = 0u;
-#pragma unroll
-        for (int np = 0; np < NT / 2; ++np) {
-          uint32_t vf[4];
-          ldsm_x4_t(vb0 + swz(kr + ((lane >> 3) & 1) * 8 + (lane & 7), 16 * np + 8 * (lane >> 4)), vf);
-          mma16816(o[2 * np], pa, vf[0], vf[1]);
-          mma16816(o[2 * np + 1], pa, vf[2], vf[3]);
-        }
+        for (int dt = 0; dt < DT; ++dt) mma16816(o[dt], va[dt], pb0, pb1);
       }
       __syncwarp();
       if (lane == 0) sep::mbar_arrive(&empty[st]);
     }
-    if (gq < G && tq == 0) {
-      wm[warp][gq] = m_run;
-      wl[warp][gq] = l_run;
+    // this lane's sums -> the column sums of heads 2tq, 2tq + 1
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      l0 += __shfl_xor_sync(0xffffffffu, l0, off);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, off);
     }
   }
   __syncthreads();
   if (abort_flag) {
-    // a wait gave up: let this CTA's copies land before the ring is reused
+    // a wait gave up: let this CTA's copies land before it can exit
     if (threadIdx.x == 4 * 32) {
       int dummy = 0;
       for (int c = issued - kPipeStages < 0 ? 0 : issued - kPipeStages; c < issued; ++c)
@@ -705,53 +748,63 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     }
     __syncthreads();
   }
-  // the ring is idle: it now holds the warps' unnormalised outputs [4][G][D]
-  float* const wo = reinterpret_cast<float*>(ring);
-  if (warp < 4 && gq < G) {
+  sep::cluster_wait();
+  if (warp < 4) {
+    // send this warp's partial: dims of slice t go to CTA t
+    const uint32_t recv_s = sep::smem_u32(recv_o) + (rank * 4 + warp) * PART * 4;
+    const uint32_t rm_s = sep::smem_u32(&rm[rank][warp][0]), rl_s = sep::smem_u32(&rl[rank][warp][0]);
+    const int h0 = 2 * tq;
+    if (h0 < G) {
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-      *reinterpret_cast<float2*>(wo + (warp * G + gq) * D + 8 * nt + 2 * tq) = make_float2(o[nt][0], o[nt][1]);
+      for (int dt = 0; dt < DT; ++dt) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int d = 16 * dt + gq + 8 * r;
+          const int t = d / DQ;
+          const uint32_t dst = sep::cluster_addr_of(recv_s + ((d - t * DQ) * G + h0) * 4, t);
+          const uint32_t bar = sep::cluster_addr(&mrg, t);
+          if (G >= 2)
+            sep::st_async_v2f32(dst, o[dt][2 * r], o[dt][2 * r + 1], bar);
+          else
+            sep::st_async_f32(dst, o[dt][2 * r], bar);
+        }
+      }
+      if (gq == 0) {
+#pragma unroll
+        for (int t = 0; t < NCL; ++t) {
+          const uint32_t bar = sep::cluster_addr(&mrg, t);
+          sep::st_async_f32(sep::cluster_addr_of(rm_s + h0 * 4, t), m0, bar);
+          sep::st_async_f32(sep::cluster_addr_of(rl_s + h0 * 4, t), l0, bar);
+          if (h0 + 1 < G) {
+            sep::st_async_f32(sep::cluster_addr_of(rm_s + (h0 + 1) * 4, t), m1, bar);
+            sep::st_async_f32(sep::cluster_addr_of(rl_s + (h0 + 1) * 4, t), l1, bar);
+          }
+        }
+      }
+    }
   }
-  cluster_sync_all();  // both CTAs' partials are visible cluster-wide
-  cg::cluster_group cl = cg::this_cluster();
-  const float* const wo_r = cl.map_shared_rank(wo, half ^ 1);
-  const float* const wm_r = cl.map_shared_rank(&wm[0][0], half ^ 1);
-  const float* const wl_r = cl.map_shared_rank(&wl[0][0], half ^ 1);
+  sep::mbar_wait_cluster(&mrg, 0, p.err);
+  // merge the NCL x 4 partials of this CTA's DQ x G outputs, one element of
+  // the [d][head] layout per thread (consecutive words)
   T* const out = static_cast<T*>(p.out);
-  constexpr int PAIRS = G * D / 2 / kPipeCluster;  // output pairs merged by each CTA
-  for (int e = threadIdx.x; e < PAIRS; e += kPipeThreads) {
-    const int idx = 2 * (half * PAIRS + e);
-    const int h = idx / D, d = idx % D;
-    float mk[8], lk[8];
-    float2 ok[8];
+  for (int f = threadIdx.x; f < PART; f += kPipeThreads) {
+    const int h = f % G, d = rank * DQ + f / G;
+    float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      mk[w] = wm[w][h];
-      lk[w] = wl[w][h];
-      ok[w] = *reinterpret_cast<const float2*>(wo + (w * G + h) * D + d);
-      mk[4 + w] = wm_r[w * G + h];
-      lk[4 + w] = wl_r[w * G + h];
-      ok[4 + w] = *reinterpret_cast<const float2*>(wo_r + (w * G + h) * D + d);
+    for (int k = 0; k < NCL * 4; ++k) M = fmaxf(M, rm[k / 4][k % 4][h]);
+    float L = 0.f, acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < NCL * 4; ++k) {
+      const float mk = rm[k / 4][k % 4][h];
+      const float wgt = mk == -INFINITY ? 0.f : exp2f(mk - M);
+      L += rl[k / 4][k % 4][h] * wgt;
+      acc += recv_o[k * PART + f] * wgt;
     }
-    float M = mk[0];
-#pragma unroll
-    for (int k = 1; k < 8; ++k) M = fmaxf(M, mk[k]);
-    float L = 0.f, ax = 0.f, ay = 0.f;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float wgt = mk[k] == -INFINITY ? 0.f : exp2f(mk[k] - M);
-      L += lk[k] * wgt;
-      ax += ok[k].x * wgt;
-      ay += ok[k].y * wgt;
-    }
-    const float inv = L > 0.f ? 1.f / L : 0.f;
-    *reinterpret_cast<__nv_bfloat162*>(out + (static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d) =
-        __floats2bfloat162_rn(ax * inv, ay * inv);
+    out[(static_cast<int64_t>(b) * p.Hq + g * G + h) * D + d] = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
     if (p.lse && d == 0)
       p.lse[static_cast<int64_t>(b) * p.Hq + g * G + h] =
           L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
   }
-  cluster_sync_all();  // keep this CTA's partials alive until the partner has read them
 }
 
 // Maximum dynamic shared memory for `kern` on the current device, set once.
@@ -769,7 +822,7 @@ bool allow_smem(K kern, int smem, bool* done) {
 template <typename T, int D, int G, bool FUSED, bool CLUSTER>
 int launch_one(const DecodeParams& p, cudaStream_t st) {
   constexpr bool TC = sizeof(T) == 2;  // bf16: streamed tensor-core kernel; fp32: exact FMA kernel
-  constexpr int smem = TC ? pipe_smem_bytes<D>() : 2 * ROWS * D * static_cast<int>(sizeof(T));
+  constexpr int smem = TC ? pipe_smem_bytes<D, G>() : 2 * ROWS * D * static_cast<int>(sizeof(T));
   const int ncl = TC ? kPipeCluster : (CLUSTER ? kMaxClusterSplits : 1);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(TC ? kPipeCluster : (CLUSTER ? kMaxClusterSplits : p.nsplit), p.Hkv, p.B);
@@ -856,7 +909,7 @@ extern "C" int sep_attn_decode(const sepcache* c, int layer, const void* q, int 
   if (!sep::aligned16(q) || !sep::aligned16(out) || !sep::aligned16(workspace)) return SEP_EALIGN;
   const WsLayout w = ws_layout(c, Hq);
   if (workspace_bytes < w.ml + w.o + w.ticket) return SEP_EINVAL;
-  DecodeParams p;
+  DecodeParams p = {};
   p.q = q;
   p.kc = c->k;
   p.vc = c->v;
@@ -909,7 +962,7 @@ extern "C" int sep_attn_decode_step(const sepcache* c, int layer, const void* q,
     const int rc = sep::cache_advance(c, is_sep_new, st);
     if (rc != SEP_OK) return rc;
   }
-  DecodeParams p;
+  DecodeParams p = {};
   p.q = q;
   p.kc = c->k;
   p.vc = c->v;
@@ -932,6 +985,7 @@ extern "C" int sep_attn_decode_step(const sepcache* c, int layer, const void* q,
   p.Hkv = c->Hkv;
   p.cap = c->cap;
   p.nsplit = (c->cap + ROWS - 1) / ROWS;
+  p.early = layer > 0;  // the step's metadata was advanced in the layer-0 call
   const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(c->D));
   p.scale_log2 = sc * 1.44269504088896340736f;
   if (c->dtype == SEP_BF16)
@@ -996,7 +1050,7 @@ extern "C" int sep_attn_decode_noalloc(const sepcache* c, int layer, const void*
   // the tickets must start at zero (the array keeps the previous call's contents)
   if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(c->B) * c->Hkv * 4, st) != cudaSuccess)
     return SEP_ECUDA;
-  DecodeParams p;
+  DecodeParams p = {};
   p.q = q;
   p.kc = c->k;
   p.vc = c->v;
