@@ -24,13 +24,16 @@
 //     from the first tile's lo); per-tile masks keep each tile's own set.
 // The kernel is persistent (one CTA per SM, items heaviest first, strided
 // over the grid).  Warps 0-3 and 4-7 are the softmax warpgroups of tiles A
-// and B (thread = query row = TMEM lane), warp 8 issues TMA loads, warp 9
-// owns TMEM and issues tcgen05.mma.  TMEM: S_A | S_B | O_A | O_B; each tile's
-// P (bf16) is written over the first 64 columns of its S and feeds the PV
-// MMA from TMEM.  While one warpgroup runs its softmax the tensor core works
-// on the other tile, and the next item's Q/K/V loads overlap the current
-// item's tail.  The running maximum moves (and O is rescaled) only when it
-// grows by more than 2^8, so P stays <= 256.
+// and B (thread = query row = TMEM lane), warp 8 issues TMA loads, warps 9
+// and 10 issue the tcgen05.mma of tiles A and B (warp 9 owns TMEM).  TMEM:
+// S_A | S_B | O_A | O_B, and for D = 64 also P_A | P_B, so that S of the next
+// block is computed while the softmax of this one still runs; for D = 128 a
+// tile's P (bf16) is written over the first 64 columns of its S.  P feeds
+// the PV MMA from TMEM.  While one warpgroup runs its softmax the tensor
+// core works on the other tile, and the next item's Q/K/V loads overlap the
+// current item's tail.  The reference maximum moves (and O is rescaled) only
+// when a block's row sum would exceed 2^16, and then to the block's exact
+// maximum.
 #include <string.h>
 
 #include "common.cuh"
@@ -40,9 +43,10 @@ namespace {
 
 constexpr int BM = 128;  // query rows per tile
 constexpr int BN = 128;  // keys per block
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kTmaWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kMmaWarp = 9;   // MMA issuer of tile A (and TMEM owner)
+constexpr int kMmaWarpB = 10; // MMA issuer of tile B
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -60,6 +64,11 @@ struct Cfg {
   static constexpr int BYTES = OFF_BAR + 512;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
+  // D = 64 leaves room for a separate P region per tile (bf16 pairs of 128
+  // keys in 64 columns): S of the next block can then be computed while the
+  // softmax of this one is still running.  D = 128 writes P over S.
+  static constexpr bool SEP_P = D == 64;
+  static constexpr uint32_t COL_P0 = SEP_P ? 384 : COL_S0, COL_P1 = SEP_P ? 448 : COL_S1;
 };
 
 template <int NST>
@@ -67,6 +76,7 @@ struct Bars {
   uint64_t q_full, q_empty;
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t s_free[2], pv_done[2];  // separate-P protocol: S read back / P*V done
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -154,6 +164,93 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   sep::mbar_wait(bar, parity, &dummy, nullptr);
 }
 
+// MMA issue for both tiles from one thread, P written over S (D = 128): per
+// block, tile A's P*V of the previous block then its S, then tile B's.
+template <int D>
+__device__ __forceinline__ void mma_single_issuer(const Params& p, uint8_t* smem, uint32_t tmem,
+                                                  Bars<Cfg<D>::NST>* bars, volatile int* abort) {
+  using C = Cfg<D>;
+  constexpr int NST = C::NST;
+  constexpr uint32_t idesc_s = sep::idesc_bf16_f32(BM, BN, false);
+  constexpr uint32_t idesc_o = sep::idesc_bf16_f32(BM, D, true);
+  // descriptors built once (see the per-tile issuers)
+  const uint64_t dq0 = sep::smem_desc_sw128(sep::smem_u32(smem + C::OFF_QA), 16);
+  const uint64_t dq1 = sep::smem_desc_sw128(sep::smem_u32(smem + C::OFF_QB), 16);
+  const uint64_t dk0 = sep::smem_desc_sw128(sep::smem_u32(smem + C::OFF_K), 16);
+  const uint64_t dv0 = sep::smem_desc_sw128(sep::smem_u32(smem + C::OFF_V), C::REG);
+  uint32_t gblk = 0, nitem = 0, pphase = 0;  // bit t: phase of p_full[t]
+  bool ok = true;
+  bool v_ready = false;  // V of the block whose PVs are being issued has landed
+  auto issue_pv = [&](int t, uint32_t vblk, bool first) -> bool {
+    if (!sep::mbar_wait(&bars->p_full[t], (pphase >> t) & 1u, abort, p.err)) return false;
+    pphase ^= 1u << t;
+    if (!v_ready && !sep::mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err))
+      return false;
+    v_ready = true;
+    if (first && nitem > 0 && !sep::mbar_wait(&bars->o_empty[t], (nitem - 1) & 1, abort, p.err))
+      return false;
+    sep::tc_fence_after();
+    const uint64_t dv = dv0 + static_cast<uint64_t>((vblk % NST) * (C::KV_BYTES >> 4));
+    const uint32_t ptm = tmem + (t ? C::COL_P1 : C::COL_P0);
+    const uint32_t otm = tmem + (t ? C::COL_O1 : C::COL_O0);
+#pragma unroll
+    for (int kk = 0; kk < BN / 16; ++kk)
+      sep::mma_bf16_ts(otm, ptm + kk * 8, dv + kk * (2048 >> 4), idesc_o, (!first || kk > 0) ? 1u : 0u);
+    return true;
+  };
+  auto issue_s = [&](int t, uint32_t kblk) {
+    const uint64_t dk = dk0 + static_cast<uint64_t>((kblk % NST) * (C::KV_BYTES >> 4));
+    const uint64_t dq = t ? dq1 : dq0;
+    const uint32_t stm = tmem + (t ? C::COL_S1 : C::COL_S0);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::REG + (kk % 4) * 32) >> 4);
+      sep::mma_bf16_ss(stm, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
+    }
+    sep::mma_commit(&bars->s_full[t]);
+  };
+  for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
+    const Item it = make_item(p, item);
+    if (!sep::mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
+    bool prev_a = false, prev_b = false;  // tile kept the previous block
+    bool pv_a = false, pv_b = false;      // tile already accumulated into O this item
+    for (int j = 0; j < it.nblk; ++j, ++gblk) {
+      if (!sep::mbar_wait(&bars->k_full[gblk % NST], (gblk / NST) & 1, abort, p.err)) {
+        ok = false;
+        break;
+      }
+      sep::tc_fence_after();
+      const bool act_a = block_active(it, 0, j, p.S), act_b = block_active(it, 1, j, p.S);
+      v_ready = false;
+      if (prev_a) {
+        if (!(ok = issue_pv(0, gblk - 1, !pv_a))) break;
+        pv_a = true;
+      }
+      if (act_a) issue_s(0, gblk);
+      if (prev_b) {
+        if (!(ok = issue_pv(1, gblk - 1, !pv_b))) break;
+        pv_b = true;
+      }
+      if (j > 0) sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
+      if (act_b) issue_s(1, gblk);
+      sep::mma_commit(&bars->k_empty[gblk % NST]);
+      if (j == it.nblk - 1) sep::mma_commit(&bars->q_empty);
+      prev_a = act_a;
+      prev_b = act_b;
+    }
+    if (!ok) break;
+    // last block's P*V of both tiles, then hand O to the epilogues
+    v_ready = false;
+    if (prev_a && !(ok = issue_pv(0, gblk - 1, !pv_a))) break;
+    sep::mma_commit(&bars->o_full[0]);
+    if (prev_b && !(ok = issue_pv(1, gblk - 1, !pv_b))) break;
+    sep::mma_commit(&bars->o_full[1]);
+    sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
+  }
+  sep::mma_commit(&bars->drain);
+  drain_wait(&bars->drain, 0);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     k_prefill_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -170,20 +267,23 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     sep::mbar_init(&bars->q_full, 1);
-    sep::mbar_init(&bars->q_empty, 1);
+    constexpr uint32_t kIssuers = C::SEP_P ? 2 : 1;  // one commit per MMA issuer
+    sep::mbar_init(&bars->q_empty, kIssuers);
     for (int s = 0; s < NST; ++s) {
       sep::mbar_init(&bars->k_full[s], 1);
-      sep::mbar_init(&bars->k_empty[s], 1);
+      sep::mbar_init(&bars->k_empty[s], kIssuers);
       sep::mbar_init(&bars->v_full[s], 1);
-      sep::mbar_init(&bars->v_empty[s], 1);
+      sep::mbar_init(&bars->v_empty[s], kIssuers);
     }
     for (int t = 0; t < 2; ++t) {
       sep::mbar_init(&bars->s_full[t], 1);
       sep::mbar_init(&bars->p_full[t], 128);
       sep::mbar_init(&bars->o_full[t], 1);
       sep::mbar_init(&bars->o_empty[t], 128);
+      sep::mbar_init(&bars->s_free[t], 128);
+      sep::mbar_init(&bars->pv_done[t], 1);
     }
-    sep::mbar_init(&bars->drain, 1);
+    sep::mbar_init(&bars->drain, kIssuers);
     bars->abort = 0;
     sep::mbar_fence_init();
   }
@@ -262,86 +362,106 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+  } else if (warp == kMmaWarp || warp == kMmaWarpB) {
+    // ------------------------------------------------------------ MMA issuers
+    // Separate P (D = 64): one issuing thread per tile, so that a tile's S
+    // and P*V wait only for that tile's softmax.  P over S (D = 128): one
+    // thread issues both tiles, P*V of a tile before its next S.  The MMAs
+    // of one thread complete in issue order; the barriers of the shared K,
+    // V and Q stages take one commit from each issuer.
+    if (!C::SEP_P) {
+      if (warp == kMmaWarp && lane == 0) mma_single_issuer<D>(p, smem, tmem, bars, abort);
+    } else if (lane == 0) {
+      const int t = warp == kMmaWarp ? 0 : 1;
       constexpr uint32_t idesc_s = sep::idesc_bf16_f32(BM, BN, false);
       constexpr uint32_t idesc_o = sep::idesc_bf16_f32(BM, D, true);
-      const uint32_t sq0 = sep::smem_u32(smem + C::OFF_QA), sq1 = sep::smem_u32(smem + C::OFF_QB);
-      uint32_t gblk = 0, nitem = 0, pphase = 0;  // bit t: phase of p_full[t]
+      // Shared-memory descriptors are built once: a K step only moves the
+      // start address, whose field (bits 0-13, address >> 4) takes the
+      // offset >> 4 without a carry (every address is below 256 KB).  Built
+      // per instruction, the descriptor arithmetic of this single thread
+      // costs about as much as the MMA itself.
+      const uint64_t dq = sep::smem_desc_sw128(sep::smem_u32(smem + (t ? C::OFF_QB : C::OFF_QA)), 16);
+      const uint64_t dk0 = sep::smem_desc_sw128(sep::smem_u32(smem + C::OFF_K), 16);
+      const uint64_t dv0 = sep::smem_desc_sw128(sep::smem_u32(smem + C::OFF_V), C::REG);
+      const uint32_t stm = tmem + (t ? C::COL_S1 : C::COL_S0);
+      const uint32_t ptm = tmem + (t ? C::COL_P1 : C::COL_P0);
+      const uint32_t otm = tmem + (t ? C::COL_O1 : C::COL_O0);
+      uint32_t gblk = 0, nitem = 0, pphase = 0;
+      uint32_t ns = 0;  // S products issued (separate-P protocol)
       bool ok = true;
       // O_t += P_t V (block `vblk` of the global stream); the first PV of an
       // item overwrites O_t, so it waits until the previous item's epilogue
-      // of tile t has read O_t.
-      bool v_ready = false;  // V of the block whose PVs are being issued has landed
-      auto issue_pv = [&](int t, uint32_t vblk, bool first) -> bool {
-        if (!sep::mbar_wait(&bars->p_full[t], (pphase >> t) & 1u, abort, p.err)) return false;
-        pphase ^= 1u << t;
-        if (!v_ready && !sep::mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err))
-          return false;
-        v_ready = true;
+      // of this tile has read O_t.
+      auto issue_pv = [&](uint32_t vblk, bool first) -> bool {
+        if (!sep::mbar_wait(&bars->p_full[t], pphase, abort, p.err)) return false;
+        pphase ^= 1u;
+        if (!sep::mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err)) return false;
         if (first && nitem > 0 && !sep::mbar_wait(&bars->o_empty[t], (nitem - 1) & 1, abort, p.err))
           return false;
         sep::tc_fence_after();
-        const uint32_t sv = sep::smem_u32(smem + C::OFF_V + (vblk % NST) * C::KV_BYTES);
-        const uint32_t ptm = tmem + (t ? C::COL_S1 : C::COL_S0);
-        const uint32_t otm = tmem + (t ? C::COL_O1 : C::COL_O0);
+        const uint64_t dv = dv0 + static_cast<uint64_t>((vblk % NST) * (C::KV_BYTES >> 4));
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sep::smem_desc_sw128(sv + kk * 2048, C::REG);
-          sep::mma_bf16_ts(otm, ptm + kk * 8, bd, idesc_o, (!first || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BN / 16; ++kk)  // 16 keys = 2048 bytes of V per step
+          sep::mma_bf16_ts(otm, ptm + kk * 8, dv + kk * (2048 >> 4), idesc_o, (!first || kk > 0) ? 1u : 0u);
+        if (C::SEP_P) sep::mma_commit(&bars->pv_done[t]);
         return true;
       };
-      auto issue_s = [&](int t, uint32_t kblk) {
-        const uint32_t sk = sep::smem_u32(smem + C::OFF_K + (kblk % NST) * C::KV_BYTES);
-        const uint32_t sq = t ? sq1 : sq0;
-        const uint32_t stm = tmem + (t ? C::COL_S1 : C::COL_S0);
+      auto issue_s = [&](uint32_t kblk) -> bool {
+        if (C::SEP_P) {
+          // S_t is free once the softmax has read the previous block's scores
+          if (ns > 0 && !sep::mbar_wait(&bars->s_free[t], (ns - 1) & 1, abort, p.err)) return false;
+          ++ns;
+          sep::tc_fence_after();
+        }
+        const uint64_t dk = dk0 + static_cast<uint64_t>((kblk % NST) * (C::KV_BYTES >> 4));
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = sep::smem_desc_sw128(sq + (kk / 4) * C::REG + (kk % 4) * 32, 16);
-          const uint64_t bd = sep::smem_desc_sw128(sk + (kk / 4) * C::REG + (kk % 4) * 32, 16);
-          sep::mma_bf16_ss(stm, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < D / 16; ++kk) {  // 16 dims: 32 bytes within a 64-column region
+          const uint64_t off = static_cast<uint64_t>(((kk / 4) * C::REG + (kk % 4) * 32) >> 4);
+          sep::mma_bf16_ss(stm, dq + off, dk + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         sep::mma_commit(&bars->s_full[t]);
+        return true;
       };
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
         const Item it = make_item(p, item);
         if (!sep::mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
-        bool prev_a = false, prev_b = false;  // tile kept the previous block
-        bool pv_a = false, pv_b = false;      // tile already accumulated into O this item
+        bool prev = false;  // this tile kept the previous block
+        bool pv = false;    // this tile already accumulated into O this item
         for (int j = 0; j < it.nblk; ++j, ++gblk) {
           if (!sep::mbar_wait(&bars->k_full[gblk % NST], (gblk / NST) & 1, abort, p.err)) {
             ok = false;
             break;
           }
           sep::tc_fence_after();
-          const bool act_a = block_active(it, 0, j, p.S), act_b = block_active(it, 1, j, p.S);
-          v_ready = false;
-          // tile A: finish the previous block's PV, then this block's S
-          if (prev_a) {
-            if (!(ok = issue_pv(0, gblk - 1, !pv_a))) break;
-            pv_a = true;
+          const bool act = block_active(it, t, j, p.S);
+          if constexpr (C::SEP_P) {
+            // S of block j (as soon as the softmax has read the previous
+            // scores), then P*V of block j - 1 once its P is there
+            if (act && !(ok = issue_s(gblk))) break;
+            sep::mma_commit(&bars->k_empty[gblk % NST]);
+            if (j == it.nblk - 1) sep::mma_commit(&bars->q_empty);
+            if (prev) {
+              if (!(ok = issue_pv(gblk - 1, !pv))) break;
+              pv = true;
+            }
+            if (j > 0) sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
+          } else {
+            // P is written over S: the previous block's P*V before this S
+            if (prev) {
+              if (!(ok = issue_pv(gblk - 1, !pv))) break;
+              pv = true;
+            }
+            if (j > 0) sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
+            if (act) issue_s(gblk);
+            sep::mma_commit(&bars->k_empty[gblk % NST]);
+            if (j == it.nblk - 1) sep::mma_commit(&bars->q_empty);
           }
-          if (act_a) issue_s(0, gblk);
-          if (prev_b) {
-            if (!(ok = issue_pv(1, gblk - 1, !pv_b))) break;
-            pv_b = true;
-          }
-          if (j > 0) sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
-          if (act_b) issue_s(1, gblk);
-          sep::mma_commit(&bars->k_empty[gblk % NST]);
-          if (j == it.nblk - 1) sep::mma_commit(&bars->q_empty);
-          prev_a = act_a;
-          prev_b = act_b;
+          prev = act;
         }
         if (!ok) break;
-        // last block's PV of both tiles, then hand O to the epilogues
-        v_ready = false;
-        if (prev_a && !(ok = issue_pv(0, gblk - 1, !pv_a))) break;
-        sep::mma_commit(&bars->o_full[0]);
-        if (prev_b && !(ok = issue_pv(1, gblk - 1, !pv_b))) break;
-        sep::mma_commit(&bars->o_full[1]);
+        // last block's P*V, then hand O to the epilogue
+        if (prev && !(ok = issue_pv(gblk - 1, !pv))) break;
+        sep::mma_commit(&bars->o_full[t]);
         sep::mma_commit(&bars->v_empty[(gblk - 1) % NST]);
       }
       sep::mma_commit(&bars->drain);
@@ -353,8 +473,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = threadIdx.x & 127;  // tile row == TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_col = tmem + lane_base + (t ? C::COL_S1 : C::COL_S0);
+    const uint32_t p_col = tmem + lane_base + (t ? C::COL_P1 : C::COL_P0);
     const uint32_t o_col = tmem + lane_base + (t ? C::COL_O1 : C::COL_O0);
     uint32_t sphase = 0, nitem = 0;
+    uint32_t npv = 0;  // P*V products of this tile issued so far (separate-P protocol)
+    // Separate-P protocol, after the scores of a block are in registers:
+    // free S_t for the next block's MMA, then wait until the previous P*V
+    // (reader of P_t, writer of O_t) is done.
+    auto s_read_pv_wait = [&]() -> bool {
+      if constexpr (C::SEP_P) {
+        sep::tc_fence_before();
+        sep::mbar_arrive(&bars->s_free[t]);
+        if (npv > 0 && !__all_sync(0xffffffffu, sep::mbar_wait(&bars->pv_done[t], (npv - 1) & 1, abort, p.err)))
+          return false;
+        ++npv;
+        sep::tc_fence_after();
+      }
+      return true;
+    };
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
       const Item it = make_item(p, item);
@@ -414,18 +550,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         sphase ^= 1;
         sep::tc_fence_after();
         // Fast path (after the block where a row first saw a key): one pass
-        // over S against the running reference m_ref, P kept in registers
-        // until every score of the row is known to be within 2^8 of m_ref.
-        // Otherwise (first block, or a score that grew past 2^8): the exact
-        // two-pass path that moves the reference and rescales O.
+        // over S against the reference m_ref, P kept in registers until the
+        // block's row sum is known to stay within 2^16.  Otherwise (first
+        // block, or scores that grew too far): the exact two-pass path, which
+        // moves the reference to the block maximum when that exceeds it by
+        // more than 2^8 and rescales O.
         bool fast_done = false;
         if (__all_sync(0xffffffffu, m_ref != -INFINITY)) {
           uint32_t pk[64];
           uint32_t ra[32], rb[32];
-          float sm[8], pm[2];
+          float2 sm2[4];  // partial row sums, four independent pairs
 #pragma unroll
-          for (int u = 0; u < 8; ++u) sm[u] = 0.f;
-          pm[0] = pm[1] = 0.f;
+          for (int u = 0; u < 4; ++u) sm2[u] = make_float2(0.f, 0.f);
+          const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+          const float2 nm2 = make_float2(-m_ref, -m_ref);
           sep::tmem_ld32(s_col, ra);
           sep::tmem_wait_ld_r32(ra);
 #pragma unroll
@@ -440,36 +578,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (__all_sync(0xffffffffu, kc == 0xffffffffu)) {
 #pragma unroll
               for (int e = 0; e < 32; e += 2) {
-                const float p0 = sep::ex2_approx(fmaf(__uint_as_float(cur[e]), p.scale_log2, -m_ref));
-                const float p1 = sep::ex2_approx(fmaf(__uint_as_float(cur[e + 1]), p.scale_log2, -m_ref));
-                sm[e & 7] += p0;
-                sm[(e + 1) & 7] += p1;
-                pm[0] = fmaxf(pm[0], p0);
-                pm[1] = fmaxf(pm[1], p1);
-                pk[16 * c + (e >> 1)] = sep::pack_bf16x2(p0, p1);
+                const float2 y = sep::ffma2(make_float2(__uint_as_float(cur[e]), __uint_as_float(cur[e + 1])), sc2, nm2);
+                const float2 pp = make_float2(sep::ex2_approx(y.x), sep::ex2_approx(y.y));
+                sm2[(e >> 1) & 3] = sep::fadd2(sm2[(e >> 1) & 3], pp);
+                pk[16 * c + (e >> 1)] = sep::pack_bf16x2(pp.x, pp.y);
               }
             } else {
 #pragma unroll
               for (int e = 0; e < 32; e += 2) {
                 const float x0 = (kc >> e) & 1u ? __uint_as_float(cur[e]) : -INFINITY;
                 const float x1 = (kc >> (e + 1)) & 1u ? __uint_as_float(cur[e + 1]) : -INFINITY;
-                const float p0 = sep::ex2_approx(fmaf(x0, p.scale_log2, -m_ref));
-                const float p1 = sep::ex2_approx(fmaf(x1, p.scale_log2, -m_ref));
-                sm[e & 7] += p0;
-                sm[(e + 1) & 7] += p1;
-                pm[0] = fmaxf(pm[0], p0);
-                pm[1] = fmaxf(pm[1], p1);
-                pk[16 * c + (e >> 1)] = sep::pack_bf16x2(p0, p1);
+                const float2 y = sep::ffma2(make_float2(x0, x1), sc2, nm2);
+                const float2 pp = make_float2(sep::ex2_approx(y.x), sep::ex2_approx(y.y));
+                sm2[(e >> 1) & 3] = sep::fadd2(sm2[(e >> 1) & 3], pp);
+                pk[16 * c + (e >> 1)] = sep::pack_bf16x2(pp.x, pp.y);
               }
             }
             if (c < 3) sep::tmem_wait_ld_r32(nxt);
           }
-          const float pmax = fmaxf(pm[0], pm[1]);
-          // 2^8 bound on P (the lazy-rescale rule); a NaN here also falls back
-          if (!__any_sync(0xffffffffu, !(pmax <= 256.f))) {
-            l += ((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7]));
-            sep::tmem_st32(s_col, pk);
-            sep::tmem_st32(s_col + 32, pk + 32);
+          const float2 s01 = sep::fadd2(sm2[0], sm2[1]), s23 = sep::fadd2(sm2[2], sm2[3]);
+          const float rowsum = (s01.x + s01.y) + (s23.x + s23.y);
+          // Every P of the block is at most its row sum: up to 2^16 (P in
+          // bf16, O and l in fp32) the block stays on the reference m_ref; an
+          // overflow or a NaN fails the test as well, and the exact path
+          // below moves the reference instead.
+          if (!__any_sync(0xffffffffu, !(rowsum <= 65536.f))) {
+            l += rowsum;
+            if (!s_read_pv_wait()) {
+              ok = false;
+              break;
+            }
+            sep::tmem_st32(p_col, pk);
+            sep::tmem_st32(p_col + 32, pk + 32);
             fast_done = true;
           }
         }
@@ -504,8 +644,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             alpha = sep::ex2_approx(m_ref - mblk);  // 0 while m_ref is -inf
             m_ref = mblk;
           }
-          // S_t of this block was issued after this tile's previous P*V, and
-          // MMAs complete in order, so that P*V is done: O_t may be rescaled.
+          // D = 128: S_t of this block was issued after this tile's previous
+          // P*V, and MMAs complete in order, so that P*V is done.  Separate P:
+          // wait for it (pass 2 below still reads S_t; it is freed after).
+          if constexpr (C::SEP_P) {
+            if (npv > 0 && !__all_sync(0xffffffffu, sep::mbar_wait(&bars->pv_done[t], (npv - 1) & 1, abort, p.err))) {
+              ok = false;
+              break;
+            }
+            sep::tc_fence_after();
+          }
           if (j > 0 && __any_sync(0xffffffffu, grow)) {
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -533,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!__any_sync(0xffffffffu, k0 != 0u)) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) r[e] = 0u;
-              sep::tmem_st16(s_col + 16 * c, r);
+              sep::tmem_st16(p_col + 16 * c, r);
               k0 = k1;
               k1 = k2;
               k2 = keep[3];
@@ -551,12 +699,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               sm[(e + 1) & 7] += p1;
               r[e >> 1] = sep::pack_bf16x2(p0, p1);
             }
-            sep::tmem_st16(s_col + 16 * c, r);
+            sep::tmem_st16(p_col + 16 * c, r);
             k0 = k1;
             k1 = k2;
             k2 = keep[3];
           }
           l = l * alpha + (((sm[0] + sm[1]) + (sm[2] + sm[3])) + ((sm[4] + sm[5]) + (sm[6] + sm[7])));
+          if constexpr (C::SEP_P) {
+            // every score of the block has been read: free S_t (the previous
+            // P*V was waited for above)
+            sep::tmem_wait_st();
+            sep::tc_fence_before();
+            sep::mbar_arrive(&bars->s_free[t]);
+            ++npv;
+          }
         }
         sep::tmem_wait_st();
         sep::tc_fence_before();
