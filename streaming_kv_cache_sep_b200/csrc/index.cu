@@ -19,6 +19,8 @@ struct SepIdSet {
 
 __global__ void k_flags_from_ids(const int32_t* __restrict__ ids, int64_t n_tok, SepIdSet set,
                                  uint8_t* __restrict__ is_sep) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the ids' producer
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (; t < n_tok; t += stride) {
@@ -30,10 +32,13 @@ __global__ void k_flags_from_ids(const int32_t* __restrict__ ids, int64_t n_tok,
   }
 }
 
-// One CTA per (chunk of kChunk positions, sequence).  Each CTA counts the
-// separators before its chunk and in the whole sequence (the flags of a
-// sequence are at most a few hundred KB, read from L2), then scans its own
-// chunk: thread t owns kPer consecutive positions.  No CTA waits on another.
+// One CTA per (chunk of kChunk positions, sequence).  Warp w of the CTA
+// owns kPer x 32 consecutive positions, lane l the positions 32e + l
+// (e < kPer), so that flag reads and prefix writes are coalesced.  A warp
+// ranks its separators with ballots, one block-wide scan of the warp totals
+// gives the offsets.  With several chunks per sequence each CTA first counts
+// the separators before its chunk and in the whole sequence (read from L2);
+// no CTA waits on another.
 constexpr int kScanThreads = 1024;
 constexpr int kPer = 16;
 constexpr int kChunk = kScanThreads * kPer;
@@ -59,50 +64,55 @@ __global__ void __launch_bounds__(kScanThreads) k_build_index(const uint8_t* __r
                                                               int32_t* __restrict__ idx,
                                                               int32_t* __restrict__ count) {
   __shared__ int red[33];
-  __shared__ int wsum[32];
+  __shared__ int wsum[33];
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the flags' producer
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.y;
   const int64_t chunk0 = static_cast<int64_t>(blockIdx.x) * kChunk;
   const uint8_t* f = is_sep + static_cast<int64_t>(b) * S;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt = (1u << lane) - 1u;
 
   // separators before the chunk, and in the whole sequence
-  int before = 0, total = 0;
-  for (int64_t p = threadIdx.x; p < S; p += kScanThreads) {
-    int v = f[p];
-    total += v;
-    before += (p < chunk0) ? v : 0;
+  int before = 0, total = -1;
+  if (gridDim.x > 1) {
+    int tot = 0;
+    for (int64_t p = threadIdx.x; p < S; p += kScanThreads) {
+      const int v = f[p] != 0;
+      tot += v;
+      before += (p < chunk0) ? v : 0;
+    }
+    before = block_sum_1024(before, red);
+    total = block_sum_1024(tot, red);
   }
-  before = block_sum_1024(before, red);
-  total = block_sum_1024(total, red);
 
-  // local counts of this thread's kPer positions
-  const int64_t p0 = chunk0 + static_cast<int64_t>(threadIdx.x) * kPer;
+  // this warp's flags: bit e of `bits` is position w0 + 32e + lane
+  const int64_t w0 = chunk0 + static_cast<int64_t>(warp) * 32 * kPer;
   uint32_t bits = 0;
+  int wtot = 0;
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
-    int64_t p = p0 + e;
-    if (p < S && f[p]) bits |= 1u << e;
+    const int64_t pos = w0 + 32 * e + lane;
+    const bool fl = pos < S && f[pos] != 0;
+    bits |= static_cast<uint32_t>(fl) << e;
   }
-  int mine = __popc(bits);
-  // exclusive scan of `mine` over the block
-  int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = mine;
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  if (lane == 31) wsum[warp] = incl;
+#pragma unroll
+  for (int e = 0; e < kPer; ++e) wtot += __popc(__ballot_sync(0xffffffffu, (bits >> e) & 1u));
+  // exclusive scan of the warp totals
+  if (lane == 0) wsum[warp] = wtot;
   __syncthreads();
   if (warp == 0) {
-    int x = wsum[lane];
+    const int x = wsum[lane];
     int xi = x;
     for (int o = 1; o < 32; o <<= 1) {
-      int y = __shfl_up_sync(0xffffffffu, xi, o);
+      const int y = __shfl_up_sync(0xffffffffu, xi, o);
       if (lane >= o) xi += y;
     }
-    wsum[lane] = xi - x;  // exclusive over warps
+    wsum[lane] = xi - x;
+    if (lane == 31) wsum[32] = xi;  // the chunk's total
   }
   __syncthreads();
-  int run = before + wsum[warp] + (incl - mine);
+  if (total < 0) total = wsum[32];  // one chunk: the sequence's total
 
   int32_t* pre = prefix + static_cast<int64_t>(b) * (S + 1);
   int32_t* ix = idx + static_cast<int64_t>(b) * S;
@@ -110,18 +120,20 @@ __global__ void __launch_bounds__(kScanThreads) k_build_index(const uint8_t* __r
     pre[0] = 0;
     count[b] = total;
   }
+  int run = before + wsum[warp];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
-    int64_t p = p0 + e;
-    if (p < S) {
-      if (bits & (1u << e)) {
-        ix[run] = static_cast<int32_t>(p);
-        ++run;
-      }
-      pre[p + 1] = run;
+    const int64_t pos = w0 + 32 * e + lane;
+    const uint32_t bal = __ballot_sync(0xffffffffu, (bits >> e) & 1u);
+    const int rank = run + __popc(bal & lt);
+    if (pos < S) {
+      const bool fl = (bits >> e) & 1u;
+      if (fl) ix[rank] = static_cast<int32_t>(pos);
+      pre[pos + 1] = rank + static_cast<int>(fl);
       // idx slots at or after the total count are padding
-      if (p >= total) ix[p] = -1;
+      if (pos >= total) ix[pos] = -1;
     }
+    run += __popc(bal);
   }
 }
 
@@ -165,8 +177,9 @@ extern "C" int sep_flags_from_ids(const int32_t* ids, int64_t n_tok, const int32
   for (int k = 0; k < n_sep_ids; ++k) set.id[k] = sep_ids[k];
   int64_t blocks = (n_tok + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  k_flags_from_ids<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      ids, n_tok, set, is_sep);
+  if (sep::launch_pdl(k_flags_from_ids, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                      static_cast<cudaStream_t>(stream), ids, n_tok, set, is_sep) != cudaSuccess)
+    return SEP_ECUDA;
   return sep::launch_status();
 }
 
@@ -175,8 +188,9 @@ extern "C" int sep_build_index(const uint8_t* is_sep, int B, int S, int32_t* pre
   if (B < 1 || S < 1 || B > 65535) return SEP_EINVAL;
   if (!is_sep || !prefix || !idx || !count) return SEP_ENULL;
   dim3 grid((S + kChunk - 1) / kChunk, B);
-  k_build_index<<<grid, kScanThreads, 0, static_cast<cudaStream_t>(stream)>>>(is_sep, S, prefix,
-                                                                              idx, count);
+  if (sep::launch_pdl(k_build_index, grid, dim3(kScanThreads), 0, static_cast<cudaStream_t>(stream),
+                      is_sep, S, prefix, idx, count) != cudaSuccess)
+    return SEP_ECUDA;
   return sep::launch_status();
 }
 

@@ -60,7 +60,10 @@ struct Cfg {
   static constexpr int OFF_QB = OFF_QA + Q_BYTES;
   static constexpr int OFF_K = OFF_QB + Q_BYTES;
   static constexpr int OFF_V = OFF_K + NST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + NST * KV_BYTES;
+  // D = 64: per-tile staging of the output tile for one tensor store
+  static constexpr int OFF_STG = OFF_V + NST * KV_BYTES;
+  static constexpr int STG_BYTES = D == 64 ? 2 * Q_BYTES : 0;
+  static constexpr int OFF_BAR = OFF_STG + STG_BYTES;
   static constexpr int BYTES = OFF_BAR + 512;
   static constexpr int ALLOC = BYTES + 1024;  // slack for 1024-byte alignment
   static constexpr uint32_t COL_S0 = 0, COL_S1 = 128, COL_O0 = 256, COL_O1 = 256 + D;
@@ -255,7 +258,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     k_prefill_tc(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_kc,
-                 const __grid_constant__ CUtensorMap tm_vc, const Params p) {
+                 const __grid_constant__ CUtensorMap tm_vc, const __grid_constant__ CUtensorMap tm_o,
+                 const Params p) {
   using C = Cfg<D>;
   constexpr int NST = C::NST;
   extern __shared__ uint8_t smem_raw[];
@@ -295,6 +299,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   sep::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+  // launched with programmatic serialization: the set-up above overlapped
+  // the previous kernel; its outputs (index, gathered rows) are read below
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (threadIdx.x == 0) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == kTmaWarp) {
     // ------------------------------------------------------------ producer
@@ -556,16 +564,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         // moves the reference to the block maximum when that exceeds it by
         // more than 2^8 and rescales O.
         bool fast_done = false;
-        if (__all_sync(0xffffffffu, m_ref != -INFINITY)) {
+        uint32_t ra[32], rb[32];
+        sep::tmem_ld32(s_col, ra);
+        sep::tmem_wait_ld_r32(ra);
+        // A row without a reference yet (its first kept block) takes the
+        // maximum of its kept scores among the first 32 keys: never above the
+        // block maximum, so P cannot underflow, and the row-sum test below
+        // catches a reference that is too low.
+        float m_use = m_ref;
+        if (__any_sync(0xffffffffu, m_ref == -INFINITY)) {
+          float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            mx[e & 3] = fmaxf(mx[e & 3], (keep[0] >> e) & 1u ? __uint_as_float(ra[e]) : -INFINITY);
+          const float m0 = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+          if (m_ref == -INFINITY) m_use = m0 * p.scale_log2;
+        }
+        if (__all_sync(0xffffffffu, m_use != -INFINITY)) {
           uint32_t pk[64];
-          uint32_t ra[32], rb[32];
           float2 sm2[4];  // partial row sums, four independent pairs
 #pragma unroll
           for (int u = 0; u < 4; ++u) sm2[u] = make_float2(0.f, 0.f);
           const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-          const float2 nm2 = make_float2(-m_ref, -m_ref);
-          sep::tmem_ld32(s_col, ra);
-          sep::tmem_wait_ld_r32(ra);
+          const float2 nm2 = make_float2(-m_use, -m_use);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             uint32_t* cur = (c & 1) ? rb : ra;
@@ -603,6 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // overflow or a NaN fails the test as well, and the exact path
           // below moves the reference instead.
           if (!__any_sync(0xffffffffu, !(rowsum <= 65536.f))) {
+            m_ref = m_use;
             l += rowsum;
             if (!s_read_pv_wait()) {
               ok = false;
@@ -726,6 +748,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       sep::tc_fence_after();
       const float inv = 1.f / l;
+      if (C::STG_BYTES > 0 && my_q0 + BM <= p.S) {
+        // whole tile: rows into a 128-byte swizzled staging tile (16-byte
+        // unit u of row r at u ^ (r & 7): one row per thread, conflict-free),
+        // then one tensor store.  A thread per row writing global memory
+        // directly touches 32 lines per warp instruction.
+        uint8_t* stg = smem + C::OFF_STG + t * C::Q_BYTES;
+        if (row == 0) sep::bulk_wait_read0();  // the previous store has read the tile
+        sep::named_bar_sync(1 + t, 128);
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          sep::tmem_ld32(o_col + 32 * c, o);
+          sep::tmem_wait_ld_r32(o);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 w;
+            w.x = sep::pack_bf16x2(__uint_as_float(o[8 * q + 0]) * inv, __uint_as_float(o[8 * q + 1]) * inv);
+            w.y = sep::pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
+            w.z = sep::pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
+            w.w = sep::pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
+            const int u = 4 * c + q;
+            *reinterpret_cast<uint4*>(stg + row * 128 + ((u ^ (row & 7)) << 4)) = w;
+          }
+        }
+        sep::fence_proxy_async_smem();
+        sep::named_bar_sync(1 + t, 128);
+        if (row == 0) {
+          sep::tma_store_2d(&tm_o, 0, static_cast<int32_t>(static_cast<int64_t>(b * p.Hq + h) * p.S + my_q0), stg);
+          sep::bulk_commit();
+        }
+      } else {
       __nv_bfloat16* orow = p.out + (static_cast<int64_t>(b * p.Hq + h) * p.S + i) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -744,12 +797,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      }
       if (p.lse && i < p.S)
         p.lse[static_cast<int64_t>(b * p.Hq + h) * p.S + i] =
             (m_ref + __log2f(l)) * 0.69314718055994530942f;
       sep::tc_fence_before();
       sep::mbar_arrive(&bars->o_empty[t]);
     }
+    if (C::STG_BYTES > 0 && row == 0) sep::bulk_wait0();  // output stores done before exit
   }
   sep::tc_fence_before();
   __syncthreads();
@@ -771,6 +826,8 @@ __global__ void __launch_bounds__(256) k_gather_sep_rows(
     const int32_t* __restrict__ prefix, const int32_t* __restrict__ idx, int Hkv, int S, int a,
     __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, int32_t* err) {
   constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the index's producer
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int g = blockIdx.y, b = blockIdx.z;
   const int r0 = blockIdx.x * 64;
   const int32_t* pre = prefix + static_cast<int64_t>(b) * (S + 1);
@@ -855,17 +912,18 @@ int launch(const void* q, const void* k, const void* v, const uint8_t* is_sep,
   const int64_t qrows = static_cast<int64_t>(B) * Hq * S;
   const int64_t krows = static_cast<int64_t>(B) * Hkv * S;
   if (qrows >= (1ll << 31) || krows >= (1ll << 31)) return SEP_EINVAL;
-  CUtensorMap mq, mk, mv, mkc, mvc;
-  if (!make_map(&mq, q, qrows, D) || !make_map(&mk, k, krows, D) || !make_map(&mv, v, krows, D) ||
+  CUtensorMap mq, mk, mv, mkc, mvc, mo;
+  if (!make_map(&mq, q, qrows, D) || !make_map(&mo, out, qrows, D) || !make_map(&mk, k, krows, D) ||
+      !make_map(&mv, v, krows, D) ||
       !make_map(&mkc, kc, krows, D) || !make_map(&mvc, vc, krows, D))
     return SEP_ECUDA;
 
   dim3 ggrid((S + 63) / 64, Hkv, B);
-  k_gather_sep_rows<D><<<ggrid, 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v), prefix, idx, Hkv,
-      S, a, static_cast<__nv_bfloat16*>(kc), static_cast<__nv_bfloat16*>(vc),
-      sep::device_error_word());
-  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  if (sep::launch_pdl(k_gather_sep_rows<D>, ggrid, dim3(256), 0, st,
+                      static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
+                      prefix, idx, Hkv, S, a, static_cast<__nv_bfloat16*>(kc),
+                      static_cast<__nv_bfloat16*>(vc), sep::device_error_word()) != cudaSuccess)
+    return SEP_ECUDA;
 
   Params p;
   p.is_sep = is_sep;
@@ -893,7 +951,9 @@ int launch(const void* q, const void* k, const void* v, const uint8_t* is_sep,
   p.lse = lse;
   p.err = sep::device_error_word();
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
-  k_prefill_tc<D><<<grid, kThreads, C::ALLOC, st>>>(mq, mk, mv, mkc, mvc, p);
+  if (sep::launch_pdl(k_prefill_tc<D>, dim3(grid), dim3(kThreads), C::ALLOC, st, mq, mk, mv, mkc,
+                      mvc, mo, p) != cudaSuccess)
+    return SEP_ECUDA;
   return sep::launch_status();
 }
 
