@@ -57,6 +57,40 @@ def _peaks():
         return dict(hbm=6650.0, bf16=1590.0, bf16_sust=1400.0, src="fallback")
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernel, from one ncu capture each (summaries under profiles/).  A figure
+# holds only for the kernel source it was taken on: when the hash of the
+# kernel's files differs, the traffic is reported as unknown (null).  `per` is the unit the
+# figure scales with: one launch, or one retained K/V row of one sequence
+# (the capture ran a smaller cache than the bench; decode traffic grows in
+# proportion to the retained rows).
+TRAFFIC = {
+    "prefill_pythia160m_b8h12_s2048_d64_bf16": dict(
+        bytes=82608128 + 9976576, per="launch", src=("prefill_tc.cu", "common.cuh"), sha1="33933b4438440541d25b84d21f8513b525cea57a"),
+}
+
+
+def _src_sha1(fnames):
+    import hashlib
+    h = hashlib.sha1()
+    for f in fnames:
+        with open(os.path.join(ROOT, "streaming_kv_cache_sep_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def _traffic(name, units):
+    t = TRAFFIC.get(name)
+    if t is None:
+        return None
+    try:
+        if _src_sha1(t["src"]) != t["sha1"]:
+            return None
+    except OSError:
+        return None
+    return int(round(t["bytes"] * (units if t["per"] == "row" else 1)))
+
+
 # ---------------------------------------------------------------- clocks
 
 
@@ -286,10 +320,21 @@ def bench_prefill(sl, args, world, rank):
     attn_s = statistics.mean(attn_ms) / 1e3
     achieved = wl.flops / attn_s / 1e12
     c = wl.cfg
+    # algorithmic bytes of one call: q, k, v read once, out and lse written
+    esz = wl.q.element_size()
+    alg_bytes = (wl.q.numel() + wl.k.numel() + wl.v.numel() + wl.out.numel()) * esz + wl.lse.numel() * 4
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16"],
-                "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4), "traffic": None,
+                "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4),
+                "traffic": _traffic(name, units=1),
+                "bytes_per_launch": int(alg_bytes), "launch_us": round(attn_s * 1e6, 3),
                 "kernel": "sep_attn_prefill (separator-row gather + tcgen05 attention)",
-                "peak_source": pk["src"] + " bf16 dense burst"}
+                "peak_source": pk["src"] + " bf16 dense burst",
+                # the same call against HBM: below the ridge point (bf16 peak /
+                # HBM bandwidth) the bytes bound the call before the FLOPs do
+                "hbm_view": {"achieved": round(alg_bytes / attn_s / 1e9, 1), "peak": pk["hbm"],
+                             "unit": "GB/s", "frac": round(alg_bytes / attn_s / 1e9 / pk["hbm"], 4),
+                             "flop_per_byte": round(wl.flops / alg_bytes, 1),
+                             "ridge_flop_per_byte": round(pk["bf16"] * 1e3 / pk["hbm"], 1)}}
     line = {
         "metric": PREFILL_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(t / K * 1e3, 5),
@@ -356,9 +401,11 @@ def _kept_pairs_rows(flags, c, rows):
 class DecodeWorkload:
     RING = 4
 
-    def __init__(self, sl, name, seed):
+    def __init__(self, sl, name, seed, layers=None):
         self.sl = sl
-        self.cfg = c = synth.WORKLOADS[name]
+        self.cfg = c = dict(synth.WORKLOADS[name])
+        if layers:
+            c["layers"] = layers
         self.B, self.Hq, self.Hkv, self.D, self.L = c["B"], c["Hq"], c["Hkv"], c["D"], c["layers"]
         self.cache = sl.SepCache(c["a"], c["s"], c["past"], c["w"], self.L, self.B, self.Hkv, self.D,
                                  dtype=torch.bfloat16)
@@ -413,7 +460,8 @@ class DecodeWorkload:
 def bench_decode(sl, args, world, rank):
     name = args.workload
     c = synth.WORKLOADS[name]
-    wl = DecodeWorkload(sl, name, synth.WORKLOAD_SEED[name] + 7919 * rank)
+    wl = DecodeWorkload(sl, name, synth.WORKLOAD_SEED[name] + 7919 * rank, layers=args.layers)
+    c = wl.cfg
     fill = min(1000, c["T"] - args.steps - args.warmup)
     for _ in range(fill):  # reach the steady-state block sizes (untimed set-up)
         wl.eager_step()
@@ -443,15 +491,18 @@ def bench_decode(sl, args, world, rank):
     kv_bytes = rows * wl.Hkv * wl.D * 2 * 2  # K and V, bf16, every sequence, one layer
     r = wl.t % wl.RING
     reps = 20
-    # the decode kernel alone over the 32 layers of the current state, replayed
-    # as one CUDA graph (so host launch overhead is not timed)
+    # the dominant kernel as the timed step runs it: the fused decode step of
+    # layers 1..L-1 (append + flush copy + attention, no bookkeeping launch),
+    # replayed as one CUDA graph.  Without the layer-0 bookkeeping a replay
+    # repeats the same plan: it rewrites the same new-token row, or copies the
+    # same rows out of place again, so every replay does the step's work.
     gdec = torch.cuda.CUDAGraph()
     s_ = torch.cuda.Stream()
     s_.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s_):
         with torch.cuda.graph(gdec, stream=s_):
-            for l in range(wl.L):
-                wl.cache.decode(l, wl.q[r, l], out=wl.out[l], lse=wl.lse[l])
+            for l in range(1, wl.L):
+                wl.layer_ops(r, l)
     torch.cuda.current_stream().wait_stream(s_)
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     for _ in range(2):
@@ -462,8 +513,12 @@ def bench_decode(sl, args, world, rank):
         gdec.replay()
     d1.record()
     torch.cuda.synchronize()
-    dec_s = d0.elapsed_time(d1) / 1e3 / (reps * wl.L)
-    achieved = kv_bytes / dec_s / 1e9
+    dec_s = d0.elapsed_time(d1) / 1e3 / (reps * (wl.L - 1))
+    # algorithmic bytes of one launch: the retained K/V rows read, the new
+    # token's K/V row written, q read, out and lse written
+    alg_bytes = kv_bytes + wl.B * (wl.Hkv * wl.D * 2 * 2 + wl.Hq * wl.D * 2 * 2 + wl.Hq * 4)
+    achieved = alg_bytes / dec_s / 1e9
+    traffic = _traffic(name, units=rows)
     pk = _peaks()
     # e2e: the step with its per-step inputs copied from pinned host memory
     # (q, k_new, v_new of every layer and the flags) and the outputs read back
@@ -508,8 +563,10 @@ def bench_decode(sl, args, world, rank):
                    "l2": "working set (~1 GB of cache) far above L2",
                    "parallelism": "replica per GPU (weak)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
-                     "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": None,
-                     "kernel": "sep_attn_decode (32 layers in one CUDA graph, per-launch mean)",
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": traffic,
+                     "bytes_per_launch": int(alg_bytes), "launch_us": round(dec_s * 1e6, 3),
+                     "kernel": "sep_attn_decode_step, layers 1..%d in one CUDA graph (fused append "
+                               "+ flush copy + attention), per-launch mean" % (wl.L - 1),
                      "peak_source": pk["src"] + " HBM copy"},
         "e2e": e2e, "clocks": clk,
         "gpu_launches": (wl.L + 1) * K,
@@ -602,6 +659,9 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true", help="omit the cpu_baseline leg")
     ap.add_argument("--skip-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--layers", type=int, default=None,
+                    help="decode: fewer layers than the workload (a small case for profilers); "
+                         "the JSON line then names the count in config.layers")
     args = ap.parse_args()
     kind = synth.WORKLOADS[args.workload]["kind"]
     if args.steps is None:
