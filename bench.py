@@ -65,6 +65,12 @@ def _peaks():
 # (the capture ran a smaller cache than the bench; decode traffic grows in
 # proportion to the retained rows).
 TRAFFIC = {
+    "decode_llama3_8b_b16_l32_t65536_d128_bf16": dict(
+        bytes=(28613120 + 256) / (420.5 * 16), per="row", src=("decode.cu", "common.cuh"),
+        sha1="752d1f5715bf6a85c3f300167961d2a1744add15"),
+    "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
+        bytes=104798720 + 29326080, per="launch", src=("prefill_tc.cu", "common.cuh"),
+        sha1="33933b4438440541d25b84d21f8513b525cea57a"),
     "prefill_pythia160m_b8h12_s2048_d64_bf16": dict(
         bytes=82608128 + 9976576, per="launch", src=("prefill_tc.cu", "common.cuh"), sha1="33933b4438440541d25b84d21f8513b525cea57a"),
 }
