@@ -43,6 +43,7 @@ import synth  # noqa: E402
 DEFAULT_WORKLOAD = "prefill_pythia160m_b8h12_s2048_d64_bf16"
 PREFILL_METRIC = "Sep-Attn prefill TFLOP/s on kept pairs"
 DECODE_METRIC = "Sep-Attn decode tokens/s over the four-block SepCache"
+INGEST_METRIC = "SepCache prompt ingestion tokens/s"
 
 
 def _peaks():
@@ -616,7 +617,193 @@ def cpu_baseline_decode(wl, budget_s=10.0):
                           T0 + 1, wl.B, wl.Hq, T0, reps, wl.B, wl.L)}
 
 
+# ---------------------------------------------------------------- prompt ingestion
+
+
+def bench_ingest(sl, args, world, rank):
+    """Prompt ingestion: every step resets the cache and ingests a T-token
+    prompt at all layers (sepcache_ingest); value = prompt tokens of all
+    sequences per second.  Each layer has its own prompt K/V, so the
+    retained rows come from HBM, and L2 is flushed between steps."""
+    name = args.workload
+    c = dict(synth.WORKLOADS[name])
+    if args.layers:
+        c["layers"] = args.layers
+    seed = synth.WORKLOAD_SEED[name] + 7919 * rank
+    B, Hkv, D, L, T = c["B"], c["Hkv"], c["D"], c["layers"], c["T"]
+    cache = sl.SepCache(c["a"], c["s"], c["past"], c["w"], L, B, Hkv, D, dtype=torch.bfloat16)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    kp = torch.randn((L, B, Hkv, T, D), generator=g, device="cuda").bfloat16()
+    vp = torch.randn((L, B, Hkv, T, D), generator=g, device="cuda").bfloat16()
+    flags = synth.bernoulli_flags(synth.rng((seed, 31)), (B, T), c["p_sep"])
+    is_sep = torch.from_numpy(flags).cuda()
+    prefix, idx, _ = sl.build_index(is_sep)
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device="cuda")
+
+    def step():
+        cache.init()
+        for l in range(L):
+            cache.ingest(l, kp[l], vp[l], is_sep, prefix, idx)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    _barrier(world)
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()  # untimed: evict L2 between steps
+        ev[i][0].record()
+        step()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk = clocks.stop()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    t = _max_over_ranks(sum(ms) / 1e3, world)
+    value = B * T * K * world / t
+    rows = int(cache.counts.sum())
+    # algorithmic bytes of a step: every retained K/V row read from the prompt
+    # and written to the cache at every layer, plus the block metadata
+    row_bytes = Hkv * D * 2
+    alg = L * rows * row_bytes * 2 * 2 + B * (cache.cap * 5 + 16 + 8)
+    step_s = statistics.mean(ms) / 1e3
+    pk = _peaks()
+    achieved = alg / step_s / 1e9
+    return {
+        "metric": INGEST_METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(t / K * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": name, "B": B, "Hkv": Hkv, "D": D, "layers": L, "T": T,
+                   "a": c["a"], "s": c["s"], "past": c["past"], "w": c["w"],
+                   "retained_rows_per_sequence": round(rows / B, 2),
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)",
+                   "parallelism": "replica per GPU (weak)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": None,
+                     "bytes_per_launch": int(alg), "launch_us": round(step_s * 1e6, 3),
+                     "kernel": "sepcache_ingest over %d layers (state at layer 0, row copies at "
+                               "every layer)" % L,
+                     "peak_source": pk["src"] + " HBM copy"},
+        "e2e": None, "clocks": clk,
+        "gpu_launches": (L + 1) * K,  # layer 0: state + rows; other layers: rows
+    }
+
+
 # ---------------------------------------------------------------- reference arm
+
+
+def run_reference_decode(args, world, c, name):
+    """The oracle's decode on host cores.  Set-up (untimed): the state machine
+    over the first 1000 tokens.  A step: the state machine for one more token
+    of every sequence, then fp64 attention of every query head of 2 of the
+    sequences at one layer (the bounded sample); the step's time is scaled to
+    all sequences and layers."""
+    import oracle
+    seed = synth.WORKLOAD_SEED[name]
+    flags = synth.decode_flags(c, seed)
+    B, L = c["B"], c["layers"]
+    wl = dict(c, B=B)
+    T0 = 1000
+    nb = 2
+    state_t, attn_t, n_rows = 0.0, 0.0, 0
+
+    def one(t, timed):
+        nonlocal state_t, attn_t, n_rows
+        t0 = time.time()
+        sim = oracle.sepcache_simulate(flags[: t + 1], c["a"], c["s"], c["past"], c["w"], [t])
+        t1 = time.time()
+        q, _, _ = synth.decode_step_qkv(wl, seed, t, 0)
+        for b in range(nb):
+            n = int(sim["counts"][0, b].sum())
+            pos = sim["pos"][0, b, :n]
+            ks = torch.stack([synth.decode_step_qkv(wl, seed, int(p2), 0)[1][b] for p2 in pos[:1]], 1)
+            kk = ks.expand(c["Hkv"], n, c["D"]).contiguous()
+            oracle.attend(q[b], kk, kk)
+        t2 = time.time()
+        if timed:
+            # the simulation replays t+1 tokens; one token of the stream costs 1/(t+1) of it
+            state_t += (t1 - t0) / (t + 1)
+            attn_t += (t2 - t1) / nb
+            n_rows += n
+    for w in range(args.warmup):
+        one(T0 + w, False)
+    t0 = time.time()
+    for k in range(args.steps):
+        one(T0 + args.warmup + k, True)
+    wall = time.time() - t0
+    per_step = state_t / args.steps + L * B * attn_t / args.steps  # one token of all sequences
+    value = B / per_step
+    sample = ("state machine per token; fp64 attention of all %d query heads of %d of %d "
+              "sequences at 1 of %d layers per step over the retained row count (one K/V row "
+              "repeated: the cost depends on the count only), scaled to all" % (
+                  c["Hq"], nb, B, L))
+    return {"impl": "reference", "metric": DECODE_METRIC, "value": round(value, 3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(wall / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name, "B": B, "Hq": c["Hq"], "Hkv": c["Hkv"], "D": c["D"],
+                       "layers": L, "a": c["a"], "s": c["s"], "past": c["past"], "w": c["w"]},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def run_reference_ingest(args, world, c, name):
+    """The oracle's way to ingest a prompt: T sequential appends of the
+    four-block state machine for every sequence, then the retained rows'
+    K/V gathered from the prompt (numpy).  Bounded sample: one layer's rows
+    per step, scaled to all layers."""
+    import oracle
+    seed = synth.WORKLOAD_SEED[name]
+    B, Hkv, D, L, T = c["B"], c["Hkv"], c["D"], c["layers"], c["T"]
+    flags = synth.bernoulli_flags(synth.rng((seed, 31)), (B, T), c["p_sep"])
+    g = synth.rng((seed, 32))
+    kp = g.standard_normal((B, Hkv, T, D), dtype=np.float32)
+    vp = g.standard_normal((B, Hkv, T, D), dtype=np.float32)
+    st_t, cp_t = 0.0, 0.0
+
+    def one(timed):
+        nonlocal st_t, cp_t
+        t0 = time.time()
+        sim = oracle.sepcache_simulate(flags.T.copy(), c["a"], c["s"], c["past"], c["w"], [T - 1])
+        t1 = time.time()
+        for b in range(B):
+            n = int(sim["counts"][0, b].sum())
+            pos = sim["pos"][0, b, :n]
+            _ = kp[b][:, pos].copy(), vp[b][:, pos].copy()
+        t2 = time.time()
+        if timed:
+            st_t += t1 - t0
+            cp_t += t2 - t1
+    for _ in range(args.warmup):
+        one(False)
+    t0 = time.time()
+    for _ in range(args.steps):
+        one(True)
+    wall = time.time() - t0
+    per_step = (st_t + L * cp_t) / args.steps
+    value = B * T / per_step
+    sample = ("state machine over %d tokens x %d sequences and the retained rows of 1 of %d "
+              "layers per step, scaled to all layers" % (T, B, L))
+    return {"impl": "reference", "metric": INGEST_METRIC, "value": round(value, 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(wall / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": name, "B": B, "Hkv": Hkv, "D": D, "layers": L, "T": T,
+                       "a": c["a"], "s": c["s"], "past": c["past"], "w": c["w"]},
+            "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": 1,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
 
 
 def run_reference(args, world, rank):
@@ -625,11 +812,10 @@ def run_reference(args, world, rank):
     import oracle
     name = args.workload
     c = synth.WORKLOADS[name]
-    if c["kind"] != "prefill":
-        wl_cores = oracle.nthreads()
-        return {"impl": "reference", "metric": DECODE_METRIC,
-                "unavailable": "reference arm implemented for prefill workloads only",
-                "cores": wl_cores}
+    if c["kind"] == "decode":
+        return run_reference_decode(args, world, c, name)
+    if c["kind"] == "ingest":
+        return run_reference_ingest(args, world, c, name)
     inp = synth.prefill_inputs(c, synth.WORKLOAD_SEED[name])
     rows, frac = _sample_rows(c, budget_hint=4.0)
     kept = _kept_pairs_rows(inp["is_sep"], c, rows)
@@ -671,7 +857,7 @@ def main():
     args = ap.parse_args()
     kind = synth.WORKLOADS[args.workload]["kind"]
     if args.steps is None:
-        args.steps = 50 if kind == "prefill" else 2000
+        args.steps = {"prefill": 50, "ingest": 20}.get(kind, 2000)
     args.warmup = max(args.warmup, 3)
 
     if args.impl == "reference":
@@ -686,6 +872,8 @@ def main():
     import streaming_kv_cache_sep_b200 as sl
     if kind == "prefill":
         line = bench_prefill(sl, args, world, rank)
+    elif kind == "ingest":
+        line = bench_ingest(sl, args, world, rank)
     else:
         line = bench_decode(sl, args, world, rank)
     status = sl.device_status()

@@ -181,6 +181,22 @@ int sepcache_append(const sepcache* cache, int layer, const void* k_new, const v
  * without a flush. */
 int sepcache_compact(const sepcache* cache, int layer, void* stream);
 
+/* Prompt ingestion (bulk append): put the T tokens of a prompt into an EMPTY
+ * cache in one call per layer, with the same result as T calls of
+ * sepcache_append (and sepcache_compact) -- the prefill of the prompt then
+ * hands over to streaming decode (the study's prefill / decode split; the
+ * cache's block rules as in sepcache_append, xugj520 article section 3.3).
+ * k, v: the prompt's keys and values [B, Hkv, T, D] in the cache dtype (the
+ * layout sep_attn_prefill reads); is_sep [B, T], prefix [B, T+1] and idx
+ * [B, T] from sep_build_index of the prompt, read at layer 0, which also
+ * writes the block bookkeeping (step becomes T).  Layers 0..layers-1 in
+ * order.  A sequence whose cache is not empty is left unchanged and the
+ * cache status word gets SEP_CACHE_ESTATE.  Errors: SEP_EINVAL (T < 1, bad
+ * layer or cache), SEP_ENULL, SEP_EALIGN (k, v not 16-byte aligned). */
+int sepcache_ingest(const sepcache* cache, int layer, const void* k, const void* v,
+                    const uint8_t* is_sep, const int32_t* prefix, const int32_t* idx, int T,
+                    void* stream);
+
 /* One whole decode step of `layer` in a single launch per layer (plus, at
  * layer 0, the bookkeeping launch): the same result as sepcache_append(layer,
  * k_new, v_new, is_sep_new) -> sepcache_compact(layer) -> sep_attn_decode(

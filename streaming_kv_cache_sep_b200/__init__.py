@@ -26,7 +26,7 @@ ABI_SYMBOLS = (
     "sep_attn_prefill_workspace", "sep_attn_prefill", "sepcache_bytes", "sepcache_carve",
     "sepcache_init", "sepcache_append", "sepcache_compact", "sep_attn_decode_workspace",
     "sep_attn_decode", "sepcache_status", "sep_device_status", "sep_attn_decode_noalloc",
-    "sep_attn_decode_step",
+    "sep_attn_decode_step", "sepcache_ingest",
 )
 
 
@@ -73,6 +73,7 @@ def _load():
     L.sepcache_init.argtypes = [ctypes.POINTER(_SepCacheC), P]
     L.sepcache_append.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, P, P, P]
     L.sepcache_compact.argtypes = [ctypes.POINTER(_SepCacheC), i32, P]
+    L.sepcache_ingest.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, P, P, P, P, i32, P]
     L.sep_attn_decode_workspace.argtypes = [ctypes.POINTER(_SepCacheC), i32]
     L.sep_attn_decode_workspace.restype = sz
     L.sep_attn_decode.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, i32, f32, P, P, P, sz, P]
@@ -275,6 +276,21 @@ class SepCache:
     def compact(self, layer: int, stream=None):
         _check("sepcache_compact", _lib.sepcache_compact(ctypes.byref(self.c), layer,
                                                          _stream(stream)))
+
+    def ingest(self, layer: int, k, v, is_sep=None, prefix=None, idx=None, stream=None):
+        """Put a prompt's T tokens into this (empty) cache at `layer`: k, v
+        [B, Hkv, T, D]; is_sep [B, T], prefix [B, T+1], idx [B, T] from
+        build_index (read at layer 0).  Same result as T appends."""
+        _need_cuda(k, v, is_sep, prefix, idx)
+        if k.dim() != 4 or k.shape != v.shape or k.shape[0] != self.B or k.shape[1] != self.Hkv \
+                or k.shape[3] != self.D:
+            raise ValueError("k, v must be [B, Hkv, T, D] matching the cache")
+        if not (k.is_contiguous() and v.is_contiguous()):
+            raise ValueError("k, v must be contiguous")
+        T = int(k.shape[2])
+        _check("sepcache_ingest", _lib.sepcache_ingest(
+            ctypes.byref(self.c), layer, _ptr(k), _ptr(v), _ptr(is_sep), _ptr(prefix), _ptr(idx), T,
+            _stream(stream)))
 
     def workspace(self, Hq: int):
         ws = self._ws.get(Hq)

@@ -203,6 +203,111 @@ __global__ void __launch_bounds__(256) k_cache_compact(uint8_t* __restrict__ kc,
   }
 }
 
+// Prompt ingestion into an empty cache: the state after T sequential
+// appends, in closed form.  With nI = min(a, T) initial tokens and nL =
+// min(w, T - nI) local ones, E = T - nI - nL tokens left the local window in
+// position order and entered the past window, which flushed after every
+// past + 1 of them: F = E / (past + 1) flushes took positions [nI, hi), hi =
+// nI + F (past + 1), and their separators fed the separator cache, which
+// keeps the newest s (the last s separators of [nI, hi) -- a slice of the
+// prompt's separator index list); the past window holds [hi, T - nL).  One
+// CTA per sequence writes the rows' positions and flags, the block sizes and
+// step = T.  A cache that is not empty is left unchanged (status bit).
+__global__ void k_cache_ingest_meta(int32_t* __restrict__ pos, uint8_t* __restrict__ flag,
+                                    int32_t* __restrict__ counts, int32_t* __restrict__ plan,
+                                    int64_t* __restrict__ step, int32_t* __restrict__ status,
+                                    int32_t* __restrict__ cur, const uint8_t* __restrict__ is_sep,
+                                    const int32_t* __restrict__ prefix,
+                                    const int32_t* __restrict__ idx, int T, int cap, int a, int s,
+                                    int past, int w) {
+  __shared__ int empty;
+  const int b = blockIdx.x;
+  int32_t* cnt = counts + 4 * b;
+  if (threadIdx.x == 0)
+    empty = step[b] == 0 && cnt[0] == 0 && cnt[1] == 0 && cnt[2] == 0 && cnt[3] == 0;
+  __syncthreads();
+  if (!empty) {
+    if (threadIdx.x == 0) atomicOr(status, SEP_CACHE_ESTATE);
+    return;
+  }
+  const uint8_t* f = is_sep + static_cast<int64_t>(b) * T;
+  const int32_t* pre = prefix + static_cast<int64_t>(b) * (T + 1);
+  const int32_t* ix = idx + static_cast<int64_t>(b) * T;
+  const int nI = a < T ? a : T;
+  const int rest = T - nI;
+  const int nL = w < rest ? w : rest;
+  const int E = rest - nL;
+  const int F = E / (past + 1);
+  const int hi = nI + F * (past + 1);
+  const int nP = E - F * (past + 1);
+  const int nsep = pre[hi] - pre[nI];
+  const int nS = s < nsep ? s : nsep;
+  const int len = nI + nS + nP + nL;
+  const int s0 = pre[hi] - nS;  // index-list entry of the oldest kept separator
+  const int l0 = T - nL;
+  int32_t* ps = pos + static_cast<int64_t>(b) * cap;
+  uint8_t* fl = flag + static_cast<int64_t>(b) * cap;
+  for (int r = threadIdx.x; r < cap; r += blockDim.x) {
+    int p = -1;
+    if (r < nI) p = r;
+    else if (r < nI + nS) p = ix[s0 + (r - nI)];
+    else if (r < nI + nS + nP) p = hi + (r - nI - nS);
+    else if (r < len) p = l0 + (r - nI - nS - nP);
+    uint8_t fv = 0;
+    if (p >= T || (p < 0 && r < len)) {
+      atomicOr(status, SEP_CACHE_ESTATE);
+      p = -1;
+    } else if (p >= 0) {
+      fv = f[p] ? 1 : 0;
+    }
+    ps[r] = p;
+    fl[r] = fv;
+  }
+  if (threadIdx.x == 0) {
+    cnt[0] = nI;
+    cnt[1] = nS;
+    cnt[2] = nP;
+    cnt[3] = nL;
+    step[b] = T;
+    cur[b] = 0;
+    int32_t* pl = plan + static_cast<int64_t>(b) * (cap + kPlanHdr);
+    pl[0] = 0;
+    pl[1] = -1;
+    pl[2] = len;
+    pl[3] = nI;
+    pl[4] = pl[5] = 0;
+    pl[6] = pl[7] = 0;
+  }
+}
+
+// One layer's K/V rows of an ingested prompt: row r of buffer 0 takes the
+// prompt's row at position pos[r] (k, v: [B][Hkv][T][D]).  Grid: (chunks,
+// kv head, b).  Skips a sequence whose ingestion did not happen (step != T).
+__global__ void __launch_bounds__(256) k_cache_ingest_rows(
+    uint8_t* __restrict__ kc, uint8_t* __restrict__ vc, const uint8_t* __restrict__ k,
+    const uint8_t* __restrict__ v, const int32_t* __restrict__ pos,
+    const int32_t* __restrict__ counts, const int64_t* __restrict__ step, int T, int layer,
+    int layers, int B, int Hkv, int cap, int row_bytes) {
+  const int g = blockIdx.y, b = blockIdx.z;
+  if (step[b] != T) return;
+  const int32_t* cnt = counts + 4 * b;
+  const int len = cnt[0] + cnt[1] + cnt[2] + cnt[3];
+  if (len < 0 || len > cap) return;
+  const int ch = row_bytes / 16;
+  const int64_t dbase = row0(0, layer, b, g, layers, B, Hkv, cap, row_bytes);
+  const int64_t sbase = (static_cast<int64_t>(b) * Hkv + g) * T * row_bytes;
+  const int32_t* ps = pos + static_cast<int64_t>(b) * cap;
+  const int total = 2 * len * ch;
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
+    const int which = e / (len * ch);
+    const int r = (e / ch) % len, c = e % ch;
+    const int p = ps[r];
+    if (p < 0 || p >= T) continue;
+    const uint4 val = reinterpret_cast<const uint4*>((which ? v : k) + sbase + static_cast<int64_t>(p) * row_bytes)[c];
+    reinterpret_cast<uint4*>((which ? vc : kc) + dbase + static_cast<int64_t>(r) * row_bytes)[c] = val;
+  }
+}
+
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct Sizes {
@@ -341,6 +446,30 @@ extern "C" int sepcache_compact(const sepcache* c, int layer, void* stream) {
   dim3 grid(2, c->Hkv, c->B);
   k_cache_compact<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), c->plan, layer, c->layers, c->B,
+      c->Hkv, c->cap, row_bytes);
+  return sep::launch_status();
+}
+
+extern "C" int sepcache_ingest(const sepcache* c, int layer, const void* k, const void* v,
+                               const uint8_t* is_sep, const int32_t* prefix, const int32_t* idx,
+                               int T, void* stream) {
+  if (!cache_ok(c)) return c ? SEP_EINVAL : SEP_ENULL;
+  if (layer < 0 || layer >= c->layers || T < 1) return SEP_EINVAL;
+  if (!k || !v || (layer == 0 && (!is_sep || !prefix || !idx))) return SEP_ENULL;
+  if (!sep::aligned16(k) || !sep::aligned16(v)) return SEP_EALIGN;
+  if (static_cast<int64_t>(c->B) * c->Hkv * T >= (1ll << 31)) return SEP_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (layer == 0) {
+    k_cache_ingest_meta<<<c->B, 256, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step,
+                                               c->status, c->cur, is_sep, prefix, idx, T, c->cap,
+                                               c->cfg.a, c->cfg.s, c->cfg.past, c->cfg.w);
+    if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  }
+  const int row_bytes = c->D * sep::elem_bytes(c->dtype);
+  dim3 grid(4, c->Hkv, c->B);
+  k_cache_ingest_rows<<<grid, 256, 0, st>>>(
+      static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), static_cast<const uint8_t*>(k),
+      static_cast<const uint8_t*>(v), c->pos, c->counts, c->step, T, layer, c->layers, c->B,
       c->Hkv, c->cap, row_bytes);
   return sep::launch_status();
 }

@@ -49,6 +49,11 @@ WORKLOADS = {
     "prefill_long_b1_s131072_d128_bf16": dict(
         kind="prefill", B=1, Hq=32, Hkv=8, S=131072, D=128, dtype="bf16", a=4, n=1024,
         p_single=0.05, p_run_start=0.05 / 3.0, run_len=3, ids=None, qkv_std=1.0),
+    # Prompt ingestion into the decode workload's cache: a 4096-token prompt
+    # of 16 sequences, 8 kv heads, D128, 32 layers, a=4 s=64 past=128 w=256
+    "ingest_llama3_8b_b16_l32_t4096_d128_bf16": dict(
+        kind="ingest", B=16, Hq=32, Hkv=8, D=128, dtype="bf16", layers=32, T=4096,
+        a=4, s=64, past=128, w=256, p_sep=0.1, qkv_std=1.0),
 }
 
 # Base seed per workload (1000 + index in the list above); parity tests add
