@@ -676,7 +676,7 @@ def bench_ingest(sl, args, world, rank):
     step_s = statistics.mean(ms) / 1e3
     pk = _peaks()
     achieved = alg / step_s / 1e9
-    return {
+    line = {
         "metric": INGEST_METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(t / K * 1e3, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -695,6 +695,10 @@ def bench_ingest(sl, args, world, rank):
         "e2e": None, "clocks": clk,
         "gpu_launches": (L + 1) * K,  # layer 0: state + rows; other layers: rows
     }
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        ref = run_reference_ingest(argparse.Namespace(steps=3, warmup=1), 1, c, name)
+        line["cpu_baseline"] = ref["cpu_baseline"]
+    return line
 
 
 # ---------------------------------------------------------------- reference arm

@@ -466,7 +466,10 @@ extern "C" int sepcache_ingest(const sepcache* c, int layer, const void* k, cons
     if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   }
   const int row_bytes = c->D * sep::elem_bytes(c->dtype);
-  dim3 grid(4, c->Hkv, c->B);
+  // one 16-byte chunk per thread for a full cache: the copy is a chain of
+  // dependent loads (row position, then data), so width hides its latency
+  const int chunks = 2 * c->cap * (row_bytes / 16);
+  dim3 grid((chunks + 255) / 256, c->Hkv, c->B);
   k_cache_ingest_rows<<<grid, 256, 0, st>>>(
       static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), static_cast<const uint8_t*>(k),
       static_cast<const uint8_t*>(v), c->pos, c->counts, c->step, T, layer, c->layers, c->B,
