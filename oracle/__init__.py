@@ -34,8 +34,10 @@ def _lib():
         L.oracle_attend.argtypes = [P, P, P, i32, i32, i32, i32, i32, dbl, P, P]
         L.oracle_sepcache_simulate.argtypes = [P, i32, i64, i32, i32, i32, i32, P, i32, i32,
                                                P, P, P, P]
+        L.oracle_rope.argtypes = [P, i32, i64, i32, P, dbl, P]
         for f in (L.oracle_flags_from_ids, L.oracle_build_index, L.oracle_count_pairs,
-                  L.oracle_prefill_rows, L.oracle_attend, L.oracle_sepcache_simulate):
+                  L.oracle_prefill_rows, L.oracle_attend, L.oracle_sepcache_simulate,
+                  L.oracle_rope):
             f.restype = ctypes.c_int
     return _LIB
 
@@ -55,7 +57,8 @@ def _ptr(a: np.ndarray):
 
 def _elems(x):
     """(contiguous numpy array of raw element bits, dtype code): fp32 -> 0,
-    bf16 bit patterns (uint16) -> 1.  Accepts numpy arrays or CPU tensors."""
+    bf16 bit patterns (uint16) -> 1, fp64 -> 2.  Accepts numpy arrays or CPU
+    tensors."""
     if hasattr(x, "numpy"):  # a torch tensor
         import torch
         x = x.detach().cpu().contiguous()
@@ -63,10 +66,14 @@ def _elems(x):
             return x.view(torch.int16).numpy().view(np.uint16), 1
         if x.dtype == torch.float32:
             return x.numpy(), 0
+        if x.dtype == torch.float64:
+            return x.numpy(), 2
         raise TypeError(x.dtype)
     x = np.ascontiguousarray(x)
     if x.dtype == np.float32:
         return x, 0
+    if x.dtype == np.float64:
+        return x, 2
     if x.dtype == np.uint16:
         return x, 1
     raise TypeError(x.dtype)
@@ -178,3 +185,37 @@ def sepcache_simulate(flags: np.ndarray, a: int, s: int, past: int, w: int, snap
     if rc != 0:
         raise ValueError("oracle_sepcache_simulate failed (%d)" % rc)
     return dict(pos=pos, flag=flg, counts=cnt, flushed=flushed)
+
+
+def rope(x, positions, theta: float) -> np.ndarray:
+    """Rotary position encoding of the rows of x [..., D] at `positions`
+    (one per row, broadcast over the leading dims), rotate-half pairing:
+    the pair (x_i, x_{i+D/2}) turns by pos * theta^(-2i/D).  fp64 out."""
+    xa, dt = _elems(x)
+    D = xa.shape[-1]
+    rows = xa.size // D
+    pos = np.ascontiguousarray(np.broadcast_to(np.asarray(positions, dtype=np.int64),
+                                               xa.shape[:-1]).reshape(-1))
+    out = np.zeros(xa.shape, dtype=np.float64)
+    rc = _lib().oracle_rope(_ptr(xa), dt, rows, D, _ptr(pos), float(theta), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_rope rejected its arguments")
+    return out
+
+
+def decode_shifted(q, k, v, theta: float, scale: float = 0.0):
+    """Decode over a cache whose keys are stored before the position is
+    encoded: the retained rows k/v [Hkv,L,D] (cache order) take the positions
+    0..L-1 they hold inside the cache, the query q [Hq,D] (the newest token,
+    the last row) takes L-1.  fp64 (out [Hq,D], lse [Hq])."""
+    ka, _ = _elems(k)
+    L = ka.shape[1]
+    kr = rope(k, np.arange(L, dtype=np.int64)[None, :], theta)
+    qr = rope(q, L - 1, theta)
+    va, dv = _elems(v)
+    return attend(qr, kr, va.astype(np.float64) if dv == 0 else _bf16_to_f64(va), scale)
+
+
+def _bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """Exact values of bf16 bit patterns (uint16)."""
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)

@@ -29,6 +29,16 @@
  * of the softmax denominator over the scaled scores; the past buffer is
  * flushed when it holds more than `past` rows, and all of it is flushed.
  *
+ *   - positional-encoding shifting for streaming: the keys kept in the cache
+ *     are stored before their position is encoded, and the rotary encoding
+ *     of a Llama model is applied at each step with the rows' positions
+ *     inside the cache ("HKUDS047: SepLLM ..." study, section on the three
+ *     versions: the streaming setting needs positional-encoding shifting;
+ *     section "Streaming-SepLLM": the Llama positional-encoding-shifting
+ *     module).  The rotary encoding itself is not spelled out on the pages;
+ *     the reading taken is the rotate-half form used by Llama models: for
+ *     i < D/2 the pair (x_i, x_{i+D/2}) turns by pos * theta^(-2i/D).
+ *
  * Arithmetic is fp64 throughout, from the exact input values (fp32 inputs
  * widen exactly; bf16 inputs are the top 16 bits of an fp32).  Threads only
  * split independent rows / sequences; each row's arithmetic is sequential.
@@ -39,9 +49,10 @@
 #include <stdlib.h>
 #include <string.h>
 
-/* element loaders: dtype 0 = fp32, 1 = bf16 (raw 16-bit patterns) */
+/* element loaders: dtype 0 = fp32, 1 = bf16 (raw 16-bit patterns), 2 = fp64 */
 static double elem(const void* base, int dtype, int64_t i) {
   if (dtype == 0) return (double)((const float*)base)[i];
+  if (dtype == 2) return ((const double*)base)[i];
   uint32_t u = ((uint32_t)((const uint16_t*)base)[i]) << 16;
   float f;
   memcpy(&f, &u, sizeof f);
@@ -400,4 +411,31 @@ int oracle_sepcache_simulate(const uint8_t* flags, int B, int64_t T, int a, int 
   free(bufp);
   free(buff);
   return rc;
+}
+
+/* ------------------------------------------------------------------ */
+/* rotary position encoding and the position-shifted decode            */
+/* ------------------------------------------------------------------ */
+
+/* Rotate each of the nrows rows of x [nrows, D] to the position pos[r]:
+ * for i < D/2, with phi = pos[r] * theta^(-2i/D),
+ *   out_i       = x_i cos(phi) - x_{i+D/2} sin(phi)
+ *   out_{i+D/2} = x_{i+D/2} cos(phi) + x_i sin(phi)
+ * i.e. the complex number x_i + j x_{i+D/2} times exp(j phi).  fp64 out. */
+int oracle_rope(const void* x, int dtype, int64_t nrows, int D, const int64_t* pos, double theta,
+                double* out) {
+  if (D < 2 || D % 2 != 0 || !(theta > 0.0)) return -1;
+  int half = D / 2;
+  for (int64_t r = 0; r < nrows; ++r) {
+    for (int i = 0; i < half; ++i) {
+      double inv_freq = pow(theta, -2.0 * (double)i / (double)D);
+      double phi = (double)pos[r] * inv_freq;
+      double c = cos(phi), sn = sin(phi);
+      double a = elem(x, dtype, r * D + i);
+      double b = elem(x, dtype, r * D + i + half);
+      out[r * D + i] = a * c - b * sn;
+      out[r * D + i + half] = b * c + a * sn;
+    }
+  }
+  return 0;
 }

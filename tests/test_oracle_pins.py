@@ -428,3 +428,100 @@ def test_attend_equals_prefill_row_on_same_set():
     o2, l2 = oracle.attend(np.ascontiguousarray(q[0, :, i]), kq, vq)
     np.testing.assert_array_equal(out, o2)
     np.testing.assert_array_equal(lse, l2)
+
+
+# ---------------------------------------------------------------------------
+# rotary position encoding and the position-shifted decode.  Streaming needs
+# positional-encoding shifting: keys are cached before the encoding and take
+# their position inside the cache at each step (HKUDS047 SepLLM study,
+# section on the three versions and section "Streaming-SepLLM").  The
+# encoding is read as the rotate-half rotary form of Llama models.
+
+def test_rope_direction_and_pairing():
+    # the pair (x_i, x_{i+D/2}) is the complex number x_i + j x_{i+D/2},
+    # turned counter-clockwise: e_0 at angle 1 -> (cos 1, 0, sin 1, 0), and
+    # e_2 (the partner of e_0) -> (-sin 1, 0, cos 1, 0)
+    c1, s1 = math.cos(1.0), math.sin(1.0)
+    x = np.eye(4)
+    out = oracle.rope(x, [1, 1, 1, 1], 10000.0)
+    np.testing.assert_allclose(out[0], [c1, 0, s1, 0], atol=1e-15)
+    np.testing.assert_allclose(out[2], [-s1, 0, c1, 0], atol=1e-15)
+    # D = 4, theta = 10^4: the second frequency is 10^4^(-1/2) = 0.01, so
+    # e_1 at position 100 also turns by 1 rad, into the pair (1, 3)
+    out = oracle.rope(x[1:2], [100], 10000.0)
+    np.testing.assert_allclose(out[0], [0, c1, 0, s1], atol=1e-13)
+    # position 0 is the identity
+    r = _rand((5, 64), 70)
+    np.testing.assert_array_equal(oracle.rope(r, 0, 500000.0), r.astype(np.float64))
+
+
+def test_rope_frequencies():
+    # D = 8, theta = 256: frequency i is 256^(-2i/8) = 4^(-i), so e_i at
+    # position 4^i turns by exactly 1 rad for every i < 4
+    c1, s1 = math.cos(1.0), math.sin(1.0)
+    for i in range(4):
+        x = np.zeros((1, 8))
+        x[0, i] = 1.0
+        out = oracle.rope(x, [4 ** i], 256.0)[0]
+        want = np.zeros(8)
+        want[i], want[i + 4] = c1, s1
+        np.testing.assert_allclose(out, want, atol=1e-13)
+
+
+def test_rope_is_a_rotation_group():
+    rng = np.random.default_rng(71)
+    x = rng.standard_normal((16, 128))
+    m = rng.integers(0, 5000, size=16)
+    n = rng.integers(0, 5000, size=16)
+    rm = oracle.rope(x, m, 500000.0)
+    # norms are kept, and turning by m then by n is turning by m + n
+    np.testing.assert_allclose(np.linalg.norm(rm, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(oracle.rope(rm, n, 500000.0), oracle.rope(x, m + n, 500000.0),
+                               atol=1e-10)
+    # turning back by -m restores x
+    np.testing.assert_allclose(oracle.rope(rm, -m, 500000.0), x, atol=1e-11)
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    rng = np.random.default_rng(72)
+    q = rng.standard_normal((1, 64))
+    k = rng.standard_normal((1, 64))
+    for m, n, t in [(10, 3, 7), (452, 0, 1000), (5, 5, 123456)]:
+        a = oracle.rope(q, m, 10000.0) @ oracle.rope(k, n, 10000.0).T
+        b = oracle.rope(q, m + t, 10000.0) @ oracle.rope(k, n + t, 10000.0).T
+        np.testing.assert_allclose(a, b, rtol=1e-9, atol=1e-10)
+
+
+@pytest.mark.parametrize("theta", [10000.0, 500000.0])
+def test_decode_shifted_is_attention_over_cache_positions(theta):
+    # keys at their cache slots 0..L-1, the query (the newest row) at L-1:
+    # torch fp64 attention over the encoded rows gives the same result
+    Hq, Hkv, L, D = 8, 2, 37, 64
+    q = _rand((Hq, D), 73)
+    k = _rand((Hkv, L, D), 74)
+    v = _rand((Hkv, L, D), 75)
+    out, lse = oracle.decode_shifted(q, k, v, theta)
+    qr = oracle.rope(q, L - 1, theta)
+    kr = oracle.rope(k, np.arange(L)[None, :], theta)
+    ref_o, ref_l = _torch_attention(qr[None, :, None, :], kr[None], v[None].astype(np.float64),
+                                    torch.ones(1, L, dtype=torch.bool), 1.0 / math.sqrt(D))
+    np.testing.assert_allclose(out, ref_o[0, :, 0], atol=1e-12)
+    np.testing.assert_allclose(lse, ref_l[0, :, 0], atol=1e-12)
+    # the same scores from the relative offsets alone: q unrotated, key j
+    # turned by j - (L-1)
+    G = Hq // Hkv
+    for h in (0, Hq - 1):
+        krel = oracle.rope(k[h // G], np.arange(L) - (L - 1), theta)
+        s = (krel @ q[h].astype(np.float64)) / math.sqrt(D)
+        np.testing.assert_allclose(lse[h], np.log(np.exp(s - s.max()).sum()) + s.max(), atol=1e-12)
+
+
+def test_decode_shifted_single_row_returns_its_value():
+    q = _rand((4, 128), 76)
+    k = _rand((1, 1, 128), 77)
+    v = _rand((1, 1, 128), 78)
+    out, lse = oracle.decode_shifted(q, k, v, 500000.0)
+    np.testing.assert_allclose(out, np.repeat(v[0].astype(np.float64), 4, axis=0), atol=1e-15)
+    # one row at slot 0 and the query at slot 0: no turn at all
+    np.testing.assert_allclose(lse, q.astype(np.float64) @ k[0, 0].astype(np.float64) / math.sqrt(128),
+                               atol=1e-12)
