@@ -416,6 +416,9 @@ class DecodeWorkload:
         self.B, self.Hq, self.Hkv, self.D, self.L = c["B"], c["Hq"], c["Hkv"], c["D"], c["layers"]
         self.cache = sl.SepCache(c["a"], c["s"], c["past"], c["w"], self.L, self.B, self.Hkv, self.D,
                                  dtype=torch.bfloat16)
+        self.rope_theta = c.get("rope_theta", 0.0)
+        if self.rope_theta:
+            self.cache.set_rope(self.rope_theta)  # keys cached un-encoded
         g = torch.Generator(device="cuda")
         g.manual_seed(seed)
         R = self.RING
@@ -565,6 +568,7 @@ def bench_decode(sl, args, world, rank):
         "data": "synthetic",
         "config": {"workload": name, "B": c["B"], "Hq": c["Hq"], "Hkv": c["Hkv"], "D": c["D"],
                    "layers": c["layers"], "a": c["a"], "s": c["s"], "past": c["past"], "w": c["w"],
+                   "rope_theta": c.get("rope_theta"),
                    "timed_tokens": [wl.t - K, wl.t] if e2e is None else None,
                    "mean_retained_rows": round(rows / wl.B, 2),
                    "l2": "working set (~1 GB of cache) far above L2",
@@ -605,7 +609,10 @@ def cpu_baseline_decode(wl, budget_s=10.0):
             n = int(sim["counts"][0, b].sum())
             kk = k[b].unsqueeze(1).expand(wl.Hkv, n, wl.D).contiguous()
             vv = v[b].unsqueeze(1).expand(wl.Hkv, n, wl.D).contiguous()
-            oracle.attend(q[b], kk, vv)
+            if wl.rope_theta:
+                oracle.decode_shifted(q[b], kk, vv, wl.rope_theta)
+            else:
+                oracle.attend(q[b], kk, vv)
         reps += 1
         if time.time() - t0 >= budget_s:
             break
@@ -730,7 +737,10 @@ def run_reference_decode(args, world, c, name):
             pos = sim["pos"][0, b, :n]
             ks = torch.stack([synth.decode_step_qkv(wl, seed, int(p2), 0)[1][b] for p2 in pos[:1]], 1)
             kk = ks.expand(c["Hkv"], n, c["D"]).contiguous()
-            oracle.attend(q[b], kk, kk)
+            if c.get("rope_theta"):
+                oracle.decode_shifted(q[b], kk, kk, c["rope_theta"])
+            else:
+                oracle.attend(q[b], kk, kk)
         t2 = time.time()
         if timed:
             # the simulation replays t+1 tokens; one token of the stream costs 1/(t+1) of it
@@ -754,7 +764,8 @@ def run_reference_decode(args, world, c, name):
             "ms_per_step": round(wall / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": name, "B": B, "Hq": c["Hq"], "Hkv": c["Hkv"], "D": c["D"],
-                       "layers": L, "a": c["a"], "s": c["s"], "past": c["past"], "w": c["w"]},
+                       "layers": L, "a": c["a"], "s": c["s"], "past": c["past"], "w": c["w"],
+                       "rope_theta": c.get("rope_theta")},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,

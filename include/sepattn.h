@@ -141,8 +141,11 @@ typedef struct {
   int64_t* step;     /* [B]       tokens appended so far */
   int32_t* status;   /* [1]       0, or SEP_CACHE_E* bits set by a kernel */
   int32_t* cur;      /* [B]       current K/V buffer (0 or 1) of each sequence */
+  float* rope;       /* [rope_rows][D/2][2] cos, sin of slot r at frequency i (fp32) */
   int32_t layers, B, Hkv, D, dtype, cap;
   sep_cache_cfg cfg;
+  float rope_theta;  /* 0: keys are stored encoded; > 0: see sepcache_set_rope */
+  int32_t rope_rows; /* max(cap, 65) */
 } sepcache;
 
 #define SEP_CACHE_EOVERFLOW 1 /* a step found more rows than the capacity */
@@ -157,6 +160,24 @@ size_t sepcache_bytes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int 
  * dtype in {SEP_F32, SEP_BF16}, layers, B, Hkv >= 1. */
 int sepcache_carve(sepcache* cache, void* buffer, size_t bytes, sep_cache_cfg cfg, int layers,
                    int B, int Hkv, int D, int dtype);
+
+/* Positional-encoding shifting for streaming (HKUDS047 study, section on
+ * the three versions: the streaming setting needs positional-encoding
+ * shifting; section "Streaming-SepLLM": the Llama positional-encoding-
+ * shifting module).  With theta > 0 the cache holds keys BEFORE their
+ * rotary encoding, and every decode call (sep_attn_decode, _noalloc, _step)
+ * encodes each retained key at its slot r inside the cache (0 .. len-1, the
+ * order I | S | P | L) and the query at len-1, the newest token's slot:
+ * for i < D/2 the pair (x_i, x_{i+D/2}) turns by r * theta^(-2i/D)
+ * (rotate-half form, as in Llama models; Llama-3 uses theta = 500000).  So
+ * positions never exceed the capacity however long the stream runs.  Keys
+ * passed to sepcache_append / _ingest / _decode_step and q passed to the
+ * decode calls must then be un-encoded; values are never encoded.  Fills the
+ * cache's cos / sin table (fp32, rounded from fp64) on `stream` and records
+ * theta in *cache.  theta = 0 switches the shifting off (keys stored already
+ * encoded, the default after sepcache_carve).  Errors: SEP_EINVAL for theta
+ * < 0, not finite, or in (0, 1]. */
+int sepcache_set_rope(sepcache* cache, float theta, void* stream);
 
 /* Reset to the empty state (no tokens; status 0). */
 int sepcache_init(const sepcache* cache, void* stream);

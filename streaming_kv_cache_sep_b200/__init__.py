@@ -26,7 +26,7 @@ ABI_SYMBOLS = (
     "sep_attn_prefill_workspace", "sep_attn_prefill", "sepcache_bytes", "sepcache_carve",
     "sepcache_init", "sepcache_append", "sepcache_compact", "sep_attn_decode_workspace",
     "sep_attn_decode", "sepcache_status", "sep_device_status", "sep_attn_decode_noalloc",
-    "sep_attn_decode_step", "sepcache_ingest",
+    "sep_attn_decode_step", "sepcache_ingest", "sepcache_set_rope",
 )
 
 
@@ -46,9 +46,10 @@ class _SepCacheC(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("pos", ctypes.c_void_p),
                 ("flag", ctypes.c_void_p), ("counts", ctypes.c_void_p), ("plan", ctypes.c_void_p),
                 ("step", ctypes.c_void_p), ("status", ctypes.c_void_p), ("cur", ctypes.c_void_p),
-                ("layers", ctypes.c_int32),
+                ("rope", ctypes.c_void_p), ("layers", ctypes.c_int32),
                 ("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32),
-                ("dtype", ctypes.c_int32), ("cap", ctypes.c_int32), ("cfg", SepCacheCfg)]
+                ("dtype", ctypes.c_int32), ("cap", ctypes.c_int32), ("cfg", SepCacheCfg),
+                ("rope_theta", ctypes.c_float), ("rope_rows", ctypes.c_int32)]
 
 
 def _load():
@@ -74,6 +75,7 @@ def _load():
     L.sepcache_append.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, P, P, P]
     L.sepcache_compact.argtypes = [ctypes.POINTER(_SepCacheC), i32, P]
     L.sepcache_ingest.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, P, P, P, P, i32, P]
+    L.sepcache_set_rope.argtypes = [ctypes.POINTER(_SepCacheC), f32, P]
     L.sep_attn_decode_workspace.argtypes = [ctypes.POINTER(_SepCacheC), i32]
     L.sep_attn_decode_workspace.restype = sz
     L.sep_attn_decode.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, i32, f32, P, P, P, sz, P]
@@ -266,6 +268,18 @@ class SepCache:
 
     def init(self, stream=None):
         _check("sepcache_init", _lib.sepcache_init(ctypes.byref(self.c), _stream(stream)))
+
+    def set_rope(self, theta: float, stream=None):
+        """Positional-encoding shifting: with theta > 0 the cache holds keys
+        before their rotary encoding and every decode encodes each retained
+        key at its slot in the cache and q at the newest slot; 0 switches it
+        off (keys stored encoded)."""
+        _check("sepcache_set_rope", _lib.sepcache_set_rope(ctypes.byref(self.c), float(theta),
+                                                           _stream(stream)))
+
+    @property
+    def rope_theta(self) -> float:
+        return float(self.c.rope_theta)
 
     def append(self, layer: int, k_new, v_new, is_sep_new=None, stream=None):
         _need_cuda(k_new, v_new, is_sep_new)

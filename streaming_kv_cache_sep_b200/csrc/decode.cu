@@ -75,6 +75,11 @@ struct DecodeParams {
   int layer, layers, B, Hq, Hkv, cap, nsplit;
   int early;  // fused step of layer >= 1: cache reads may precede the grid-dependency wait
   float scale_log2;
+  // positional-encoding shifting: keys are stored un-encoded and encoded at
+  // their slot in the cache, q at the newest slot len - 1; rope[r][i] =
+  // (cos, sin) of r * theta^(-2i/D), rope_rows >= max(cap, 65).  null: off
+  const float* rope;
+  int rope_rows;
 };
 
 // The last part of a split: its unnormalised partial (po, sm = max, sl = sum,
@@ -265,11 +270,26 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const Dec
   // this lane's query slices of the group's heads, pre-scaled (log2 domain)
   const T* qg = static_cast<const T*>(p.q) + (static_cast<int64_t>(b) * p.Hq + g * G) * D;
   float qv[G][DPL];
+  const int mq = len > 0 ? len - 1 : 0;  // the newest token's slot
 #pragma unroll
   for (int h = 0; h < G; ++h)
 #pragma unroll
     for (int i = 0; i < NI; ++i) {
       ld8(qg + h * D + 64 * i + 8 * c8, &qv[h][8 * i]);
+      if (p.rope) {
+        // encode at slot mq: dims d < D/2 pair with d + D/2
+        const int d0 = 64 * i + 8 * c8;
+        const bool lo = d0 < D / 2;
+        const int dp = lo ? d0 + D / 2 : d0 - D / 2;
+        float y[8];
+        ld8(qg + h * D + dp, y);
+        const float* cs = p.rope + static_cast<int64_t>(mq) * D + 2 * (lo ? d0 : dp);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = qv[h][8 * i + e];
+          qv[h][8 * i + e] = lo ? x * cs[2 * e] - y[e] * cs[2 * e + 1] : x * cs[2 * e] + y[e] * cs[2 * e + 1];
+        }
+      }
 #pragma unroll
       for (int e = 0; e < 8; ++e) qv[h][8 * i + e] *= p.scale_log2;
     }
@@ -317,6 +337,19 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const Dec
       }
       __syncthreads();
     }
+  }
+
+  if (p.rope) {
+    // encode the split's K rows in place at their slots r0 + r (the cache
+    // keeps them un-encoded)
+    for (int e = threadIdx.x; e < nrows * (D / 2); e += kThreads) {
+      const int r = e / (D / 2), i = e % (D / 2);
+      const float2 cs = reinterpret_cast<const float2*>(p.rope)[static_cast<int64_t>(r0 + r) * (D / 2) + i];
+      const float x = to_f(sk[r * D + i]), y = to_f(sk[r * D + i + D / 2]);
+      sk[r * D + i] = from_f<T>(x * cs.x - y * cs.y);
+      sk[r * D + i + D / 2] = from_f<T>(y * cs.x + x * cs.y);
+    }
+    __syncthreads();
   }
 
   // scores: warp w takes 4-row groups w, w+4, ...; lane (rr, c8) covers dims
@@ -487,13 +520,66 @@ __host__ __device__ constexpr int pipe_smem_bytes() {
   return pipe_stages<D, G>() * pipe_stage_bytes<D>() + 4 * G * D * 4 + 1024;  // + alignment slack
 }
 
+// packed fp32 pairs (one f32x2 instruction per pair)
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// Turn the bf16 pairs lo = (x_f, x_f+1) and hi = (x_{f+D/2}, x_{f+1+D/2})
+// by the angles with cosines c = (c_f, c_f+1) and sines s: x_f + j x_{f+D/2}
+// times exp(j phi), in fp32 (packed pairs).  The results go out as tf32
+// operands (l: dims f, f+1; h: dims f+D/2, f+1+D/2): the fp32 bit patterns
+// as they are, of which the tensor core reads the top 19 bits (sign, 8-bit
+// exponent, 10-bit fraction), so the encoded scores carry less than 2^-10
+// relative error per operand instead of bf16's 2^-9.
+__device__ __forceinline__ void rope_tf32(uint32_t lo, uint32_t hi, float2 c, float2 s,
+                                          uint32_t (&l)[2], uint32_t (&h)[2]) {
+  const float2 a = make_float2(__uint_as_float(lo << 16), __uint_as_float(lo & 0xffff0000u));
+  const float2 b = make_float2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u));
+  const float2 lv = fsub2(fmul2(a, c), fmul2(b, s));
+  const float2 hv = sep::ffma2(a, s, fmul2(b, c));
+  l[0] = __float_as_uint(lv.x);
+  l[1] = __float_as_uint(lv.y);
+  h[0] = __float_as_uint(hv.x);
+  h[1] = __float_as_uint(hv.y);
+}
+// (c, s) times (mc, ms) as complex numbers, two frequencies at once
+__device__ __forceinline__ void cturn(float2& c, float2& s, float2 mc, float2 ms) {
+  const float2 nc = fsub2(fmul2(c, mc), fmul2(s, ms));
+  s = sep::ffma2(c, ms, fmul2(s, mc));
+  c = nc;
+}
+// c (16x8 fp32) += a (16x8 tf32, row-major fragment) * b (8x8 tf32, col fragment)
+__device__ __forceinline__ void mma1688(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
 // Byte offset of (row r, element d) in one tensor's D/64 swizzled tiles.
 __device__ __forceinline__ uint32_t swz(int r, int d) {
   return static_cast<uint32_t>((d >> 6) * kTileBytes + r * 128 +
                                ((((d >> 3) & 7) ^ (r & 7)) << 4) + (d & 7) * 2);
 }
 
-template <int D, int G, bool FUSED>
+template <int D, int G, bool FUSED, bool ROPE>
 __global__ void __launch_bounds__(kPipeThreads, 2)
     k_decode_pipe(const DecodeParams p, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v) {
@@ -516,6 +602,8 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
       (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   float* const recv_o = reinterpret_cast<float*>(ring + kPipeStages * SB);  // [NCL][4][PART]
   __shared__ float rm[NCL][4][G], rl[NCL][4][G];  // every warp's running max (log2) and sum
+  // rotary turns by 8 and by 64 slots: cosines and sines per frequency
+  __shared__ __align__(16) float rope_c[2][ROPE ? D / 2 : 2], rope_s[2][ROPE ? D / 2 : 2];
   __shared__ __align__(8) uint64_t full[kPipeStages], empty[kPipeStages], mrg;
   __shared__ int abort_flag;
 
@@ -628,6 +716,31 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
     asm volatile("griddepcontrol.wait;" ::: "memory");  // before this warp's stores in the merge
   } else {
     // ---------------------------------------------------------- consumers
+    const int kr = 16 * warp;  // this warp's rows of each chunk
+    // Rotary table reads go before the grid-dependency wait: the table is
+    // written by a launch that lets no later kernel start before it ends.
+    // cq/ck: (cos, sin) pairs of the lane's dims f, f + 1 (index 2kk + h,
+    // f = 16kk + 8h + 2tq) at the query's slot and at the lane's first row.
+    float4 cq[ROPE ? DT : 1], ck[ROPE ? DT : 1];
+    if constexpr (ROPE) {
+      for (int e = threadIdx.x; e < D; e += 128) {
+        const int t = e / (D / 2), i = e % (D / 2);
+        const float2 cs = reinterpret_cast<const float2*>(p.rope)[(t ? 64 : 8) * (D / 2) + i];
+        rope_c[t][i] = cs.x;
+        rope_s[t][i] = cs.y;
+      }
+      const int mq = len > 0 ? len - 1 : 0;  // the query: the newest token's slot
+      int r1 = rs + kr + gq;
+      if (r1 > p.rope_rows - 1) r1 = p.rope_rows - 1;  // rows past len: never used
+#pragma unroll
+      for (int kk = 0; kk < DT / 2; ++kk)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int f = 16 * kk + 8 * h + 2 * tq;
+          cq[2 * kk + h] = *reinterpret_cast<const float4*>(p.rope + static_cast<int64_t>(mq) * D + 2 * f);
+          ck[2 * kk + h] = *reinterpret_cast<const float4*>(p.rope + static_cast<int64_t>(r1) * D + 2 * f);
+        }
+    }
     asm volatile("griddepcontrol.wait;" ::: "memory");  // q, k_new, v_new
     uint32_t qb[DT][2];  // Q^T as the B operand: dims x heads (heads >= G are zero)
     {
@@ -639,13 +752,54 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         qb[kk][1] = in ? *reinterpret_cast<const uint32_t*>(qg + gq * D + 16 * kk + 8 + 2 * tq) : 0u;
       }
     }
-    const int kr = 16 * warp;  // this warp's rows of each chunk
+    // Positional-encoding shifting.  The lane's fragments hold dims f =
+    // 16kk + 8h + 2tq + {0, 1} (kk < DT/2, h in {0, 1}: register h of the B
+    // operand, registers 2h and 2h + 1 (rows gq, gq + 8) of the A operand),
+    // and the partner dim f + D/2 sits in the same register of tile
+    // kk + DT/2, so the rotation needs no data exchange.  ec/es[2kk + h]:
+    // cos / sin at dims f, f + 1 of the lane's row rs + 64c + kr + gq of
+    // chunk c, advanced chunk to chunk by the turn of 64 slots; row gq + 8
+    // is one turn of 8 further.  The encoded scores use tf32 operands: a dot
+    // product may take its terms in any order shared by both operands, so a
+    // 16-dim tile is two k = 8 products, one over the lane's even dims
+    // (2tq, 2tq + 8) and one over its odd dims, read straight from the bf16
+    // fragments' registers.  qf[t][2h + e]: encoded q at dim 16t + 8h + 2tq + e.
+    float2 ec[ROPE ? DT : 1], es[ROPE ? DT : 1];
+    uint32_t qf[ROPE ? DT : 1][4];
+    if constexpr (ROPE) {
+      sep::named_bar_sync(1, 128);  // rope_c / rope_s are filled
+#pragma unroll
+      for (int kk = 0; kk < DT / 2; ++kk)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int i = 2 * kk + h;
+          uint32_t lq[2], hq[2];
+          rope_tf32(qb[kk][h], qb[kk + DT / 2][h], make_float2(cq[i].x, cq[i].z),
+                    make_float2(cq[i].y, cq[i].w), lq, hq);
+          qf[kk][2 * h] = lq[0];
+          qf[kk][2 * h + 1] = lq[1];
+          qf[kk + DT / 2][2 * h] = hq[0];
+          qf[kk + DT / 2][2 * h + 1] = hq[1];
+          ec[i] = make_float2(ck[i].x, ck[i].z);
+          es[i] = make_float2(ck[i].y, ck[i].w);
+        }
+    }
     for (int c = 0; c < nchunks; ++c) {
       const int st = c % kPipeStages;
       const int r0 = rs + c * ROWS;
       const int nr = re - r0 < ROWS ? re - r0 : ROWS;
       uint8_t* const kt = ring + st * SB;
       uint8_t* const vt = kt + NB * kTileBytes;
+      if constexpr (ROPE) {
+        if (c > 0) {
+#pragma unroll
+          for (int i = 0; i < DT; ++i) {
+            const int f = 16 * (i / 2) + 8 * (i & 1) + 2 * tq;
+            cturn(ec[i], es[i], *reinterpret_cast<const float2*>(&rope_c[1][f]),
+                  *reinterpret_cast<const float2*>(&rope_s[1][f]));
+          }
+        }
+      }
       if (!__all_sync(0xffffffffu, sep::mbar_wait(&full[st], (c / kPipeStages) & 1, &abort_flag, p.err)))
         break;
       if (kr < nr) {
@@ -683,8 +837,33 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
           ldsm_x4_t(vb + swz(kr + (lane & 7) + (lane >> 4) * 8, 16 * dt + ((lane >> 3) & 1) * 8), va[dt]);
         // S^T = K Q^T for the warp's 16 keys (rows) x 8 heads, four chains
         float sacc[4][4] = {};
+        if constexpr (ROPE) {
 #pragma unroll
-        for (int kk = 0; kk < DT; ++kk) mma16816(sacc[kk & 3], ka[kk], qb[kk][0], qb[kk][1]);
+          for (int kk = 0; kk < DT / 2; ++kk) {
+            // encoded K of tile kk (kl) and of its partner tile kk + DT/2
+            // (kh): [register of the bf16 fragment][even / odd dim]
+            uint32_t kl[4][2], kh[4][2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int f = 16 * kk + 8 * h + 2 * tq, i = 2 * kk + h;
+              rope_tf32(ka[kk][2 * h], ka[kk + DT / 2][2 * h], ec[i], es[i], kl[2 * h], kh[2 * h]);
+              float2 c8 = ec[i], s8 = es[i];
+              cturn(c8, s8, *reinterpret_cast<const float2*>(&rope_c[0][f]),
+                    *reinterpret_cast<const float2*>(&rope_s[0][f]));
+              rope_tf32(ka[kk][2 * h + 1], ka[kk + DT / 2][2 * h + 1], c8, s8, kl[2 * h + 1],
+                        kh[2 * h + 1]);
+            }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              mma1688(sacc[e], kl[0][e], kl[1][e], kl[2][e], kl[3][e], qf[kk][e], qf[kk][2 + e]);
+              mma1688(sacc[2 + e], kh[0][e], kh[1][e], kh[2][e], kh[3][e], qf[kk + DT / 2][e],
+                      qf[kk + DT / 2][2 + e]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < DT; ++kk) mma16816(sacc[kk & 3], ka[kk], qb[kk][0], qb[kk][1]);
+        }
         // x0/x1: key kr + gq, heads 2tq / 2tq + 1; x2/x3: key kr + gq + 8
         float x[4];
 #pragma unroll
@@ -851,8 +1030,9 @@ int launch_one(const DecodeParams& p, cudaStream_t st) {
     CUtensorMap mk, mv;
     if (!sep::make_rows_map(&mk, p.kc, rows, D, ROWS) || !sep::make_rows_map(&mv, p.vc, rows, D, ROWS))
       return SEP_ECUDA;
-    auto kern = k_decode_pipe<D, G, FUSED>;
-    if (!allow_smem(kern, smem, attr_set)) return SEP_ECUDA;
+    static bool attr_rope[64] = {false};
+    auto kern = p.rope ? k_decode_pipe<D, G, FUSED, true> : k_decode_pipe<D, G, FUSED, false>;
+    if (!allow_smem(kern, smem, p.rope ? attr_rope : attr_set)) return SEP_ECUDA;
     if (cudaLaunchKernelEx(&cfg, kern, p, mk, mv) != cudaSuccess) return SEP_ECUDA;
   } else {
     auto kern = k_decode<T, D, G, FUSED, CLUSTER>;
@@ -934,6 +1114,8 @@ extern "C" int sep_attn_decode(const sepcache* c, int layer, const void* q, int 
   p.nsplit = (c->cap + ROWS - 1) / ROWS;
   const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(c->D));
   p.scale_log2 = sc * 1.44269504088896340736f;
+  p.rope = c->rope_theta > 0.f ? c->rope : nullptr;
+  p.rope_rows = c->rope_rows;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (c->dtype == SEP_BF16)
     return c->D == 64 ? launch_g<__nv_bfloat16, 64>(p, G, st) : launch_g<__nv_bfloat16, 128>(p, G, st);
@@ -988,6 +1170,8 @@ extern "C" int sep_attn_decode_step(const sepcache* c, int layer, const void* q,
   p.early = layer > 0;  // the step's metadata was advanced in the layer-0 call
   const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(c->D));
   p.scale_log2 = sc * 1.44269504088896340736f;
+  p.rope = c->rope_theta > 0.f ? c->rope : nullptr;
+  p.rope_rows = c->rope_rows;
   if (c->dtype == SEP_BF16)
     return c->D == 64 ? launch_g<__nv_bfloat16, 64, true>(p, G, st)
                       : launch_g<__nv_bfloat16, 128, true>(p, G, st);
@@ -1074,6 +1258,8 @@ extern "C" int sep_attn_decode_noalloc(const sepcache* c, int layer, const void*
   p.nsplit = nsplit;
   const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(c->D));
   p.scale_log2 = sc * 1.44269504088896340736f;
+  p.rope = c->rope_theta > 0.f ? c->rope : nullptr;
+  p.rope_rows = c->rope_rows;
   if (c->dtype == SEP_BF16)
     return c->D == 64 ? launch_g<__nv_bfloat16, 64>(p, G, st) : launch_g<__nv_bfloat16, 128>(p, G, st);
   return c->D == 64 ? launch_g<float, 64>(p, G, st) : launch_g<float, 128>(p, G, st);

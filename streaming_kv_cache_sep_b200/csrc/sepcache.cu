@@ -311,9 +311,13 @@ __global__ void __launch_bounds__(256) k_cache_ingest_rows(
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct Sizes {
-  size_t k, v, pos, flag, counts, plan, step, status, cur;
-  size_t total() const { return k + v + pos + flag + counts + plan + step + status + cur; }
+  size_t k, v, pos, flag, counts, plan, step, status, cur, rope;
+  size_t total() const { return k + v + pos + flag + counts + plan + step + status + cur + rope; }
 };
+
+// rows of the rotary table: every slot, and at least 65 so that the decode
+// kernels can read the turns by 8 and by 64 slots
+int rope_rows_of(int64_t cap) { return static_cast<int>(cap > 65 ? cap : 65); }
 
 Sizes sizes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
   const int64_t cap = static_cast<int64_t>(cfg.a) + cfg.s + cfg.past + cfg.w + 1;
@@ -327,6 +331,7 @@ Sizes sizes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
   z.step = round256(static_cast<size_t>(B) * 8);
   z.status = 256;
   z.cur = round256(static_cast<size_t>(B) * 4);
+  z.rope = round256(static_cast<size_t>(rope_rows_of(cap)) * D * 4);
   return z;
 }
 
@@ -341,7 +346,7 @@ bool cfg_ok(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
 
 bool cache_ok(const sepcache* c) {
   return c && c->k && c->v && c->pos && c->flag && c->counts && c->plan && c->step && c->status &&
-         c->cur &&
+         c->cur && c->rope && c->rope_rows == rope_rows_of(c->cap) && c->rope_theta >= 0.f &&
          cfg_ok(c->cfg, c->layers, c->B, c->Hkv, c->D, c->dtype) &&
          c->cap == c->cfg.a + c->cfg.s + c->cfg.past + c->cfg.w + 1;
 }
@@ -383,6 +388,8 @@ extern "C" int sepcache_carve(sepcache* cache, void* buffer, size_t bytes, sep_c
   cache->status = reinterpret_cast<int32_t*>(p);
   p += z.status;
   cache->cur = reinterpret_cast<int32_t*>(p);
+  p += z.cur;
+  cache->rope = reinterpret_cast<float*>(p);
   cache->layers = layers;
   cache->B = B;
   cache->Hkv = Hkv;
@@ -390,7 +397,41 @@ extern "C" int sepcache_carve(sepcache* cache, void* buffer, size_t bytes, sep_c
   cache->dtype = dtype;
   cache->cap = cfg.a + cfg.s + cfg.past + cfg.w + 1;
   cache->cfg = cfg;
+  cache->rope_theta = 0.f;
+  cache->rope_rows = rope_rows_of(cache->cap);
   return SEP_OK;
+}
+
+namespace {
+// cos / sin of slot r at frequency i: phi = r * theta^(-2i/D), evaluated in
+// fp64 and rounded to fp32
+__global__ void k_rope_table(float* tab, int rows, int D, double theta) {
+  const int half = D / 2;
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= rows * half) return;
+  const int r = e / half, i = e % half;
+  const double phi = static_cast<double>(r) * pow(theta, -2.0 * i / D);
+  double sn, cs;
+  sincos(phi, &sn, &cs);
+  tab[2 * e] = static_cast<float>(cs);
+  tab[2 * e + 1] = static_cast<float>(sn);
+}
+}  // namespace
+
+extern "C" int sepcache_set_rope(sepcache* c, float theta, void* stream) {
+  if (!c) return SEP_ENULL;
+  if (!cache_ok(c)) return SEP_EINVAL;
+  if (!(theta >= 0.f) || !isfinite(theta) || (theta > 0.f && theta <= 1.f)) return SEP_EINVAL;
+  if (theta == 0.f) {
+    c->rope_theta = 0.f;
+    return SEP_OK;
+  }
+  const int n = c->rope_rows * (c->D / 2);
+  k_rope_table<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      c->rope, c->rope_rows, c->D, static_cast<double>(theta));
+  const int rc = sep::launch_status();
+  if (rc == SEP_OK) c->rope_theta = theta;
+  return rc;
 }
 
 extern "C" int sepcache_init(const sepcache* c, void* stream) {

@@ -54,6 +54,11 @@ WORKLOADS = {
     "ingest_llama3_8b_b16_l32_t4096_d128_bf16": dict(
         kind="ingest", B=16, Hq=32, Hkv=8, D=128, dtype="bf16", layers=32, T=4096,
         a=4, s=64, past=128, w=256, p_sep=0.1, qkv_std=1.0),
+    # The decode workload with positional-encoding shifting: keys cached
+    # un-encoded, rotary base 500000 (Llama-3), encoded at their cache slots
+    "decode_rope_llama3_8b_b16_l32_t65536_d128_bf16": dict(
+        kind="decode", B=16, Hq=32, Hkv=8, D=128, dtype="bf16", layers=32, T=65536,
+        a=4, s=64, past=128, w=256, p_sep=0.1, qkv_std=1.0, rope_theta=500000.0),
 }
 
 # Base seed per workload (1000 + index in the list above); parity tests add

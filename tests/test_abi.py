@@ -83,7 +83,8 @@ def test_cache_layout_and_validation(sl):
     nb = L.sepcache_bytes(cfg, 32, 16, 8, 128, 1)
     cap = 4 + 64 + 128 + 256 + 1
     kv = 32 * 16 * 8 * cap * 128 * 2
-    assert nb >= 4 * kv and nb < 4 * kv + 256 * 1024  # K and V, two buffers each
+    # K and V, two buffers each; the metadata and the rotary table are small
+    assert nb >= 4 * kv and nb < 4 * kv + 512 * 1024
     assert L.sepcache_bytes(sl.SepCacheCfg(4, 64, 128, 0), 1, 1, 1, 128, 1) == 0  # w >= 1
     assert L.sepcache_bytes(sl.SepCacheCfg(-1, 64, 128, 4), 1, 1, 1, 128, 1) == 0
     assert L.sepcache_bytes(cfg, 1, 1, 1, 96, 1) == 0
@@ -92,7 +93,22 @@ def test_cache_layout_and_validation(sl):
     assert L.sepcache_carve(ctypes.byref(c), base, nb, cfg, 32, 16, 8, 128, 1) == 0
     assert c.cap == cap and c.k == (1 << 20) and c.v - c.k >= 2 * kv
     assert all(getattr(c, f) % 256 == 0
-               for f in ("pos", "flag", "counts", "plan", "step", "status", "cur"))
+               for f in ("pos", "flag", "counts", "plan", "step", "status", "cur", "rope"))
+    # rotary table: max(cap, 65) rows of D/2 (cos, sin) pairs, at the end
+    assert c.rope_rows == cap and c.rope_theta == 0.0
+    assert c.rope + cap * 128 * 4 <= (1 << 20) + nb
+    # positional-encoding shifting: theta 0 (off) enqueues nothing; negative
+    # or (0, 1] is refused before anything is enqueued
+    assert L.sepcache_set_rope(ctypes.byref(c), 0.0, None) == 0 and c.rope_theta == 0.0
+    assert L.sepcache_set_rope(ctypes.byref(c), -5.0, None) == -1
+    assert L.sepcache_set_rope(ctypes.byref(c), 1.0, None) == -1
+    assert L.sepcache_set_rope(ctypes.byref(c), float("nan"), None) == -1
+    assert L.sepcache_set_rope(None, 10000.0, None) == -6
+    small = sl._SepCacheC()
+    cfg_s = sl.SepCacheCfg(1, 1, 1, 1)
+    assert L.sepcache_carve(ctypes.byref(small), base, L.sepcache_bytes(cfg_s, 1, 1, 1, 64, 1),
+                            cfg_s, 1, 1, 1, 64, 1) == 0
+    assert small.rope_rows == 65  # the turns by 8 and 64 slots are always in the table
     assert L.sepcache_carve(ctypes.byref(c), ctypes.c_void_p((1 << 20) + 16), nb, cfg, 32, 16, 8,
                             128, 1) == -3
     assert L.sepcache_carve(ctypes.byref(c), base, nb - 1, cfg, 32, 16, 8, 128, 1) == -1
