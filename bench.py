@@ -67,8 +67,11 @@ def _peaks():
 # proportion to the retained rows).
 TRAFFIC = {
     "decode_llama3_8b_b16_l32_t65536_d128_bf16": dict(
-        bytes=(28613120 + 256) / (420.5 * 16), per="row", src=("decode.cu", "common.cuh"),
-        sha1="752d1f5715bf6a85c3f300167961d2a1744add15"),
+        bytes=(28613632 + 0) / (420.5 * 16), per="row", src=("decode.cu", "common.cuh"),
+        sha1="1ff00ea8ff526fc5d2f3bebd8de2529b9ee09d05"),
+    "decode_rope_llama3_8b_b16_l32_t65536_d128_bf16": dict(
+        bytes=(28884992 + 0) / (421.19 * 16), per="row", src=("decode.cu", "common.cuh"),
+        sha1="1ff00ea8ff526fc5d2f3bebd8de2529b9ee09d05"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
         bytes=104798720 + 29326080, per="launch", src=("prefill_tc.cu", "common.cuh"),
         sha1="33933b4438440541d25b84d21f8513b525cea57a"),
