@@ -33,7 +33,7 @@ def _lib():
                                           dbl, P, i64, P, P, i32]
         L.oracle_attend.argtypes = [P, P, P, i32, i32, i32, i32, i32, dbl, P, P]
         L.oracle_sepcache_simulate.argtypes = [P, i32, i64, i32, i32, i32, i32, P, i32, i32,
-                                               P, P, P, P]
+                                               P, P, P, P, i32, P]
         L.oracle_rope.argtypes = [P, i32, i64, i32, P, dbl, P]
         for f in (L.oracle_flags_from_ids, L.oracle_build_index, L.oracle_count_pairs,
                   L.oracle_prefill_rows, L.oracle_attend, L.oracle_sepcache_simulate,
@@ -161,13 +161,19 @@ def attend(q, k, v, scale: float = 0.0):
     return out, lse
 
 
+NO_ACCUMULATION = 1   # a flush keeps only the flushed past window's separators
+UNBOUNDED_SEPS = 2    # separators are never evicted (overflow past s is flagged)
+TOTAL_TRIGGER = 4     # flush when the whole cache exceeds a+s+past+w
+
+
 def sepcache_simulate(flags: np.ndarray, a: int, s: int, past: int, w: int, snap_steps,
-                      cap: int | None = None, want_flushed: bool = False):
+                      cap: int | None = None, want_flushed: bool = False, mode: int = 0):
     """Run the four-block cache over flags [T,B].
 
     Returns dict(pos [nsnap,B,cap] int32 (-1 padded), flag [nsnap,B,cap] uint8,
-    counts [nsnap,B,4] int32 = (|I|,|S|,|P|,|L|), flushed [T,B] uint8 or None),
-    the cache being read after the token of each snap step."""
+    counts [nsnap,B,4] int32 = (|I|,|S|,|P|,|L|), flushed [T,B] uint8 or None,
+    overflowed [B] uint8), the cache being read after the token of each snap
+    step.  mode: a sum of NO_ACCUMULATION, UNBOUNDED_SEPS, TOTAL_TRIGGER."""
     f = np.ascontiguousarray(flags, dtype=np.uint8)
     T, B = f.shape
     snaps = np.ascontiguousarray(np.asarray(snap_steps, dtype=np.int64))
@@ -177,14 +183,15 @@ def sepcache_simulate(flags: np.ndarray, a: int, s: int, past: int, w: int, snap
     flg = np.zeros((snaps.size, B, cap), dtype=np.uint8)
     cnt = np.zeros((snaps.size, B, 4), dtype=np.int32)
     flushed = np.zeros((T, B), dtype=np.uint8) if want_flushed else None
+    overflowed = np.zeros((B,), dtype=np.uint8)
     rc = _lib().oracle_sepcache_simulate(
         _ptr(f), B, T, a, s, past, w, _ptr(snaps), snaps.size, cap, _ptr(pos), _ptr(flg),
-        _ptr(cnt), _ptr(flushed) if flushed is not None else None)
+        _ptr(cnt), _ptr(flushed) if flushed is not None else None, int(mode), _ptr(overflowed))
     if rc == -2:
         raise AssertionError("cache exceeded a+s+past+w")
     if rc != 0:
         raise ValueError("oracle_sepcache_simulate failed (%d)" % rc)
-    return dict(pos=pos, flag=flg, counts=cnt, flushed=flushed)
+    return dict(pos=pos, flag=flg, counts=cnt, flushed=flushed, overflowed=overflowed)
 
 
 def rope(x, positions, theta: float) -> np.ndarray:

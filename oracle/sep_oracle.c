@@ -321,12 +321,27 @@ static void blk_push(blk* x, int32_t p, uint8_t f) {
  * After the token at step snap_steps[k] the cache I|S|P|L is written to
  * snap_pos/snap_flag [nsnap,B,cap] (-1 / 0 padded) and the block sizes to
  * snap_counts [nsnap,B,4] = (|I|,|S|,|P|,|L|).  flushed [T,B] (optional)
- * marks the steps whose token triggered a flush.  snap_steps ascending. */
+ * marks the steps whose token triggered a flush.  snap_steps ascending.
+ *
+ * mode bits, the KV manager's switches and its compression condition
+ * ("HKUDS047: SepLLM ..." study, section "KV Cache Manager": the
+ * SEP_ACCUMULATION and USE_MAX_SEP_CACHE branches of the compression step,
+ * and compression when the sequence exceeds cache_size):
+ *   1  no accumulation: a flush keeps only the separators of the flushed
+ *      past window (the old separator cache is dropped), newest s of them;
+ *   2  no maximum on the separator cache: separators are never evicted; the
+ *      s rows are its capacity, and a flush that would need more sets
+ *      overflowed[b] and keeps the newest s;
+ *   4  total-length trigger: flush when |I|+|S|+|P|+|L| > a+s+past+w instead
+ *      of when |P| > past (the same once |S| = s).
+ * overflowed [B] (optional) receives the mode-2 overflow flag. */
 int oracle_sepcache_simulate(const uint8_t* flags, int B, int64_t T, int a, int s, int past, int w,
                              const int64_t* snap_steps, int nsnap, int cap, int32_t* snap_pos,
-                             uint8_t* snap_flag, int32_t* snap_counts, uint8_t* flushed) {
-  if (a < 0 || s < 0 || past < 0 || w < 1) return -1;
-  int capI = a + 1, capS = s + 1, capP = past + 2, capL = w + 2;
+                             uint8_t* snap_flag, int32_t* snap_counts, uint8_t* flushed, int mode,
+                             uint8_t* overflowed) {
+  if (a < 0 || s < 0 || past < 0 || w < 1 || (mode & ~7) != 0) return -1;
+  /* under the total-length trigger the past window holds up to past + s */
+  int capI = a + 1, capS = s + 1, capP = past + s + 2, capL = w + 2;
   int32_t* bufp = (int32_t*)malloc(sizeof(int32_t) * (size_t)(capI + capS + capP + capL) * 2);
   uint8_t* buff = (uint8_t*)malloc((size_t)(capI + capS + capP + capL) * 2);
   for (int k = 0; k < nsnap; ++k)
@@ -362,14 +377,17 @@ int oracle_sepcache_simulate(const uint8_t* flags, int B, int64_t T, int a, int 
           L.n--;
         }
       }
-      /* 2. flush the past window when it overflows */
-      if (P.n > past) {
+      /* 2. flush the past window when it overflows (or the whole cache,
+       *    under the total-length trigger) */
+      int over = (mode & 4) ? (I.n + Sb.n + P.n + L.n > a + s + past + w) : (P.n > past);
+      if (over) {
         int nc = 0;
-        for (int r = 0; r < Sb.n; ++r) {
-          cp[nc] = Sb.pos[r];
-          cf[nc] = Sb.flag[r];
-          nc++;
-        }
+        if (!(mode & 1))
+          for (int r = 0; r < Sb.n; ++r) {
+            cp[nc] = Sb.pos[r];
+            cf[nc] = Sb.flag[r];
+            nc++;
+          }
         for (int r = 0; r < P.n; ++r)
           if (P.flag[r]) {
             cp[nc] = P.pos[r];
@@ -377,6 +395,7 @@ int oracle_sepcache_simulate(const uint8_t* flags, int B, int64_t T, int a, int 
             nc++;
           }
         int keep = nc < s ? nc : s;
+        if ((mode & 2) && nc > s && overflowed) overflowed[b] = 1;
         Sb.n = 0;
         for (int r = nc - keep; r < nc; ++r) blk_push(&Sb, cp[r], cf[r]);
         P.n = 0;

@@ -299,9 +299,9 @@ def test_flags_from_ids():
 # ---------------------------------------------------------------- SepCache
 
 
-def _read_trace():
-    meta, steps = {}, []
-    with open(os.path.join(GOLD, "sepcache_trace_a1_s2_p2_w2.txt")) as fh:
+def _read_trace(name="sepcache_trace_a1_s2_p2_w2.txt"):
+    meta, steps = {"mode": 0}, []
+    with open(os.path.join(GOLD, name)) as fh:
         for line in fh:
             line = line.strip()
             if line.startswith("# a="):
@@ -321,12 +321,15 @@ def _read_trace():
     return meta, steps
 
 
-def test_sepcache_golden_trace():
-    meta, steps = _read_trace()
+@pytest.mark.parametrize("name", ["sepcache_trace_a1_s2_p2_w2.txt",
+                                  "sepcache_trace_a1_s2_p2_w2_noacc.txt",
+                                  "sepcache_trace_a1_s2_p2_w2_total.txt"])
+def test_sepcache_golden_trace(name):
+    meta, steps = _read_trace(name)
     T = len(steps)
     flags = np.array([[f] for (_, f, _, _) in steps], dtype=np.uint8)
     sim = oracle.sepcache_simulate(flags, meta["a"], meta["s"], meta["past"], meta["w"],
-                                   np.arange(T), want_flushed=True)
+                                   np.arange(T), want_flushed=True, mode=meta["mode"])
     for k, (t, f, blocks, flushed) in enumerate(steps):
         cnt = sim["counts"][k, 0]
         assert list(cnt) == [len(x) for x in blocks], t
@@ -525,3 +528,96 @@ def test_decode_shifted_single_row_returns_its_value():
     # one row at slot 0 and the query at slot 0: no turn at all
     np.testing.assert_allclose(lse, q.astype(np.float64) @ k[0, 0].astype(np.float64) / math.sqrt(128),
                                atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# cache variants.  The KV manager's compression step, read off the study's
+# pseudocode ("HKUDS047: SepLLM ..." study, section "KV Cache Manager") and
+# written here as a whole-cache recomputation per token -- a different
+# formulation from the oracle's block state machine: when the cache is over
+# its budget, initial = first a tokens, local = last w, past window = the
+# tokens between the separator block and the local window; new separators =
+# the flagged tokens of the past window; seps = old + new (accumulation) or
+# new; seps = last s of them (maximum on; with the maximum off, more than s
+# is the flagged overflow and the newest s stay).
+
+
+def _pseudocode_cache(flags, a, s, past, w, mode):
+    acc = not (mode & oracle.NO_ACCUMULATION)
+    use_max = not (mode & oracle.UNBOUNDED_SEPS)
+    total_trigger = bool(mode & oracle.TOTAL_TRIGGER)
+    init, seps, rest = [], [], []  # rest = past window + local window, in order
+    states, overflow = [], False
+    for t, f in enumerate(flags):
+        if len(init) < a:
+            init.append(t)
+        else:
+            rest.append(t)
+        n_past = max(0, len(rest) - w)
+        size = len(init) + len(seps) + len(rest)
+        over = size > a + s + past + w if total_trigger else n_past > past
+        if over:
+            past_window, local = rest[:n_past], rest[n_past:]
+            new = [p for p in past_window if flags[p]]
+            seps = (seps + new) if acc else new
+            if len(seps) > s:
+                overflow = overflow or not use_max
+                seps = seps[len(seps) - s:]
+            rest = local
+        n_past = max(0, len(rest) - w)
+        states.append((list(init), list(seps), rest[:n_past], rest[n_past:]))
+    return states, overflow
+
+
+@pytest.mark.parametrize("mode", range(8))
+@pytest.mark.parametrize("a,s,past,w", [(1, 2, 2, 2), (3, 5, 4, 6), (0, 3, 0, 2), (2, 1, 3, 1)])
+def test_sepcache_variants_match_pseudocode(mode, a, s, past, w):
+    T, B = 400, 3
+    rng = np.random.default_rng(1000 + 17 * mode + a + s + past + w)
+    flags = (rng.random((T, B)) < 0.3).astype(np.uint8)
+    sim = oracle.sepcache_simulate(flags, a, s, past, w, np.arange(T), mode=mode)
+    for b in range(B):
+        states, overflow = _pseudocode_cache(flags[:, b], a, s, past, w, mode)
+        for t in range(T):
+            I, S, P, L = states[t]
+            assert list(sim["counts"][t, b]) == [len(I), len(S), len(P), len(L)], (mode, b, t)
+            want = I + S + P + L
+            assert list(sim["pos"][t, b, : len(want)]) == want, (mode, b, t)
+        assert bool(sim["overflowed"][b]) == overflow, (mode, b)
+
+
+def test_sepcache_variant_special_cases():
+    T, B = 2000, 4
+    flags = (np.random.default_rng(91).random((T, B)) < 0.1).astype(np.uint8)
+    a, s, past, w = 4, 64, 128, 256
+    base = oracle.sepcache_simulate(flags, a, s, past, w, np.arange(T))
+    # with no maximum the cache is the default one until the first eviction,
+    # which is flagged
+    unb = oracle.sepcache_simulate(flags, a, s, past, w, np.arange(T), mode=oracle.UNBOUNDED_SEPS)
+    np.testing.assert_array_equal(unb["pos"], base["pos"])
+    big = oracle.sepcache_simulate(flags, a, 4096, past, w, [T - 1], mode=oracle.UNBOUNDED_SEPS)
+    assert not big["overflowed"].any()
+    n_flushed_seps = big["counts"][0, :, 1]
+    assert (unb["overflowed"] == (n_flushed_seps > s)).all()
+    # without accumulation every separator of the cache came from the last
+    # flushed past window, which spans past + 1 positions
+    noacc = oracle.sepcache_simulate(flags, a, s, past, w, np.arange(T), mode=oracle.NO_ACCUMULATION)
+    for t in range(T):
+        for b in range(B):
+            nI, nS, nP, nL = noacc["counts"][t, b]
+            S = noacc["pos"][t, b, nI:nI + nS]
+            if nS:
+                assert S[-1] - S[0] <= past and flags[S, b].all()
+    # the total-length trigger never lets the cache exceed a+s+past+w and
+    # flushes exactly when it would; once S is full it flushes like the
+    # past-window trigger
+    tot = oracle.sepcache_simulate(flags, a, s, past, w, np.arange(T), mode=oracle.TOTAL_TRIGGER,
+                                   want_flushed=True)
+    sizes = tot["counts"].sum(-1)
+    assert sizes.max() <= a + s + past + w
+    for t in range(1, T):
+        for b in range(B):
+            if tot["flushed"][t, b]:
+                assert sizes[t - 1, b] == a + s + past + w
+            if tot["counts"][t - 1, b, 1] == s and tot["flushed"][t, b]:
+                assert tot["counts"][t - 1, b, 2] == past
