@@ -44,6 +44,7 @@ DEFAULT_WORKLOAD = "prefill_pythia160m_b8h12_s2048_d64_bf16"
 PREFILL_METRIC = "Sep-Attn prefill TFLOP/s on kept pairs"
 DECODE_METRIC = "Sep-Attn decode tokens/s over the four-block SepCache"
 INGEST_METRIC = "SepCache prompt ingestion tokens/s"
+GENERATE_METRIC = "Sep-Attn mask-based generation tokens/s over full histories"
 
 
 def _peaks():
@@ -711,6 +712,161 @@ def bench_ingest(sl, args, world, rank):
     return line
 
 
+# ---------------------------------------------------------------- mask-based generation
+
+
+def _kept_rows_last(flags, T, a, n):
+    """Kept keys of query T-1 per sequence: window + initial + separators."""
+    lo = max(0, T - n)
+    a0 = min(a, lo)
+    return (T - lo) + a0 + flags[:, a0:lo].astype(np.int64).sum(1)
+
+
+def bench_generate(sl, args, world, rank):
+    """Mask-based generation: one token of all sequences through every layer,
+    each layer attending over its own full history of S tokens with the kept
+    set of the newest row (sep_attn_decode_masked per layer, one CUDA graph
+    per step).  value = tokens/s.  The kept rows of 32 layers (~2 GB) are far
+    larger than L2."""
+    name = args.workload
+    c = dict(synth.WORKLOADS[name])
+    if args.layers:
+        c["layers"] = args.layers
+    seed = synth.WORKLOAD_SEED[name] + 7919 * rank
+    B, Hq, Hkv, D, L, S = c["B"], c["Hq"], c["Hkv"], c["D"], c["layers"], c["S"]
+    a, n, T = c["a"], c["n"], S
+    g = torch.Generator(device="cuda")
+    g.manual_seed(seed)
+    k = torch.randn((L, B, Hkv, S, D), generator=g, device="cuda").bfloat16()
+    v = torch.randn((L, B, Hkv, S, D), generator=g, device="cuda").bfloat16()
+    q = torch.randn((L, B, Hq, D), generator=g, device="cuda").bfloat16()
+    flags = synth.bernoulli_flags(synth.rng((seed, 51)), (B, S), c["p_sep"])
+    is_sep = torch.from_numpy(flags).cuda()
+    prefix, idx, _ = sl.build_index(is_sep)
+    out = torch.empty((L, B, Hq, D), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((L, B, Hq), dtype=torch.float32, device="cuda")
+
+    def layer(l):
+        sl.decode_masked(q[l], k[l], v[l], prefix, idx, T, a, n, out=out[l], lse=lse[l])
+
+    gstep = torch.cuda.CUDAGraph()
+    s_ = torch.cuda.Stream()
+    s_.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s_):
+        for l in range(L):  # once eagerly, then captured
+            layer(l)
+        with torch.cuda.graph(gstep, stream=s_):
+            for l in range(L):
+                layer(l)
+    torch.cuda.current_stream().wait_stream(s_)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup):
+        gstep.replay()
+    torch.cuda.synchronize()
+    K = args.steps
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    _barrier(world)
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record()
+    for _ in range(K):
+        gstep.replay()
+    s1.record()
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk = clocks.stop()
+    local_s = s0.elapsed_time(s1) / 1e3
+    t = _max_over_ranks(local_s, world)
+    value = B * K * world / t
+    # the dominant kernel: one layer's launch, the mean over this rank's graph
+    per_launch = local_s / (K * L)
+    kept = _kept_rows_last(flags, T, a, n)
+    alg = int(kept.sum()) * Hkv * D * 2 * 2 + B * Hq * (D * 2 * 2 + 4)
+    achieved = alg / per_launch / 1e9
+    pk = _peaks()
+    e2e = None
+    if not args.skip_e2e:
+        hq = q.cpu().pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        hlse = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
+        Ke = min(K, 100)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(Ke):
+            q.copy_(hq, non_blocking=True)
+            gstep.replay()
+            hout.copy_(out, non_blocking=True)
+            hlse.copy_(lse, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        te = _max_over_ranks(e0.elapsed_time(e1) / 1e3, world)
+        e2e = {"value": round(B * Ke * world / te, 2), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(hq.numel() * 2),
+               "d2h_bytes_per_step": int(hout.numel() * 2 + hlse.numel() * 4)}
+    line = {
+        "metric": GENERATE_METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(t / K * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": name, "B": B, "Hq": Hq, "Hkv": Hkv, "D": D, "layers": L,
+                   "history": T, "a": a, "n": n,
+                   "mean_kept_rows": round(float(kept.mean()), 2),
+                   "l2": "kept rows of all layers (~2 GB) far above L2",
+                   "parallelism": "replica per GPU (weak)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4),
+                     "traffic": _traffic(name, units=1),
+                     "bytes_per_launch": alg, "launch_us": round(per_launch * 1e6, 3),
+                     "kernel": "sep_attn_decode_masked of one layer (gathered kept rows), "
+                               "per-launch mean over the step graph",
+                     "peak_source": pk["src"] + " HBM copy"},
+        "e2e": e2e, "clocks": clk,
+        "gpu_launches": L * K,
+    }
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        ref = run_reference_generate(argparse.Namespace(steps=2, warmup=1), 1, c, name)
+        line["cpu_baseline"] = ref["cpu_baseline"]
+    return line
+
+
+def run_reference_generate(args, world, c, name):
+    """The oracle's mask-based generation on host cores: fp64 attention of
+    every query head of one sequence over its kept set at one layer per step
+    (the bounded sample); the step's time is scaled to all sequences and
+    layers."""
+    import oracle
+    seed = synth.WORKLOAD_SEED[name]
+    B, Hq, Hkv, D, L, S = c["B"], c["Hq"], c["Hkv"], c["D"], c["layers"], c["S"]
+    g = synth.rng((seed, 52))
+    flags = synth.bernoulli_flags(synth.rng((seed, 51)), (1, S), c["p_sep"])
+    q = synth.normal(g, (1, Hq, D), 1.0, "bf16")
+    k = synth.normal(g, (1, Hkv, S, D), 1.0, "bf16")
+    v = synth.normal(g, (1, Hkv, S, D), 1.0, "bf16")
+    for _ in range(args.warmup):
+        oracle.decode_masked(q, k, v, flags, S, c["a"], c["n"])
+    t0 = time.time()
+    for _ in range(args.steps):
+        oracle.decode_masked(q, k, v, flags, S, c["a"], c["n"])
+    wall = time.time() - t0
+    per_seq_layer = wall / args.steps
+    per_step = per_seq_layer * B * L  # one token of every sequence through every layer
+    value = B / per_step
+    sample = ("fp64 attention of all %d query heads of 1 of %d sequences at 1 of %d layers per "
+              "step, scaled to all" % (Hq, B, L))
+    return {"impl": "reference", "metric": GENERATE_METRIC, "value": round(value, 3),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(wall / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name, "B": B, "Hq": Hq, "Hkv": Hkv, "D": D, "layers": L,
+                       "history": S, "a": c["a"], "n": c["n"]},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s",
+                             "cores": oracle.nthreads(), "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
 # ---------------------------------------------------------------- reference arm
 
 
@@ -834,6 +990,8 @@ def run_reference(args, world, rank):
         return run_reference_decode(args, world, c, name)
     if c["kind"] == "ingest":
         return run_reference_ingest(args, world, c, name)
+    if c["kind"] == "generate":
+        return run_reference_generate(args, world, c, name)
     inp = synth.prefill_inputs(c, synth.WORKLOAD_SEED[name])
     rows, frac = _sample_rows(c, budget_hint=4.0)
     kept = _kept_pairs_rows(inp["is_sep"], c, rows)
@@ -875,7 +1033,7 @@ def main():
     args = ap.parse_args()
     kind = synth.WORKLOADS[args.workload]["kind"]
     if args.steps is None:
-        args.steps = {"prefill": 50, "ingest": 20}.get(kind, 2000)
+        args.steps = {"prefill": 50, "ingest": 20, "generate": 200}.get(kind, 2000)
     args.warmup = max(args.warmup, 3)
 
     if args.impl == "reference":
@@ -892,6 +1050,8 @@ def main():
         line = bench_prefill(sl, args, world, rank)
     elif kind == "ingest":
         line = bench_ingest(sl, args, world, rank)
+    elif kind == "generate":
+        line = bench_generate(sl, args, world, rank)
     else:
         line = bench_decode(sl, args, world, rank)
     status = sl.device_status()

@@ -122,7 +122,25 @@ int sep_attn_prefill(const void* q, const void* k, const void* v, int dtype, con
  * 0 with past = 0 is the StreamingLLM special case). */
 typedef struct {
   int32_t a, s, past, w;
+  int32_t mode; /* 0, or a sum of the SEP_CACHE_* variant bits below */
 } sep_cache_cfg;
+
+/* Variants of the KV manager's compression step ("HKUDS047: SepLLM ..."
+ * study, section "KV Cache Manager": the SEP_ACCUMULATION and
+ * USE_MAX_SEP_CACHE switches, and compression once the sequence exceeds
+ * cache_size).  Mode 0 is the default: separators accumulate, the separator
+ * cache keeps its newest s, and the past window is flushed when it holds
+ * more than `past` tokens. */
+#define SEP_CACHE_NO_ACCUMULATION 1 /* a flush keeps only the flushed past window's
+                                       separators (newest s); the old ones are dropped */
+#define SEP_CACHE_UNBOUNDED_SEPS 2  /* separators are never evicted: s is the block's
+                                       capacity, and a flush that needs more sets
+                                       SEP_CACHE_ESEPS in the status word (the newest s
+                                       stay) */
+#define SEP_CACHE_TOTAL_TRIGGER 4   /* flush when the whole cache holds more than
+                                       a+s+past+w tokens (the past window may then hold
+                                       up to past+s); the same as the default once the
+                                       separator cache is full */
 
 /* Cache state.  Every pointer is device memory inside one caller-owned
  * buffer laid out by sepcache_carve().  Rows of each (layer, b, kv head)
@@ -150,13 +168,14 @@ typedef struct {
 
 #define SEP_CACHE_EOVERFLOW 1 /* a step found more rows than the capacity */
 #define SEP_CACHE_ESTATE 2    /* corrupt block counts */
+#define SEP_CACHE_ESEPS 4     /* SEP_CACHE_UNBOUNDED_SEPS: more separators than s rows */
 
 /* Bytes of the single buffer holding a cache (256-byte aligned pieces). */
 size_t sepcache_bytes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype);
 
 /* Fill *cache with pointers into `buffer` (device, >= sepcache_bytes(),
  * 256-byte aligned) and the sizes.  Host-only; enqueues nothing.
- * Validation: a >= 0, s >= 0, past >= 0, w >= 1, D in {64, 128},
+ * Validation: a >= 0, s >= 0, past >= 0, w >= 1, mode bits in 0..7, D in {64, 128},
  * dtype in {SEP_F32, SEP_BF16}, layers, B, Hkv >= 1. */
 int sepcache_carve(sepcache* cache, void* buffer, size_t bytes, sep_cache_cfg cfg, int layers,
                    int B, int Hkv, int D, int dtype);
@@ -260,6 +279,30 @@ int sep_attn_decode(const sepcache* cache, int layer, const void* q, int Hq, flo
  * the GPU (other streams, other threads) race on it. */
 int sep_attn_decode_noalloc(const sepcache* cache, int layer, const void* q, int Hq, float scale,
                             void* out, float* lse, void* stream);
+
+/* Mask-based generation: the decode of the generate mask ("HKUDS047:
+ * SepLLM ..." study, section "SepAttention": build_generate_mask applies the
+ * prefill mask's rule to a query of length 1), over a full KV history with
+ * no row evicted.  The newest token of each sequence, at position T - 1,
+ * attends over k, v [B, Hkv, S, D] (rows 0 .. T-1 hold the history) with
+ * the kept set of its row
+ *   { j <= T-1 : j < a  or  is_sep[j]  or  T-1-j < n },
+ * read as the initial rows [0, min(a, lo)), the separators in
+ * [min(a, lo), lo) taken from idx, and the window [lo, T), lo = max(0, T-n).
+ * q [B, Hq, D] and out [B, Hq, D] in dtype; lse [B, Hq] fp32 (may be NULL).
+ * prefix [B, S+1], idx [B, S]: sep_build_index of the flags [B, S] (flags at
+ * positions >= T are never used).  scale <= 0 means 1/sqrt(D).  Same query
+ * head grouping and limits as sep_attn_decode (Hq/Hkv in {1, 2, 4, 8}),
+ * D in {64, 128}, 1 <= T <= S, a >= 0, n >= 1.  bf16 runs on warp-level
+ * tensor cores with the rows gathered by 16-byte asynchronous copies (no
+ * workspace: may be NULL); fp32 runs the exact FMA kernel and needs
+ * sep_attn_decode_masked_workspace() bytes, zero-filled before first use,
+ * 16-byte aligned; calls sharing it must not overlap on the GPU. */
+size_t sep_attn_decode_masked_workspace(int B, int Hq, int Hkv, int S, int D);
+int sep_attn_decode_masked(const void* q, const void* k, const void* v, int dtype,
+                           const int32_t* prefix, const int32_t* idx, int B, int Hq, int Hkv,
+                           int S, int T, int D, int a, int n, float scale, void* out, float* lse,
+                           void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronise `stream`, copy the cache status word to *host_status (host)
  * and return SEP_EDEVICE if it is nonzero, SEP_OK otherwise. */

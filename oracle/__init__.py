@@ -226,3 +226,23 @@ def decode_shifted(q, k, v, theta: float, scale: float = 0.0):
 def _bf16_to_f64(bits: np.ndarray) -> np.ndarray:
     """Exact values of bf16 bit patterns (uint16)."""
     return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def decode_masked(q, k, v, is_sep, T: int, a: int, n: int, scale: float = 0.0):
+    """Mask-based generation: q [B,Hq,D] is the query of token T-1, which
+    attends over k/v [B,Hkv,S,D] with its row's kept set -- the prefill rule
+    for that one row (the generate mask applies the prefill mask's rule to a
+    query of length 1).  fp64 (out [B,Hq,D], lse [B,Hq])."""
+    qa, dq = _elems(q)
+    ka, _ = _elems(k)
+    va, _ = _elems(v)
+    B, Hq, D = qa.shape
+    S = ka.shape[2]
+    qfull = np.zeros((B, Hq, T, D), dtype=qa.dtype)
+    qfull[:, :, T - 1, :] = qa
+    kT = np.ascontiguousarray(ka[:, :, :T, :])
+    vT = np.ascontiguousarray(va[:, :, :T, :])
+    f = np.ascontiguousarray(np.asarray(is_sep, dtype=np.uint8)[:, :T])
+    rows = np.array([(b * Hq + h) * T + (T - 1) for b in range(B) for h in range(Hq)], dtype=np.int64)
+    out, lse = prefill_rows(qfull, kT, vT, f, a, n, rows, scale)
+    return out.reshape(B, Hq, D), lse.reshape(B, Hq)

@@ -27,6 +27,7 @@ ABI_SYMBOLS = (
     "sepcache_init", "sepcache_append", "sepcache_compact", "sep_attn_decode_workspace",
     "sep_attn_decode", "sepcache_status", "sep_device_status", "sep_attn_decode_noalloc",
     "sep_attn_decode_step", "sepcache_ingest", "sepcache_set_rope",
+    "sep_attn_decode_masked_workspace", "sep_attn_decode_masked",
 )
 
 
@@ -39,7 +40,14 @@ class SepError(RuntimeError):
 
 class SepCacheCfg(ctypes.Structure):
     _fields_ = [("a", ctypes.c_int32), ("s", ctypes.c_int32), ("past", ctypes.c_int32),
-                ("w", ctypes.c_int32)]
+                ("w", ctypes.c_int32), ("mode", ctypes.c_int32)]
+
+
+# variant bits of SepCacheCfg.mode (the KV manager's switches)
+NO_ACCUMULATION = 1   # a flush keeps only the flushed past window's separators
+UNBOUNDED_SEPS = 2    # separators are never evicted; more than s sets CACHE_ESEPS
+TOTAL_TRIGGER = 4     # flush when the whole cache exceeds a+s+past+w
+CACHE_EOVERFLOW, CACHE_ESTATE, CACHE_ESEPS = 1, 2, 4  # cache status bits
 
 
 class _SepCacheC(ctypes.Structure):
@@ -76,6 +84,10 @@ def _load():
     L.sepcache_compact.argtypes = [ctypes.POINTER(_SepCacheC), i32, P]
     L.sepcache_ingest.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, P, P, P, P, i32, P]
     L.sepcache_set_rope.argtypes = [ctypes.POINTER(_SepCacheC), f32, P]
+    L.sep_attn_decode_masked_workspace.argtypes = [i32, i32, i32, i32, i32]
+    L.sep_attn_decode_masked_workspace.restype = sz
+    L.sep_attn_decode_masked.argtypes = [P, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i32,
+                                         i32, f32, P, P, P, sz, P]
     L.sep_attn_decode_workspace.argtypes = [ctypes.POINTER(_SepCacheC), i32]
     L.sep_attn_decode_workspace.restype = sz
     L.sep_attn_decode.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, i32, f32, P, P, P, sz, P]
@@ -87,7 +99,7 @@ def _load():
     for name in ABI_SYMBOLS:
         fn = getattr(L, name)
         if name not in ("sep_strerror", "sep_attn_prefill_workspace", "sepcache_bytes",
-                        "sep_attn_decode_workspace"):
+                        "sep_attn_decode_workspace", "sep_attn_decode_masked_workspace"):
             fn.restype = ctypes.c_int
     return L
 
@@ -197,6 +209,39 @@ def prefill(q, k, v, is_sep, prefix, idx, a: int, n: int, scale: float = 0.0, ou
     return out, lse
 
 
+_masked_ws = {}
+
+
+def decode_masked(q, k, v, prefix, idx, T: int, a: int, n: int, scale: float = 0.0, out=None,
+                  lse=None, want_lse: bool = True, workspace=None, stream=None):
+    """Mask-based generation over a full history: q [B,Hq,D] (token T-1)
+    attends over k/v [B,Hkv,S,D] rows 0..T-1 with the Sep-Attention kept set
+    of its row; prefix/idx from build_index of the flags [B,S].
+    Returns (out [B,Hq,D], lse [B,Hq])."""
+    _need_cuda(q, k, v, prefix, idx, out, lse, workspace)
+    B, Hq, D = q.shape
+    Hkv, S = k.shape[1], k.shape[2]
+    dt = _dtype_code(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    wsb = 0
+    if dt == SEP_F32:
+        need = int(_lib.sep_attn_decode_masked_workspace(B, Hq, Hkv, S, D))
+        if workspace is None:
+            key = (q.device, B, Hq, Hkv, S, D)
+            workspace = _masked_ws.get(key)
+            if workspace is None:
+                workspace = torch.zeros((need,), dtype=torch.uint8, device=q.device)
+                _masked_ws[key] = workspace
+        wsb = workspace.numel()
+    _check("sep_attn_decode_masked", _lib.sep_attn_decode_masked(
+        _ptr(q), _ptr(k), _ptr(v), dt, _ptr(prefix), _ptr(idx), B, Hq, Hkv, S, int(T), D, a, n,
+        float(scale), _ptr(out), _ptr(lse), _ptr(workspace), wsb, _stream(stream)))
+    return out, lse
+
+
 def device_status(clear: bool = True, stream=None) -> int:
     """Synchronise and return the library's device error bits (0 = none)."""
     bits = ctypes.c_int32(0)
@@ -212,8 +257,8 @@ class SepCache:
     device buffer.  Sizes: a initial, s separator, past window, w local."""
 
     def __init__(self, a: int, s: int, past: int, w: int, layers: int, B: int, Hkv: int, D: int,
-                 dtype=torch.bfloat16, device="cuda", stream=None):
-        self.cfg = SepCacheCfg(a, s, past, w)
+                 dtype=torch.bfloat16, device="cuda", stream=None, mode: int = 0):
+        self.cfg = SepCacheCfg(a, s, past, w, mode)
         self.dt = SEP_BF16 if dtype == torch.bfloat16 else SEP_F32
         nbytes = int(_lib.sepcache_bytes(self.cfg, layers, B, Hkv, D, self.dt))
         if nbytes == 0:

@@ -19,6 +19,7 @@
 //     the previous kernel on the stream drains, and waits for it before its
 //     first global read.
 #include <cooperative_groups.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "internal.h"
@@ -80,7 +81,45 @@ struct DecodeParams {
   // (cos, sin) of r * theta^(-2i/D), rope_rows >= max(cap, 65).  null: off
   const float* rope;
   int rope_rows;
+  // mask-based generation over a full history (null prefix: the cache path).
+  // kc, vc: k, v [B][Hkv][S][D]; the query is token T - 1; its kept set is
+  // [0, min(a, lo)), the separators in [min(a, lo), lo) (idx[b][prefix[b][.]]),
+  // and the window [lo, T), lo = max(0, T - n)
+  const int32_t* prefix;  // [B][S + 1]
+  const int32_t* idx;     // [B][S]
+  int S, T, a, n;
 };
+
+// The kept rows of the generating token: count and the history row of the
+// i-th kept row (ascending positions).
+struct GenRows {
+  int lo, a0, pa, nsep, len;
+  const int32_t* ix;
+  __device__ __forceinline__ GenRows(const DecodeParams& p, int b) {
+    lo = p.T - p.n > 0 ? p.T - p.n : 0;
+    a0 = p.a < lo ? p.a : lo;
+    const int32_t* pre = p.prefix + static_cast<int64_t>(b) * (p.S + 1);
+    pa = pre[a0];
+    nsep = pre[lo] - pa;
+    len = a0 + nsep + (p.T - lo);
+    ix = p.idx + static_cast<int64_t>(b) * p.S;
+  }
+  __device__ __forceinline__ int row(int i) const {
+    return i < a0 ? i : (i < a0 + nsep ? ix[pa + i - a0] : lo + (i - a0 - nsep));
+  }
+};
+
+// 16-byte asynchronous copy global -> shared; src_bytes = 0 writes zeros
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// arrive on `bar` once this thread's earlier cp.async copies have landed
+// (the barrier's expected count includes this arrival)
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(sep::smem_u32(bar))
+               : "memory");
+}
 
 // The last part of a split: its unnormalised partial (po, sm = max, sl = sum,
 // in this CTA's shared memory, rows with no keys at -inf / 0) is merged with
@@ -236,12 +275,14 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const Dec
   // metadata: independent loads issued together
   const int32_t* cnt = p.counts + 4 * b;
   const int32_t* pl = p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr);
-  const int c0 = cnt[0], c1 = cnt[1], c2 = cnt[2], c3 = cnt[3];
-  const int buf = p.cur[b] & 1;  // current after this step's bookkeeping
+  const bool gen = p.prefix != nullptr;  // mask-based generation over k, v
+  const int c0 = gen ? 0 : cnt[0], c1 = gen ? 0 : cnt[1], c2 = gen ? 0 : cnt[2], c3 = gen ? 0 : cnt[3];
+  const int buf = gen ? 0 : p.cur[b] & 1;  // current after this step's bookkeeping
   const int flush = FUSED ? pl[0] : 0;
   const int slot = FUSED ? pl[1] : -1;
   const int sbuf = FUSED ? (pl[4] & 1) : buf;
   int len = c0 + c1 + c2 + c3;
+  if (gen) len = GenRows(p, b).len;
   if (len < 0 || len > p.cap) len = 0;
   const int r0 = split * ROWS;
   const int nrows = len - r0 < 0 ? 0 : (len - r0 < ROWS ? len - r0 : ROWS);
@@ -258,7 +299,20 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const Dec
     sep::mbar_fence_init();
   }
   __syncthreads();
-  const bool bulk = nrows > 0 && !flush;
+  const bool bulk = nrows > 0 && !flush && !gen;
+  if (gen && nrows > 0) {
+    // the split's kept rows, gathered from k, v [B][Hkv][S][D]
+    const GenRows gr(p, b);
+    const int64_t hbase = (static_cast<int64_t>(b) * p.Hkv + g) * p.S;
+    constexpr int CU = D * static_cast<int>(sizeof(T)) / 16;
+    for (int e = threadIdx.x; e < 2 * nrows * CU; e += kThreads) {
+      const int which = e / (nrows * CU), r = (e / CU) % nrows, c = e % CU;
+      const int64_t hr = hbase + gr.row(r0 + r);
+      reinterpret_cast<uint4*>((which ? sv : sk) + r * D)[c] =
+          reinterpret_cast<const uint4*>(static_cast<const T*>(which ? p.vc : p.kc) + hr * D)[c];
+    }
+    __syncthreads();
+  }
   if (threadIdx.x == 0 && bulk) {
     const uint32_t bytes = static_cast<uint32_t>(nrows * D * sizeof(T));
     sep::mbar_arrive_expect_tx(&bar, 2 * bytes);
@@ -579,7 +633,7 @@ __device__ __forceinline__ uint32_t swz(int r, int d) {
                                ((((d >> 3) & 7) ^ (r & 7)) << 4) + (d & 7) * 2);
 }
 
-template <int D, int G, bool FUSED, bool ROPE>
+template <int D, int G, bool FUSED, bool ROPE, bool GATHER>
 __global__ void __launch_bounds__(kPipeThreads, 2)
     k_decode_pipe(const DecodeParams p, const __grid_constant__ CUtensorMap map_k,
                   const __grid_constant__ CUtensorMap map_v) {
@@ -614,14 +668,16 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   if (threadIdx.x == 0) {
     abort_flag = 0;
     for (int st = 0; st < kPipeStages; ++st) {
-      sep::mbar_init(&full[st], 1);
+      sep::mbar_init(&full[st], GATHER ? 32 : 1);  // gathers: one arrival per producer lane
       sep::mbar_init(&empty[st], 4);
     }
     sep::mbar_init(&mrg, 1);
     sep::mbar_fence_init();
     sep::mbar_arrive_expect_tx(&mrg, kMergeBytes);  // completes once every partial is here
-    sep::tma_prefetch_desc(&map_k);
-    sep::tma_prefetch_desc(&map_v);
+    if constexpr (!GATHER) {
+      sep::tma_prefetch_desc(&map_k);
+      sep::tma_prefetch_desc(&map_v);
+    }
     // let the next grid on the stream launch now: its CTAs take SM slots as
     // soon as ours retire and start their copies while ours drain (its own
     // grid-dependency wait still orders it after this grid)
@@ -634,10 +690,16 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   // at least two launches back, so they are read before waiting on the
   // previous grid; q, k_new, v_new and every store still come after the wait.
   if (!p.early) asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int32_t* cnt = p.counts + 4 * b;
-  const int32_t* pl = p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr);
-  int len = cnt[0] + cnt[1] + cnt[2] + cnt[3];
-  const int buf = p.cur[b] & 1;
+  const int32_t* pl = FUSED ? p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr) : nullptr;
+  int len;
+  int buf = 0;
+  if constexpr (GATHER) {
+    len = GenRows(p, b).len;
+  } else {
+    const int32_t* cnt = p.counts + 4 * b;
+    len = cnt[0] + cnt[1] + cnt[2] + cnt[3];
+    buf = p.cur[b] & 1;
+  }
   const int flush = FUSED ? pl[0] : 0;
   const int slot = FUSED ? pl[1] : -1;
   const int sbuf = FUSED ? (pl[4] & 1) : buf;
@@ -647,7 +709,9 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   const int re = rs + per < len ? rs + per : len;
   const int nchunks = (re - rs + ROWS - 1) / ROWS;
   // first row of this (buffer, layer, b, kv head) in the [rows, D] view
+  // (gathers: first row of (b, kv head) in the [B * Hkv * S, D] view of k, v)
   auto row_of = [&](int bb) -> int64_t {
+    if constexpr (GATHER) return (static_cast<int64_t>(b) * p.Hkv + g) * p.S;
     return (((static_cast<int64_t>(bb) * p.layers + p.layer) * p.B + b) * p.Hkv + g) * p.cap;
   };
   const int64_t row0 = row_of(buf);
@@ -677,7 +741,28 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
       if (c >= kPipeStages &&
           !__all_sync(0xffffffffu, sep::mbar_wait(&empty[st], ((c / kPipeStages) - 1) & 1, &abort_flag, p.err)))
         break;
-      if (FUSED && flush) {
+      if constexpr (GATHER) {
+        // the chunk's kept rows by 16-byte copies: CH lanes per row (one
+        // 256- or 128-byte row segment per instruction group), rows past the
+        // chunk's end zero-filled; each lane then arrives on the stage's
+        // barrier once its copies have landed
+        const GenRows gr(p, b);
+        int hr[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) hr[u] = 32 * u + lane < nr ? gr.row(r0 + 32 * u + lane) : -1;
+        constexpr int RPI = 32 / CH;  // rows per warp instruction
+        const uint32_t kts = sep::smem_u32(kt), vts = sep::smem_u32(vt);
+#pragma unroll 4
+        for (int it = 0; it < ROWS / RPI; ++it) {
+          const int q = it * RPI + lane / CH, cc = lane % CH;
+          const int src = __shfl_sync(0xffffffffu, (it * RPI) >> 5 ? hr[1] : hr[0], q & 31);
+          const int64_t off = (row0 + (src < 0 ? 0 : src)) * D + 8 * cc;
+          const uint32_t nb = src < 0 ? 0u : 16u;
+          cp_async16(kts + swz(q, 8 * cc), kc + off, nb);
+          cp_async16(vts + swz(q, 8 * cc), vc + off, nb);
+        }
+        cp_async_arrive(&full[st]);
+      } else if (FUSED && flush) {
         // rows of the post-flush layout come from their source rows in the
         // old buffer (the new token from k_new/v_new); each is also stored
         // at its destination in the new buffer
@@ -1024,15 +1109,26 @@ int launch_one(const DecodeParams& p, cudaStream_t st) {
   cfg.numAttrs = na;
   static bool attr_set[64] = {false};
   if constexpr (TC) {
-    // the K and V arrays as [2 * layers * B * Hkv * cap, D] rows
-    const int64_t rows = 2LL * p.layers * p.B * p.Hkv * p.cap;
-    if (rows > 0x7fffffffLL) return SEP_ETOOBIG;
     CUtensorMap mk, mv;
-    if (!sep::make_rows_map(&mk, p.kc, rows, D, ROWS) || !sep::make_rows_map(&mv, p.vc, rows, D, ROWS))
-      return SEP_ECUDA;
-    static bool attr_rope[64] = {false};
-    auto kern = p.rope ? k_decode_pipe<D, G, FUSED, true> : k_decode_pipe<D, G, FUSED, false>;
-    if (!allow_smem(kern, smem, p.rope ? attr_rope : attr_set)) return SEP_ECUDA;
+    static bool attr_rope[64] = {false}, attr_gen[64] = {false};
+    auto kern = p.rope ? k_decode_pipe<D, G, FUSED, true, false> : k_decode_pipe<D, G, FUSED, false, false>;
+    bool* done = p.rope ? attr_rope : attr_set;
+    if constexpr (!FUSED) {
+      if (p.prefix) {  // rows gathered by index: the tensor maps stay unused
+        memset(&mk, 0, sizeof mk);
+        memset(&mv, 0, sizeof mv);
+        kern = k_decode_pipe<D, G, false, false, true>;
+        done = attr_gen;
+      }
+    }
+    if (!p.prefix) {
+      // the K and V arrays as [2 * layers * B * Hkv * cap, D] rows
+      const int64_t rows = 2LL * p.layers * p.B * p.Hkv * p.cap;
+      if (rows > 0x7fffffffLL) return SEP_ETOOBIG;
+      if (!sep::make_rows_map(&mk, p.kc, rows, D, ROWS) || !sep::make_rows_map(&mv, p.vc, rows, D, ROWS))
+        return SEP_ECUDA;
+    }
+    if (!allow_smem(kern, smem, done)) return SEP_ECUDA;
     if (cudaLaunchKernelEx(&cfg, kern, p, mk, mv) != cudaSuccess) return SEP_ECUDA;
   } else {
     auto kern = k_decode<T, D, G, FUSED, CLUSTER>;
@@ -1059,14 +1155,15 @@ bool cache_ok(const sepcache* c) { return sep::cache_valid(c); }
 struct WsLayout {
   size_t ml, o, ticket;
 };
-WsLayout ws_layout(const sepcache* c, int Hq) {
-  const size_t nsplit = (c->cap + ROWS - 1) / ROWS;
+WsLayout ws_layout_of(int B, int Hq, int Hkv, int rows, int D) {
+  const size_t nsplit = (rows + ROWS - 1) / ROWS;
   WsLayout w;
-  w.ml = (static_cast<size_t>(c->B) * Hq * nsplit * 2 * 4 + 255) / 256 * 256;
-  w.o = (static_cast<size_t>(c->B) * Hq * nsplit * c->D * 4 + 255) / 256 * 256;
-  w.ticket = (static_cast<size_t>(c->B) * c->Hkv * 4 + 255) / 256 * 256;
+  w.ml = (static_cast<size_t>(B) * Hq * nsplit * 2 * 4 + 255) / 256 * 256;
+  w.o = (static_cast<size_t>(B) * Hq * nsplit * D * 4 + 255) / 256 * 256;
+  w.ticket = (static_cast<size_t>(B) * Hkv * 4 + 255) / 256 * 256;
   return w;
 }
+WsLayout ws_layout(const sepcache* c, int Hq) { return ws_layout_of(c->B, Hq, c->Hkv, c->cap, c->D); }
 
 }  // namespace
 
@@ -1263,4 +1360,79 @@ extern "C" int sep_attn_decode_noalloc(const sepcache* c, int layer, const void*
   if (c->dtype == SEP_BF16)
     return c->D == 64 ? launch_g<__nv_bfloat16, 64>(p, G, st) : launch_g<__nv_bfloat16, 128>(p, G, st);
   return c->D == 64 ? launch_g<float, 64>(p, G, st) : launch_g<float, 128>(p, G, st);
+}
+
+// ---------------------------------------------------------------------------
+// Mask-based generation: the newest token attends over the full history with
+// the Sep-Attention kept set of its row (the study's generate mask: the
+// prefill mask's rule for a query of length 1), no rows evicted.
+namespace {
+bool gen_args_ok(int B, int Hq, int Hkv, int S, int T, int D, int a, int n, int dtype) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || B > 65535 || Hkv > 65535) return false;
+  const int G = Hq / Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return false;
+  if (S < 1 || T < 1 || T > S || a < 0 || n < 1) return false;
+  if (static_cast<int64_t>(B) * Hkv * S >= (1LL << 31)) return false;
+  (void)D;
+  (void)dtype;
+  return true;
+}
+}  // namespace
+
+extern "C" size_t sep_attn_decode_masked_workspace(int B, int Hq, int Hkv, int S, int D) {
+  if (!gen_args_ok(B, Hq, Hkv, S, S, D, 0, 1, SEP_BF16) || (D != 64 && D != 128)) return 0;
+  const WsLayout w = ws_layout_of(B, Hq, Hkv, S, D);
+  return w.ml + w.o + w.ticket;
+}
+
+extern "C" int sep_attn_decode_masked(const void* q, const void* k, const void* v, int dtype,
+                                      const int32_t* prefix, const int32_t* idx, int B, int Hq,
+                                      int Hkv, int S, int T, int D, int a, int n, float scale,
+                                      void* out, float* lse, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  if (dtype != SEP_F32 && dtype != SEP_BF16) return SEP_EDTYPE;
+  if (D != 64 && D != 128) return SEP_EDTYPE;
+  if (!gen_args_ok(B, Hq, Hkv, S, T, D, a, n, dtype)) return SEP_EINVAL;
+  if (!q || !k || !v || !prefix || !idx || !out) return SEP_ENULL;
+  if (!sep::aligned16(q) || !sep::aligned16(k) || !sep::aligned16(v) || !sep::aligned16(out))
+    return SEP_EALIGN;
+  const WsLayout w = ws_layout_of(B, Hq, Hkv, T, D);
+  if (dtype == SEP_F32) {  // the exact kernel merges splits through the workspace
+    if (!workspace) return SEP_ENULL;
+    if (!sep::aligned16(workspace)) return SEP_EALIGN;
+    if (workspace_bytes < w.ml + w.o + w.ticket) return SEP_EINVAL;
+  }
+  DecodeParams p = {};
+  p.q = q;
+  p.kc = k;
+  p.vc = v;
+  p.out = out;
+  p.lse = lse;
+  if (workspace) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.part_ml = reinterpret_cast<float*>(ws);
+    p.part_o = reinterpret_cast<float*>(ws + w.ml);
+    p.ticket = reinterpret_cast<int32_t*>(ws + w.ml + w.o);
+  }
+  p.err = sep::device_error_word();
+  p.layer = 0;
+  p.layers = 1;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.cap = T;  // at most T kept rows
+  p.nsplit = (T + ROWS - 1) / ROWS;
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(D));
+  p.scale_log2 = sc * 1.44269504088896340736f;
+  p.prefix = prefix;
+  p.idx = idx;
+  p.S = S;
+  p.T = T;
+  p.a = a;
+  p.n = n;
+  const int G = Hq / Hkv;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dtype == SEP_BF16)
+    return D == 64 ? launch_g<__nv_bfloat16, 64>(p, G, st) : launch_g<__nv_bfloat16, 128>(p, G, st);
+  return D == 64 ? launch_g<float, 64>(p, G, st) : launch_g<float, 128>(p, G, st);
 }

@@ -7,6 +7,10 @@
 //   P  past window: tokens that slid out of the local window; when it holds
 //      more than `past` tokens it is flushed -- its separators join S (which
 //      then keeps its newest s entries) and it empties;
+//      (variants, the KV manager's switches: without accumulation a flush
+//      keeps only P's separators; with an unbounded separator cache an
+//      eviction is an error; with the total-length trigger P is flushed when
+//      the whole cache holds more than a + s + past + w tokens)
 //   L  local window: the newest w tokens.
 // Rows of each (layer, b, kv head) are stored I | S | P | L in increasing
 // position order.  P and L are one contiguous run of recent positions, so a
@@ -44,7 +48,7 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
                                 int32_t* __restrict__ counts, int32_t* __restrict__ plan,
                                 int64_t* __restrict__ step, int32_t* __restrict__ status,
                                 int32_t* __restrict__ cur, const uint8_t* __restrict__ is_sep_new,
-                                int B, int cap, int a, int s, int past, int w) {
+                                int B, int cap, int a, int s, int past, int w, int mode) {
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
   if (b >= B) return;
@@ -57,8 +61,10 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
   const int cb = cur[b] & 1;
   const uint8_t f = is_sep_new[b] ? 1 : 0;
   int len = nI + nS + nP + nL;
-  const bool bad = nI < 0 || nS < 0 || nP < 0 || nL < 0 || nI > a || nS > s || nP > past ||
-                   nL > w || len > cap - 1 || (nI < a && len != nI);
+  const bool total_trigger = (mode & SEP_CACHE_TOTAL_TRIGGER) != 0;
+  const bool bad = nI < 0 || nS < 0 || nP < 0 || nL < 0 || nI > a || nS > s ||
+                   nP > (total_trigger ? past + s : past) || nL > w || len > cap - 1 ||
+                   (nI < a && len != nI);
   __syncwarp();
   if (bad) {
     if (lane == 0) {
@@ -88,17 +94,20 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
   }
   ++len;
   __syncwarp();
-  // 2. flush the past window when it overflows
-  const bool flush = nP > past;
+  // 2. flush the past window when it overflows (or, with the total-length
+  //    trigger, when the whole cache does)
+  const bool flush = total_trigger ? len > a + s + past + w : nP > past;
+  const bool accumulate = (mode & SEP_CACHE_NO_ACCUMULATION) == 0;
   int new_len = len;
   if (flush) {
     const int eS = nI + nS, eP = eS + nP;
-    int ncand = nS;
+    int ncand = accumulate ? nS : 0;
     for (int base = eS; base < eP; base += 32) {
       const int r = base + lane;
       ncand += __popc(__ballot_sync(0xffffffffu, r < eP && fl[r] != 0));
     }
     const int drop = ncand > s ? ncand - s : 0;
+    if (drop > 0 && (mode & SEP_CACHE_UNBOUNDED_SEPS) && lane == 0) atomicOr(status, SEP_CACHE_ESEPS);
     for (int r = lane; r < nI; r += 32) pl[kPlanHdr + r] = r;  // initial rows keep their place
     int rank = 0, dst = nI;
     for (int base = nI; base < len; base += 32) {
@@ -106,7 +115,7 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
       const bool valid = r < len;
       const int32_t my_pos = valid ? ps[r] : -1;
       const uint8_t my_flag = valid ? fl[r] : 0;
-      const bool is_cand = valid && r < eP && (r < eS || my_flag != 0);
+      const bool is_cand = valid && r < eP && (r < eS ? accumulate : my_flag != 0);
       const bool is_local = valid && r >= eP;
       const uint32_t candb = __ballot_sync(0xffffffffu, is_cand);
       const int my_rank = rank + __popc(candb & lanemask_lt());
@@ -213,14 +222,19 @@ __global__ void __launch_bounds__(256) k_cache_compact(uint8_t* __restrict__ kc,
 // prompt's separator index list); the past window holds [hi, T - nL).  One
 // CTA per sequence writes the rows' positions and flags, the block sizes and
 // step = T.  A cache that is not empty is left unchanged (status bit).
+// Variants: without accumulation the separator cache holds the newest s
+// separators of the last flushed block [hi - past - 1, hi) -- again the end
+// of the index list up to hi; with the total-length trigger a flush happens
+// when the past window exceeds past + s - |S|, so the block ends depend on
+// the separator counts and one thread walks them (one step per flush).
 __global__ void k_cache_ingest_meta(int32_t* __restrict__ pos, uint8_t* __restrict__ flag,
                                     int32_t* __restrict__ counts, int32_t* __restrict__ plan,
                                     int64_t* __restrict__ step, int32_t* __restrict__ status,
                                     int32_t* __restrict__ cur, const uint8_t* __restrict__ is_sep,
                                     const int32_t* __restrict__ prefix,
                                     const int32_t* __restrict__ idx, int T, int cap, int a, int s,
-                                    int past, int w) {
-  __shared__ int empty;
+                                    int past, int w, int mode) {
+  __shared__ int empty, sh_hi, sh_ns, sh_ovf;
   const int b = blockIdx.x;
   int32_t* cnt = counts + 4 * b;
   if (threadIdx.x == 0)
@@ -237,11 +251,43 @@ __global__ void k_cache_ingest_meta(int32_t* __restrict__ pos, uint8_t* __restri
   const int rest = T - nI;
   const int nL = w < rest ? w : rest;
   const int E = rest - nL;
-  const int F = E / (past + 1);
-  const int hi = nI + F * (past + 1);
-  const int nP = E - F * (past + 1);
-  const int nsep = pre[hi] - pre[nI];
-  const int nS = s < nsep ? s : nsep;
+  const bool accumulate = (mode & SEP_CACHE_NO_ACCUMULATION) == 0;
+  if (threadIdx.x == 0) {
+    int hi = nI, ns = 0, ovf = 0;
+    if (mode & SEP_CACHE_TOTAL_TRIGGER) {
+      // the k-th flush takes the past window once it holds past + s - |S| + 1
+      for (;;) {
+        const int blen = past + s - ns + 1;
+        if (hi + blen > nI + E) break;
+        const int cnt = pre[hi + blen] - pre[hi];
+        const int cand = (accumulate ? ns : 0) + cnt;
+        ovf |= cand > s;
+        ns = cand < s ? cand : s;
+        hi += blen;
+      }
+    } else {
+      const int F = E / (past + 1);
+      hi = nI + F * (past + 1);
+      if (F > 0) {
+        const int cand = accumulate ? pre[hi] - pre[nI] : pre[hi] - pre[hi - past - 1];
+        ns = cand < s ? cand : s;
+        if (accumulate) {
+          ovf = cand > s;
+        } else {
+          for (int k = 0; k < F && !ovf; ++k)
+            ovf = pre[nI + (k + 1) * (past + 1)] - pre[nI + k * (past + 1)] > s;
+        }
+      }
+    }
+    sh_hi = hi;
+    sh_ns = ns;
+    sh_ovf = ovf;
+  }
+  __syncthreads();
+  const int hi = sh_hi;
+  const int nS = sh_ns;
+  const int nP = E - (hi - nI);
+  if (sh_ovf && (mode & SEP_CACHE_UNBOUNDED_SEPS) && threadIdx.x == 0) atomicOr(status, SEP_CACHE_ESEPS);
   const int len = nI + nS + nP + nL;
   const int s0 = pre[hi] - nS;  // index-list entry of the oldest kept separator
   const int l0 = T - nL;
@@ -336,7 +382,7 @@ Sizes sizes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
 }
 
 bool cfg_ok(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
-  if (cfg.a < 0 || cfg.s < 0 || cfg.past < 0 || cfg.w < 1) return false;
+  if (cfg.a < 0 || cfg.s < 0 || cfg.past < 0 || cfg.w < 1 || (cfg.mode & ~7) != 0) return false;
   if (layers < 1 || B < 1 || Hkv < 1 || B > 65535) return false;
   if (dtype != SEP_F32 && dtype != SEP_BF16) return false;
   if (D != 64 && D != 128) return false;
@@ -452,7 +498,7 @@ namespace sep {
 int cache_advance(const sepcache* c, const uint8_t* is_sep_new, cudaStream_t st) {
   k_cache_advance<<<c->B, 32, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step, c->status,
                                         c->cur, is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
-                                        c->cfg.past, c->cfg.w);
+                                        c->cfg.past, c->cfg.w, c->cfg.mode);
   return launch_status();
 }
 bool cache_valid(const sepcache* c) { return cache_ok(c); }
@@ -468,7 +514,7 @@ extern "C" int sepcache_append(const sepcache* c, int layer, const void* k_new, 
   if (layer == 0) {
     k_cache_advance<<<c->B, 32, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step, c->status,
                                           c->cur, is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
-                                          c->cfg.past, c->cfg.w);
+                                          c->cfg.past, c->cfg.w, c->cfg.mode);
     if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   }
   const int row_bytes = c->D * sep::elem_bytes(c->dtype);
@@ -503,7 +549,7 @@ extern "C" int sepcache_ingest(const sepcache* c, int layer, const void* k, cons
   if (layer == 0) {
     k_cache_ingest_meta<<<c->B, 256, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step,
                                                c->status, c->cur, is_sep, prefix, idx, T, c->cap,
-                                               c->cfg.a, c->cfg.s, c->cfg.past, c->cfg.w);
+                                               c->cfg.a, c->cfg.s, c->cfg.past, c->cfg.w, c->cfg.mode);
     if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   }
   const int row_bytes = c->D * sep::elem_bytes(c->dtype);

@@ -59,6 +59,12 @@ WORKLOADS = {
     "decode_rope_llama3_8b_b16_l32_t65536_d128_bf16": dict(
         kind="decode", B=16, Hq=32, Hkv=8, D=128, dtype="bf16", layers=32, T=65536,
         a=4, s=64, past=128, w=256, p_sep=0.1, qkv_std=1.0, rope_theta=500000.0),
+    # Mask-based generation over full 8k-token histories (no eviction),
+    # Llama-3-8B shape: 16 sequences, 32 q / 8 kv heads, D128, 32 layers,
+    # a=4 n=256
+    "generate_masked_llama3_8b_b16_s8192_d128_bf16": dict(
+        kind="generate", B=16, Hq=32, Hkv=8, D=128, dtype="bf16", layers=32, S=8192,
+        a=4, n=256, p_sep=0.1, qkv_std=1.0),
 }
 
 # Base seed per workload (1000 + index in the list above); parity tests add

@@ -30,7 +30,8 @@ def sl():
 class Stream:
     """Drive a SepCache through the C ABI with ring-cycled synthetic inputs."""
 
-    def __init__(self, sl, a, s, past, w, B, Hkv, Hq, D, layers, dtype, seed, T, fused=False):
+    def __init__(self, sl, a, s, past, w, B, Hkv, Hq, D, layers, dtype, seed, T, fused=False,
+                 mode=0):
         self.fused = fused
         self.sl = sl
         self.cfg = dict(a=a, s=s, past=past, w=w)
@@ -48,7 +49,7 @@ class Stream:
         self.dv = [x.cuda() for x in self.ring_v]
         self.flags = synth.bernoulli_flags(synth.rng((seed, 10)), (T, B), 0.1)
         self.dflags = torch.from_numpy(self.flags).cuda()
-        self.cache = sl.SepCache(a, s, past, w, layers, B, Hkv, D, dtype=dtype)
+        self.cache = sl.SepCache(a, s, past, w, layers, B, Hkv, D, dtype=dtype, mode=mode)
         self.t = 0
 
     def step(self, decode_layers=()):

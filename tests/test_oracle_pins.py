@@ -621,3 +621,27 @@ def test_sepcache_variant_special_cases():
                 assert sizes[t - 1, b] == a + s + past + w
             if tot["counts"][t - 1, b, 1] == s and tot["flushed"][t, b]:
                 assert tot["counts"][t - 1, b, 2] == past
+
+
+def test_decode_masked_limits():
+    # the generate mask is the prefill rule for the last row: with n >= T it
+    # is dense attention of token T-1; with no separators, sinks + window
+    B, Hq, Hkv, S, D, T = 2, 4, 2, 40, 64, 33
+    q = _rand((B, Hq, D), 80)
+    k = _rand((B, Hkv, S, D), 81)
+    v = _rand((B, Hkv, S, D), 82)
+    flags = (np.random.default_rng(83).random((B, S)) < 0.3).astype(np.uint8)
+    out, lse = oracle.decode_masked(q, k, v, flags, T, 2, T)
+    qq = q[:, :, None, :]
+    mask = torch.ones(1, T, dtype=torch.bool)
+    ref_o, ref_l = _torch_attention(qq, k[:, :, :T], v[:, :, :T], mask, 1.0 / math.sqrt(D))
+    np.testing.assert_allclose(out, ref_o[:, :, 0], atol=1e-12)
+    np.testing.assert_allclose(lse, ref_l[:, :, 0], atol=1e-12)
+    a, n = 3, 5
+    out, lse = oracle.decode_masked(q, k, v, np.zeros_like(flags), T, a, n)
+    keep = torch.zeros(1, T, dtype=torch.bool)
+    keep[0, :a] = True
+    keep[0, T - n:] = True
+    ref_o, ref_l = _torch_attention(qq, k[:, :, :T], v[:, :, :T], keep, 1.0 / math.sqrt(D))
+    np.testing.assert_allclose(out, ref_o[:, :, 0], atol=1e-12)
+    np.testing.assert_allclose(lse, ref_l[:, :, 0], atol=1e-12)
