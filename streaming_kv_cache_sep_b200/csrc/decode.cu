@@ -732,6 +732,15 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
 
   if (warp == 4) {
     // ---------------------------------------------------------- producer
+    // gathers: the history rows of the lane's two rows of the next chunk,
+    // looked up one chunk ahead so the index loads overlap the copies
+    int hn[2] = {-1, -1};
+    if constexpr (GATHER) {
+      const GenRows gr(p, b);
+      const int nr0 = re - rs < ROWS ? re - rs : ROWS;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) hn[u] = 32 * u + lane < nr0 ? gr.row(rs + 32 * u + lane) : -1;
+    }
     for (int c = 0; c < nchunks; ++c) {
       const int st = c % kPipeStages;
       const int r0 = rs + c * ROWS;
@@ -747,9 +756,12 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         // chunk's end zero-filled; each lane then arrives on the stage's
         // barrier once its copies have landed
         const GenRows gr(p, b);
-        int hr[2];
+        const int hr[2] = {hn[0], hn[1]};
+        {
+          const int r1 = r0 + ROWS, nr1 = re - r1 < ROWS ? re - r1 : ROWS;
 #pragma unroll
-        for (int u = 0; u < 2; ++u) hr[u] = 32 * u + lane < nr ? gr.row(r0 + 32 * u + lane) : -1;
+          for (int u = 0; u < 2; ++u) hn[u] = 32 * u + lane < nr1 ? gr.row(r1 + 32 * u + lane) : -1;
+        }
         constexpr int RPI = 32 / CH;  // rows per warp instruction
         const uint32_t kts = sep::smem_u32(kt), vts = sep::smem_u32(vt);
 #pragma unroll 4
