@@ -35,9 +35,11 @@ def _lib():
         L.oracle_sepcache_simulate.argtypes = [P, i32, i64, i32, i32, i32, i32, P, i32, i32,
                                                P, P, P, P, i32, P]
         L.oracle_rope.argtypes = [P, i32, i64, i32, P, dbl, P]
+        L.oracle_prefill_backward.argtypes = [P, P, P, i32, P, i32, P, i32, i32, i32, i32, i32,
+                                              i32, i32, dbl, P, P, P, i32]
         for f in (L.oracle_flags_from_ids, L.oracle_build_index, L.oracle_count_pairs,
                   L.oracle_prefill_rows, L.oracle_attend, L.oracle_sepcache_simulate,
-                  L.oracle_rope):
+                  L.oracle_rope, L.oracle_prefill_backward):
             f.restype = ctypes.c_int
     return _LIB
 
@@ -246,3 +248,26 @@ def decode_masked(q, k, v, is_sep, T: int, a: int, n: int, scale: float = 0.0):
     rows = np.array([(b * Hq + h) * T + (T - 1) for b in range(B) for h in range(Hq)], dtype=np.int64)
     out, lse = prefill_rows(qfull, kT, vT, f, a, n, rows, scale)
     return out.reshape(B, Hq, D), lse.reshape(B, Hq)
+
+
+def prefill_backward(q, k, v, dout, is_sep, a: int, n: int, scale: float = 0.0,
+                     threads: int | None = None):
+    """Gradients (dq [B,Hq,S,D], dk, dv [B,Hkv,S,D], fp64) of
+    sum(out * dout) through Sep-Attention, out recomputed in fp64."""
+    qa, dq_ = _elems(q)
+    ka, dk_ = _elems(k)
+    va, dv_ = _elems(v)
+    oa, do_ = _elems(dout)
+    assert dq_ == dk_ == dv_
+    B, Hq, S, D = qa.shape
+    Hkv = ka.shape[1]
+    f = np.ascontiguousarray(is_sep, dtype=np.uint8)
+    gq = np.zeros((B, Hq, S, D), dtype=np.float64)
+    gk = np.zeros((B, Hkv, S, D), dtype=np.float64)
+    gv = np.zeros((B, Hkv, S, D), dtype=np.float64)
+    rc = _lib().oracle_prefill_backward(_ptr(qa), _ptr(ka), _ptr(va), dq_, _ptr(oa), do_, _ptr(f),
+                                        B, Hq, Hkv, S, D, a, n, float(scale), _ptr(gq), _ptr(gk),
+                                        _ptr(gv), threads or nthreads())
+    if rc != 0:
+        raise ValueError("oracle_prefill_backward rejected its arguments")
+    return gq, gk, gv

@@ -458,3 +458,106 @@ int oracle_rope(const void* x, int dtype, int64_t nrows, int D, const int64_t* p
   }
   return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* Sep-Attention backward                                              */
+/* ------------------------------------------------------------------ */
+/* Gradients of L = sum_{b,h,i,d} out[b,h,i,d] * dout[b,h,i,d] with respect
+ * to q, k, v, where out is the Sep-Attention of the prefill (kept set of row
+ * i: {j <= i : j < a or is_sep[j] or i - j < n}; the training use of the
+ * sparse attention, "HKUDS047: SepLLM ..." study, section on the three
+ * versions: Training-SepLLM).  For each row i over its kept keys j:
+ *   s_j = scale q_i.k_j,  p_j = exp(s_j - m) / sum_t exp(s_t - m),
+ *   out_i = sum_j p_j v_j,  delta_i = dout_i . out_i,
+ *   dv_j += p_j dout_i,  ds_j = p_j (dout_i . v_j - delta_i),
+ *   dq_i += scale sum_j ds_j k_j,  dk_j += scale ds_j q_i.
+ * (the chain rule through the softmax: d s_j = p_j (d p-term - sum_t p_t d p-term)).
+ * q, dout [B,Hq,S,D]; k, v [B,Hkv,S,D] (dtype 0 fp32, 1 bf16 bits, 2 fp64;
+ * dout has its own dtype); dq [B,Hq,S,D], dk, dv [B,Hkv,S,D] fp64 out.
+ * Threads split (b, kv head) units; every query head of a group runs in the
+ * same thread, so its dk/dv sums are race-free. */
+typedef struct {
+  const void *q, *k, *v, *dout;
+  int dtype, dtype_o;
+  const uint8_t* is_sep;
+  int B, Hq, Hkv, S, D, a, n;
+  double scale;
+  double *dq, *dk, *dv;
+} bwd_ctx;
+
+static void bwd_range(void* vctx, int64_t begin, int64_t end, int tid) {
+  (void)tid;
+  bwd_ctx* c = (bwd_ctx*)vctx;
+  int G = c->Hq / c->Hkv, D = c->D, S = c->S;
+  int64_t* krow = (int64_t*)malloc(sizeof(int64_t) * (size_t)S);
+  double* p = (double*)malloc(sizeof(double) * (size_t)S);
+  double qd[512], od[512], go[512];
+  for (int64_t u = begin; u < end; ++u) {
+    int64_t b = u / c->Hkv, g = u % c->Hkv;
+    const uint8_t* sep_row = c->is_sep + b * S;
+    int64_t kv_base = (b * c->Hkv + g) * (int64_t)S;
+    for (int64_t h = g * G; h < (g + 1) * G; ++h) {
+      int64_t qrow0 = (b * c->Hq + h) * (int64_t)S;
+      for (int64_t i = 0; i < S; ++i) {
+        int64_t qi = qrow0 + i;
+        for (int d = 0; d < D; ++d) {
+          qd[d] = elem(c->q, c->dtype, qi * D + d);
+          go[d] = elem(c->dout, c->dtype_o, qi * D + d);
+        }
+        int64_t nk = 0;
+        for (int64_t j = 0; j <= i; ++j)
+          if (kept(sep_row, c->a, c->n, i, j)) krow[nk++] = kv_base + j;
+        double m = -INFINITY;
+        for (int64_t t = 0; t < nk; ++t) {
+          double s = 0.0;
+          for (int d = 0; d < D; ++d) s += qd[d] * elem(c->k, c->dtype, krow[t] * D + d);
+          s *= c->scale;
+          p[t] = s;
+          if (s > m) m = s;
+        }
+        double l = 0.0;
+        for (int64_t t = 0; t < nk; ++t) {
+          p[t] = exp(p[t] - m);
+          l += p[t];
+        }
+        for (int d = 0; d < D; ++d) od[d] = 0.0;
+        for (int64_t t = 0; t < nk; ++t) {
+          p[t] /= l;
+          for (int d = 0; d < D; ++d) od[d] += p[t] * elem(c->v, c->dtype, krow[t] * D + d);
+        }
+        double delta = 0.0;
+        for (int d = 0; d < D; ++d) delta += go[d] * od[d];
+        double* dqi = c->dq + qi * D;
+        for (int64_t t = 0; t < nk; ++t) {
+          double dp = 0.0;
+          for (int d = 0; d < D; ++d) dp += go[d] * elem(c->v, c->dtype, krow[t] * D + d);
+          double ds = p[t] * (dp - delta);
+          double* dkj = c->dk + krow[t] * D;
+          double* dvj = c->dv + krow[t] * D;
+          for (int d = 0; d < D; ++d) {
+            dvj[d] += p[t] * go[d];
+            dkj[d] += c->scale * ds * qd[d];
+            dqi[d] += c->scale * ds * elem(c->k, c->dtype, krow[t] * D + d);
+          }
+        }
+      }
+    }
+  }
+  free(krow);
+  free(p);
+}
+
+int oracle_prefill_backward(const void* q, const void* k, const void* v, int dtype,
+                            const void* dout, int dtype_o, const uint8_t* is_sep, int B, int Hq,
+                            int Hkv, int S, int D, int a, int n, double scale, double* dq,
+                            double* dk, double* dv, int nthreads) {
+  if (D > 512 || Hkv <= 0 || Hq % Hkv != 0 || S < 1 || n < 1 || a < 0) return -1;
+  if (scale <= 0.0) scale = 1.0 / sqrt((double)D);
+  if (nthreads < 1) nthreads = 1;
+  memset(dq, 0, sizeof(double) * (size_t)B * Hq * S * D);
+  memset(dk, 0, sizeof(double) * (size_t)B * Hkv * S * D);
+  memset(dv, 0, sizeof(double) * (size_t)B * Hkv * S * D);
+  bwd_ctx c = {q, k, v, dout, dtype, dtype_o, is_sep, B, Hq, Hkv, S, D, a, n, scale, dq, dk, dv};
+  parallel_for((int64_t)B * Hkv, 1, nthreads, bwd_range, &c);
+  return 0;
+}
