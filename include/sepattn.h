@@ -111,6 +111,28 @@ int sep_attn_prefill(const void* q, const void* k, const void* v, int dtype, con
                      int a, int n, float scale, void* out, float* lse, void* workspace,
                      size_t workspace_bytes, void* stream);
 
+/* Sep-Attention backward (the training use of the sparse attention:
+ * "HKUDS047: SepLLM ..." study, section on the three versions,
+ * Training-SepLLM).  Gradients of sum(out * dout) with respect to q, k, v
+ * through sep_attn_prefill's attention (same kept set, scale and query-head
+ * grouping): per kept pair (i, j), with p_ij the forward probability rebuilt
+ * from lse and delta_i = dout_i . out_i,
+ *   dv_j += p_ij dout_i,  ds_ij = p_ij (dout_i . v_j - delta_i),
+ *   dk_j += scale ds_ij q_i,  dq_i += scale ds_ij k_j
+ * (dk, dv summed over the query heads of each kv head).
+ * q, out, dout, dq: [B, Hq, S, D]; k, v, dk, dv: [B, Hkv, S, D]; lse
+ * [B, Hq, S] fp32 from sep_attn_prefill; is_sep, prefix, idx as for the
+ * prefill.  dtype SEP_BF16 only (fp32 accumulation; SEP_EDTYPE otherwise),
+ * D in {64, 128}.  workspace: sep_attn_backward_workspace() bytes, 256-byte
+ * aligned, contents arbitrary (the call clears what it needs); calls sharing
+ * it must not overlap on the GPU.  Every output element is written. */
+size_t sep_attn_backward_workspace(int B, int Hq, int Hkv, int S, int D);
+int sep_attn_backward(const void* q, const void* k, const void* v, const void* out,
+                      const float* lse, const void* dout, int dtype, const uint8_t* is_sep,
+                      const int32_t* prefix, const int32_t* idx, int B, int Hq, int Hkv, int S,
+                      int D, int a, int n, float scale, void* dq, void* dk, void* dv,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------------------------- */
 /* Streaming decode over the four-block SepCache                            */
 /* ---------------------------------------------------------------------- */

@@ -28,6 +28,7 @@ ABI_SYMBOLS = (
     "sep_attn_decode", "sepcache_status", "sep_device_status", "sep_attn_decode_noalloc",
     "sep_attn_decode_step", "sepcache_ingest", "sepcache_set_rope",
     "sep_attn_decode_masked_workspace", "sep_attn_decode_masked",
+    "sep_attn_backward_workspace", "sep_attn_backward",
 )
 
 
@@ -84,6 +85,10 @@ def _load():
     L.sepcache_compact.argtypes = [ctypes.POINTER(_SepCacheC), i32, P]
     L.sepcache_ingest.argtypes = [ctypes.POINTER(_SepCacheC), i32, P, P, P, P, P, i32, P]
     L.sepcache_set_rope.argtypes = [ctypes.POINTER(_SepCacheC), f32, P]
+    L.sep_attn_backward_workspace.argtypes = [i32, i32, i32, i32, i32]
+    L.sep_attn_backward_workspace.restype = sz
+    L.sep_attn_backward.argtypes = [P, P, P, P, P, P, i32, P, P, P, i32, i32, i32, i32, i32, i32,
+                                    i32, f32, P, P, P, P, sz, P]
     L.sep_attn_decode_masked_workspace.argtypes = [i32, i32, i32, i32, i32]
     L.sep_attn_decode_masked_workspace.restype = sz
     L.sep_attn_decode_masked.argtypes = [P, P, P, i32, P, P, i32, i32, i32, i32, i32, i32, i32,
@@ -99,7 +104,8 @@ def _load():
     for name in ABI_SYMBOLS:
         fn = getattr(L, name)
         if name not in ("sep_strerror", "sep_attn_prefill_workspace", "sepcache_bytes",
-                        "sep_attn_decode_workspace", "sep_attn_decode_masked_workspace"):
+                        "sep_attn_decode_workspace", "sep_attn_decode_masked_workspace",
+                        "sep_attn_backward_workspace"):
             fn.restype = ctypes.c_int
     return L
 
@@ -207,6 +213,28 @@ def prefill(q, k, v, is_sep, prefix, idx, a: int, n: int, scale: float = 0.0, ou
         a, n, float(scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
         _stream(stream)))
     return out, lse
+
+
+def backward(q, k, v, out, lse, dout, is_sep, prefix, idx, a: int, n: int, scale: float = 0.0,
+             dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of sum(out * dout) through Sep-Attention: q/out/dout
+    [B,Hq,S,D], k/v [B,Hkv,S,D] bf16, lse [B,Hq,S] from prefill.
+    Returns (dq, dk, dv)."""
+    _need_cuda(q, k, v, out, lse, dout, is_sep, prefix, idx, dq, dk, dv, workspace)
+    B, Hq, S, D = q.shape
+    Hkv = k.shape[1]
+    dt = _dtype_code(q)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = int(_lib.sep_attn_backward_workspace(B, Hq, Hkv, S, D))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
+    _check("sep_attn_backward", _lib.sep_attn_backward(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), dt, _ptr(is_sep),
+        _ptr(prefix), _ptr(idx), B, Hq, Hkv, S, D, a, n, float(scale), _ptr(dq), _ptr(dk),
+        _ptr(dv), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
 
 
 _masked_ws = {}

@@ -1,0 +1,492 @@
+// Sep-Attention backward (bf16, D in {64, 128}) on warp-level tensor cores.
+//
+// Gradients of sum(out * dout) through the prefill's sparse attention (the
+// training use of Sep-Attention: "HKUDS047: SepLLM ..." study, section on the
+// three versions, Training-SepLLM; kept set of query i from section
+// "SepAttention": {j <= i : j < a or is_sep[j] or i - j < n}).  Per kept pair
+// (i, j), with p_ij the forward's probability (rebuilt from the saved lse)
+// and delta_i = dout_i . out_i:
+//   dv_j += p_ij dout_i,   ds_ij = p_ij (dout_i . v_j - delta_i),
+//   dk_j += scale ds_ij q_i,   dq_i += scale ds_ij k_j.
+//
+// Key-centric work split.  The kept pairs fall into two disjoint families:
+//   * global keys (j < a or a separator) are kept by every query i >= j;
+//     they are taken 64 at a time from the separator index list, and each
+//     block visits the query tiles after its first position, at most
+//     kChunkTiles tiles per CTA;
+//   * local keys (all others) are kept only by queries i in [j, j + n); they
+//     are taken as 64 consecutive positions, and each block visits the query
+//     tiles that reach it, with the global keys of the block masked out.
+// A CTA (four warps, one work item) keeps its 64 keys' K and V in shared
+// memory and the dK and dV of its keys in registers (warp w: keys 16w ..
+// 16w + 15) over all query heads of the kv group and all its query tiles.
+// Per 64-row query tile the warps form S^T = K Q^T and dP^T = V dO^T for
+// their keys (the keys as the 16 rows of the mma tile), P and dS in
+// registers, dV += P^T dO and dK += dS^T Q; dS goes to shared memory and each
+// warp then forms dQ for 16 queries (dS K) and adds it into an fp32
+// accumulator with vector reductions.  At the end the item adds its dK and
+// dV into fp32 accumulators.  A delta pass runs before, and a pass after
+// converts the accumulators (times scale for dq and dk) to bf16.
+#include <string.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace {
+
+constexpr int BR = 64;          // query rows per tile
+constexpr int BC = 64;          // keys per work item
+constexpr int kThreads = 128;   // four warps
+constexpr int kChunkTiles = 8;  // query tiles per item of global keys
+constexpr int kTileBytes = 64 * 128;  // 64 rows x 64 bf16, 128-byte swizzled
+
+// Byte offset of (row r, element d) in a tensor's D/64 swizzled 64-row tiles.
+__device__ __forceinline__ uint32_t swz(int r, int d) {
+  return static_cast<uint32_t>((d >> 6) * kTileBytes + r * 128 +
+                               ((((d >> 3) & 7) ^ (r & 7)) << 4) + (d & 7) * 2);
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// c (16x8 fp32) += a (16x16 bf16, row-major fragment) * b (16x8 bf16, col fragment)
+__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void red_add_v2(float* p, float x, float y) {
+  asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(x), "f"(y) : "memory");
+}
+
+struct BwdParams {
+  const __nv_bfloat16 *q, *k, *v, *dout;
+  const float* lse;    // [B][Hq][S] natural log
+  const float* delta;  // [B][Hq][S]
+  const uint8_t* is_sep;
+  const int32_t *prefix, *idx;
+  float *dq_acc, *dk_acc, *dv_acc;
+  int32_t* err;
+  int B, Hq, Hkv, S, a, n;
+  int nwin;     // window items per (b, kv head) = ceil(S / 64)
+  int nchunk;   // chunks per block of global keys = ceil(ceil(S / 64) / kChunkTiles)
+  float scale_log2;
+};
+
+// delta[b,h,i] = sum_d dout . out, one warp per row
+template <int D>
+__global__ void k_bwd_delta(const __nv_bfloat16* __restrict__ out,
+                            const __nv_bfloat16* __restrict__ dout, float* __restrict__ delta,
+                            int64_t rows) {
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  constexpr int PER = D / 32;  // 2 or 4 elements per lane
+  float acc = 0.f;
+  const __nv_bfloat16* o = out + row * D + lane * PER;
+  const __nv_bfloat16* g = dout + row * D + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc += __bfloat162float(o[e]) * __bfloat162float(g[e]);
+#pragma unroll
+  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) delta[row] = acc;
+}
+
+// fp32 accumulators -> bf16 gradients (dq, dk scaled)
+__global__ void k_bwd_convert(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dst,
+                              int64_t n4, float mul) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 x = reinterpret_cast<const float4*>(acc)[i];
+    __nv_bfloat162 lo = __floats2bfloat162_rn(x.x * mul, x.y * mul);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(x.z * mul, x.w * mul);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&lo);
+    u.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(dst)[i] = u;
+  }
+}
+
+// Shared memory of one CTA (dynamic): K, V [64][D]; Q, dO [2][64][D]; dS^T
+// [64 keys][64 queries], all bf16 swizzled; then the per-tile and per-key
+// scalars.
+template <int D>
+struct Smem {
+  static constexpr int T = (D / 64) * kTileBytes;  // one 64-row tensor
+  static constexpr int K = 0, V = T, Q = 2 * T, DO = 4 * T, DS = 6 * T;
+  static constexpr int LSE = DS + kTileBytes;      // [2][64] fp32 (log2 domain)
+  static constexpr int DEL = LSE + 2 * 64 * 4;     // [2][64] fp32
+  static constexpr int POS = DEL + 2 * 64 * 4;     // [64] int32 key positions
+  static constexpr int LOCAL = POS + 64 * 4;       // [64] int32: key may be used
+  static constexpr int BYTES = LOCAL + 64 * 4;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 2) k_sep_bwd(const BwdParams p) {
+  constexpr int DT = D / 16, NT = D / 8;
+  using SM = Smem<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t sbase = sep::smem_u32(smem);
+  float* const lse_s = reinterpret_cast<float*>(smem + SM::LSE);
+  float* const del_s = reinterpret_cast<float*>(smem + SM::DEL);
+  int32_t* const pos_s = reinterpret_cast<int32_t*>(smem + SM::POS);
+  int32_t* const use_s = reinterpret_cast<int32_t*>(smem + SM::LOCAL);
+
+  const int item = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int S = p.S, G = p.Hq / p.Hkv;
+  const int nT = (S + BR - 1) / BR;
+  const int32_t* pre = p.prefix + static_cast<int64_t>(b) * (S + 1);
+  const int32_t* ix = p.idx + static_cast<int64_t>(b) * S;
+  const uint8_t* fl = p.is_sep + static_cast<int64_t>(b) * S;
+  const int a0 = p.a < S ? p.a : S;
+  const int nglob = a0 + (pre[S] - pre[a0]);  // global keys: initial, then separators >= a
+
+  // ---- the item: its keys and its query tiles
+  const bool window = item < p.nwin;
+  int kb, t0, t1;
+  if (window) {
+    kb = item;
+    t0 = kb;  // queries from the block's first key on
+    const int last = kb * BC + BC - 1 + p.n - 1;  // the last query a key of the block can reach
+    t1 = (last < S - 1 ? last : S - 1) / BR + 1;
+  } else {
+    kb = (item - p.nwin) / p.nchunk;
+    const int chunk = (item - p.nwin) % p.nchunk;
+    if (kb * BC >= nglob) return;
+    const int t = kb * BC;
+    const int pmin = t < a0 ? t : ix[pre[a0] + t - a0];
+    t0 = pmin / BR + chunk * kChunkTiles;
+    t1 = t0 + kChunkTiles < nT ? t0 + kChunkTiles : nT;
+    if (t0 >= nT) return;
+  }
+  // key positions and whether a key takes part in this item's pairs
+  if (threadIdx.x < BC) {
+    const int r = threadIdx.x;
+    int pos = -1, use = 0;
+    if (window) {
+      pos = kb * BC + r;
+      use = pos < S && !(pos < p.a || fl[pos]);  // local keys only
+      if (pos >= S) pos = -1;
+    } else {
+      const int t = kb * BC + r;
+      if (t < nglob) {
+        pos = t < a0 ? t : ix[pre[a0] + t - a0];
+        use = 1;
+      }
+    }
+    pos_s[r] = pos;
+    use_s[r] = use;
+  }
+  __syncthreads();
+  // K and V rows of the block (zero rows where there is no key)
+  const int64_t kvrow0 = (static_cast<int64_t>(b) * p.Hkv + g) * S;
+  for (int e = threadIdx.x; e < BC * (D / 8); e += kThreads) {
+    const int r = e / (D / 8), c = e % (D / 8);
+    const int pos = pos_s[r];
+    const int64_t off = (kvrow0 + (pos < 0 ? 0 : pos)) * D + 8 * c;
+    const uint32_t nb = pos < 0 ? 0u : 16u;
+    cp_async16(sbase + SM::K + swz(r, 8 * c), p.k + off, nb);
+    cp_async16(sbase + SM::V + swz(r, 8 * c), p.v + off, nb);
+  }
+  cp_async_commit();
+
+  // the visits: (head, query tile) pairs, heads outer
+  const int ntile = t1 - t0;
+  const int nvisit = G * ntile;
+  auto load_visit = [&](int v, int buf) {
+    const int h = g * G + v / ntile, t = t0 + v % ntile;
+    const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
+    for (int e = threadIdx.x; e < BR * (D / 8); e += kThreads) {
+      const int r = e / (D / 8), c = e % (D / 8);
+      const int i = t * BR + r;
+      const int64_t off = (qrow0 + (i < S ? i : 0)) * D + 8 * c;
+      const uint32_t nb = i < S ? 16u : 0u;
+      cp_async16(sbase + SM::Q + buf * SM::T + swz(r, 8 * c), p.q + off, nb);
+      cp_async16(sbase + SM::DO + buf * SM::T + swz(r, 8 * c), p.dout + off, nb);
+    }
+    if (threadIdx.x < BR) {
+      const int i = t * BR + threadIdx.x;
+      lse_s[buf * 64 + threadIdx.x] = i < S ? p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
+      del_s[buf * 64 + threadIdx.x] = i < S ? p.delta[qrow0 + i] : 0.f;
+    }
+    cp_async_commit();
+  };
+  if (nvisit > 0) load_visit(0, 0);
+
+  float dk[NT][4], dv[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) dk[nt][e] = dv[nt][e] = 0.f;
+
+  const int kr = 16 * warp;  // this warp's keys
+  for (int v = 0; v < nvisit; ++v) {
+    const int buf = v & 1;
+    const int h = g * G + v / ntile, t = t0 + v % ntile;
+    const int i0 = t * BR;
+    if (v + 1 < nvisit) {
+      load_visit(v + 1, buf ^ 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();  // this visit's tiles (and K, V) are in shared memory
+    const uint32_t qs = sbase + SM::Q + buf * SM::T, ds_ = sbase + SM::DO + buf * SM::T;
+    const uint32_t ks = sbase + SM::K, vs = sbase + SM::V, dss = sbase + SM::DS;
+    const float* lse2 = lse_s + buf * 64;
+    const float* del = del_s + buf * 64;
+    // key rows of this lane: kr + gq and kr + gq + 8
+    const int jp0 = pos_s[kr + gq], jp1 = pos_s[kr + gq + 8];
+    const int u0 = use_s[kr + gq], u1 = use_s[kr + gq + 8];
+    // ---------------- phase A: 16 queries at a time
+#pragma unroll 1
+    for (int sb = 0; sb < BR / 16; ++sb) {
+      float s[2][4] = {}, dp[2][4] = {};
+#pragma unroll
+      for (int kk = 0; kk < DT; ++kk) {
+        uint32_t ka[4], va[4], qb[4], ob[4];
+        ldsm_x4(ks + swz(kr + (lane & 7) + ((lane >> 3) & 1) * 8, 16 * kk + (lane >> 4) * 8), ka);
+        ldsm_x4(vs + swz(kr + (lane & 7) + ((lane >> 3) & 1) * 8, 16 * kk + (lane >> 4) * 8), va);
+        // B = Q^T / dO^T: matrices (queries 0-7 | 8-15) x (dims 16kk | 16kk+8)
+        const int qr = 16 * sb + (lane & 7) + (lane >> 4) * 8, qc = 16 * kk + ((lane >> 3) & 1) * 8;
+        ldsm_x4(qs + swz(qr, qc), qb);
+        ldsm_x4(ds_ + swz(qr, qc), ob);
+        mma16816(s[0], ka, qb[0], qb[1]);
+        mma16816(s[1], ka, qb[2], qb[3]);
+        mma16816(dp[0], va, ob[0], ob[1]);
+        mma16816(dp[1], va, ob[2], ob[3]);
+      }
+      // P and dS: element e of n-tile nt is key kr + gq (+8 for e >= 2),
+      // query 16sb + 8nt + 2tq + (e & 1)
+      uint32_t pa[4], sa[4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        float pv[4], dsv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int q = 16 * sb + 8 * nt + 2 * tq + (e & 1);
+          const int i = i0 + q;
+          const int j = e < 2 ? jp0 : jp1;
+          const int use = e < 2 ? u0 : u1;
+          bool kept = use && j >= 0 && i < S && j <= i;
+          if (window) kept = kept && i - j < p.n;
+          const float pe = kept ? exp2f(s[nt][e] * p.scale_log2 - lse2[q]) : 0.f;
+          pv[e] = pe;
+          dsv[e] = pe * (dp[nt][e] - del[q]);
+        }
+        pa[2 * nt] = sep::pack_bf16x2(pv[0], pv[1]);
+        pa[2 * nt + 1] = sep::pack_bf16x2(pv[2], pv[3]);
+        sa[2 * nt] = sep::pack_bf16x2(dsv[0], dsv[1]);
+        sa[2 * nt + 1] = sep::pack_bf16x2(dsv[2], dsv[3]);
+        // dS^T to shared memory: rows keys, columns queries
+        const int q0 = 16 * sb + 8 * nt + 2 * tq;
+        *reinterpret_cast<uint32_t*>(smem + SM::DS + swz(kr + gq, q0)) = sa[2 * nt];
+        *reinterpret_cast<uint32_t*>(smem + SM::DS + swz(kr + gq + 8, q0)) = sa[2 * nt + 1];
+      }
+      // A fragments of P^T / dS^T (keys x 16 queries): registers 0, 1 of
+      // n-tile 0 and 0, 1 of n-tile 1
+      const uint32_t ap[4] = {pa[0], pa[1], pa[2], pa[3]};
+      const uint32_t as[4] = {sa[0], sa[1], sa[2], sa[3]};
+      // dV += P^T dO, dK += dS^T Q: B = dO / Q (queries x dims) by ldmatrix.trans
+#pragma unroll
+      for (int dn = 0; dn < NT; dn += 2) {
+        uint32_t ob[4], qb[4];
+        const int rr = 16 * sb + (lane & 7) + ((lane >> 3) & 1) * 8, cc = 8 * dn + (lane >> 4) * 8;
+        ldsm_x4_t(ds_ + swz(rr, cc), ob);
+        ldsm_x4_t(qs + swz(rr, cc), qb);
+        mma16816(dv[dn], ap, ob[0], ob[1]);
+        mma16816(dv[dn + 1], ap, ob[2], ob[3]);
+        mma16816(dk[dn], as, qb[0], qb[1]);
+        mma16816(dk[dn + 1], as, qb[2], qb[3]);
+      }
+    }
+    __syncthreads();  // dS^T of all keys is in shared memory
+    // ---------------- phase B: dQ of queries 16w .. 16w + 15 = dS K
+    {
+      float dq[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dq[nt][e] = 0.f;
+#pragma unroll
+      for (int kt = 0; kt < BC / 16; ++kt) {
+        // A = dS (queries x keys) from dS^T by ldmatrix.trans: matrices
+        // (keys 16kt | +8) x (queries 16w | +8)
+        uint32_t aa[4];
+        {
+          const int m = lane >> 3, r = lane & 7;
+          const int key = 16 * kt + (m >> 1) * 8 + r, q = 16 * warp + (m & 1) * 8;
+          ldsm_x4_t(dss + swz(key, q), aa);
+        }
+#pragma unroll
+        for (int dn = 0; dn < NT; dn += 2) {
+          // B = K (keys x dims) by ldmatrix.trans: matrices (keys | +8) x (dims 8dn | +8)
+          uint32_t kb4[4];
+          const int m = lane >> 3, r = lane & 7;
+          const int key = 16 * kt + (m & 1) * 8 + r, d = 8 * dn + (m >> 1) * 8;
+          ldsm_x4_t(ks + swz(key, d), kb4);
+          mma16816(dq[dn], aa, kb4[0], kb4[1]);
+          mma16816(dq[dn + 1], aa, kb4[2], kb4[3]);
+        }
+      }
+      const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int i = i0 + 16 * warp + gq + 8 * half;
+        if (i < S) {
+          float* dst = p.dq_acc + (qrow0 + i) * D + 2 * tq;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) red_add_v2(dst + 8 * nt, dq[nt][2 * half], dq[nt][2 * half + 1]);
+        }
+      }
+    }
+    __syncthreads();  // the buffers of this visit may be refilled
+  }
+  // ---------------- the item's dK and dV
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int key = kr + gq + 8 * half;
+    const int j = pos_s[key];
+    if (j >= 0 && use_s[key]) {
+      float* dkp = p.dk_acc + (kvrow0 + j) * D + 2 * tq;
+      float* dvp = p.dv_acc + (kvrow0 + j) * D + 2 * tq;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        red_add_v2(dkp + 8 * nt, dk[nt][2 * half], dk[nt][2 * half + 1]);
+        red_add_v2(dvp + 8 * nt, dv[nt][2 * half], dv[nt][2 * half + 1]);
+      }
+    }
+  }
+}
+
+struct BwdWs {
+  size_t delta, dq, dk, dv;
+};
+BwdWs bwd_ws(int B, int Hq, int Hkv, int S, int D) {
+  auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  BwdWs w;
+  w.delta = r256(static_cast<size_t>(B) * Hq * S * 4);
+  w.dq = r256(static_cast<size_t>(B) * Hq * S * D * 4);
+  w.dk = r256(static_cast<size_t>(B) * Hkv * S * D * 4);
+  w.dv = w.dk;
+  return w;
+}
+
+template <int D>
+int launch_bwd(const BwdParams& p0, const void* out, void* dq, void* dk, void* dv, void* ws,
+               cudaStream_t st) {
+  BwdParams p = p0;
+  const BwdWs w = bwd_ws(p.B, p.Hq, p.Hkv, p.S, D);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  float* delta = reinterpret_cast<float*>(base);
+  p.delta = delta;
+  p.dq_acc = reinterpret_cast<float*>(base + w.delta);
+  p.dk_acc = reinterpret_cast<float*>(base + w.delta + w.dq);
+  p.dv_acc = reinterpret_cast<float*>(base + w.delta + w.dq + w.dk);
+  if (cudaMemsetAsync(p.dq_acc, 0, w.dq + w.dk + w.dv, st) != cudaSuccess) return SEP_ECUDA;
+  const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.S;
+  k_bwd_delta<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(out), p.dout, delta, rows);
+  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  constexpr int smem = Smem<D>::BYTES;
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(k_sep_bwd<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return SEP_ECUDA;
+    attr_done[dev] = true;
+  }
+  dim3 grid(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B);
+  k_sep_bwd<D><<<grid, kThreads, smem, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  const float sc = p.scale_log2 / 1.44269504088896340736f;
+  struct {
+    const float* acc;
+    void* dst;
+    int64_t n;
+    float mul;
+  } conv[3] = {{p.dq_acc, dq, rows * D, sc},
+               {p.dk_acc, dk, static_cast<int64_t>(p.B) * p.Hkv * p.S * D, sc},
+               {p.dv_acc, dv, static_cast<int64_t>(p.B) * p.Hkv * p.S * D, 1.f}};
+  for (auto& c : conv) {
+    const int64_t n4 = c.n / 4;
+    const int blocks = static_cast<int>(n4 / 256 + 1 < 148 * 16 ? n4 / 256 + 1 : 148 * 16);
+    k_bwd_convert<<<blocks, 256, 0, st>>>(c.acc, static_cast<__nv_bfloat16*>(c.dst), n4, c.mul);
+    if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  }
+  return sep::launch_status();
+}
+
+}  // namespace
+
+extern "C" size_t sep_attn_backward_workspace(int B, int Hq, int Hkv, int S, int D) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Hq % Hkv != 0 || (D != 64 && D != 128)) return 0;
+  const BwdWs w = bwd_ws(B, Hq, Hkv, S, D);
+  return w.delta + w.dq + w.dk + w.dv;
+}
+
+extern "C" int sep_attn_backward(const void* q, const void* k, const void* v, const void* out,
+                                 const float* lse, const void* dout, int dtype,
+                                 const uint8_t* is_sep, const int32_t* prefix, const int32_t* idx,
+                                 int B, int Hq, int Hkv, int S, int D, int a, int n, float scale,
+                                 void* dq, void* dk, void* dv, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (dtype != SEP_BF16) return SEP_EDTYPE;
+  if (D != 64 && D != 128) return SEP_EDTYPE;
+  if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Hq % Hkv != 0 || a < 0 || n < 1) return SEP_EINVAL;
+  if (B > 65535 || Hkv > 65535 || static_cast<int64_t>(B) * Hq * S * D >= (1LL << 40))
+    return SEP_EINVAL;
+  if (!q || !k || !v || !out || !lse || !dout || !is_sep || !prefix || !idx || !dq || !dk || !dv ||
+      !workspace)
+    return SEP_ENULL;
+  if (!sep::aligned16(q) || !sep::aligned16(k) || !sep::aligned16(v) || !sep::aligned16(out) ||
+      !sep::aligned16(dout) || !sep::aligned16(dq) || !sep::aligned16(dk) || !sep::aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return SEP_EALIGN;
+  if (workspace_bytes < sep_attn_backward_workspace(B, Hq, Hkv, S, D)) return SEP_EINVAL;
+  BwdParams p = {};
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.dout = static_cast<const __nv_bfloat16*>(dout);
+  p.lse = lse;
+  p.is_sep = is_sep;
+  p.prefix = prefix;
+  p.idx = idx;
+  p.err = sep::device_error_word();
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.S = S;
+  p.a = a;
+  p.n = n;
+  p.nwin = (S + BC - 1) / BC;
+  p.nchunk = (p.nwin + kChunkTiles - 1) / kChunkTiles;
+  const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(D));
+  p.scale_log2 = sc * 1.44269504088896340736f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return D == 64 ? launch_bwd<64>(p, out, dq, dk, dv, workspace, st)
+                 : launch_bwd<128>(p, out, dq, dk, dv, workspace, st);
+}
