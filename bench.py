@@ -45,6 +45,7 @@ PREFILL_METRIC = "Sep-Attn prefill TFLOP/s on kept pairs"
 DECODE_METRIC = "Sep-Attn decode tokens/s over the four-block SepCache"
 INGEST_METRIC = "SepCache prompt ingestion tokens/s"
 GENERATE_METRIC = "Sep-Attn mask-based generation tokens/s over full histories"
+BACKWARD_METRIC = "Sep-Attn backward TFLOP/s on kept pairs"
 
 
 def _peaks():
@@ -712,6 +713,165 @@ def bench_ingest(sl, args, world, rank):
     return line
 
 
+# ---------------------------------------------------------------- backward
+
+
+def bench_backward(sl, args, world, rank):
+    """Backward of the prefill workload: the gradients of q, k, v for a
+    seeded dout, given the forward's out and lse (computed once, untimed).
+    value = 10 D FLOP per kept pair and head (the five products S, dP, dV,
+    dK, dQ) / device time of sep_attn_backward.  L2 flushed between steps."""
+    name = args.workload
+    wl = PrefillWorkload(sl, name, synth.WORKLOAD_SEED[name] + 7919 * rank)
+    c = wl.cfg
+    B, Hq, Hkv, S, D = c["B"], c["Hq"], c["Hkv"], c["S"], c["D"]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(synth.WORKLOAD_SEED[name] + 17 + 7919 * rank)
+    dout = torch.randn(wl.q.shape, generator=g, device="cuda").bfloat16()
+    wl.step()  # forward: index, out, lse
+    dq, dk, dv = torch.empty_like(wl.q), torch.empty_like(wl.k), torch.empty_like(wl.v)
+    ws = torch.empty((int(sl.lib().sep_attn_backward_workspace(B, Hq, Hkv, S, D)),),
+                     dtype=torch.uint8, device="cuda")
+    flops = 10.0 * D * wl.kept_pairs
+
+    def bwd():
+        sl.backward(wl.q, wl.k, wl.v, wl.out, wl.lse, dout, wl.is_sep, wl.prefix, wl.idx,
+                    c["a"], c["n"], dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    flush = torch.empty((256 << 20,), dtype=torch.uint8, device="cuda")
+    for _ in range(args.warmup):
+        flush.zero_()
+        bwd()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K)]
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
+    _barrier(world)
+    torch.cuda.synchronize()
+    for i in range(K):
+        flush.zero_()  # untimed: evict L2 between steps
+        ev[i][0].record()
+        bwd()
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    _barrier(world)
+    clk = clocks.stop()
+    ms = [a_.elapsed_time(b_) for a_, b_ in ev]
+    t = _max_over_ranks(sum(ms) / 1e3, world)
+    value = flops * K * world / t / 1e12
+    step_s = statistics.mean(ms) / 1e3
+    pk = _peaks()
+    achieved = flops / step_s / 1e12
+    e2e = None
+    if not args.skip_e2e:
+        h = wl.host
+        hq, hk, hv = (x.pin_memory() for x in (h["q"], h["k"], h["v"]))
+        hout, hdo = wl.out.cpu().pin_memory(), dout.cpu().pin_memory()
+        hlse = wl.lse.cpu().pin_memory()
+        hsep = torch.from_numpy(h["is_sep"]).pin_memory()
+        gq_h = torch.empty(dq.shape, dtype=dq.dtype).pin_memory()
+        gk_h = torch.empty(dk.shape, dtype=dk.dtype).pin_memory()
+        gv_h = torch.empty(dv.shape, dtype=dv.dtype).pin_memory()
+        dout_d, out_d, lse_d = torch.empty_like(dout), torch.empty_like(wl.out), torch.empty_like(wl.lse)
+
+        def e2e_step():
+            wl.q.copy_(hq, non_blocking=True)
+            wl.k.copy_(hk, non_blocking=True)
+            wl.v.copy_(hv, non_blocking=True)
+            out_d.copy_(hout, non_blocking=True)
+            lse_d.copy_(hlse, non_blocking=True)
+            dout_d.copy_(hdo, non_blocking=True)
+            wl.is_sep.copy_(hsep, non_blocking=True)
+            sl.build_index(wl.is_sep, out=(wl.prefix, wl.idx, wl.count))
+            sl.backward(wl.q, wl.k, wl.v, out_d, lse_d, dout_d, wl.is_sep, wl.prefix, wl.idx,
+                        c["a"], c["n"], dq=dq, dk=dk, dv=dv, workspace=ws)
+            gq_h.copy_(dq, non_blocking=True)
+            gk_h.copy_(dk, non_blocking=True)
+            gv_h.copy_(dv, non_blocking=True)
+        e2e_step()
+        torch.cuda.synchronize()
+        Ke = max(3, K // 2)
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(Ke):
+            e2e_step()
+        s1.record()
+        torch.cuda.synchronize()
+        te = _max_over_ranks(s0.elapsed_time(s1) / 1e3, world)
+        bi = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hout, hdo, hlse, hsep))
+        bo = sum(x.numel() * x.element_size() for x in (gq_h, gk_h, gv_h))
+        e2e = {"value": round(flops * Ke * world / te / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(bi), "d2h_bytes_per_step": int(bo)}
+    line = {
+        "metric": BACKWARD_METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(t / K * 1e3, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": name, "B": B, "Hq": Hq, "Hkv": Hkv, "S": S, "D": D, "a": c["a"],
+                   "n": c["n"], "kept_pairs": wl.kept_pairs,
+                   "gflop_per_step": round(flops / 1e9, 3),
+                   "l2": "flushed between timed steps (256 MiB write, outside the events)",
+                   "parallelism": "replica per GPU (weak)"},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16"],
+                     "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4),
+                     "traffic": _traffic(name, units=1), "launch_us": round(step_s * 1e6, 3),
+                     "kernel": "sep_attn_backward (delta pass, k_sep_bwd on warp-level "
+                               "mma.sync tensor cores, fp32 -> bf16 pass)",
+                     "peak_source": pk["src"] + " bf16 dense burst (tcgen05 path; the kernel "
+                                    "issues warp-level mma.sync)"},
+        "e2e": e2e, "clocks": clk,
+        "gpu_launches": 5 * K,  # delta, backward, three conversions (plus one memset)
+    }
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        ref = run_reference_backward(argparse.Namespace(steps=1, warmup=0), 1, c, name)
+        line["cpu_baseline"] = ref["cpu_baseline"]
+    return line
+
+
+def run_reference_backward(args, world, c, name):
+    """The oracle's backward on host cores over a bounded sample: the first
+    sequence's first S' tokens (S' <= 1024), all query heads; the kept pairs
+    of the sample give its FLOPs (10 D per pair)."""
+    import oracle
+    inp = synth.prefill_inputs(c, synth.WORKLOAD_SEED[name])
+    Sp = min(c["S"], 1024)
+    q = np.ascontiguousarray(_bits(inp["q"])[:1, :, :Sp])
+    k = np.ascontiguousarray(_bits(inp["k"])[:1, :, :Sp])
+    v = np.ascontiguousarray(_bits(inp["v"])[:1, :, :Sp])
+    dout = q.copy()
+    flags = np.ascontiguousarray(inp["is_sep"][:1, :Sp])
+    kept = int(oracle.count_pairs(flags, c["a"], c["n"]).sum()) * c["Hq"]
+    for _ in range(args.warmup):
+        oracle.prefill_backward(q, k, v, dout, flags, c["a"], c["n"])
+    t0 = time.time()
+    for _ in range(args.steps):
+        oracle.prefill_backward(q, k, v, dout, flags, c["a"], c["n"])
+    dt = (time.time() - t0) / args.steps
+    value = 10.0 * c["D"] * kept / dt / 1e12
+    sample = "sequence 0, tokens 0..%d, all %d query heads (%d kept pairs) per step" % (
+        Sp - 1, c["Hq"], kept)
+    return {"impl": "reference", "metric": BACKWARD_METRIC, "value": round(value, 6),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": name, "B": c["B"], "Hq": c["Hq"], "Hkv": c["Hkv"], "S": c["S"],
+                       "D": c["D"], "a": c["a"], "n": c["n"]},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s",
+                             "cores": min(oracle.nthreads(), c["Hkv"]), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def _bits(t):
+    """bf16 tensor -> raw bits (uint16) for the oracle; fp32 tensor as is."""
+    if t.dtype == torch.bfloat16:
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+    return t.contiguous().numpy()
+
+
 # ---------------------------------------------------------------- mask-based generation
 
 
@@ -992,6 +1152,8 @@ def run_reference(args, world, rank):
         return run_reference_ingest(args, world, c, name)
     if c["kind"] == "generate":
         return run_reference_generate(args, world, c, name)
+    if c["kind"] == "backward":
+        return run_reference_backward(args, world, c, name)
     inp = synth.prefill_inputs(c, synth.WORKLOAD_SEED[name])
     rows, frac = _sample_rows(c, budget_hint=4.0)
     kept = _kept_pairs_rows(inp["is_sep"], c, rows)
@@ -1033,7 +1195,7 @@ def main():
     args = ap.parse_args()
     kind = synth.WORKLOADS[args.workload]["kind"]
     if args.steps is None:
-        args.steps = {"prefill": 50, "ingest": 20, "generate": 200}.get(kind, 2000)
+        args.steps = {"prefill": 50, "ingest": 20, "generate": 200, "backward": 20}.get(kind, 2000)
     args.warmup = max(args.warmup, 3)
 
     if args.impl == "reference":
@@ -1052,6 +1214,8 @@ def main():
         line = bench_ingest(sl, args, world, rank)
     elif kind == "generate":
         line = bench_generate(sl, args, world, rank)
+    elif kind == "backward":
+        line = bench_backward(sl, args, world, rank)
     else:
         line = bench_decode(sl, args, world, rank)
     status = sl.device_status()

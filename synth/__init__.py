@@ -65,6 +65,13 @@ WORKLOADS = {
     "generate_masked_llama3_8b_b16_s8192_d128_bf16": dict(
         kind="generate", B=16, Hq=32, Hkv=8, D=128, dtype="bf16", layers=32, S=8192,
         a=4, n=256, p_sep=0.1, qkv_std=1.0),
+    # Backward of the prefill workloads (training): gradients of q, k, v
+    "backward_llama3_8b_b1_s8192_d128_bf16": dict(
+        kind="backward", B=1, Hq=32, Hkv=8, S=8192, D=128, dtype="bf16", a=4, n=256,
+        p_sep=0.1, ids=None, qkv_std=1.0),
+    "backward_pythia160m_b8h12_s2048_d64_bf16": dict(
+        kind="backward", B=8, Hq=12, Hkv=12, S=2048, D=64, dtype="bf16", a=4, n=64,
+        p_sep=0.08, ids="pythia50k", qkv_std=1.0 / 8.0),
 }
 
 # Base seed per workload (1000 + index in the list above); parity tests add
