@@ -139,8 +139,9 @@ struct Smem {
   static constexpr int BYTES = LOCAL + 64 * 4;
 };
 
+// D = 64 fits three CTAs per SM (registers <= 168), D = 128 two
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2) k_sep_bwd(const BwdParams p) {
+__global__ void __launch_bounds__(kThreads, D == 64 ? 3 : 2) k_sep_bwd(const BwdParams p) {
   constexpr int DT = D / 16, NT = D / 8;
   using SM = Smem<D>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -258,6 +259,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_sep_bwd(const BwdParams p) {
     // key rows of this lane: kr + gq and kr + gq + 8
     const int jp0 = pos_s[kr + gq], jp1 = pos_s[kr + gq + 8];
     const int u0 = use_s[kr + gq], u1 = use_s[kr + gq + 8];
+    // the warp's last key position: a global-key item keeps every valid key
+    // for queries after it, so those sub-blocks need no element mask
+    int jmax = jp0 > jp1 ? jp0 : jp1;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) jmax = max(jmax, __shfl_xor_sync(0xffffffffu, jmax, off));
     // ---------------- phase A: 16 queries at a time
 #pragma unroll 1
     for (int sb = 0; sb < BR / 16; ++sb) {
@@ -279,6 +285,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_sep_bwd(const BwdParams p) {
       // P and dS: element e of n-tile nt is key kr + gq (+8 for e >= 2),
       // query 16sb + 8nt + 2tq + (e & 1)
       uint32_t pa[4], sa[4];
+      // (D = 128 runs at the register limit, where the extra path costs more
+      // than it saves: measured)
+      const bool all_kept = D == 64 && !window && i0 + 16 * sb >= jmax && i0 + 16 * sb + 15 < S;
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         float pv[4], dsv[4];
@@ -288,8 +297,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_sep_bwd(const BwdParams p) {
           const int i = i0 + q;
           const int j = e < 2 ? jp0 : jp1;
           const int use = e < 2 ? u0 : u1;
-          bool kept = use && j >= 0 && i < S && j <= i;
-          if (window) kept = kept && i - j < p.n;
+          bool kept;
+          if (all_kept) {
+            kept = use;
+          } else {
+            kept = use && j >= 0 && i < S && j <= i;
+            if (window) kept = kept && i - j < p.n;
+          }
           const float pe = kept ? exp2f(s[nt][e] * p.scale_log2 - lse2[q]) : 0.f;
           pv[e] = pe;
           dsv[e] = pe * (dp[nt][e] - del[q]);
@@ -321,42 +335,46 @@ __global__ void __launch_bounds__(kThreads, 2) k_sep_bwd(const BwdParams p) {
       }
     }
     __syncthreads();  // dS^T of all keys is in shared memory
-    // ---------------- phase B: dQ of queries 16w .. 16w + 15 = dS K
+    // ---------------- phase B: dQ of queries 16w .. 16w + 15 = dS K, one
+    // half of the dims at a time (half the accumulator registers)
     {
-      float dq[NT][4];
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dq[nt][e] = 0.f;
-#pragma unroll
-      for (int kt = 0; kt < BC / 16; ++kt) {
-        // A = dS (queries x keys) from dS^T by ldmatrix.trans: matrices
-        // (keys 16kt | +8) x (queries 16w | +8)
-        uint32_t aa[4];
-        {
-          const int m = lane >> 3, r = lane & 7;
-          const int key = 16 * kt + (m >> 1) * 8 + r, q = 16 * warp + (m & 1) * 8;
-          ldsm_x4_t(dss + swz(key, q), aa);
-        }
-#pragma unroll
-        for (int dn = 0; dn < NT; dn += 2) {
-          // B = K (keys x dims) by ldmatrix.trans: matrices (keys | +8) x (dims 8dn | +8)
-          uint32_t kb4[4];
-          const int m = lane >> 3, r = lane & 7;
-          const int key = 16 * kt + (m & 1) * 8 + r, d = 8 * dn + (m >> 1) * 8;
-          ldsm_x4_t(ks + swz(key, d), kb4);
-          mma16816(dq[dn], aa, kb4[0], kb4[1]);
-          mma16816(dq[dn + 1], aa, kb4[2], kb4[3]);
-        }
-      }
       const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
+#pragma unroll 1
+      for (int dh = 0; dh < 2; ++dh) {
+        float dq[NT / 2][4];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int i = i0 + 16 * warp + gq + 8 * half;
-        if (i < S) {
-          float* dst = p.dq_acc + (qrow0 + i) * D + 2 * tq;
+        for (int nt = 0; nt < NT / 2; ++nt)
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt) red_add_v2(dst + 8 * nt, dq[nt][2 * half], dq[nt][2 * half + 1]);
+          for (int e = 0; e < 4; ++e) dq[nt][e] = 0.f;
+#pragma unroll
+        for (int kt = 0; kt < BC / 16; ++kt) {
+          // A = dS (queries x keys) from dS^T by ldmatrix.trans: matrices
+          // (keys 16kt | +8) x (queries 16w | +8)
+          uint32_t aa[4];
+          {
+            const int m = lane >> 3, r = lane & 7;
+            const int key = 16 * kt + (m >> 1) * 8 + r, q = 16 * warp + (m & 1) * 8;
+            ldsm_x4_t(dss + swz(key, q), aa);
+          }
+#pragma unroll
+          for (int dn = 0; dn < NT / 2; dn += 2) {
+            // B = K (keys x dims) by ldmatrix.trans: matrices (keys | +8) x (dims | +8)
+            uint32_t kb4[4];
+            const int m = lane >> 3, r = lane & 7;
+            const int key = 16 * kt + (m & 1) * 8 + r, d = 8 * (dh * (NT / 2) + dn) + (m >> 1) * 8;
+            ldsm_x4_t(ks + swz(key, d), kb4);
+            mma16816(dq[dn], aa, kb4[0], kb4[1]);
+            mma16816(dq[dn + 1], aa, kb4[2], kb4[3]);
+          }
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int i = i0 + 16 * warp + gq + 8 * half;
+          if (i < S) {
+            float* dst = p.dq_acc + (qrow0 + i) * D + (D / 2) * dh + 2 * tq;
+#pragma unroll
+            for (int nt = 0; nt < NT / 2; ++nt) red_add_v2(dst + 8 * nt, dq[nt][2 * half], dq[nt][2 * half + 1]);
+          }
         }
       }
     }
@@ -370,10 +388,18 @@ __global__ void __launch_bounds__(kThreads, 2) k_sep_bwd(const BwdParams p) {
     if (j >= 0 && use_s[key]) {
       float* dkp = p.dk_acc + (kvrow0 + j) * D + 2 * tq;
       float* dvp = p.dv_acc + (kvrow0 + j) * D + 2 * tq;
+      if (window) {  // a local key's pairs all belong to this item: plain stores
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        red_add_v2(dkp + 8 * nt, dk[nt][2 * half], dk[nt][2 * half + 1]);
-        red_add_v2(dvp + 8 * nt, dv[nt][2 * half], dv[nt][2 * half + 1]);
+        for (int nt = 0; nt < NT; ++nt) {
+          *reinterpret_cast<float2*>(dkp + 8 * nt) = make_float2(dk[nt][2 * half], dk[nt][2 * half + 1]);
+          *reinterpret_cast<float2*>(dvp + 8 * nt) = make_float2(dv[nt][2 * half], dv[nt][2 * half + 1]);
+        }
+      } else {  // global keys: one item per chunk of query tiles
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          red_add_v2(dkp + 8 * nt, dk[nt][2 * half], dk[nt][2 * half + 1]);
+          red_add_v2(dvp + 8 * nt, dv[nt][2 * half], dv[nt][2 * half + 1]);
+        }
       }
     }
   }
