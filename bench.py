@@ -69,11 +69,20 @@ def _peaks():
 # proportion to the retained rows).
 TRAFFIC = {
     "decode_llama3_8b_b16_l32_t65536_d128_bf16": dict(
-        bytes=(28613632 + 0) / (420.5 * 16), per="row", src=("decode.cu", "common.cuh"),
-        sha1="1ff00ea8ff526fc5d2f3bebd8de2529b9ee09d05"),
+        bytes=(28613888 + 1536) / (420.5 * 16), per="row", src=("decode.cu", "common.cuh"),
+        sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
     "decode_rope_llama3_8b_b16_l32_t65536_d128_bf16": dict(
-        bytes=(28884992 + 0) / (421.19 * 16), per="row", src=("decode.cu", "common.cuh"),
-        sha1="1ff00ea8ff526fc5d2f3bebd8de2529b9ee09d05"),
+        bytes=(28885248 + 0) / (421.19 * 16), per="row", src=("decode.cu", "common.cuh"),
+        sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
+    "generate_masked_llama3_8b_b16_s8192_d128_bf16": dict(
+        bytes=69485568 + 1160448, per="launch", src=("decode.cu", "common.cuh"),
+        sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
+    "backward_llama3_8b_b1_s8192_d128_bf16": dict(
+        bytes=318605568 + 161198080, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="6e9731b99d0a106d28786a56bbffc5ca59fd6ccd"),
+    "backward_pythia160m_b8h12_s2048_d64_bf16": dict(
+        bytes=161130240 + 105582848, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="6e9731b99d0a106d28786a56bbffc5ca59fd6ccd"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
         bytes=104798720 + 29326080, per="launch", src=("prefill_tc.cu", "common.cuh"),
         sha1="33933b4438440541d25b84d21f8513b525cea57a"),
