@@ -339,14 +339,18 @@ __global__ void __launch_bounds__(256) k_cache_ingest_rows(
   const int32_t* cnt = counts + 4 * b;
   const int len = cnt[0] + cnt[1] + cnt[2] + cnt[3];
   if (len < 0 || len > cap) return;
-  const int ch = row_bytes / 16;
+  const int ch = row_bytes / 16;  // 16-byte chunks per row: a power of two (8, 16 or 32)
+  const int lg = __ffs(ch) - 1;
   const int64_t dbase = row0(0, layer, b, g, layers, B, Hkv, cap, row_bytes);
   const int64_t sbase = (static_cast<int64_t>(b) * Hkv + g) * T * row_bytes;
   const int32_t* ps = pos + static_cast<int64_t>(b) * cap;
-  const int total = 2 * len * ch;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-    const int which = e / (len * ch);
-    const int r = (e / ch) % len, c = e % ch;
+  const int half = len << lg;  // chunks of K; V follows
+  // one chunk per thread, the K rows first, then the V rows (shifts and a
+  // compare, no division)
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < 2 * half; e += gridDim.x * blockDim.x) {
+    const bool which = e >= half;
+    const int e1 = which ? e - half : e;
+    const int r = e1 >> lg, c = e1 & (ch - 1);
     const int p = ps[r];
     if (p < 0 || p >= T) continue;
     const uint4 val = reinterpret_cast<const uint4*>((which ? v : k) + sbase + static_cast<int64_t>(p) * row_bytes)[c];
