@@ -405,6 +405,569 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 3 : 2) k_sep_bwd(const Bwd
   }
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 form (D = 128), two kernels on the operand forms of the forward:
+//   k_sep_bwd_tc_kv (key-centric, 128 keys in TMEM lanes, 128-query tiles,
+//     Q and dO double-buffered): S^T = K Q^T and dP^T = V dO^T (SS); warps
+//     0-3 (thread = key row) turn them into P^T and dS^T, written back as
+//     bf16 over the first 64 columns of each; dV += P^T dO and dK += dS^T Q
+//     (TS, B MN-major).  TMEM: S^T [0,128) dP^T [128,256) dV [256,384)
+//     dK [384,512).
+//   k_sep_bwd_tc_q (query-centric, 128 queries in TMEM lanes, over the kept
+//     key blocks of its tile as the forward does: the global keys before the
+//     window unmasked, then the window blocks with the element mask; K and V
+//     double-buffered): S = Q K^T and dP = dO V^T (SS); thread = query row
+//     forms dS, written back as bf16; dQ += dS K (TS, B = K MN-major).  The
+//     CTA owns its queries, so dQ is stored once, as bf16, with no
+//     reduction.  TMEM: S [0,128) dP [128,256) dQ [256,384).
+// Warps 0-7 share the 128 TMEM lanes two by two (warp w: lanes 32 (w & 3) ..
+// +31, columns [64 (w >> 2), +64) of each 128-column tile); the two warps of
+// a lane quarter load all their scores before either stores the bf16 P / dS
+// over them.  Warp 8 allocates TMEM; its lane 0 issues the MMAs while the
+// other lanes wait for it, and the warp reaches the block barrier together.
+constexpr int TBK = 128;  // keys per block (TMEM lanes of the key-centric kernel)
+constexpr int TBQ = 128;  // queries per tile
+constexpr int kTcThreads = 288;  // warps 0-7: softmax, loads, readout; warp 8: TMEM and MMA issue
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 256;
+constexpr int kT128 = 128 * 128;  // one 128-row x 64-column swizzled tile
+constexpr int kTcChunkTiles = 4;  // query tiles per item of global keys
+
+__device__ __forceinline__ uint32_t swz128(int r, int d) {
+  return static_cast<uint32_t>((d >> 6) * kT128 + r * 128 + ((((d >> 3) & 7) ^ (r & 7)) << 4) +
+                               (d & 7) * 2);
+}
+// packed fp32 pairs (one f32x2 instruction per pair)
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// kind::f16 instruction descriptor with bf16 A/B, fp32 D and each operand's
+// major-ness (bit 15: A MN-major, bit 16: B MN-major)
+__host__ __device__ constexpr uint32_t idesc_mn(int M, int N, bool a_mn, bool b_mn) {
+  return sep::idesc_bf16_f32(M, N, b_mn) | ((a_mn ? 1u : 0u) << 15);
+}
+// Rows [0, 128) of a [rows, 128] bf16 tensor into a swizzled 128-row tile
+// pair, one 16-byte chunk per copy; row_of(r) < 0 gives a zero row.
+template <typename RowOf>
+__device__ __forceinline__ void load_rows128(uint32_t dst, const __nv_bfloat16* src, RowOf row_of,
+                                             int tid, int nthreads) {
+  for (int e = tid; e < 128 * 16; e += nthreads) {
+    const int r = e >> 4, c = e & 15;
+    const int64_t row = row_of(r);
+    cp_async16(dst + swz128(r, 8 * c), src + (row < 0 ? 0 : row) * 128 + 8 * c, row < 0 ? 0u : 16u);
+  }
+}
+
+struct KvSmem {
+  static constexpr int K = 0, V = 2 * kT128, Q = 4 * kT128, DO = 8 * kT128;  // Q, dO: [2] x 2 tiles
+  static constexpr int LSE = 12 * kT128;  // [2][128] fp32: -lse (log2 domain)
+  static constexpr int DEL = LSE + 1024;  // [2][128] fp32
+  static constexpr int POS = DEL + 1024;  // [128] int32
+  static constexpr int USE = POS + 512;   // [128] int32
+  static constexpr int BYTES = USE + 512 + 1024;  // + alignment slack
+};
+struct TcBars {
+  uint64_t full, s_full, p_full, m_full, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_kv(const BwdParams p) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* const smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ TcBars bars;
+  const uint32_t sb_ = sep::smem_u32(smem);
+  float* const lse_s = reinterpret_cast<float*>(smem + KvSmem::LSE);
+  float* const del_s = reinterpret_cast<float*>(smem + KvSmem::DEL);
+  int32_t* const pos_s = reinterpret_cast<int32_t*>(smem + KvSmem::POS);
+  int32_t* const use_s = reinterpret_cast<int32_t*>(smem + KvSmem::USE);
+
+  const int item = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.S, G = p.Hq / p.Hkv;
+  const int nT = (S + TBQ - 1) / TBQ;
+  const int32_t* pre = p.prefix + static_cast<int64_t>(b) * (S + 1);
+  const int32_t* ix = p.idx + static_cast<int64_t>(b) * S;
+  const uint8_t* fl = p.is_sep + static_cast<int64_t>(b) * S;
+  const int a0 = p.a < S ? p.a : S;
+  const int nglob = a0 + (pre[S] - pre[a0]);
+
+  const bool window = item < p.nwin;
+  int kb, t0, t1;
+  if (window) {
+    kb = item;
+    t0 = kb;
+    const int last = kb * TBK + TBK - 1 + p.n - 1;
+    t1 = (last < S - 1 ? last : S - 1) / TBQ + 1;
+  } else {
+    kb = (item - p.nwin) / p.nchunk;
+    const int chunk = (item - p.nwin) % p.nchunk;
+    if (kb * TBK >= nglob) return;
+    const int t = kb * TBK;
+    const int pmin = t < a0 ? t : ix[pre[a0] + t - a0];
+    t0 = pmin / TBQ + chunk * kTcChunkTiles;
+    t1 = t0 + kTcChunkTiles < nT ? t0 + kTcChunkTiles : nT;
+    if (t0 >= nT) return;
+  }
+  const int ntile = t1 - t0;
+  const int nvisit = G * ntile;
+
+  if (threadIdx.x == 0) {
+    sep::mbar_init(&bars.full, 1);
+    sep::mbar_init(&bars.s_full, 1);
+    sep::mbar_init(&bars.p_full, 1);
+    sep::mbar_init(&bars.m_full, 1);
+    sep::mbar_init(&bars.drain, 1);
+    bars.abort = 0;
+    sep::mbar_fence_init();
+  }
+  if (threadIdx.x < TBK) {
+    const int r = threadIdx.x;
+    int pos = -1, use = 0;
+    if (window) {
+      pos = kb * TBK + r;
+      use = pos < S && !(pos < p.a || fl[pos]);
+      if (pos >= S) pos = -1;
+    } else {
+      const int t = kb * TBK + r;
+      if (t < nglob) {
+        pos = t < a0 ? t : ix[pre[a0] + t - a0];
+        use = 1;
+      }
+    }
+    pos_s[r] = pos;
+    use_s[r] = use;
+  }
+  if (warp == 8) {
+    sep::tmem_alloc(&bars.tmem_base, 512);
+    sep::tmem_relinquish();
+  }
+  sep::tc_fence_before();
+  __syncthreads();
+  sep::tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+  volatile int* abort = &bars.abort;
+  const int64_t kvrow0 = (static_cast<int64_t>(b) * p.Hkv + g) * S;
+
+  if (warp < 8) {
+    // ------------------------------------------------ compute warps
+    const int tid = threadIdx.x;
+    const int lq = warp & 3, ch = warp >> 2;
+    const int r = 32 * lq + lane;  // key row = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(32 * lq) << 16;
+    load_rows128(sb_ + KvSmem::K, p.k, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
+    load_rows128(sb_ + KvSmem::V, p.v, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
+    auto load_visit = [&](int v, int buf) {
+      const int h = g * G + v / ntile, t = t0 + v % ntile;
+      const int i0 = t * TBQ;
+      const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
+      auto rowq = [&](int rr) -> int64_t { return i0 + rr < S ? qrow0 + i0 + rr : -1; };
+      load_rows128(sb_ + KvSmem::Q + buf * 2 * kT128, p.q, rowq, tid, 256);
+      load_rows128(sb_ + KvSmem::DO + buf * 2 * kT128, p.dout, rowq, tid, 256);
+      if (tid < TBQ) {
+        const int i = i0 + tid;
+        lse_s[buf * 128 + tid] = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
+        del_s[buf * 128 + tid] = i < S ? p.delta[qrow0 + i] : 0.f;
+      }
+      cp_async_commit();
+    };
+    load_visit(0, 0);  // the same group as K and V
+    const int jp = pos_s[r], use = use_s[r];
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+    bool ok = true;
+    for (int v = 0; v < nvisit && ok; ++v) {
+      const int buf = v & 1;
+      const int t = t0 + v % ntile;
+      const int i0 = t * TBQ;
+      if (v > 0 && (!sep::mbar_wait(&bars.m_full, (v - 1) & 1, abort, p.err) || *abort)) {
+        ok = false;  // the products of visit v-1 have read buffer (v+1) & 1
+        break;
+      }
+      if (v + 1 < nvisit) {
+        load_visit(v + 1, buf ^ 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      sep::fence_proxy_async_smem();
+      sep::named_bar_sync(1, 256);
+      if (tid == 0) sep::mbar_arrive(&bars.full);
+      if (!sep::mbar_wait(&bars.s_full, v & 1, abort, p.err) || *abort) {
+        ok = false;
+        break;
+      }
+      sep::tc_fence_after();
+      // the query columns this key row keeps: [qa, qb)
+      int qa = 0, qb = 0;
+      if (use && jp >= 0) {
+        qa = jp - i0 > 0 ? jp - i0 : 0;
+        qb = S - i0 < TBQ ? S - i0 : TBQ;
+        if (window && jp + p.n - i0 < qb) qb = jp + p.n - i0;
+      }
+      uint32_t sv[64], dv_[64];
+      sep::tmem_ld32(tmem + lane_base + kColS + 64 * ch, sv);
+      sep::tmem_ld32(tmem + lane_base + kColS + 64 * ch + 32, sv + 32);
+      sep::tmem_ld32(tmem + lane_base + kColDP + 64 * ch, dv_);
+      sep::tmem_ld32(tmem + lane_base + kColDP + 64 * ch + 32, dv_ + 32);
+      sep::tmem_wait_ld_r32(sv);
+      sep::tmem_wait_ld_r32(sv + 32);
+      sep::tmem_wait_ld_r32(dv_);
+      sep::tmem_wait_ld_r32(dv_ + 32);
+      sep::named_bar_sync(2 + lq, 64);  // the partner warp has read its scores too
+      const float* nl = lse_s + buf * 128 + 64 * ch;
+      const float* dl = del_s + buf * 128 + 64 * ch;
+      uint32_t pp[32], dd[32];
+#pragma unroll
+      for (int e = 0; e < 64; e += 2) {
+        const int q = 64 * ch + e;
+        const float2 x = sep::ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2,
+                                    *reinterpret_cast<const float2*>(nl + e));
+        const float p0 = (q >= qa && q < qb) ? sep::ex2_approx(x.x) : 0.f;
+        const float p1 = (q + 1 >= qa && q + 1 < qb) ? sep::ex2_approx(x.y) : 0.f;
+        const float2 ds = fmul2(make_float2(p0, p1),
+                                fsub2(make_float2(__uint_as_float(dv_[e]), __uint_as_float(dv_[e + 1])),
+                                      *reinterpret_cast<const float2*>(dl + e)));
+        pp[e / 2] = sep::pack_bf16x2(p0, p1);
+        dd[e / 2] = sep::pack_bf16x2(ds.x, ds.y);
+      }
+      sep::tmem_st32(tmem + lane_base + kColS + 32 * ch, pp);
+      sep::tmem_st32(tmem + lane_base + kColDP + 32 * ch, dd);
+      sep::tmem_wait_st();
+      sep::tc_fence_before();
+      sep::named_bar_sync(1, 256);
+      if (tid == 0) sep::mbar_arrive(&bars.p_full);
+    }
+    if (ok && nvisit > 0 && sep::mbar_wait(&bars.m_full, (nvisit - 1) & 1, abort, p.err) && !*abort) {
+      sep::tc_fence_after();
+      // dK and dV of this key row, columns [64 ch, +64): every lane loads
+      // (warp-wide), rows with a key store
+      const bool mine = jp >= 0 && use;
+      float* dkp = p.dk_acc + (kvrow0 + (mine ? jp : 0)) * D + 64 * ch;
+      float* dvp = p.dv_acc + (kvrow0 + (mine ? jp : 0)) * D + 64 * ch;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t kv[32], vv[32];
+        sep::tmem_ld32(tmem + lane_base + kColDK + 64 * ch + 32 * c, kv);
+        sep::tmem_ld32(tmem + lane_base + kColDV + 64 * ch + 32 * c, vv);
+        sep::tmem_wait_ld_r32(kv);
+        sep::tmem_wait_ld_r32(vv);
+        if (mine) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            if (window) {
+              *reinterpret_cast<float2*>(dkp + 32 * c + e) = make_float2(__uint_as_float(kv[e]), __uint_as_float(kv[e + 1]));
+              *reinterpret_cast<float2*>(dvp + 32 * c + e) = make_float2(__uint_as_float(vv[e]), __uint_as_float(vv[e + 1]));
+            } else {
+              red_add_v2(dkp + 32 * c + e, __uint_as_float(kv[e]), __uint_as_float(kv[e + 1]));
+              red_add_v2(dvp + 32 * c + e, __uint_as_float(vv[e]), __uint_as_float(vv[e + 1]));
+            }
+          }
+        }
+      }
+    }
+    cp_async_wait<0>();
+  } else {
+    if (lane == 0) {
+      // ---------------------------------------------- MMA issue (one thread)
+      constexpr uint32_t id_s = idesc_mn(128, 128, false, false);
+      constexpr uint32_t id_o = idesc_mn(128, D, false, true);
+      const uint64_t dK = sep::smem_desc_sw128(sb_ + KvSmem::K, 16);
+      const uint64_t dV = sep::smem_desc_sw128(sb_ + KvSmem::V, 16);
+      for (int v = 0; v < nvisit; ++v) {
+        const int buf = v & 1;
+        if (!sep::mbar_wait(&bars.full, v & 1, abort, p.err)) break;
+        sep::tc_fence_after();
+        const uint32_t qa = sb_ + KvSmem::Q + buf * 2 * kT128, oa = sb_ + KvSmem::DO + buf * 2 * kT128;
+        const uint64_t dQ = sep::smem_desc_sw128(qa, 16), dO = sep::smem_desc_sw128(oa, 16);
+        const uint64_t dQmn = sep::smem_desc_sw128(qa, kT128), dOmn = sep::smem_desc_sw128(oa, kT128);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
+          sep::mma_bf16_ss(tmem + kColS, dK + off, dQ + off, id_s, kk > 0 ? 1u : 0u);
+          sep::mma_bf16_ss(tmem + kColDP, dV + off, dO + off, id_s, kk > 0 ? 1u : 0u);
+        }
+        sep::mma_commit(&bars.s_full);
+        if (!sep::mbar_wait(&bars.p_full, v & 1, abort, p.err)) break;
+        sep::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < TBQ / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
+          const uint32_t acc = (v > 0 || kk > 0) ? 1u : 0u;
+          sep::mma_bf16_ts(tmem + kColDV, tmem + kColS + kk * 8, dOmn + off, id_o, acc);
+          sep::mma_bf16_ts(tmem + kColDK, tmem + kColDP + kk * 8, dQmn + off, id_o, acc);
+        }
+        sep::mma_commit(&bars.m_full);
+      }
+      sep::mma_commit(&bars.drain);  // every MMA completes before TMEM is released
+      int keep = 0;
+      sep::mbar_wait(&bars.drain, 0, &keep, nullptr);
+    }
+    __syncwarp();
+  }
+  sep::tc_fence_before();
+  __syncthreads();
+  sep::tc_fence_after();
+  if (warp == 8) {
+    __syncwarp();
+    sep::tmem_dealloc(tmem, 512);
+  }
+}
+
+struct QSmem {
+  static constexpr int Q = 0, DO = 2 * kT128;
+  static constexpr int K = 4 * kT128, V = 6 * kT128;  // [2] buffers, 4 tiles apart
+  static constexpr int POS = 12 * kT128;  // [2][128] int32 key positions
+  static constexpr int GLB = POS + 1024;  // [2][128] int32: key kept by every later query
+  static constexpr int BYTES = GLB + 1024 + 1024;
+};
+
+__global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams p,
+                                                                __nv_bfloat16* __restrict__ dq) {
+  constexpr int D = 128;
+  extern __shared__ uint8_t dsm_raw[];
+  uint8_t* const smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ TcBars bars;
+  const uint32_t sb_ = sep::smem_u32(smem);
+  int32_t* const pos_s = reinterpret_cast<int32_t*>(smem + QSmem::POS);
+  int32_t* const glb_s = reinterpret_cast<int32_t*>(smem + QSmem::GLB);
+
+  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.S, G = p.Hq / p.Hkv, g = h / G;
+  const int i0 = t * TBQ;
+  const int qlast = (i0 + TBQ < S ? i0 + TBQ : S) - 1;
+  const int32_t* pre = p.prefix + static_cast<int64_t>(b) * (S + 1);
+  const int32_t* ix = p.idx + static_cast<int64_t>(b) * S;
+  const uint8_t* fl = p.is_sep + static_cast<int64_t>(b) * S;
+  // the tile's kept keys: global keys before the first row's window, then
+  // the window positions [lo, qlast]
+  const int lo = i0 - p.n + 1 > 0 ? i0 - p.n + 1 : 0;
+  const int al = p.a < lo ? p.a : lo;
+  const int nglo = al + (pre[lo] - pre[al]);
+  const int nbg = (nglo + TBK - 1) / TBK;
+  const int nbw = (qlast - lo + TBK) / TBK;
+  const int nblk = nbg + nbw;
+  const int64_t kvrow0 = (static_cast<int64_t>(b) * p.Hkv + g) * S;
+  const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
+
+  if (threadIdx.x == 0) {
+    sep::mbar_init(&bars.full, 1);
+    sep::mbar_init(&bars.s_full, 1);
+    sep::mbar_init(&bars.p_full, 1);
+    sep::mbar_init(&bars.m_full, 1);
+    sep::mbar_init(&bars.drain, 1);
+    bars.abort = 0;
+    sep::mbar_fence_init();
+  }
+  if (warp == 8) {
+    sep::tmem_alloc(&bars.tmem_base, 512);
+    sep::tmem_relinquish();
+  }
+  sep::tc_fence_before();
+  __syncthreads();
+  sep::tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+  volatile int* abort = &bars.abort;
+
+  if (warp < 8) {
+    const int tid = threadIdx.x;
+    const int lq = warp & 3, ch = warp >> 2;
+    const int r = 32 * lq + lane;  // query row = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>(32 * lq) << 16;
+    const int i = i0 + r;
+    const float nlse2 = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
+    const float dl = i < S ? p.delta[qrow0 + i] : 0.f;
+    auto rowq = [&](int rr) -> int64_t { return i0 + rr < S ? qrow0 + i0 + rr : -1; };
+    load_rows128(sb_ + QSmem::Q, p.q, rowq, tid, 256);
+    load_rows128(sb_ + QSmem::DO, p.dout, rowq, tid, 256);
+    auto load_block = [&](int j, int buf) {
+      // key positions of block j (threads 0..127: one key each), then rows
+      if (tid < TBK) {
+        int pos = -1, glb = 0;
+        if (j < nbg) {
+          const int e = j * TBK + tid;
+          if (e < nglo) {
+            pos = e < al ? e : ix[pre[al] + e - al];
+            glb = 1;
+          }
+        } else {
+          const int q = lo + (j - nbg) * TBK + tid;
+          if (q <= qlast) {
+            pos = q;
+            glb = q < p.a || fl[q];
+          }
+        }
+        pos_s[buf * 128 + tid] = pos;
+        glb_s[buf * 128 + tid] = glb;
+      }
+      sep::named_bar_sync(1, 256);  // every position is written before the row copies read them
+      auto rowk = [&](int rr) -> int64_t { const int q = pos_s[buf * 128 + rr]; return q < 0 ? -1 : kvrow0 + q; };
+      load_rows128(sb_ + QSmem::K + buf * 4 * kT128, p.k, rowk, tid, 256);
+      load_rows128(sb_ + QSmem::V + buf * 4 * kT128, p.v, rowk, tid, 256);
+      cp_async_commit();
+    };
+    load_block(0, 0);  // with Q and dO
+    const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+    const float2 nl2 = make_float2(nlse2, nlse2), dl2 = make_float2(dl, dl);
+    bool ok = true;
+    for (int j = 0; j < nblk && ok; ++j) {
+      const int buf = j & 1;
+      if (j > 0 && (!sep::mbar_wait(&bars.m_full, (j - 1) & 1, abort, p.err) || *abort)) {
+        ok = false;  // the products of block j-1 have read buffer (j+1) & 1
+        break;
+      }
+      if (j + 1 < nblk) {
+        load_block(j + 1, buf ^ 1);
+        cp_async_wait<1>();
+      } else {
+        cp_async_wait<0>();
+      }
+      sep::fence_proxy_async_smem();
+      sep::named_bar_sync(1, 256);
+      if (tid == 0) sep::mbar_arrive(&bars.full);
+      if (!sep::mbar_wait(&bars.s_full, j & 1, abort, p.err) || *abort) {
+        ok = false;
+        break;
+      }
+      sep::tc_fence_after();
+      const int32_t* gb = glb_s + buf * 128 + 64 * ch;
+      // the key columns this query row keeps: global blocks, every valid
+      // key; window blocks (contiguous positions from `base`), keys at most
+      // n - 1 back, or global ones, never past the row or the tile
+      int ka, kb2;
+      const bool win = j >= nbg;
+      int wlo = 0;
+      if (!win) {
+        ka = 0;
+        kb2 = nglo - j * TBK < TBK ? nglo - j * TBK : TBK;
+        if (i >= S) kb2 = 0;
+      } else {
+        const int base = lo + (j - nbg) * TBK;
+        ka = 0;
+        kb2 = i - base + 1;  // keys at positions <= i
+        const int lim = qlast - base + 1;
+        if (kb2 > lim) kb2 = lim;
+        if (kb2 > TBK) kb2 = TBK;
+        if (i >= S) kb2 = 0;
+        wlo = i - base - p.n + 1;  // keys before this column need the global flag
+      }
+      uint32_t sv[64], dv_[64];
+      sep::tmem_ld32(tmem + lane_base + kColS + 64 * ch, sv);
+      sep::tmem_ld32(tmem + lane_base + kColS + 64 * ch + 32, sv + 32);
+      sep::tmem_ld32(tmem + lane_base + kColDP + 64 * ch, dv_);
+      sep::tmem_ld32(tmem + lane_base + kColDP + 64 * ch + 32, dv_ + 32);
+      sep::tmem_wait_ld_r32(sv);
+      sep::tmem_wait_ld_r32(sv + 32);
+      sep::tmem_wait_ld_r32(dv_);
+      sep::tmem_wait_ld_r32(dv_ + 32);
+      sep::named_bar_sync(2 + lq, 64);  // the partner warp has read its scores too
+      uint32_t dd[32];
+#pragma unroll
+      for (int e = 0; e < 64; e += 2) {
+        const int kc = 64 * ch + e;
+        const float2 x = sep::ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, nl2);
+        bool k0 = kc >= ka && kc < kb2, k1 = kc + 1 >= ka && kc + 1 < kb2;
+        if (win) {
+          k0 = k0 && (kc >= wlo || gb[e]);
+          k1 = k1 && (kc + 1 >= wlo || gb[e + 1]);
+        }
+        const float p0 = k0 ? sep::ex2_approx(x.x) : 0.f;
+        const float p1 = k1 ? sep::ex2_approx(x.y) : 0.f;
+        const float2 ds = fmul2(make_float2(p0, p1),
+                                fsub2(make_float2(__uint_as_float(dv_[e]), __uint_as_float(dv_[e + 1])), dl2));
+        dd[e / 2] = sep::pack_bf16x2(ds.x, ds.y);
+      }
+      sep::tmem_st32(tmem + lane_base + kColS + 32 * ch, dd);
+      sep::tmem_wait_st();
+      sep::tc_fence_before();
+      sep::named_bar_sync(1, 256);
+      if (tid == 0) sep::mbar_arrive(&bars.p_full);
+    }
+    if (ok && sep::mbar_wait(&bars.m_full, (nblk - 1) & 1, abort, p.err) && !*abort) {
+      sep::tc_fence_after();
+      const float sc = p.scale_log2 * 0.69314718055994530942f;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t qv[32];
+        sep::tmem_ld32(tmem + lane_base + kColDQ + 64 * ch + 32 * c, qv);
+        sep::tmem_wait_ld_r32(qv);
+        if (i < S) {
+          uint4* dst = reinterpret_cast<uint4*>(dq + (qrow0 + i) * D + 64 * ch + 32 * c);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            dst[u] = make_uint4(sep::pack_bf16x2(__uint_as_float(qv[8 * u]) * sc, __uint_as_float(qv[8 * u + 1]) * sc),
+                                sep::pack_bf16x2(__uint_as_float(qv[8 * u + 2]) * sc, __uint_as_float(qv[8 * u + 3]) * sc),
+                                sep::pack_bf16x2(__uint_as_float(qv[8 * u + 4]) * sc, __uint_as_float(qv[8 * u + 5]) * sc),
+                                sep::pack_bf16x2(__uint_as_float(qv[8 * u + 6]) * sc, __uint_as_float(qv[8 * u + 7]) * sc));
+        }
+      }
+    }
+    cp_async_wait<0>();
+  } else {
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_mn(128, 128, false, false);
+      constexpr uint32_t id_o = idesc_mn(128, D, false, true);
+      const uint64_t dQ = sep::smem_desc_sw128(sb_ + QSmem::Q, 16);
+      const uint64_t dO = sep::smem_desc_sw128(sb_ + QSmem::DO, 16);
+      for (int j = 0; j < nblk; ++j) {
+        const int buf = j & 1;
+        if (!sep::mbar_wait(&bars.full, j & 1, abort, p.err)) break;
+        sep::tc_fence_after();
+        const uint32_t ka = sb_ + QSmem::K + buf * 4 * kT128, va = sb_ + QSmem::V + buf * 4 * kT128;
+        const uint64_t dK = sep::smem_desc_sw128(ka, 16), dV = sep::smem_desc_sw128(va, 16);
+        const uint64_t dKmn = sep::smem_desc_sw128(ka, kT128);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
+          sep::mma_bf16_ss(tmem + kColS, dQ + off, dK + off, id_s, kk > 0 ? 1u : 0u);
+          sep::mma_bf16_ss(tmem + kColDP, dO + off, dV + off, id_s, kk > 0 ? 1u : 0u);
+        }
+        sep::mma_commit(&bars.s_full);
+        if (!sep::mbar_wait(&bars.p_full, j & 1, abort, p.err)) break;
+        sep::tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < TBK / 16; ++kk) {
+          const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
+          sep::mma_bf16_ts(tmem + kColDQ, tmem + kColS + kk * 8, dKmn + off, id_o,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        sep::mma_commit(&bars.m_full);
+      }
+      sep::mma_commit(&bars.drain);
+      int keep = 0;
+      sep::mbar_wait(&bars.drain, 0, &keep, nullptr);
+    }
+    __syncwarp();
+  }
+  sep::tc_fence_before();
+  __syncthreads();
+  sep::tc_fence_after();
+  if (warp == 8) {
+    __syncwarp();
+    sep::tmem_dealloc(tmem, 512);
+  }
+}
+
+// D = 128 runs the tcgen05 kernels
+constexpr bool kTcBackward = true;
+
 struct BwdWs {
   size_t delta, dq, dk, dv;
 };
@@ -418,6 +981,28 @@ BwdWs bwd_ws(int B, int Hq, int Hkv, int S, int D) {
   return w;
 }
 
+// the tcgen05 kernels (D = 128): dK, dV key-centric; dQ query-centric
+int launch_bwd_tc(BwdParams p, void* dq, cudaStream_t st) {
+  static bool attr_done[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(k_sep_bwd_tc_kv, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             KvSmem::BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(k_sep_bwd_tc_q, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             QSmem::BYTES) != cudaSuccess)
+      return SEP_ECUDA;
+    attr_done[dev] = true;
+  }
+  p.nwin = (p.S + TBK - 1) / TBK;
+  p.nchunk = (p.nwin + kTcChunkTiles - 1) / kTcChunkTiles;
+  k_sep_bwd_tc_kv<<<dim3(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B), kTcThreads, KvSmem::BYTES, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  k_sep_bwd_tc_q<<<dim3((p.S + TBQ - 1) / TBQ, p.Hq, p.B), kTcThreads, QSmem::BYTES, st>>>(
+      p, static_cast<__nv_bfloat16*>(dq));
+  return cudaGetLastError() == cudaSuccess ? SEP_OK : SEP_ECUDA;
+}
+
 template <int D>
 int launch_bwd(const BwdParams& p0, const void* out, void* dq, void* dk, void* dv, void* ws,
                cudaStream_t st) {
@@ -429,11 +1014,20 @@ int launch_bwd(const BwdParams& p0, const void* out, void* dq, void* dk, void* d
   p.dq_acc = reinterpret_cast<float*>(base + w.delta);
   p.dk_acc = reinterpret_cast<float*>(base + w.delta + w.dq);
   p.dv_acc = reinterpret_cast<float*>(base + w.delta + w.dq + w.dk);
-  if (cudaMemsetAsync(p.dq_acc, 0, w.dq + w.dk + w.dv, st) != cudaSuccess) return SEP_ECUDA;
+  const bool tc = D == 128 && kTcBackward;  // dq is then written directly, in bf16
+  if (tc) {
+    if (cudaMemsetAsync(p.dk_acc, 0, w.dk + w.dv, st) != cudaSuccess) return SEP_ECUDA;
+  } else if (cudaMemsetAsync(p.dq_acc, 0, w.dq + w.dk + w.dv, st) != cudaSuccess) {
+    return SEP_ECUDA;
+  }
   const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.S;
   k_bwd_delta<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
       static_cast<const __nv_bfloat16*>(out), p.dout, delta, rows);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  if (tc) {
+    const int rc = launch_bwd_tc(p, dq, st);
+    if (rc != SEP_OK) return rc;
+  } else {
   constexpr int smem = Smem<D>::BYTES;
   static bool attr_done[64] = {false};
   int dev = 0;
@@ -447,6 +1041,7 @@ int launch_bwd(const BwdParams& p0, const void* out, void* dq, void* dk, void* d
   dim3 grid(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B);
   k_sep_bwd<D><<<grid, kThreads, smem, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  }
   const float sc = p.scale_log2 / 1.44269504088896340736f;
   struct {
     const float* acc;
@@ -457,6 +1052,7 @@ int launch_bwd(const BwdParams& p0, const void* out, void* dq, void* dk, void* d
                {p.dk_acc, dk, static_cast<int64_t>(p.B) * p.Hkv * p.S * D, sc},
                {p.dv_acc, dv, static_cast<int64_t>(p.B) * p.Hkv * p.S * D, 1.f}};
   for (auto& c : conv) {
+    if (tc && c.dst == dq) continue;  // already written
     const int64_t n4 = c.n / 4;
     const int blocks = static_cast<int>(n4 / 256 + 1 < 148 * 16 ? n4 / 256 + 1 : 148 * 16);
     k_bwd_convert<<<blocks, 256, 0, st>>>(c.acc, static_cast<__nv_bfloat16*>(c.dst), n4, c.mul);
