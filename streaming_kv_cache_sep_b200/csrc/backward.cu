@@ -482,11 +482,14 @@ struct KvSmem {
 };
 struct TcBars {
   uint64_t full, s_full, p_full, m_full, drain;
+  uint64_t tile[2];  // tensor-copy completion of a Q / dO buffer (key-centric kernel)
   uint32_t tmem_base;
   int abort;
 };
 
-__global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_kv(const BwdParams p) {
+__global__ void __launch_bounds__(kTcThreads, 1)
+    k_sep_bwd_tc_kv(const BwdParams p, const __grid_constant__ CUtensorMap map_q,
+                    const __grid_constant__ CUtensorMap map_do) {
   constexpr int D = 128;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* const smem = reinterpret_cast<uint8_t*>(
@@ -534,6 +537,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_kv(const BwdParams
     sep::mbar_init(&bars.p_full, 1);
     sep::mbar_init(&bars.m_full, 1);
     sep::mbar_init(&bars.drain, 1);
+    sep::mbar_init(&bars.tile[0], 1);
+    sep::mbar_init(&bars.tile[1], 1);
     bars.abort = 0;
     sep::mbar_fence_init();
   }
@@ -573,21 +578,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_kv(const BwdParams
     const uint32_t lane_base = static_cast<uint32_t>(32 * lq) << 16;
     load_rows128(sb_ + KvSmem::K, p.k, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
     load_rows128(sb_ + KvSmem::V, p.v, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
-    auto load_visit = [&](int v, int buf) {
+    cp_async_commit();
+    // lse (negated, log2 domain) and delta of visit v's queries: thread
+    // tid < 128 loads its query's pair (into registers one visit ahead)
+    auto row_stats = [&](int v, float& nl, float& dl) {
       const int h = g * G + v / ntile, t = t0 + v % ntile;
-      const int i0 = t * TBQ;
+      const int i = t * TBQ + tid;
       const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
-      auto rowq = [&](int rr) -> int64_t { return i0 + rr < S ? qrow0 + i0 + rr : -1; };
-      load_rows128(sb_ + KvSmem::Q + buf * 2 * kT128, p.q, rowq, tid, 256);
-      load_rows128(sb_ + KvSmem::DO + buf * 2 * kT128, p.dout, rowq, tid, 256);
-      if (tid < TBQ) {
-        const int i = i0 + tid;
-        lse_s[buf * 128 + tid] = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
-        del_s[buf * 128 + tid] = i < S ? p.delta[qrow0 + i] : 0.f;
-      }
-      cp_async_commit();
+      nl = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
+      dl = i < S ? p.delta[qrow0 + i] : 0.f;
     };
-    load_visit(0, 0);  // the same group as K and V
+    if (tid < TBQ) {
+      float nl, dl;
+      row_stats(0, nl, dl);
+      lse_s[tid] = nl;
+      del_s[tid] = dl;
+    }
+    cp_async_wait<0>();  // K and V
+    sep::fence_proxy_async_smem();
+    sep::named_bar_sync(1, 256);
+    if (tid == 0) sep::mbar_arrive(&bars.full);  // K and V are in shared memory
     const int jp = pos_s[r], use = use_s[r];
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
@@ -595,19 +605,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_kv(const BwdParams
       const int buf = v & 1;
       const int t = t0 + v % ntile;
       const int i0 = t * TBQ;
-      if (v > 0 && (!sep::mbar_wait(&bars.m_full, (v - 1) & 1, abort, p.err) || *abort)) {
-        ok = false;  // the products of visit v-1 have read buffer (v+1) & 1
-        break;
-      }
-      if (v + 1 < nvisit) {
-        load_visit(v + 1, buf ^ 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      sep::fence_proxy_async_smem();
-      sep::named_bar_sync(1, 256);
-      if (tid == 0) sep::mbar_arrive(&bars.full);
+      float nl_next = 0.f, dl_next = 0.f;
+      if (v + 1 < nvisit && tid < TBQ) row_stats(v + 1, nl_next, dl_next);
       if (!sep::mbar_wait(&bars.s_full, v & 1, abort, p.err) || *abort) {
         ok = false;
         break;
@@ -648,6 +647,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_kv(const BwdParams
       }
       sep::tmem_st32(tmem + lane_base + kColS + 32 * ch, pp);
       sep::tmem_st32(tmem + lane_base + kColDP + 32 * ch, dd);
+      if (v + 1 < nvisit && tid < TBQ) {  // buffer (v+1) & 1 was last read by visit v-1
+        lse_s[(buf ^ 1) * 128 + tid] = nl_next;
+        del_s[(buf ^ 1) * 128 + tid] = dl_next;
+      }
       sep::tmem_wait_st();
       sep::tc_fence_before();
       sep::named_bar_sync(1, 256);
@@ -689,9 +692,25 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_kv(const BwdParams
       constexpr uint32_t id_o = idesc_mn(128, D, false, true);
       const uint64_t dK = sep::smem_desc_sw128(sb_ + KvSmem::K, 16);
       const uint64_t dV = sep::smem_desc_sw128(sb_ + KvSmem::V, 16);
-      for (int v = 0; v < nvisit; ++v) {
+      // Q and dO tiles of visit v into buffer v & 1 by the tensor-copy
+      // engine (two 64-column tiles each; rows past the head belong to the
+      // next head or are zero-filled past the array, and their P is 0)
+      auto load_tiles = [&](int v) {
+        const int h = g * G + v / ntile, t = t0 + v % ntile;
+        const int32_t row = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hq + h) * S + t * TBQ);
         const int buf = v & 1;
-        if (!sep::mbar_wait(&bars.full, v & 1, abort, p.err)) break;
+        sep::mbar_arrive_expect_tx(&bars.tile[buf], 4 * kT128);
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          sep::tma_load_2d(smem + KvSmem::Q + buf * 2 * kT128 + c * kT128, &map_q, 64 * c, row, &bars.tile[buf]);
+          sep::tma_load_2d(smem + KvSmem::DO + buf * 2 * kT128 + c * kT128, &map_do, 64 * c, row, &bars.tile[buf]);
+        }
+      };
+      if (nvisit > 0) load_tiles(0);
+      bool kv_in = sep::mbar_wait(&bars.full, 0, abort, p.err);  // K and V
+      for (int v = 0; v < nvisit && kv_in; ++v) {
+        const int buf = v & 1;
+        if (!sep::mbar_wait(&bars.tile[buf], (v >> 1) & 1, abort, p.err)) break;
         sep::tc_fence_after();
         const uint32_t qa = sb_ + KvSmem::Q + buf * 2 * kT128, oa = sb_ + KvSmem::DO + buf * 2 * kT128;
         const uint64_t dQ = sep::smem_desc_sw128(qa, 16), dO = sep::smem_desc_sw128(oa, 16);
@@ -704,6 +723,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_kv(const BwdParams
         }
         sep::mma_commit(&bars.s_full);
         if (!sep::mbar_wait(&bars.p_full, v & 1, abort, p.err)) break;
+        // the scores of visit v are complete, so (in order) are the products
+        // of visit v-1: buffer (v+1) & 1 may be refilled
+        if (v + 1 < nvisit) load_tiles(v + 1);
         sep::tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < TBQ / 16; ++kk) {
@@ -996,7 +1018,12 @@ int launch_bwd_tc(BwdParams p, void* dq, cudaStream_t st) {
   }
   p.nwin = (p.S + TBK - 1) / TBK;
   p.nchunk = (p.nwin + kTcChunkTiles - 1) / kTcChunkTiles;
-  k_sep_bwd_tc_kv<<<dim3(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B), kTcThreads, KvSmem::BYTES, st>>>(p);
+  const int64_t qrows = static_cast<int64_t>(p.B) * p.Hq * p.S;
+  if (qrows > 0x7fffffffLL) return SEP_ETOOBIG;
+  CUtensorMap mq, mdo;
+  if (!sep::make_rows_map(&mq, p.q, qrows, 128, TBQ) || !sep::make_rows_map(&mdo, p.dout, qrows, 128, TBQ))
+    return SEP_ECUDA;
+  k_sep_bwd_tc_kv<<<dim3(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B), kTcThreads, KvSmem::BYTES, st>>>(p, mq, mdo);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   k_sep_bwd_tc_q<<<dim3((p.S + TBQ - 1) / TBQ, p.Hq, p.B), kTcThreads, QSmem::BYTES, st>>>(
       p, static_cast<__nv_bfloat16*>(dq));
