@@ -78,11 +78,11 @@ TRAFFIC = {
         bytes=69485568 + 1160448, per="launch", src=("decode.cu", "common.cuh"),
         sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
     "backward_llama3_8b_b1_s8192_d128_bf16": dict(
-        bytes=318605568 + 161198080, per="launch", src=("backward.cu", "common.cuh"),
-        sha1="6e9731b99d0a106d28786a56bbffc5ca59fd6ccd"),
+        bytes=223200000 + 208900000, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="ccc1d51920b8eb0ffa71d1c0b81985af9610007c"),
     "backward_pythia160m_b8h12_s2048_d64_bf16": dict(
-        bytes=161130240 + 105582848, per="launch", src=("backward.cu", "common.cuh"),
-        sha1="6e9731b99d0a106d28786a56bbffc5ca59fd6ccd"),
+        bytes=161018624 + 101916928, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="ccc1d51920b8eb0ffa71d1c0b81985af9610007c"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
         bytes=104798720 + 29326080, per="launch", src=("prefill_tc.cu", "common.cuh"),
         sha1="33933b4438440541d25b84d21f8513b525cea57a"),
@@ -827,12 +827,16 @@ def bench_backward(sl, args, world, rank):
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16"],
                      "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4),
                      "traffic": _traffic(name, units=1), "launch_us": round(step_s * 1e6, 3),
-                     "kernel": "sep_attn_backward (delta pass, k_sep_bwd on warp-level "
-                               "mma.sync tensor cores, fp32 -> bf16 pass)",
-                     "peak_source": pk["src"] + " bf16 dense burst (tcgen05 path; the kernel "
-                                    "issues warp-level mma.sync)"},
+                     "kernel": ("sep_attn_backward: delta pass, k_sep_bwd_tc_kv (dK, dV) + "
+                                "k_sep_bwd_tc_q (dQ) on tcgen05, fp32 -> bf16 pass; traffic = "
+                                "the two tcgen05 kernels" if D == 128 else
+                                "sep_attn_backward: delta pass, k_sep_bwd on warp-level mma.sync, "
+                                "fp32 -> bf16 pass; traffic = k_sep_bwd"),
+                     "peak_source": pk["src"] + " bf16 dense burst"},
         "e2e": e2e, "clocks": clk,
-        "gpu_launches": 5 * K,  # delta, backward, three conversions (plus one memset)
+        # D = 128: delta, two tcgen05 kernels, two conversions; D = 64: delta, one
+        # kernel, three conversions (plus one memset either way)
+        "gpu_launches": 5 * K,
     }
     if rank == 0 and world == 1 and not args.skip_cpu:
         ref = run_reference_backward(argparse.Namespace(steps=1, warmup=0), 1, c, name)

@@ -1,4 +1,5 @@
-// Sep-Attention backward (bf16, D in {64, 128}) on warp-level tensor cores.
+// Sep-Attention backward (bf16, D in {64, 128}): warp-level tensor cores
+// (mma.sync) for D = 64, tcgen05 for D = 128 (second part of this file).
 //
 // Gradients of sum(out * dout) through the prefill's sparse attention (the
 // training use of Sep-Attention: "HKUDS047: SepLLM ..." study, section on the
@@ -423,7 +424,8 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 3 : 2) k_sep_bwd(const Bwd
 // Warps 0-7 share the 128 TMEM lanes two by two (warp w: lanes 32 (w & 3) ..
 // +31, columns [64 (w >> 2), +64) of each 128-column tile); the two warps of
 // a lane quarter load all their scores before either stores the bf16 P / dS
-// over them.  Warp 8 allocates TMEM; its lane 0 issues the MMAs while the
+// over them.  Warp 8 allocates TMEM; its lane 0 issues the MMAs (and, in the
+// key-centric kernel, the tensor copies of the Q and dO tiles) while the
 // other lanes wait for it, and the warp reaches the block barrier together.
 constexpr int TBK = 128;  // keys per block (TMEM lanes of the key-centric kernel)
 constexpr int TBQ = 128;  // queries per tile

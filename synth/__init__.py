@@ -72,6 +72,11 @@ WORKLOADS = {
     "backward_pythia160m_b8h12_s2048_d64_bf16": dict(
         kind="backward", B=8, Hq=12, Hkv=12, S=2048, D=64, dtype="bf16", a=4, n=64,
         p_sep=0.08, ids="pythia50k", qkv_std=1.0 / 8.0),
+    # The Llama-3-8B backward on 2k tokens: the size a full counter capture
+    # of the D128 backward kernels takes
+    "backward_llama3_8b_b1_s2048_d128_bf16": dict(
+        kind="backward", B=1, Hq=32, Hkv=8, S=2048, D=128, dtype="bf16", a=4, n=256,
+        p_sep=0.1, ids=None, qkv_std=1.0),
 }
 
 # Base seed per workload (1000 + index in the list above); parity tests add
