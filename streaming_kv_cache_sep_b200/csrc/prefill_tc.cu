@@ -162,9 +162,23 @@ __device__ __forceinline__ uint32_t bits_le(int x) {
   return x < 0 ? 0u : (x >= 31 ? 0xffffffffu : (0xffffffffu >> (31 - x)));
 }
 
+// mbarrier phase wait: one (potentially blocking) try inline, the bounded
+// retry loop out of line.  Inlined at each of the kernel's wait sites the
+// loop costs some 9 KB of instructions; one shared copy keeps the code that
+// the warps run per item small enough for the instruction cache.
+__device__ __noinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            int32_t* err_word) {
+  return sep::mbar_wait(bar, parity, abort, err_word);
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int32_t* err_word) {
+  return sep::mbar_try_wait(bar, parity) || mbar_wait_loop(bar, parity, abort, err_word);
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   int dummy = 0;
-  sep::mbar_wait(bar, parity, &dummy, nullptr);
+  mbar_wait(bar, parity, &dummy, nullptr);
 }
 
 // MMA issue for both tiles from one thread, P written over S (D = 128): per
@@ -185,12 +199,12 @@ __device__ __forceinline__ void mma_single_issuer(const Params& p, uint8_t* smem
   bool ok = true;
   bool v_ready = false;  // V of the block whose PVs are being issued has landed
   auto issue_pv = [&](int t, uint32_t vblk, bool first) -> bool {
-    if (!sep::mbar_wait(&bars->p_full[t], (pphase >> t) & 1u, abort, p.err)) return false;
+    if (!mbar_wait(&bars->p_full[t], (pphase >> t) & 1u, abort, p.err)) return false;
     pphase ^= 1u << t;
-    if (!v_ready && !sep::mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err))
+    if (!v_ready && !mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err))
       return false;
     v_ready = true;
-    if (first && nitem > 0 && !sep::mbar_wait(&bars->o_empty[t], (nitem - 1) & 1, abort, p.err))
+    if (first && nitem > 0 && !mbar_wait(&bars->o_empty[t], (nitem - 1) & 1, abort, p.err))
       return false;
     sep::tc_fence_after();
     const uint64_t dv = dv0 + static_cast<uint64_t>((vblk % NST) * (C::KV_BYTES >> 4));
@@ -214,11 +228,11 @@ __device__ __forceinline__ void mma_single_issuer(const Params& p, uint8_t* smem
   };
   for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
     const Item it = make_item(p, item);
-    if (!sep::mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
+    if (!mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
     bool prev_a = false, prev_b = false;  // tile kept the previous block
     bool pv_a = false, pv_b = false;      // tile already accumulated into O this item
     for (int j = 0; j < it.nblk; ++j, ++gblk) {
-      if (!sep::mbar_wait(&bars->k_full[gblk % NST], (gblk / NST) & 1, abort, p.err)) {
+      if (!mbar_wait(&bars->k_full[gblk % NST], (gblk / NST) & 1, abort, p.err)) {
         ok = false;
         break;
       }
@@ -320,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
         const Item it = make_item(p, item);
         const int64_t kv_row0 = static_cast<int64_t>(it.b * p.Hkv + it.g) * p.S;
-        if (nitem > 0 && !sep::mbar_wait(&bars->q_empty, (nitem - 1) & 1, abort, p.err)) break;
+        if (nitem > 0 && !mbar_wait(&bars->q_empty, (nitem - 1) & 1, abort, p.err)) break;
         sep::mbar_arrive_expect_tx(&bars->q_full, 2 * C::Q_BYTES);
         for (int t = 0; t < 2; ++t) {
           const int64_t qrow = static_cast<int64_t>(it.b * p.Hq + it.h[t]) * p.S + it.q0[t];
@@ -338,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int64_t row = kv_row0 + (gathered ? static_cast<int64_t>(j) * BN
                                                   : it.win_lo + static_cast<int64_t>(j - it.nblk_g) * BN);
           if (gblk >= static_cast<uint32_t>(NST) &&
-              !sep::mbar_wait(&bars->k_empty[st], (use - 1) & 1, abort, p.err)) {
+              !mbar_wait(&bars->k_empty[st], (use - 1) & 1, abort, p.err)) {
             ok = false;
             break;
           }
@@ -349,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              r * 64, static_cast<int32_t>(row), &bars->k_full[st]);
           last_k[st] = static_cast<int>(gblk);
           if (gblk >= static_cast<uint32_t>(NST) &&
-              !sep::mbar_wait(&bars->v_empty[st], (use - 1) & 1, abort, p.err)) {
+              !mbar_wait(&bars->v_empty[st], (use - 1) & 1, abort, p.err)) {
             ok = false;
             break;
           }
@@ -401,10 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // item overwrites O_t, so it waits until the previous item's epilogue
       // of this tile has read O_t.
       auto issue_pv = [&](uint32_t vblk, bool first) -> bool {
-        if (!sep::mbar_wait(&bars->p_full[t], pphase, abort, p.err)) return false;
+        if (!mbar_wait(&bars->p_full[t], pphase, abort, p.err)) return false;
         pphase ^= 1u;
-        if (!sep::mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err)) return false;
-        if (first && nitem > 0 && !sep::mbar_wait(&bars->o_empty[t], (nitem - 1) & 1, abort, p.err))
+        if (!mbar_wait(&bars->v_full[vblk % NST], (vblk / NST) & 1, abort, p.err)) return false;
+        if (first && nitem > 0 && !mbar_wait(&bars->o_empty[t], (nitem - 1) & 1, abort, p.err))
           return false;
         sep::tc_fence_after();
         const uint64_t dv = dv0 + static_cast<uint64_t>((vblk % NST) * (C::KV_BYTES >> 4));
@@ -417,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_s = [&](uint32_t kblk) -> bool {
         if (C::SEP_P) {
           // S_t is free once the softmax has read the previous block's scores
-          if (ns > 0 && !sep::mbar_wait(&bars->s_free[t], (ns - 1) & 1, abort, p.err)) return false;
+          if (ns > 0 && !mbar_wait(&bars->s_free[t], (ns - 1) & 1, abort, p.err)) return false;
           ++ns;
           sep::tc_fence_after();
         }
@@ -432,11 +446,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
         const Item it = make_item(p, item);
-        if (!sep::mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
+        if (!mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
         bool prev = false;  // this tile kept the previous block
         bool pv = false;    // this tile already accumulated into O this item
         for (int j = 0; j < it.nblk; ++j, ++gblk) {
-          if (!sep::mbar_wait(&bars->k_full[gblk % NST], (gblk / NST) & 1, abort, p.err)) {
+          if (!mbar_wait(&bars->k_full[gblk % NST], (gblk / NST) & 1, abort, p.err)) {
             ok = false;
             break;
           }
@@ -492,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (C::SEP_P) {
         sep::tc_fence_before();
         sep::mbar_arrive(&bars->s_free[t]);
-        if (npv > 0 && !__all_sync(0xffffffffu, sep::mbar_wait(&bars->pv_done[t], (npv - 1) & 1, abort, p.err)))
+        if (npv > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[t], (npv - 1) & 1, abort, p.err)))
           return false;
         ++npv;
         sep::tc_fence_after();
@@ -551,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       ~bits_le(jlo - 1 - 32 * c);
           }
         }
-        if (!__all_sync(0xffffffffu, sep::mbar_wait(&bars->s_full[t], sphase, abort, p.err))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], sphase, abort, p.err))) {
           ok = false;
           break;
         }
@@ -670,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // P*V, and MMAs complete in order, so that P*V is done.  Separate P:
           // wait for it (pass 2 below still reads S_t; it is freed after).
           if constexpr (C::SEP_P) {
-            if (npv > 0 && !__all_sync(0xffffffffu, sep::mbar_wait(&bars->pv_done[t], (npv - 1) & 1, abort, p.err))) {
+            if (npv > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars->pv_done[t], (npv - 1) & 1, abort, p.err))) {
               ok = false;
               break;
             }
@@ -742,7 +756,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
       // epilogue: O_t / l -> out (bf16), lse
-      if (!__all_sync(0xffffffffu, sep::mbar_wait(&bars->o_full[t], nitem & 1, abort, p.err))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars->o_full[t], nitem & 1, abort, p.err))) {
         ok = false;
         break;
       }
