@@ -84,10 +84,11 @@ TRAFFIC = {
         bytes=161018624 + 101916928, per="launch", src=("backward.cu", "common.cuh"),
         sha1="ccc1d51920b8eb0ffa71d1c0b81985af9610007c"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
-        bytes=104798720 + 29326080, per="launch", src=("prefill_tc.cu", "common.cuh"),
-        sha1="33933b4438440541d25b84d21f8513b525cea57a"),
+        bytes=104788480 + 29667840, per="launch", src=("prefill_tc.cu", "common.cuh"),
+        sha1="0ccfa2f810f1862257e2228d4f7439111558f44b"),
     "prefill_pythia160m_b8h12_s2048_d64_bf16": dict(
-        bytes=82608128 + 9976576, per="launch", src=("prefill_tc.cu", "common.cuh"), sha1="33933b4438440541d25b84d21f8513b525cea57a"),
+        bytes=82165248 + 8908800, per="launch", src=("prefill_tc.cu", "common.cuh"),
+        sha1="0ccfa2f810f1862257e2228d4f7439111558f44b"),
 }
 
 
