@@ -241,22 +241,16 @@ class PrefillWorkload:
         kept = int(sl.count_pairs(prefix, cfg["a"], cfg["n"]).sum().item()) * cfg["Hq"]
         self.kept_pairs = kept
         self.flops = 4.0 * cfg["D"] * kept
-        self.launches_per_step = (1 if self.has_ids else 0) + 1 + (2 if dt == 1 else 1)
+        # front: one launch (flags and index from ids, or the index from
+        # flags); sep_attn_prefill: the separator-row gather and attention
+        self.launches_per_step = 1 + (2 if dt == 1 else 1)
 
     def front(self):
         if self.has_ids:
-            self._flags_into()
-        self.sl.build_index(self.is_sep, out=(self.prefix, self.idx, self.count))
-
-    def _flags_into(self):
-        import ctypes
-        arr = (ctypes.c_int32 * len(self.sep_ids))(*self.sep_ids)
-        rc = self.sl.lib().sep_flags_from_ids(
-            ctypes.c_void_p(self.ids.data_ptr()), self.ids.numel(), ctypes.cast(arr, ctypes.c_void_p),
-            len(self.sep_ids), ctypes.c_void_p(self.is_sep.data_ptr()),
-            ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-        if rc != 0:
-            raise RuntimeError("sep_flags_from_ids failed %d" % rc)
+            self.sl.build_index_from_ids(self.ids, self.sep_ids,
+                                         out=(self.is_sep, self.prefix, self.idx, self.count))
+        else:
+            self.sl.build_index(self.is_sep, out=(self.prefix, self.idx, self.count))
 
     def attn(self):
         c = self.cfg

@@ -79,6 +79,14 @@ int sep_flags_from_ids(const int32_t* ids, int64_t n_tok, const int32_t* sep_ids
 int sep_build_index(const uint8_t* is_sep, int B, int S, int32_t* prefix, int32_t* idx,
                     int32_t* count, void* stream);
 
+/* sep_flags_from_ids followed by sep_build_index in one launch: ids int32
+ * [B, S] -> is_sep uint8 [B, S] (written), prefix [B, S+1], idx [B, S],
+ * count [B], with the same results as the two calls.  sep_ids: HOST int32
+ * array, 1 <= n_sep_ids <= 32.  B >= 1, S >= 1. */
+int sep_build_index_from_ids(const int32_t* ids, int B, int S, const int32_t* sep_ids,
+                             int n_sep_ids, uint8_t* is_sep, int32_t* prefix, int32_t* idx,
+                             int32_t* count, void* stream);
+
 /* Kept (query, key) pairs of one head of each sequence (the retention
  * statistics of the HKUDS047 study, section "Forward Input Wrapper").
  * prefix: from sep_build_index; kept_pairs: int64 [B]. a >= 0, n >= 1. */

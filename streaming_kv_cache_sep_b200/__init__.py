@@ -22,7 +22,8 @@ SEP_BF16 = 1
 
 # every symbol include/sepattn.h declares
 ABI_SYMBOLS = (
-    "sep_strerror", "sep_version", "sep_flags_from_ids", "sep_build_index", "sep_count_pairs",
+    "sep_strerror", "sep_version", "sep_flags_from_ids", "sep_build_index",
+    "sep_build_index_from_ids", "sep_count_pairs",
     "sep_attn_prefill_workspace", "sep_attn_prefill", "sepcache_bytes", "sepcache_carve",
     "sepcache_init", "sepcache_append", "sepcache_compact", "sep_attn_decode_workspace",
     "sep_attn_decode", "sepcache_status", "sep_device_status", "sep_attn_decode_noalloc",
@@ -71,6 +72,7 @@ def _load():
     L.sep_version.argtypes = []
     L.sep_flags_from_ids.argtypes = [P, i64, P, i32, P, P]
     L.sep_build_index.argtypes = [P, i32, i32, P, P, P, P]
+    L.sep_build_index_from_ids.argtypes = [P, i32, i32, P, i32, P, P, P, P, P]
     L.sep_count_pairs.argtypes = [P, i32, i32, i32, i32, P, P]
     L.sep_attn_prefill_workspace.argtypes = [i32, i32, i32, i32, i32, i32]
     L.sep_attn_prefill_workspace.restype = sz
@@ -174,6 +176,26 @@ def build_index(is_sep: torch.Tensor, out=None, stream=None):
     _check("sep_build_index", _lib.sep_build_index(_ptr(is_sep), B, S, _ptr(prefix), _ptr(idx),
                                                    _ptr(count), _stream(stream)))
     return prefix, idx, count
+
+
+def build_index_from_ids(ids: torch.Tensor, sep_ids, out=None, stream=None):
+    """flags_from_ids then build_index in one launch: ids int32 [B,S] ->
+    (is_sep uint8 [B,S], prefix [B,S+1], idx [B,S], count [B]) on the device."""
+    _need_cuda(ids)
+    assert ids.dtype == torch.int32 and ids.dim() == 2
+    B, S = ids.shape
+    dev = ids.device
+    if out is None:
+        out = (torch.empty((B, S), dtype=torch.uint8, device=dev),
+               torch.empty((B, S + 1), dtype=torch.int32, device=dev),
+               torch.empty((B, S), dtype=torch.int32, device=dev),
+               torch.empty((B,), dtype=torch.int32, device=dev))
+    is_sep, prefix, idx, count = out
+    arr = (ctypes.c_int32 * len(sep_ids))(*[int(x) for x in sep_ids])
+    _check("sep_build_index_from_ids", _lib.sep_build_index_from_ids(
+        _ptr(ids), B, S, ctypes.cast(arr, ctypes.c_void_p), len(sep_ids), _ptr(is_sep),
+        _ptr(prefix), _ptr(idx), _ptr(count), _stream(stream)))
+    return is_sep, prefix, idx, count
 
 
 def count_pairs(prefix: torch.Tensor, a: int, n: int, out=None, stream=None) -> torch.Tensor:

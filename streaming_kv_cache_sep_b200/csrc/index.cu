@@ -32,26 +32,29 @@ __global__ void k_flags_from_ids(const int32_t* __restrict__ ids, int64_t n_tok,
   }
 }
 
-// One CTA per (chunk of kChunk positions, sequence).  Warp w of the CTA
-// owns kPer x 32 consecutive positions, lane l the positions 32e + l
-// (e < kPer), so that flag reads and prefix writes are coalesced.  A warp
-// ranks its separators with ballots, one block-wide scan of the warp totals
-// gives the offsets.  With several chunks per sequence each CTA first counts
-// the separators before its chunk and in the whole sequence (read from L2);
-// no CTA waits on another.
+// One CTA per (chunk of positions, sequence); a chunk is kPer positions per
+// thread, and a CTA has as many warps as its chunk needs (at most 32).  Warp
+// w of the CTA owns kPer x 32 consecutive positions, lane l the positions
+// 32e + l (e < kPer), so that flag reads and prefix writes are coalesced.  A
+// warp ranks its separators with ballots, one block-wide scan of the warp
+// totals gives the offsets.  With several chunks per sequence each CTA first
+// counts the separators before its chunk and in the whole sequence (read
+// from L2); no CTA waits on another.  FROM_IDS: the flags are computed from
+// the token ids here (and written out), so one launch replaces the flag
+// kernel and this one.
 constexpr int kScanThreads = 1024;
 constexpr int kPer = 16;
-constexpr int kChunk = kScanThreads * kPer;
+constexpr int kChunkMax = kScanThreads * kPer;
 
-__device__ __forceinline__ int block_sum_1024(int v, int* red) {
+__device__ __forceinline__ int block_sum(int v, int* red) {
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5, l = threadIdx.x & 31, nw = blockDim.x >> 5;
   __syncthreads();
   if (l == 0) red[w] = v;
   __syncthreads();
   int s = 0;
   if (w == 0) {
-    s = red[l];
+    s = l < nw ? red[l] : 0;
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (l == 0) red[32] = s;
   }
@@ -59,42 +62,71 @@ __device__ __forceinline__ int block_sum_1024(int v, int* red) {
   return red[32];
 }
 
-__global__ void __launch_bounds__(kScanThreads) k_build_index(const uint8_t* __restrict__ is_sep,
-                                                              int S, int32_t* __restrict__ prefix,
-                                                              int32_t* __restrict__ idx,
-                                                              int32_t* __restrict__ count) {
+// Membership in the id set: the host pads id[n..32) with id[0], so all 32
+// fixed slots are compared (fixed indices keep the set in the parameter bank).
+__device__ __forceinline__ bool in_set(int32_t v, const SepIdSet& set) {
+  bool f = false;
+#pragma unroll
+  for (int k = 0; k < kMaxSepIds; ++k) f |= (v == set.id[k]);
+  return f;
+}
+
+template <bool FROM_IDS>
+__global__ void __launch_bounds__(kScanThreads) k_build_index(
+    const uint8_t* __restrict__ is_sep, const int32_t* __restrict__ ids, const SepIdSet set,
+    uint8_t* __restrict__ is_sep_out, int S, int32_t* __restrict__ prefix,
+    int32_t* __restrict__ idx, int32_t* __restrict__ count) {
   __shared__ int red[33];
   __shared__ int wsum[33];
-  asm volatile("griddepcontrol.wait;" ::: "memory");  // the flags' producer
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the flags' (or ids') producer
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int b = blockIdx.y;
-  const int64_t chunk0 = static_cast<int64_t>(blockIdx.x) * kChunk;
+  const int chunk0 = static_cast<int>(blockIdx.x * blockDim.x) * kPer;  // < S < 2^31
   const uint8_t* f = is_sep + static_cast<int64_t>(b) * S;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int32_t* tok = ids + static_cast<int64_t>(b) * S;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
   const uint32_t lt = (1u << lane) - 1u;
+  auto flag_at = [&](int p) -> bool { return FROM_IDS ? in_set(tok[p], set) : f[p] != 0; };
 
   // separators before the chunk, and in the whole sequence
   int before = 0, total = -1;
   if (gridDim.x > 1) {
     int tot = 0;
-    for (int64_t p = threadIdx.x; p < S; p += kScanThreads) {
-      const int v = f[p] != 0;
+    for (int p = threadIdx.x; p < S; p += blockDim.x) {
+      const int v = flag_at(p);
       tot += v;
       before += (p < chunk0) ? v : 0;
     }
-    before = block_sum_1024(before, red);
-    total = block_sum_1024(tot, red);
+    before = block_sum(before, red);
+    total = block_sum(tot, red);
   }
 
   // this warp's flags: bit e of `bits` is position w0 + 32e + lane
-  const int64_t w0 = chunk0 + static_cast<int64_t>(warp) * 32 * kPer;
+  const int w0 = chunk0 + warp * 32 * kPer;
   uint32_t bits = 0;
   int wtot = 0;
+  if (FROM_IDS) {
+    // all loads first: a flag store between them would keep the compiler
+    // from having the kPer loads in flight together
+    int32_t tv[kPer];
 #pragma unroll
-  for (int e = 0; e < kPer; ++e) {
-    const int64_t pos = w0 + 32 * e + lane;
-    const bool fl = pos < S && f[pos] != 0;
-    bits |= static_cast<uint32_t>(fl) << e;
+    for (int e = 0; e < kPer; ++e) {
+      const int pos = w0 + 32 * e + lane;
+      tv[e] = pos < S ? tok[pos] : 0;
+    }
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const int pos = w0 + 32 * e + lane;
+      const bool fl = pos < S && in_set(tv[e], set);
+      if (pos < S) is_sep_out[static_cast<int64_t>(b) * S + pos] = fl ? 1 : 0;
+      bits |= static_cast<uint32_t>(fl) << e;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+      const int pos = w0 + 32 * e + lane;
+      bits |= static_cast<uint32_t>(pos < S && f[pos] != 0) << e;
+    }
   }
 #pragma unroll
   for (int e = 0; e < kPer; ++e) wtot += __popc(__ballot_sync(0xffffffffu, (bits >> e) & 1u));
@@ -102,7 +134,7 @@ __global__ void __launch_bounds__(kScanThreads) k_build_index(const uint8_t* __r
   if (lane == 0) wsum[warp] = wtot;
   __syncthreads();
   if (warp == 0) {
-    const int x = wsum[lane];
+    const int x = lane < nwarps ? wsum[lane] : 0;
     int xi = x;
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, xi, o);
@@ -123,7 +155,7 @@ __global__ void __launch_bounds__(kScanThreads) k_build_index(const uint8_t* __r
   int run = before + wsum[warp];
 #pragma unroll
   for (int e = 0; e < kPer; ++e) {
-    const int64_t pos = w0 + 32 * e + lane;
+    const int pos = w0 + 32 * e + lane;
     const uint32_t bal = __ballot_sync(0xffffffffu, (bits >> e) & 1u);
     const int rank = run + __popc(bal & lt);
     if (pos < S) {
@@ -135,6 +167,13 @@ __global__ void __launch_bounds__(kScanThreads) k_build_index(const uint8_t* __r
     }
     run += __popc(bal);
   }
+}
+
+// Threads of a scan CTA: one chunk of S when it fits, whole warps.
+int scan_threads(int S) {
+  if (S > kChunkMax) return kScanThreads;
+  const int warps = (S + 32 * kPer - 1) / (32 * kPer);
+  return warps * 32;
 }
 
 // Closed form of one row's kept count: window [lo, i] + initial tokens left
@@ -187,9 +226,34 @@ extern "C" int sep_build_index(const uint8_t* is_sep, int B, int S, int32_t* pre
                                int32_t* count, void* stream) {
   if (B < 1 || S < 1 || B > 65535) return SEP_EINVAL;
   if (!is_sep || !prefix || !idx || !count) return SEP_ENULL;
-  dim3 grid((S + kChunk - 1) / kChunk, B);
-  if (sep::launch_pdl(k_build_index, grid, dim3(kScanThreads), 0, static_cast<cudaStream_t>(stream),
-                      is_sep, S, prefix, idx, count) != cudaSuccess)
+  const int threads = scan_threads(S);
+  const int chunk = threads * kPer;
+  SepIdSet none;
+  memset(&none, 0, sizeof none);
+  dim3 grid((S + chunk - 1) / chunk, B);
+  if (sep::launch_pdl(k_build_index<false>, grid, dim3(threads), 0,
+                      static_cast<cudaStream_t>(stream), is_sep, static_cast<const int32_t*>(nullptr),
+                      none, static_cast<uint8_t*>(nullptr), S, prefix, idx, count) != cudaSuccess)
+    return SEP_ECUDA;
+  return sep::launch_status();
+}
+
+extern "C" int sep_build_index_from_ids(const int32_t* ids, int B, int S, const int32_t* sep_ids,
+                                        int n_sep_ids, uint8_t* is_sep, int32_t* prefix,
+                                        int32_t* idx, int32_t* count, void* stream) {
+  if (B < 1 || S < 1 || B > 65535 || n_sep_ids < 1 || n_sep_ids > kMaxSepIds) return SEP_EINVAL;
+  if (!sep_ids) return SEP_ENULL;
+  if (!ids || !is_sep || !prefix || !idx || !count) return SEP_ENULL;
+  SepIdSet set;
+  memset(&set, 0, sizeof set);
+  set.n = n_sep_ids;
+  for (int k = 0; k < kMaxSepIds; ++k) set.id[k] = sep_ids[k < n_sep_ids ? k : 0];
+  const int threads = scan_threads(S);
+  const int chunk = threads * kPer;
+  dim3 grid((S + chunk - 1) / chunk, B);
+  if (sep::launch_pdl(k_build_index<true>, grid, dim3(threads), 0,
+                      static_cast<cudaStream_t>(stream), static_cast<const uint8_t*>(nullptr), ids,
+                      set, is_sep, S, prefix, idx, count) != cudaSuccess)
     return SEP_ECUDA;
   return sep::launch_status();
 }

@@ -75,6 +75,14 @@ def test_index_rejects_bad_arguments(sl):
     assert L.sep_flags_from_ids(FAKE, 10, ids, 0, FAKE, None) == -1
     assert L.sep_flags_from_ids(FAKE, -1, ids, 3, FAKE, None) == -1
     assert L.sep_flags_from_ids(None, 0, ids, 3, None, None) == 0  # empty is a no-op
+    F = FAKE
+    assert L.sep_build_index_from_ids(F, 0, 10, ids, 3, F, F, F, F, None) == -1
+    assert L.sep_build_index_from_ids(F, 1, 0, ids, 3, F, F, F, F, None) == -1
+    assert L.sep_build_index_from_ids(F, 1, 10, ids, 0, F, F, F, F, None) == -1
+    assert L.sep_build_index_from_ids(F, 1, 10, ids, 33, F, F, F, F, None) == -1
+    assert L.sep_build_index_from_ids(F, 1, 10, None, 3, F, F, F, F, None) == -6
+    assert L.sep_build_index_from_ids(None, 1, 10, ids, 3, F, F, F, F, None) == -6
+    assert L.sep_build_index_from_ids(F, 1, 10, ids, 3, F, F, None, F, None) == -6
 
 
 def test_cache_layout_and_validation(sl):

@@ -90,6 +90,34 @@ def test_build_index_bit_exact(sl, case):
     np.testing.assert_array_equal(count.cpu().numpy(), c0)
 
 
+@pytest.mark.parametrize("B,S,n_ids", [(8, 2048, 9), (1, 256, 9), (2, 16385, 3), (1, 40000, 32),
+                                        (3, 1, 1), (2, 777, 5)])
+def test_build_index_from_ids_bit_exact(sl, B, S, n_ids):
+    """One-launch flags + index from token ids against the oracle's two steps."""
+    g = np.random.default_rng(B * 100003 + S + n_ids)
+    sep_ids = [int(x) for x in g.choice(1000, size=n_ids, replace=False)]
+    ids = g.integers(0, 60, size=(B, S)).astype(np.int32)  # dense hits among ids < 60
+    ids[:, ::7] = sep_ids[-1]
+    flags, prefix, idx, count = sl.build_index_from_ids(_cuda(ids), sep_ids)
+    want_flags = oracle.flags_from_ids(ids, sep_ids)
+    p0, i0, c0 = oracle.build_index(want_flags)
+    np.testing.assert_array_equal(flags.cpu().numpy(), want_flags)
+    np.testing.assert_array_equal(prefix.cpu().numpy(), p0)
+    np.testing.assert_array_equal(idx.cpu().numpy(), i0)
+    np.testing.assert_array_equal(count.cpu().numpy(), c0)
+
+
+def test_build_index_from_ids_workload(sl):
+    name = "prefill_pythia160m_b8h12_s2048_d64_bf16"
+    inp = synth.prefill_inputs(synth.WORKLOADS[name], synth.WORKLOAD_SEED[name])
+    flags, prefix, idx, count = sl.build_index_from_ids(_cuda(inp["ids"]), list(inp["sep_ids"]))
+    p0, i0, c0 = oracle.build_index(inp["is_sep"])
+    np.testing.assert_array_equal(flags.cpu().numpy(), inp["is_sep"])
+    np.testing.assert_array_equal(prefix.cpu().numpy(), p0)
+    np.testing.assert_array_equal(idx.cpu().numpy(), i0)
+    np.testing.assert_array_equal(count.cpu().numpy(), c0)
+
+
 def test_flags_from_ids_bit_exact(sl):
     for name in ("prefill_tiny_b1h1_s256_d64_f32", "prefill_pythia160m_b8h12_s2048_d64_bf16"):
         cfg = synth.WORKLOADS[name]
