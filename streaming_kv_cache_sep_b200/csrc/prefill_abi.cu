@@ -6,7 +6,7 @@
 
 extern "C" size_t sep_attn_prefill_workspace(int B, int Hq, int Hkv, int S, int D, int dtype) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || D < 1) return 0;
-  if (dtype == SEP_BF16) return 256 + sep::prefill_tc_workspace(B, Hkv, S, D);
+  if (dtype == SEP_BF16) return sep::prefill_tc_workspace(B, Hkv, S, D);
   return 256;
 }
 
@@ -32,5 +32,5 @@ extern "C" int sep_attn_prefill(const void* q, const void* k, const void* v, int
                             static_cast<const float*>(v), prefix, idx, B, Hq, Hkv, S, D, a, n, sc,
                             static_cast<float*>(out), lse, st);
   return sep::prefill_tc(q, k, v, is_sep, prefix, idx, B, Hq, Hkv, S, D, a, n, sc, out, lse,
-                         static_cast<uint8_t*>(workspace) + 256, st);
+                         workspace, st);
 }

@@ -81,6 +81,8 @@ struct Bars {
   uint64_t s_full[2], p_full[2], o_full[2], o_empty[2];
   uint64_t s_free[2], pv_done[2];  // separate-P protocol: S read back / P*V done
   uint64_t drain;
+  uint64_t it_full[4], it_empty[4];  // work-item ring (dynamic scheduling)
+  int item_q[4];
   uint32_t tmem_base;
   int abort;
 };
@@ -95,6 +97,7 @@ struct Params {
   __nv_bfloat16* out;
   float* lse;
   int32_t* err;
+  int32_t* sched;  // next work item (zeroed by the gather kernel before each launch)
 };
 
 // Geometry of one work item, computed identically by every role.
@@ -181,6 +184,41 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   mbar_wait(bar, parity, &dummy, nullptr);
 }
 
+// Dynamic work distribution.  The producer thread takes item indices from a
+// global counter (the index order is heaviest first, so each CTA takes the
+// heaviest item left when it is ready for one) and publishes its k-th item
+// in slot k % 4 of a ring; the MMA issuers and the softmax warps take the
+// items from the ring in the same order.  An index >= n_items ends the loop;
+// -1 means the CTA is aborting.
+template <int NST>
+__device__ __forceinline__ int publish_item(Bars<NST>* bars, uint32_t k, const Params& p,
+                                            volatile int* abort) {
+  const uint32_t slot = k & 3u;
+  if (k >= 4 && !mbar_wait(&bars->it_empty[slot], ((k >> 2) - 1) & 1, abort, p.err)) return -1;
+  int item = atomicAdd(p.sched, 1);
+  if (item > p.n_items) item = p.n_items;
+  bars->item_q[slot] = item;
+  sep::mbar_arrive(&bars->it_full[slot]);  // release: the slot's value is visible to the takers
+  return item;
+}
+
+// whole_warp: all 32 lanes take the item and lane 0 frees the slot for them.
+template <int NST>
+__device__ __forceinline__ int take_item(Bars<NST>* bars, uint32_t k, const Params& p,
+                                         volatile int* abort, bool whole_warp) {
+  const uint32_t slot = k & 3u;
+  const bool got = mbar_wait(&bars->it_full[slot], (k >> 2) & 1, abort, p.err);
+  if (whole_warp ? !__all_sync(0xffffffffu, got) : !got) return -1;
+  const int item = *reinterpret_cast<volatile int*>(&bars->item_q[slot]);
+  if (whole_warp) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) sep::mbar_arrive(&bars->it_empty[slot]);
+  } else {
+    sep::mbar_arrive(&bars->it_empty[slot]);
+  }
+  return item;
+}
+
 // MMA issue for both tiles from one thread, P written over S (D = 128): per
 // block, tile A's P*V of the previous block then its S, then tile B's.
 template <int D>
@@ -226,7 +264,9 @@ __device__ __forceinline__ void mma_single_issuer(const Params& p, uint8_t* smem
     }
     sep::mma_commit(&bars->s_full[t]);
   };
-  for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
+  for (; ok; ++nitem) {
+    const int item = take_item<NST>(bars, nitem, p, abort, false);
+    if (item < 0 || item >= p.n_items) break;
     const Item it = make_item(p, item);
     if (!mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
     bool prev_a = false, prev_b = false;  // tile kept the previous block
@@ -302,6 +342,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       sep::mbar_init(&bars->pv_done[t], 1);
     }
     sep::mbar_init(&bars->drain, kIssuers);
+    for (int k = 0; k < 4; ++k) {
+      sep::mbar_init(&bars->it_full[k], 1);
+      sep::mbar_init(&bars->it_empty[k], kIssuers + 8);  // issuers + softmax warps
+    }
     bars->abort = 0;
     sep::mbar_fence_init();
   }
@@ -331,7 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s2 = 0; s2 < NST; ++s2) last_k[s2] = last_v[s2] = -1;
       int last_q = -1;
       bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
+      for (; ok; ++nitem) {
+        const int item = publish_item<NST>(bars, nitem, p, abort);
+        if (item < 0 || item >= p.n_items) break;
         const Item it = make_item(p, item);
         const int64_t kv_row0 = static_cast<int64_t>(it.b * p.Hkv + it.g) * p.S;
         if (nitem > 0 && !mbar_wait(&bars->q_empty, (nitem - 1) & 1, abort, p.err)) break;
@@ -444,7 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         sep::mma_commit(&bars->s_full[t]);
         return true;
       };
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
+      for (; ok; ++nitem) {
+        const int item = take_item<NST>(bars, nitem, p, abort, false);
+        if (item < 0 || item >= p.n_items) break;
         const Item it = make_item(p, item);
         if (!mbar_wait(&bars->q_full, nitem & 1, abort, p.err)) break;
         bool prev = false;  // this tile kept the previous block
@@ -514,7 +562,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
     bool ok = true;
-    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x, ++nitem) {
+    for (; ok; ++nitem) {
+      const int item = take_item<NST>(bars, nitem, p, abort, true);
+      if (item < 0 || item >= p.n_items) break;
       const Item it = make_item(p, item);
       // this tile's scalars (the rest of the item is not needed here)
       const int my_q0 = t ? it.q0[1] : it.q0[0];
@@ -833,15 +883,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 // followed by every separator at a position >= a into the compact buffers
 // Kc/Vc [B, Hkv, S, D]; rows from the end of that list up to 128 (at least)
 // and up to the next multiple of 128 are zero-filled, so whole 128-row tiles
-// read finite values.  One CTA copies 64 rows.
+// read finite values.  One CTA copies 64 rows.  The first thread also zeroes
+// the attention kernel's work-item counter (every earlier kernel on the
+// stream, the previous attention launch included, has completed here).
 template <int D>
 __global__ void __launch_bounds__(256) k_gather_sep_rows(
     const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
     const int32_t* __restrict__ prefix, const int32_t* __restrict__ idx, int Hkv, int S, int a,
-    __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, int32_t* err) {
+    __nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, int32_t* err,
+    int32_t* __restrict__ sched) {
   constexpr int CH = D * 2 / 16;  // 16-byte chunks per row
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the index's producer
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x == 0) *sched = 0;
   const int g = blockIdx.y, b = blockIdx.z;
   const int r0 = blockIdx.x * 64;
   const int32_t* pre = prefix + static_cast<int64_t>(b) * (S + 1);
@@ -912,7 +966,7 @@ int num_sms() {
 template <int D>
 int launch(const void* q, const void* k, const void* v, const uint8_t* is_sep,
            const int32_t* prefix, const int32_t* idx, int B, int Hq, int Hkv, int S, int a, int n,
-           float scale, void* out, float* lse, void* kc, void* vc, cudaStream_t st) {
+           float scale, void* out, float* lse, void* kc, void* vc, int32_t* sched, cudaStream_t st) {
   using C = Cfg<D>;
   static bool attr_set[64] = {false};
   int dev = 0;
@@ -936,7 +990,7 @@ int launch(const void* q, const void* k, const void* v, const uint8_t* is_sep,
   if (sep::launch_pdl(k_gather_sep_rows<D>, ggrid, dim3(256), 0, st,
                       static_cast<const __nv_bfloat16*>(k), static_cast<const __nv_bfloat16*>(v),
                       prefix, idx, Hkv, S, a, static_cast<__nv_bfloat16*>(kc),
-                      static_cast<__nv_bfloat16*>(vc), sep::device_error_word()) != cudaSuccess)
+                      static_cast<__nv_bfloat16*>(vc), sep::device_error_word(), sched) != cudaSuccess)
     return SEP_ECUDA;
 
   Params p;
@@ -964,6 +1018,7 @@ int launch(const void* q, const void* k, const void* v, const uint8_t* is_sep,
   p.out = static_cast<__nv_bfloat16*>(out);
   p.lse = lse;
   p.err = sep::device_error_word();
+  p.sched = sched;
   const int grid = p.n_items < num_sms() ? p.n_items : num_sms();
   if (sep::launch_pdl(k_prefill_tc<D>, dim3(grid), dim3(kThreads), C::ALLOC, st, mq, mk, mv, mkc,
                       mvc, mo, p) != cudaSuccess)
@@ -974,22 +1029,25 @@ int launch(const void* q, const void* k, const void* v, const uint8_t* is_sep,
 }  // namespace
 
 namespace sep {
+// Workspace: 256 bytes of head (the work-item counter) and the compact K and
+// V row lists.
 size_t prefill_tc_workspace(int B, int Hkv, int S, int D) {
-  return 2 * ((static_cast<size_t>(B) * Hkv * S * D * 2 + 255) / 256 * 256);
+  return 256 + 2 * ((static_cast<size_t>(B) * Hkv * S * D * 2 + 255) / 256 * 256);
 }
 
 int prefill_tc(const void* q, const void* k, const void* v, const uint8_t* is_sep,
                const int32_t* prefix, const int32_t* idx, int B, int Hq, int Hkv, int S, int D,
                int a, int n, float scale, void* out, float* lse, void* workspace, cudaStream_t st) {
   const size_t half = (static_cast<size_t>(B) * Hkv * S * D * 2 + 255) / 256 * 256;
-  void* kc = workspace;
-  void* vc = static_cast<uint8_t*>(workspace) + half;
+  int32_t* sched = static_cast<int32_t*>(workspace);
+  void* kc = static_cast<uint8_t*>(workspace) + 256;
+  void* vc = static_cast<uint8_t*>(kc) + half;
   if (D == 64)
     return launch<64>(q, k, v, is_sep, prefix, idx, B, Hq, Hkv, S, a, n, scale, out, lse, kc, vc,
-                      st);
+                      sched, st);
   if (D == 128)
     return launch<128>(q, k, v, is_sep, prefix, idx, B, Hq, Hkv, S, a, n, scale, out, lse, kc, vc,
-                       st);
+                       sched, st);
   return SEP_EDTYPE;
 }
 }  // namespace sep
