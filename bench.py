@@ -84,11 +84,11 @@ TRAFFIC = {
         bytes=161018624 + 101916928, per="launch", src=("backward.cu", "common.cuh"),
         sha1="ccc1d51920b8eb0ffa71d1c0b81985af9610007c"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
-        bytes=104788480 + 29667840, per="launch", src=("prefill_tc.cu", "common.cuh"),
-        sha1="0ccfa2f810f1862257e2228d4f7439111558f44b"),
+        bytes=104931328 + 30614528, per="launch", src=("prefill_tc.cu", "common.cuh"),
+        sha1="7c01b1b5569fa46bbbed9d0e03a0aa812f51443e"),
     "prefill_pythia160m_b8h12_s2048_d64_bf16": dict(
-        bytes=82165248 + 8908800, per="launch", src=("prefill_tc.cu", "common.cuh"),
-        sha1="0ccfa2f810f1862257e2228d4f7439111558f44b"),
+        bytes=82398208 + 8301312, per="launch", src=("prefill_tc.cu", "common.cuh"),
+        sha1="7c01b1b5569fa46bbbed9d0e03a0aa812f51443e"),
 }
 
 
