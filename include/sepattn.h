@@ -97,9 +97,10 @@ int sep_count_pairs(const int32_t* prefix, int B, int S, int a, int n, int64_t* 
 /* Prefill / training forward                                               */
 /* ---------------------------------------------------------------------- */
 
-/* Workspace bytes sep_attn_prefill needs for these sizes (bf16: room for the
- * compacted initial+separator K and V rows of every (b, kv head), i.e. two
- * buffers of k's size, plus 256 bytes; fp32: 256 bytes). */
+/* Workspace bytes sep_attn_prefill needs for these sizes (bf16: 256 bytes
+ * of head, which hold the attention kernel's work-item counter, then room
+ * for the compacted initial+separator K and V rows of every (b, kv head),
+ * i.e. two buffers of k's size; fp32: 256 bytes). */
 size_t sep_attn_prefill_workspace(int B, int Hq, int Hkv, int S, int D, int dtype);
 
 /* Sep-Attention over whole sequences:
