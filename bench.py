@@ -85,10 +85,10 @@ TRAFFIC = {
         sha1="ccc1d51920b8eb0ffa71d1c0b81985af9610007c"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
         bytes=104931328 + 30614528, per="launch", src=("prefill_tc.cu", "common.cuh"),
-        sha1="7c01b1b5569fa46bbbed9d0e03a0aa812f51443e"),
+        sha1="49dc56e530bf1481bf356ca09d0d136ab3caf701"),
     "prefill_pythia160m_b8h12_s2048_d64_bf16": dict(
         bytes=82398208 + 8301312, per="launch", src=("prefill_tc.cu", "common.cuh"),
-        sha1="7c01b1b5569fa46bbbed9d0e03a0aa812f51443e"),
+        sha1="49dc56e530bf1481bf356ca09d0d136ab3caf701"),
 }
 
 

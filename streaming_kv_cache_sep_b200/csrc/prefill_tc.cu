@@ -22,8 +22,10 @@
 //   * otherwise: rows [q0, q0+128) and [q0+128, q0+256) of one head -- the
 //     stream is the union (the larger gathered prefix and the window range
 //     from the first tile's lo); per-tile masks keep each tile's own set.
-// The kernel is persistent (one CTA per SM, items heaviest first, strided
-// over the grid).  Warps 0-3 and 4-7 are the softmax warpgroups of tiles A
+// The kernel is persistent (one CTA per SM); items are numbered heaviest
+// first and handed out dynamically (a global counter read by the producer,
+// passed to the other roles through a shared-memory ring, see publish_item).
+// Warps 0-3 and 4-7 are the softmax warpgroups of tiles A
 // and B (thread = query row = TMEM lane), warp 8 issues TMA loads, warps 9
 // and 10 issue the tcgen05.mma of tiles A and B (warp 9 owns TMEM).  TMEM:
 // S_A | S_B | O_A | O_B, and for D = 64 also P_A | P_B, so that S of the next
