@@ -40,7 +40,9 @@ import torch  # noqa: E402
 
 import synth  # noqa: E402
 
-DEFAULT_WORKLOAD = "prefill_pythia160m_b8h12_s2048_d64_bf16"
+# The default line is the largest single-GPU configuration: the 131,072-token
+# long-context prefill (B1, 32 query / 8 kv heads, D128, a4, n1024).
+DEFAULT_WORKLOAD = "prefill_long_b1_s131072_d128_bf16"
 PREFILL_METRIC = "Sep-Attn prefill TFLOP/s on kept pairs"
 DECODE_METRIC = "Sep-Attn decode tokens/s over the four-block SepCache"
 INGEST_METRIC = "SepCache prompt ingestion tokens/s"

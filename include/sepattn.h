@@ -70,7 +70,11 @@ int sep_flags_from_ids(const int32_t* ids, int64_t n_tok, const int32_t* sep_ids
                        uint8_t* is_sep, void* stream);
 
 /* Per-sequence prefix-scan compaction of the separator flags (the
- * separator index lists used to gather separator rows).
+ * separator index lists used to gather separator rows).  The flags are the
+ * separator columns of the Sep-Attention mask ("HKUDS047: SepLLM ..." study,
+ * section "SepAttention": build_prefill_mask marks every column whose token
+ * is a separator; jieyibu.net explainer, section 1.2), so these lists name
+ * exactly the keys that every later query keeps beyond its window.
  *   prefix [B, S+1]: prefix[b][j] = number of separators among positions < j
  *   idx    [B, S]  : positions of the separators of sequence b in increasing
  *                    order, then -1 up to S
@@ -103,7 +107,11 @@ int sep_count_pairs(const int32_t* prefix, int B, int S, int a, int n, int64_t* 
  * i.e. two buffers of k's size; fp32: 256 bytes). */
 size_t sep_attn_prefill_workspace(int B, int Hq, int Hkv, int S, int D, int dtype);
 
-/* Sep-Attention over whole sequences:
+/* Sep-Attention over whole sequences ("HKUDS047: SepLLM ..." study, section
+ * "SepAttention": build_prefill_mask = (separator columns | initial columns |
+ * local triangular window) AND the causal lower triangle; jieyibu.net
+ * explainer, section 1.2: scores outside the mask are -inf before the
+ * softmax):
  *   out[b,h,i,:] = sum_{j in K_i} softmax_j(scale * q_i . k_j) v_j,
  *   K_i = { j <= i : j < a or is_sep[b,j] or i - j < n },
  *   lse[b,h,i]  = ln sum_{j in K_i} exp(scale * q_i . k_j).
@@ -167,7 +175,12 @@ typedef struct {
 #define SEP_CACHE_UNBOUNDED_SEPS 2  /* separators are never evicted: s is the block's
                                        capacity, and a flush that needs more sets
                                        SEP_CACHE_ESEPS in the status word (the newest s
-                                       stay) */
+                                       stay).  The page's list without a maximum simply
+                                       grows; a device cache has a fixed capacity, so a
+                                       caller gets those semantics by sizing s for the
+                                       whole stream (at least its separator count), and
+                                       this bit then only reports a cache sized too
+                                       small */
 #define SEP_CACHE_TOTAL_TRIGGER 4   /* flush when the whole cache holds more than
                                        a+s+past+w tokens (the past window may then hold
                                        up to past+s); the same as the default once the
@@ -244,9 +257,13 @@ int sepcache_init(const sepcache* cache, void* stream);
 int sepcache_append(const sepcache* cache, int layer, const void* k_new, const void* v_new,
                     const uint8_t* is_sep_new, void* stream);
 
-/* Apply this step's flush to `layer`: the separators of the past window join
- * the separator cache, which keeps its newest s entries, the past window
- * empties and the local window slides down.  The surviving rows (found by an
+/* Apply this step's flush to `layer` ("HKUDS047: SepLLM ..." study, section
+ * "KV Cache Manager": the compression step; xugj520 article, section 3.3
+ * table: the past window keeps only its separators, which join the
+ * separator cache, and that cache evicts its oldest entries beyond s): the
+ * separators of the past window join the separator cache, which keeps its
+ * newest s entries, the past window empties and the local window slides
+ * down.  The surviving rows (found by an
  * order-preserving warp-ballot stream compaction at layer 0's append) are
  * copied, in order, into the sequence's other K/V buffer.  A no-op on steps
  * without a flush. */
@@ -283,7 +300,11 @@ int sep_attn_decode_step(const sepcache* cache, int layer, const void* q, const 
 /* Workspace bytes sep_attn_decode needs (split-K partials and counters). */
 size_t sep_attn_decode_workspace(const sepcache* cache, int Hq);
 
-/* Attention of the newest token over the retained rows of `layer`:
+/* Attention of the newest token over the retained rows of `layer` (the
+ * streaming decode over the four cache blocks: xugj520 article, section 3.3
+ * table; jieyibu.net explainer, section 1.3: the query attends over the
+ * initial, separator, past-window and local-window rows only; the softmax is
+ * that of sep_attn_prefill restricted to those rows):
  * q [B, Hq, D] (cache dtype), out [B, Hq, D] (cache dtype), lse [B, Hq]
  * fp32 (may be NULL).  Hq % Hkv == 0 and Hq / Hkv <= 8.  workspace: at least
  * sep_attn_decode_workspace() bytes, zero-filled before its first use (the
@@ -301,13 +322,17 @@ int sep_attn_decode(const sepcache* cache, int layer, const void* q, int Hq, flo
  * sep_attn_decode, without the workspace: the split-K partials and tickets
  * live in a fixed scratch array inside the library (about 4.1 MiB, held by
  * every GPU that loads the library until the process exits).
- * Limits: B * Hq * ceil((a+s+past+w+1) / 64) <= 8192 and B * Hkv <= 4096;
- * larger sizes return SEP_ETOOBIG before anything is enqueued.
- * The first call on a device looks up the array's device address (with
- * that device current); make that first call before any stream capture.
- * Each call clears the tickets on `stream` before its kernel and calls no
- * allocating routine.  All calls share the array, so calls that overlap on
- * the GPU (other streams, other threads) race on it. */
+ * Only an fp32 cache with more than 8 splits of 64 rows (a+s+past+w+1 >
+ * 512) merges its splits through that array; bf16 caches and smaller fp32
+ * caches merge inside a thread-block cluster and do not use it.  For the
+ * fp32 case the limits are B * Hq * ceil((a+s+past+w+1) / 64) <= 8192 and
+ * B * Hkv <= 4096; larger sizes return SEP_ETOOBIG before anything is
+ * enqueued.  In that case the first call on a device looks up the array's
+ * device address (with that device current); make that first call before
+ * any stream capture, and do not use this entry point on a device after
+ * cudaDeviceReset.  Each such call clears the tickets on `stream` before
+ * its kernel.  No call allocates.  All calls share the array, so calls that
+ * overlap on the GPU (other streams, other threads) race on it. */
 int sep_attn_decode_noalloc(const sepcache* cache, int layer, const void* q, int Hq, float scale,
                             void* out, float* lse, void* stream);
 

@@ -21,6 +21,8 @@
 #include <cooperative_groups.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -686,9 +688,20 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   // completes long before the first remote store (after the chunk loop):
   // every CTA's barriers are initialised by then
   sep::cluster_arrive_relaxed();
-  // With p.early the cache metadata and this layer's rows were last written
-  // at least two launches back, so they are read before waiting on the
-  // previous grid; q, k_new, v_new and every store still come after the wait.
+  // With p.early (fused step, layer >= 1) the cache metadata (counts, cur,
+  // plan) and this layer's rows are read before waiting on the previous
+  // grid; q, k_new, v_new and every store still come after the wait.  This
+  // is safe because of how the step is ordered, not because of distance in
+  // the stream: the step's bookkeeping kernel (k_cache_advance, launched
+  // with the layer-0 call) is a plain launch WITHOUT programmatic stream
+  // serialization, so it starts only after every kernel of the previous step
+  // has completed (each waits on its predecessor before it ends), and the
+  // layer-0 decode, which does wait, starts only after it.  A grid of this
+  // step at layer >= 1 can start only once layer 0 has started, so the
+  // metadata it reads is this step's, and the rows of this layer were last
+  // written by this layer's launch of the previous step, which has ended.
+  // If the bookkeeping launch ever became a programmatic launch, these reads
+  // would race with the previous step's layers.
   if (!p.early) asm volatile("griddepcontrol.wait;" ::: "memory");
   const int32_t* pl = FUSED ? p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr) : nullptr;
   int len;
@@ -1298,6 +1311,13 @@ extern "C" int sep_attn_decode_step(const sepcache* c, int layer, const void* q,
 // fixed scratch array inside the library instead.  Every GPU that loads the
 // library holds the array (about 4.1 MiB) until the process exits; every
 // call shares it, so calls that overlap on the GPU race on it.
+//
+// Only one kernel form reads or writes the array: the exact fp32 decode of a
+// cache with more than kMaxClusterSplits splits of 64 rows, whose splits
+// merge through memory with an atomic ticket.  The bf16 kernel and the fp32
+// kernel with at most kMaxClusterSplits splits merge inside a thread-block
+// cluster and never touch it, so the size limits and the ticket clear apply
+// to the first form only.
 namespace {
 
 constexpr int kNoAllocMaxPartials = 8192;  // B * Hq * splits, splits = ceil(cap / 64)
@@ -1306,11 +1326,23 @@ constexpr size_t kNoAllocMlBytes = static_cast<size_t>(kNoAllocMaxPartials) * 2 
 constexpr size_t kNoAllocOBytes = static_cast<size_t>(kNoAllocMaxPartials) * 128 * 4;
 constexpr size_t kNoAllocTicketBytes = static_cast<size_t>(kNoAllocMaxTickets) * 4;
 constexpr size_t kNoAllocBytes = kNoAllocMlBytes + kNoAllocOBytes + kNoAllocTicketBytes;
-
-__device__ __align__(256) uint8_t g_decode_scratch[kNoAllocBytes];
-
 constexpr int kNoAllocMaxDevices = 64;
-uint8_t* g_decode_scratch_addr[kNoAllocMaxDevices];  // device address, per device
+
+}  // namespace
+
+// The scratch itself.  In host code this name is only a stand-in for the
+// array, not its device address: the address is looked up per device.
+static __device__ __align__(256) uint8_t g_decode_scratch[kNoAllocBytes];
+
+namespace {
+
+// Device address of the scratch array, per device.  Set once per device
+// (the first call on it, with that device current); a race between two
+// host threads making that first call stores the same value twice, and the
+// atomic makes that well defined.  The address is not refreshed after
+// cudaDeviceReset: a process that resets a device must not use this entry
+// point on it afterwards.
+std::atomic<uint8_t*> g_decode_scratch_addr[kNoAllocMaxDevices];
 
 }  // namespace
 
@@ -1325,25 +1357,34 @@ extern "C" int sep_attn_decode_noalloc(const sepcache* c, int layer, const void*
   if (!q || !out) return SEP_ENULL;
   if (!sep::aligned16(q) || !sep::aligned16(out)) return SEP_EALIGN;
   const int nsplit = (c->cap + ROWS - 1) / ROWS;
-  if (static_cast<int64_t>(c->B) * Hq * nsplit > kNoAllocMaxPartials ||
-      static_cast<int64_t>(c->B) * c->Hkv > kNoAllocMaxTickets)
-    return SEP_ETOOBIG;
-  // set-up, once per device with that device current: the device address of
-  // the scratch array (the host-side symbol itself is not a device address)
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) return SEP_ECUDA;
-  if (!g_decode_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) return SEP_ECUDA;
-    g_decode_scratch_addr[dev] = static_cast<uint8_t*>(p);
-  }
-  uint8_t* scratch = g_decode_scratch_addr[dev];
+  // the only kernel form that merges through the scratch array
+  const bool uses_scratch = c->dtype == SEP_F32 && nsplit > kMaxClusterSplits;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int32_t* tickets = reinterpret_cast<int32_t*>(scratch + kNoAllocMlBytes + kNoAllocOBytes);
-  // the tickets must start at zero (the array keeps the previous call's contents)
-  if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(c->B) * c->Hkv * 4, st) != cudaSuccess)
-    return SEP_ECUDA;
   DecodeParams p = {};
+  if (uses_scratch) {
+    if (static_cast<int64_t>(c->B) * Hq * nsplit > kNoAllocMaxPartials ||
+        static_cast<int64_t>(c->B) * c->Hkv > kNoAllocMaxTickets)
+      return SEP_ETOOBIG;
+    // set-up, once per device with that device current: the device address
+    // of the scratch array (the host-side symbol is not a device address)
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices)
+      return SEP_ECUDA;
+    uint8_t* scratch = g_decode_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!scratch) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_decode_scratch) != cudaSuccess || !ptr) return SEP_ECUDA;
+      scratch = static_cast<uint8_t*>(ptr);
+      g_decode_scratch_addr[dev].store(scratch, std::memory_order_release);
+    }
+    int32_t* tickets = reinterpret_cast<int32_t*>(scratch + kNoAllocMlBytes + kNoAllocOBytes);
+    // the tickets must start at zero (the array keeps the previous call's contents)
+    if (cudaMemsetAsync(tickets, 0, static_cast<size_t>(c->B) * c->Hkv * 4, st) != cudaSuccess)
+      return SEP_ECUDA;
+    p.part_ml = reinterpret_cast<float*>(scratch);
+    p.part_o = reinterpret_cast<float*>(scratch + kNoAllocMlBytes);
+    p.ticket = tickets;
+  }
   p.q = q;
   p.kc = c->k;
   p.vc = c->v;
@@ -1355,9 +1396,6 @@ extern "C" int sep_attn_decode_noalloc(const sepcache* c, int layer, const void*
   p.layers = c->layers;
   p.out = out;
   p.lse = lse;
-  p.part_ml = reinterpret_cast<float*>(scratch);
-  p.part_o = reinterpret_cast<float*>(scratch + kNoAllocMlBytes);
-  p.ticket = tickets;
   p.err = sep::device_error_word();
   p.layer = layer;
   p.B = c->B;

@@ -22,5 +22,5 @@ bool cache_valid(const sepcache* c);
 constexpr int kCachePlanHdr = 8;  // plan header words per sequence (see sepcache.cu)
 // Tensor map of a bf16 [rows, D] row-major array (D = 64 or 128): tiles of
 // 64 columns x box_rows rows, 128-byte swizzled.  Defined in prefill_tc.cu.
-bool make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int D, int box_rows);  // plan header words per sequence (see sepcache.cu)
+bool make_rows_map(CUtensorMap* m, const void* base, int64_t rows, int D, int box_rows);
 }  // namespace sep

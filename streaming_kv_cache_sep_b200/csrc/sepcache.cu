@@ -500,6 +500,10 @@ extern "C" int sepcache_init(const sepcache* c, void* stream) {
 
 namespace sep {
 int cache_advance(const sepcache* c, const uint8_t* is_sep_new, cudaStream_t st) {
+  // A plain launch, and it must stay one (no programmatic stream
+  // serialization): it starts only after every kernel of the previous step
+  // has completed, which is what lets the fused decode of layers >= 1 read
+  // the cache metadata and its layer's rows before its grid-dependency wait.
   k_cache_advance<<<c->B, 32, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step, c->status,
                                         c->cur, is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
                                         c->cfg.past, c->cfg.w, c->cfg.mode);
@@ -516,6 +520,7 @@ extern "C" int sepcache_append(const sepcache* c, int layer, const void* k_new, 
   if (!sep::aligned16(k_new) || !sep::aligned16(v_new)) return SEP_EALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (layer == 0) {
+    // a plain launch (no programmatic serialization), as in cache_advance
     k_cache_advance<<<c->B, 32, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step, c->status,
                                           c->cur, is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
                                           c->cfg.past, c->cfg.w, c->cfg.mode);

@@ -77,6 +77,11 @@ WORKLOADS = {
     "backward_llama3_8b_b1_s2048_d128_bf16": dict(
         kind="backward", B=1, Hq=32, Hkv=8, S=2048, D=128, dtype="bf16", a=4, n=256,
         p_sep=0.1, ids=None, qkv_std=1.0),
+    # The long-context prefill on 32k tokens (same flags recipe and window):
+    # the size a full counter capture of the D128 prefill kernel takes
+    "prefill_long_b1_s32768_d128_bf16": dict(
+        kind="prefill", B=1, Hq=32, Hkv=8, S=32768, D=128, dtype="bf16", a=4, n=1024,
+        p_single=0.05, p_run_start=0.05 / 3.0, run_len=3, ids=None, qkv_std=1.0),
 }
 
 # Base seed per workload (1000 + index in the list above); parity tests add
