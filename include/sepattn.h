@@ -190,19 +190,17 @@ typedef struct {
  * buffer laid out by sepcache_carve().  Rows of each (layer, b, kv head)
  * are stored in increasing position order: initial | separator | past |
  * local, cap = c + 1 rows (one spare row holds the newest token between
- * sepcache_append and sepcache_compact).  K/V rows live in two buffers per
- * sequence; a flush copies the surviving rows into the other buffer, which
- * then becomes current (cur[b]). */
+ * sepcache_append and sepcache_compact).  A flush compacts the surviving
+ * rows in place (each moves to a row at or below its own, in order). */
 typedef struct {
-  void* k;           /* [2][layers][B][Hkv][cap][D] dtype */
-  void* v;           /* [2][layers][B][Hkv][cap][D] dtype */
+  void* k;           /* [layers][B][Hkv][cap][D] dtype */
+  void* v;           /* [layers][B][Hkv][cap][D] dtype */
   int32_t* pos;      /* [B][cap]  token position of each row, -1 when empty */
   uint8_t* flag;     /* [B][cap]  separator flag of each row */
   int32_t* counts;   /* [B][4]    rows in blocks I, S, P, L */
   int32_t* plan;     /* [B][cap+8] this step's slot / flush / buffers / move list */
   int64_t* step;     /* [B]       tokens appended so far */
   int32_t* status;   /* [1]       0, or SEP_CACHE_E* bits set by a kernel */
-  int32_t* cur;      /* [B]       current K/V buffer (0 or 1) of each sequence */
   float* rope;       /* [rope_rows][D/2][2] cos, sin of slot r at frequency i (fp32) */
   int32_t layers, B, Hkv, D, dtype, cap;
   sep_cache_cfg cfg;
@@ -264,9 +262,9 @@ int sepcache_append(const sepcache* cache, int layer, const void* k_new, const v
  * separators of the past window join the separator cache, which keeps its
  * newest s entries, the past window empties and the local window slides
  * down.  The surviving rows (found by an
- * order-preserving warp-ballot stream compaction at layer 0's append) are
- * copied, in order, into the sequence's other K/V buffer.  A no-op on steps
- * without a flush. */
+ * order-preserving warp-ballot stream compaction at layer 0's append) move
+ * in place, in ascending order, each to a row at or below its own.  A no-op
+ * on steps without a flush. */
 int sepcache_compact(const sepcache* cache, int layer, void* stream);
 
 /* Prompt ingestion (bulk append): put the T tokens of a prompt into an EMPTY
@@ -288,10 +286,13 @@ int sepcache_ingest(const sepcache* cache, int layer, const void* k, const void*
 /* One whole decode step of `layer` in a single launch per layer (plus, at
  * layer 0, the bookkeeping launch): the same result as sepcache_append(layer,
  * k_new, v_new, is_sep_new) -> sepcache_compact(layer) -> sep_attn_decode(
- * layer, q, ...).  Each decode CTA writes the new token's row and, on a
- * flush step, copies its share of the surviving rows into the other buffer
- * while it loads them.  Same arguments as those calls; is_sep_new is read
- * at layer 0 only.  Layers are stepped in order 0..layers-1 each token. */
+ * layer, q, ...).  Each decode CTA writes the new token's row; on a flush
+ * step the CTAs of a (sequence, kv head) load the surviving rows from their
+ * old places and compact them in place (the first CTA of the pair while it
+ * loads its share, the second, whose destinations may be the first one's
+ * sources, once the first has loaded everything).  Same arguments as those
+ * calls; is_sep_new is read at layer 0 only.  Layers are stepped in order
+ * 0..layers-1 each token. */
 int sep_attn_decode_step(const sepcache* cache, int layer, const void* q, const void* k_new,
                          const void* v_new, const uint8_t* is_sep_new, int Hq, float scale,
                          void* out, float* lse, void* workspace, size_t workspace_bytes,

@@ -55,8 +55,7 @@ CACHE_EOVERFLOW, CACHE_ESTATE, CACHE_ESEPS = 1, 2, 4  # cache status bits
 class _SepCacheC(ctypes.Structure):
     _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("pos", ctypes.c_void_p),
                 ("flag", ctypes.c_void_p), ("counts", ctypes.c_void_p), ("plan", ctypes.c_void_p),
-                ("step", ctypes.c_void_p), ("status", ctypes.c_void_p), ("cur", ctypes.c_void_p),
-                ("rope", ctypes.c_void_p), ("layers", ctypes.c_int32),
+                ("step", ctypes.c_void_p), ("status", ctypes.c_void_p), ("rope", ctypes.c_void_p), ("layers", ctypes.c_int32),
                 ("B", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("D", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("cap", ctypes.c_int32), ("cfg", SepCacheCfg),
                 ("rope_theta", ctypes.c_float), ("rope_rows", ctypes.c_int32)]
@@ -331,19 +330,14 @@ class SepCache:
             n *= d
         return self.buffer[off: off + n * esz].view(dtype).view(*shape)
 
-    # device views of the cache state; K/V have two buffers per sequence and
-    # cur[b] names the current one
+    # device views of the cache state
     @property
     def k(self):
-        return self._view(self.c.k, (2, self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
+        return self._view(self.c.k, (self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
 
     @property
     def v(self):
-        return self._view(self.c.v, (2, self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
-
-    @property
-    def cur(self):
-        return self._view(self.c.cur, (self.B,), torch.int32)
+        return self._view(self.c.v, (self.layers, self.B, self.Hkv, self.cap, self.D), self.dtype)
 
     @property
     def pos(self):

@@ -430,7 +430,9 @@ __global__ void __launch_bounds__(kThreads, D == 64 ? 3 : 2) k_sep_bwd(const Bwd
 constexpr int TBK = 128;  // keys per block (TMEM lanes of the key-centric kernel)
 constexpr int TBQ = 128;  // queries per tile
 constexpr int kTcThreads = 288;  // warps 0-7: softmax, loads, readout; warp 8: TMEM and MMA issue
-constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384, kColDQ = 256;
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDQ = 256;
+template <int D>
+constexpr uint32_t col_dk() { return kColDV + D; }  // dK after the D columns of dV
 constexpr int kT128 = 128 * 128;  // one 128-row x 64-column swizzled tile
 constexpr int kTcChunkTiles = 4;  // query tiles per item of global keys
 
@@ -462,21 +464,25 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
 __host__ __device__ constexpr uint32_t idesc_mn(int M, int N, bool a_mn, bool b_mn) {
   return sep::idesc_bf16_f32(M, N, b_mn) | ((a_mn ? 1u : 0u) << 15);
 }
-// Rows [0, 128) of a [rows, 128] bf16 tensor into a swizzled 128-row tile
-// pair, one 16-byte chunk per copy; row_of(r) < 0 gives a zero row.
-template <typename RowOf>
-__device__ __forceinline__ void load_rows128(uint32_t dst, const __nv_bfloat16* src, RowOf row_of,
-                                             int tid, int nthreads) {
-  for (int e = tid; e < 128 * 16; e += nthreads) {
-    const int r = e >> 4, c = e & 15;
+// Rows [0, 128) of a [rows, D] bf16 tensor into D/64 swizzled 128-row
+// tiles, one 16-byte chunk per copy; row_of(r) < 0 gives a zero row.
+template <int D, typename RowOf>
+__device__ __forceinline__ void load_rows(uint32_t dst, const __nv_bfloat16* src, RowOf row_of,
+                                          int tid, int nthreads) {
+  constexpr int CH = D / 8;  // 16-byte chunks per row
+  for (int e = tid; e < 128 * CH; e += nthreads) {
+    const int r = e / CH, c = e % CH;
     const int64_t row = row_of(r);
-    cp_async16(dst + swz128(r, 8 * c), src + (row < 0 ? 0 : row) * 128 + 8 * c, row < 0 ? 0u : 16u);
+    cp_async16(dst + swz128(r, 8 * c), src + (row < 0 ? 0 : row) * D + 8 * c, row < 0 ? 0u : 16u);
   }
 }
 
+// NB = D/64 tiles of 128 rows x 64 columns per 128-row tensor
+template <int D>
 struct KvSmem {
-  static constexpr int K = 0, V = 2 * kT128, Q = 4 * kT128, DO = 8 * kT128;  // Q, dO: [2] x 2 tiles
-  static constexpr int LSE = 12 * kT128;  // [2][128] fp32: -lse (log2 domain)
+  static constexpr int NB = D / 64;
+  static constexpr int K = 0, V = NB * kT128, Q = 2 * NB * kT128, DO = 4 * NB * kT128;  // Q, dO: [2] x NB tiles
+  static constexpr int LSE = 6 * NB * kT128;  // [2][128] fp32: -lse (log2 domain)
   static constexpr int DEL = LSE + 1024;  // [2][128] fp32
   static constexpr int POS = DEL + 1024;  // [128] int32
   static constexpr int USE = POS + 512;   // [128] int32
@@ -489,10 +495,13 @@ struct TcBars {
   int abort;
 };
 
+template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_sep_bwd_tc_kv(const BwdParams p, const __grid_constant__ CUtensorMap map_q,
                     const __grid_constant__ CUtensorMap map_do) {
-  constexpr int D = 128;
+  using KvSmem = ::KvSmem<D>;
+  constexpr int NB = D / 64;
+  constexpr uint32_t kColDK = col_dk<D>();
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* const smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -578,8 +587,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int lq = warp & 3, ch = warp >> 2;
     const int r = 32 * lq + lane;  // key row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * lq) << 16;
-    load_rows128(sb_ + KvSmem::K, p.k, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
-    load_rows128(sb_ + KvSmem::V, p.v, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
+    load_rows<D>(sb_ + KvSmem::K, p.k, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
+    load_rows<D>(sb_ + KvSmem::V, p.v, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
     cp_async_commit();
     // lse (negated, log2 domain) and delta of visit v's queries: thread
     // tid < 128 loads its query's pair (into registers one visit ahead)
@@ -660,16 +669,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     if (ok && nvisit > 0 && sep::mbar_wait(&bars.m_full, (nvisit - 1) & 1, abort, p.err) && !*abort) {
       sep::tc_fence_after();
-      // dK and dV of this key row, columns [64 ch, +64): every lane loads
-      // (warp-wide), rows with a key store
+      // dK and dV of this key row, columns [D/2 ch, +D/2): every lane
+      // loads (warp-wide), rows with a key store
       const bool mine = jp >= 0 && use;
-      float* dkp = p.dk_acc + (kvrow0 + (mine ? jp : 0)) * D + 64 * ch;
-      float* dvp = p.dv_acc + (kvrow0 + (mine ? jp : 0)) * D + 64 * ch;
+      float* dkp = p.dk_acc + (kvrow0 + (mine ? jp : 0)) * D + (D / 2) * ch;
+      float* dvp = p.dv_acc + (kvrow0 + (mine ? jp : 0)) * D + (D / 2) * ch;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t kv[32], vv[32];
-        sep::tmem_ld32(tmem + lane_base + kColDK + 64 * ch + 32 * c, kv);
-        sep::tmem_ld32(tmem + lane_base + kColDV + 64 * ch + 32 * c, vv);
+        sep::tmem_ld32(tmem + lane_base + kColDK + (D / 2) * ch + 32 * c, kv);
+        sep::tmem_ld32(tmem + lane_base + kColDV + (D / 2) * ch + 32 * c, vv);
         sep::tmem_wait_ld_r32(kv);
         sep::tmem_wait_ld_r32(vv);
         if (mine) {
@@ -701,11 +710,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int h = g * G + v / ntile, t = t0 + v % ntile;
         const int32_t row = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hq + h) * S + t * TBQ);
         const int buf = v & 1;
-        sep::mbar_arrive_expect_tx(&bars.tile[buf], 4 * kT128);
+        sep::mbar_arrive_expect_tx(&bars.tile[buf], 2 * NB * kT128);
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          sep::tma_load_2d(smem + KvSmem::Q + buf * 2 * kT128 + c * kT128, &map_q, 64 * c, row, &bars.tile[buf]);
-          sep::tma_load_2d(smem + KvSmem::DO + buf * 2 * kT128 + c * kT128, &map_do, 64 * c, row, &bars.tile[buf]);
+        for (int c = 0; c < NB; ++c) {
+          sep::tma_load_2d(smem + KvSmem::Q + buf * NB * kT128 + c * kT128, &map_q, 64 * c, row, &bars.tile[buf]);
+          sep::tma_load_2d(smem + KvSmem::DO + buf * NB * kT128 + c * kT128, &map_do, 64 * c, row, &bars.tile[buf]);
         }
       };
       if (nvisit > 0) load_tiles(0);
@@ -714,7 +723,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int buf = v & 1;
         if (!sep::mbar_wait(&bars.tile[buf], (v >> 1) & 1, abort, p.err)) break;
         sep::tc_fence_after();
-        const uint32_t qa = sb_ + KvSmem::Q + buf * 2 * kT128, oa = sb_ + KvSmem::DO + buf * 2 * kT128;
+        const uint32_t qa = sb_ + KvSmem::Q + buf * NB * kT128, oa = sb_ + KvSmem::DO + buf * NB * kT128;
         const uint64_t dQ = sep::smem_desc_sw128(qa, 16), dO = sep::smem_desc_sw128(oa, 16);
         const uint64_t dQmn = sep::smem_desc_sw128(qa, kT128), dOmn = sep::smem_desc_sw128(oa, kT128);
 #pragma unroll
@@ -753,17 +762,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
+template <int D>
 struct QSmem {
-  static constexpr int Q = 0, DO = 2 * kT128;
-  static constexpr int K = 4 * kT128, V = 6 * kT128;  // [2] buffers, 4 tiles apart
-  static constexpr int POS = 12 * kT128;  // [2][128] int32 key positions
+  static constexpr int NB = D / 64;
+  static constexpr int Q = 0, DO = NB * kT128;
+  static constexpr int K = 2 * NB * kT128, V = 3 * NB * kT128;  // [2] buffers, 2 NB tiles apart
+  static constexpr int POS = 6 * NB * kT128;  // [2][128] int32 key positions
   static constexpr int GLB = POS + 1024;  // [2][128] int32: key kept by every later query
   static constexpr int BYTES = GLB + 1024 + 1024;
 };
 
+template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams p,
                                                                 __nv_bfloat16* __restrict__ dq) {
-  constexpr int D = 128;
+  using QSmem = ::QSmem<D>;
+  constexpr int NB = D / 64;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* const smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -819,8 +832,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams 
     const float nlse2 = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
     const float dl = i < S ? p.delta[qrow0 + i] : 0.f;
     auto rowq = [&](int rr) -> int64_t { return i0 + rr < S ? qrow0 + i0 + rr : -1; };
-    load_rows128(sb_ + QSmem::Q, p.q, rowq, tid, 256);
-    load_rows128(sb_ + QSmem::DO, p.dout, rowq, tid, 256);
+    load_rows<D>(sb_ + QSmem::Q, p.q, rowq, tid, 256);
+    load_rows<D>(sb_ + QSmem::DO, p.dout, rowq, tid, 256);
     auto load_block = [&](int j, int buf) {
       // key positions of block j (threads 0..127: one key each), then rows
       if (tid < TBK) {
@@ -843,8 +856,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams 
       }
       sep::named_bar_sync(1, 256);  // every position is written before the row copies read them
       auto rowk = [&](int rr) -> int64_t { const int q = pos_s[buf * 128 + rr]; return q < 0 ? -1 : kvrow0 + q; };
-      load_rows128(sb_ + QSmem::K + buf * 4 * kT128, p.k, rowk, tid, 256);
-      load_rows128(sb_ + QSmem::V + buf * 4 * kT128, p.v, rowk, tid, 256);
+      load_rows<D>(sb_ + QSmem::K + buf * 2 * NB * kT128, p.k, rowk, tid, 256);
+      load_rows<D>(sb_ + QSmem::V + buf * 2 * NB * kT128, p.v, rowk, tid, 256);
       cp_async_commit();
     };
     load_block(0, 0);  // with Q and dO
@@ -928,12 +941,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams 
       sep::tc_fence_after();
       const float sc = p.scale_log2 * 0.69314718055994530942f;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t qv[32];
-        sep::tmem_ld32(tmem + lane_base + kColDQ + 64 * ch + 32 * c, qv);
+        sep::tmem_ld32(tmem + lane_base + kColDQ + (D / 2) * ch + 32 * c, qv);
         sep::tmem_wait_ld_r32(qv);
         if (i < S) {
-          uint4* dst = reinterpret_cast<uint4*>(dq + (qrow0 + i) * D + 64 * ch + 32 * c);
+          uint4* dst = reinterpret_cast<uint4*>(dq + (qrow0 + i) * D + (D / 2) * ch + 32 * c);
 #pragma unroll
           for (int u = 0; u < 4; ++u)
             dst[u] = make_uint4(sep::pack_bf16x2(__uint_as_float(qv[8 * u]) * sc, __uint_as_float(qv[8 * u + 1]) * sc),
@@ -954,7 +967,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams 
         const int buf = j & 1;
         if (!sep::mbar_wait(&bars.full, j & 1, abort, p.err)) break;
         sep::tc_fence_after();
-        const uint32_t ka = sb_ + QSmem::K + buf * 4 * kT128, va = sb_ + QSmem::V + buf * 4 * kT128;
+        const uint32_t ka = sb_ + QSmem::K + buf * 2 * NB * kT128, va = sb_ + QSmem::V + buf * 2 * NB * kT128;
         const uint64_t dK = sep::smem_desc_sw128(ka, 16), dV = sep::smem_desc_sw128(va, 16);
         const uint64_t dKmn = sep::smem_desc_sw128(ka, kT128);
 #pragma unroll
@@ -989,8 +1002,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams 
   }
 }
 
-// D = 128 runs the tcgen05 kernels
-constexpr bool kTcBackward = true;
+// D = 128 runs the tcgen05 kernels.  At D = 64 they are correct too (the
+// same kernels with one 64-column tile per 128-row tensor) but slower than
+// the warp-level kernel on the Pythia-160M shape (0.54 against 0.37 ms per
+// step): TMEM holds one CTA per SM and the items there are small.
+template <int D>
+constexpr bool tc_backward() { return D == 128; }
 
 struct BwdWs {
   size_t delta, dq, dk, dv;
@@ -1005,16 +1022,17 @@ BwdWs bwd_ws(int B, int Hq, int Hkv, int S, int D) {
   return w;
 }
 
-// the tcgen05 kernels (D = 128): dK, dV key-centric; dQ query-centric
+// the tcgen05 kernels: dK, dV key-centric; dQ query-centric
+template <int D>
 int launch_bwd_tc(BwdParams p, void* dq, cudaStream_t st) {
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(k_sep_bwd_tc_kv, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             KvSmem::BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(k_sep_bwd_tc_q, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             QSmem::BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_sep_bwd_tc_kv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             KvSmem<D>::BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(k_sep_bwd_tc_q<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             QSmem<D>::BYTES) != cudaSuccess)
       return SEP_ECUDA;
     attr_done[dev] = true;
   }
@@ -1023,11 +1041,11 @@ int launch_bwd_tc(BwdParams p, void* dq, cudaStream_t st) {
   const int64_t qrows = static_cast<int64_t>(p.B) * p.Hq * p.S;
   if (qrows > 0x7fffffffLL) return SEP_ETOOBIG;
   CUtensorMap mq, mdo;
-  if (!sep::make_rows_map(&mq, p.q, qrows, 128, TBQ) || !sep::make_rows_map(&mdo, p.dout, qrows, 128, TBQ))
+  if (!sep::make_rows_map(&mq, p.q, qrows, D, TBQ) || !sep::make_rows_map(&mdo, p.dout, qrows, D, TBQ))
     return SEP_ECUDA;
-  k_sep_bwd_tc_kv<<<dim3(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B), kTcThreads, KvSmem::BYTES, st>>>(p, mq, mdo);
+  k_sep_bwd_tc_kv<D><<<dim3(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B), kTcThreads, KvSmem<D>::BYTES, st>>>(p, mq, mdo);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  k_sep_bwd_tc_q<<<dim3((p.S + TBQ - 1) / TBQ, p.Hq, p.B), kTcThreads, QSmem::BYTES, st>>>(
+  k_sep_bwd_tc_q<D><<<dim3((p.S + TBQ - 1) / TBQ, p.Hq, p.B), kTcThreads, QSmem<D>::BYTES, st>>>(
       p, static_cast<__nv_bfloat16*>(dq));
   return cudaGetLastError() == cudaSuccess ? SEP_OK : SEP_ECUDA;
 }
@@ -1043,7 +1061,7 @@ int launch_bwd(const BwdParams& p0, const void* out, void* dq, void* dk, void* d
   p.dq_acc = reinterpret_cast<float*>(base + w.delta);
   p.dk_acc = reinterpret_cast<float*>(base + w.delta + w.dq);
   p.dv_acc = reinterpret_cast<float*>(base + w.delta + w.dq + w.dk);
-  const bool tc = D == 128 && kTcBackward;  // dq is then written directly, in bf16
+  constexpr bool tc = tc_backward<D>();  // dq is then written directly, in bf16
   if (tc) {
     if (cudaMemsetAsync(p.dk_acc, 0, w.dk + w.dv, st) != cudaSuccess) return SEP_ECUDA;
   } else if (cudaMemsetAsync(p.dq_acc, 0, w.dq + w.dk + w.dv, st) != cudaSuccess) {
@@ -1054,7 +1072,7 @@ int launch_bwd(const BwdParams& p0, const void* out, void* dq, void* dk, void* d
       static_cast<const __nv_bfloat16*>(out), p.dout, delta, rows);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   if (tc) {
-    const int rc = launch_bwd_tc(p, dq, st);
+    const int rc = launch_bwd_tc<D>(p, dq, st);
     if (rc != SEP_OK) return rc;
   } else {
   constexpr int smem = Smem<D>::BYTES;

@@ -65,7 +65,6 @@ struct DecodeParams {
   const void* kc;
   const void* vc;
   const int32_t* counts;
-  const int32_t* cur;   // [B] current K/V buffer
   const int32_t* plan;  // [B][cap + header] this step's plan (fused step only)
   const void* k_new;    // [B][Hkv][D] (fused step only)
   const void* v_new;
@@ -125,9 +124,11 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 
 // The last part of a split: its unnormalised partial (po, sm = max, sl = sum,
 // in this CTA's shared memory, rows with no keys at -inf / 0) is merged with
-// the other splits of the (b, kv head) and written out.
+// the other splits of the (b, kv head) and written out.  Returns true in
+// exactly one CTA of the (b, kv head), at a point where every split has
+// finished reading its K/V rows (the CTA that may then move rows in place).
 template <typename T, int D, int G, bool CLUSTER, int NCL = kMaxClusterSplits>
-__device__ __forceinline__ void decode_finish(const DecodeParams& p, float (*po)[D], float* sm,
+__device__ __forceinline__ bool decode_finish(const DecodeParams& p, float (*po)[D], float* sm,
                                               float* sl, int nsplit_b, int split, int b, int g) {
   __shared__ int is_last;
   __shared__ float Ms[G], Ls[G];
@@ -148,7 +149,7 @@ __device__ __forceinline__ void decode_finish(const DecodeParams& p, float (*po)
       cg::this_cluster().sync();
       cg::this_cluster().sync();
     }
-    return;
+    return split == 0;
   }
   if (CLUSTER) {
     // after the cluster barrier CTA `split` merges outputs
@@ -181,9 +182,9 @@ __device__ __forceinline__ void decode_finish(const DecodeParams& p, float (*po)
         p.lse[static_cast<int64_t>(b) * p.Hq + hq0 + h] = (M + log2f(L)) * 0.69314718055994530942f;
     }
     cl.sync();  // keep this CTA's partial alive until every reader is done
-    return;
+    return split == 0;
   }
-  if (split >= nsplit_b) return;
+  if (split >= nsplit_b) return false;
   // write this split's partial to the workspace
   for (int e = threadIdx.x; e < G * D; e += kThreads) {
     const int h = e / D, d = e % D;
@@ -203,7 +204,7 @@ __device__ __forceinline__ void decode_finish(const DecodeParams& p, float (*po)
     if (is_last) atomicExch(tk, 0);  // ready for the next call
   }
   __syncthreads();
-  if (!is_last) return;
+  if (!is_last) return false;
   __threadfence();
   // merge the partials of every split of this (b, kv head).  Loads that do
   // not depend on each other are issued together: one lane per split for the
@@ -245,6 +246,52 @@ __device__ __forceinline__ void decode_finish(const DecodeParams& p, float (*po)
   if (p.lse && threadIdx.x < G)
     p.lse[static_cast<int64_t>(b) * p.Hq + hq0 + threadIdx.x] =
         (Ms[threadIdx.x] + log2f(Ls[threadIdx.x])) * 0.69314718055994530942f;
+  return true;
+}
+
+// In-place flush of one layer's destination rows [from, len) of one (b, kv
+// head), by one CTA of nthreads threads, once every reader of their old
+// rows is done: destination row r takes source row plan.src[r] >= r (src
+// increasing; the new token, src == slot, from k_new / v_new).  Ascending chunks of `rows` rows staged
+// in shared memory (sk, sv), every source of a chunk read before any of its
+// destinations is written, so no row is overwritten before it is read.
+// Rows with src[r] == r (the initial block, and separators that stay) are
+// left alone; the new token's row (src == slot) is always written.
+template <typename T, int D>
+__device__ __forceinline__ void compact_in_place(const DecodeParams& p, int b, int g, int from,
+                                                 int len, int slot, int rows, int nthreads, T* sk,
+                                                 T* sv) {
+  constexpr int CH = D * static_cast<int>(sizeof(T)) / 16;
+  const int32_t* pl = p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr);
+  const int64_t base = (((static_cast<int64_t>(p.layer) * p.B + b) * p.Hkv + g) * p.cap) * D;
+  T* const kc = static_cast<T*>(const_cast<void*>(p.kc));
+  T* const vc = static_cast<T*>(const_cast<void*>(p.vc));
+  const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+  const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
+  const int first = pl[3] > from ? pl[3] : from;
+  for (int c0 = first; c0 < len; c0 += rows) {
+    const int nr = len - c0 < rows ? len - c0 : rows;
+    for (int e = threadIdx.x; e < 2 * nr * CH; e += nthreads) {
+      const int which = e / (nr * CH), r = (e / CH) % nr, c = e % CH;
+      const int src = pl[sep::kCachePlanHdr + c0 + r];
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (src == slot) {
+        val = (which ? vn : kn)[c];
+      } else if (src >= 0 && src < p.cap) {
+        val = reinterpret_cast<const uint4*>((which ? vc : kc) + base + static_cast<int64_t>(src) * D)[c];
+      }
+      reinterpret_cast<uint4*>((which ? sv : sk) + r * D)[c] = val;
+    }
+    __syncthreads();  // every source of the chunk has been read
+    for (int e = threadIdx.x; e < 2 * nr * CH; e += nthreads) {
+      const int which = e / (nr * CH), r = (e / CH) % nr, c = e % CH;
+      const int src = pl[sep::kCachePlanHdr + c0 + r];
+      if (src == c0 + r && src != slot) continue;  // the row stays
+      reinterpret_cast<uint4*>((which ? vc : kc) + base + static_cast<int64_t>(c0 + r) * D)[c] =
+          reinterpret_cast<const uint4*>((which ? sv : sk) + r * D)[c];
+    }
+    __syncthreads();
+  }
 }
 
 // FUSED: one decode step of the layer -- the CTA also writes the new token's
@@ -279,10 +326,8 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const Dec
   const int32_t* pl = p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr);
   const bool gen = p.prefix != nullptr;  // mask-based generation over k, v
   const int c0 = gen ? 0 : cnt[0], c1 = gen ? 0 : cnt[1], c2 = gen ? 0 : cnt[2], c3 = gen ? 0 : cnt[3];
-  const int buf = gen ? 0 : p.cur[b] & 1;  // current after this step's bookkeeping
   const int flush = FUSED ? pl[0] : 0;
   const int slot = FUSED ? pl[1] : -1;
-  const int sbuf = FUSED ? (pl[4] & 1) : buf;
   int len = c0 + c1 + c2 + c3;
   if (gen) len = GenRows(p, b).len;
   if (len < 0 || len > p.cap) len = 0;
@@ -290,11 +335,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const Dec
   const int nrows = len - r0 < 0 ? 0 : (len - r0 < ROWS ? len - r0 : ROWS);
   if (!CLUSTER && nrows == 0) return;
   const int nsplit_b = (len + ROWS - 1) / ROWS;
-  // element offset of row 0 of (buffer, layer, b, g)
-  auto base_of = [&](int bb) -> int64_t {
-    return ((((static_cast<int64_t>(bb) * p.layers + p.layer) * p.B + b) * p.Hkv + g) * p.cap) * D;
-  };
-  const int64_t kv_base = base_of(buf) + static_cast<int64_t>(r0) * D;
+  // element offset of row 0 of (layer, b, g)
+  const int64_t base = (((static_cast<int64_t>(p.layer) * p.B + b) * p.Hkv + g) * p.cap) * D;
+  const int64_t kv_base = base + static_cast<int64_t>(r0) * D;
   if (threadIdx.x == 0) {
     abort_flag = 0;
     sep::mbar_init(&bar, 1);
@@ -351,10 +394,9 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const Dec
     }
   constexpr int CH = D * static_cast<int>(sizeof(T)) / 16;  // 16-byte chunks per row
   if (FUSED && flush && nrows > 0) {
-    // rows of the post-flush layout come from their source rows in the old
-    // buffer (the new token from k_new/v_new); each is also stored at its
-    // destination in the new buffer
-    const int64_t sbase = base_of(sbuf);
+    // rows of the post-flush layout come from their source rows (the new
+    // token from k_new/v_new); the rows move in place only after every split
+    // of the (b, kv head) has read its sources (compact_in_place)
     const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
     const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
     for (int e = threadIdx.x; e < 2 * nrows * CH; e += kThreads) {
@@ -364,12 +406,10 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const Dec
       if (src == slot) {
         val = (which ? vn : kn)[c];
       } else if (src >= 0 && src < p.cap) {
-        val = reinterpret_cast<const uint4*>(static_cast<const T*>(which ? p.vc : p.kc) + sbase +
+        val = reinterpret_cast<const uint4*>(static_cast<const T*>(which ? p.vc : p.kc) + base +
                                              static_cast<int64_t>(src) * D)[c];
       }
       reinterpret_cast<uint4*>((which ? sv : sk) + r * D)[c] = val;
-      reinterpret_cast<uint4*>(const_cast<T*>(static_cast<const T*>(which ? p.vc : p.kc)) + kv_base +
-                               static_cast<int64_t>(r) * D)[c] = val;
     }
     __syncthreads();
   } else if (bulk) {
@@ -506,7 +546,12 @@ __global__ void __launch_bounds__(kThreads, (G <= 4 ? 5 : 3)) k_decode(const Dec
     sl[threadIdx.x] = 0.f;
   }
   __syncthreads();
-  decode_finish<T, D, G, CLUSTER>(p, po, sm, sl, nsplit_b, split, b, g);
+  const bool owner = decode_finish<T, D, G, CLUSTER>(p, po, sm, sl, nsplit_b, split, b, g);
+  if (FUSED && flush && owner) {
+    // every split has read its sources: move the rows in place
+    __syncthreads();
+    compact_in_place<T, D>(p, b, g, 0, len, slot, ROWS, kThreads, sk, sv);
+  }
 }
 
 // ---- warp-level tensor-core helpers (bf16 in, fp32 accumulate)
@@ -688,7 +733,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   // completes long before the first remote store (after the chunk loop):
   // every CTA's barriers are initialised by then
   sep::cluster_arrive_relaxed();
-  // With p.early (fused step, layer >= 1) the cache metadata (counts, cur,
+  // With p.early (fused step, layer >= 1) the cache metadata (counts and
   // plan) and this layer's rows are read before waiting on the previous
   // grid; q, k_new, v_new and every store still come after the wait.  This
   // is safe because of how the step is ordered, not because of distance in
@@ -705,29 +750,23 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   if (!p.early) asm volatile("griddepcontrol.wait;" ::: "memory");
   const int32_t* pl = FUSED ? p.plan + static_cast<int64_t>(b) * (p.cap + sep::kCachePlanHdr) : nullptr;
   int len;
-  int buf = 0;
   if constexpr (GATHER) {
     len = GenRows(p, b).len;
   } else {
     const int32_t* cnt = p.counts + 4 * b;
     len = cnt[0] + cnt[1] + cnt[2] + cnt[3];
-    buf = p.cur[b] & 1;
   }
   const int flush = FUSED ? pl[0] : 0;
   const int slot = FUSED ? pl[1] : -1;
-  const int sbuf = FUSED ? (pl[4] & 1) : buf;
   if (len < 0 || len > p.cap) len = 0;
   const int per = ((len + NCL - 1) / NCL + 15) / 16 * 16;  // rows per CTA (multiple of 16)
   const int rs = rank * per < len ? rank * per : len;
   const int re = rs + per < len ? rs + per : len;
   const int nchunks = (re - rs + ROWS - 1) / ROWS;
-  // first row of this (buffer, layer, b, kv head) in the [rows, D] view
-  // (gathers: first row of (b, kv head) in the [B * Hkv * S, D] view of k, v)
-  auto row_of = [&](int bb) -> int64_t {
-    if constexpr (GATHER) return (static_cast<int64_t>(b) * p.Hkv + g) * p.S;
-    return (((static_cast<int64_t>(bb) * p.layers + p.layer) * p.B + b) * p.Hkv + g) * p.cap;
-  };
-  const int64_t row0 = row_of(buf);
+  // first row of this (layer, b, kv head) in the [rows, D] view (gathers:
+  // first row of (b, kv head) in the [B * Hkv * S, D] view of k, v)
+  const int64_t row0 = GATHER ? (static_cast<int64_t>(b) * p.Hkv + g) * p.S
+                              : ((static_cast<int64_t>(p.layer) * p.B + b) * p.Hkv + g) * p.cap;
   T* const kc = static_cast<T*>(const_cast<void*>(p.kc));
   T* const vc = static_cast<T*>(const_cast<void*>(p.vc));
   __syncthreads();
@@ -788,11 +827,13 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
         }
         cp_async_arrive(&full[st]);
       } else if (FUSED && flush) {
-        // rows of the post-flush layout come from their source rows in the
-        // old buffer (the new token from k_new/v_new); each is also stored
-        // at its destination in the new buffer
+        // rows of the post-flush layout come from their source rows (the
+        // new token from k_new/v_new).  The first CTA of the pair also
+        // stores each row at its destination, in place: its destinations
+        // lie below every source of the second CTA and below the sources of
+        // its own later chunks.  The second CTA's destinations may be the
+        // first one's sources, so it moves its rows after the merge.
         asm volatile("griddepcontrol.wait;" ::: "memory");
-        const int64_t srow = row_of(sbuf);
         const uint4* kn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.k_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
         const uint4* vn = reinterpret_cast<const uint4*>(static_cast<const T*>(p.v_new) + (static_cast<int64_t>(b) * p.Hkv + g) * D);
         for (int e = lane; e < 2 * nr * CH; e += 32) {
@@ -802,10 +843,11 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
           if (src == slot) {
             val = (which ? vn : kn)[cc];
           } else if (src >= 0 && src < p.cap) {
-            val = reinterpret_cast<const uint4*>((which ? vc : kc) + (srow + src) * D)[cc];
+            val = reinterpret_cast<const uint4*>((which ? vc : kc) + (row0 + src) * D)[cc];
           }
           *reinterpret_cast<uint4*>((which ? vt : kt) + swz(r, 8 * cc)) = val;
-          reinterpret_cast<uint4*>((which ? vc : kc) + (row0 + r0 + r) * D)[cc] = val;
+          if (rank == 0 && (src != r0 + r || src == slot))  // a row that stays is not rewritten
+            reinterpret_cast<uint4*>((which ? vc : kc) + (row0 + r0 + r) * D)[cc] = val;
         }
         sep::fence_proxy_async_smem();  // later tensor copies refill these bytes
         __syncwarp();
@@ -1094,6 +1136,16 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
       p.lse[static_cast<int64_t>(b) * p.Hq + g * G + h] =
           L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
   }
+  if constexpr (FUSED) {
+    if (flush && rank > 0 && rs < re) {
+      // The merge has received the first CTA's partials, sent after it had
+      // loaded every one of its rows: its sources are all read, so this
+      // CTA's rows can now move in place (staged through ring stage 0).
+      __syncthreads();
+      compact_in_place<T, D>(p, b, g, rs, re, slot, ROWS, kPipeThreads, reinterpret_cast<T*>(ring),
+                             reinterpret_cast<T*>(ring + ROWS * D * 2));
+    }
+  }
 }
 
 // Maximum dynamic shared memory for `kern` on the current device, set once.
@@ -1147,8 +1199,8 @@ int launch_one(const DecodeParams& p, cudaStream_t st) {
       }
     }
     if (!p.prefix) {
-      // the K and V arrays as [2 * layers * B * Hkv * cap, D] rows
-      const int64_t rows = 2LL * p.layers * p.B * p.Hkv * p.cap;
+      // the K and V arrays as [layers * B * Hkv * cap, D] rows
+      const int64_t rows = static_cast<int64_t>(p.layers) * p.B * p.Hkv * p.cap;
       if (rows > 0x7fffffffLL) return SEP_ETOOBIG;
       if (!sep::make_rows_map(&mk, p.kc, rows, D, ROWS) || !sep::make_rows_map(&mv, p.vc, rows, D, ROWS))
         return SEP_ECUDA;
@@ -1216,7 +1268,6 @@ extern "C" int sep_attn_decode(const sepcache* c, int layer, const void* q, int 
   p.kc = c->k;
   p.vc = c->v;
   p.counts = c->counts;
-  p.cur = c->cur;
   p.plan = c->plan;
   p.k_new = nullptr;
   p.v_new = nullptr;
@@ -1271,7 +1322,6 @@ extern "C" int sep_attn_decode_step(const sepcache* c, int layer, const void* q,
   p.kc = c->k;
   p.vc = c->v;
   p.counts = c->counts;
-  p.cur = c->cur;
   p.plan = c->plan;
   p.k_new = k_new;
   p.v_new = v_new;
@@ -1389,7 +1439,6 @@ extern "C" int sep_attn_decode_noalloc(const sepcache* c, int layer, const void*
   p.kc = c->k;
   p.vc = c->v;
   p.counts = c->counts;
-  p.cur = c->cur;
   p.plan = c->plan;
   p.k_new = nullptr;
   p.v_new = nullptr;

@@ -14,13 +14,13 @@
 //   L  local window: the newest w tokens.
 // Rows of each (layer, b, kv head) are stored I | S | P | L in increasing
 // position order.  P and L are one contiguous run of recent positions, so a
-// token sliding from L to P moves no data; only a flush moves rows.  The
-// K/V rows live in two buffers per sequence: a flush copies the surviving
-// rows, in order, from the current buffer into the other one (out of place,
-// so every row can be copied in parallel and the decode of the same step can
-// fetch its rows from either side without hazards), and that buffer becomes
-// current.  The surviving rows are found with an order-preserving
-// warp-ballot stream compaction of the I | S | P | L rows.
+// token sliding from L to P moves no data; only a flush moves rows.  A flush
+// compacts the surviving rows in place: the survivors are found with an
+// order-preserving warp-ballot stream compaction of the I | S | P | L rows,
+// so destination row r takes source row src[r] >= r, with src increasing.
+// Copying the rows in ascending chunks, every source of a chunk read before
+// any destination of that chunk is written, therefore never overwrites a
+// row that is still to be read.
 //
 // Bookkeeping is shared by all layers: sepcache_append at layer 0 runs the
 // state machine for the new token and records this step's plan (the row the
@@ -33,7 +33,7 @@
 
 namespace {
 
-// plan[b] = {flush, slot, new_len, nI, src_buf, dst_buf, -, -, src row of each
+// plan[b] = {flush, slot, new_len, nI, -, -, -, -, source row of each
 // destination row (flush steps)...}
 constexpr int kPlanHdr = 8;
 
@@ -47,8 +47,8 @@ __device__ __forceinline__ uint32_t lanemask_lt() {
 __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__ flag,
                                 int32_t* __restrict__ counts, int32_t* __restrict__ plan,
                                 int64_t* __restrict__ step, int32_t* __restrict__ status,
-                                int32_t* __restrict__ cur, const uint8_t* __restrict__ is_sep_new,
-                                int B, int cap, int a, int s, int past, int w, int mode) {
+                                const uint8_t* __restrict__ is_sep_new, int B, int cap, int a,
+                                int s, int past, int w, int mode) {
   const int b = blockIdx.x;
   const int lane = threadIdx.x;
   if (b >= B) return;
@@ -58,7 +58,6 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
   uint8_t* fl = flag + static_cast<int64_t>(b) * cap;
   int nI = cnt[0], nS = cnt[1], nP = cnt[2], nL = cnt[3];
   const int64_t t = step[b];
-  const int cb = cur[b] & 1;
   const uint8_t f = is_sep_new[b] ? 1 : 0;
   int len = nI + nS + nP + nL;
   const bool total_trigger = (mode & SEP_CACHE_TOTAL_TRIGGER) != 0;
@@ -73,7 +72,6 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
       pl[1] = -1;
       pl[2] = len > cap ? cap : (len < 0 ? 0 : len);
       pl[3] = 0;
-      pl[4] = pl[5] = cb;
     }
     return;
   }
@@ -146,9 +144,6 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
     pl[1] = slot;
     pl[2] = new_len;
     pl[3] = nI;
-    pl[4] = cb;                   // rows are read from (and the token written to)
-    pl[5] = flush ? 1 - cb : cb;  // rows are current in after this step
-    cur[b] = pl[5];
     cnt[0] = nI;
     cnt[1] = nS;
     cnt[2] = nP;
@@ -157,58 +152,75 @@ __global__ void k_cache_advance(int32_t* __restrict__ pos, uint8_t* __restrict__
   }
 }
 
-// Byte offset of row 0 of (buffer, layer, b, kv head).
-__device__ __forceinline__ int64_t row0(int buf, int layer, int b, int g, int layers, int B,
-                                        int Hkv, int cap, int row_bytes) {
-  return ((((static_cast<int64_t>(buf) * layers + layer) * B + b) * Hkv + g) * cap) * row_bytes;
+// Byte offset of row 0 of (layer, b, kv head).
+__device__ __forceinline__ int64_t row0(int layer, int b, int g, int B, int Hkv, int cap,
+                                        int row_bytes) {
+  return (((static_cast<int64_t>(layer) * B + b) * Hkv + g) * cap) * row_bytes;
 }
 
-// Write the new token's K and V rows of one layer at this step's slot of the
-// buffer the step reads from.
+// Write the new token's K and V rows of one layer at this step's slot.
 __global__ void k_cache_write(uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
                               const uint8_t* __restrict__ k_new, const uint8_t* __restrict__ v_new,
-                              const int32_t* __restrict__ plan, int layer, int layers, int B,
-                              int Hkv, int cap, int row_bytes) {
+                              const int32_t* __restrict__ plan, int layer, int B, int Hkv, int cap,
+                              int row_bytes) {
   const int b = blockIdx.x;
   const int32_t* pl = plan + static_cast<int64_t>(b) * (cap + kPlanHdr);
-  const int slot = pl[1], sb = pl[4] & 1;
+  const int slot = pl[1];
   if (slot < 0 || slot >= cap) return;
   const int ch = row_bytes / 16;
   const int per = Hkv * ch;
   for (int e = threadIdx.x; e < 2 * per; e += blockDim.x) {
     const int which = e / per, g = (e % per) / ch, c = e % ch;
-    const int64_t dst = row0(sb, layer, b, g, layers, B, Hkv, cap, row_bytes) +
-                        static_cast<int64_t>(slot) * row_bytes;
+    const int64_t dst = row0(layer, b, g, B, Hkv, cap, row_bytes) + static_cast<int64_t>(slot) * row_bytes;
     const int64_t src = (static_cast<int64_t>(b) * Hkv + g) * row_bytes;
     const uint4 val = reinterpret_cast<const uint4*>((which ? v_new : k_new) + src)[c];
     reinterpret_cast<uint4*>((which ? vc : kc) + dst)[c] = val;
   }
 }
 
-// Apply this step's flush to one layer: destination row r of the other
-// buffer takes source row plan.src[r] of the current one.  Out of place, so
-// every 16-byte chunk is copied independently.  Grid: (chunks, kv head, b).
-__global__ void __launch_bounds__(256) k_cache_compact(uint8_t* __restrict__ kc,
-                                                       uint8_t* __restrict__ vc,
-                                                       const int32_t* __restrict__ plan, int layer,
-                                                       int layers, int B, int Hkv, int cap,
-                                                       int row_bytes) {
-  const int g = blockIdx.y, b = blockIdx.z;
+// Apply this step's flush to one layer, in place: destination row r takes
+// source row plan.src[r] >= r (increasing in r).  One CTA per (K or V, kv
+// head, b) walks the destination rows in ascending chunks of kChunkRows; it
+// reads every source row of a chunk into registers, synchronises, then
+// writes the chunk.  A chunk's destinations lie below the sources of every
+// later chunk, so nothing is overwritten before it is read.  Rows that do
+// not move (the initial block, and any row with src[r] == r) are skipped.
+constexpr int kCompactThreads = 256;
+constexpr int kCompactUnits = 4;  // 16-byte units per thread and chunk
+__global__ void __launch_bounds__(kCompactThreads) k_cache_compact(uint8_t* __restrict__ kc,
+                                                                   uint8_t* __restrict__ vc,
+                                                                   const int32_t* __restrict__ plan,
+                                                                   int layer, int B, int Hkv,
+                                                                   int cap, int row_bytes) {
+  const int which = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int32_t* pl = plan + static_cast<int64_t>(b) * (cap + kPlanHdr);
   if (pl[0] == 0) return;
-  const int new_len = pl[2], sb = pl[4] & 1, db = pl[5] & 1;
+  const int new_len = pl[2] < cap ? pl[2] : cap;
+  const int first = pl[3] > 0 ? pl[3] : 0;  // the initial rows keep their place
   const int ch = row_bytes / 16;
-  const int64_t sbase = row0(sb, layer, b, g, layers, B, Hkv, cap, row_bytes);
-  const int64_t dbase = row0(db, layer, b, g, layers, B, Hkv, cap, row_bytes);
-  const int total = 2 * new_len * ch;
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < total; e += gridDim.x * blockDim.x) {
-    const int which = e / (new_len * ch);
-    const int r = (e / ch) % new_len, c = e % ch;
-    const int src = pl[kPlanHdr + r];
-    if (src < 0 || src >= cap) continue;
-    uint8_t* base = which ? vc : kc;
-    const uint4 val = reinterpret_cast<const uint4*>(base + sbase + static_cast<int64_t>(src) * row_bytes)[c];
-    reinterpret_cast<uint4*>(base + dbase + static_cast<int64_t>(r) * row_bytes)[c] = val;
+  const int chunk_rows = kCompactThreads * kCompactUnits / ch;
+  uint8_t* base = (which ? vc : kc) + row0(layer, b, g, B, Hkv, cap, row_bytes);
+  for (int r0 = first; r0 < new_len; r0 += chunk_rows) {
+    uint4 val[kCompactUnits];
+    int dst[kCompactUnits];
+#pragma unroll
+    for (int u = 0; u < kCompactUnits; ++u) {
+      const int e = u * kCompactThreads + threadIdx.x;
+      const int r = r0 + e / ch, c = e % ch;
+      dst[u] = -1;
+      if (r < new_len) {
+        const int src = pl[kPlanHdr + r];
+        if (src >= 0 && src < cap && src != r) {
+          val[u] = reinterpret_cast<const uint4*>(base + static_cast<int64_t>(src) * row_bytes)[c];
+          dst[u] = r * ch + c;
+        }
+      }
+    }
+    __syncthreads();  // every source of the chunk has been read
+#pragma unroll
+    for (int u = 0; u < kCompactUnits; ++u)
+      if (dst[u] >= 0) reinterpret_cast<uint4*>(base)[dst[u]] = val[u];
+    __syncthreads();
   }
 }
 
@@ -230,7 +242,7 @@ __global__ void __launch_bounds__(256) k_cache_compact(uint8_t* __restrict__ kc,
 __global__ void k_cache_ingest_meta(int32_t* __restrict__ pos, uint8_t* __restrict__ flag,
                                     int32_t* __restrict__ counts, int32_t* __restrict__ plan,
                                     int64_t* __restrict__ step, int32_t* __restrict__ status,
-                                    int32_t* __restrict__ cur, const uint8_t* __restrict__ is_sep,
+                                    const uint8_t* __restrict__ is_sep,
                                     const int32_t* __restrict__ prefix,
                                     const int32_t* __restrict__ idx, int T, int cap, int a, int s,
                                     int past, int w, int mode) {
@@ -315,7 +327,6 @@ __global__ void k_cache_ingest_meta(int32_t* __restrict__ pos, uint8_t* __restri
     cnt[2] = nP;
     cnt[3] = nL;
     step[b] = T;
-    cur[b] = 0;
     int32_t* pl = plan + static_cast<int64_t>(b) * (cap + kPlanHdr);
     pl[0] = 0;
     pl[1] = -1;
@@ -326,14 +337,14 @@ __global__ void k_cache_ingest_meta(int32_t* __restrict__ pos, uint8_t* __restri
   }
 }
 
-// One layer's K/V rows of an ingested prompt: row r of buffer 0 takes the
+// One layer's K/V rows of an ingested prompt: row r takes the
 // prompt's row at position pos[r] (k, v: [B][Hkv][T][D]).  Grid: (chunks,
 // kv head, b).  Skips a sequence whose ingestion did not happen (step != T).
 __global__ void __launch_bounds__(256) k_cache_ingest_rows(
     uint8_t* __restrict__ kc, uint8_t* __restrict__ vc, const uint8_t* __restrict__ k,
     const uint8_t* __restrict__ v, const int32_t* __restrict__ pos,
-    const int32_t* __restrict__ counts, const int64_t* __restrict__ step, int T, int layer,
-    int layers, int B, int Hkv, int cap, int row_bytes) {
+    const int32_t* __restrict__ counts, const int64_t* __restrict__ step, int T, int layer, int B,
+    int Hkv, int cap, int row_bytes) {
   const int g = blockIdx.y, b = blockIdx.z;
   if (step[b] != T) return;
   const int32_t* cnt = counts + 4 * b;
@@ -341,7 +352,7 @@ __global__ void __launch_bounds__(256) k_cache_ingest_rows(
   if (len < 0 || len > cap) return;
   const int ch = row_bytes / 16;  // 16-byte chunks per row: a power of two (8, 16 or 32)
   const int lg = __ffs(ch) - 1;
-  const int64_t dbase = row0(0, layer, b, g, layers, B, Hkv, cap, row_bytes);
+  const int64_t dbase = row0(layer, b, g, B, Hkv, cap, row_bytes);
   const int64_t sbase = (static_cast<int64_t>(b) * Hkv + g) * T * row_bytes;
   const int32_t* ps = pos + static_cast<int64_t>(b) * cap;
   const int half = len << lg;  // chunks of K; V follows
@@ -361,8 +372,8 @@ __global__ void __launch_bounds__(256) k_cache_ingest_rows(
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
 
 struct Sizes {
-  size_t k, v, pos, flag, counts, plan, step, status, cur, rope;
-  size_t total() const { return k + v + pos + flag + counts + plan + step + status + cur + rope; }
+  size_t k, v, pos, flag, counts, plan, step, status, rope;
+  size_t total() const { return k + v + pos + flag + counts + plan + step + status + rope; }
 };
 
 // rows of the rotary table: every slot, and at least 65 so that the decode
@@ -372,7 +383,7 @@ int rope_rows_of(int64_t cap) { return static_cast<int>(cap > 65 ? cap : 65); }
 Sizes sizes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
   const int64_t cap = static_cast<int64_t>(cfg.a) + cfg.s + cfg.past + cfg.w + 1;
   Sizes z;
-  z.k = round256(2 * static_cast<size_t>(layers) * B * Hkv * cap * D * sep::elem_bytes(dtype));
+  z.k = round256(static_cast<size_t>(layers) * B * Hkv * cap * D * sep::elem_bytes(dtype));
   z.v = z.k;
   z.pos = round256(static_cast<size_t>(B) * cap * 4);
   z.flag = round256(static_cast<size_t>(B) * cap);
@@ -380,7 +391,6 @@ Sizes sizes(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
   z.plan = round256(static_cast<size_t>(B) * (cap + kPlanHdr) * 4);
   z.step = round256(static_cast<size_t>(B) * 8);
   z.status = 256;
-  z.cur = round256(static_cast<size_t>(B) * 4);
   z.rope = round256(static_cast<size_t>(rope_rows_of(cap)) * D * 4);
   return z;
 }
@@ -396,7 +406,7 @@ bool cfg_ok(sep_cache_cfg cfg, int layers, int B, int Hkv, int D, int dtype) {
 
 bool cache_ok(const sepcache* c) {
   return c && c->k && c->v && c->pos && c->flag && c->counts && c->plan && c->step && c->status &&
-         c->cur && c->rope && c->rope_rows == rope_rows_of(c->cap) && c->rope_theta >= 0.f &&
+         c->rope && c->rope_rows == rope_rows_of(c->cap) && c->rope_theta >= 0.f &&
          cfg_ok(c->cfg, c->layers, c->B, c->Hkv, c->D, c->dtype) &&
          c->cap == c->cfg.a + c->cfg.s + c->cfg.past + c->cfg.w + 1;
 }
@@ -437,8 +447,6 @@ extern "C" int sepcache_carve(sepcache* cache, void* buffer, size_t bytes, sep_c
   p += z.step;
   cache->status = reinterpret_cast<int32_t*>(p);
   p += z.status;
-  cache->cur = reinterpret_cast<int32_t*>(p);
-  p += z.cur;
   cache->rope = reinterpret_cast<float*>(p);
   cache->layers = layers;
   cache->B = B;
@@ -493,8 +501,7 @@ extern "C" int sepcache_init(const sepcache* c, void* stream) {
             cudaMemsetAsync(c->counts, 0, c->B * 16, st) == cudaSuccess &&
             cudaMemsetAsync(c->plan, 0, c->B * (cap + kPlanHdr) * 4, st) == cudaSuccess &&
             cudaMemsetAsync(c->step, 0, c->B * 8, st) == cudaSuccess &&
-            cudaMemsetAsync(c->status, 0, 4, st) == cudaSuccess &&
-            cudaMemsetAsync(c->cur, 0, c->B * 4, st) == cudaSuccess;
+            cudaMemsetAsync(c->status, 0, 4, st) == cudaSuccess;
   return ok ? SEP_OK : SEP_ECUDA;
 }
 
@@ -505,8 +512,8 @@ int cache_advance(const sepcache* c, const uint8_t* is_sep_new, cudaStream_t st)
   // has completed, which is what lets the fused decode of layers >= 1 read
   // the cache metadata and its layer's rows before its grid-dependency wait.
   k_cache_advance<<<c->B, 32, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step, c->status,
-                                        c->cur, is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
-                                        c->cfg.past, c->cfg.w, c->cfg.mode);
+                                        is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s, c->cfg.past,
+                                        c->cfg.w, c->cfg.mode);
   return launch_status();
 }
 bool cache_valid(const sepcache* c) { return cache_ok(c); }
@@ -522,16 +529,16 @@ extern "C" int sepcache_append(const sepcache* c, int layer, const void* k_new, 
   if (layer == 0) {
     // a plain launch (no programmatic serialization), as in cache_advance
     k_cache_advance<<<c->B, 32, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step, c->status,
-                                          c->cur, is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s,
-                                          c->cfg.past, c->cfg.w, c->cfg.mode);
+                                          is_sep_new, c->B, c->cap, c->cfg.a, c->cfg.s, c->cfg.past,
+                                          c->cfg.w, c->cfg.mode);
     if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   }
   const int row_bytes = c->D * sep::elem_bytes(c->dtype);
   const int threads = 2 * c->Hkv * row_bytes / 16 < 512 ? 2 * c->Hkv * row_bytes / 16 : 512;
   k_cache_write<<<c->B, (threads + 31) / 32 * 32, 0, st>>>(
       static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v),
-      static_cast<const uint8_t*>(k_new), static_cast<const uint8_t*>(v_new), c->plan, layer,
-      c->layers, c->B, c->Hkv, c->cap, row_bytes);
+      static_cast<const uint8_t*>(k_new), static_cast<const uint8_t*>(v_new), c->plan, layer, c->B,
+      c->Hkv, c->cap, row_bytes);
   return sep::launch_status();
 }
 
@@ -540,9 +547,9 @@ extern "C" int sepcache_compact(const sepcache* c, int layer, void* stream) {
   if (layer < 0 || layer >= c->layers) return SEP_EINVAL;
   const int row_bytes = c->D * sep::elem_bytes(c->dtype);
   dim3 grid(2, c->Hkv, c->B);
-  k_cache_compact<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), c->plan, layer, c->layers, c->B,
-      c->Hkv, c->cap, row_bytes);
+  k_cache_compact<<<grid, kCompactThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), c->plan, layer, c->B, c->Hkv,
+      c->cap, row_bytes);
   return sep::launch_status();
 }
 
@@ -557,7 +564,7 @@ extern "C" int sepcache_ingest(const sepcache* c, int layer, const void* k, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (layer == 0) {
     k_cache_ingest_meta<<<c->B, 256, 0, st>>>(c->pos, c->flag, c->counts, c->plan, c->step,
-                                               c->status, c->cur, is_sep, prefix, idx, T, c->cap,
+                                               c->status, is_sep, prefix, idx, T, c->cap,
                                                c->cfg.a, c->cfg.s, c->cfg.past, c->cfg.w, c->cfg.mode);
     if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   }
@@ -568,8 +575,8 @@ extern "C" int sepcache_ingest(const sepcache* c, int layer, const void* k, cons
   dim3 grid((chunks + 255) / 256, c->Hkv, c->B);
   k_cache_ingest_rows<<<grid, 256, 0, st>>>(
       static_cast<uint8_t*>(c->k), static_cast<uint8_t*>(c->v), static_cast<const uint8_t*>(k),
-      static_cast<const uint8_t*>(v), c->pos, c->counts, c->step, T, layer, c->layers, c->B,
-      c->Hkv, c->cap, row_bytes);
+      static_cast<const uint8_t*>(v), c->pos, c->counts, c->step, T, layer, c->B, c->Hkv, c->cap,
+      row_bytes);
   return sep::launch_status();
 }
 

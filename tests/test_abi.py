@@ -91,17 +91,18 @@ def test_cache_layout_and_validation(sl):
     nb = L.sepcache_bytes(cfg, 32, 16, 8, 128, 1)
     cap = 4 + 64 + 128 + 256 + 1
     kv = 32 * 16 * 8 * cap * 128 * 2
-    # K and V, two buffers each; the metadata and the rotary table are small
-    assert nb >= 4 * kv and nb < 4 * kv + 512 * 1024
+    # K and V, one buffer each (flushes compact in place); the metadata and
+    # the rotary table are small
+    assert nb >= 2 * kv and nb < 2 * kv + 512 * 1024
     assert L.sepcache_bytes(sl.SepCacheCfg(4, 64, 128, 0), 1, 1, 1, 128, 1) == 0  # w >= 1
     assert L.sepcache_bytes(sl.SepCacheCfg(-1, 64, 128, 4), 1, 1, 1, 128, 1) == 0
     assert L.sepcache_bytes(cfg, 1, 1, 1, 96, 1) == 0
     c = sl._SepCacheC()
     base = ctypes.c_void_p(1 << 20)
     assert L.sepcache_carve(ctypes.byref(c), base, nb, cfg, 32, 16, 8, 128, 1) == 0
-    assert c.cap == cap and c.k == (1 << 20) and c.v - c.k >= 2 * kv
+    assert c.cap == cap and c.k == (1 << 20) and c.v - c.k >= kv
     assert all(getattr(c, f) % 256 == 0
-               for f in ("pos", "flag", "counts", "plan", "step", "status", "cur", "rope"))
+               for f in ("pos", "flag", "counts", "plan", "step", "status", "rope"))
     # rotary table: max(cap, 65) rows of D/2 (cos, sin) pairs, at the end
     assert c.rope_rows == cap and c.rope_theta == 0.0
     assert c.rope + cap * 128 * 4 <= (1 << 20) + nb

@@ -82,3 +82,10 @@ def test_backward_pythia160m_shape(sl):
     # B8, 12 heads (MHA), D64, S2048, a=4, n=64, 8 % separators, data / 8
     got, ref = _run(sl, 8, 12, 12, 2048, 64, 4, 64, 0.08, seed=1002, std=1.0 / 8.0)
     print(_check(got, ref, "pythia"))
+
+
+def test_backward_llama3_8b_shape(sl):
+    # the bench's Llama-3-8B shape: B1, 32 query / 8 kv heads, D128, S8192,
+    # a=4, n=256, 10 % separators; every element of dq, dk and dv checked
+    got, ref = _run(sl, 1, 32, 8, 8192, 128, 4, 256, 0.1, seed=1003)
+    print(_check(got, ref, "llama3-8k"))

@@ -88,15 +88,14 @@ def _check_meta(st, snap, k):
 
 def _check_kv(st, snap, k):
     c = st.cache
-    K, V, cur = c.k.cpu(), c.v.cpu(), c.cur.cpu()
+    K, V = c.k.cpu(), c.v.cpu()
     for b in range(st.B):
         n = int(snap["counts"][k, b].sum())
         pos = snap["pos"][k, b, :n]
-        cb = int(cur[b])
         for l in range(st.layers):
             kr, vr = st.kv_rows(l, pos, b)
-            assert torch.equal(K[cb, l, b, :, :n], kr), (k, b, l)
-            assert torch.equal(V[cb, l, b, :, :n], vr), (k, b, l)
+            assert torch.equal(K[l, b, :, :n], kr), (k, b, l)
+            assert torch.equal(V[l, b, :, :n], vr), (k, b, l)
 
 
 def _check_decode(st, snap, k, outs, t):
@@ -142,6 +141,30 @@ def test_small_caches_every_step(sl, shape, fused):
         if t % 7 == 0 or t < 40:
             _check_kv(st, snap, t)
         _check_decode(st, snap, t, outs, t)
+    assert st.cache.status() == 0
+    assert sl.device_status() == 0
+
+
+@pytest.mark.parametrize("fused", [False, True], ids=["separate", "fused"])
+def test_fp32_more_than_eight_splits_every_step(sl, fused):
+    """An exact (fp32) cache of up to 643 rows: ten 64-row splits, merged
+    through the workspace by the last split to finish; on flush steps the
+    fused step's rows move in place only after every split has read its
+    sources.  Late in the stream the sequences retain more than 512 rows."""
+    a, s, past, w, B, Hkv, Hq, D = 2, 160, 40, 440, 2, 1, 2, 64
+    T = 1300
+    st = Stream(sl, a, s, past, w, B, Hkv, Hq, D, 2, torch.float32, seed=7777, T=T, fused=fused)
+    snap = oracle.sepcache_simulate(st.flags, a, s, past, w, np.arange(T))
+    flushes = {a + w + k * (past + 1) - 1 for k in range(1, 40)}
+    for t in range(T):
+        dec = (0, 1) if (t % 7 == 0 or t in flushes or t + 1 in flushes) else ()
+        outs = st.step(decode_layers=dec)
+        _check_meta(st, snap, t)
+        if t % 13 == 0 or t in flushes:
+            _check_kv(st, snap, t)
+        if dec:
+            _check_decode(st, snap, t, outs, t)
+    assert int(snap["counts"][T - 1].sum(1).min()) > 8 * 64
     assert st.cache.status() == 0
     assert sl.device_status() == 0
 

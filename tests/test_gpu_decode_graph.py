@@ -76,7 +76,6 @@ def test_graph_replayed_decode_step_matches_oracle(sl):
         np.testing.assert_array_equal(c.counts.cpu().numpy(), snap["counts"][k], err_msg=str(t))
         np.testing.assert_array_equal(c.pos.cpu().numpy(), snap["pos"][k], err_msg=str(t))
         np.testing.assert_array_equal(c.flag.cpu().numpy(), snap["flag"][k], err_msg=str(t))
-        cur = c.cur.cpu().numpy()
         out = wl.out.double().cpu().numpy()
         lse = wl.lse.double().cpu().numpy()
         r = t % R
@@ -88,9 +87,8 @@ def test_graph_replayed_decode_step_matches_oracle(sl):
                 kr = hk[ring_idx, l, b].transpose(0, 1).contiguous()  # [Hkv, n, D]
                 vr = hv[ring_idx, l, b].transpose(0, 1).contiguous()
                 if l in kv_layers:
-                    cb = int(cur[b])
-                    assert torch.equal(c.k[cb, l, b, :, :n].cpu(), kr), (t, l, b)
-                    assert torch.equal(c.v[cb, l, b, :, :n].cpu(), vr), (t, l, b)
+                    assert torch.equal(c.k[l, b, :, :n].cpu(), kr), (t, l, b)
+                    assert torch.equal(c.v[l, b, :, :n].cpu(), vr), (t, l, b)
                 want, want_lse = oracle.attend(hq[r, l, b], kr, vr)
                 d = out[l, b] - want
                 assert np.abs(d).max() <= 2e-2 and np.sqrt((d * d).mean()) <= 2e-3, (t, l, b)

@@ -41,14 +41,14 @@ def _check_state(cache, snap, k_snap, B, layers, kv_of):
     np.testing.assert_array_equal(cache.counts.cpu().numpy(), snap["counts"][k_snap])
     np.testing.assert_array_equal(cache.pos.cpu().numpy(), snap["pos"][k_snap])
     np.testing.assert_array_equal(cache.flag.cpu().numpy(), snap["flag"][k_snap])
-    K, V, cur = cache.k.cpu(), cache.v.cpu(), cache.cur.cpu()
+    K, V = cache.k.cpu(), cache.v.cpu()
     for b in range(B):
         n = int(snap["counts"][k_snap, b].sum())
         pos = snap["pos"][k_snap, b, :n]
         for l in range(layers):
             kr, vr = kv_of(l, b, pos)
-            assert torch.equal(K[int(cur[b]), l, b, :, :n], kr), (b, l)
-            assert torch.equal(V[int(cur[b]), l, b, :, :n], vr), (b, l)
+            assert torch.equal(K[l, b, :, :n], kr), (b, l)
+            assert torch.equal(V[l, b, :, :n], vr), (b, l)
 
 
 CASES = [
