@@ -86,11 +86,14 @@ TRAFFIC = {
         bytes=161018624 + 101916928, per="launch", src=("backward.cu", "common.cuh"),
         sha1="ccc1d51920b8eb0ffa71d1c0b81985af9610007c"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
-        bytes=104931328 + 30614528, per="launch", src=("prefill_tc.cu", "common.cuh"),
-        sha1="49dc56e530bf1481bf356ca09d0d136ab3caf701"),
+        bytes=104811776 + 20765440, per="launch", src=("prefill_tc.cu", "common.cuh"),
+        sha1="0a11e6db6fab1045752f3db57e190bbd825b7948"),
     "prefill_pythia160m_b8h12_s2048_d64_bf16": dict(
-        bytes=82398208 + 8301312, per="launch", src=("prefill_tc.cu", "common.cuh"),
-        sha1="49dc56e530bf1481bf356ca09d0d136ab3caf701"),
+        bytes=81602304 + 5924096, per="launch", src=("prefill_tc.cu", "common.cuh"),
+        sha1="0a11e6db6fab1045752f3db57e190bbd825b7948"),
+    "prefill_long_b1_s131072_d128_bf16": dict(
+        bytes=2237840128 + 1067599872, per="launch", src=("prefill_tc.cu", "common.cuh"),
+        sha1="0a11e6db6fab1045752f3db57e190bbd825b7948"),
 }
 
 

@@ -772,6 +772,13 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
   __syncthreads();
 
   int issued = 0;  // producer: chunks whose copies were started
+  // With more chunks than ring stages, the last (shortest) chunk is loaded
+  // first: its stage is released almost at once, so the copy of the chunk
+  // that has to wait for a free stage starts about one chunk earlier.  Flush
+  // steps keep the ascending order (the in-place moves rely on it), and so
+  // do the rotary and gather forms (their row state advances chunk by chunk).
+  const bool tail_first = !ROPE && !GATHER && !(FUSED && flush) && nchunks > kPipeStages;
+  auto chunk_of = [&](int ci) -> int { return tail_first ? (ci == 0 ? nchunks - 1 : ci - 1) : ci; };
   // consumer state.  O^T tiles: o[dt] holds dims 16dt + gq (+8) x heads
   // 2tq, 2tq + 1; the reference max of those two heads (equal across the
   // lanes of a column) and this lane's share of their sums.
@@ -793,14 +800,15 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
 #pragma unroll
       for (int u = 0; u < 2; ++u) hn[u] = 32 * u + lane < nr0 ? gr.row(rs + 32 * u + lane) : -1;
     }
-    for (int c = 0; c < nchunks; ++c) {
-      const int st = c % kPipeStages;
+    for (int ci = 0; ci < nchunks; ++ci) {
+      const int c = chunk_of(ci);
+      const int st = ci % kPipeStages;
       const int r0 = rs + c * ROWS;
       const int nr = re - r0 < ROWS ? re - r0 : ROWS;
       uint8_t* const kt = ring + st * SB;
       uint8_t* const vt = kt + NB * kTileBytes;
-      if (c >= kPipeStages &&
-          !__all_sync(0xffffffffu, sep::mbar_wait(&empty[st], ((c / kPipeStages) - 1) & 1, &abort_flag, p.err)))
+      if (ci >= kPipeStages &&
+          !__all_sync(0xffffffffu, sep::mbar_wait(&empty[st], ((ci / kPipeStages) - 1) & 1, &abort_flag, p.err)))
         break;
       if constexpr (GATHER) {
         // the chunk's kept rows by 16-byte copies: CH lanes per row (one
@@ -863,7 +871,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
           sep::tma_load_2d_hint(vt + j * kTileBytes, &map_v, 64 * j, static_cast<int32_t>(row0 + r0), &full[st], pol);
         }
       }
-      issued = c + 1;
+      issued = ci + 1;
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");  // before this warp's stores in the merge
   } else {
@@ -936,14 +944,15 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
           es[i] = make_float2(ck[i].y, ck[i].w);
         }
     }
-    for (int c = 0; c < nchunks; ++c) {
-      const int st = c % kPipeStages;
+    for (int ci = 0; ci < nchunks; ++ci) {
+      const int c = chunk_of(ci);
+      const int st = ci % kPipeStages;
       const int r0 = rs + c * ROWS;
       const int nr = re - r0 < ROWS ? re - r0 : ROWS;
       uint8_t* const kt = ring + st * SB;
       uint8_t* const vt = kt + NB * kTileBytes;
       if constexpr (ROPE) {
-        if (c > 0) {
+        if (c > 0) {  // (chunks in ascending order)
 #pragma unroll
           for (int i = 0; i < DT; ++i) {
             const int f = 16 * (i / 2) + 8 * (i & 1) + 2 * tq;
@@ -952,7 +961,7 @@ __global__ void __launch_bounds__(kPipeThreads, 2)
           }
         }
       }
-      if (!__all_sync(0xffffffffu, sep::mbar_wait(&full[st], (c / kPipeStages) & 1, &abort_flag, p.err)))
+      if (!__all_sync(0xffffffffu, sep::mbar_wait(&full[st], (ci / kPipeStages) & 1, &abort_flag, p.err)))
         break;
       if (kr < nr) {
         bool wrote = false;

@@ -372,6 +372,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       sep::tma_prefetch_desc(&tm_v);
       sep::tma_prefetch_desc(&tm_kc);
       sep::tma_prefetch_desc(&tm_vc);
+      // L2 policies: a Q tile is read once; the compact initial+separator
+      // rows of a (b, kv head) are read by every later tile of it, so they
+      // are kept over the streams of Q and of the outputs
+      const uint64_t pol_q = sep::l2_evict_first_policy();
+      const uint64_t pol_g = sep::l2_evict_last_policy();
       uint32_t gblk = 0, nitem = 0;
       int last_k[NST], last_v[NST];
       for (int s2 = 0; s2 < NST; ++s2) last_k[s2] = last_v[s2] = -1;
@@ -389,8 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* dst = smem + (t ? C::OFF_QB : C::OFF_QA);
 #pragma unroll
           for (int r = 0; r < D / 64; ++r)
-            sep::tma_load_2d(dst + r * C::REG, &tm_q, r * 64, static_cast<int32_t>(qrow),
-                             &bars->q_full);
+            sep::tma_load_2d_hint(dst + r * C::REG, &tm_q, r * 64, static_cast<int32_t>(qrow),
+                                  &bars->q_full, pol_q);
         }
         last_q = static_cast<int>(nitem);
         for (int j = 0; j < it.nblk; ++j, ++gblk) {
@@ -406,9 +411,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           sep::mbar_arrive_expect_tx(&bars->k_full[st], C::KV_BYTES);
 #pragma unroll
-          for (int r = 0; r < D / 64; ++r)
-            sep::tma_load_2d(smem + C::OFF_K + st * C::KV_BYTES + r * C::REG, gathered ? &tm_kc : &tm_k,
-                             r * 64, static_cast<int32_t>(row), &bars->k_full[st]);
+          for (int r = 0; r < D / 64; ++r) {
+            if (gathered)
+              sep::tma_load_2d_hint(smem + C::OFF_K + st * C::KV_BYTES + r * C::REG, &tm_kc, r * 64,
+                                    static_cast<int32_t>(row), &bars->k_full[st], pol_g);
+            else
+              sep::tma_load_2d(smem + C::OFF_K + st * C::KV_BYTES + r * C::REG, &tm_k, r * 64,
+                               static_cast<int32_t>(row), &bars->k_full[st]);
+          }
           last_k[st] = static_cast<int>(gblk);
           if (gblk >= static_cast<uint32_t>(NST) &&
               !mbar_wait(&bars->v_empty[st], (use - 1) & 1, abort, p.err)) {
@@ -417,9 +427,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           sep::mbar_arrive_expect_tx(&bars->v_full[st], C::KV_BYTES);
 #pragma unroll
-          for (int r = 0; r < D / 64; ++r)
-            sep::tma_load_2d(smem + C::OFF_V + st * C::KV_BYTES + r * C::REG, gathered ? &tm_vc : &tm_v,
-                             r * 64, static_cast<int32_t>(row), &bars->v_full[st]);
+          for (int r = 0; r < D / 64; ++r) {
+            if (gathered)
+              sep::tma_load_2d_hint(smem + C::OFF_V + st * C::KV_BYTES + r * C::REG, &tm_vc, r * 64,
+                                    static_cast<int32_t>(row), &bars->v_full[st], pol_g);
+            else
+              sep::tma_load_2d(smem + C::OFF_V + st * C::KV_BYTES + r * C::REG, &tm_v, r * 64,
+                               static_cast<int32_t>(row), &bars->v_full[st]);
+          }
           last_v[st] = static_cast<int>(gblk);
         }
       }
@@ -841,7 +856,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         sep::fence_proxy_async_smem();
         sep::named_bar_sync(1 + t, 128);
         if (row == 0) {
-          sep::tma_store_2d(&tm_o, 0, static_cast<int32_t>(static_cast<int64_t>(b * p.Hq + h) * p.S + my_q0), stg);
+          sep::tma_store_2d_hint(&tm_o, 0, static_cast<int32_t>(static_cast<int64_t>(b * p.Hq + h) * p.S + my_q0),
+                                 stg, sep::l2_evict_first_policy());
           sep::bulk_commit();
         }
       } else {
@@ -859,14 +875,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             w.y = sep::pack_bf16x2(__uint_as_float(o[8 * q + 2]) * inv, __uint_as_float(o[8 * q + 3]) * inv);
             w.z = sep::pack_bf16x2(__uint_as_float(o[8 * q + 4]) * inv, __uint_as_float(o[8 * q + 5]) * inv);
             w.w = sep::pack_bf16x2(__uint_as_float(o[8 * q + 6]) * inv, __uint_as_float(o[8 * q + 7]) * inv);
-            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q) = w;
+            __stcs(reinterpret_cast<uint4*>(orow + 32 * c + 8 * q), w);  // streamed out
           }
         }
       }
       }
       if (p.lse && i < p.S)
-        p.lse[static_cast<int64_t>(b * p.Hq + h) * p.S + i] =
-            (m_ref + __log2f(l)) * 0.69314718055994530942f;
+        __stcs(p.lse + static_cast<int64_t>(b * p.Hq + h) * p.S + i, (m_ref + __log2f(l)) * 0.69314718055994530942f);
       sep::tc_fence_before();
       sep::mbar_arrive(&bars->o_empty[t]);
     }
