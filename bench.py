@@ -71,8 +71,8 @@ def _peaks():
 # proportion to the retained rows).
 TRAFFIC = {
     "decode_llama3_8b_b16_l32_t65536_d128_bf16": dict(
-        bytes=(28613888 + 1536) / (420.5 * 16), per="row", src=("decode.cu", "common.cuh"),
-        sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
+        bytes=(28617472 + 0) / (420.5 * 16), per="row", src=("decode.cu", "common.cuh"),
+        sha1="15a13239d28cd65b3fab191c803aa3c5a4c49bee"),
     "decode_rope_llama3_8b_b16_l32_t65536_d128_bf16": dict(
         bytes=(28885248 + 0) / (421.19 * 16), per="row", src=("decode.cu", "common.cuh"),
         sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
@@ -80,11 +80,11 @@ TRAFFIC = {
         bytes=69485568 + 1160448, per="launch", src=("decode.cu", "common.cuh"),
         sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
     "backward_llama3_8b_b1_s8192_d128_bf16": dict(
-        bytes=223200000 + 208900000, per="launch", src=("backward.cu", "common.cuh"),
-        sha1="ccc1d51920b8eb0ffa71d1c0b81985af9610007c"),
+        bytes=498886144 + 68659200, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="11bd4cf8a0687eacce0e46894d94b9b4981cc760"),
     "backward_pythia160m_b8h12_s2048_d64_bf16": dict(
-        bytes=161018624 + 101916928, per="launch", src=("backward.cu", "common.cuh"),
-        sha1="ccc1d51920b8eb0ffa71d1c0b81985af9610007c"),
+        bytes=288590848 + 31880192, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="11bd4cf8a0687eacce0e46894d94b9b4981cc760"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
         bytes=104811776 + 20765440, per="launch", src=("prefill_tc.cu", "common.cuh"),
         sha1="0a11e6db6fab1045752f3db57e190bbd825b7948"),
@@ -861,15 +861,12 @@ def bench_backward(sl, args, world, rank):
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16"],
                      "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4),
                      "traffic": _traffic(name, units=1), "launch_us": round(step_s * 1e6, 3),
-                     "kernel": ("sep_attn_backward: delta pass, k_sep_bwd_tc_kv (dK, dV) + "
-                                "k_sep_bwd_tc_q (dQ) on tcgen05, fp32 -> bf16 pass; traffic = "
-                                "the two tcgen05 kernels" if D == 128 else
-                                "sep_attn_backward: delta pass, k_sep_bwd on warp-level mma.sync, "
-                                "fp32 -> bf16 pass; traffic = k_sep_bwd"),
+                     "kernel": ("sep_attn_backward: delta pass, separator-row gather, "
+                                "k_bwd_kv (dK, dV) + k_bwd_q (dQ) on tcgen05, separator-key "
+                                "scatter; traffic = all five launches"),
                      "peak_source": pk["src"] + " bf16 dense burst"},
         "e2e": e2e, "clocks": clk,
-        # D = 128: delta, two tcgen05 kernels, two conversions; D = 64: delta, one
-        # kernel, three conversions (plus one memset either way)
+        # delta, gather, two tcgen05 kernels, scatter
         "gpu_launches": 5 * K,
     }
     if rank == 0 and world == 1 and not args.skip_cpu:

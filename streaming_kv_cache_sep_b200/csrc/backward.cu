@@ -1,5 +1,4 @@
-// Sep-Attention backward (bf16, D in {64, 128}): warp-level tensor cores
-// (mma.sync) for D = 64, tcgen05 for D = 128 (second part of this file).
+// Sep-Attention backward (bf16, D in {64, 128}) on tcgen05 tensor cores.
 //
 // Gradients of sum(out * dout) through the prefill's sparse attention (the
 // training use of Sep-Attention: "HKUDS047: SepLLM ..." study, section on the
@@ -10,24 +9,17 @@
 //   dv_j += p_ij dout_i,   ds_ij = p_ij (dout_i . v_j - delta_i),
 //   dk_j += scale ds_ij q_i,   dq_i += scale ds_ij k_j.
 //
-// Key-centric work split.  The kept pairs fall into two disjoint families:
+// Key-centric work split for dK and dV.  The kept pairs fall into two
+// disjoint families:
 //   * global keys (j < a or a separator) are kept by every query i >= j;
-//     they are taken 64 at a time from the separator index list, and each
-//     block visits the query tiles after its first position, at most
-//     kChunkTiles tiles per CTA;
+//     they are taken 128 at a time from the compact list of global keys, and
+//     each block visits the query tiles after its first position, at most
+//     kTcChunkTiles tiles per CTA;
 //   * local keys (all others) are kept only by queries i in [j, j + n); they
-//     are taken as 64 consecutive positions, and each block visits the query
+//     are taken as 128 consecutive positions, and each block visits the query
 //     tiles that reach it, with the global keys of the block masked out.
-// A CTA (four warps, one work item) keeps its 64 keys' K and V in shared
-// memory and the dK and dV of its keys in registers (warp w: keys 16w ..
-// 16w + 15) over all query heads of the kv group and all its query tiles.
-// Per 64-row query tile the warps form S^T = K Q^T and dP^T = V dO^T for
-// their keys (the keys as the 16 rows of the mma tile), P and dS in
-// registers, dV += P^T dO and dK += dS^T Q; dS goes to shared memory and each
-// warp then forms dQ for 16 queries (dS K) and adds it into an fp32
-// accumulator with vector reductions.  At the end the item adds its dK and
-// dV into fp32 accumulators.  A delta pass runs before, and a pass after
-// converts the accumulators (times scale for dq and dk) to bf16.
+// dQ is query-centric: each CTA owns 128 queries of one head and visits the
+// key blocks its tile keeps.  A delta pass runs first.
 #include <string.h>
 
 #include "common.cuh"
@@ -35,45 +27,6 @@
 
 namespace {
 
-constexpr int BR = 64;          // query rows per tile
-constexpr int BC = 64;          // keys per work item
-constexpr int kThreads = 128;   // four warps
-constexpr int kChunkTiles = 4;  // query tiles per item of global keys (measured: 4 < 8 < 16)
-constexpr int kTileBytes = 64 * 128;  // 64 rows x 64 bf16, 128-byte swizzled
-
-// Byte offset of (row r, element d) in a tensor's D/64 swizzled 64-row tiles.
-__device__ __forceinline__ uint32_t swz(int r, int d) {
-  return static_cast<uint32_t>((d >> 6) * kTileBytes + r * 128 +
-                               ((((d >> 3) & 7) ^ (r & 7)) << 4) + (d & 7) * 2);
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(addr));
-}
-// c (16x8 fp32) += a (16x16 bf16, row-major fragment) * b (16x8 bf16, col fragment)
-__device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-      "{%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 __device__ __forceinline__ void red_add_v2(float* p, float x, float y) {
   asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(p), "f"(x), "f"(y) : "memory");
 }
@@ -84,11 +37,11 @@ struct BwdParams {
   const float* delta;  // [B][Hq][S]
   const uint8_t* is_sep;
   const int32_t *prefix, *idx;
-  float *dq_acc, *dk_acc, *dv_acc;
+  float *dk_acc, *dv_acc;  // fp32 dK, dV rows of the compact global-key lists
   int32_t* err;
   int B, Hq, Hkv, S, a, n;
-  int nwin;     // window items per (b, kv head) = ceil(S / 64)
-  int nchunk;   // chunks per block of global keys = ceil(ceil(S / 64) / kChunkTiles)
+  int nwin;    // window items per (b, kv head) = ceil(S / 128)
+  int nchunk;  // chunks per block of global keys = ceil(ceil(S / 128) / kTcChunkTiles)
   float scale_log2;
 };
 
@@ -111,335 +64,50 @@ __global__ void k_bwd_delta(const __nv_bfloat16* __restrict__ out,
   if (lane == 0) delta[row] = acc;
 }
 
-// fp32 accumulators -> bf16 gradients (dq, dk scaled)
-__global__ void k_bwd_convert(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dst,
-                              int64_t n4, float mul) {
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const float4 x = reinterpret_cast<const float4*>(acc)[i];
-    __nv_bfloat162 lo = __floats2bfloat162_rn(x.x * mul, x.y * mul);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(x.z * mul, x.w * mul);
-    uint2 u;
-    u.x = *reinterpret_cast<uint32_t*>(&lo);
-    u.y = *reinterpret_cast<uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(dst)[i] = u;
-  }
-}
-
-// Shared memory of one CTA (dynamic): K, V [64][D]; Q, dO [2][64][D]; dS^T
-// [64 keys][64 queries], all bf16 swizzled; then the per-tile and per-key
-// scalars.
-template <int D>
-struct Smem {
-  static constexpr int T = (D / 64) * kTileBytes;  // one 64-row tensor
-  static constexpr int K = 0, V = T, Q = 2 * T, DO = 4 * T, DS = 6 * T;
-  static constexpr int LSE = DS + kTileBytes;      // [2][64] fp32 (log2 domain)
-  static constexpr int DEL = LSE + 2 * 64 * 4;     // [2][64] fp32
-  static constexpr int POS = DEL + 2 * 64 * 4;     // [64] int32 key positions
-  static constexpr int LOCAL = POS + 64 * 4;       // [64] int32: key may be used
-  static constexpr int BYTES = LOCAL + 64 * 4;
-};
-
-// D = 64 fits three CTAs per SM (registers <= 168), D = 128 two
-template <int D>
-__global__ void __launch_bounds__(kThreads, D == 64 ? 3 : 2) k_sep_bwd(const BwdParams p) {
-  constexpr int DT = D / 16, NT = D / 8;
-  using SM = Smem<D>;
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const uint32_t sbase = sep::smem_u32(smem);
-  float* const lse_s = reinterpret_cast<float*>(smem + SM::LSE);
-  float* const del_s = reinterpret_cast<float*>(smem + SM::DEL);
-  int32_t* const pos_s = reinterpret_cast<int32_t*>(smem + SM::POS);
-  int32_t* const use_s = reinterpret_cast<int32_t*>(smem + SM::LOCAL);
-
-  const int item = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gq = lane >> 2, tq = lane & 3;
-  const int S = p.S, G = p.Hq / p.Hkv;
-  const int nT = (S + BR - 1) / BR;
-  const int32_t* pre = p.prefix + static_cast<int64_t>(b) * (S + 1);
-  const int32_t* ix = p.idx + static_cast<int64_t>(b) * S;
-  const uint8_t* fl = p.is_sep + static_cast<int64_t>(b) * S;
-  const int a0 = p.a < S ? p.a : S;
-  const int nglob = a0 + (pre[S] - pre[a0]);  // global keys: initial, then separators >= a
-
-  // ---- the item: its keys and its query tiles
-  const bool window = item < p.nwin;
-  int kb, t0, t1;
-  if (window) {
-    kb = item;
-    t0 = kb;  // queries from the block's first key on
-    const int last = kb * BC + BC - 1 + p.n - 1;  // the last query a key of the block can reach
-    t1 = (last < S - 1 ? last : S - 1) / BR + 1;
-  } else {
-    kb = (item - p.nwin) / p.nchunk;
-    const int chunk = (item - p.nwin) % p.nchunk;
-    if (kb * BC >= nglob) return;
-    const int t = kb * BC;
-    const int pmin = t < a0 ? t : ix[pre[a0] + t - a0];
-    t0 = pmin / BR + chunk * kChunkTiles;
-    t1 = t0 + kChunkTiles < nT ? t0 + kChunkTiles : nT;
-    if (t0 >= nT) return;
-  }
-  // key positions and whether a key takes part in this item's pairs
-  if (threadIdx.x < BC) {
-    const int r = threadIdx.x;
-    int pos = -1, use = 0;
-    if (window) {
-      pos = kb * BC + r;
-      use = pos < S && !(pos < p.a || fl[pos]);  // local keys only
-      if (pos >= S) pos = -1;
-    } else {
-      const int t = kb * BC + r;
-      if (t < nglob) {
-        pos = t < a0 ? t : ix[pre[a0] + t - a0];
-        use = 1;
-      }
-    }
-    pos_s[r] = pos;
-    use_s[r] = use;
-  }
-  __syncthreads();
-  // K and V rows of the block (zero rows where there is no key)
-  const int64_t kvrow0 = (static_cast<int64_t>(b) * p.Hkv + g) * S;
-  for (int e = threadIdx.x; e < BC * (D / 8); e += kThreads) {
-    const int r = e / (D / 8), c = e % (D / 8);
-    const int pos = pos_s[r];
-    const int64_t off = (kvrow0 + (pos < 0 ? 0 : pos)) * D + 8 * c;
-    const uint32_t nb = pos < 0 ? 0u : 16u;
-    cp_async16(sbase + SM::K + swz(r, 8 * c), p.k + off, nb);
-    cp_async16(sbase + SM::V + swz(r, 8 * c), p.v + off, nb);
-  }
-  cp_async_commit();
-
-  // the visits: (head, query tile) pairs, heads outer
-  const int ntile = t1 - t0;
-  const int nvisit = G * ntile;
-  auto load_visit = [&](int v, int buf) {
-    const int h = g * G + v / ntile, t = t0 + v % ntile;
-    const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
-    for (int e = threadIdx.x; e < BR * (D / 8); e += kThreads) {
-      const int r = e / (D / 8), c = e % (D / 8);
-      const int i = t * BR + r;
-      const int64_t off = (qrow0 + (i < S ? i : 0)) * D + 8 * c;
-      const uint32_t nb = i < S ? 16u : 0u;
-      cp_async16(sbase + SM::Q + buf * SM::T + swz(r, 8 * c), p.q + off, nb);
-      cp_async16(sbase + SM::DO + buf * SM::T + swz(r, 8 * c), p.dout + off, nb);
-    }
-    if (threadIdx.x < BR) {
-      const int i = t * BR + threadIdx.x;
-      lse_s[buf * 64 + threadIdx.x] = i < S ? p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
-      del_s[buf * 64 + threadIdx.x] = i < S ? p.delta[qrow0 + i] : 0.f;
-    }
-    cp_async_commit();
-  };
-  if (nvisit > 0) load_visit(0, 0);
-
-  float dk[NT][4], dv[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) dk[nt][e] = dv[nt][e] = 0.f;
-
-  const int kr = 16 * warp;  // this warp's keys
-  for (int v = 0; v < nvisit; ++v) {
-    const int buf = v & 1;
-    const int h = g * G + v / ntile, t = t0 + v % ntile;
-    const int i0 = t * BR;
-    if (v + 1 < nvisit) {
-      load_visit(v + 1, buf ^ 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();  // this visit's tiles (and K, V) are in shared memory
-    const uint32_t qs = sbase + SM::Q + buf * SM::T, ds_ = sbase + SM::DO + buf * SM::T;
-    const uint32_t ks = sbase + SM::K, vs = sbase + SM::V, dss = sbase + SM::DS;
-    const float* lse2 = lse_s + buf * 64;
-    const float* del = del_s + buf * 64;
-    // key rows of this lane: kr + gq and kr + gq + 8
-    const int jp0 = pos_s[kr + gq], jp1 = pos_s[kr + gq + 8];
-    const int u0 = use_s[kr + gq], u1 = use_s[kr + gq + 8];
-    // the warp's last key position: a global-key item keeps every valid key
-    // for queries after it, so those sub-blocks need no element mask
-    int jmax = jp0 > jp1 ? jp0 : jp1;
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) jmax = max(jmax, __shfl_xor_sync(0xffffffffu, jmax, off));
-    // ---------------- phase A: 16 queries at a time
-#pragma unroll 1
-    for (int sb = 0; sb < BR / 16; ++sb) {
-      float s[2][4] = {}, dp[2][4] = {};
-#pragma unroll
-      for (int kk = 0; kk < DT; ++kk) {
-        uint32_t ka[4], va[4], qb[4], ob[4];
-        ldsm_x4(ks + swz(kr + (lane & 7) + ((lane >> 3) & 1) * 8, 16 * kk + (lane >> 4) * 8), ka);
-        ldsm_x4(vs + swz(kr + (lane & 7) + ((lane >> 3) & 1) * 8, 16 * kk + (lane >> 4) * 8), va);
-        // B = Q^T / dO^T: matrices (queries 0-7 | 8-15) x (dims 16kk | 16kk+8)
-        const int qr = 16 * sb + (lane & 7) + (lane >> 4) * 8, qc = 16 * kk + ((lane >> 3) & 1) * 8;
-        ldsm_x4(qs + swz(qr, qc), qb);
-        ldsm_x4(ds_ + swz(qr, qc), ob);
-        mma16816(s[0], ka, qb[0], qb[1]);
-        mma16816(s[1], ka, qb[2], qb[3]);
-        mma16816(dp[0], va, ob[0], ob[1]);
-        mma16816(dp[1], va, ob[2], ob[3]);
-      }
-      // P and dS: element e of n-tile nt is key kr + gq (+8 for e >= 2),
-      // query 16sb + 8nt + 2tq + (e & 1)
-      uint32_t pa[4], sa[4];
-      // (D = 128 runs at the register limit, where the extra path costs more
-      // than it saves: measured)
-      const bool all_kept = D == 64 && !window && i0 + 16 * sb >= jmax && i0 + 16 * sb + 15 < S;
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        float pv[4], dsv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int q = 16 * sb + 8 * nt + 2 * tq + (e & 1);
-          const int i = i0 + q;
-          const int j = e < 2 ? jp0 : jp1;
-          const int use = e < 2 ? u0 : u1;
-          bool kept;
-          if (all_kept) {
-            kept = use;
-          } else {
-            kept = use && j >= 0 && i < S && j <= i;
-            if (window) kept = kept && i - j < p.n;
-          }
-          const float pe = kept ? exp2f(s[nt][e] * p.scale_log2 - lse2[q]) : 0.f;
-          pv[e] = pe;
-          dsv[e] = pe * (dp[nt][e] - del[q]);
-        }
-        pa[2 * nt] = sep::pack_bf16x2(pv[0], pv[1]);
-        pa[2 * nt + 1] = sep::pack_bf16x2(pv[2], pv[3]);
-        sa[2 * nt] = sep::pack_bf16x2(dsv[0], dsv[1]);
-        sa[2 * nt + 1] = sep::pack_bf16x2(dsv[2], dsv[3]);
-        // dS^T to shared memory: rows keys, columns queries
-        const int q0 = 16 * sb + 8 * nt + 2 * tq;
-        *reinterpret_cast<uint32_t*>(smem + SM::DS + swz(kr + gq, q0)) = sa[2 * nt];
-        *reinterpret_cast<uint32_t*>(smem + SM::DS + swz(kr + gq + 8, q0)) = sa[2 * nt + 1];
-      }
-      // A fragments of P^T / dS^T (keys x 16 queries): registers 0, 1 of
-      // n-tile 0 and 0, 1 of n-tile 1
-      const uint32_t ap[4] = {pa[0], pa[1], pa[2], pa[3]};
-      const uint32_t as[4] = {sa[0], sa[1], sa[2], sa[3]};
-      // dV += P^T dO, dK += dS^T Q: B = dO / Q (queries x dims) by ldmatrix.trans
-#pragma unroll
-      for (int dn = 0; dn < NT; dn += 2) {
-        uint32_t ob[4], qb[4];
-        const int rr = 16 * sb + (lane & 7) + ((lane >> 3) & 1) * 8, cc = 8 * dn + (lane >> 4) * 8;
-        ldsm_x4_t(ds_ + swz(rr, cc), ob);
-        ldsm_x4_t(qs + swz(rr, cc), qb);
-        mma16816(dv[dn], ap, ob[0], ob[1]);
-        mma16816(dv[dn + 1], ap, ob[2], ob[3]);
-        mma16816(dk[dn], as, qb[0], qb[1]);
-        mma16816(dk[dn + 1], as, qb[2], qb[3]);
-      }
-    }
-    __syncthreads();  // dS^T of all keys is in shared memory
-    // ---------------- phase B: dQ of queries 16w .. 16w + 15 = dS K, one
-    // half of the dims at a time (half the accumulator registers)
-    {
-      const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
-#pragma unroll 1
-      for (int dh = 0; dh < 2; ++dh) {
-        float dq[NT / 2][4];
-#pragma unroll
-        for (int nt = 0; nt < NT / 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) dq[nt][e] = 0.f;
-#pragma unroll
-        for (int kt = 0; kt < BC / 16; ++kt) {
-          // A = dS (queries x keys) from dS^T by ldmatrix.trans: matrices
-          // (keys 16kt | +8) x (queries 16w | +8)
-          uint32_t aa[4];
-          {
-            const int m = lane >> 3, r = lane & 7;
-            const int key = 16 * kt + (m >> 1) * 8 + r, q = 16 * warp + (m & 1) * 8;
-            ldsm_x4_t(dss + swz(key, q), aa);
-          }
-#pragma unroll
-          for (int dn = 0; dn < NT / 2; dn += 2) {
-            // B = K (keys x dims) by ldmatrix.trans: matrices (keys | +8) x (dims | +8)
-            uint32_t kb4[4];
-            const int m = lane >> 3, r = lane & 7;
-            const int key = 16 * kt + (m & 1) * 8 + r, d = 8 * (dh * (NT / 2) + dn) + (m >> 1) * 8;
-            ldsm_x4_t(ks + swz(key, d), kb4);
-            mma16816(dq[dn], aa, kb4[0], kb4[1]);
-            mma16816(dq[dn + 1], aa, kb4[2], kb4[3]);
-          }
-        }
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int i = i0 + 16 * warp + gq + 8 * half;
-          if (i < S) {
-            float* dst = p.dq_acc + (qrow0 + i) * D + (D / 2) * dh + 2 * tq;
-#pragma unroll
-            for (int nt = 0; nt < NT / 2; ++nt) red_add_v2(dst + 8 * nt, dq[nt][2 * half], dq[nt][2 * half + 1]);
-          }
-        }
-      }
-    }
-    __syncthreads();  // the buffers of this visit may be refilled
-  }
-  // ---------------- the item's dK and dV
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int key = kr + gq + 8 * half;
-    const int j = pos_s[key];
-    if (j >= 0 && use_s[key]) {
-      float* dkp = p.dk_acc + (kvrow0 + j) * D + 2 * tq;
-      float* dvp = p.dv_acc + (kvrow0 + j) * D + 2 * tq;
-      if (window) {  // a local key's pairs all belong to this item: plain stores
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          *reinterpret_cast<float2*>(dkp + 8 * nt) = make_float2(dk[nt][2 * half], dk[nt][2 * half + 1]);
-          *reinterpret_cast<float2*>(dvp + 8 * nt) = make_float2(dv[nt][2 * half], dv[nt][2 * half + 1]);
-        }
-      } else {  // global keys: one item per chunk of query tiles
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          red_add_v2(dkp + 8 * nt, dk[nt][2 * half], dk[nt][2 * half + 1]);
-          red_add_v2(dvp + 8 * nt, dv[nt][2 * half], dv[nt][2 * half + 1]);
-        }
-      }
-    }
-  }
-}
-
 // ---------------------------------------------------------------------------
-// tcgen05 form (D = 128), two kernels on the operand forms of the forward:
-//   k_sep_bwd_tc_kv (key-centric, 128 keys in TMEM lanes, 128-query tiles,
-//     Q and dO double-buffered): S^T = K Q^T and dP^T = V dO^T (SS); warps
-//     0-3 (thread = key row) turn them into P^T and dS^T, written back as
-//     bf16 over the first 64 columns of each; dV += P^T dO and dK += dS^T Q
-//     (TS, B MN-major).  TMEM: S^T [0,128) dP^T [128,256) dV [256,384)
-//     dK [384,512).
-//   k_sep_bwd_tc_q (query-centric, 128 queries in TMEM lanes, over the kept
-//     key blocks of its tile as the forward does: the global keys before the
-//     window unmasked, then the window blocks with the element mask; K and V
-//     double-buffered): S = Q K^T and dP = dO V^T (SS); thread = query row
-//     forms dS, written back as bf16; dQ += dS K (TS, B = K MN-major).  The
-//     CTA owns its queries, so dQ is stored once, as bf16, with no
-//     reduction.  TMEM: S [0,128) dP [128,256) dQ [256,384).
-// Warps 0-7 share the 128 TMEM lanes two by two (warp w: lanes 32 (w & 3) ..
-// +31, columns [64 (w >> 2), +64) of each 128-column tile); the two warps of
-// a lane quarter load all their scores before either stores the bf16 P / dS
-// over them.  Warp 8 allocates TMEM; its lane 0 issues the MMAs (and, in the
-// key-centric kernel, the tensor copies of the Q and dO tiles) while the
-// other lanes wait for it, and the warp reaches the block barrier together.
-constexpr int TBK = 128;  // keys per block (TMEM lanes of the key-centric kernel)
+// Two software-pipelined tcgen05 kernels on the operand forms of the forward.
+//   k_bwd_kv (key-centric, 128 keys in TMEM lanes, K and V resident): in
+//     units of 64 queries of one head (each unit's Q and dO rows stream
+//     through a ring of kNst shared-memory stages filled by the tensor-copy
+//     engine): S^T = K Q^T and dP^T = V dO^T (SS, N = 64) into one of two
+//     score buffers; the compute warps turn them into P^T and dS^T, written
+//     back as bf16 over the first 16 columns of each warp's 32; then
+//     dV += P^T dO and dK += dS^T Q (TS, B MN-major).  The MMA warp issues
+//     the scores of unit u before the gradient products of unit u-1, so the
+//     tensor pipe computes while the compute warps work on the other
+//     buffer.  TMEM: S0 [0,64) dP0 [64,128) S1 [128,192) dP1 [192,256)
+//     dV [256,256+D) dK [256+D,256+2D).
+//   k_bwd_q (query-centric, 128 queries in TMEM lanes, Q and dO resident):
+//     over the kept key blocks of its tile as the forward does -- the global
+//     keys before the window from the compact list, then the window blocks
+//     with the element mask -- in units of 64 keys streamed through the
+//     ring: S = Q K^T and dP = dO V^T (SS), dS written back as bf16,
+//     dQ += dS K (TS, B = K MN-major).  The CTA owns its queries, so dQ is
+//     stored once, as bf16.  TMEM: S0 dP0 S1 dP1 as above, dQ [256, 256+D).
+// Warps 0-7 are the compute warps (warp w: TMEM lanes 32 (w & 3) .. +31,
+// columns [32 (w >> 2), +32) of each 64-column score tile), warp 8
+// allocates TMEM and its lane 0 issues the MMAs, warp 9 issues the tensor
+// copies and stages the per-unit statistics (key-centric) or global-flag
+// words (query-centric).  A ring stage is released by the commit of the
+// last product that reads it.  Every wait is bounded.
+//
+// Key rows: the global keys (initial tokens and separators) are read from a
+// compact copy [B, Hkv, S, D] (k_bwd_prep), so every K/V block is one
+// tensor copy.  Window keys' dK and dV are owned by one item and stored as
+// bf16; the global keys' partial sums go to fp32 rows of the compact list
+// (zeroed by k_bwd_prep) and k_bwd_scatter writes them to their positions.
+
+constexpr int TBK = 128;  // keys per block
 constexpr int TBQ = 128;  // queries per tile
-constexpr int kTcThreads = 288;  // warps 0-7: softmax, loads, readout; warp 8: TMEM and MMA issue
-constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDQ = 256;
+constexpr int kTcThreads = 320;
+constexpr int kNst = 4;           // stages of the 64-row operand ring
+constexpr int kT64 = 64 * 128;    // one 64-row x 64-column swizzled tile
+constexpr uint32_t kColAcc = 256;    // dV (key-centric) / dQ (query-centric)
 template <int D>
-constexpr uint32_t col_dk() { return kColDV + D; }  // dK after the D columns of dV
+constexpr uint32_t col_dk() { return kColAcc + D; }  // dK after the D columns of dV
 constexpr int kT128 = 128 * 128;  // one 128-row x 64-column swizzled tile
 constexpr int kTcChunkTiles = 4;  // query tiles per item of global keys
 
-__device__ __forceinline__ uint32_t swz128(int r, int d) {
-  return static_cast<uint32_t>((d >> 6) * kT128 + r * 128 + ((((d >> 3) & 7) ^ (r & 7)) << 4) +
-                               (d & 7) * 2);
-}
 // packed fp32 pairs (one f32x2 instruction per pair)
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   float2 d;
@@ -464,63 +132,207 @@ __device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
 __host__ __device__ constexpr uint32_t idesc_mn(int M, int N, bool a_mn, bool b_mn) {
   return sep::idesc_bf16_f32(M, N, b_mn) | ((a_mn ? 1u : 0u) << 15);
 }
-// Rows [0, 128) of a [rows, D] bf16 tensor into D/64 swizzled 128-row
-// tiles, one 16-byte chunk per copy; row_of(r) < 0 gives a zero row.
-template <int D, typename RowOf>
-__device__ __forceinline__ void load_rows(uint32_t dst, const __nv_bfloat16* src, RowOf row_of,
-                                          int tid, int nthreads) {
-  constexpr int CH = D / 8;  // 16-byte chunks per row
-  for (int e = tid; e < 128 * CH; e += nthreads) {
-    const int r = e / CH, c = e % CH;
-    const int64_t row = row_of(r);
-    cp_async16(dst + swz128(r, 8 * c), src + (row < 0 ? 0 : row) * D + 8 * c, row < 0 ? 0u : 16u);
+// TMEM column of the bf16 operand of k-step kk (16 rows of K) of a unit
+// whose values were stored by the compute warps at [base + 32 ch, +16)
+__device__ __forceinline__ uint32_t unit_acol(uint32_t base, int kk) {
+  return base + 32u * static_cast<uint32_t>(kk >> 1) + 8u * static_cast<uint32_t>(kk & 1);
+}
+// 128 rows starting at `row` of a [rows, D] tensor map into NB 64-column
+// swizzled tiles at `dst`, completing on `bar`
+template <int D>
+__device__ __forceinline__ void load_tile128(uint8_t* dst, const CUtensorMap* map, int32_t row,
+                                             uint64_t* bar) {
+#pragma unroll
+  for (int c = 0; c < D / 64; ++c) sep::tma_load_2d(dst + c * kT128, map, 64 * c, row, bar);
+}
+
+// The compact list of global keys of (b, kv head): initial tokens [0,
+// min(a, S)), then separators at positions >= a, in order.
+struct GlobalList {
+  const int32_t* pre;
+  const int32_t* ix;
+  int a0, total;
+  __device__ GlobalList(const BwdParams& p, int b) {
+    pre = p.prefix + static_cast<int64_t>(b) * (p.S + 1);
+    ix = p.idx + static_cast<int64_t>(b) * p.S;
+    a0 = p.a < p.S ? p.a : p.S;
+    total = a0 + (pre[p.S] - pre[a0]);
+  }
+  __device__ int pos(int t) const { return t < a0 ? t : ix[pre[a0] + t - a0]; }
+};
+
+// Copies the global keys' K/V rows into the compact buffers (rows past the
+// list and up to the next multiple of 128, at least 128 and at most S, are
+// zero-filled so whole tiles read finite values) and zeroes the fp32
+// dK/dV rows of the list.  One CTA per 64 rows of (b, kv head).
+template <int D>
+__global__ void __launch_bounds__(256) k_bwd_prep(const BwdParams p, __nv_bfloat16* __restrict__ kc,
+                                                  __nv_bfloat16* __restrict__ vc) {
+  constexpr int CH = D / 8;  // 16-byte chunks per bf16 row
+  const int g = blockIdx.y, b = blockIdx.z, r0 = blockIdx.x * 64;
+  const GlobalList gl(p, b);
+  int lim = (gl.total + TBK - 1) / TBK * TBK;
+  if (lim < TBK) lim = TBK;
+  if (lim > p.S) lim = p.S;
+  if (r0 >= lim) return;
+  const int64_t base = (static_cast<int64_t>(b) * p.Hkv + g) * p.S;
+  for (int e = threadIdx.x; e < 64 * CH; e += 256) {
+    const int r = r0 + e / CH, c = e % CH;
+    if (r >= lim) break;
+    uint4 kv = make_uint4(0, 0, 0, 0), vv = make_uint4(0, 0, 0, 0);
+    if (r < gl.total) {
+      const int pos = gl.pos(r);
+      if (pos >= 0 && pos < p.S) {
+        kv = reinterpret_cast<const uint4*>(p.k + (base + pos) * D)[c];
+        vv = reinterpret_cast<const uint4*>(p.v + (base + pos) * D)[c];
+      } else {
+        atomicOr(p.err, sep::ERR_BAD_INDEX);
+      }
+      const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+      reinterpret_cast<float4*>(p.dk_acc + (base + r) * D)[2 * c] = z;
+      reinterpret_cast<float4*>(p.dk_acc + (base + r) * D)[2 * c + 1] = z;
+      reinterpret_cast<float4*>(p.dv_acc + (base + r) * D)[2 * c] = z;
+      reinterpret_cast<float4*>(p.dv_acc + (base + r) * D)[2 * c + 1] = z;
+    }
+    reinterpret_cast<uint4*>(kc + (base + r) * D)[c] = kv;
+    reinterpret_cast<uint4*>(vc + (base + r) * D)[c] = vv;
   }
 }
 
-// NB = D/64 tiles of 128 rows x 64 columns per 128-row tensor
+// The global keys' fp32 dK (times scale) and dV sums -> bf16 rows at their
+// positions.
+template <int D>
+__global__ void __launch_bounds__(256) k_bwd_scatter(const BwdParams p, float scale,
+                                                     __nv_bfloat16* __restrict__ dk,
+                                                     __nv_bfloat16* __restrict__ dv) {
+  constexpr int CH = D / 8;
+  const int g = blockIdx.y, b = blockIdx.z, r0 = blockIdx.x * 64;
+  const GlobalList gl(p, b);
+  if (r0 >= gl.total) return;
+  const int64_t base = (static_cast<int64_t>(b) * p.Hkv + g) * p.S;
+  for (int e = threadIdx.x; e < 64 * CH; e += 256) {
+    const int r = r0 + e / CH, c = e % CH;
+    if (r >= gl.total) break;
+    const int pos = gl.pos(r);
+    if (pos < 0 || pos >= p.S) continue;  // flagged by k_bwd_prep
+    const float4* ks = reinterpret_cast<const float4*>(p.dk_acc + (base + r) * D) + 2 * c;
+    const float4* vs = reinterpret_cast<const float4*>(p.dv_acc + (base + r) * D) + 2 * c;
+    const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
+    reinterpret_cast<uint4*>(dk + (base + pos) * D)[c] =
+        make_uint4(sep::pack_bf16x2(k0.x * scale, k0.y * scale), sep::pack_bf16x2(k0.z * scale, k0.w * scale),
+                   sep::pack_bf16x2(k1.x * scale, k1.y * scale), sep::pack_bf16x2(k1.z * scale, k1.w * scale));
+    reinterpret_cast<uint4*>(dv + (base + pos) * D)[c] =
+        make_uint4(sep::pack_bf16x2(v0.x, v0.y), sep::pack_bf16x2(v0.z, v0.w),
+                   sep::pack_bf16x2(v1.x, v1.y), sep::pack_bf16x2(v1.z, v1.w));
+  }
+}
+
+// Bounded wait by every lane of a warp on the same phase; true on all lanes
+// or on none.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          int32_t* err) {
+  const bool ok = sep::mbar_wait(bar, parity, abort, err);
+  return __all_sync(0xffffffffu, ok);
+}
+// Adds `bytes` of expected tensor-copy data to the current phase of `bar`
+// without an arrival.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(sep::smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+// Bits [a, b) of a 32-bit word, a and b clamped to [0, 32].
+__device__ __forceinline__ uint32_t bit_range(int a, int b) {
+  a = a < 0 ? 0 : (a > 32 ? 32 : a);
+  b = b < 0 ? 0 : (b > 32 ? 32 : b);
+  if (b <= a) return 0u;
+  const uint32_t hi = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+  return hi & ~((1u << a) - 1u);
+}
+// One thread's 32 scores s and dP of a unit -> P = 2^(s scale_log2 + nl)
+// and dS = P (dP - dl), each packed to bf16 pairs.  Columns whose bit of
+// `keep` is clear (MASK) get a score of -inf, so P = 0 and dS = 0 there.
+// COLSTATS: nl and dl per column (float4 reads of nl[], dl[]), else the
+// row's nl2, dl2.
+template <bool MASK, bool COLSTATS>
+__device__ __forceinline__ void probs_grads(const uint32_t (&sv)[32], const uint32_t (&dpv)[32],
+                                            const float* nl, const float* dl, float2 nl2, float2 dl2,
+                                            float2 sc2, uint32_t keep, uint32_t (&pp)[16],
+                                            uint32_t (&dd)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    float4 n4 = make_float4(0.f, 0.f, 0.f, 0.f), d4 = n4;
+    if constexpr (COLSTATS) {
+      n4 = *reinterpret_cast<const float4*>(nl + e);
+      d4 = *reinterpret_cast<const float4*>(dl + e);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int f = e + 2 * h;
+      const float2 nn = COLSTATS ? (h ? make_float2(n4.z, n4.w) : make_float2(n4.x, n4.y)) : nl2;
+      const float2 dm = COLSTATS ? (h ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y)) : dl2;
+      float2 x = sep::ffma2(make_float2(__uint_as_float(sv[f]), __uint_as_float(sv[f + 1])), sc2, nn);
+      if constexpr (MASK) {
+        x.x = (keep >> f) & 1u ? x.x : -INFINITY;
+        x.y = (keep >> (f + 1)) & 1u ? x.y : -INFINITY;
+      }
+      const float p0 = sep::ex2_approx(x.x), p1 = sep::ex2_approx(x.y);
+      const float2 ds = fmul2(make_float2(p0, p1),
+                              fsub2(make_float2(__uint_as_float(dpv[f]), __uint_as_float(dpv[f + 1])), dm));
+      pp[f / 2] = sep::pack_bf16x2(p0, p1);
+      dd[f / 2] = sep::pack_bf16x2(ds.x, ds.y);
+    }
+  }
+}
+
+// Shared memory of the key-centric kernel: K, V [128][D] (swizzled
+// 64-column tiles); a ring of kNst unit stages, each the unit's Q and dO
+// rows [64][D]; -lse (log2 domain) and delta [kNst][64] fp32; key
+// positions and use flags [128] int32.
 template <int D>
 struct KvSmem {
   static constexpr int NB = D / 64;
-  static constexpr int K = 0, V = NB * kT128, Q = 2 * NB * kT128, DO = 4 * NB * kT128;  // Q, dO: [2] x NB tiles
-  static constexpr int LSE = 6 * NB * kT128;  // [2][128] fp32: -lse (log2 domain)
-  static constexpr int DEL = LSE + 1024;  // [2][128] fp32
-  static constexpr int POS = DEL + 1024;  // [128] int32
-  static constexpr int USE = POS + 512;   // [128] int32
+  static constexpr int K = 0, V = NB * kT128, RING = 2 * NB * kT128;
+  static constexpr int STAGE = 2 * NB * kT64;  // Q tiles, then dO tiles
+  static constexpr int LSE = RING + kNst * STAGE;
+  static constexpr int DEL = LSE + kNst * 64 * 4;
+  static constexpr int POS = DEL + kNst * 64 * 4;
+  static constexpr int USE = POS + 512;
   static constexpr int BYTES = USE + 512 + 1024;  // + alignment slack
 };
-struct TcBars {
-  uint64_t full, s_full, p_full, m_full, drain;
-  uint64_t tile[2];  // tensor-copy completion of a Q / dO buffer (key-centric kernel)
+struct KvBars {
+  uint64_t kv_full, fin, drain;
+  uint64_t st_full[kNst], st_free[kNst], s_full[2], p_full[2];
   uint32_t tmem_base;
   int abort;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
-    k_sep_bwd_tc_kv(const BwdParams p, const __grid_constant__ CUtensorMap map_q,
-                    const __grid_constant__ CUtensorMap map_do) {
-  using KvSmem = ::KvSmem<D>;
+    k_bwd_kv(const BwdParams p, const __grid_constant__ CUtensorMap map_q,
+             const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_k,
+             const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kc,
+             const __grid_constant__ CUtensorMap map_vc, __nv_bfloat16* __restrict__ dk,
+             __nv_bfloat16* __restrict__ dv) {
+  using Sm = KvSmem<D>;
   constexpr int NB = D / 64;
   constexpr uint32_t kColDK = col_dk<D>();
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* const smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ TcBars bars;
+  __shared__ KvBars bars;
   const uint32_t sb_ = sep::smem_u32(smem);
-  float* const lse_s = reinterpret_cast<float*>(smem + KvSmem::LSE);
-  float* const del_s = reinterpret_cast<float*>(smem + KvSmem::DEL);
-  int32_t* const pos_s = reinterpret_cast<int32_t*>(smem + KvSmem::POS);
-  int32_t* const use_s = reinterpret_cast<int32_t*>(smem + KvSmem::USE);
+  float* const lse_s = reinterpret_cast<float*>(smem + Sm::LSE);
+  float* const del_s = reinterpret_cast<float*>(smem + Sm::DEL);
+  int32_t* const pos_s = reinterpret_cast<int32_t*>(smem + Sm::POS);
+  int32_t* const use_s = reinterpret_cast<int32_t*>(smem + Sm::USE);
 
   const int item = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.S, G = p.Hq / p.Hkv;
   const int nT = (S + TBQ - 1) / TBQ;
-  const int32_t* pre = p.prefix + static_cast<int64_t>(b) * (S + 1);
-  const int32_t* ix = p.idx + static_cast<int64_t>(b) * S;
   const uint8_t* fl = p.is_sep + static_cast<int64_t>(b) * S;
-  const int a0 = p.a < S ? p.a : S;
-  const int nglob = a0 + (pre[S] - pre[a0]);
+  const GlobalList gl(p, b);
 
   const bool window = item < p.nwin;
   int kb, t0, t1;
@@ -532,26 +344,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else {
     kb = (item - p.nwin) / p.nchunk;
     const int chunk = (item - p.nwin) % p.nchunk;
-    if (kb * TBK >= nglob) return;
-    const int t = kb * TBK;
-    const int pmin = t < a0 ? t : ix[pre[a0] + t - a0];
-    t0 = pmin / TBQ + chunk * kTcChunkTiles;
+    if (kb * TBK >= gl.total) return;
+    t0 = gl.pos(kb * TBK) / TBQ + chunk * kTcChunkTiles;
     t1 = t0 + kTcChunkTiles < nT ? t0 + kTcChunkTiles : nT;
     if (t0 >= nT) return;
   }
   const int ntile = t1 - t0;
   const int nvisit = G * ntile;
+  const int nunit = 2 * nvisit;
+  const int64_t kvrow0 = (static_cast<int64_t>(b) * p.Hkv + g) * S;
+  // unit u: queries [64 (u & 1), +64) of the tile of visit u >> 1, whose
+  // first row in the [B * Hq * S] view is unit_row(u)
+  auto unit_row = [&](int u) -> int64_t {
+    const int v = u >> 1;
+    return (static_cast<int64_t>(b) * p.Hq + g * G + v / ntile) * S + (t0 + v % ntile) * TBQ +
+           64 * (u & 1);
+  };
+  // the unit's Q and dO rows into stage u % kNst (its bytes, no arrival)
+  auto load_unit = [&](int u) {
+    const int st = u % kNst;
+    uint8_t* dst = smem + Sm::RING + st * Sm::STAGE;
+    const int32_t row = static_cast<int32_t>(unit_row(u));
+    mbar_expect_tx(&bars.st_full[st], Sm::STAGE);
+#pragma unroll
+    for (int c = 0; c < NB; ++c) {
+      sep::tma_load_2d(dst + c * kT64, &map_q, 64 * c, row, &bars.st_full[st]);
+      sep::tma_load_2d(dst + (NB + c) * kT64, &map_do, 64 * c, row, &bars.st_full[st]);
+    }
+  };
 
-  if (threadIdx.x == 0) {
-    sep::mbar_init(&bars.full, 1);
-    sep::mbar_init(&bars.s_full, 1);
-    sep::mbar_init(&bars.p_full, 1);
-    sep::mbar_init(&bars.m_full, 1);
+  if (threadIdx.x == 9 * 32) {
+    // the load warp's first lane: barriers, then at once the K / V copies
+    // and the first kNst units (the ring starts free)
+    sep::mbar_init(&bars.kv_full, 1);
+    sep::mbar_init(&bars.fin, 1);
     sep::mbar_init(&bars.drain, 1);
-    sep::mbar_init(&bars.tile[0], 1);
-    sep::mbar_init(&bars.tile[1], 1);
-    bars.abort = 0;
+    for (int i = 0; i < kNst; ++i) {
+      sep::mbar_init(&bars.st_full[i], 32);  // the load warp's lanes, after the statistics
+      sep::mbar_init(&bars.st_free[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      sep::mbar_init(&bars.s_full[i], 1);
+      sep::mbar_init(&bars.p_full[i], 8);
+    }
+    // a wait of an earlier CTA gave up: this one ends at its first wait too
+    bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
     sep::mbar_fence_init();
+    sep::mbar_arrive_expect_tx(&bars.kv_full, 2 * NB * kT128);
+    const int32_t row = static_cast<int32_t>(kvrow0 + kb * TBK);
+    load_tile128<D>(smem + Sm::K, window ? &map_k : &map_kc, row, &bars.kv_full);
+    load_tile128<D>(smem + Sm::V, window ? &map_v : &map_vc, row, &bars.kv_full);
+    for (int u = 0; u < kNst && u < nunit; ++u) load_unit(u);
   }
   if (threadIdx.x < TBK) {
     const int r = threadIdx.x;
@@ -562,8 +405,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (pos >= S) pos = -1;
     } else {
       const int t = kb * TBK + r;
-      if (t < nglob) {
-        pos = t < a0 ? t : ix[pre[a0] + t - a0];
+      if (t < gl.total) {
+        pos = gl.pos(t);
         use = 1;
       }
     }
@@ -579,177 +422,209 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   sep::tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
   volatile int* abort = &bars.abort;
-  const int64_t kvrow0 = (static_cast<int64_t>(b) * p.Hkv + g) * S;
 
   if (warp < 8) {
     // ------------------------------------------------ compute warps
-    const int tid = threadIdx.x;
     const int lq = warp & 3, ch = warp >> 2;
     const int r = 32 * lq + lane;  // key row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * lq) << 16;
-    load_rows<D>(sb_ + KvSmem::K, p.k, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
-    load_rows<D>(sb_ + KvSmem::V, p.v, [&](int rr) { const int q = pos_s[rr]; return q < 0 ? -1 : kvrow0 + q; }, tid, 256);
-    cp_async_commit();
-    // lse (negated, log2 domain) and delta of visit v's queries: thread
-    // tid < 128 loads its query's pair (into registers one visit ahead)
-    auto row_stats = [&](int v, float& nl, float& dl) {
-      const int h = g * G + v / ntile, t = t0 + v % ntile;
-      const int i = t * TBQ + tid;
-      const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
-      nl = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
-      dl = i < S ? p.delta[qrow0 + i] : 0.f;
-    };
-    if (tid < TBQ) {
-      float nl, dl;
-      row_stats(0, nl, dl);
-      lse_s[tid] = nl;
-      del_s[tid] = dl;
-    }
-    cp_async_wait<0>();  // K and V
-    sep::fence_proxy_async_smem();
-    sep::named_bar_sync(1, 256);
-    if (tid == 0) sep::mbar_arrive(&bars.full);  // K and V are in shared memory
     const int jp = pos_s[r], use = use_s[r];
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     bool ok = true;
-    for (int v = 0; v < nvisit && ok; ++v) {
-      const int buf = v & 1;
-      const int t = t0 + v % ntile;
-      const int i0 = t * TBQ;
-      float nl_next = 0.f, dl_next = 0.f;
-      if (v + 1 < nvisit && tid < TBQ) row_stats(v + 1, nl_next, dl_next);
-      if (!sep::mbar_wait(&bars.s_full, v & 1, abort, p.err) || *abort) {
+    for (int u = 0; u < nunit && ok; ++u) {
+      const int v = u >> 1, hh = u & 1, sb = u & 1, st = u % kNst;
+      const int i0 = (t0 + v % ntile) * TBQ;
+      if (!warp_wait(&bars.st_full[st], (u / kNst) & 1, abort, p.err)) {
+        ok = false;  // (the unit's statistics are in shared memory)
+        break;
+      }
+      if (!warp_wait(&bars.s_full[sb], (u >> 1) & 1, abort, p.err)) {
         ok = false;
         break;
       }
       sep::tc_fence_after();
-      // the query columns this key row keeps: [qa, qb)
+      // the unit columns this key row keeps: [qa, qb) relative to column
+      // 64 hh + 32 ch of the tile
       int qa = 0, qb = 0;
       if (use && jp >= 0) {
         qa = jp - i0 > 0 ? jp - i0 : 0;
         qb = S - i0 < TBQ ? S - i0 : TBQ;
         if (window && jp + p.n - i0 < qb) qb = jp + p.n - i0;
       }
-      uint32_t sv[64], dv_[64];
-      sep::tmem_ld32(tmem + lane_base + kColS + 64 * ch, sv);
-      sep::tmem_ld32(tmem + lane_base + kColS + 64 * ch + 32, sv + 32);
-      sep::tmem_ld32(tmem + lane_base + kColDP + 64 * ch, dv_);
-      sep::tmem_ld32(tmem + lane_base + kColDP + 64 * ch + 32, dv_ + 32);
-      sep::tmem_wait_ld_r32(sv);
-      sep::tmem_wait_ld_r32(sv + 32);
-      sep::tmem_wait_ld_r32(dv_);
-      sep::tmem_wait_ld_r32(dv_ + 32);
-      sep::named_bar_sync(2 + lq, 64);  // the partner warp has read its scores too
-      const float* nl = lse_s + buf * 128 + 64 * ch;
-      const float* dl = del_s + buf * 128 + 64 * ch;
-      uint32_t pp[32], dd[32];
+      const int c0 = 64 * hh + 32 * ch;
+      const uint32_t keep = bit_range(qa - c0, qb - c0);
+      const uint32_t cs = 128u * sb + 32u * ch;
+      uint32_t pp[16], dd[16];
+      if (__all_sync(0xffffffffu, keep == 0u)) {
+        // no column of the warp's rows is kept: P^T and dS^T are zero
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
-        const int q = 64 * ch + e;
-        const float2 x = sep::ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2,
-                                    *reinterpret_cast<const float2*>(nl + e));
-        const float p0 = (q >= qa && q < qb) ? sep::ex2_approx(x.x) : 0.f;
-        const float p1 = (q + 1 >= qa && q + 1 < qb) ? sep::ex2_approx(x.y) : 0.f;
-        const float2 ds = fmul2(make_float2(p0, p1),
-                                fsub2(make_float2(__uint_as_float(dv_[e]), __uint_as_float(dv_[e + 1])),
-                                      *reinterpret_cast<const float2*>(dl + e)));
-        pp[e / 2] = sep::pack_bf16x2(p0, p1);
-        dd[e / 2] = sep::pack_bf16x2(ds.x, ds.y);
+        for (int e = 0; e < 16; ++e) pp[e] = dd[e] = 0u;
+      } else {
+        uint32_t sv[32], dv_[32];
+        sep::tmem_ld32(tmem + lane_base + cs, sv);
+        sep::tmem_ld32(tmem + lane_base + cs + 64, dv_);
+        sep::tmem_wait_ld_r32(sv);
+        sep::tmem_wait_ld_r32(dv_);
+        const float* nl = lse_s + st * 64 + 32 * ch;
+        const float* dl = del_s + st * 64 + 32 * ch;
+        const float2 z2 = make_float2(0.f, 0.f);
+        if (__all_sync(0xffffffffu, keep == 0xffffffffu))
+          probs_grads<false, true>(sv, dv_, nl, dl, z2, z2, sc2, keep, pp, dd);
+        else
+          probs_grads<true, true>(sv, dv_, nl, dl, z2, z2, sc2, keep, pp, dd);
       }
-      sep::tmem_st32(tmem + lane_base + kColS + 32 * ch, pp);
-      sep::tmem_st32(tmem + lane_base + kColDP + 32 * ch, dd);
-      if (v + 1 < nvisit && tid < TBQ) {  // buffer (v+1) & 1 was last read by visit v-1
-        lse_s[(buf ^ 1) * 128 + tid] = nl_next;
-        del_s[(buf ^ 1) * 128 + tid] = dl_next;
-      }
+      sep::tmem_st16(tmem + lane_base + cs, pp);
+      sep::tmem_st16(tmem + lane_base + cs + 64, dd);
       sep::tmem_wait_st();
       sep::tc_fence_before();
-      sep::named_bar_sync(1, 256);
-      if (tid == 0) sep::mbar_arrive(&bars.p_full);
+      __syncwarp();
+      if (lane == 0) sep::mbar_arrive(&bars.p_full[sb]);
     }
-    if (ok && nvisit > 0 && sep::mbar_wait(&bars.m_full, (nvisit - 1) & 1, abort, p.err) && !*abort) {
+    if (ok && warp_wait(&bars.fin, 0, abort, p.err)) {
       sep::tc_fence_after();
-      // dK and dV of this key row, columns [D/2 ch, +D/2): every lane
-      // loads (warp-wide), rows with a key store
+      // dK and dV of this key row, columns [D/2 ch, +D/2): every lane loads
+      // (warp-wide); a window key is stored as bf16, a global key's partial
+      // sum is added to its fp32 row of the compact list
       const bool mine = jp >= 0 && use;
-      float* dkp = p.dk_acc + (kvrow0 + (mine ? jp : 0)) * D + (D / 2) * ch;
-      float* dvp = p.dv_acc + (kvrow0 + (mine ? jp : 0)) * D + (D / 2) * ch;
+      const int64_t row = kvrow0 + (window ? (mine ? jp : 0) : kb * TBK + r);
+      const float sc = p.scale_log2 * 0.69314718055994530942f;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t kv[32], vv[32];
-        sep::tmem_ld32(tmem + lane_base + kColDK + (D / 2) * ch + 32 * c, kv);
-        sep::tmem_ld32(tmem + lane_base + kColDV + (D / 2) * ch + 32 * c, vv);
+        const int col = (D / 2) * ch + 32 * c;
+        sep::tmem_ld32(tmem + lane_base + kColDK + col, kv);
+        sep::tmem_ld32(tmem + lane_base + kColAcc + col, vv);
         sep::tmem_wait_ld_r32(kv);
         sep::tmem_wait_ld_r32(vv);
-        if (mine) {
+        if (!mine) continue;
+        if (window) {
+          uint4* kd = reinterpret_cast<uint4*>(dk + row * D + col);
+          uint4* vd = reinterpret_cast<uint4*>(dv + row * D + col);
+#pragma unroll
+          for (int u4 = 0; u4 < 4; ++u4) {
+            kd[u4] = make_uint4(sep::pack_bf16x2(__uint_as_float(kv[8 * u4]) * sc, __uint_as_float(kv[8 * u4 + 1]) * sc),
+                                sep::pack_bf16x2(__uint_as_float(kv[8 * u4 + 2]) * sc, __uint_as_float(kv[8 * u4 + 3]) * sc),
+                                sep::pack_bf16x2(__uint_as_float(kv[8 * u4 + 4]) * sc, __uint_as_float(kv[8 * u4 + 5]) * sc),
+                                sep::pack_bf16x2(__uint_as_float(kv[8 * u4 + 6]) * sc, __uint_as_float(kv[8 * u4 + 7]) * sc));
+            vd[u4] = make_uint4(sep::pack_bf16x2(__uint_as_float(vv[8 * u4]), __uint_as_float(vv[8 * u4 + 1])),
+                                sep::pack_bf16x2(__uint_as_float(vv[8 * u4 + 2]), __uint_as_float(vv[8 * u4 + 3])),
+                                sep::pack_bf16x2(__uint_as_float(vv[8 * u4 + 4]), __uint_as_float(vv[8 * u4 + 5])),
+                                sep::pack_bf16x2(__uint_as_float(vv[8 * u4 + 6]), __uint_as_float(vv[8 * u4 + 7])));
+          }
+        } else {
+          float* kp = p.dk_acc + row * D + col;
+          float* vp = p.dv_acc + row * D + col;
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            if (window) {
-              *reinterpret_cast<float2*>(dkp + 32 * c + e) = make_float2(__uint_as_float(kv[e]), __uint_as_float(kv[e + 1]));
-              *reinterpret_cast<float2*>(dvp + 32 * c + e) = make_float2(__uint_as_float(vv[e]), __uint_as_float(vv[e + 1]));
-            } else {
-              red_add_v2(dkp + 32 * c + e, __uint_as_float(kv[e]), __uint_as_float(kv[e + 1]));
-              red_add_v2(dvp + 32 * c + e, __uint_as_float(vv[e]), __uint_as_float(vv[e + 1]));
-            }
+            red_add_v2(kp + e, __uint_as_float(kv[e]), __uint_as_float(kv[e + 1]));
+            red_add_v2(vp + e, __uint_as_float(vv[e]), __uint_as_float(vv[e + 1]));
           }
         }
       }
     }
-    cp_async_wait<0>();
-  } else {
+  } else if (warp == 8) {
     if (lane == 0) {
       // ---------------------------------------------- MMA issue (one thread)
-      constexpr uint32_t id_s = idesc_mn(128, 128, false, false);
+      constexpr uint32_t id_s = idesc_mn(128, 64, false, false);
       constexpr uint32_t id_o = idesc_mn(128, D, false, true);
-      const uint64_t dK = sep::smem_desc_sw128(sb_ + KvSmem::K, 16);
-      const uint64_t dV = sep::smem_desc_sw128(sb_ + KvSmem::V, 16);
-      // Q and dO tiles of visit v into buffer v & 1 by the tensor-copy
-      // engine (two 64-column tiles each; rows past the head belong to the
-      // next head or are zero-filled past the array, and their P is 0)
-      auto load_tiles = [&](int v) {
-        const int h = g * G + v / ntile, t = t0 + v % ntile;
-        const int32_t row = static_cast<int32_t>((static_cast<int64_t>(b) * p.Hq + h) * S + t * TBQ);
-        const int buf = v & 1;
-        sep::mbar_arrive_expect_tx(&bars.tile[buf], 2 * NB * kT128);
+      const uint64_t dK = sep::smem_desc_sw128(sb_ + Sm::K, 16);
+      const uint64_t dV = sep::smem_desc_sw128(sb_ + Sm::V, 16);
+      bool ok = nvisit > 0 && sep::mbar_wait(&bars.kv_full, 0, abort, p.err);
+      for (int u = 0; u <= nunit && ok; ++u) {
+        if (u < nunit) {
+          // scores of unit u into buffer u & 1 (its previous contents, unit
+          // u-2, were read by the products issued before this point)
+          const int st = u % kNst;
+          if (!sep::mbar_wait(&bars.st_full[st], (u / kNst) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          sep::tc_fence_after();
+          const uint32_t qa = sb_ + Sm::RING + st * Sm::STAGE, oa = qa + NB * kT64;
+          const uint64_t dQ = sep::smem_desc_sw128(qa, 16), dO = sep::smem_desc_sw128(oa, 16);
+          const uint32_t cs = 128u * (u & 1);
 #pragma unroll
-        for (int c = 0; c < NB; ++c) {
-          sep::tma_load_2d(smem + KvSmem::Q + buf * NB * kT128 + c * kT128, &map_q, 64 * c, row, &bars.tile[buf]);
-          sep::tma_load_2d(smem + KvSmem::DO + buf * NB * kT128 + c * kT128, &map_do, 64 * c, row, &bars.tile[buf]);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t kofs = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
+            const uint64_t oq = static_cast<uint64_t>(((kk / 4) * kT64 + (kk % 4) * 32) >> 4);
+            sep::mma_bf16_ss(tmem + cs, dK + kofs, dQ + oq, id_s, kk > 0 ? 1u : 0u);
+            sep::mma_bf16_ss(tmem + cs + 64, dV + kofs, dO + oq, id_s, kk > 0 ? 1u : 0u);
+          }
+          sep::mma_commit(&bars.s_full[u & 1]);
         }
-      };
-      if (nvisit > 0) load_tiles(0);
-      bool kv_in = sep::mbar_wait(&bars.full, 0, abort, p.err);  // K and V
-      for (int v = 0; v < nvisit && kv_in; ++v) {
-        const int buf = v & 1;
-        if (!sep::mbar_wait(&bars.tile[buf], (v >> 1) & 1, abort, p.err)) break;
-        sep::tc_fence_after();
-        const uint32_t qa = sb_ + KvSmem::Q + buf * NB * kT128, oa = sb_ + KvSmem::DO + buf * NB * kT128;
-        const uint64_t dQ = sep::smem_desc_sw128(qa, 16), dO = sep::smem_desc_sw128(oa, 16);
-        const uint64_t dQmn = sep::smem_desc_sw128(qa, kT128), dOmn = sep::smem_desc_sw128(oa, kT128);
+        if (u >= 1) {
+          // gradient products of unit w = u - 1 once its P^T and dS^T are in
+          const int w = u - 1, wst = w % kNst;
+          if (!sep::mbar_wait(&bars.p_full[w & 1], (w >> 1) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          sep::tc_fence_after();
+          const uint32_t qa = sb_ + Sm::RING + wst * Sm::STAGE, oa = qa + NB * kT64;
+          const uint64_t dQmn = sep::smem_desc_sw128(qa, kT64), dOmn = sep::smem_desc_sw128(oa, kT64);
+          const uint32_t cs = 128u * (w & 1);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
-          sep::mma_bf16_ss(tmem + kColS, dK + off, dQ + off, id_s, kk > 0 ? 1u : 0u);
-          sep::mma_bf16_ss(tmem + kColDP, dV + off, dO + off, id_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
+            const uint32_t acc = (w > 0 || kk > 0) ? 1u : 0u;
+            sep::mma_bf16_ts(tmem + kColAcc, tmem + unit_acol(cs, kk), dOmn + off, id_o, acc);
+            sep::mma_bf16_ts(tmem + kColDK, tmem + unit_acol(cs + 64, kk), dQmn + off, id_o, acc);
+          }
+          sep::mma_commit(&bars.st_free[wst]);  // the stage may be refilled
         }
-        sep::mma_commit(&bars.s_full);
-        if (!sep::mbar_wait(&bars.p_full, v & 1, abort, p.err)) break;
-        // the scores of visit v are complete, so (in order) are the products
-        // of visit v-1: buffer (v+1) & 1 may be refilled
-        if (v + 1 < nvisit) load_tiles(v + 1);
-        sep::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < TBQ / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
-          const uint32_t acc = (v > 0 || kk > 0) ? 1u : 0u;
-          sep::mma_bf16_ts(tmem + kColDV, tmem + kColS + kk * 8, dOmn + off, id_o, acc);
-          sep::mma_bf16_ts(tmem + kColDK, tmem + kColDP + kk * 8, dQmn + off, id_o, acc);
-        }
-        sep::mma_commit(&bars.m_full);
       }
+      if (ok) sep::mma_commit(&bars.fin);
       sep::mma_commit(&bars.drain);  // every MMA completes before TMEM is released
       int keep = 0;
       sep::mbar_wait(&bars.drain, 0, &keep, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ loads (warp 9)
+    // (K, V and the first kNst units were started before the block
+    // barrier.)  Per unit: the copies once its stage is free, then the
+    // unit's -lse (log2 domain) and delta, read one unit ahead into
+    // registers (rows lane, lane + 32), then the 32 arrivals that complete
+    // the stage with its bytes.
+    int issued = nunit < kNst ? nunit : kNst;  // units whose copies were started
+    float nlr[2], dlr[2];
+    auto fetch = [&](int u) {
+      if (u >= nunit) return;
+      const int64_t row0 = unit_row(u);
+      const int i0 = (t0 + (u >> 1) % ntile) * TBQ + 64 * (u & 1);
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int e = lane + 32 * m;
+        nlr[m] = i0 + e < S ? -p.lse[row0 + e] * 1.44269504088896340736f : 0.f;
+        dlr[m] = i0 + e < S ? p.delta[row0 + e] : 0.f;
+      }
+    };
+    fetch(0);
+    for (int u = 0; u < nunit; ++u) {
+      const int st = u % kNst;
+      if (u >= kNst) {
+        bool go = true;
+        if (lane == 0) {
+          go = sep::mbar_wait(&bars.st_free[st], ((u / kNst) - 1) & 1, abort, p.err);
+          if (go) load_unit(u);
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+        issued = u + 1;
+      }
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        lse_s[st * 64 + lane + 32 * m] = nlr[m];
+        del_s[st * 64 + lane + 32 * m] = dlr[m];
+      }
+      fetch(u + 1);
+      sep::mbar_arrive(&bars.st_full[st]);
+    }
+    // after an abort, let the started copies land before the CTA can exit
+    if (lane == 0 && *abort) {
+      int dummy = 0;
+      if (nvisit > 0) sep::mbar_wait(&bars.kv_full, 0, &dummy, nullptr);
+      for (int u = issued - kNst < 0 ? 0 : issued - kNst; u < issued; ++u)
+        sep::mbar_wait(&bars.st_full[u % kNst], (u / kNst) & 1, &dummy, nullptr);
     }
     __syncwarp();
   }
@@ -762,28 +637,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
+// Shared memory of the query-centric kernel: Q, dO [128][D] (swizzled
+// 64-column tiles); a ring of kNst unit stages, each the unit's K and V rows
+// [64][D]; the global flags of each stage's keys as [kNst][2] 32-bit words
+// (bit k of word m: key 32 m + k of the unit).
 template <int D>
 struct QSmem {
   static constexpr int NB = D / 64;
-  static constexpr int Q = 0, DO = NB * kT128;
-  static constexpr int K = 2 * NB * kT128, V = 3 * NB * kT128;  // [2] buffers, 2 NB tiles apart
-  static constexpr int POS = 6 * NB * kT128;  // [2][128] int32 key positions
-  static constexpr int GLB = POS + 1024;  // [2][128] int32: key kept by every later query
+  static constexpr int Q = 0, DO = NB * kT128, RING = 2 * NB * kT128;
+  static constexpr int STAGE = 2 * NB * kT64;  // K tiles, then V tiles
+  static constexpr int GLB = RING + kNst * STAGE;
   static constexpr int BYTES = GLB + 1024 + 1024;
+};
+struct QBars {
+  uint64_t q_full, fin, drain;
+  uint64_t st_full[kNst], st_free[kNst], s_full[2], p_full[2];
+  uint32_t tmem_base;
+  int abort;
 };
 
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams p,
-                                                                __nv_bfloat16* __restrict__ dq) {
-  using QSmem = ::QSmem<D>;
+__global__ void __launch_bounds__(kTcThreads, 1)
+    k_bwd_q(const BwdParams p, const __grid_constant__ CUtensorMap map_q,
+            const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_k,
+            const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kc,
+            const __grid_constant__ CUtensorMap map_vc, __nv_bfloat16* __restrict__ dq) {
+  using Sm = QSmem<D>;
   constexpr int NB = D / 64;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* const smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  __shared__ TcBars bars;
+  __shared__ QBars bars;
   const uint32_t sb_ = sep::smem_u32(smem);
-  int32_t* const pos_s = reinterpret_cast<int32_t*>(smem + QSmem::POS);
-  int32_t* const glb_s = reinterpret_cast<int32_t*>(smem + QSmem::GLB);
+  uint32_t* const glb_w = reinterpret_cast<uint32_t*>(smem + Sm::GLB);
 
   const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -791,27 +677,60 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams 
   const int i0 = t * TBQ;
   const int qlast = (i0 + TBQ < S ? i0 + TBQ : S) - 1;
   const int32_t* pre = p.prefix + static_cast<int64_t>(b) * (S + 1);
-  const int32_t* ix = p.idx + static_cast<int64_t>(b) * S;
   const uint8_t* fl = p.is_sep + static_cast<int64_t>(b) * S;
-  // the tile's kept keys: global keys before the first row's window, then
-  // the window positions [lo, qlast]
+  // the tile's kept keys: global keys before the first row's window (the
+  // head of the compact list), then the window positions [lo, qlast]
   const int lo = i0 - p.n + 1 > 0 ? i0 - p.n + 1 : 0;
   const int al = p.a < lo ? p.a : lo;
   const int nglo = al + (pre[lo] - pre[al]);
   const int nbg = (nglo + TBK - 1) / TBK;
   const int nbw = (qlast - lo + TBK) / TBK;
   const int nblk = nbg + nbw;
+  const int nunit = 2 * nblk;
   const int64_t kvrow0 = (static_cast<int64_t>(b) * p.Hkv + g) * S;
   const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
+  // unit u: keys [64 (u & 1), +64) of block u >> 1 -- rows of the compact
+  // list (global blocks) or positions (window blocks) from unit_key(u)
+  auto unit_key = [&](int u) -> int {
+    const int j = u >> 1;
+    return (j < nbg ? j * TBK : lo + (j - nbg) * TBK) + 64 * (u & 1);
+  };
+  // the unit's K and V rows into stage u % kNst (its bytes; the load warp's
+  // 32 arrivals follow once the stage's global-flag words are written)
+  auto load_unit = [&](int u) {
+    const int st = u % kNst;
+    const bool win = (u >> 1) >= nbg;
+    uint8_t* dst = smem + Sm::RING + st * Sm::STAGE;
+    const int32_t row = static_cast<int32_t>(kvrow0 + unit_key(u));
+    mbar_expect_tx(&bars.st_full[st], Sm::STAGE);
+#pragma unroll
+    for (int c = 0; c < NB; ++c) {
+      sep::tma_load_2d(dst + c * kT64, win ? &map_k : &map_kc, 64 * c, row, &bars.st_full[st]);
+      sep::tma_load_2d(dst + (NB + c) * kT64, win ? &map_v : &map_vc, 64 * c, row, &bars.st_full[st]);
+    }
+  };
 
-  if (threadIdx.x == 0) {
-    sep::mbar_init(&bars.full, 1);
-    sep::mbar_init(&bars.s_full, 1);
-    sep::mbar_init(&bars.p_full, 1);
-    sep::mbar_init(&bars.m_full, 1);
+  if (threadIdx.x == 9 * 32) {
+    // the load warp's first lane: barriers, then at once the Q / dO copies
+    // and the first kNst units (the ring starts free)
+    sep::mbar_init(&bars.q_full, 1);
+    sep::mbar_init(&bars.fin, 1);
     sep::mbar_init(&bars.drain, 1);
-    bars.abort = 0;
+    for (int i = 0; i < kNst; ++i) {
+      sep::mbar_init(&bars.st_full[i], 32);
+      sep::mbar_init(&bars.st_free[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      sep::mbar_init(&bars.s_full[i], 1);
+      sep::mbar_init(&bars.p_full[i], 8);
+    }
+    // a wait of an earlier CTA gave up: this one ends at its first wait too
+    bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
     sep::mbar_fence_init();
+    sep::mbar_arrive_expect_tx(&bars.q_full, 2 * NB * kT128);
+    load_tile128<D>(smem + Sm::Q, &map_q, static_cast<int32_t>(qrow0 + i0), &bars.q_full);
+    load_tile128<D>(smem + Sm::DO, &map_do, static_cast<int32_t>(qrow0 + i0), &bars.q_full);
+    for (int u = 0; u < kNst && u < nunit; ++u) load_unit(u);
   }
   if (warp == 8) {
     sep::tmem_alloc(&bars.tmem_base, 512);
@@ -824,172 +743,178 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams 
   volatile int* abort = &bars.abort;
 
   if (warp < 8) {
-    const int tid = threadIdx.x;
     const int lq = warp & 3, ch = warp >> 2;
     const int r = 32 * lq + lane;  // query row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * lq) << 16;
     const int i = i0 + r;
     const float nlse2 = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
     const float dl = i < S ? p.delta[qrow0 + i] : 0.f;
-    auto rowq = [&](int rr) -> int64_t { return i0 + rr < S ? qrow0 + i0 + rr : -1; };
-    load_rows<D>(sb_ + QSmem::Q, p.q, rowq, tid, 256);
-    load_rows<D>(sb_ + QSmem::DO, p.dout, rowq, tid, 256);
-    auto load_block = [&](int j, int buf) {
-      // key positions of block j (threads 0..127: one key each), then rows
-      if (tid < TBK) {
-        int pos = -1, glb = 0;
-        if (j < nbg) {
-          const int e = j * TBK + tid;
-          if (e < nglo) {
-            pos = e < al ? e : ix[pre[al] + e - al];
-            glb = 1;
-          }
-        } else {
-          const int q = lo + (j - nbg) * TBK + tid;
-          if (q <= qlast) {
-            pos = q;
-            glb = q < p.a || fl[q];
-          }
-        }
-        pos_s[buf * 128 + tid] = pos;
-        glb_s[buf * 128 + tid] = glb;
-      }
-      sep::named_bar_sync(1, 256);  // every position is written before the row copies read them
-      auto rowk = [&](int rr) -> int64_t { const int q = pos_s[buf * 128 + rr]; return q < 0 ? -1 : kvrow0 + q; };
-      load_rows<D>(sb_ + QSmem::K + buf * 2 * NB * kT128, p.k, rowk, tid, 256);
-      load_rows<D>(sb_ + QSmem::V + buf * 2 * NB * kT128, p.v, rowk, tid, 256);
-      cp_async_commit();
-    };
-    load_block(0, 0);  // with Q and dO
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
     const float2 nl2 = make_float2(nlse2, nlse2), dl2 = make_float2(dl, dl);
     bool ok = true;
-    for (int j = 0; j < nblk && ok; ++j) {
-      const int buf = j & 1;
-      if (j > 0 && (!sep::mbar_wait(&bars.m_full, (j - 1) & 1, abort, p.err) || *abort)) {
-        ok = false;  // the products of block j-1 have read buffer (j+1) & 1
+    for (int u = 0; u < nunit && ok; ++u) {
+      const int j = u >> 1, hh = u & 1, sb = u & 1, st = u % kNst;
+      if (!warp_wait(&bars.st_full[st], (u / kNst) & 1, abort, p.err)) {
+        ok = false;  // (the unit's global-flag words are in shared memory)
         break;
       }
-      if (j + 1 < nblk) {
-        load_block(j + 1, buf ^ 1);
-        cp_async_wait<1>();
-      } else {
-        cp_async_wait<0>();
-      }
-      sep::fence_proxy_async_smem();
-      sep::named_bar_sync(1, 256);
-      if (tid == 0) sep::mbar_arrive(&bars.full);
-      if (!sep::mbar_wait(&bars.s_full, j & 1, abort, p.err) || *abort) {
+      if (!warp_wait(&bars.s_full[sb], (u >> 1) & 1, abort, p.err)) {
         ok = false;
         break;
       }
       sep::tc_fence_after();
-      const int32_t* gb = glb_s + buf * 128 + 64 * ch;
-      // the key columns this query row keeps: global blocks, every valid
-      // key; window blocks (contiguous positions from `base`), keys at most
-      // n - 1 back, or global ones, never past the row or the tile
-      int ka, kb2;
-      const bool win = j >= nbg;
-      int wlo = 0;
-      if (!win) {
-        ka = 0;
-        kb2 = nglo - j * TBK < TBK ? nglo - j * TBK : TBK;
-        if (i >= S) kb2 = 0;
+      // the unit's key columns this query row keeps, relative to column
+      // c0 = 64 hh + 32 ch of the block: global blocks, every listed key;
+      // window blocks (contiguous positions from `base`), keys at or before
+      // the row (and the tile), within n - 1 of it unless global
+      const int c0 = 64 * hh + 32 * ch;
+      uint32_t keep;
+      if (j < nbg) {
+        keep = bit_range(-c0, (nglo - j * TBK < TBK ? nglo - j * TBK : TBK) - c0);
       } else {
         const int base = lo + (j - nbg) * TBK;
-        ka = 0;
-        kb2 = i - base + 1;  // keys at positions <= i
-        const int lim = qlast - base + 1;
-        if (kb2 > lim) kb2 = lim;
-        if (kb2 > TBK) kb2 = TBK;
-        if (i >= S) kb2 = 0;
-        wlo = i - base - p.n + 1;  // keys before this column need the global flag
+        int kb2 = i - base + 1;  // keys at positions <= i, in the tile's range
+        if (kb2 > qlast - base + 1) kb2 = qlast - base + 1;
+        keep = bit_range(-c0, kb2 - c0) &
+               (bit_range(i - base - p.n + 1 - c0, 32) | glb_w[st * 2 + ch]);
       }
-      uint32_t sv[64], dv_[64];
-      sep::tmem_ld32(tmem + lane_base + kColS + 64 * ch, sv);
-      sep::tmem_ld32(tmem + lane_base + kColS + 64 * ch + 32, sv + 32);
-      sep::tmem_ld32(tmem + lane_base + kColDP + 64 * ch, dv_);
-      sep::tmem_ld32(tmem + lane_base + kColDP + 64 * ch + 32, dv_ + 32);
-      sep::tmem_wait_ld_r32(sv);
-      sep::tmem_wait_ld_r32(sv + 32);
-      sep::tmem_wait_ld_r32(dv_);
-      sep::tmem_wait_ld_r32(dv_ + 32);
-      sep::named_bar_sync(2 + lq, 64);  // the partner warp has read its scores too
-      uint32_t dd[32];
+      if (i >= S) keep = 0u;
+      const uint32_t cs = 128u * sb + 32u * ch;
+      uint32_t pp[16], dd[16];
+      if (__all_sync(0xffffffffu, keep == 0u)) {
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
-        const int kc = 64 * ch + e;
-        const float2 x = sep::ffma2(make_float2(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, nl2);
-        bool k0 = kc >= ka && kc < kb2, k1 = kc + 1 >= ka && kc + 1 < kb2;
-        if (win) {
-          k0 = k0 && (kc >= wlo || gb[e]);
-          k1 = k1 && (kc + 1 >= wlo || gb[e + 1]);
-        }
-        const float p0 = k0 ? sep::ex2_approx(x.x) : 0.f;
-        const float p1 = k1 ? sep::ex2_approx(x.y) : 0.f;
-        const float2 ds = fmul2(make_float2(p0, p1),
-                                fsub2(make_float2(__uint_as_float(dv_[e]), __uint_as_float(dv_[e + 1])), dl2));
-        dd[e / 2] = sep::pack_bf16x2(ds.x, ds.y);
+        for (int e = 0; e < 16; ++e) dd[e] = 0u;
+      } else {
+        uint32_t sv[32], dv_[32];
+        sep::tmem_ld32(tmem + lane_base + cs, sv);
+        sep::tmem_ld32(tmem + lane_base + cs + 64, dv_);
+        sep::tmem_wait_ld_r32(sv);
+        sep::tmem_wait_ld_r32(dv_);
+        if (__all_sync(0xffffffffu, keep == 0xffffffffu))
+          probs_grads<false, false>(sv, dv_, nullptr, nullptr, nl2, dl2, sc2, keep, pp, dd);
+        else
+          probs_grads<true, false>(sv, dv_, nullptr, nullptr, nl2, dl2, sc2, keep, pp, dd);
       }
-      sep::tmem_st32(tmem + lane_base + kColS + 32 * ch, dd);
+      sep::tmem_st16(tmem + lane_base + cs, dd);
       sep::tmem_wait_st();
       sep::tc_fence_before();
-      sep::named_bar_sync(1, 256);
-      if (tid == 0) sep::mbar_arrive(&bars.p_full);
+      __syncwarp();
+      if (lane == 0) sep::mbar_arrive(&bars.p_full[sb]);
     }
-    if (ok && sep::mbar_wait(&bars.m_full, (nblk - 1) & 1, abort, p.err) && !*abort) {
+    if (ok && warp_wait(&bars.fin, 0, abort, p.err)) {
       sep::tc_fence_after();
       const float sc = p.scale_log2 * 0.69314718055994530942f;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t qv[32];
-        sep::tmem_ld32(tmem + lane_base + kColDQ + (D / 2) * ch + 32 * c, qv);
+        const int col = (D / 2) * ch + 32 * c;
+        sep::tmem_ld32(tmem + lane_base + kColAcc + col, qv);
         sep::tmem_wait_ld_r32(qv);
         if (i < S) {
-          uint4* dst = reinterpret_cast<uint4*>(dq + (qrow0 + i) * D + (D / 2) * ch + 32 * c);
+          uint4* dst = reinterpret_cast<uint4*>(dq + (qrow0 + i) * D + col);
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            dst[u] = make_uint4(sep::pack_bf16x2(__uint_as_float(qv[8 * u]) * sc, __uint_as_float(qv[8 * u + 1]) * sc),
-                                sep::pack_bf16x2(__uint_as_float(qv[8 * u + 2]) * sc, __uint_as_float(qv[8 * u + 3]) * sc),
-                                sep::pack_bf16x2(__uint_as_float(qv[8 * u + 4]) * sc, __uint_as_float(qv[8 * u + 5]) * sc),
-                                sep::pack_bf16x2(__uint_as_float(qv[8 * u + 6]) * sc, __uint_as_float(qv[8 * u + 7]) * sc));
+          for (int u4 = 0; u4 < 4; ++u4)
+            dst[u4] = make_uint4(sep::pack_bf16x2(__uint_as_float(qv[8 * u4]) * sc, __uint_as_float(qv[8 * u4 + 1]) * sc),
+                                 sep::pack_bf16x2(__uint_as_float(qv[8 * u4 + 2]) * sc, __uint_as_float(qv[8 * u4 + 3]) * sc),
+                                 sep::pack_bf16x2(__uint_as_float(qv[8 * u4 + 4]) * sc, __uint_as_float(qv[8 * u4 + 5]) * sc),
+                                 sep::pack_bf16x2(__uint_as_float(qv[8 * u4 + 6]) * sc, __uint_as_float(qv[8 * u4 + 7]) * sc));
         }
       }
     }
-    cp_async_wait<0>();
-  } else {
+  } else if (warp == 8) {
     if (lane == 0) {
-      constexpr uint32_t id_s = idesc_mn(128, 128, false, false);
+      constexpr uint32_t id_s = idesc_mn(128, 64, false, false);
       constexpr uint32_t id_o = idesc_mn(128, D, false, true);
-      const uint64_t dQ = sep::smem_desc_sw128(sb_ + QSmem::Q, 16);
-      const uint64_t dO = sep::smem_desc_sw128(sb_ + QSmem::DO, 16);
-      for (int j = 0; j < nblk; ++j) {
-        const int buf = j & 1;
-        if (!sep::mbar_wait(&bars.full, j & 1, abort, p.err)) break;
-        sep::tc_fence_after();
-        const uint32_t ka = sb_ + QSmem::K + buf * 2 * NB * kT128, va = sb_ + QSmem::V + buf * 2 * NB * kT128;
-        const uint64_t dK = sep::smem_desc_sw128(ka, 16), dV = sep::smem_desc_sw128(va, 16);
-        const uint64_t dKmn = sep::smem_desc_sw128(ka, kT128);
+      const uint64_t dQ = sep::smem_desc_sw128(sb_ + Sm::Q, 16);
+      const uint64_t dO = sep::smem_desc_sw128(sb_ + Sm::DO, 16);
+      bool ok = sep::mbar_wait(&bars.q_full, 0, abort, p.err);
+      for (int u = 0; u <= nunit && ok; ++u) {
+        if (u < nunit) {
+          const int st = u % kNst;
+          if (!sep::mbar_wait(&bars.st_full[st], (u / kNst) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          sep::tc_fence_after();
+          const uint32_t ka = sb_ + Sm::RING + st * Sm::STAGE, va = ka + NB * kT64;
+          const uint64_t dK = sep::smem_desc_sw128(ka, 16), dV = sep::smem_desc_sw128(va, 16);
+          const uint32_t cs = 128u * (u & 1);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
-          sep::mma_bf16_ss(tmem + kColS, dQ + off, dK + off, id_s, kk > 0 ? 1u : 0u);
-          sep::mma_bf16_ss(tmem + kColDP, dO + off, dV + off, id_s, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t oq = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
+            const uint64_t okv = static_cast<uint64_t>(((kk / 4) * kT64 + (kk % 4) * 32) >> 4);
+            sep::mma_bf16_ss(tmem + cs, dQ + oq, dK + okv, id_s, kk > 0 ? 1u : 0u);
+            sep::mma_bf16_ss(tmem + cs + 64, dO + oq, dV + okv, id_s, kk > 0 ? 1u : 0u);
+          }
+          sep::mma_commit(&bars.s_full[u & 1]);
         }
-        sep::mma_commit(&bars.s_full);
-        if (!sep::mbar_wait(&bars.p_full, j & 1, abort, p.err)) break;
-        sep::tc_fence_after();
+        if (u >= 1) {
+          const int w = u - 1, wst = w % kNst;
+          if (!sep::mbar_wait(&bars.p_full[w & 1], (w >> 1) & 1, abort, p.err)) {
+            ok = false;
+            break;
+          }
+          sep::tc_fence_after();
+          const uint64_t dKmn = sep::smem_desc_sw128(sb_ + Sm::RING + wst * Sm::STAGE, kT64);
+          const uint32_t cs = 128u * (w & 1);
 #pragma unroll
-        for (int kk = 0; kk < TBK / 16; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
-          sep::mma_bf16_ts(tmem + kColDQ, tmem + kColS + kk * 8, dKmn + off, id_o,
-                           (j > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
+            sep::mma_bf16_ts(tmem + kColAcc, tmem + unit_acol(cs, kk), dKmn + off, id_o,
+                             (w > 0 || kk > 0) ? 1u : 0u);
+          }
+          sep::mma_commit(&bars.st_free[wst]);  // the stage may be refilled
         }
-        sep::mma_commit(&bars.m_full);
       }
+      if (ok) sep::mma_commit(&bars.fin);
       sep::mma_commit(&bars.drain);
       int keep = 0;
       sep::mbar_wait(&bars.drain, 0, &keep, nullptr);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ loads (warp 9)
+    // (Q, dO and the first kNst units were started before the block
+    // barrier.)  Per unit: the copies once its stage is free, then the
+    // global-flag words of a window unit (flags read one unit ahead into
+    // registers), then the 32 arrivals that complete the stage with its
+    // bytes.
+    int issued = nunit < kNst ? nunit : kNst;  // units whose copies were started
+    bool fnext[2];  // flags of keys lane, lane + 32 of the next unit
+    auto fetch = [&](int u) {
+      const bool win = u < nunit && (u >> 1) >= nbg;
+      const int base = win ? unit_key(u) : 0;
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const int q = base + lane + 32 * m;
+        fnext[m] = win && q <= qlast && (q < p.a || fl[q] != 0);
+      }
+    };
+    fetch(0);
+    for (int u = 0; u < nunit; ++u) {
+      const int st = u % kNst;
+      if (u >= kNst) {
+        bool go = true;
+        if (lane == 0) {
+          go = sep::mbar_wait(&bars.st_free[st], ((u / kNst) - 1) & 1, abort, p.err);
+          if (go) load_unit(u);
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+        issued = u + 1;
+      }
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint32_t w = __ballot_sync(0xffffffffu, fnext[m]);
+        if (lane == m) glb_w[st * 2 + m] = w;
+      }
+      fetch(u + 1);
+      sep::mbar_arrive(&bars.st_full[st]);
+    }
+    if (lane == 0 && *abort) {
+      int dummy = 0;
+      sep::mbar_wait(&bars.q_full, 0, &dummy, nullptr);
+      for (int u = issued - kNst < 0 ? 0 : issued - kNst; u < issued; ++u)
+        sep::mbar_wait(&bars.st_full[u % kNst], (u / kNst) & 1, &dummy, nullptr);
     }
     __syncwarp();
   }
@@ -1002,109 +927,76 @@ __global__ void __launch_bounds__(kTcThreads, 1) k_sep_bwd_tc_q(const BwdParams 
   }
 }
 
-// D = 128 runs the tcgen05 kernels.  At D = 64 they are correct too (the
-// same kernels with one 64-column tile per 128-row tensor) but slower than
-// the warp-level kernel on the Pythia-160M shape (0.54 against 0.37 ms per
-// step): TMEM holds one CTA per SM and the items there are small.
-template <int D>
-constexpr bool tc_backward() { return D == 128; }
-
+// Workspace: delta [B, Hq, S] fp32; fp32 dK and dV rows of the compact
+// global-key lists [B, Hkv, S, D] each; the compact bf16 K and V copies
+// [B, Hkv, S, D] each.
 struct BwdWs {
-  size_t delta, dq, dk, dv;
+  size_t delta, dk, dv, kc, vc;
+  size_t total() const { return delta + dk + dv + kc + vc; }
 };
 BwdWs bwd_ws(int B, int Hq, int Hkv, int S, int D) {
   auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
   BwdWs w;
   w.delta = r256(static_cast<size_t>(B) * Hq * S * 4);
-  w.dq = r256(static_cast<size_t>(B) * Hq * S * D * 4);
   w.dk = r256(static_cast<size_t>(B) * Hkv * S * D * 4);
   w.dv = w.dk;
+  w.kc = r256(static_cast<size_t>(B) * Hkv * S * D * 2);
+  w.vc = w.kc;
   return w;
 }
 
-// the tcgen05 kernels: dK, dV key-centric; dQ query-centric
 template <int D>
-int launch_bwd_tc(BwdParams p, void* dq, cudaStream_t st) {
+int launch_bwd(BwdParams p, const void* out, void* dq, void* dk, void* dv, void* ws,
+               cudaStream_t st) {
   static bool attr_done[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(k_sep_bwd_tc_kv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(k_bwd_kv<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              KvSmem<D>::BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(k_sep_bwd_tc_q<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(k_bwd_q<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              QSmem<D>::BYTES) != cudaSuccess)
       return SEP_ECUDA;
     attr_done[dev] = true;
   }
-  p.nwin = (p.S + TBK - 1) / TBK;
-  p.nchunk = (p.nwin + kTcChunkTiles - 1) / kTcChunkTiles;
-  const int64_t qrows = static_cast<int64_t>(p.B) * p.Hq * p.S;
-  if (qrows > 0x7fffffffLL) return SEP_ETOOBIG;
-  CUtensorMap mq, mdo;
-  if (!sep::make_rows_map(&mq, p.q, qrows, D, TBQ) || !sep::make_rows_map(&mdo, p.dout, qrows, D, TBQ))
-    return SEP_ECUDA;
-  k_sep_bwd_tc_kv<D><<<dim3(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B), kTcThreads, KvSmem<D>::BYTES, st>>>(p, mq, mdo);
-  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  k_sep_bwd_tc_q<D><<<dim3((p.S + TBQ - 1) / TBQ, p.Hq, p.B), kTcThreads, QSmem<D>::BYTES, st>>>(
-      p, static_cast<__nv_bfloat16*>(dq));
-  return cudaGetLastError() == cudaSuccess ? SEP_OK : SEP_ECUDA;
-}
-
-template <int D>
-int launch_bwd(const BwdParams& p0, const void* out, void* dq, void* dk, void* dv, void* ws,
-               cudaStream_t st) {
-  BwdParams p = p0;
   const BwdWs w = bwd_ws(p.B, p.Hq, p.Hkv, p.S, D);
   uint8_t* base = static_cast<uint8_t*>(ws);
   float* delta = reinterpret_cast<float*>(base);
   p.delta = delta;
-  p.dq_acc = reinterpret_cast<float*>(base + w.delta);
-  p.dk_acc = reinterpret_cast<float*>(base + w.delta + w.dq);
-  p.dv_acc = reinterpret_cast<float*>(base + w.delta + w.dq + w.dk);
-  constexpr bool tc = tc_backward<D>();  // dq is then written directly, in bf16
-  if (tc) {
-    if (cudaMemsetAsync(p.dk_acc, 0, w.dk + w.dv, st) != cudaSuccess) return SEP_ECUDA;
-  } else if (cudaMemsetAsync(p.dq_acc, 0, w.dq + w.dk + w.dv, st) != cudaSuccess) {
+  p.dk_acc = reinterpret_cast<float*>(base + w.delta);
+  p.dv_acc = reinterpret_cast<float*>(base + w.delta + w.dk);
+  __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(base + w.delta + w.dk + w.dv);
+  __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(base + w.delta + w.dk + w.dv + w.kc);
+  p.nwin = (p.S + TBK - 1) / TBK;
+  p.nchunk = (p.nwin + kTcChunkTiles - 1) / kTcChunkTiles;
+  const int64_t qrows = static_cast<int64_t>(p.B) * p.Hq * p.S;
+  const int64_t krows = static_cast<int64_t>(p.B) * p.Hkv * p.S;
+  if (qrows > 0x7fffffffLL) return SEP_ETOOBIG;
+  // 128-row boxes for the operands a CTA keeps (K, V of the key-centric
+  // kernel; Q, dO of the query-centric one), 64-row boxes for the ring units
+  CUtensorMap mq, mdo, mk, mv, mkc, mvc, uq, udo, uk, uv, ukc, uvc;
+  if (!sep::make_rows_map(&mq, p.q, qrows, D, TBQ) || !sep::make_rows_map(&mdo, p.dout, qrows, D, TBQ) ||
+      !sep::make_rows_map(&mk, p.k, krows, D, TBK) || !sep::make_rows_map(&mv, p.v, krows, D, TBK) ||
+      !sep::make_rows_map(&mkc, kc, krows, D, TBK) || !sep::make_rows_map(&mvc, vc, krows, D, TBK) ||
+      !sep::make_rows_map(&uq, p.q, qrows, D, 64) || !sep::make_rows_map(&udo, p.dout, qrows, D, 64) ||
+      !sep::make_rows_map(&uk, p.k, krows, D, 64) || !sep::make_rows_map(&uv, p.v, krows, D, 64) ||
+      !sep::make_rows_map(&ukc, kc, krows, D, 64) || !sep::make_rows_map(&uvc, vc, krows, D, 64))
     return SEP_ECUDA;
-  }
-  const int64_t rows = static_cast<int64_t>(p.B) * p.Hq * p.S;
-  k_bwd_delta<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(out), p.dout, delta, rows);
+  k_bwd_delta<D><<<static_cast<unsigned>((qrows + 7) / 8), 256, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(out), p.dout, delta, qrows);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  if (tc) {
-    const int rc = launch_bwd_tc<D>(p, dq, st);
-    if (rc != SEP_OK) return rc;
-  } else {
-  constexpr int smem = Smem<D>::BYTES;
-  static bool attr_done[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(k_sep_bwd<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-      return SEP_ECUDA;
-    attr_done[dev] = true;
-  }
-  dim3 grid(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B);
-  k_sep_bwd<D><<<grid, kThreads, smem, st>>>(p);
+  const dim3 rgrid((p.S + 63) / 64, p.Hkv, p.B);
+  k_bwd_prep<D><<<rgrid, 256, 0, st>>>(p, kc, vc);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  }
-  const float sc = p.scale_log2 / 1.44269504088896340736f;
-  struct {
-    const float* acc;
-    void* dst;
-    int64_t n;
-    float mul;
-  } conv[3] = {{p.dq_acc, dq, rows * D, sc},
-               {p.dk_acc, dk, static_cast<int64_t>(p.B) * p.Hkv * p.S * D, sc},
-               {p.dv_acc, dv, static_cast<int64_t>(p.B) * p.Hkv * p.S * D, 1.f}};
-  for (auto& c : conv) {
-    if (tc && c.dst == dq) continue;  // already written
-    const int64_t n4 = c.n / 4;
-    const int blocks = static_cast<int>(n4 / 256 + 1 < 148 * 16 ? n4 / 256 + 1 : 148 * 16);
-    k_bwd_convert<<<blocks, 256, 0, st>>>(c.acc, static_cast<__nv_bfloat16*>(c.dst), n4, c.mul);
-    if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  }
+  k_bwd_kv<D><<<dim3(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B), kTcThreads, KvSmem<D>::BYTES, st>>>(
+      p, uq, udo, mk, mv, mkc, mvc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  k_bwd_q<D><<<dim3((p.S + TBQ - 1) / TBQ, p.Hq, p.B), kTcThreads, QSmem<D>::BYTES, st>>>(
+      p, mq, mdo, uk, uv, ukc, uvc, static_cast<__nv_bfloat16*>(dq));
+  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  k_bwd_scatter<D><<<rgrid, 256, 0, st>>>(p, p.scale_log2 / 1.44269504088896340736f,
+                                           static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
+  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   return sep::launch_status();
 }
 
@@ -1112,8 +1004,7 @@ int launch_bwd(const BwdParams& p0, const void* out, void* dq, void* dk, void* d
 
 extern "C" size_t sep_attn_backward_workspace(int B, int Hq, int Hkv, int S, int D) {
   if (B < 1 || Hq < 1 || Hkv < 1 || S < 1 || Hq % Hkv != 0 || (D != 64 && D != 128)) return 0;
-  const BwdWs w = bwd_ws(B, Hq, Hkv, S, D);
-  return w.delta + w.dq + w.dk + w.dv;
+  return bwd_ws(B, Hq, Hkv, S, D).total();
 }
 
 extern "C" int sep_attn_backward(const void* q, const void* k, const void* v, const void* out,
@@ -1151,8 +1042,6 @@ extern "C" int sep_attn_backward(const void* q, const void* k, const void* v, co
   p.S = S;
   p.a = a;
   p.n = n;
-  p.nwin = (S + BC - 1) / BC;
-  p.nchunk = (p.nwin + kChunkTiles - 1) / kChunkTiles;
   const float sc = scale > 0.f ? scale : 1.f / sqrtf(static_cast<float>(D));
   p.scale_log2 = sc * 1.44269504088896340736f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
