@@ -38,6 +38,8 @@ struct BwdParams {
   const uint8_t* is_sep;
   const int32_t *prefix, *idx;
   float *dk_acc, *dv_acc;  // fp32 dK, dV rows of the compact global-key lists
+  int2* items;             // global-key work items (k_bwd_plan)
+  int32_t* item_count;     // their number
   int32_t* err;
   int B, Hq, Hkv, S, a, n;
   int nwin;    // window items per (b, kv head) = ceil(S / 128)
@@ -285,24 +287,96 @@ __device__ __forceinline__ void probs_grads(const uint32_t (&sv)[32], const uint
   }
 }
 
-// Shared memory of the key-centric kernel: K, V [128][D] (swizzled
-// 64-column tiles); a ring of kNst unit stages, each the unit's Q and dO
-// rows [64][D]; -lse (log2 domain) and delta [kNst][64] fp32; key
-// positions and use flags [128] int32.
+// ---- work items
+//
+// Key-centric items: the global-key items (listed by k_bwd_plan, heaviest
+// first), each for every kv head, then the window items (b, kv head, block
+// of 128 positions).  Query-centric items: (b, head, tile of 128 queries),
+// tiles with more kept keys (later positions) first.  Both kernels are
+// persistent: CTA c takes items c, c + gridDim.x, ... in order, so every
+// role of the CTA walks the same sequence without handing items around.
+
+// The global-key items: for every sequence b and block kb of 128 global
+// keys, the chunks of kTcChunkTiles query tiles from the tile of the
+// block's first key to the last tile, as (b, kb << 16 | chunk).  One warp.
+__global__ void __launch_bounds__(32) k_bwd_plan(const BwdParams p) {
+  const int lane = threadIdx.x;
+  const int nT = (p.S + TBQ - 1) / TBQ;
+  int e = 0;
+  for (int b = 0; b < p.B; ++b) {
+    const GlobalList gl(p, b);
+    const int nb = (gl.total + TBK - 1) / TBK;
+    for (int k0 = 0; k0 < nb; k0 += 32) {
+      const int kb = k0 + lane;
+      int nch = 0;
+      if (kb < nb) {
+        const int pos = gl.pos(kb * TBK);
+        const int t0 = (pos >= 0 && pos < p.S ? pos : 0) / TBQ;
+        nch = (nT - t0 + kTcChunkTiles - 1) / kTcChunkTiles;
+      }
+      int incl = nch;  // inclusive prefix over the warp
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      for (int c = 0; c < nch; ++c) p.items[e + incl - nch + c] = make_int2(b, (kb << 16) | c);
+      e += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  if (lane == 0) *p.item_count = e;
+}
+
+struct KvItem {
+  int b, g, kb, t0, ntile;
+  bool window;
+};
+__device__ __forceinline__ KvItem kv_item(const BwdParams& p, int i, int nglob) {
+  KvItem it;
+  const int nT = (p.S + TBQ - 1) / TBQ;
+  if (i < nglob) {
+    const int2 ent = p.items[i / p.Hkv];
+    it.g = i % p.Hkv;
+    it.b = ent.x;
+    it.kb = ent.y >> 16;
+    const GlobalList gl(p, it.b);
+    const int pos = gl.pos(it.kb * TBK);
+    it.t0 = (pos >= 0 && pos < p.S ? pos : 0) / TBQ + (ent.y & 0xffff) * kTcChunkTiles;
+    const int t1 = it.t0 + kTcChunkTiles < nT ? it.t0 + kTcChunkTiles : nT;
+    it.ntile = t1 - it.t0;
+    it.window = false;
+  } else {
+    const int w = i - nglob;
+    it.kb = w % p.nwin;
+    it.g = (w / p.nwin) % p.Hkv;
+    it.b = w / (p.nwin * p.Hkv);
+    it.t0 = it.kb;
+    const int last = it.kb * TBK + TBK - 1 + p.n - 1;
+    it.ntile = (last < p.S - 1 ? last : p.S - 1) / TBQ + 1 - it.t0;
+    it.window = true;
+  }
+  return it;
+}
+
+// Shared memory of the key-centric kernel: KVB buffers of an item's K and V
+// [128][D] (swizzled 64-column tiles; two buffers where they fit, so the
+// next item's keys load during the current one); a ring of kNst unit
+// stages, each the unit's Q and dO rows [64][D]; -lse (log2 domain) and
+// delta [kNst][64] fp32.
 template <int D>
 struct KvSmem {
   static constexpr int NB = D / 64;
-  static constexpr int K = 0, V = NB * kT128, RING = 2 * NB * kT128;
+  static constexpr int KVB = D == 64 ? 2 : 1;
+  static constexpr int KVSZ = 2 * NB * kT128;  // K tiles, then V tiles
+  static constexpr int RING = KVB * KVSZ;
   static constexpr int STAGE = 2 * NB * kT64;  // Q tiles, then dO tiles
   static constexpr int LSE = RING + kNst * STAGE;
   static constexpr int DEL = LSE + kNst * 64 * 4;
-  static constexpr int POS = DEL + kNst * 64 * 4;
-  static constexpr int USE = POS + 512;
-  static constexpr int BYTES = USE + 512 + 1024;  // + alignment slack
+  static constexpr int BYTES = DEL + kNst * 64 * 4 + 1024;  // + alignment slack
 };
 struct KvBars {
-  uint64_t kv_full, fin, drain;
-  uint64_t st_full[kNst], st_free[kNst], s_full[2], p_full[2];
+  uint64_t kv_full[2], kv_free[2], st_full[kNst], st_free[kNst], s_full[2], p_full[2];
+  uint64_t fin, acc_free, drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -316,6 +390,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
              __nv_bfloat16* __restrict__ dv) {
   using Sm = KvSmem<D>;
   constexpr int NB = D / 64;
+  constexpr int KVB = Sm::KVB;
   constexpr uint32_t kColDK = col_dk<D>();
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* const smem = reinterpret_cast<uint8_t*>(
@@ -324,61 +399,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t sb_ = sep::smem_u32(smem);
   float* const lse_s = reinterpret_cast<float*>(smem + Sm::LSE);
   float* const del_s = reinterpret_cast<float*>(smem + Sm::DEL);
-  int32_t* const pos_s = reinterpret_cast<int32_t*>(smem + Sm::POS);
-  int32_t* const use_s = reinterpret_cast<int32_t*>(smem + Sm::USE);
 
-  const int item = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.S, G = p.Hq / p.Hkv;
-  const int nT = (S + TBQ - 1) / TBQ;
-  const uint8_t* fl = p.is_sep + static_cast<int64_t>(b) * S;
-  const GlobalList gl(p, b);
-
-  const bool window = item < p.nwin;
-  int kb, t0, t1;
-  if (window) {
-    kb = item;
-    t0 = kb;
-    const int last = kb * TBK + TBK - 1 + p.n - 1;
-    t1 = (last < S - 1 ? last : S - 1) / TBQ + 1;
-  } else {
-    kb = (item - p.nwin) / p.nchunk;
-    const int chunk = (item - p.nwin) % p.nchunk;
-    if (kb * TBK >= gl.total) return;
-    t0 = gl.pos(kb * TBK) / TBQ + chunk * kTcChunkTiles;
-    t1 = t0 + kTcChunkTiles < nT ? t0 + kTcChunkTiles : nT;
-    if (t0 >= nT) return;
-  }
-  const int ntile = t1 - t0;
-  const int nvisit = G * ntile;
-  const int nunit = 2 * nvisit;
-  const int64_t kvrow0 = (static_cast<int64_t>(b) * p.Hkv + g) * S;
-  // unit u: queries [64 (u & 1), +64) of the tile of visit u >> 1, whose
-  // first row in the [B * Hq * S] view is unit_row(u)
-  auto unit_row = [&](int u) -> int64_t {
+  const int nglob = *p.item_count * p.Hkv;
+  const int nitems = nglob + p.B * p.Hkv * p.nwin;
+  // first row of unit u of item `it` (queries [64 (u & 1), +64) of the
+  // tile of visit u >> 1) in the [B * Hq * S] view
+  auto unit_row = [&](const KvItem& it, int u) -> int64_t {
     const int v = u >> 1;
-    return (static_cast<int64_t>(b) * p.Hq + g * G + v / ntile) * S + (t0 + v % ntile) * TBQ +
-           64 * (u & 1);
-  };
-  // the unit's Q and dO rows into stage u % kNst (its bytes, no arrival)
-  auto load_unit = [&](int u) {
-    const int st = u % kNst;
-    uint8_t* dst = smem + Sm::RING + st * Sm::STAGE;
-    const int32_t row = static_cast<int32_t>(unit_row(u));
-    mbar_expect_tx(&bars.st_full[st], Sm::STAGE);
-#pragma unroll
-    for (int c = 0; c < NB; ++c) {
-      sep::tma_load_2d(dst + c * kT64, &map_q, 64 * c, row, &bars.st_full[st]);
-      sep::tma_load_2d(dst + (NB + c) * kT64, &map_do, 64 * c, row, &bars.st_full[st]);
-    }
+    return (static_cast<int64_t>(it.b) * p.Hq + it.g * G + v / it.ntile) * S +
+           (it.t0 + v % it.ntile) * TBQ + 64 * (u & 1);
   };
 
   if (threadIdx.x == 9 * 32) {
-    // the load warp's first lane: barriers, then at once the K / V copies
-    // and the first kNst units (the ring starts free)
-    sep::mbar_init(&bars.kv_full, 1);
-    sep::mbar_init(&bars.fin, 1);
-    sep::mbar_init(&bars.drain, 1);
+    for (int i = 0; i < KVB; ++i) {
+      sep::mbar_init(&bars.kv_full[i], 1);
+      sep::mbar_init(&bars.kv_free[i], 1);
+    }
     for (int i = 0; i < kNst; ++i) {
       sep::mbar_init(&bars.st_full[i], 32);  // the load warp's lanes, after the statistics
       sep::mbar_init(&bars.st_free[i], 1);
@@ -387,31 +425,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       sep::mbar_init(&bars.s_full[i], 1);
       sep::mbar_init(&bars.p_full[i], 8);
     }
+    sep::mbar_init(&bars.fin, 1);
+    sep::mbar_init(&bars.acc_free, 8);
+    sep::mbar_init(&bars.drain, 1);
     // a wait of an earlier CTA gave up: this one ends at its first wait too
     bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
     sep::mbar_fence_init();
-    sep::mbar_arrive_expect_tx(&bars.kv_full, 2 * NB * kT128);
-    const int32_t row = static_cast<int32_t>(kvrow0 + kb * TBK);
-    load_tile128<D>(smem + Sm::K, window ? &map_k : &map_kc, row, &bars.kv_full);
-    load_tile128<D>(smem + Sm::V, window ? &map_v : &map_vc, row, &bars.kv_full);
-    for (int u = 0; u < kNst && u < nunit; ++u) load_unit(u);
-  }
-  if (threadIdx.x < TBK) {
-    const int r = threadIdx.x;
-    int pos = -1, use = 0;
-    if (window) {
-      pos = kb * TBK + r;
-      use = pos < S && !(pos < p.a || fl[pos]);
-      if (pos >= S) pos = -1;
-    } else {
-      const int t = kb * TBK + r;
-      if (t < gl.total) {
-        pos = gl.pos(t);
-        use = 1;
-      }
-    }
-    pos_s[r] = pos;
-    use_s[r] = use;
   }
   if (warp == 8) {
     sep::tmem_alloc(&bars.tmem_base, 512);
@@ -428,66 +447,88 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int lq = warp & 3, ch = warp >> 2;
     const int r = 32 * lq + lane;  // key row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * lq) << 16;
-    const int jp = pos_s[r], use = use_s[r];
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
+    const float sc = p.scale_log2 * 0.69314718055994530942f;
     bool ok = true;
-    for (int u = 0; u < nunit && ok; ++u) {
-      const int v = u >> 1, hh = u & 1, sb = u & 1, st = u % kNst;
-      const int i0 = (t0 + v % ntile) * TBQ;
-      if (!warp_wait(&bars.st_full[st], (u / kNst) & 1, abort, p.err)) {
-        ok = false;  // (the unit's statistics are in shared memory)
-        break;
+    uint32_t U = 0, I = 0;  // units and items of this CTA so far
+    for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
+      const KvItem it = kv_item(p, i, nglob);
+      const int nunit = 2 * G * it.ntile;
+      const int64_t kvrow0 = (static_cast<int64_t>(it.b) * p.Hkv + it.g) * S;
+      // this thread's key: position jp, kept by this item's queries?
+      int jp = -1, use = 0;
+      if (it.window) {
+        const int q = it.kb * TBK + r;
+        if (q < S) {
+          jp = q;
+          use = !(q < p.a || p.is_sep[static_cast<int64_t>(it.b) * S + q]);
+        }
+      } else {
+        const GlobalList gl(p, it.b);
+        const int t = it.kb * TBK + r;
+        if (t < gl.total) {
+          jp = gl.pos(t);
+          use = 1;
+        }
       }
-      if (!warp_wait(&bars.s_full[sb], (u >> 1) & 1, abort, p.err)) {
+      for (int u = 0; u < nunit; ++u) {
+        const uint32_t gu = U + u;
+        const int v = u >> 1, hh = u & 1, sb = gu & 1, st = gu % kNst;
+        const int i0 = (it.t0 + v % it.ntile) * TBQ;
+        if (!warp_wait(&bars.st_full[st], (gu / kNst) & 1, abort, p.err) ||
+            !warp_wait(&bars.s_full[sb], (gu >> 1) & 1, abort, p.err)) {
+          ok = false;
+          break;
+        }
+        sep::tc_fence_after();
+        // the unit columns this key row keeps: [qa, qb) relative to column
+        // 64 hh + 32 ch of the tile
+        int qa = 0, qb = 0;
+        if (use && jp >= 0) {
+          qa = jp - i0 > 0 ? jp - i0 : 0;
+          qb = S - i0 < TBQ ? S - i0 : TBQ;
+          if (it.window && jp + p.n - i0 < qb) qb = jp + p.n - i0;
+        }
+        const int c0 = 64 * hh + 32 * ch;
+        const uint32_t keep = bit_range(qa - c0, qb - c0);
+        const uint32_t cs = 128u * sb + 32u * ch;
+        uint32_t pp[16], dd[16];
+        if (__all_sync(0xffffffffu, keep == 0u)) {
+          // no column of the warp's rows is kept: P^T and dS^T are zero
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pp[e] = dd[e] = 0u;
+        } else {
+          uint32_t sv[32], dv_[32];
+          sep::tmem_ld32(tmem + lane_base + cs, sv);
+          sep::tmem_ld32(tmem + lane_base + cs + 64, dv_);
+          sep::tmem_wait_ld_r32(sv);
+          sep::tmem_wait_ld_r32(dv_);
+          const float* nl = lse_s + st * 64 + 32 * ch;
+          const float* dl = del_s + st * 64 + 32 * ch;
+          const float2 z2 = make_float2(0.f, 0.f);
+          if (__all_sync(0xffffffffu, keep == 0xffffffffu))
+            probs_grads<false, true>(sv, dv_, nl, dl, z2, z2, sc2, keep, pp, dd);
+          else
+            probs_grads<true, true>(sv, dv_, nl, dl, z2, z2, sc2, keep, pp, dd);
+        }
+        sep::tmem_st16(tmem + lane_base + cs, pp);
+        sep::tmem_st16(tmem + lane_base + cs + 64, dd);
+        sep::tmem_wait_st();
+        sep::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sep::mbar_arrive(&bars.p_full[sb]);
+      }
+      if (!ok || !warp_wait(&bars.fin, I & 1, abort, p.err)) {
         ok = false;
         break;
       }
       sep::tc_fence_after();
-      // the unit columns this key row keeps: [qa, qb) relative to column
-      // 64 hh + 32 ch of the tile
-      int qa = 0, qb = 0;
-      if (use && jp >= 0) {
-        qa = jp - i0 > 0 ? jp - i0 : 0;
-        qb = S - i0 < TBQ ? S - i0 : TBQ;
-        if (window && jp + p.n - i0 < qb) qb = jp + p.n - i0;
-      }
-      const int c0 = 64 * hh + 32 * ch;
-      const uint32_t keep = bit_range(qa - c0, qb - c0);
-      const uint32_t cs = 128u * sb + 32u * ch;
-      uint32_t pp[16], dd[16];
-      if (__all_sync(0xffffffffu, keep == 0u)) {
-        // no column of the warp's rows is kept: P^T and dS^T are zero
-#pragma unroll
-        for (int e = 0; e < 16; ++e) pp[e] = dd[e] = 0u;
-      } else {
-        uint32_t sv[32], dv_[32];
-        sep::tmem_ld32(tmem + lane_base + cs, sv);
-        sep::tmem_ld32(tmem + lane_base + cs + 64, dv_);
-        sep::tmem_wait_ld_r32(sv);
-        sep::tmem_wait_ld_r32(dv_);
-        const float* nl = lse_s + st * 64 + 32 * ch;
-        const float* dl = del_s + st * 64 + 32 * ch;
-        const float2 z2 = make_float2(0.f, 0.f);
-        if (__all_sync(0xffffffffu, keep == 0xffffffffu))
-          probs_grads<false, true>(sv, dv_, nl, dl, z2, z2, sc2, keep, pp, dd);
-        else
-          probs_grads<true, true>(sv, dv_, nl, dl, z2, z2, sc2, keep, pp, dd);
-      }
-      sep::tmem_st16(tmem + lane_base + cs, pp);
-      sep::tmem_st16(tmem + lane_base + cs + 64, dd);
-      sep::tmem_wait_st();
-      sep::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) sep::mbar_arrive(&bars.p_full[sb]);
-    }
-    if (ok && warp_wait(&bars.fin, 0, abort, p.err)) {
-      sep::tc_fence_after();
       // dK and dV of this key row, columns [D/2 ch, +D/2): every lane loads
-      // (warp-wide); a window key is stored as bf16, a global key's partial
-      // sum is added to its fp32 row of the compact list
+      // (warp-wide); once the last load is in, the accumulators are handed
+      // back to the next item.  A window key is stored as bf16, a global
+      // key's partial sum is added to its fp32 row of the compact list.
       const bool mine = jp >= 0 && use;
-      const int64_t row = kvrow0 + (window ? (mine ? jp : 0) : kb * TBK + r);
-      const float sc = p.scale_log2 * 0.69314718055994530942f;
+      const int64_t row = kvrow0 + (it.window ? (mine ? jp : 0) : it.kb * TBK + r);
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t kv[32], vv[32];
@@ -496,8 +537,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         sep::tmem_ld32(tmem + lane_base + kColAcc + col, vv);
         sep::tmem_wait_ld_r32(kv);
         sep::tmem_wait_ld_r32(vv);
+        if (c == D / 64 - 1) {
+          sep::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) sep::mbar_arrive(&bars.acc_free);
+        }
         if (!mine) continue;
-        if (window) {
+        if (it.window) {
           uint4* kd = reinterpret_cast<uint4*>(dk + row * D + col);
           uint4* vd = reinterpret_cast<uint4*>(dv + row * D + col);
 #pragma unroll
@@ -521,59 +567,78 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
+      U += nunit;
     }
   } else if (warp == 8) {
     if (lane == 0) {
       // ---------------------------------------------- MMA issue (one thread)
       constexpr uint32_t id_s = idesc_mn(128, 64, false, false);
       constexpr uint32_t id_o = idesc_mn(128, D, false, true);
-      const uint64_t dK = sep::smem_desc_sw128(sb_ + Sm::K, 16);
-      const uint64_t dV = sep::smem_desc_sw128(sb_ + Sm::V, 16);
-      bool ok = nvisit > 0 && sep::mbar_wait(&bars.kv_full, 0, abort, p.err);
-      for (int u = 0; u <= nunit && ok; ++u) {
-        if (u < nunit) {
-          // scores of unit u into buffer u & 1 (its previous contents, unit
-          // u-2, were read by the products issued before this point)
-          const int st = u % kNst;
-          if (!sep::mbar_wait(&bars.st_full[st], (u / kNst) & 1, abort, p.err)) {
-            ok = false;
-            break;
-          }
-          sep::tc_fence_after();
-          const uint32_t qa = sb_ + Sm::RING + st * Sm::STAGE, oa = qa + NB * kT64;
-          const uint64_t dQ = sep::smem_desc_sw128(qa, 16), dO = sep::smem_desc_sw128(oa, 16);
-          const uint32_t cs = 128u * (u & 1);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t kofs = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
-            const uint64_t oq = static_cast<uint64_t>(((kk / 4) * kT64 + (kk % 4) * 32) >> 4);
-            sep::mma_bf16_ss(tmem + cs, dK + kofs, dQ + oq, id_s, kk > 0 ? 1u : 0u);
-            sep::mma_bf16_ss(tmem + cs + 64, dV + kofs, dO + oq, id_s, kk > 0 ? 1u : 0u);
-          }
-          sep::mma_commit(&bars.s_full[u & 1]);
+      bool ok = true;
+      uint32_t U = 0, I = 0;
+      for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
+        const KvItem it = kv_item(p, i, nglob);
+        const int nunit = 2 * G * it.ntile;
+        const int kbuf = I % KVB;
+        if (!sep::mbar_wait(&bars.kv_full[kbuf], (I / KVB) & 1, abort, p.err)) {
+          ok = false;
+          break;
         }
-        if (u >= 1) {
-          // gradient products of unit w = u - 1 once its P^T and dS^T are in
-          const int w = u - 1, wst = w % kNst;
-          if (!sep::mbar_wait(&bars.p_full[w & 1], (w >> 1) & 1, abort, p.err)) {
-            ok = false;
-            break;
-          }
-          sep::tc_fence_after();
-          const uint32_t qa = sb_ + Sm::RING + wst * Sm::STAGE, oa = qa + NB * kT64;
-          const uint64_t dQmn = sep::smem_desc_sw128(qa, kT64), dOmn = sep::smem_desc_sw128(oa, kT64);
-          const uint32_t cs = 128u * (w & 1);
+        const uint64_t dK = sep::smem_desc_sw128(sb_ + kbuf * Sm::KVSZ, 16);
+        const uint64_t dV = sep::smem_desc_sw128(sb_ + kbuf * Sm::KVSZ + NB * kT128, 16);
+        for (int u = 0; u <= nunit; ++u) {
+          if (u < nunit) {
+            // scores of unit u into buffer (U + u) & 1 (its previous
+            // contents were read by the products issued before this point)
+            const uint32_t gu = U + u;
+            const int st = gu % kNst;
+            if (!sep::mbar_wait(&bars.st_full[st], (gu / kNst) & 1, abort, p.err)) {
+              ok = false;
+              break;
+            }
+            sep::tc_fence_after();
+            const uint32_t qa = sb_ + Sm::RING + st * Sm::STAGE, oa = qa + NB * kT64;
+            const uint64_t dQ = sep::smem_desc_sw128(qa, 16), dO = sep::smem_desc_sw128(oa, 16);
+            const uint32_t cs = 128u * (gu & 1);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
-            const uint32_t acc = (w > 0 || kk > 0) ? 1u : 0u;
-            sep::mma_bf16_ts(tmem + kColAcc, tmem + unit_acol(cs, kk), dOmn + off, id_o, acc);
-            sep::mma_bf16_ts(tmem + kColDK, tmem + unit_acol(cs + 64, kk), dQmn + off, id_o, acc);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t kofs = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
+              const uint64_t qofs = static_cast<uint64_t>(((kk / 4) * kT64 + (kk % 4) * 32) >> 4);
+              sep::mma_bf16_ss(tmem + cs, dK + kofs, dQ + qofs, id_s, kk > 0 ? 1u : 0u);
+              sep::mma_bf16_ss(tmem + cs + 64, dV + kofs, dO + qofs, id_s, kk > 0 ? 1u : 0u);
+            }
+            sep::mma_commit(&bars.s_full[gu & 1]);
+            if (u == nunit - 1) sep::mma_commit(&bars.kv_free[kbuf]);  // the item's K, V are read
           }
-          sep::mma_commit(&bars.st_free[wst]);  // the stage may be refilled
+          if (u >= 1) {
+            // gradient products of unit u - 1 once its P^T and dS^T are in
+            // (and, for the item's first, once the previous item's dK, dV
+            // have been read out)
+            const uint32_t w = U + u - 1;
+            const int wst = w % kNst;
+            if (!sep::mbar_wait(&bars.p_full[w & 1], (w >> 1) & 1, abort, p.err) ||
+                (u == 1 && I > 0 && !sep::mbar_wait(&bars.acc_free, (I - 1) & 1, abort, p.err))) {
+              ok = false;
+              break;
+            }
+            sep::tc_fence_after();
+            const uint32_t qa = sb_ + Sm::RING + wst * Sm::STAGE, oa = qa + NB * kT64;
+            const uint64_t dQmn = sep::smem_desc_sw128(qa, kT64), dOmn = sep::smem_desc_sw128(oa, kT64);
+            const uint32_t cs = 128u * (w & 1);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
+              const uint32_t acc = (u > 1 || kk > 0) ? 1u : 0u;
+              sep::mma_bf16_ts(tmem + kColAcc, tmem + unit_acol(cs, kk), dOmn + off, id_o, acc);
+              sep::mma_bf16_ts(tmem + kColDK, tmem + unit_acol(cs + 64, kk), dQmn + off, id_o, acc);
+            }
+            sep::mma_commit(&bars.st_free[wst]);  // the stage may be refilled
+          }
         }
+        if (!ok) break;
+        sep::mma_commit(&bars.fin);
+        U += nunit;
       }
-      if (ok) sep::mma_commit(&bars.fin);
       sep::mma_commit(&bars.drain);  // every MMA completes before TMEM is released
       int keep = 0;
       sep::mbar_wait(&bars.drain, 0, &keep, nullptr);
@@ -581,50 +646,75 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------ loads (warp 9)
-    // (K, V and the first kNst units were started before the block
-    // barrier.)  Per unit: the copies once its stage is free, then the
-    // unit's -lse (log2 domain) and delta, read one unit ahead into
-    // registers (rows lane, lane + 32), then the 32 arrivals that complete
-    // the stage with its bytes.
-    int issued = nunit < kNst ? nunit : kNst;  // units whose copies were started
-    float nlr[2], dlr[2];
-    auto fetch = [&](int u) {
-      if (u >= nunit) return;
-      const int64_t row0 = unit_row(u);
-      const int i0 = (t0 + (u >> 1) % ntile) * TBQ + 64 * (u & 1);
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const int e = lane + 32 * m;
-        nlr[m] = i0 + e < S ? -p.lse[row0 + e] * 1.44269504088896340736f : 0.f;
-        dlr[m] = i0 + e < S ? p.delta[row0 + e] : 0.f;
-      }
-    };
-    fetch(0);
-    for (int u = 0; u < nunit; ++u) {
-      const int st = u % kNst;
-      if (u >= kNst) {
-        bool go = true;
-        if (lane == 0) {
-          go = sep::mbar_wait(&bars.st_free[st], ((u / kNst) - 1) & 1, abort, p.err);
-          if (go) load_unit(u);
+    // Per item: its K and V once their buffer is free; per unit: the copies
+    // once its stage is free, the unit's -lse (log2 domain) and delta (rows
+    // lane, lane + 32), then the 32 arrivals that complete the stage with
+    // its bytes.
+    uint32_t U = 0, I = 0;
+    uint32_t issued_u = 0, issued_i = 0;  // copies started (units, items)
+    bool ok = true;
+    for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
+      const KvItem it = kv_item(p, i, nglob);
+      const int nunit = 2 * G * it.ntile;
+      const int kbuf = I % KVB;
+      bool go = true;
+      if (lane == 0) {
+        if (I >= KVB) go = sep::mbar_wait(&bars.kv_free[kbuf], ((I - KVB) / KVB) & 1, abort, p.err);
+        if (go) {
+          sep::mbar_arrive_expect_tx(&bars.kv_full[kbuf], Sm::KVSZ);
+          const int32_t row = static_cast<int32_t>((static_cast<int64_t>(it.b) * p.Hkv + it.g) * S + it.kb * TBK);
+          load_tile128<D>(smem + kbuf * Sm::KVSZ, it.window ? &map_k : &map_kc, row, &bars.kv_full[kbuf]);
+          load_tile128<D>(smem + kbuf * Sm::KVSZ + NB * kT128, it.window ? &map_v : &map_vc, row,
+                          &bars.kv_full[kbuf]);
         }
-        if (!__shfl_sync(0xffffffffu, go, 0)) break;
-        issued = u + 1;
       }
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      issued_i = I + 1;
+      for (int u = 0; u < nunit; ++u) {
+        const uint32_t gu = U + u;
+        const int st = gu % kNst;
+        const int64_t row0 = unit_row(it, u);
+        const int i0 = (it.t0 + (u >> 1) % it.ntile) * TBQ + 64 * (u & 1);
+        float nlr[2], dlr[2];  // loads in flight during the wait below
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        lse_s[st * 64 + lane + 32 * m] = nlr[m];
-        del_s[st * 64 + lane + 32 * m] = dlr[m];
+        for (int m = 0; m < 2; ++m) {
+          const int e = lane + 32 * m;
+          nlr[m] = i0 + e < S ? -p.lse[row0 + e] * 1.44269504088896340736f : 0.f;
+          dlr[m] = i0 + e < S ? p.delta[row0 + e] : 0.f;
+        }
+        if (lane == 0) {
+          if (gu >= kNst) go = sep::mbar_wait(&bars.st_free[st], ((gu / kNst) - 1) & 1, abort, p.err);
+          if (go) {
+            uint8_t* dst = smem + Sm::RING + st * Sm::STAGE;
+            mbar_expect_tx(&bars.st_full[st], Sm::STAGE);
+#pragma unroll
+            for (int c = 0; c < NB; ++c) {
+              sep::tma_load_2d(dst + c * kT64, &map_q, 64 * c, static_cast<int32_t>(row0), &bars.st_full[st]);
+              sep::tma_load_2d(dst + (NB + c) * kT64, &map_do, 64 * c, static_cast<int32_t>(row0), &bars.st_full[st]);
+            }
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) {
+          ok = false;
+          break;
+        }
+        issued_u = gu + 1;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          lse_s[st * 64 + lane + 32 * m] = nlr[m];
+          del_s[st * 64 + lane + 32 * m] = dlr[m];
+        }
+        sep::mbar_arrive(&bars.st_full[st]);
       }
-      fetch(u + 1);
-      sep::mbar_arrive(&bars.st_full[st]);
+      U += nunit;
     }
     // after an abort, let the started copies land before the CTA can exit
     if (lane == 0 && *abort) {
       int dummy = 0;
-      if (nvisit > 0) sep::mbar_wait(&bars.kv_full, 0, &dummy, nullptr);
-      for (int u = issued - kNst < 0 ? 0 : issued - kNst; u < issued; ++u)
-        sep::mbar_wait(&bars.st_full[u % kNst], (u / kNst) & 1, &dummy, nullptr);
+      for (uint32_t j = issued_i > KVB ? issued_i - KVB : 0; j < issued_i; ++j)
+        sep::mbar_wait(&bars.kv_full[j % KVB], (j / KVB) & 1, &dummy, nullptr);
+      for (uint32_t g2 = issued_u > kNst ? issued_u - kNst : 0; g2 < issued_u; ++g2)
+        sep::mbar_wait(&bars.st_full[g2 % kNst], (g2 / kNst) & 1, &dummy, nullptr);
     }
     __syncwarp();
   }
@@ -637,24 +727,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-// Shared memory of the query-centric kernel: Q, dO [128][D] (swizzled
-// 64-column tiles); a ring of kNst unit stages, each the unit's K and V rows
-// [64][D]; the global flags of each stage's keys as [kNst][2] 32-bit words
-// (bit k of word m: key 32 m + k of the unit).
+// Shared memory of the query-centric kernel: QB buffers of an item's Q and
+// dO [128][D] (swizzled 64-column tiles; two where they fit); a ring of kNst
+// unit stages, each the unit's K and V rows [64][D]; the global flags of
+// each stage's keys as [kNst][2] 32-bit words (bit k of word m: key 32 m + k
+// of the unit).
 template <int D>
 struct QSmem {
   static constexpr int NB = D / 64;
-  static constexpr int Q = 0, DO = NB * kT128, RING = 2 * NB * kT128;
+  static constexpr int QB = D == 64 ? 2 : 1;
+  static constexpr int QSZ = 2 * NB * kT128;  // Q tiles, then dO tiles
+  static constexpr int RING = QB * QSZ;
   static constexpr int STAGE = 2 * NB * kT64;  // K tiles, then V tiles
   static constexpr int GLB = RING + kNst * STAGE;
   static constexpr int BYTES = GLB + 1024 + 1024;
 };
 struct QBars {
-  uint64_t q_full, fin, drain;
-  uint64_t st_full[kNst], st_free[kNst], s_full[2], p_full[2];
+  uint64_t q_full[2], q_free[2], st_full[kNst], st_free[kNst], s_full[2], p_full[2];
+  uint64_t fin, acc_free, drain;
   uint32_t tmem_base;
   int abort;
 };
+struct QItem {
+  int b, h, t, lo, qlast, nglo, nbg, nblk;
+};
+__device__ __forceinline__ QItem q_item(const BwdParams& p, int i) {
+  QItem it;
+  const int nT = (p.S + TBQ - 1) / TBQ;
+  const int bh = p.B * p.Hq;
+  it.t = nT - 1 - i / bh;
+  it.h = (i % bh) % p.Hq;
+  it.b = (i % bh) / p.Hq;
+  const int i0 = it.t * TBQ;
+  it.qlast = (i0 + TBQ < p.S ? i0 + TBQ : p.S) - 1;
+  // the tile's kept keys: global keys before the first row's window (the
+  // head of the compact list), then the window positions [lo, qlast]
+  it.lo = i0 - p.n + 1 > 0 ? i0 - p.n + 1 : 0;
+  const int32_t* pre = p.prefix + static_cast<int64_t>(it.b) * (p.S + 1);
+  const int al = p.a < it.lo ? p.a : it.lo;
+  it.nglo = al + (pre[it.lo] - pre[al]);
+  it.nbg = (it.nglo + TBK - 1) / TBK;
+  it.nblk = it.nbg + (it.qlast - it.lo + TBK) / TBK;
+  return it;
+}
 
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -664,6 +779,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const __grid_constant__ CUtensorMap map_vc, __nv_bfloat16* __restrict__ dq) {
   using Sm = QSmem<D>;
   constexpr int NB = D / 64;
+  constexpr int QB = Sm::QB;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* const smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -671,51 +787,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t sb_ = sep::smem_u32(smem);
   uint32_t* const glb_w = reinterpret_cast<uint32_t*>(smem + Sm::GLB);
 
-  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int S = p.S, G = p.Hq / p.Hkv, g = h / G;
-  const int i0 = t * TBQ;
-  const int qlast = (i0 + TBQ < S ? i0 + TBQ : S) - 1;
-  const int32_t* pre = p.prefix + static_cast<int64_t>(b) * (S + 1);
-  const uint8_t* fl = p.is_sep + static_cast<int64_t>(b) * S;
-  // the tile's kept keys: global keys before the first row's window (the
-  // head of the compact list), then the window positions [lo, qlast]
-  const int lo = i0 - p.n + 1 > 0 ? i0 - p.n + 1 : 0;
-  const int al = p.a < lo ? p.a : lo;
-  const int nglo = al + (pre[lo] - pre[al]);
-  const int nbg = (nglo + TBK - 1) / TBK;
-  const int nbw = (qlast - lo + TBK) / TBK;
-  const int nblk = nbg + nbw;
-  const int nunit = 2 * nblk;
-  const int64_t kvrow0 = (static_cast<int64_t>(b) * p.Hkv + g) * S;
-  const int64_t qrow0 = (static_cast<int64_t>(b) * p.Hq + h) * S;
-  // unit u: keys [64 (u & 1), +64) of block u >> 1 -- rows of the compact
-  // list (global blocks) or positions (window blocks) from unit_key(u)
-  auto unit_key = [&](int u) -> int {
+  const int S = p.S, G = p.Hq / p.Hkv;
+  const int nitems = p.B * p.Hq * ((S + TBQ - 1) / TBQ);
+  // unit u of item `it`: keys [64 (u & 1), +64) of block u >> 1 -- rows of
+  // the compact list (global blocks) or positions (window blocks)
+  auto unit_key = [&](const QItem& it, int u) -> int {
     const int j = u >> 1;
-    return (j < nbg ? j * TBK : lo + (j - nbg) * TBK) + 64 * (u & 1);
-  };
-  // the unit's K and V rows into stage u % kNst (its bytes; the load warp's
-  // 32 arrivals follow once the stage's global-flag words are written)
-  auto load_unit = [&](int u) {
-    const int st = u % kNst;
-    const bool win = (u >> 1) >= nbg;
-    uint8_t* dst = smem + Sm::RING + st * Sm::STAGE;
-    const int32_t row = static_cast<int32_t>(kvrow0 + unit_key(u));
-    mbar_expect_tx(&bars.st_full[st], Sm::STAGE);
-#pragma unroll
-    for (int c = 0; c < NB; ++c) {
-      sep::tma_load_2d(dst + c * kT64, win ? &map_k : &map_kc, 64 * c, row, &bars.st_full[st]);
-      sep::tma_load_2d(dst + (NB + c) * kT64, win ? &map_v : &map_vc, 64 * c, row, &bars.st_full[st]);
-    }
+    return (j < it.nbg ? j * TBK : it.lo + (j - it.nbg) * TBK) + 64 * (u & 1);
   };
 
   if (threadIdx.x == 9 * 32) {
-    // the load warp's first lane: barriers, then at once the Q / dO copies
-    // and the first kNst units (the ring starts free)
-    sep::mbar_init(&bars.q_full, 1);
-    sep::mbar_init(&bars.fin, 1);
-    sep::mbar_init(&bars.drain, 1);
+    for (int i = 0; i < QB; ++i) {
+      sep::mbar_init(&bars.q_full[i], 1);
+      sep::mbar_init(&bars.q_free[i], 1);
+    }
     for (int i = 0; i < kNst; ++i) {
       sep::mbar_init(&bars.st_full[i], 32);
       sep::mbar_init(&bars.st_free[i], 1);
@@ -724,13 +810,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       sep::mbar_init(&bars.s_full[i], 1);
       sep::mbar_init(&bars.p_full[i], 8);
     }
+    sep::mbar_init(&bars.fin, 1);
+    sep::mbar_init(&bars.acc_free, 8);
+    sep::mbar_init(&bars.drain, 1);
     // a wait of an earlier CTA gave up: this one ends at its first wait too
     bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
     sep::mbar_fence_init();
-    sep::mbar_arrive_expect_tx(&bars.q_full, 2 * NB * kT128);
-    load_tile128<D>(smem + Sm::Q, &map_q, static_cast<int32_t>(qrow0 + i0), &bars.q_full);
-    load_tile128<D>(smem + Sm::DO, &map_do, static_cast<int32_t>(qrow0 + i0), &bars.q_full);
-    for (int u = 0; u < kNst && u < nunit; ++u) load_unit(u);
   }
   if (warp == 8) {
     sep::tmem_alloc(&bars.tmem_base, 512);
@@ -746,70 +831,81 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int lq = warp & 3, ch = warp >> 2;
     const int r = 32 * lq + lane;  // query row = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>(32 * lq) << 16;
-    const int i = i0 + r;
-    const float nlse2 = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
-    const float dl = i < S ? p.delta[qrow0 + i] : 0.f;
     const float2 sc2 = make_float2(p.scale_log2, p.scale_log2);
-    const float2 nl2 = make_float2(nlse2, nlse2), dl2 = make_float2(dl, dl);
+    const float sc = p.scale_log2 * 0.69314718055994530942f;
     bool ok = true;
-    for (int u = 0; u < nunit && ok; ++u) {
-      const int j = u >> 1, hh = u & 1, sb = u & 1, st = u % kNst;
-      if (!warp_wait(&bars.st_full[st], (u / kNst) & 1, abort, p.err)) {
-        ok = false;  // (the unit's global-flag words are in shared memory)
-        break;
+    uint32_t U = 0, I = 0;
+    for (int ii = blockIdx.x; ii < nitems && ok; ii += gridDim.x, ++I) {
+      const QItem it = q_item(p, ii);
+      const int nunit = 2 * it.nblk;
+      const int i = it.t * TBQ + r;
+      const int64_t qrow0 = (static_cast<int64_t>(it.b) * p.Hq + it.h) * S;
+      const float nlse2 = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
+      const float dl = i < S ? p.delta[qrow0 + i] : 0.f;
+      const float2 nl2 = make_float2(nlse2, nlse2), dl2 = make_float2(dl, dl);
+      for (int u = 0; u < nunit; ++u) {
+        const uint32_t gu = U + u;
+        const int j = u >> 1, hh = u & 1, sb = gu & 1, st = gu % kNst;
+        if (!warp_wait(&bars.st_full[st], (gu / kNst) & 1, abort, p.err) ||
+            !warp_wait(&bars.s_full[sb], (gu >> 1) & 1, abort, p.err)) {
+          ok = false;  // (st_full: the unit's global-flag words are in shared memory)
+          break;
+        }
+        sep::tc_fence_after();
+        // the unit's key columns this query row keeps, relative to column
+        // c0 = 64 hh + 32 ch of the block: global blocks, every listed key;
+        // window blocks (contiguous positions from `base`), keys at or
+        // before the row (and the tile), within n - 1 of it unless global
+        const int c0 = 64 * hh + 32 * ch;
+        uint32_t keep;
+        if (j < it.nbg) {
+          keep = bit_range(-c0, (it.nglo - j * TBK < TBK ? it.nglo - j * TBK : TBK) - c0);
+        } else {
+          const int base = it.lo + (j - it.nbg) * TBK;
+          int kb2 = i - base + 1;  // keys at positions <= i, in the tile's range
+          if (kb2 > it.qlast - base + 1) kb2 = it.qlast - base + 1;
+          keep = bit_range(-c0, kb2 - c0) &
+                 (bit_range(i - base - p.n + 1 - c0, 32) | glb_w[st * 2 + ch]);
+        }
+        if (i >= S) keep = 0u;
+        const uint32_t cs = 128u * sb + 32u * ch;
+        uint32_t pp[16], dd[16];
+        if (__all_sync(0xffffffffu, keep == 0u)) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) dd[e] = 0u;
+        } else {
+          uint32_t sv[32], dv_[32];
+          sep::tmem_ld32(tmem + lane_base + cs, sv);
+          sep::tmem_ld32(tmem + lane_base + cs + 64, dv_);
+          sep::tmem_wait_ld_r32(sv);
+          sep::tmem_wait_ld_r32(dv_);
+          if (__all_sync(0xffffffffu, keep == 0xffffffffu))
+            probs_grads<false, false>(sv, dv_, nullptr, nullptr, nl2, dl2, sc2, keep, pp, dd);
+          else
+            probs_grads<true, false>(sv, dv_, nullptr, nullptr, nl2, dl2, sc2, keep, pp, dd);
+        }
+        sep::tmem_st16(tmem + lane_base + cs, dd);
+        sep::tmem_wait_st();
+        sep::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) sep::mbar_arrive(&bars.p_full[sb]);
       }
-      if (!warp_wait(&bars.s_full[sb], (u >> 1) & 1, abort, p.err)) {
+      if (!ok || !warp_wait(&bars.fin, I & 1, abort, p.err)) {
         ok = false;
         break;
       }
       sep::tc_fence_after();
-      // the unit's key columns this query row keeps, relative to column
-      // c0 = 64 hh + 32 ch of the block: global blocks, every listed key;
-      // window blocks (contiguous positions from `base`), keys at or before
-      // the row (and the tile), within n - 1 of it unless global
-      const int c0 = 64 * hh + 32 * ch;
-      uint32_t keep;
-      if (j < nbg) {
-        keep = bit_range(-c0, (nglo - j * TBK < TBK ? nglo - j * TBK : TBK) - c0);
-      } else {
-        const int base = lo + (j - nbg) * TBK;
-        int kb2 = i - base + 1;  // keys at positions <= i, in the tile's range
-        if (kb2 > qlast - base + 1) kb2 = qlast - base + 1;
-        keep = bit_range(-c0, kb2 - c0) &
-               (bit_range(i - base - p.n + 1 - c0, 32) | glb_w[st * 2 + ch]);
-      }
-      if (i >= S) keep = 0u;
-      const uint32_t cs = 128u * sb + 32u * ch;
-      uint32_t pp[16], dd[16];
-      if (__all_sync(0xffffffffu, keep == 0u)) {
-#pragma unroll
-        for (int e = 0; e < 16; ++e) dd[e] = 0u;
-      } else {
-        uint32_t sv[32], dv_[32];
-        sep::tmem_ld32(tmem + lane_base + cs, sv);
-        sep::tmem_ld32(tmem + lane_base + cs + 64, dv_);
-        sep::tmem_wait_ld_r32(sv);
-        sep::tmem_wait_ld_r32(dv_);
-        if (__all_sync(0xffffffffu, keep == 0xffffffffu))
-          probs_grads<false, false>(sv, dv_, nullptr, nullptr, nl2, dl2, sc2, keep, pp, dd);
-        else
-          probs_grads<true, false>(sv, dv_, nullptr, nullptr, nl2, dl2, sc2, keep, pp, dd);
-      }
-      sep::tmem_st16(tmem + lane_base + cs, dd);
-      sep::tmem_wait_st();
-      sep::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) sep::mbar_arrive(&bars.p_full[sb]);
-    }
-    if (ok && warp_wait(&bars.fin, 0, abort, p.err)) {
-      sep::tc_fence_after();
-      const float sc = p.scale_log2 * 0.69314718055994530942f;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t qv[32];
         const int col = (D / 2) * ch + 32 * c;
         sep::tmem_ld32(tmem + lane_base + kColAcc + col, qv);
         sep::tmem_wait_ld_r32(qv);
+        if (c == D / 64 - 1) {
+          sep::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) sep::mbar_arrive(&bars.acc_free);
+        }
         if (i < S) {
           uint4* dst = reinterpret_cast<uint4*>(dq + (qrow0 + i) * D + col);
 #pragma unroll
@@ -820,53 +916,70 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                  sep::pack_bf16x2(__uint_as_float(qv[8 * u4 + 6]) * sc, __uint_as_float(qv[8 * u4 + 7]) * sc));
         }
       }
+      U += nunit;
     }
   } else if (warp == 8) {
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_mn(128, 64, false, false);
       constexpr uint32_t id_o = idesc_mn(128, D, false, true);
-      const uint64_t dQ = sep::smem_desc_sw128(sb_ + Sm::Q, 16);
-      const uint64_t dO = sep::smem_desc_sw128(sb_ + Sm::DO, 16);
-      bool ok = sep::mbar_wait(&bars.q_full, 0, abort, p.err);
-      for (int u = 0; u <= nunit && ok; ++u) {
-        if (u < nunit) {
-          const int st = u % kNst;
-          if (!sep::mbar_wait(&bars.st_full[st], (u / kNst) & 1, abort, p.err)) {
-            ok = false;
-            break;
-          }
-          sep::tc_fence_after();
-          const uint32_t ka = sb_ + Sm::RING + st * Sm::STAGE, va = ka + NB * kT64;
-          const uint64_t dK = sep::smem_desc_sw128(ka, 16), dV = sep::smem_desc_sw128(va, 16);
-          const uint32_t cs = 128u * (u & 1);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t oq = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
-            const uint64_t okv = static_cast<uint64_t>(((kk / 4) * kT64 + (kk % 4) * 32) >> 4);
-            sep::mma_bf16_ss(tmem + cs, dQ + oq, dK + okv, id_s, kk > 0 ? 1u : 0u);
-            sep::mma_bf16_ss(tmem + cs + 64, dO + oq, dV + okv, id_s, kk > 0 ? 1u : 0u);
-          }
-          sep::mma_commit(&bars.s_full[u & 1]);
+      bool ok = true;
+      uint32_t U = 0, I = 0;
+      for (int ii = blockIdx.x; ii < nitems && ok; ii += gridDim.x, ++I) {
+        const QItem it = q_item(p, ii);
+        const int nunit = 2 * it.nblk;
+        const int qbuf = I % QB;
+        if (!sep::mbar_wait(&bars.q_full[qbuf], (I / QB) & 1, abort, p.err)) {
+          ok = false;
+          break;
         }
-        if (u >= 1) {
-          const int w = u - 1, wst = w % kNst;
-          if (!sep::mbar_wait(&bars.p_full[w & 1], (w >> 1) & 1, abort, p.err)) {
-            ok = false;
-            break;
-          }
-          sep::tc_fence_after();
-          const uint64_t dKmn = sep::smem_desc_sw128(sb_ + Sm::RING + wst * Sm::STAGE, kT64);
-          const uint32_t cs = 128u * (w & 1);
+        const uint64_t dQ = sep::smem_desc_sw128(sb_ + qbuf * Sm::QSZ, 16);
+        const uint64_t dO = sep::smem_desc_sw128(sb_ + qbuf * Sm::QSZ + NB * kT128, 16);
+        for (int u = 0; u <= nunit; ++u) {
+          if (u < nunit) {
+            const uint32_t gu = U + u;
+            const int st = gu % kNst;
+            if (!sep::mbar_wait(&bars.st_full[st], (gu / kNst) & 1, abort, p.err)) {
+              ok = false;
+              break;
+            }
+            sep::tc_fence_after();
+            const uint32_t ka = sb_ + Sm::RING + st * Sm::STAGE, va = ka + NB * kT64;
+            const uint64_t dK = sep::smem_desc_sw128(ka, 16), dV = sep::smem_desc_sw128(va, 16);
+            const uint32_t cs = 128u * (gu & 1);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
-            sep::mma_bf16_ts(tmem + kColAcc, tmem + unit_acol(cs, kk), dKmn + off, id_o,
-                             (w > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t oq = static_cast<uint64_t>(((kk / 4) * kT128 + (kk % 4) * 32) >> 4);
+              const uint64_t okv = static_cast<uint64_t>(((kk / 4) * kT64 + (kk % 4) * 32) >> 4);
+              sep::mma_bf16_ss(tmem + cs, dQ + oq, dK + okv, id_s, kk > 0 ? 1u : 0u);
+              sep::mma_bf16_ss(tmem + cs + 64, dO + oq, dV + okv, id_s, kk > 0 ? 1u : 0u);
+            }
+            sep::mma_commit(&bars.s_full[gu & 1]);
+            if (u == nunit - 1) sep::mma_commit(&bars.q_free[qbuf]);  // the item's Q, dO are read
           }
-          sep::mma_commit(&bars.st_free[wst]);  // the stage may be refilled
+          if (u >= 1) {
+            const uint32_t w = U + u - 1;
+            const int wst = w % kNst;
+            if (!sep::mbar_wait(&bars.p_full[w & 1], (w >> 1) & 1, abort, p.err) ||
+                (u == 1 && I > 0 && !sep::mbar_wait(&bars.acc_free, (I - 1) & 1, abort, p.err))) {
+              ok = false;
+              break;
+            }
+            sep::tc_fence_after();
+            const uint64_t dKmn = sep::smem_desc_sw128(sb_ + Sm::RING + wst * Sm::STAGE, kT64);
+            const uint32_t cs = 128u * (w & 1);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
+              sep::mma_bf16_ts(tmem + kColAcc, tmem + unit_acol(cs, kk), dKmn + off, id_o,
+                               (u > 1 || kk > 0) ? 1u : 0u);
+            }
+            sep::mma_commit(&bars.st_free[wst]);  // the stage may be refilled
+          }
         }
+        if (!ok) break;
+        sep::mma_commit(&bars.fin);
+        U += nunit;
       }
-      if (ok) sep::mma_commit(&bars.fin);
       sep::mma_commit(&bars.drain);
       int keep = 0;
       sep::mbar_wait(&bars.drain, 0, &keep, nullptr);
@@ -874,47 +987,74 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------ loads (warp 9)
-    // (Q, dO and the first kNst units were started before the block
-    // barrier.)  Per unit: the copies once its stage is free, then the
-    // global-flag words of a window unit (flags read one unit ahead into
-    // registers), then the 32 arrivals that complete the stage with its
-    // bytes.
-    int issued = nunit < kNst ? nunit : kNst;  // units whose copies were started
-    bool fnext[2];  // flags of keys lane, lane + 32 of the next unit
-    auto fetch = [&](int u) {
-      const bool win = u < nunit && (u >> 1) >= nbg;
-      const int base = win ? unit_key(u) : 0;
-#pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const int q = base + lane + 32 * m;
-        fnext[m] = win && q <= qlast && (q < p.a || fl[q] != 0);
-      }
-    };
-    fetch(0);
-    for (int u = 0; u < nunit; ++u) {
-      const int st = u % kNst;
-      if (u >= kNst) {
-        bool go = true;
-        if (lane == 0) {
-          go = sep::mbar_wait(&bars.st_free[st], ((u / kNst) - 1) & 1, abort, p.err);
-          if (go) load_unit(u);
+    // Per item: its Q and dO once their buffer is free; per unit: the copies
+    // once its stage is free, then the global-flag words of a window unit,
+    // then the 32 arrivals that complete the stage with its bytes.
+    uint32_t U = 0, I = 0;
+    uint32_t issued_u = 0, issued_i = 0;
+    bool ok = true;
+    for (int ii = blockIdx.x; ii < nitems && ok; ii += gridDim.x, ++I) {
+      const QItem it = q_item(p, ii);
+      const int nunit = 2 * it.nblk;
+      const int qbuf = I % QB;
+      const int64_t kvrow0 = (static_cast<int64_t>(it.b) * p.Hkv + it.h / G) * S;
+      const uint8_t* fl = p.is_sep + static_cast<int64_t>(it.b) * S;
+      bool go = true;
+      if (lane == 0) {
+        if (I >= QB) go = sep::mbar_wait(&bars.q_free[qbuf], ((I - QB) / QB) & 1, abort, p.err);
+        if (go) {
+          const int32_t row = static_cast<int32_t>((static_cast<int64_t>(it.b) * p.Hq + it.h) * S + it.t * TBQ);
+          sep::mbar_arrive_expect_tx(&bars.q_full[qbuf], Sm::QSZ);
+          load_tile128<D>(smem + qbuf * Sm::QSZ, &map_q, row, &bars.q_full[qbuf]);
+          load_tile128<D>(smem + qbuf * Sm::QSZ + NB * kT128, &map_do, row, &bars.q_full[qbuf]);
         }
-        if (!__shfl_sync(0xffffffffu, go, 0)) break;
-        issued = u + 1;
       }
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      issued_i = I + 1;
+      for (int u = 0; u < nunit; ++u) {
+        const uint32_t gu = U + u;
+        const int st = gu % kNst;
+        const bool win = (u >> 1) >= it.nbg;
+        const int key0 = unit_key(it, u);
+        bool f[2];  // global flags of keys lane, lane + 32 (loads in flight during the wait)
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const uint32_t w = __ballot_sync(0xffffffffu, fnext[m]);
-        if (lane == m) glb_w[st * 2 + m] = w;
+        for (int m = 0; m < 2; ++m) {
+          const int q = key0 + lane + 32 * m;
+          f[m] = win && q <= it.qlast && (q < p.a || fl[q] != 0);
+        }
+        if (lane == 0) {
+          if (gu >= kNst) go = sep::mbar_wait(&bars.st_free[st], ((gu / kNst) - 1) & 1, abort, p.err);
+          if (go) {
+            uint8_t* dst = smem + Sm::RING + st * Sm::STAGE;
+            const int32_t row = static_cast<int32_t>(kvrow0 + key0);
+            mbar_expect_tx(&bars.st_full[st], Sm::STAGE);
+#pragma unroll
+            for (int c = 0; c < NB; ++c) {
+              sep::tma_load_2d(dst + c * kT64, win ? &map_k : &map_kc, 64 * c, row, &bars.st_full[st]);
+              sep::tma_load_2d(dst + (NB + c) * kT64, win ? &map_v : &map_vc, 64 * c, row, &bars.st_full[st]);
+            }
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) {
+          ok = false;
+          break;
+        }
+        issued_u = gu + 1;
+#pragma unroll
+        for (int m = 0; m < 2; ++m) {
+          const uint32_t w = __ballot_sync(0xffffffffu, f[m]);
+          if (lane == m) glb_w[st * 2 + m] = w;
+        }
+        sep::mbar_arrive(&bars.st_full[st]);
       }
-      fetch(u + 1);
-      sep::mbar_arrive(&bars.st_full[st]);
+      U += nunit;
     }
     if (lane == 0 && *abort) {
       int dummy = 0;
-      sep::mbar_wait(&bars.q_full, 0, &dummy, nullptr);
-      for (int u = issued - kNst < 0 ? 0 : issued - kNst; u < issued; ++u)
-        sep::mbar_wait(&bars.st_full[u % kNst], (u / kNst) & 1, &dummy, nullptr);
+      for (uint32_t j = issued_i > QB ? issued_i - QB : 0; j < issued_i; ++j)
+        sep::mbar_wait(&bars.q_full[j % QB], (j / QB) & 1, &dummy, nullptr);
+      for (uint32_t g2 = issued_u > kNst ? issued_u - kNst : 0; g2 < issued_u; ++g2)
+        sep::mbar_wait(&bars.st_full[g2 % kNst], (g2 / kNst) & 1, &dummy, nullptr);
     }
     __syncwarp();
   }
@@ -929,20 +1069,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // Workspace: delta [B, Hq, S] fp32; fp32 dK and dV rows of the compact
 // global-key lists [B, Hkv, S, D] each; the compact bf16 K and V copies
-// [B, Hkv, S, D] each.
+// [B, Hkv, S, D] each; the global-key work items (at most B x ceil(S/128) x
+// ceil(ceil(S/128)/kTcChunkTiles) pairs of int32) after their count.
 struct BwdWs {
-  size_t delta, dk, dv, kc, vc;
-  size_t total() const { return delta + dk + dv + kc + vc; }
+  size_t delta, dk, dv, kc, vc, items;
+  size_t total() const { return delta + dk + dv + kc + vc + items; }
 };
 BwdWs bwd_ws(int B, int Hq, int Hkv, int S, int D) {
   auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
+  const size_t nwin = (static_cast<size_t>(S) + TBK - 1) / TBK;
+  const size_t nchunk = (nwin + kTcChunkTiles - 1) / kTcChunkTiles;
   BwdWs w;
   w.delta = r256(static_cast<size_t>(B) * Hq * S * 4);
   w.dk = r256(static_cast<size_t>(B) * Hkv * S * D * 4);
   w.dv = w.dk;
   w.kc = r256(static_cast<size_t>(B) * Hkv * S * D * 2);
   w.vc = w.kc;
+  w.items = 256 + r256(static_cast<size_t>(B) * nwin * nchunk * 8);
   return w;
+}
+
+int num_sms() {
+  static int sms[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!sms[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    sms[dev] = v > 0 ? v : 148;
+  }
+  return sms[dev];
 }
 
 template <int D>
@@ -967,6 +1124,8 @@ int launch_bwd(BwdParams p, const void* out, void* dq, void* dk, void* dv, void*
   p.dv_acc = reinterpret_cast<float*>(base + w.delta + w.dk);
   __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(base + w.delta + w.dk + w.dv);
   __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(base + w.delta + w.dk + w.dv + w.kc);
+  p.item_count = reinterpret_cast<int32_t*>(base + w.delta + w.dk + w.dv + w.kc + w.vc);
+  p.items = reinterpret_cast<int2*>(base + w.delta + w.dk + w.dv + w.kc + w.vc + 256);
   p.nwin = (p.S + TBK - 1) / TBK;
   p.nchunk = (p.nwin + kTcChunkTiles - 1) / kTcChunkTiles;
   const int64_t qrows = static_cast<int64_t>(p.B) * p.Hq * p.S;
@@ -988,10 +1147,15 @@ int launch_bwd(BwdParams p, const void* out, void* dq, void* dk, void* dv, void*
   const dim3 rgrid((p.S + 63) / 64, p.Hkv, p.B);
   k_bwd_prep<D><<<rgrid, 256, 0, st>>>(p, kc, vc);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  k_bwd_kv<D><<<dim3(p.nwin + p.nwin * p.nchunk, p.Hkv, p.B), kTcThreads, KvSmem<D>::BYTES, st>>>(
+  k_bwd_plan<<<1, 32, 0, st>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  // persistent: one CTA per SM (shared memory and TMEM hold one)
+  const int sms = num_sms();
+  k_bwd_kv<D><<<sms, kTcThreads, KvSmem<D>::BYTES, st>>>(
       p, uq, udo, mk, mv, mkc, mvc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  k_bwd_q<D><<<dim3((p.S + TBQ - 1) / TBQ, p.Hq, p.B), kTcThreads, QSmem<D>::BYTES, st>>>(
+  const int64_t qitems = static_cast<int64_t>(p.B) * p.Hq * ((p.S + TBQ - 1) / TBQ);
+  k_bwd_q<D><<<static_cast<unsigned>(qitems < sms ? qitems : sms), kTcThreads, QSmem<D>::BYTES, st>>>(
       p, mq, mdo, uk, uv, ukc, uvc, static_cast<__nv_bfloat16*>(dq));
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   k_bwd_scatter<D><<<rgrid, 256, 0, st>>>(p, p.scale_log2 / 1.44269504088896340736f,
