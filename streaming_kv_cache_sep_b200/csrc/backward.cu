@@ -13,8 +13,9 @@
 // disjoint families:
 //   * global keys (j < a or a separator) are kept by every query i >= j;
 //     they are taken 128 at a time from the compact list of global keys, and
-//     each block visits the query tiles after its first position, at most
-//     kTcChunkTiles tiles per CTA;
+//     each block visits the query tiles from its first key's on, split into
+//     chunks of kTcChunkTiles tiles aligned to multiples of kTcChunkTiles
+//     (one work item per block, chunk and kv head);
 //   * local keys (all others) are kept only by queries i in [j, j + n); they
 //     are taken as 128 consecutive positions, and each block visits the query
 //     tiles that reach it, with the global keys of the block masked out.
@@ -78,14 +79,16 @@ __global__ void k_bwd_delta(const __nv_bfloat16* __restrict__ out,
 //     the scores of unit u before the gradient products of unit u-1, so the
 //     tensor pipe computes while the compute warps work on the other
 //     buffer.  TMEM: S0 [0,64) dP0 [64,128) S1 [128,192) dP1 [192,256)
-//     dV [256,256+D) dK [256+D,256+2D).
+//     dV [256,256+D) dK [256+D,256+2D), and at D = 64 a second dV, dK pair
+//     [384,512) for every other item.
 //   k_bwd_q (query-centric, 128 queries in TMEM lanes, Q and dO resident):
 //     over the kept key blocks of its tile as the forward does -- the global
 //     keys before the window from the compact list, then the window blocks
 //     with the element mask -- in units of 64 keys streamed through the
 //     ring: S = Q K^T and dP = dO V^T (SS), dS written back as bf16,
 //     dQ += dS K (TS, B = K MN-major).  The CTA owns its queries, so dQ is
-//     stored once, as bf16.  TMEM: S0 dP0 S1 dP1 as above, dQ [256, 256+D).
+//     stored once, as bf16.  TMEM: S0 dP0 S1 dP1 as above, dQ of every
+//     other item in [256, 256+D) and [256+D, 256+2D).
 // Warps 0-7 are the compute warps (warp w: TMEM lanes 32 (w & 3) .. +31,
 // columns [32 (w >> 2), +32) of each 64-column score tile), warp 8
 // allocates TMEM and its lane 0 issues the MMAs, warp 9 issues the tensor
@@ -104,9 +107,7 @@ constexpr int TBQ = 128;  // queries per tile
 constexpr int kTcThreads = 320;
 constexpr int kNst = 4;           // stages of the 64-row operand ring
 constexpr int kT64 = 64 * 128;    // one 64-row x 64-column swizzled tile
-constexpr uint32_t kColAcc = 256;    // dV (key-centric) / dQ (query-centric)
-template <int D>
-constexpr uint32_t col_dk() { return kColAcc + D; }  // dK after the D columns of dV
+constexpr uint32_t kColAcc = 256;    // accumulators: dV, dK (key-centric) / dQ (query-centric)
 constexpr int kT128 = 128 * 128;  // one 128-row x 64-column swizzled tile
 constexpr int kTcChunkTiles = 4;  // query tiles per item of global keys
 
@@ -289,42 +290,65 @@ __device__ __forceinline__ void probs_grads(const uint32_t (&sv)[32], const uint
 
 // ---- work items
 //
-// Key-centric items: the global-key items (listed by k_bwd_plan, heaviest
-// first), each for every kv head, then the window items (b, kv head, block
-// of 128 positions).  Query-centric items: (b, head, tile of 128 queries),
+// Key-centric items: the global-key items (listed by k_bwd_plan), for kv
+// head 0, then for head 1, ..., then the window items (b, kv head, block of
+// 128 positions).  Query-centric items: (b, head, tile of 128 queries),
 // tiles with more kept keys (later positions) first.  Both kernels are
 // persistent: CTA c takes items c, c + gridDim.x, ... in order, so every
 // role of the CTA walks the same sequence without handing items around.
 
-// The global-key items: for every sequence b and block kb of 128 global
-// keys, the chunks of kTcChunkTiles query tiles from the tile of the
-// block's first key to the last tile, as (b, kb << 16 | chunk).  One warp.
-__global__ void __launch_bounds__(32) k_bwd_plan(const BwdParams p) {
-  const int lane = threadIdx.x;
+// The global-key items: for every sequence b, chunk c of kTcChunkTiles
+// query tiles [c kTcChunkTiles, +kTcChunkTiles) and block kb of 128 global
+// keys whose first key lies before the chunk's end, the item (b,
+// kb << 16 | c), in the order (b, c, kb): the items a CTA runs side by side
+// read the same query tiles.  One CTA; warp w takes sequences w, w + 32 ...:
+// their item counts, then (after one thread's prefix over the sequences)
+// their items.  p.item_count[1 + b] holds sequence b's offset.
+constexpr int kPlanWarps = 32;
+__global__ void __launch_bounds__(32 * kPlanWarps) k_bwd_plan(const BwdParams p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nT = (p.S + TBQ - 1) / TBQ;
-  int e = 0;
-  for (int b = 0; b < p.B; ++b) {
+  const int nC = (nT + kTcChunkTiles - 1) / kTcChunkTiles;
+  int32_t* const off = p.item_count + 1;
+  // chunk of the first tile of block kb of sequence b
+  auto first_chunk = [&](const GlobalList& gl, int kb) {
+    const int pos = gl.pos(kb * TBK);
+    return (pos >= 0 && pos < p.S ? pos : 0) / TBQ / kTcChunkTiles;
+  };
+  for (int b = warp; b < p.B; b += kPlanWarps) {
     const GlobalList gl(p, b);
     const int nb = (gl.total + TBK - 1) / TBK;
-    for (int k0 = 0; k0 < nb; k0 += 32) {
-      const int kb = k0 + lane;
-      int nch = 0;
-      if (kb < nb) {
-        const int pos = gl.pos(kb * TBK);
-        const int t0 = (pos >= 0 && pos < p.S ? pos : 0) / TBQ;
-        nch = (nT - t0 + kTcChunkTiles - 1) / kTcChunkTiles;
-      }
-      int incl = nch;  // inclusive prefix over the warp
+    int n = 0;  // block kb has items for chunks first_chunk .. nC - 1
+    for (int kb = lane; kb < nb; kb += 32) n += nC - first_chunk(gl, kb);
 #pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
+    for (int o = 16; o; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+    if (lane == 0) off[b] = n;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int e = 0;
+    for (int b = 0; b < p.B; ++b) {
+      const int n = off[b];
+      off[b] = e;
+      e += n;
+    }
+    *p.item_count = e;
+  }
+  __syncthreads();
+  for (int b = warp; b < p.B; b += kPlanWarps) {
+    const GlobalList gl(p, b);
+    const int nb = (gl.total + TBK - 1) / TBK;
+    int e = off[b];
+    for (int c = 0; c < nC; ++c) {
+      for (int k0 = 0; k0 < nb; k0 += 32) {
+        const int kb = k0 + lane;
+        const bool on = kb < nb && first_chunk(gl, kb) <= c;
+        const uint32_t m = __ballot_sync(0xffffffffu, on);
+        if (on) p.items[e + __popc(m & ((1u << lane) - 1u))] = make_int2(b, (kb << 16) | c);
+        e += __popc(m);
       }
-      for (int c = 0; c < nch; ++c) p.items[e + incl - nch + c] = make_int2(b, (kb << 16) | c);
-      e += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
-  if (lane == 0) *p.item_count = e;
 }
 
 struct KvItem {
@@ -335,14 +359,16 @@ __device__ __forceinline__ KvItem kv_item(const BwdParams& p, int i, int nglob) 
   KvItem it;
   const int nT = (p.S + TBQ - 1) / TBQ;
   if (i < nglob) {
-    const int2 ent = p.items[i / p.Hkv];
-    it.g = i % p.Hkv;
+    const int nge = nglob / p.Hkv;
+    const int2 ent = p.items[i % nge];
+    it.g = i / nge;
     it.b = ent.x;
     it.kb = ent.y >> 16;
     const GlobalList gl(p, it.b);
     const int pos = gl.pos(it.kb * TBK);
-    it.t0 = (pos >= 0 && pos < p.S ? pos : 0) / TBQ + (ent.y & 0xffff) * kTcChunkTiles;
-    const int t1 = it.t0 + kTcChunkTiles < nT ? it.t0 + kTcChunkTiles : nT;
+    const int first = (pos >= 0 && pos < p.S ? pos : 0) / TBQ, c0 = (ent.y & 0xffff) * kTcChunkTiles;
+    it.t0 = first > c0 ? first : c0;
+    const int t1 = c0 + kTcChunkTiles < nT ? c0 + kTcChunkTiles : nT;
     it.ntile = t1 - it.t0;
     it.window = false;
   } else {
@@ -356,6 +382,34 @@ __device__ __forceinline__ KvItem kv_item(const BwdParams& p, int i, int nglob) 
     it.window = true;
   }
   return it;
+}
+
+// An item and this compute thread's key row in it: position jp, and
+// whether the item's queries keep it (window items leave global keys out).
+struct KvRow {
+  KvItem it;
+  int jp, use;
+};
+__device__ __forceinline__ KvRow kv_row(const BwdParams& p, int i, int nglob, int r) {
+  KvRow x;
+  x.it = kv_item(p, i, nglob);
+  x.jp = -1;
+  x.use = 0;
+  if (x.it.window) {
+    const int q = x.it.kb * TBK + r;
+    if (q < p.S) {
+      x.jp = q;
+      x.use = !(q < p.a || p.is_sep[static_cast<int64_t>(x.it.b) * p.S + q]);
+    }
+  } else {
+    const GlobalList gl(p, x.it.b);
+    const int t = x.it.kb * TBK + r;
+    if (t < gl.total) {
+      x.jp = gl.pos(t);
+      x.use = 1;
+    }
+  }
+  return x;
 }
 
 // Shared memory of the key-centric kernel: KVB buffers of an item's K and V
@@ -376,7 +430,7 @@ struct KvSmem {
 };
 struct KvBars {
   uint64_t kv_full[2], kv_free[2], st_full[kNst], st_free[kNst], s_full[2], p_full[2];
-  uint64_t fin, acc_free, drain;
+  uint64_t fin[2], acc_free[2], drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -391,7 +445,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using Sm = KvSmem<D>;
   constexpr int NB = D / 64;
   constexpr int KVB = Sm::KVB;
-  constexpr uint32_t kColDK = col_dk<D>();
+  // dV, dK accumulator buffers (columns [256, 512)): two where they fit, so
+  // an item's products need not wait for the previous item's read-out
+  constexpr int ACCB = D == 64 ? 2 : 1;
   extern __shared__ uint8_t dsm_raw[];
   uint8_t* const smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -425,8 +481,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       sep::mbar_init(&bars.s_full[i], 1);
       sep::mbar_init(&bars.p_full[i], 8);
     }
-    sep::mbar_init(&bars.fin, 1);
-    sep::mbar_init(&bars.acc_free, 8);
+    for (int i = 0; i < 2; ++i) {
+      sep::mbar_init(&bars.fin[i], 1);
+      sep::mbar_init(&bars.acc_free[i], 8);
+    }
     sep::mbar_init(&bars.drain, 1);
     // a wait of an earlier CTA gave up: this one ends at its first wait too
     bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
@@ -451,26 +509,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float sc = p.scale_log2 * 0.69314718055994530942f;
     bool ok = true;
     uint32_t U = 0, I = 0;  // units and items of this CTA so far
+    // every role decodes the next item (dependent global loads) while it
+    // works on the current one
+    KvRow cur = blockIdx.x < nitems ? kv_row(p, blockIdx.x, nglob, r) : KvRow{};
     for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
-      const KvItem it = kv_item(p, i, nglob);
+      const KvRow nxt = i + static_cast<int>(gridDim.x) < nitems ? kv_row(p, i + gridDim.x, nglob, r) : cur;
+      const KvItem it = cur.it;
+      const int jp = cur.jp, use = cur.use;
+      cur = nxt;
       const int nunit = 2 * G * it.ntile;
       const int64_t kvrow0 = (static_cast<int64_t>(it.b) * p.Hkv + it.g) * S;
-      // this thread's key: position jp, kept by this item's queries?
-      int jp = -1, use = 0;
-      if (it.window) {
-        const int q = it.kb * TBK + r;
-        if (q < S) {
-          jp = q;
-          use = !(q < p.a || p.is_sep[static_cast<int64_t>(it.b) * S + q]);
-        }
-      } else {
-        const GlobalList gl(p, it.b);
-        const int t = it.kb * TBK + r;
-        if (t < gl.total) {
-          jp = gl.pos(t);
-          use = 1;
-        }
-      }
       for (int u = 0; u < nunit; ++u) {
         const uint32_t gu = U + u;
         const int v = u >> 1, hh = u & 1, sb = gu & 1, st = gu % kNst;
@@ -518,29 +566,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         if (lane == 0) sep::mbar_arrive(&bars.p_full[sb]);
       }
-      if (!ok || !warp_wait(&bars.fin, I & 1, abort, p.err)) {
+      const int abuf = I % ACCB;
+      if (!ok || !warp_wait(&bars.fin[abuf], (I / ACCB) & 1, abort, p.err)) {
         ok = false;
         break;
       }
       sep::tc_fence_after();
       // dK and dV of this key row, columns [D/2 ch, +D/2): every lane loads
       // (warp-wide); once the last load is in, the accumulators are handed
-      // back to the next item.  A window key is stored as bf16, a global
+      // back for a later item.  A window key is stored as bf16, a global
       // key's partial sum is added to its fp32 row of the compact list.
       const bool mine = jp >= 0 && use;
       const int64_t row = kvrow0 + (it.window ? (mine ? jp : 0) : it.kb * TBK + r);
+      const uint32_t cdv = kColAcc + 2u * D * abuf, cdk = cdv + D;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t kv[32], vv[32];
         const int col = (D / 2) * ch + 32 * c;
-        sep::tmem_ld32(tmem + lane_base + kColDK + col, kv);
-        sep::tmem_ld32(tmem + lane_base + kColAcc + col, vv);
+        sep::tmem_ld32(tmem + lane_base + cdk + col, kv);
+        sep::tmem_ld32(tmem + lane_base + cdv + col, vv);
         sep::tmem_wait_ld_r32(kv);
         sep::tmem_wait_ld_r32(vv);
         if (c == D / 64 - 1) {
           sep::tc_fence_before();
           __syncwarp();
-          if (lane == 0) sep::mbar_arrive(&bars.acc_free);
+          if (lane == 0) sep::mbar_arrive(&bars.acc_free[abuf]);
         }
         if (!mine) continue;
         if (it.window) {
@@ -576,10 +626,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t id_o = idesc_mn(128, D, false, true);
       bool ok = true;
       uint32_t U = 0, I = 0;
+      KvItem cur = blockIdx.x < nitems ? kv_item(p, blockIdx.x, nglob) : KvItem{};
       for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
-        const KvItem it = kv_item(p, i, nglob);
+        const KvItem it = cur;
+        cur = i + static_cast<int>(gridDim.x) < nitems ? kv_item(p, i + gridDim.x, nglob) : cur;
         const int nunit = 2 * G * it.ntile;
-        const int kbuf = I % KVB;
+        const int kbuf = I % KVB, abuf = I % ACCB;
+        const uint32_t cdv = kColAcc + 2u * D * abuf, cdk = cdv + D;
         if (!sep::mbar_wait(&bars.kv_full[kbuf], (I / KVB) & 1, abort, p.err)) {
           ok = false;
           break;
@@ -617,7 +670,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t w = U + u - 1;
             const int wst = w % kNst;
             if (!sep::mbar_wait(&bars.p_full[w & 1], (w >> 1) & 1, abort, p.err) ||
-                (u == 1 && I > 0 && !sep::mbar_wait(&bars.acc_free, (I - 1) & 1, abort, p.err))) {
+                (u == 1 && I >= ACCB &&
+                 !sep::mbar_wait(&bars.acc_free[abuf], ((I - ACCB) / ACCB) & 1, abort, p.err))) {
               ok = false;
               break;
             }
@@ -629,14 +683,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
               const uint32_t acc = (u > 1 || kk > 0) ? 1u : 0u;
-              sep::mma_bf16_ts(tmem + kColAcc, tmem + unit_acol(cs, kk), dOmn + off, id_o, acc);
-              sep::mma_bf16_ts(tmem + kColDK, tmem + unit_acol(cs + 64, kk), dQmn + off, id_o, acc);
+              sep::mma_bf16_ts(tmem + cdv, tmem + unit_acol(cs, kk), dOmn + off, id_o, acc);
+              sep::mma_bf16_ts(tmem + cdk, tmem + unit_acol(cs + 64, kk), dQmn + off, id_o, acc);
             }
             sep::mma_commit(&bars.st_free[wst]);  // the stage may be refilled
           }
         }
         if (!ok) break;
-        sep::mma_commit(&bars.fin);
+        sep::mma_commit(&bars.fin[abuf]);
         U += nunit;
       }
       sep::mma_commit(&bars.drain);  // every MMA completes before TMEM is released
@@ -653,8 +707,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t U = 0, I = 0;
     uint32_t issued_u = 0, issued_i = 0;  // copies started (units, items)
     bool ok = true;
+    KvItem cur = blockIdx.x < nitems ? kv_item(p, blockIdx.x, nglob) : KvItem{};
     for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
-      const KvItem it = kv_item(p, i, nglob);
+      const KvItem it = cur;
+      cur = i + static_cast<int>(gridDim.x) < nitems ? kv_item(p, i + gridDim.x, nglob) : cur;
       const int nunit = 2 * G * it.ntile;
       const int kbuf = I % KVB;
       bool go = true;
@@ -744,7 +800,7 @@ struct QSmem {
 };
 struct QBars {
   uint64_t q_full[2], q_free[2], st_full[kNst], st_free[kNst], s_full[2], p_full[2];
-  uint64_t fin, acc_free, drain;
+  uint64_t fin[2], acc_free[2], drain;
   uint32_t tmem_base;
   int abort;
 };
@@ -810,8 +866,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       sep::mbar_init(&bars.s_full[i], 1);
       sep::mbar_init(&bars.p_full[i], 8);
     }
-    sep::mbar_init(&bars.fin, 1);
-    sep::mbar_init(&bars.acc_free, 8);
+    for (int i = 0; i < 2; ++i) {
+      sep::mbar_init(&bars.fin[i], 1);
+      sep::mbar_init(&bars.acc_free[i], 8);
+    }
     sep::mbar_init(&bars.drain, 1);
     // a wait of an earlier CTA gave up: this one ends at its first wait too
     bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
@@ -835,13 +893,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float sc = p.scale_log2 * 0.69314718055994530942f;
     bool ok = true;
     uint32_t U = 0, I = 0;
+    // every role decodes the next item while it works on the current one
+    auto row_stats = [&](const QItem& x, float& nl, float& dlv) {
+      const int i = x.t * TBQ + r;
+      const int64_t q0 = (static_cast<int64_t>(x.b) * p.Hq + x.h) * S;
+      nl = i < S ? -p.lse[q0 + i] * 1.44269504088896340736f : 0.f;
+      dlv = i < S ? p.delta[q0 + i] : 0.f;
+    };
+    QItem cur = blockIdx.x < nitems ? q_item(p, blockIdx.x) : QItem{};
+    float cur_nl = 0.f, cur_dl = 0.f;
+    if (blockIdx.x < nitems) row_stats(cur, cur_nl, cur_dl);
     for (int ii = blockIdx.x; ii < nitems && ok; ii += gridDim.x, ++I) {
-      const QItem it = q_item(p, ii);
+      const QItem it = cur;
+      const float nlse2 = cur_nl, dl = cur_dl;
+      if (ii + static_cast<int>(gridDim.x) < nitems) {
+        cur = q_item(p, ii + gridDim.x);
+        row_stats(cur, cur_nl, cur_dl);
+      }
       const int nunit = 2 * it.nblk;
       const int i = it.t * TBQ + r;
       const int64_t qrow0 = (static_cast<int64_t>(it.b) * p.Hq + it.h) * S;
-      const float nlse2 = i < S ? -p.lse[qrow0 + i] * 1.44269504088896340736f : 0.f;
-      const float dl = i < S ? p.delta[qrow0 + i] : 0.f;
       const float2 nl2 = make_float2(nlse2, nlse2), dl2 = make_float2(dl, dl);
       for (int u = 0; u < nunit; ++u) {
         const uint32_t gu = U + u;
@@ -865,7 +936,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           int kb2 = i - base + 1;  // keys at positions <= i, in the tile's range
           if (kb2 > it.qlast - base + 1) kb2 = it.qlast - base + 1;
           keep = bit_range(-c0, kb2 - c0) &
-                 (bit_range(i - base - p.n + 1 - c0, 32) | glb_w[st * 2 + ch]);
+               (bit_range(i - base - p.n + 1 - c0, 32) | glb_w[st * 2 + ch]);
         }
         if (i >= S) keep = 0u;
         const uint32_t cs = 128u * sb + 32u * ch;
@@ -890,7 +961,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         if (lane == 0) sep::mbar_arrive(&bars.p_full[sb]);
       }
-      if (!ok || !warp_wait(&bars.fin, I & 1, abort, p.err)) {
+      const int abuf = I & 1;
+      if (!ok || !warp_wait(&bars.fin[abuf], (I >> 1) & 1, abort, p.err)) {
         ok = false;
         break;
       }
@@ -899,12 +971,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int c = 0; c < D / 64; ++c) {
         uint32_t qv[32];
         const int col = (D / 2) * ch + 32 * c;
-        sep::tmem_ld32(tmem + lane_base + kColAcc + col, qv);
+        sep::tmem_ld32(tmem + lane_base + kColAcc + D * abuf + col, qv);
         sep::tmem_wait_ld_r32(qv);
         if (c == D / 64 - 1) {
           sep::tc_fence_before();
           __syncwarp();
-          if (lane == 0) sep::mbar_arrive(&bars.acc_free);
+          if (lane == 0) sep::mbar_arrive(&bars.acc_free[abuf]);
         }
         if (i < S) {
           uint4* dst = reinterpret_cast<uint4*>(dq + (qrow0 + i) * D + col);
@@ -924,10 +996,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t id_o = idesc_mn(128, D, false, true);
       bool ok = true;
       uint32_t U = 0, I = 0;
+      QItem cur = blockIdx.x < nitems ? q_item(p, blockIdx.x) : QItem{};
       for (int ii = blockIdx.x; ii < nitems && ok; ii += gridDim.x, ++I) {
-        const QItem it = q_item(p, ii);
+        const QItem it = cur;
+        cur = ii + static_cast<int>(gridDim.x) < nitems ? q_item(p, ii + gridDim.x) : cur;
         const int nunit = 2 * it.nblk;
-        const int qbuf = I % QB;
+        const int qbuf = I % QB, abuf = I & 1;
+        const uint32_t cdq = kColAcc + static_cast<uint32_t>(D) * abuf;
         if (!sep::mbar_wait(&bars.q_full[qbuf], (I / QB) & 1, abort, p.err)) {
           ok = false;
           break;
@@ -960,7 +1035,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t w = U + u - 1;
             const int wst = w % kNst;
             if (!sep::mbar_wait(&bars.p_full[w & 1], (w >> 1) & 1, abort, p.err) ||
-                (u == 1 && I > 0 && !sep::mbar_wait(&bars.acc_free, (I - 1) & 1, abort, p.err))) {
+                (u == 1 && I >= 2 && !sep::mbar_wait(&bars.acc_free[abuf], ((I - 2) >> 1) & 1, abort, p.err))) {
               ok = false;
               break;
             }
@@ -970,14 +1045,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t off = static_cast<uint64_t>(kk * (2048 >> 4));
-              sep::mma_bf16_ts(tmem + kColAcc, tmem + unit_acol(cs, kk), dKmn + off, id_o,
+              sep::mma_bf16_ts(tmem + cdq, tmem + unit_acol(cs, kk), dKmn + off, id_o,
                                (u > 1 || kk > 0) ? 1u : 0u);
             }
             sep::mma_commit(&bars.st_free[wst]);  // the stage may be refilled
           }
         }
         if (!ok) break;
-        sep::mma_commit(&bars.fin);
+        sep::mma_commit(&bars.fin[abuf]);
         U += nunit;
       }
       sep::mma_commit(&bars.drain);
@@ -993,8 +1068,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t U = 0, I = 0;
     uint32_t issued_u = 0, issued_i = 0;
     bool ok = true;
+    QItem cur = blockIdx.x < nitems ? q_item(p, blockIdx.x) : QItem{};
     for (int ii = blockIdx.x; ii < nitems && ok; ii += gridDim.x, ++I) {
-      const QItem it = q_item(p, ii);
+      const QItem it = cur;
+      cur = ii + static_cast<int>(gridDim.x) < nitems ? q_item(p, ii + gridDim.x) : cur;
       const int nunit = 2 * it.nblk;
       const int qbuf = I % QB;
       const int64_t kvrow0 = (static_cast<int64_t>(it.b) * p.Hkv + it.h / G) * S;
@@ -1070,7 +1147,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // Workspace: delta [B, Hq, S] fp32; fp32 dK and dV rows of the compact
 // global-key lists [B, Hkv, S, D] each; the compact bf16 K and V copies
 // [B, Hkv, S, D] each; the global-key work items (at most B x ceil(S/128) x
-// ceil(ceil(S/128)/kTcChunkTiles) pairs of int32) after their count.
+// ceil(ceil(S/128)/kTcChunkTiles) pairs of int32) after their count and the
+// per-sequence offsets.
 struct BwdWs {
   size_t delta, dk, dv, kc, vc, items;
   size_t total() const { return delta + dk + dv + kc + vc + items; }
@@ -1085,7 +1163,7 @@ BwdWs bwd_ws(int B, int Hq, int Hkv, int S, int D) {
   w.dv = w.dk;
   w.kc = r256(static_cast<size_t>(B) * Hkv * S * D * 2);
   w.vc = w.kc;
-  w.items = 256 + r256(static_cast<size_t>(B) * nwin * nchunk * 8);
+  w.items = r256(4 + static_cast<size_t>(B) * 4) + r256(static_cast<size_t>(B) * nwin * nchunk * 8);
   return w;
 }
 
@@ -1125,7 +1203,8 @@ int launch_bwd(BwdParams p, const void* out, void* dq, void* dk, void* dv, void*
   __nv_bfloat16* kc = reinterpret_cast<__nv_bfloat16*>(base + w.delta + w.dk + w.dv);
   __nv_bfloat16* vc = reinterpret_cast<__nv_bfloat16*>(base + w.delta + w.dk + w.dv + w.kc);
   p.item_count = reinterpret_cast<int32_t*>(base + w.delta + w.dk + w.dv + w.kc + w.vc);
-  p.items = reinterpret_cast<int2*>(base + w.delta + w.dk + w.dv + w.kc + w.vc + 256);
+  p.items = reinterpret_cast<int2*>(base + w.delta + w.dk + w.dv + w.kc + w.vc +
+                                    (4 + static_cast<size_t>(p.B) * 4 + 255) / 256 * 256);
   p.nwin = (p.S + TBK - 1) / TBK;
   p.nchunk = (p.nwin + kTcChunkTiles - 1) / kTcChunkTiles;
   const int64_t qrows = static_cast<int64_t>(p.B) * p.Hq * p.S;
@@ -1147,7 +1226,7 @@ int launch_bwd(BwdParams p, const void* out, void* dq, void* dk, void* dv, void*
   const dim3 rgrid((p.S + 63) / 64, p.Hkv, p.B);
   k_bwd_prep<D><<<rgrid, 256, 0, st>>>(p, kc, vc);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  k_bwd_plan<<<1, 32, 0, st>>>(p);
+  k_bwd_plan<<<1, 32 * kPlanWarps, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   // persistent: one CTA per SM (shared memory and TMEM hold one)
   const int sms = num_sms();
