@@ -80,11 +80,11 @@ TRAFFIC = {
         bytes=69485568 + 1160448, per="launch", src=("decode.cu", "common.cuh"),
         sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
     "backward_llama3_8b_b1_s8192_d128_bf16": dict(
-        bytes=498886144 + 68659200, per="launch", src=("backward.cu", "common.cuh"),
-        sha1="11bd4cf8a0687eacce0e46894d94b9b4981cc760"),
+        bytes=438024192 + 69230336, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="2a223a1a60781ce45cbab4f3a3ad5c7f37003178"),
     "backward_pythia160m_b8h12_s2048_d64_bf16": dict(
-        bytes=288590848 + 31880192, per="launch", src=("backward.cu", "common.cuh"),
-        sha1="11bd4cf8a0687eacce0e46894d94b9b4981cc760"),
+        bytes=264635904 + 35314944, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="2a223a1a60781ce45cbab4f3a3ad5c7f37003178"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
         bytes=104811776 + 20765440, per="launch", src=("prefill_tc.cu", "common.cuh"),
         sha1="0a11e6db6fab1045752f3db57e190bbd825b7948"),
@@ -861,12 +861,12 @@ def bench_backward(sl, args, world, rank):
         "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": pk["bf16"],
                      "unit": "TFLOP/s", "frac": round(achieved / pk["bf16"], 4),
                      "traffic": _traffic(name, units=1), "launch_us": round(step_s * 1e6, 3),
-                     "kernel": ("sep_attn_backward: delta pass, separator-row gather, "
-                                "k_bwd_kv (dK, dV) + k_bwd_q (dQ) on tcgen05, separator-key "
-                                "scatter; traffic = all five launches"),
+                     "kernel": ("sep_attn_backward: separator-row gather, item plan, "
+                                "k_bwd_q (dQ, delta) + k_bwd_kv (dK, dV) on tcgen05, "
+                                "separator-key scatter; traffic = all five launches"),
                      "peak_source": pk["src"] + " bf16 dense burst"},
         "e2e": e2e, "clocks": clk,
-        # delta, gather, two tcgen05 kernels, scatter
+        # gather, plan, two tcgen05 kernels, scatter
         "gpu_launches": 5 * K,
     }
     if rank == 0 and world == 1 and not args.skip_cpu:

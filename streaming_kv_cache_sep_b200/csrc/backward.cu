@@ -20,7 +20,8 @@
 //     are taken as 128 consecutive positions, and each block visits the query
 //     tiles that reach it, with the global keys of the block masked out.
 // dQ is query-centric: each CTA owns 128 queries of one head and visits the
-// key blocks its tile keeps.  A delta pass runs first.
+// key blocks its tile keeps; it also forms delta_i from its tile of out and
+// dout and writes it for the key-centric kernel, which runs after it.
 #include <string.h>
 
 #include "common.cuh"
@@ -35,7 +36,7 @@ __device__ __forceinline__ void red_add_v2(float* p, float x, float y) {
 struct BwdParams {
   const __nv_bfloat16 *q, *k, *v, *dout;
   const float* lse;    // [B][Hq][S] natural log
-  const float* delta;  // [B][Hq][S]
+  float* delta;        // [B][Hq][S]: written by the query-centric kernel
   const uint8_t* is_sep;
   const int32_t *prefix, *idx;
   float *dk_acc, *dv_acc;  // fp32 dK, dV rows of the compact global-key lists
@@ -47,25 +48,6 @@ struct BwdParams {
   int nchunk;  // chunks per block of global keys = ceil(ceil(S / 128) / kTcChunkTiles)
   float scale_log2;
 };
-
-// delta[b,h,i] = sum_d dout . out, one warp per row
-template <int D>
-__global__ void k_bwd_delta(const __nv_bfloat16* __restrict__ out,
-                            const __nv_bfloat16* __restrict__ dout, float* __restrict__ delta,
-                            int64_t rows) {
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= rows) return;
-  constexpr int PER = D / 32;  // 2 or 4 elements per lane
-  float acc = 0.f;
-  const __nv_bfloat16* o = out + row * D + lane * PER;
-  const __nv_bfloat16* g = dout + row * D + lane * PER;
-#pragma unroll
-  for (int e = 0; e < PER; ++e) acc += __bfloat162float(o[e]) * __bfloat162float(g[e]);
-#pragma unroll
-  for (int off = 16; off; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) delta[row] = acc;
-}
 
 // ---------------------------------------------------------------------------
 // Two software-pipelined tcgen05 kernels on the operand forms of the forward.
@@ -81,7 +63,8 @@ __global__ void k_bwd_delta(const __nv_bfloat16* __restrict__ out,
 //     buffer.  TMEM: S0 [0,64) dP0 [64,128) S1 [128,192) dP1 [192,256)
 //     dV [256,256+D) dK [256+D,256+2D), and at D = 64 a second dV, dK pair
 //     [384,512) for every other item.
-//   k_bwd_q (query-centric, 128 queries in TMEM lanes, Q and dO resident):
+//   k_bwd_q (query-centric, 128 queries in TMEM lanes, Q, dO and out
+//     resident; delta of each row from dO and out first):
 //     over the kept key blocks of its tile as the forward does -- the global
 //     keys before the window from the compact list, then the window blocks
 //     with the element mask -- in units of 64 keys streamed through the
@@ -290,21 +273,25 @@ __device__ __forceinline__ void probs_grads(const uint32_t (&sv)[32], const uint
 
 // ---- work items
 //
-// Key-centric items: the global-key items (listed by k_bwd_plan), for kv
-// head 0, then for head 1, ..., then the window items (b, kv head, block of
-// 128 positions).  Query-centric items: (b, head, tile of 128 queries),
+// Key-centric items: listed by k_bwd_plan (global-key blocks on chunks of
+// query tiles, and window blocks of 128 positions).  Query-centric items: (b, head, tile of 128 queries),
 // tiles with more kept keys (later positions) first.  Both kernels are
 // persistent: CTA c takes items c, c + gridDim.x, ... in order, so every
 // role of the CTA walks the same sequence without handing items around.
 
-// The global-key items: for every sequence b, chunk c of kTcChunkTiles
-// query tiles [c kTcChunkTiles, +kTcChunkTiles) and block kb of 128 global
-// keys whose first key lies before the chunk's end, the item (b,
-// kb << 16 | c), in the order (b, c, kb): the items a CTA runs side by side
-// read the same query tiles.  One CTA; warp w takes sequences w, w + 32 ...:
-// their item counts, then (after one thread's prefix over the sequences)
-// their items.  p.item_count[1 + b] holds sequence b's offset.
+// The key-centric items, per sequence b and kv head g (b-major, then g):
+// for each chunk c of kTcChunkTiles query tiles [c kTcChunkTiles,
+// +kTcChunkTiles), the global-key items (blocks kb of 128 global keys whose
+// first key lies before the chunk's end), then the window items (blocks kb
+// of 128 positions): the items a CTA runs side by side read the query tiles
+// of one kv head, and the heavier come first.  Entry: (b Hkv + g, kb << 16 | c), with
+// c = 0xffff for a window item.  One CTA; warp w takes sequences w, w + 32
+// ...: their item counts, then (after one thread's prefix over the
+// sequences) the items of (b, g) pairs.  p.item_count[1 + b] holds sequence
+// b's offset.
 constexpr int kPlanWarps = 32;
+constexpr int kPlanCache = 512;  // blocks whose first chunk a warp keeps in shared memory
+constexpr int kWindowItem = 0xffff;
 __global__ void __launch_bounds__(32 * kPlanWarps) k_bwd_plan(const BwdParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nT = (p.S + TBQ - 1) / TBQ;
@@ -322,7 +309,7 @@ __global__ void __launch_bounds__(32 * kPlanWarps) k_bwd_plan(const BwdParams p)
     for (int kb = lane; kb < nb; kb += 32) n += nC - first_chunk(gl, kb);
 #pragma unroll
     for (int o = 16; o; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
-    if (lane == 0) off[b] = n;
+    if (lane == 0) off[b] = n + p.nwin;  // items per kv head
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -330,24 +317,34 @@ __global__ void __launch_bounds__(32 * kPlanWarps) k_bwd_plan(const BwdParams p)
     for (int b = 0; b < p.B; ++b) {
       const int n = off[b];
       off[b] = e;
-      e += n;
+      e += n * p.Hkv;
     }
     *p.item_count = e;
   }
   __syncthreads();
-  for (int b = warp; b < p.B; b += kPlanWarps) {
+  // (b, g) pairs across the warps; each warp caches its blocks' first chunks
+  __shared__ int16_t fc_s[kPlanWarps][kPlanCache];
+  for (int pr = warp; pr < p.B * p.Hkv; pr += kPlanWarps) {
+    const int b = pr / p.Hkv, g = pr % p.Hkv;
     const GlobalList gl(p, b);
     const int nb = (gl.total + TBK - 1) / TBK;
-    int e = off[b];
+    const bool cached = nb <= kPlanCache;
+    if (cached)
+      for (int kb = lane; kb < nb; kb += 32) fc_s[warp][kb] = static_cast<int16_t>(first_chunk(gl, kb));
+    __syncwarp();
+    const int per = ((b + 1 < p.B ? off[b + 1] : *p.item_count) - off[b]) / p.Hkv;  // items per head
+    int e = off[b] + g * per;
     for (int c = 0; c < nC; ++c) {
       for (int k0 = 0; k0 < nb; k0 += 32) {
         const int kb = k0 + lane;
-        const bool on = kb < nb && first_chunk(gl, kb) <= c;
+        const bool on = kb < nb && (cached ? fc_s[warp][kb] : first_chunk(gl, kb)) <= c;
         const uint32_t m = __ballot_sync(0xffffffffu, on);
-        if (on) p.items[e + __popc(m & ((1u << lane) - 1u))] = make_int2(b, (kb << 16) | c);
+        if (on) p.items[e + __popc(m & ((1u << lane) - 1u))] = make_int2(pr, (kb << 16) | c);
         e += __popc(m);
       }
     }
+    for (int kb = lane; kb < p.nwin; kb += 32) p.items[e + kb] = make_int2(pr, (kb << 16) | kWindowItem);
+    __syncwarp();
   }
 }
 
@@ -355,27 +352,23 @@ struct KvItem {
   int b, g, kb, t0, ntile;
   bool window;
 };
-__device__ __forceinline__ KvItem kv_item(const BwdParams& p, int i, int nglob) {
+__device__ __forceinline__ KvItem kv_item(const BwdParams& p, int i) {
   KvItem it;
   const int nT = (p.S + TBQ - 1) / TBQ;
-  if (i < nglob) {
-    const int nge = nglob / p.Hkv;
-    const int2 ent = p.items[i % nge];
-    it.g = i / nge;
-    it.b = ent.x;
-    it.kb = ent.y >> 16;
+  const int2 ent = p.items[i];
+  it.b = ent.x / p.Hkv;
+  it.g = ent.x % p.Hkv;
+  it.kb = ent.y >> 16;
+  const int c = ent.y & 0xffff;
+  if (c != kWindowItem) {
     const GlobalList gl(p, it.b);
     const int pos = gl.pos(it.kb * TBK);
-    const int first = (pos >= 0 && pos < p.S ? pos : 0) / TBQ, c0 = (ent.y & 0xffff) * kTcChunkTiles;
+    const int first = (pos >= 0 && pos < p.S ? pos : 0) / TBQ, c0 = c * kTcChunkTiles;
     it.t0 = first > c0 ? first : c0;
     const int t1 = c0 + kTcChunkTiles < nT ? c0 + kTcChunkTiles : nT;
     it.ntile = t1 - it.t0;
     it.window = false;
   } else {
-    const int w = i - nglob;
-    it.kb = w % p.nwin;
-    it.g = (w / p.nwin) % p.Hkv;
-    it.b = w / (p.nwin * p.Hkv);
     it.t0 = it.kb;
     const int last = it.kb * TBK + TBK - 1 + p.n - 1;
     it.ntile = (last < p.S - 1 ? last : p.S - 1) / TBQ + 1 - it.t0;
@@ -390,9 +383,9 @@ struct KvRow {
   KvItem it;
   int jp, use;
 };
-__device__ __forceinline__ KvRow kv_row(const BwdParams& p, int i, int nglob, int r) {
+__device__ __forceinline__ KvRow kv_row(const BwdParams& p, int i, int r) {
   KvRow x;
-  x.it = kv_item(p, i, nglob);
+  x.it = kv_item(p, i);
   x.jp = -1;
   x.use = 0;
   if (x.it.window) {
@@ -458,8 +451,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.S, G = p.Hq / p.Hkv;
-  const int nglob = *p.item_count * p.Hkv;
-  const int nitems = nglob + p.B * p.Hkv * p.nwin;
+  const int nitems = *p.item_count;
   // first row of unit u of item `it` (queries [64 (u & 1), +64) of the
   // tile of visit u >> 1) in the [B * Hq * S] view
   auto unit_row = [&](const KvItem& it, int u) -> int64_t {
@@ -511,9 +503,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t U = 0, I = 0;  // units and items of this CTA so far
     // every role decodes the next item (dependent global loads) while it
     // works on the current one
-    KvRow cur = blockIdx.x < nitems ? kv_row(p, blockIdx.x, nglob, r) : KvRow{};
+    KvRow cur = blockIdx.x < nitems ? kv_row(p, blockIdx.x, r) : KvRow{};
     for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
-      const KvRow nxt = i + static_cast<int>(gridDim.x) < nitems ? kv_row(p, i + gridDim.x, nglob, r) : cur;
+      const KvRow nxt = i + static_cast<int>(gridDim.x) < nitems ? kv_row(p, i + gridDim.x, r) : cur;
       const KvItem it = cur.it;
       const int jp = cur.jp, use = cur.use;
       cur = nxt;
@@ -626,10 +618,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr uint32_t id_o = idesc_mn(128, D, false, true);
       bool ok = true;
       uint32_t U = 0, I = 0;
-      KvItem cur = blockIdx.x < nitems ? kv_item(p, blockIdx.x, nglob) : KvItem{};
+      KvItem cur = blockIdx.x < nitems ? kv_item(p, blockIdx.x) : KvItem{};
       for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
         const KvItem it = cur;
-        cur = i + static_cast<int>(gridDim.x) < nitems ? kv_item(p, i + gridDim.x, nglob) : cur;
+        cur = i + static_cast<int>(gridDim.x) < nitems ? kv_item(p, i + gridDim.x) : cur;
         const int nunit = 2 * G * it.ntile;
         const int kbuf = I % KVB, abuf = I % ACCB;
         const uint32_t cdv = kColAcc + 2u * D * abuf, cdk = cdv + D;
@@ -707,10 +699,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t U = 0, I = 0;
     uint32_t issued_u = 0, issued_i = 0;  // copies started (units, items)
     bool ok = true;
-    KvItem cur = blockIdx.x < nitems ? kv_item(p, blockIdx.x, nglob) : KvItem{};
+    KvItem cur = blockIdx.x < nitems ? kv_item(p, blockIdx.x) : KvItem{};
     for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
       const KvItem it = cur;
-      cur = i + static_cast<int>(gridDim.x) < nitems ? kv_item(p, i + gridDim.x, nglob) : cur;
+      cur = i + static_cast<int>(gridDim.x) < nitems ? kv_item(p, i + gridDim.x) : cur;
       const int nunit = 2 * G * it.ntile;
       const int kbuf = I % KVB;
       bool go = true;
@@ -783,8 +775,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-// Shared memory of the query-centric kernel: QB buffers of an item's Q and
-// dO [128][D] (swizzled 64-column tiles; two where they fit); a ring of kNst
+// Shared memory of the query-centric kernel: QB buffers of an item's Q, dO
+// and out [128][D] (swizzled 64-column tiles; two where they fit); a ring of kNst
 // unit stages, each the unit's K and V rows [64][D]; the global flags of
 // each stage's keys as [kNst][2] 32-bit words (bit k of word m: key 32 m + k
 // of the unit).
@@ -792,7 +784,7 @@ template <int D>
 struct QSmem {
   static constexpr int NB = D / 64;
   static constexpr int QB = D == 64 ? 2 : 1;
-  static constexpr int QSZ = 2 * NB * kT128;  // Q tiles, then dO tiles
+  static constexpr int QSZ = 3 * NB * kT128;  // Q tiles, dO tiles, out tiles
   static constexpr int RING = QB * QSZ;
   static constexpr int STAGE = 2 * NB * kT64;  // K tiles, then V tiles
   static constexpr int GLB = RING + kNst * STAGE;
@@ -830,7 +822,8 @@ __device__ __forceinline__ QItem q_item(const BwdParams& p, int i) {
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_bwd_q(const BwdParams p, const __grid_constant__ CUtensorMap map_q,
-            const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_k,
+            const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_o,
+            const __grid_constant__ CUtensorMap map_k,
             const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_kc,
             const __grid_constant__ CUtensorMap map_vc, __nv_bfloat16* __restrict__ dq) {
   using Sm = QSmem<D>;
@@ -856,7 +849,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (threadIdx.x == 9 * 32) {
     for (int i = 0; i < QB; ++i) {
       sep::mbar_init(&bars.q_full[i], 1);
-      sep::mbar_init(&bars.q_free[i], 1);
+      sep::mbar_init(&bars.q_free[i], 9);  // the last score products' commit, the 8 compute warps
     }
     for (int i = 0; i < kNst; ++i) {
       sep::mbar_init(&bars.st_full[i], 32);
@@ -894,25 +887,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     uint32_t U = 0, I = 0;
     // every role decodes the next item while it works on the current one
-    auto row_stats = [&](const QItem& x, float& nl, float& dlv) {
+    auto row_nl = [&](const QItem& x) {
       const int i = x.t * TBQ + r;
-      const int64_t q0 = (static_cast<int64_t>(x.b) * p.Hq + x.h) * S;
-      nl = i < S ? -p.lse[q0 + i] * 1.44269504088896340736f : 0.f;
-      dlv = i < S ? p.delta[q0 + i] : 0.f;
+      return i < S ? -p.lse[(static_cast<int64_t>(x.b) * p.Hq + x.h) * S + i] * 1.44269504088896340736f : 0.f;
     };
     QItem cur = blockIdx.x < nitems ? q_item(p, blockIdx.x) : QItem{};
-    float cur_nl = 0.f, cur_dl = 0.f;
-    if (blockIdx.x < nitems) row_stats(cur, cur_nl, cur_dl);
+    float cur_nl = blockIdx.x < nitems ? row_nl(cur) : 0.f;
     for (int ii = blockIdx.x; ii < nitems && ok; ii += gridDim.x, ++I) {
       const QItem it = cur;
-      const float nlse2 = cur_nl, dl = cur_dl;
+      const float nlse2 = cur_nl;
       if (ii + static_cast<int>(gridDim.x) < nitems) {
         cur = q_item(p, ii + gridDim.x);
-        row_stats(cur, cur_nl, cur_dl);
+        cur_nl = row_nl(cur);
       }
       const int nunit = 2 * it.nblk;
       const int i = it.t * TBQ + r;
       const int64_t qrow0 = (static_cast<int64_t>(it.b) * p.Hq + it.h) * S;
+      // delta of this row: dout . out over its D columns (both warps of the
+      // lane quarter form it; the first stores it for the key-centric kernel)
+      const int qbuf = I % QB;
+      if (!warp_wait(&bars.q_full[qbuf], (I / QB) & 1, abort, p.err)) {
+        ok = false;
+        break;
+      }
+      float dl = 0.f;
+      {
+        const uint8_t* dos = smem + qbuf * Sm::QSZ + NB * kT128;
+        const uint8_t* os = dos + NB * kT128;
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          const uint32_t off = static_cast<uint32_t>((c >> 3) * kT128 + r * 128 + ((((c & 7) ^ (r & 7))) << 4));
+          const uint4 a4 = *reinterpret_cast<const uint4*>(dos + off);
+          const uint4 b4 = *reinterpret_cast<const uint4*>(os + off);
+          const uint32_t aw[4] = {a4.x, a4.y, a4.z, a4.w}, bw[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            dl = fmaf(__uint_as_float(aw[e] << 16), __uint_as_float(bw[e] << 16), dl);
+            dl = fmaf(__uint_as_float(aw[e] & 0xffff0000u), __uint_as_float(bw[e] & 0xffff0000u), dl);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) sep::mbar_arrive(&bars.q_free[qbuf]);  // this warp is done with dO and out
+      if (i >= S) dl = 0.f;
+      else if (ch == 0) p.delta[qrow0 + i] = dl;
       const float2 nl2 = make_float2(nlse2, nlse2), dl2 = make_float2(dl, dl);
       for (int u = 0; u < nunit; ++u) {
         const uint32_t gu = U + u;
@@ -1084,6 +1102,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           sep::mbar_arrive_expect_tx(&bars.q_full[qbuf], Sm::QSZ);
           load_tile128<D>(smem + qbuf * Sm::QSZ, &map_q, row, &bars.q_full[qbuf]);
           load_tile128<D>(smem + qbuf * Sm::QSZ + NB * kT128, &map_do, row, &bars.q_full[qbuf]);
+          load_tile128<D>(smem + qbuf * Sm::QSZ + 2 * NB * kT128, &map_o, row, &bars.q_full[qbuf]);
         }
       }
       if (!__shfl_sync(0xffffffffu, go, 0)) break;
@@ -1147,8 +1166,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // Workspace: delta [B, Hq, S] fp32; fp32 dK and dV rows of the compact
 // global-key lists [B, Hkv, S, D] each; the compact bf16 K and V copies
 // [B, Hkv, S, D] each; the global-key work items (at most B x ceil(S/128) x
-// ceil(ceil(S/128)/kTcChunkTiles) pairs of int32) after their count and the
-// per-sequence offsets.
+// ceil(ceil(S/128)/kTcChunkTiles) x Hkv global items and B x ceil(S/128) x
+// Hkv window items, pairs of int32) after their count and the per-sequence
+// offsets.
 struct BwdWs {
   size_t delta, dk, dv, kc, vc, items;
   size_t total() const { return delta + dk + dv + kc + vc + items; }
@@ -1163,7 +1183,8 @@ BwdWs bwd_ws(int B, int Hq, int Hkv, int S, int D) {
   w.dv = w.dk;
   w.kc = r256(static_cast<size_t>(B) * Hkv * S * D * 2);
   w.vc = w.kc;
-  w.items = r256(4 + static_cast<size_t>(B) * 4) + r256(static_cast<size_t>(B) * nwin * nchunk * 8);
+  w.items = r256(4 + static_cast<size_t>(B) * 4) +
+            r256(static_cast<size_t>(B) * Hkv * nwin * (nchunk + 1) * 8);
   return w;
 }
 
@@ -1212,17 +1233,15 @@ int launch_bwd(BwdParams p, const void* out, void* dq, void* dk, void* dv, void*
   if (qrows > 0x7fffffffLL) return SEP_ETOOBIG;
   // 128-row boxes for the operands a CTA keeps (K, V of the key-centric
   // kernel; Q, dO of the query-centric one), 64-row boxes for the ring units
-  CUtensorMap mq, mdo, mk, mv, mkc, mvc, uq, udo, uk, uv, ukc, uvc;
+  CUtensorMap mq, mdo, mo, mk, mv, mkc, mvc, uq, udo, uk, uv, ukc, uvc;
   if (!sep::make_rows_map(&mq, p.q, qrows, D, TBQ) || !sep::make_rows_map(&mdo, p.dout, qrows, D, TBQ) ||
+      !sep::make_rows_map(&mo, out, qrows, D, TBQ) ||
       !sep::make_rows_map(&mk, p.k, krows, D, TBK) || !sep::make_rows_map(&mv, p.v, krows, D, TBK) ||
       !sep::make_rows_map(&mkc, kc, krows, D, TBK) || !sep::make_rows_map(&mvc, vc, krows, D, TBK) ||
       !sep::make_rows_map(&uq, p.q, qrows, D, 64) || !sep::make_rows_map(&udo, p.dout, qrows, D, 64) ||
       !sep::make_rows_map(&uk, p.k, krows, D, 64) || !sep::make_rows_map(&uv, p.v, krows, D, 64) ||
       !sep::make_rows_map(&ukc, kc, krows, D, 64) || !sep::make_rows_map(&uvc, vc, krows, D, 64))
     return SEP_ECUDA;
-  k_bwd_delta<D><<<static_cast<unsigned>((qrows + 7) / 8), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(out), p.dout, delta, qrows);
-  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   const dim3 rgrid((p.S + 63) / 64, p.Hkv, p.B);
   k_bwd_prep<D><<<rgrid, 256, 0, st>>>(p, kc, vc);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
@@ -1230,12 +1249,13 @@ int launch_bwd(BwdParams p, const void* out, void* dq, void* dk, void* dv, void*
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   // persistent: one CTA per SM (shared memory and TMEM hold one)
   const int sms = num_sms();
-  k_bwd_kv<D><<<sms, kTcThreads, KvSmem<D>::BYTES, st>>>(
-      p, uq, udo, mk, mv, mkc, mvc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
-  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  // dQ and delta first, then dK and dV (which read delta)
   const int64_t qitems = static_cast<int64_t>(p.B) * p.Hq * ((p.S + TBQ - 1) / TBQ);
   k_bwd_q<D><<<static_cast<unsigned>(qitems < sms ? qitems : sms), kTcThreads, QSmem<D>::BYTES, st>>>(
-      p, mq, mdo, uk, uv, ukc, uvc, static_cast<__nv_bfloat16*>(dq));
+      p, mq, mdo, mo, uk, uv, ukc, uvc, static_cast<__nv_bfloat16*>(dq));
+  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  k_bwd_kv<D><<<sms, kTcThreads, KvSmem<D>::BYTES, st>>>(
+      p, uq, udo, mk, mv, mkc, mvc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
   k_bwd_scatter<D><<<rgrid, 256, 0, st>>>(p, p.scale_log2 / 1.44269504088896340736f,
                                            static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
