@@ -743,7 +743,8 @@ def bench_ingest(sl, args, world, rank):
                    "l2": "flushed between timed steps (256 MiB write, outside the events)",
                    "parallelism": "replica per GPU (weak)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": pk["hbm"],
-                     "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4), "traffic": None,
+                     "unit": "GB/s", "frac": round(achieved / pk["hbm"], 4),
+                     "traffic": _traffic(name, units=1),
                      "bytes_per_launch": int(alg), "launch_us": round(step_s * 1e6, 3),
                      "kernel": "sepcache_ingest over %d layers (state at layer 0, row copies at "
                                "every layer)" % L,
