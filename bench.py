@@ -74,11 +74,15 @@ TRAFFIC = {
         bytes=(28617472 + 0) / (420.5 * 16), per="row", src=("decode.cu", "common.cuh"),
         sha1="15a13239d28cd65b3fab191c803aa3c5a4c49bee"),
     "decode_rope_llama3_8b_b16_l32_t65536_d128_bf16": dict(
-        bytes=(28885248 + 0) / (421.19 * 16), per="row", src=("decode.cu", "common.cuh"),
-        sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
+        bytes=(28890368 + 0) / (421.19 * 16), per="row", src=("decode.cu", "common.cuh"),
+        sha1="15a13239d28cd65b3fab191c803aa3c5a4c49bee"),
     "generate_masked_llama3_8b_b16_s8192_d128_bf16": dict(
-        bytes=69485568 + 1160448, per="launch", src=("decode.cu", "common.cuh"),
-        sha1="ba4365934dd4b41e4875743a7a5f9d3d9de0a56c"),
+        bytes=69489920 + 773120, per="launch", src=("decode.cu", "common.cuh"),
+        sha1="15a13239d28cd65b3fab191c803aa3c5a4c49bee"),
+    # one ingestion step: the state kernel and the 32 layers' row copies
+    "ingest_llama3_8b_b16_l32_t4096_d128_bf16": dict(
+        bytes=879904256 + 2625280, per="launch", src=("sepcache.cu", "common.cuh"),
+        sha1="0d11d7ce0b1432ab13e322fbddf2eb9d687f9376"),
     "backward_llama3_8b_b1_s8192_d128_bf16": dict(
         bytes=438024192 + 69230336, per="launch", src=("backward.cu", "common.cuh"),
         sha1="2a223a1a60781ce45cbab4f3a3ad5c7f37003178"),

@@ -77,6 +77,11 @@ def _index_cases():
     alt[0, ::2] = 1
     alt[1, 16383:16386] = 1  # a run across the 16384-position chunk edge
     cases.append(("alternating_and_edge_run", alt))
+    # several chunks with flag bytes other than 1 (any nonzero byte is a
+    # separator): rows 16-byte aligned (S % 16 == 0) and not (S odd)
+    for S in (40000, 40001):
+        f = rng.choice(np.array([0, 0, 0, 0, 1, 2, 127, 128, 255], np.uint8), size=(2, S))
+        cases.append(("nonzero_bytes_%d" % S, f))
     return cases
 
 
