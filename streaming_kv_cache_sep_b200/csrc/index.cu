@@ -88,14 +88,37 @@ __global__ void __launch_bounds__(kScanThreads) k_build_index(
   const uint32_t lt = (1u << lane) - 1u;
   auto flag_at = [&](int p) -> bool { return FROM_IDS ? in_set(tok[p], set) : f[p] != 0; };
 
-  // separators before the chunk, and in the whole sequence
+  // separators before the chunk, and in the whole sequence (every chunk's
+  // CTA counts the whole sequence; with flags in 16-byte-aligned rows, 16
+  // flags per load: a byte's top bit is set where the byte is nonzero, and
+  // the four 0/1 bytes of a word are summed by a multiply)
   int before = 0, total = -1;
   if (gridDim.x > 1) {
     int tot = 0;
-    for (int p = threadIdx.x; p < S; p += blockDim.x) {
-      const int v = flag_at(p);
-      tot += v;
-      before += (p < chunk0) ? v : 0;
+    if (!FROM_IDS && (reinterpret_cast<uintptr_t>(f) & 15u) == 0) {
+      const uint4* f4 = reinterpret_cast<const uint4*>(f);
+      const int n16 = S >> 4;  // chunk0 is a multiple of 16
+      for (int q = threadIdx.x; q < n16; q += blockDim.x) {
+        const uint4 w = f4[q];
+        auto nz4 = [](uint32_t x) {  // nonzero bytes of x
+          const uint32_t hi = (((x & 0x7f7f7f7fu) + 0x7f7f7f7fu) | x) & 0x80808080u;
+          return static_cast<int>(((hi >> 7) * 0x01010101u) >> 24);
+        };
+        const int v = nz4(w.x) + nz4(w.y) + nz4(w.z) + nz4(w.w);
+        tot += v;
+        before += (16 * q < chunk0) ? v : 0;
+      }
+      for (int p = (n16 << 4) + threadIdx.x; p < S; p += blockDim.x) {
+        const int v = f[p] != 0;
+        tot += v;
+        before += (p < chunk0) ? v : 0;
+      }
+    } else {
+      for (int p = threadIdx.x; p < S; p += blockDim.x) {
+        const int v = flag_at(p);
+        tot += v;
+        before += (p < chunk0) ? v : 0;
+      }
     }
     before = block_sum(before, red);
     total = block_sum(tot, red);
