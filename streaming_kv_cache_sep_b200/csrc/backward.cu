@@ -14,7 +14,7 @@
 //   * global keys (j < a or a separator) are kept by every query i >= j;
 //     they are taken 128 at a time from the compact list of global keys, and
 //     each block visits the query tiles from its first key's on, split into
-//     chunks of kTcChunkTiles tiles aligned to multiples of kTcChunkTiles
+//     chunks of ctiles tiles aligned to multiples of ctiles (chunk_tiles<D>)
 //     (one work item per block, chunk and kv head);
 //   * local keys (all others) are kept only by queries i in [j, j + n); they
 //     are taken as 128 consecutive positions, and each block visits the query
@@ -45,7 +45,8 @@ struct BwdParams {
   int32_t* err;
   int B, Hq, Hkv, S, a, n;
   int nwin;    // window items per (b, kv head) = ceil(S / 128)
-  int nchunk;  // chunks per block of global keys = ceil(ceil(S / 128) / kTcChunkTiles)
+  int ctiles;  // query tiles per chunk of a global-key item (chunk_tiles<D>)
+  int nchunk;  // chunks per block of global keys = ceil(ceil(S / 128) / ctiles)
   float scale_log2;
 };
 
@@ -92,7 +93,13 @@ constexpr int kNst = 4;           // stages of the 64-row operand ring
 constexpr int kT64 = 64 * 128;    // one 64-row x 64-column swizzled tile
 constexpr uint32_t kColAcc = 256;    // accumulators: dV, dK (key-centric) / dQ (query-centric)
 constexpr int kT128 = 128 * 128;  // one 128-row x 64-column swizzled tile
-constexpr int kTcChunkTiles = 4;  // query tiles per item of global keys
+// Query tiles per chunk of a global-key item, measured per head dimension
+// (Llama-3 8k shape at D = 128: 4 tiles 0.541 ms, 8 0.595, 16 0.646;
+// Pythia-160M shape at D = 64: 4 tiles 0.239 ms, 8 0.218, 16 0.238).  At
+// D = 64 the key-centric kernel double-buffers K and V, so fewer, longer
+// items cost no reload bubble.
+template <int D>
+constexpr int chunk_tiles() { return D == 64 ? 8 : 4; }
 
 // packed fp32 pairs (one f32x2 instruction per pair)
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
@@ -280,8 +287,8 @@ __device__ __forceinline__ void probs_grads(const uint32_t (&sv)[32], const uint
 // role of the CTA walks the same sequence without handing items around.
 
 // The key-centric items, per sequence b and kv head g (b-major, then g):
-// for each chunk c of kTcChunkTiles query tiles [c kTcChunkTiles,
-// +kTcChunkTiles), the global-key items (blocks kb of 128 global keys whose
+// for each chunk c of p.ctiles query tiles [c ctiles, +ctiles), the
+// global-key items (blocks kb of 128 global keys whose
 // first key lies before the chunk's end), then the window items (blocks kb
 // of 128 positions): the items a CTA runs side by side read the query tiles
 // of one kv head, and the heavier come first.  Entry: (b Hkv + g, kb << 16 | c), with
@@ -295,12 +302,12 @@ constexpr int kWindowItem = 0xffff;
 __global__ void __launch_bounds__(32 * kPlanWarps) k_bwd_plan(const BwdParams p) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nT = (p.S + TBQ - 1) / TBQ;
-  const int nC = (nT + kTcChunkTiles - 1) / kTcChunkTiles;
+  const int nC = (nT + p.ctiles - 1) / p.ctiles;
   int32_t* const off = p.item_count + 1;
   // chunk of the first tile of block kb of sequence b
   auto first_chunk = [&](const GlobalList& gl, int kb) {
     const int pos = gl.pos(kb * TBK);
-    return (pos >= 0 && pos < p.S ? pos : 0) / TBQ / kTcChunkTiles;
+    return (pos >= 0 && pos < p.S ? pos : 0) / TBQ / p.ctiles;
   };
   for (int b = warp; b < p.B; b += kPlanWarps) {
     const GlobalList gl(p, b);
@@ -363,9 +370,9 @@ __device__ __forceinline__ KvItem kv_item(const BwdParams& p, int i) {
   if (c != kWindowItem) {
     const GlobalList gl(p, it.b);
     const int pos = gl.pos(it.kb * TBK);
-    const int first = (pos >= 0 && pos < p.S ? pos : 0) / TBQ, c0 = c * kTcChunkTiles;
+    const int first = (pos >= 0 && pos < p.S ? pos : 0) / TBQ, c0 = c * p.ctiles;
     it.t0 = first > c0 ? first : c0;
-    const int t1 = c0 + kTcChunkTiles < nT ? c0 + kTcChunkTiles : nT;
+    const int t1 = c0 + p.ctiles < nT ? c0 + p.ctiles : nT;
     it.ntile = t1 - it.t0;
     it.window = false;
   } else {
@@ -1166,7 +1173,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // Workspace: delta [B, Hq, S] fp32; fp32 dK and dV rows of the compact
 // global-key lists [B, Hkv, S, D] each; the compact bf16 K and V copies
 // [B, Hkv, S, D] each; the global-key work items (at most B x ceil(S/128) x
-// ceil(ceil(S/128)/kTcChunkTiles) x Hkv global items and B x ceil(S/128) x
+// ceil(ceil(S/128)/chunk_tiles) x Hkv global items and B x ceil(S/128) x
 // Hkv window items, pairs of int32) after their count and the per-sequence
 // offsets.
 struct BwdWs {
@@ -1176,7 +1183,8 @@ struct BwdWs {
 BwdWs bwd_ws(int B, int Hq, int Hkv, int S, int D) {
   auto r256 = [](size_t x) { return (x + 255) / 256 * 256; };
   const size_t nwin = (static_cast<size_t>(S) + TBK - 1) / TBK;
-  const size_t nchunk = (nwin + kTcChunkTiles - 1) / kTcChunkTiles;
+  const int ct = D == 64 ? chunk_tiles<64>() : chunk_tiles<128>();
+  const size_t nchunk = (nwin + ct - 1) / ct;
   BwdWs w;
   w.delta = r256(static_cast<size_t>(B) * Hq * S * 4);
   w.dk = r256(static_cast<size_t>(B) * Hkv * S * D * 4);
@@ -1227,7 +1235,8 @@ int launch_bwd(BwdParams p, const void* out, void* dq, void* dk, void* dv, void*
   p.items = reinterpret_cast<int2*>(base + w.delta + w.dk + w.dv + w.kc + w.vc +
                                     (4 + static_cast<size_t>(p.B) * 4 + 255) / 256 * 256);
   p.nwin = (p.S + TBK - 1) / TBK;
-  p.nchunk = (p.nwin + kTcChunkTiles - 1) / kTcChunkTiles;
+  p.ctiles = chunk_tiles<D>();
+  p.nchunk = (p.nwin + p.ctiles - 1) / p.ctiles;
   const int64_t qrows = static_cast<int64_t>(p.B) * p.Hq * p.S;
   const int64_t krows = static_cast<int64_t>(p.B) * p.Hkv * p.S;
   if (qrows > 0x7fffffffLL) return SEP_ETOOBIG;
