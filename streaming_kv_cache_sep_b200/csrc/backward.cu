@@ -154,20 +154,39 @@ struct GlobalList {
   __device__ int pos(int t) const { return t < a0 ? t : ix[pre[a0] + t - a0]; }
 };
 
+// Programmatic launch: let the next grid on the stream start launching
+// (pdl_trigger), and wait until the grids before this one have completed
+// with their stores visible (pdl_wait; returns at once without a
+// programmatic dependency).
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Copies the global keys' K/V rows into the compact buffers (rows past the
 // list and up to the next multiple of 128, at least 128 and at most S, are
 // zero-filled so whole tiles read finite values) and zeroes the fp32
 // dK/dV rows of the list.  One CTA per 64 rows of (b, kv head).
+//
+// Runs alongside k_bwd_plan (launched just before it, programmatically):
+// both read only the index.  CTA (0, 0, 0) waits for the plan grid before
+// it ends, so the completion of this grid, which the next launch waits for,
+// also implies the plan's.
 template <int D>
 __global__ void __launch_bounds__(256) k_bwd_prep(const BwdParams p, __nv_bfloat16* __restrict__ kc,
                                                   __nv_bfloat16* __restrict__ vc) {
   constexpr int CH = D / 8;  // 16-byte chunks per bf16 row
+  if (threadIdx.x == 0) pdl_trigger();
+  const bool chain = (blockIdx.x | blockIdx.y | blockIdx.z) == 0;
   const int g = blockIdx.y, b = blockIdx.z, r0 = blockIdx.x * 64;
   const GlobalList gl(p, b);
   int lim = (gl.total + TBK - 1) / TBK * TBK;
   if (lim < TBK) lim = TBK;
   if (lim > p.S) lim = p.S;
-  if (r0 >= lim) return;
+  if (r0 >= lim) {
+    if (chain) pdl_wait();
+    return;
+  }
   const int64_t base = (static_cast<int64_t>(b) * p.Hkv + g) * p.S;
   for (int e = threadIdx.x; e < 64 * CH; e += 256) {
     const int r = r0 + e / CH, c = e % CH;
@@ -190,6 +209,7 @@ __global__ void __launch_bounds__(256) k_bwd_prep(const BwdParams p, __nv_bfloat
     reinterpret_cast<uint4*>(kc + (base + r) * D)[c] = kv;
     reinterpret_cast<uint4*>(vc + (base + r) * D)[c] = vv;
   }
+  if (chain) pdl_wait();
 }
 
 // The global keys' fp32 dK (times scale) and dV sums -> bf16 rows at their
@@ -200,6 +220,9 @@ __global__ void __launch_bounds__(256) k_bwd_scatter(const BwdParams p, float sc
                                                      __nv_bfloat16* __restrict__ dv) {
   constexpr int CH = D / 8;
   const int g = blockIdx.y, b = blockIdx.z, r0 = blockIdx.x * 64;
+  // every CTA waits for the key-centric kernel (its sums), so this grid
+  // completes only after it
+  pdl_wait();
   const GlobalList gl(p, b);
   if (r0 >= gl.total) return;
   const int64_t base = (static_cast<int64_t>(b) * p.Hkv + g) * p.S;
@@ -300,6 +323,7 @@ constexpr int kPlanWarps = 32;
 constexpr int kPlanCache = 512;  // blocks whose first chunk a warp keeps in shared memory
 constexpr int kWindowItem = 0xffff;
 __global__ void __launch_bounds__(32 * kPlanWarps) k_bwd_plan(const BwdParams p) {
+  if (threadIdx.x == 0) pdl_trigger();  // k_bwd_prep runs alongside
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nT = (p.S + TBQ - 1) / TBQ;
   const int nC = (nT + p.ctiles - 1) / p.ctiles;
@@ -458,7 +482,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.S, G = p.Hq / p.Hkv;
-  const int nitems = *p.item_count;
   // first row of unit u of item `it` (queries [64 (u & 1), +64) of the
   // tile of visit u >> 1) in the [B * Hq * S] view
   auto unit_row = [&](const KvItem& it, int u) -> int64_t {
@@ -485,17 +508,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       sep::mbar_init(&bars.acc_free[i], 8);
     }
     sep::mbar_init(&bars.drain, 1);
-    // a wait of an earlier CTA gave up: this one ends at its first wait too
-    bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
     sep::mbar_fence_init();
+    pdl_trigger();  // the next kernel's CTAs take SMs as this grid's retire
   }
   if (warp == 8) {
     sep::tmem_alloc(&bars.tmem_base, 512);
     sep::tmem_relinquish();
   }
+  // everything above overlaps the previous kernel; its outputs are read below
+  pdl_wait();
+  if (threadIdx.x == 9 * 32)  // a wait of an earlier CTA gave up: this one ends at its first wait too
+    bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
   sep::tc_fence_before();
   __syncthreads();
   sep::tc_fence_after();
+  const int nitems = *p.item_count;  // written by k_bwd_plan
   const uint32_t tmem = bars.tmem_base;
   volatile int* abort = &bars.abort;
 
@@ -871,14 +898,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       sep::mbar_init(&bars.acc_free[i], 8);
     }
     sep::mbar_init(&bars.drain, 1);
-    // a wait of an earlier CTA gave up: this one ends at its first wait too
-    bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
     sep::mbar_fence_init();
+    pdl_trigger();  // the next kernel's CTAs take SMs as this grid's retire
   }
   if (warp == 8) {
     sep::tmem_alloc(&bars.tmem_base, 512);
     sep::tmem_relinquish();
   }
+  // everything above overlaps the previous kernel; its outputs are read below
+  pdl_wait();
+  if (threadIdx.x == 9 * 32)  // a wait of an earlier CTA gave up: this one ends at its first wait too
+    bars.abort = (*reinterpret_cast<volatile int32_t*>(p.err) & sep::ERR_WAIT_TIMEOUT) ? 1 : 0;
   sep::tc_fence_before();
   __syncthreads();
   sep::tc_fence_after();
@@ -1252,23 +1282,33 @@ int launch_bwd(BwdParams p, const void* out, void* dq, void* dk, void* dv, void*
       !sep::make_rows_map(&ukc, kc, krows, D, 64) || !sep::make_rows_map(&uvc, vc, krows, D, 64))
     return SEP_ECUDA;
   const dim3 rgrid((p.S + 63) / 64, p.Hkv, p.B);
-  k_bwd_prep<D><<<rgrid, 256, 0, st>>>(p, kc, vc);
-  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  // Launch chain.  The plan is a plain launch: it starts once all earlier
+  // work on the stream has completed.  Every later kernel is a programmatic
+  // launch that overlaps the tail of the one before and runs
+  // griddepcontrol.wait before it reads any output of this call: k_bwd_prep
+  // runs alongside the plan (it reads only the index) and one of its CTAs
+  // waits for the plan before it ends, so each wait covers every launch
+  // before it.  The plan must stay a plain launch.
   k_bwd_plan<<<1, 32 * kPlanWarps, 0, st>>>(p);
   if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  if (sep::launch_pdl(k_bwd_prep<D>, rgrid, dim3(256), 0, st, p, kc, vc) != cudaSuccess)
+    return SEP_ECUDA;
   // persistent: one CTA per SM (shared memory and TMEM hold one)
   const int sms = num_sms();
   // dQ and delta first, then dK and dV (which read delta)
   const int64_t qitems = static_cast<int64_t>(p.B) * p.Hq * ((p.S + TBQ - 1) / TBQ);
-  k_bwd_q<D><<<static_cast<unsigned>(qitems < sms ? qitems : sms), kTcThreads, QSmem<D>::BYTES, st>>>(
-      p, mq, mdo, mo, uk, uv, ukc, uvc, static_cast<__nv_bfloat16*>(dq));
-  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  k_bwd_kv<D><<<sms, kTcThreads, KvSmem<D>::BYTES, st>>>(
-      p, uq, udo, mk, mv, mkc, mvc, static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
-  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
-  k_bwd_scatter<D><<<rgrid, 256, 0, st>>>(p, p.scale_log2 / 1.44269504088896340736f,
-                                           static_cast<__nv_bfloat16*>(dk), static_cast<__nv_bfloat16*>(dv));
-  if (cudaGetLastError() != cudaSuccess) return SEP_ECUDA;
+  if (sep::launch_pdl(k_bwd_q<D>, dim3(static_cast<unsigned>(qitems < sms ? qitems : sms)),
+                     dim3(kTcThreads), QSmem<D>::BYTES, st, p, mq, mdo, mo, uk, uv, ukc, uvc,
+                     static_cast<__nv_bfloat16*>(dq)) != cudaSuccess)
+    return SEP_ECUDA;
+  if (sep::launch_pdl(k_bwd_kv<D>, dim3(sms), dim3(kTcThreads), KvSmem<D>::BYTES, st, p, uq, udo, mk,
+                     mv, mkc, mvc, static_cast<__nv_bfloat16*>(dk),
+                     static_cast<__nv_bfloat16*>(dv)) != cudaSuccess)
+    return SEP_ECUDA;
+  if (sep::launch_pdl(k_bwd_scatter<D>, rgrid, dim3(256), 0, st, p,
+                     p.scale_log2 / 1.44269504088896340736f, static_cast<__nv_bfloat16*>(dk),
+                     static_cast<__nv_bfloat16*>(dv)) != cudaSuccess)
+    return SEP_ECUDA;
   return sep::launch_status();
 }
 
