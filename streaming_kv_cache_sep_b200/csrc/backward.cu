@@ -381,6 +381,7 @@ __global__ void __launch_bounds__(32 * kPlanWarps) k_bwd_plan(const BwdParams p)
 
 struct KvItem {
   int b, g, kb, t0, ntile;
+  int nh;  // 64-row units per query head: two per tile, less a last half no row of which keeps a key
   bool window;
 };
 __device__ __forceinline__ KvItem kv_item(const BwdParams& p, int i) {
@@ -405,8 +406,19 @@ __device__ __forceinline__ KvItem kv_item(const BwdParams& p, int i) {
     it.ntile = (last < p.S - 1 ? last : p.S - 1) / TBQ + 1 - it.t0;
     it.window = true;
   }
+  // the last query that keeps a key of the item: the window's end (window
+  // keys), or the sequence's (global keys); at a short window (n <= 64) the
+  // second half of a window item's last tile lies past it
+  int lastq = it.window ? it.kb * TBK + TBK - 1 + p.n - 1 : p.S - 1;
+  if (lastq > p.S - 1) lastq = p.S - 1;
+  it.nh = 2 * it.ntile - ((it.t0 + it.ntile - 1) * TBQ + 64 > lastq ? 1 : 0);
   return it;
 }
+// Unit u of a key-centric item: query head u / nh (of the kv head's group),
+// tile t0 + (u % nh) / 2, rows [64 ((u % nh) & 1), +64) of the tile.
+__device__ __forceinline__ int kv_unit_head(const KvItem& it, int u) { return u / it.nh; }
+__device__ __forceinline__ int kv_unit_tile(const KvItem& it, int u) { return it.t0 + ((u % it.nh) >> 1); }
+__device__ __forceinline__ int kv_unit_half(const KvItem& it, int u) { return (u % it.nh) & 1; }
 
 // An item and this compute thread's key row in it: position jp, and
 // whether the item's queries keep it (window items leave global keys out).
@@ -482,12 +494,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = p.S, G = p.Hq / p.Hkv;
-  // first row of unit u of item `it` (queries [64 (u & 1), +64) of the
-  // tile of visit u >> 1) in the [B * Hq * S] view
+  // first row of unit u of item `it` in the [B * Hq * S] view
   auto unit_row = [&](const KvItem& it, int u) -> int64_t {
-    const int v = u >> 1;
-    return (static_cast<int64_t>(it.b) * p.Hq + it.g * G + v / it.ntile) * S +
-           (it.t0 + v % it.ntile) * TBQ + 64 * (u & 1);
+    return (static_cast<int64_t>(it.b) * p.Hq + it.g * G + kv_unit_head(it, u)) * S +
+           kv_unit_tile(it, u) * TBQ + 64 * kv_unit_half(it, u);
   };
 
   if (threadIdx.x == 9 * 32) {
@@ -543,12 +553,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const KvItem it = cur.it;
       const int jp = cur.jp, use = cur.use;
       cur = nxt;
-      const int nunit = 2 * G * it.ntile;
+      const int nunit = G * it.nh;
       const int64_t kvrow0 = (static_cast<int64_t>(it.b) * p.Hkv + it.g) * S;
       for (int u = 0; u < nunit; ++u) {
         const uint32_t gu = U + u;
-        const int v = u >> 1, hh = u & 1, sb = gu & 1, st = gu % kNst;
-        const int i0 = (it.t0 + v % it.ntile) * TBQ;
+        const int hh = kv_unit_half(it, u), sb = gu & 1, st = gu % kNst;
+        const int i0 = kv_unit_tile(it, u) * TBQ;
         if (!warp_wait(&bars.st_full[st], (gu / kNst) & 1, abort, p.err) ||
             !warp_wait(&bars.s_full[sb], (gu >> 1) & 1, abort, p.err)) {
           ok = false;
@@ -656,7 +666,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
         const KvItem it = cur;
         cur = i + static_cast<int>(gridDim.x) < nitems ? kv_item(p, i + gridDim.x) : cur;
-        const int nunit = 2 * G * it.ntile;
+        const int nunit = G * it.nh;
         const int kbuf = I % KVB, abuf = I % ACCB;
         const uint32_t cdv = kColAcc + 2u * D * abuf, cdk = cdv + D;
         if (!sep::mbar_wait(&bars.kv_full[kbuf], (I / KVB) & 1, abort, p.err)) {
@@ -737,7 +747,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int i = blockIdx.x; i < nitems && ok; i += gridDim.x, ++I) {
       const KvItem it = cur;
       cur = i + static_cast<int>(gridDim.x) < nitems ? kv_item(p, i + gridDim.x) : cur;
-      const int nunit = 2 * G * it.ntile;
+      const int nunit = G * it.nh;
       const int kbuf = I % KVB;
       bool go = true;
       if (lane == 0) {
@@ -756,7 +766,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t gu = U + u;
         const int st = gu % kNst;
         const int64_t row0 = unit_row(it, u);
-        const int i0 = (it.t0 + (u >> 1) % it.ntile) * TBQ + 64 * (u & 1);
+        const int i0 = kv_unit_tile(it, u) * TBQ + 64 * kv_unit_half(it, u);
         float nlr[2], dlr[2];  // loads in flight during the wait below
 #pragma unroll
         for (int m = 0; m < 2; ++m) {
@@ -832,6 +842,7 @@ struct QBars {
 };
 struct QItem {
   int b, h, t, lo, qlast, nglo, nbg, nblk;
+  int nunit;  // 64-key units: two per block, less a last window half past the tile's last row
 };
 __device__ __forceinline__ QItem q_item(const BwdParams& p, int i) {
   QItem it;
@@ -850,6 +861,9 @@ __device__ __forceinline__ QItem q_item(const BwdParams& p, int i) {
   it.nglo = al + (pre[it.lo] - pre[al]);
   it.nbg = (it.nglo + TBK - 1) / TBK;
   it.nblk = it.nbg + (it.qlast - it.lo + TBK) / TBK;
+  // the last window block's second half starts past qlast at a short
+  // window (n <= 64): no row of the tile keeps any of its keys
+  it.nunit = 2 * it.nblk - (it.lo + (it.nblk - it.nbg - 1) * TBK + 64 > it.qlast ? 1 : 0);
   return it;
 }
 
@@ -937,7 +951,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         cur = q_item(p, ii + gridDim.x);
         cur_nl = row_nl(cur);
       }
-      const int nunit = 2 * it.nblk;
+      const int nunit = it.nunit;
       const int i = it.t * TBQ + r;
       const int64_t qrow0 = (static_cast<int64_t>(it.b) * p.Hq + it.h) * S;
       // delta of this row: dout . out over its D columns (both warps of the
@@ -1055,7 +1069,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int ii = blockIdx.x; ii < nitems && ok; ii += gridDim.x, ++I) {
         const QItem it = cur;
         cur = ii + static_cast<int>(gridDim.x) < nitems ? q_item(p, ii + gridDim.x) : cur;
-        const int nunit = 2 * it.nblk;
+        const int nunit = it.nunit;
         const int qbuf = I % QB, abuf = I & 1;
         const uint32_t cdq = kColAcc + static_cast<uint32_t>(D) * abuf;
         if (!sep::mbar_wait(&bars.q_full[qbuf], (I / QB) & 1, abort, p.err)) {
@@ -1127,7 +1141,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int ii = blockIdx.x; ii < nitems && ok; ii += gridDim.x, ++I) {
       const QItem it = cur;
       cur = ii + static_cast<int>(gridDim.x) < nitems ? q_item(p, ii + gridDim.x) : cur;
-      const int nunit = 2 * it.nblk;
+      const int nunit = it.nunit;
       const int qbuf = I % QB;
       const int64_t kvrow0 = (static_cast<int64_t>(it.b) * p.Hkv + it.h / G) * S;
       const uint8_t* fl = p.is_sep + static_cast<int64_t>(it.b) * S;

@@ -68,6 +68,7 @@ CASES = [
     (1, 2, 2, 190, 64, 2, 8, 1.0),       # every token a separator
     (1, 4, 1, 600, 128, 4, 64, 0.0),     # no separators: sinks + window
     (2, 8, 8, 700, 64, 4, 100, 0.08),    # many chunks of global keys
+    (1, 8, 2, 430, 128, 4, 48, 0.12),    # GQA, short window, last tile under 64 rows
 ]
 
 
