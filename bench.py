@@ -84,11 +84,11 @@ TRAFFIC = {
         bytes=879904256 + 2625280, per="launch", src=("sepcache.cu", "common.cuh"),
         sha1="0d11d7ce0b1432ab13e322fbddf2eb9d687f9376"),
     "backward_llama3_8b_b1_s8192_d128_bf16": dict(
-        bytes=436127232 + 68668672, per="launch", src=("backward.cu", "common.cuh"),
-        sha1="3d8a85abf0ac3a08c8a413852c5f4d31028f237d"),
+        bytes=433952512 + 67951872, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="0f3a298c018e77b40779bd9f5771a864484deb97"),
     "backward_pythia160m_b8h12_s2048_d64_bf16": dict(
-        bytes=264452864 + 34534912, per="launch", src=("backward.cu", "common.cuh"),
-        sha1="3d8a85abf0ac3a08c8a413852c5f4d31028f237d"),
+        bytes=263013376 + 32558592, per="launch", src=("backward.cu", "common.cuh"),
+        sha1="0f3a298c018e77b40779bd9f5771a864484deb97"),
     "prefill_llama3_8b_b1_s8192_d128_bf16": dict(
         bytes=104811776 + 20765440, per="launch", src=("prefill_tc.cu", "common.cuh"),
         sha1="0a11e6db6fab1045752f3db57e190bbd825b7948"),
