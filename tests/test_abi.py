@@ -136,3 +136,139 @@ def test_cache_layout_and_validation(sl):
     assert L.sep_attn_decode(ctypes.byref(c), 0, FAKE, 8 * 16, 0.0, FAKE, None, FAKE, ws, None) == -1
     assert L.sep_attn_decode(ctypes.byref(c), 0, FAKE, 32, 0.0, FAKE, None, FAKE, ws - 1, None) == -1
     assert L.sep_attn_decode(ctypes.byref(c), 0, None, 32, 0.0, FAKE, None, FAKE, ws, None) == -6
+
+
+def test_backward_rejects_bad_arguments(sl):
+    L = sl.lib()
+    need = L.sep_attn_backward_workspace(1, 4, 2, 16, 64)
+    assert need > 0
+    assert L.sep_attn_backward_workspace(1, 4, 2, 16, 96) == 0
+    assert L.sep_attn_backward_workspace(1, 3, 2, 16, 64) == 0
+    assert L.sep_attn_backward_workspace(0, 4, 2, 16, 64) == 0
+    assert L.sep_attn_backward_workspace(1, 4, 2, 0, 64) == 0
+    # grows with the sequence (fp32 dK/dV sums, compact rows, the item list)
+    assert L.sep_attn_backward_workspace(1, 4, 2, 4096, 128) > L.sep_attn_backward_workspace(1, 4, 2, 16, 128)
+    order = ("q", "k", "v", "out", "lse", "dout", "dtype", "is_sep", "prefix", "idx", "B", "Hq",
+             "Hkv", "S", "D", "a", "n", "scale", "dq", "dk", "dv", "ws", "wsb")
+
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, out=FAKE, lse=FAKE, dout=FAKE, dtype=1, is_sep=FAKE,
+                 prefix=FAKE, idx=FAKE, B=1, Hq=4, Hkv=2, S=16, D=64, a=4, n=8, scale=0.0,
+                 dq=FAKE, dk=FAKE, dv=FAKE, ws=FAKE, wsb=need)
+        a.update(kw)
+        return L.sep_attn_backward(*[a[x] for x in order], None)
+
+    assert call(dtype=0) == -2  # bf16 only
+    assert call(D=96) == -2
+    for bad in (dict(B=0), dict(S=0), dict(Hq=3), dict(a=-1), dict(n=0), dict(B=70000)):
+        assert call(**bad) == -1, bad
+    for name in ("q", "k", "v", "out", "lse", "dout", "is_sep", "prefix", "idx", "dq", "dk", "dv",
+                 "ws"):
+        assert call(**{name: None}) == -6, name
+    for name in ("q", "k", "v", "out", "dout", "dq", "dk", "dv"):
+        assert call(**{name: ctypes.c_void_p(4100)}) == -3, name
+    assert call(ws=ctypes.c_void_p(4096 + 16)) == -3  # the workspace is 256-byte aligned
+    assert call(wsb=need - 1) == -1
+
+
+def test_masked_generation_rejects_bad_arguments(sl):
+    L = sl.lib()
+    need = L.sep_attn_decode_masked_workspace(2, 8, 2, 64, 128)
+    assert need > 0
+    assert L.sep_attn_decode_masked_workspace(2, 8, 2, 64, 96) == 0
+    assert L.sep_attn_decode_masked_workspace(2, 6, 2, 64, 128) == 0  # 3 query heads per kv head
+    order = ("q", "k", "v", "dtype", "prefix", "idx", "B", "Hq", "Hkv", "S", "T", "D", "a", "n",
+             "scale", "out", "lse", "ws", "wsb")
+
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, dtype=1, prefix=FAKE, idx=FAKE, B=2, Hq=8, Hkv=2, S=64,
+                 T=40, D=128, a=4, n=16, scale=0.0, out=FAKE, lse=None, ws=None, wsb=0)
+        a.update(kw)
+        return L.sep_attn_decode_masked(*[a[x] for x in order], None)
+
+    assert call(dtype=2) == -2
+    assert call(D=96) == -2
+    for bad in (dict(T=0), dict(T=65), dict(Hq=6), dict(Hq=32), dict(Hq=7), dict(a=-1), dict(n=0),
+                dict(B=0), dict(S=0, T=0)):
+        assert call(**bad) == -1, bad
+    for name in ("q", "k", "v", "prefix", "idx", "out"):
+        assert call(**{name: None}) == -6, name
+    for name in ("q", "k", "v", "out"):
+        assert call(**{name: ctypes.c_void_p(4100)}) == -3, name
+    # fp32 merges its splits through the caller's workspace
+    assert call(dtype=0) == -6
+    assert call(dtype=0, ws=ctypes.c_void_p(4100), wsb=need) == -3
+    assert call(dtype=0, ws=FAKE, wsb=16) == -1
+
+
+def _carved(sl, cfg, layers, B, Hkv, D, dtype):
+    L = sl.lib()
+    nb = L.sepcache_bytes(cfg, layers, B, Hkv, D, dtype)
+    assert nb > 0
+    c = sl._SepCacheC()
+    assert L.sepcache_carve(ctypes.byref(c), ctypes.c_void_p(1 << 20), nb, cfg, layers, B, Hkv, D,
+                            dtype) == 0
+    return c
+
+
+def test_ingest_and_decode_step_reject_bad_arguments(sl):
+    L = sl.lib()
+    c = _carved(sl, sl.SepCacheCfg(4, 64, 128, 256), 32, 16, 8, 128, 1)
+    cp = ctypes.byref(c)
+    F = FAKE
+    # ingestion: cache, layer and T first, then pointers, then alignment
+    assert L.sepcache_ingest(None, 0, F, F, F, F, F, 10, None) == -6
+    assert L.sepcache_ingest(cp, 32, F, F, F, F, F, 10, None) == -1
+    assert L.sepcache_ingest(cp, -1, F, F, F, F, F, 10, None) == -1
+    assert L.sepcache_ingest(cp, 0, F, F, F, F, F, 0, None) == -1
+    assert L.sepcache_ingest(cp, 0, None, F, F, F, F, 10, None) == -6
+    assert L.sepcache_ingest(cp, 0, F, F, None, F, F, 10, None) == -6  # layer 0 reads the index
+    assert L.sepcache_ingest(cp, 1, ctypes.c_void_p(4100), F, None, None, None, 10, None) == -3
+    assert L.sepcache_ingest(cp, 1, F, F, None, None, None, 1 << 24, None) == -1  # B Hkv T >= 2^31
+    # a cache whose fields do not agree is refused by every call
+    bad = _carved(sl, sl.SepCacheCfg(4, 64, 128, 256), 32, 16, 8, 128, 1)
+    bad.cap += 1
+    assert L.sepcache_ingest(ctypes.byref(bad), 1, F, F, None, None, None, 10, None) == -1
+    assert L.sepcache_append(ctypes.byref(bad), 1, F, F, None, None) == -1
+    assert L.sep_attn_decode_workspace(ctypes.byref(bad), 32) == 0
+    # the fused step: layer, head grouping, pointers, alignment, workspace size
+    ws = L.sep_attn_decode_workspace(cp, 32)
+    assert ws > 0
+
+    def step(layer=1, q=F, kn=F, vn=F, is_sep=None, Hq=32, out=F, w=F, wb=ws, cache=cp):
+        return L.sep_attn_decode_step(cache, layer, q, kn, vn, is_sep, Hq, 0.0, out, None, w, wb,
+                                      None)
+
+    assert step(cache=None) == -6
+    assert step(cache=ctypes.byref(bad)) == -1
+    assert step(layer=32) == -1
+    assert step(Hq=24) == -1   # 3 query heads per kv head
+    assert step(Hq=128) == -1  # 16 query heads per kv head
+    assert step(Hq=30) == -1   # not a multiple of Hkv
+    assert step(layer=0) == -6  # layer 0 advances the cache from is_sep_new
+    for kw in (dict(q=None), dict(kn=None), dict(vn=None), dict(out=None), dict(w=None)):
+        assert step(**kw) == -6, kw
+    for kw in (dict(q=ctypes.c_void_p(4100)), dict(kn=ctypes.c_void_p(4104)),
+               dict(vn=ctypes.c_void_p(4108)), dict(out=ctypes.c_void_p(4100)),
+               dict(w=ctypes.c_void_p(4100))):
+        assert step(**kw) == -3, kw
+    assert step(wb=ws - 1) == -1
+
+
+def test_noalloc_decode_rejects_bad_arguments(sl):
+    L = sl.lib()
+    c = _carved(sl, sl.SepCacheCfg(4, 64, 128, 256), 2, 2, 2, 64, 1)
+    cp = ctypes.byref(c)
+    assert L.sep_attn_decode_noalloc(None, 0, FAKE, 4, 0.0, FAKE, None, None) == -6
+    assert L.sep_attn_decode_noalloc(cp, 2, FAKE, 4, 0.0, FAKE, None, None) == -1
+    assert L.sep_attn_decode_noalloc(cp, 0, FAKE, 6, 0.0, FAKE, None, None) == -1
+    assert L.sep_attn_decode_noalloc(cp, 0, FAKE, 3, 0.0, FAKE, None, None) == -1
+    assert L.sep_attn_decode_noalloc(cp, 0, None, 4, 0.0, FAKE, None, None) == -6
+    assert L.sep_attn_decode_noalloc(cp, 0, FAKE, 4, 0.0, None, None, None) == -6
+    assert L.sep_attn_decode_noalloc(cp, 0, ctypes.c_void_p(4100), 4, 0.0, FAKE, None, None) == -3
+    # an fp32 cache of more than 512 rows merges through the fixed scratch:
+    # B * Hq * ceil(cap / 64) partials beyond its 8192 slots are refused
+    # before anything is enqueued
+    big = _carved(sl, sl.SepCacheCfg(4, 300, 200, 100), 1, 64, 8, 64, 0)
+    assert big.cap == 605
+    assert L.sep_attn_decode_noalloc(ctypes.byref(big), 0, FAKE, 64, 0.0, FAKE, None, None) == -7
