@@ -145,6 +145,32 @@ def _need_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("expected contiguous CUDA tensors")
+    dev = next((t.device for t in ts if t is not None), None)
+    for t in ts:
+        if t is not None and t.device != dev:
+            raise ValueError("expected every tensor on %s, got one on %s" % (dev, t.device))
+
+
+def _expect(t, name, dtype, shape):
+    """The C calls take bare pointers and trust the sizes they are given, so
+    the binding checks each tensor's dtype and shape against the layout the
+    call documents (None: an optional tensor that was not passed)."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise TypeError("%s: expected %s, got %s" % (name, dtype, t.dtype))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s: expected shape %s, got %s" % (name, tuple(shape), tuple(t.shape)))
+
+
+def _dims(t, name, n):
+    if t.dim() != n:
+        raise ValueError("%s: expected %d dimensions, got shape %s" % (name, n, tuple(t.shape)))
+    return tuple(t.shape)
+
+
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
 
 
 # ------------------------------------------------------------------ index
@@ -152,8 +178,8 @@ def _need_cuda(*ts):
 
 def flags_from_ids(ids: torch.Tensor, sep_ids, stream=None) -> torch.Tensor:
     """uint8 flags: 1 where ids is one of sep_ids (a host list, <= 32 ids)."""
+    _expect(ids, "ids", torch.int32, ids.shape)
     _need_cuda(ids)
-    assert ids.dtype == torch.int32
     out = torch.empty(ids.shape, dtype=torch.uint8, device=ids.device)
     arr = (ctypes.c_int32 * len(sep_ids))(*[int(x) for x in sep_ids])
     _check("sep_flags_from_ids", _lib.sep_flags_from_ids(
@@ -164,8 +190,15 @@ def flags_from_ids(ids: torch.Tensor, sep_ids, stream=None) -> torch.Tensor:
 
 def build_index(is_sep: torch.Tensor, out=None, stream=None):
     """(prefix [B,S+1], idx [B,S] (-1 padded), count [B]) int32 on the device."""
+    B, S = _dims(is_sep, "is_sep", 2)
+    _expect(is_sep, "is_sep", torch.uint8, (B, S))
+    if out is not None:
+        prefix, idx, count = out
+        _expect(prefix, "prefix", torch.int32, (B, S + 1))
+        _expect(idx, "idx", torch.int32, (B, S))
+        _expect(count, "count", torch.int32, (B,))
+        _need_cuda(is_sep, prefix, idx, count)
     _need_cuda(is_sep)
-    B, S = is_sep.shape
     dev = is_sep.device
     if out is None:
         out = (torch.empty((B, S + 1), dtype=torch.int32, device=dev),
@@ -180,9 +213,16 @@ def build_index(is_sep: torch.Tensor, out=None, stream=None):
 def build_index_from_ids(ids: torch.Tensor, sep_ids, out=None, stream=None):
     """flags_from_ids then build_index in one launch: ids int32 [B,S] ->
     (is_sep uint8 [B,S], prefix [B,S+1], idx [B,S], count [B]) on the device."""
+    B, S = _dims(ids, "ids", 2)
+    _expect(ids, "ids", torch.int32, (B, S))
+    if out is not None:
+        is_sep, prefix, idx, count = out
+        _expect(is_sep, "is_sep", torch.uint8, (B, S))
+        _expect(prefix, "prefix", torch.int32, (B, S + 1))
+        _expect(idx, "idx", torch.int32, (B, S))
+        _expect(count, "count", torch.int32, (B,))
+        _need_cuda(ids, is_sep, prefix, idx, count)
     _need_cuda(ids)
-    assert ids.dtype == torch.int32 and ids.dim() == 2
-    B, S = ids.shape
     dev = ids.device
     if out is None:
         out = (torch.empty((B, S), dtype=torch.uint8, device=dev),
@@ -199,8 +239,10 @@ def build_index_from_ids(ids: torch.Tensor, sep_ids, out=None, stream=None):
 
 def count_pairs(prefix: torch.Tensor, a: int, n: int, out=None, stream=None) -> torch.Tensor:
     """Kept (query, key) pairs per sequence for one head, int64 [B]."""
-    _need_cuda(prefix)
-    B, S1 = prefix.shape
+    B, S1 = _dims(prefix, "prefix", 2)
+    _expect(prefix, "prefix", torch.int32, (B, S1))
+    _expect(out, "out", torch.int64, (B,))
+    _need_cuda(prefix, out)
     out = out if out is not None else torch.empty((B,), dtype=torch.int64, device=prefix.device)
     _check("sep_count_pairs", _lib.sep_count_pairs(_ptr(prefix), B, S1 - 1, a, n, _ptr(out),
                                                    _stream(stream)))
@@ -218,20 +260,27 @@ def prefill(q, k, v, is_sep, prefix, idx, a: int, n: int, scale: float = 0.0, ou
             lse=None, workspace=None, want_lse: bool = True, stream=None):
     """Sep-Attention over whole sequences.  q [B,Hq,S,D], k/v [B,Hkv,S,D]
     (bf16 -> tcgen05 path, fp32 -> exact FMA path).  Returns (out, lse)."""
-    _need_cuda(q, k, v, is_sep, prefix, idx, out, lse, workspace)
-    B, Hq, S, D = q.shape
-    Hkv = k.shape[1]
+    B, Hq, S, D = _dims(q, "q", 4)
     dt = _dtype_code(q)
+    Hkv = _dims(k, "k", 4)[1]
+    _expect(k, "k", q.dtype, (B, Hkv, S, D))
+    _expect(v, "v", q.dtype, (B, Hkv, S, D))
+    _expect(is_sep, "is_sep", torch.uint8, (B, S))
+    _expect(prefix, "prefix", torch.int32, (B, S + 1))
+    _expect(idx, "idx", torch.int32, (B, S))
+    _expect(out, "out", q.dtype, (B, Hq, S, D))
+    _expect(lse, "lse", torch.float32, (B, Hq, S))
+    _need_cuda(q, k, v, is_sep, prefix, idx, out, lse, workspace)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
     need = prefill_workspace_bytes(B, Hq, Hkv, S, D, dt)
-    if workspace is None or workspace.numel() < need:
+    if workspace is None or _nbytes(workspace) < need:
         workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
     _check("sep_attn_prefill", _lib.sep_attn_prefill(
         _ptr(q), _ptr(k), _ptr(v), dt, _ptr(is_sep), _ptr(prefix), _ptr(idx), B, Hq, Hkv, S, D,
-        a, n, float(scale), _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(),
+        a, n, float(scale), _ptr(out), _ptr(lse), _ptr(workspace), _nbytes(workspace),
         _stream(stream)))
     return out, lse
 
@@ -241,20 +290,31 @@ def backward(q, k, v, out, lse, dout, is_sep, prefix, idx, a: int, n: int, scale
     """Gradients of sum(out * dout) through Sep-Attention: q/out/dout
     [B,Hq,S,D], k/v [B,Hkv,S,D] bf16, lse [B,Hq,S] from prefill.
     Returns (dq, dk, dv)."""
-    _need_cuda(q, k, v, out, lse, dout, is_sep, prefix, idx, dq, dk, dv, workspace)
-    B, Hq, S, D = q.shape
-    Hkv = k.shape[1]
+    B, Hq, S, D = _dims(q, "q", 4)
     dt = _dtype_code(q)
+    Hkv = _dims(k, "k", 4)[1]
+    _expect(k, "k", q.dtype, (B, Hkv, S, D))
+    _expect(v, "v", q.dtype, (B, Hkv, S, D))
+    _expect(out, "out", q.dtype, (B, Hq, S, D))
+    _expect(lse, "lse", torch.float32, (B, Hq, S))
+    _expect(dout, "dout", q.dtype, (B, Hq, S, D))
+    _expect(is_sep, "is_sep", torch.uint8, (B, S))
+    _expect(prefix, "prefix", torch.int32, (B, S + 1))
+    _expect(idx, "idx", torch.int32, (B, S))
+    _expect(dq, "dq", q.dtype, (B, Hq, S, D))
+    _expect(dk, "dk", q.dtype, (B, Hkv, S, D))
+    _expect(dv, "dv", q.dtype, (B, Hkv, S, D))
+    _need_cuda(q, k, v, out, lse, dout, is_sep, prefix, idx, dq, dk, dv, workspace)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     need = int(_lib.sep_attn_backward_workspace(B, Hq, Hkv, S, D))
-    if workspace is None or workspace.numel() < need:
+    if workspace is None or _nbytes(workspace) < need:
         workspace = torch.empty((need,), dtype=torch.uint8, device=q.device)
     _check("sep_attn_backward", _lib.sep_attn_backward(
         _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dout), dt, _ptr(is_sep),
         _ptr(prefix), _ptr(idx), B, Hq, Hkv, S, D, a, n, float(scale), _ptr(dq), _ptr(dk),
-        _ptr(dv), _ptr(workspace), workspace.numel(), _stream(stream)))
+        _ptr(dv), _ptr(workspace), _nbytes(workspace), _stream(stream)))
     return dq, dk, dv
 
 
@@ -267,10 +327,16 @@ def decode_masked(q, k, v, prefix, idx, T: int, a: int, n: int, scale: float = 0
     attends over k/v [B,Hkv,S,D] rows 0..T-1 with the Sep-Attention kept set
     of its row; prefix/idx from build_index of the flags [B,S].
     Returns (out [B,Hq,D], lse [B,Hq])."""
-    _need_cuda(q, k, v, prefix, idx, out, lse, workspace)
-    B, Hq, D = q.shape
-    Hkv, S = k.shape[1], k.shape[2]
+    B, Hq, D = _dims(q, "q", 3)
     dt = _dtype_code(q)
+    _, Hkv, S, _ = _dims(k, "k", 4)
+    _expect(k, "k", q.dtype, (B, Hkv, S, D))
+    _expect(v, "v", q.dtype, (B, Hkv, S, D))
+    _expect(prefix, "prefix", torch.int32, (B, S + 1))
+    _expect(idx, "idx", torch.int32, (B, S))
+    _expect(out, "out", q.dtype, (B, Hq, D))
+    _expect(lse, "lse", torch.float32, (B, Hq))
+    _need_cuda(q, k, v, prefix, idx, out, lse, workspace)
     if out is None:
         out = torch.empty_like(q)
     if lse is None and want_lse:
@@ -284,7 +350,7 @@ def decode_masked(q, k, v, prefix, idx, T: int, a: int, n: int, scale: float = 0
             if workspace is None:
                 workspace = torch.zeros((need,), dtype=torch.uint8, device=q.device)
                 _masked_ws[key] = workspace
-        wsb = workspace.numel()
+        wsb = _nbytes(workspace)
     _check("sep_attn_decode_masked", _lib.sep_attn_decode_masked(
         _ptr(q), _ptr(k), _ptr(v), dt, _ptr(prefix), _ptr(idx), B, Hq, Hkv, S, int(T), D, a, n,
         float(scale), _ptr(out), _ptr(lse), _ptr(workspace), wsb, _stream(stream)))

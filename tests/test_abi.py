@@ -272,3 +272,80 @@ def test_noalloc_decode_rejects_bad_arguments(sl):
     big = _carved(sl, sl.SepCacheCfg(4, 300, 200, 100), 1, 64, 8, 64, 0)
     assert big.cap == 605
     assert L.sep_attn_decode_noalloc(ctypes.byref(big), 0, FAKE, 64, 0.0, FAKE, None, None) == -7
+
+
+def test_binding_checks_layouts_before_the_device(sl):
+    """The Python binding checks each tensor's dtype and shape against the
+    documented layout before it hands bare pointers to the library (CPU
+    tensors here: a correct layout gets as far as the device check)."""
+    import torch
+    bf, f32, u8, i32 = torch.bfloat16, torch.float32, torch.uint8, torch.int32
+    B, Hq, Hkv, S, D = 2, 4, 2, 40, 64
+    q = torch.zeros((B, Hq, S, D), dtype=bf)
+    k = torch.zeros((B, Hkv, S, D), dtype=bf)
+    v = torch.zeros((B, Hkv, S, D), dtype=bf)
+    fl = torch.zeros((B, S), dtype=u8)
+    pre = torch.zeros((B, S + 1), dtype=i32)
+    idx = torch.zeros((B, S), dtype=i32)
+    cuda_msg = "expected contiguous CUDA tensors"
+
+    with pytest.raises(ValueError, match=cuda_msg):
+        sl.prefill(q, k, v, fl, pre, idx, 4, 8)
+    with pytest.raises(TypeError, match="k:"):
+        sl.prefill(q, k.float(), v, fl, pre, idx, 4, 8)
+    with pytest.raises(ValueError, match="v: expected shape"):
+        sl.prefill(q, k, v[:, :, :S - 1].contiguous(), fl, pre, idx, 4, 8)
+    with pytest.raises(TypeError, match="is_sep:"):
+        sl.prefill(q, k, v, fl.bool(), pre, idx, 4, 8)
+    with pytest.raises(TypeError, match="prefix:"):
+        sl.prefill(q, k, v, fl, pre.long(), idx, 4, 8)
+    with pytest.raises(ValueError, match="prefix: expected shape"):
+        sl.prefill(q, k, v, fl, pre[:, :S].contiguous(), idx, 4, 8)
+    with pytest.raises(ValueError, match="idx: expected shape"):
+        sl.prefill(q, k, v, fl, pre, idx[:1].contiguous(), 4, 8)
+    with pytest.raises(TypeError, match="lse:"):
+        sl.prefill(q, k, v, fl, pre, idx, 4, 8, lse=torch.zeros((B, Hq, S), dtype=bf))
+    with pytest.raises(ValueError, match="out: expected shape"):
+        sl.prefill(q, k, v, fl, pre, idx, 4, 8, out=torch.zeros((B, Hq, S, 2 * D), dtype=bf))
+    with pytest.raises(ValueError, match="q: expected 4"):
+        sl.prefill(q[0], k, v, fl, pre, idx, 4, 8)
+    with pytest.raises(TypeError, match="unsupported dtype"):
+        sl.prefill(q.half(), k.half(), v.half(), fl, pre, idx, 4, 8)
+
+    lse = torch.zeros((B, Hq, S), dtype=f32)
+    with pytest.raises(ValueError, match=cuda_msg):
+        sl.backward(q, k, v, q, lse, q, fl, pre, idx, 4, 8)
+    with pytest.raises(ValueError, match="dout: expected shape"):
+        sl.backward(q, k, v, q, lse, q[:, :2].contiguous(), fl, pre, idx, 4, 8)
+    with pytest.raises(ValueError, match="lse: expected shape"):
+        sl.backward(q, k, v, q, lse[:, :, :4].contiguous(), q, fl, pre, idx, 4, 8)
+    with pytest.raises(ValueError, match="dk: expected shape"):
+        sl.backward(q, k, v, q, lse, q, fl, pre, idx, 4, 8, dk=torch.zeros_like(q))
+
+    qd = torch.zeros((B, Hq, D), dtype=bf)
+    with pytest.raises(ValueError, match=cuda_msg):
+        sl.decode_masked(qd, k, v, pre, idx, S, 4, 8)
+    with pytest.raises(ValueError, match="k: expected shape"):
+        sl.decode_masked(qd, k[:, :, :, :32].contiguous(), v, pre, idx, S, 4, 8)
+    with pytest.raises(ValueError, match="lse: expected shape"):
+        sl.decode_masked(qd, k, v, pre, idx, S, 4, 8, lse=torch.zeros((B, Hq, 1), dtype=f32))
+
+    with pytest.raises(ValueError, match=cuda_msg):
+        sl.build_index(fl)
+    with pytest.raises(TypeError, match="is_sep:"):
+        sl.build_index(fl.int())
+    with pytest.raises(ValueError, match="is_sep: expected 2"):
+        sl.build_index(fl[0])
+    with pytest.raises(ValueError, match="prefix: expected shape"):
+        sl.build_index(fl, out=(idx, idx, torch.zeros((B,), dtype=i32)))
+    ids = torch.zeros((B, S), dtype=i32)
+    with pytest.raises(TypeError, match="ids:"):
+        sl.flags_from_ids(ids.long(), [1, 2])
+    with pytest.raises(TypeError, match="ids:"):
+        sl.build_index_from_ids(ids.long(), [1, 2])
+    with pytest.raises(ValueError, match=cuda_msg):
+        sl.build_index_from_ids(ids, [1, 2])
+    with pytest.raises(TypeError, match="prefix:"):
+        sl.count_pairs(pre.long(), 4, 8)
+    with pytest.raises(TypeError, match="out:"):
+        sl.count_pairs(pre, 4, 8, out=torch.zeros((B,), dtype=i32))
