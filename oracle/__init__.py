@@ -81,6 +81,13 @@ def _elems(x):
     raise TypeError(x.dtype)
 
 
+def _shape(name, a, shape):
+    """The C routines take bare pointers: every array must have the layout
+    its sizes imply."""
+    if tuple(a.shape) != tuple(shape):
+        raise ValueError("%s: expected shape %s, got %s" % (name, tuple(shape), tuple(a.shape)))
+
+
 def flags_from_ids(ids: np.ndarray, sep_ids) -> np.ndarray:
     ids = np.ascontiguousarray(ids, dtype=np.int32)
     sep = np.ascontiguousarray(np.asarray(sep_ids, dtype=np.int32))
@@ -124,6 +131,9 @@ def prefill_rows(q, k, v, is_sep, a: int, n: int, rows=None, scale: float = 0.0,
     B, Hq, S, D = qa.shape
     Hkv = ka.shape[1]
     f = np.ascontiguousarray(is_sep, dtype=np.uint8)
+    _shape("k", ka, (B, Hkv, S, D))
+    _shape("v", va, (B, Hkv, S, D))
+    _shape("is_sep", f, (B, S))
     if rows is None:
         rows = np.arange(B * Hq * S, dtype=np.int64)
     rows = np.ascontiguousarray(rows, dtype=np.int64)
@@ -154,6 +164,8 @@ def attend(q, k, v, scale: float = 0.0):
     assert dq == dk == dv
     Hq, D = qa.shape
     Hkv, L, _ = ka.shape
+    _shape("k", ka, (Hkv, L, D))
+    _shape("v", va, (Hkv, L, D))
     out = np.zeros((Hq, D), dtype=np.float64)
     lse = np.zeros((Hq,), dtype=np.float64)
     rc = _lib().oracle_attend(_ptr(qa), _ptr(ka), _ptr(va), dq, Hq, Hkv, L, D, float(scale),
@@ -262,6 +274,10 @@ def prefill_backward(q, k, v, dout, is_sep, a: int, n: int, scale: float = 0.0,
     B, Hq, S, D = qa.shape
     Hkv = ka.shape[1]
     f = np.ascontiguousarray(is_sep, dtype=np.uint8)
+    _shape("k", ka, (B, Hkv, S, D))
+    _shape("v", va, (B, Hkv, S, D))
+    _shape("dout", oa, (B, Hq, S, D))
+    _shape("is_sep", f, (B, S))
     gq = np.zeros((B, Hq, S, D), dtype=np.float64)
     gk = np.zeros((B, Hkv, S, D), dtype=np.float64)
     gv = np.zeros((B, Hkv, S, D), dtype=np.float64)

@@ -436,8 +436,24 @@ class SepCache:
     def rope_theta(self) -> float:
         return float(self.c.rope_theta)
 
+    # layout checks of the per-token tensors (the library reads B * Hkv rows
+    # of D elements in the cache dtype, B flags and B * Hq query rows)
+    def _check_new(self, k_new, v_new, is_sep_new):
+        shape = (self.B, self.Hkv, self.D)
+        _expect(k_new, "k_new", self.dtype, shape)
+        _expect(v_new, "v_new", self.dtype, shape)
+        _expect(is_sep_new, "is_sep_new", torch.uint8, (self.B,))
+
+    def _check_query(self, q, out, lse) -> int:
+        Hq = _dims(q, "q", 3)[1]
+        _expect(q, "q", self.dtype, (self.B, Hq, self.D))
+        _expect(out, "out", self.dtype, (self.B, Hq, self.D))
+        _expect(lse, "lse", torch.float32, (self.B, Hq))
+        return Hq
+
     def append(self, layer: int, k_new, v_new, is_sep_new=None, stream=None):
-        _need_cuda(k_new, v_new, is_sep_new)
+        self._check_new(k_new, v_new, is_sep_new)
+        _need_cuda(k_new, v_new, is_sep_new, self.buffer)
         _check("sepcache_append", _lib.sepcache_append(
             ctypes.byref(self.c), layer, _ptr(k_new), _ptr(v_new), _ptr(is_sep_new),
             _stream(stream)))
@@ -450,13 +466,13 @@ class SepCache:
         """Put a prompt's T tokens into this (empty) cache at `layer`: k, v
         [B, Hkv, T, D]; is_sep [B, T], prefix [B, T+1], idx [B, T] from
         build_index (read at layer 0).  Same result as T appends."""
-        _need_cuda(k, v, is_sep, prefix, idx)
-        if k.dim() != 4 or k.shape != v.shape or k.shape[0] != self.B or k.shape[1] != self.Hkv \
-                or k.shape[3] != self.D:
-            raise ValueError("k, v must be [B, Hkv, T, D] matching the cache")
-        if not (k.is_contiguous() and v.is_contiguous()):
-            raise ValueError("k, v must be contiguous")
-        T = int(k.shape[2])
+        T = _dims(k, "k", 4)[2]
+        _expect(k, "k", self.dtype, (self.B, self.Hkv, T, self.D))
+        _expect(v, "v", self.dtype, (self.B, self.Hkv, T, self.D))
+        _expect(is_sep, "is_sep", torch.uint8, (self.B, T))
+        _expect(prefix, "prefix", torch.int32, (self.B, T + 1))
+        _expect(idx, "idx", torch.int32, (self.B, T))
+        _need_cuda(k, v, is_sep, prefix, idx, self.buffer)
         _check("sepcache_ingest", _lib.sepcache_ingest(
             ctypes.byref(self.c), layer, _ptr(k), _ptr(v), _ptr(is_sep), _ptr(prefix), _ptr(idx), T,
             _stream(stream)))
@@ -471,8 +487,9 @@ class SepCache:
 
     def decode(self, layer: int, q, scale: float = 0.0, out=None, lse=None, want_lse=True,
                stream=None):
-        _need_cuda(q, out, lse)
-        B, Hq, D = q.shape
+        Hq = self._check_query(q, out, lse)
+        _need_cuda(q, out, lse, self.buffer)
+        B = self.B
         if out is None:
             out = torch.empty_like(q)
         if lse is None and want_lse:
@@ -487,8 +504,10 @@ class SepCache:
                     out=None, lse=None, want_lse=True, stream=None):
         """append + compact + decode of one layer in one launch (plus the
         layer-0 bookkeeping launch)."""
-        _need_cuda(q, k_new, v_new, is_sep_new, out, lse)
-        B, Hq, D = q.shape
+        Hq = self._check_query(q, out, lse)
+        self._check_new(k_new, v_new, is_sep_new)
+        _need_cuda(q, k_new, v_new, is_sep_new, out, lse, self.buffer)
+        B = self.B
         if out is None:
             out = torch.empty_like(q)
         if lse is None and want_lse:
@@ -503,8 +522,9 @@ class SepCache:
                        want_lse=True, stream=None):
         """decode() for callers that cannot allocate: no workspace; the
         library's fixed scratch holds the partials (see the header)."""
-        _need_cuda(q, out, lse)
-        B, Hq, D = q.shape
+        Hq = self._check_query(q, out, lse)
+        _need_cuda(q, out, lse, self.buffer)
+        B = self.B
         if out is None:
             out = torch.empty_like(q)
         if lse is None and want_lse:
