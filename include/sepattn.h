@@ -142,7 +142,11 @@ int sep_attn_prefill(const void* q, const void* k, const void* v, int dtype, con
  * prefill.  dtype SEP_BF16 only (fp32 accumulation; SEP_EDTYPE otherwise),
  * D in {64, 128}.  workspace: sep_attn_backward_workspace() bytes, 256-byte
  * aligned, contents arbitrary (the call clears what it needs); calls sharing
- * it must not overlap on the GPU.  Every output element is written. */
+ * it must not overlap on the GPU.  Every output element is written.  The
+ * call's five kernels overlap one another's set-up on the stream
+ * (programmatic launches), but its first launch starts only after earlier
+ * work on `stream` has completed, and its last one ends only after all of
+ * the call's work, so stream order holds as for any call. */
 size_t sep_attn_backward_workspace(int B, int Hq, int Hkv, int S, int D);
 int sep_attn_backward(const void* q, const void* k, const void* v, const void* out,
                       const float* lse, const void* dout, int dtype, const uint8_t* is_sep,
