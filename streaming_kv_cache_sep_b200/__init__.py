@@ -192,19 +192,17 @@ def build_index(is_sep: torch.Tensor, out=None, stream=None):
     """(prefix [B,S+1], idx [B,S] (-1 padded), count [B]) int32 on the device."""
     B, S = _dims(is_sep, "is_sep", 2)
     _expect(is_sep, "is_sep", torch.uint8, (B, S))
-    if out is not None:
-        prefix, idx, count = out
-        _expect(prefix, "prefix", torch.int32, (B, S + 1))
-        _expect(idx, "idx", torch.int32, (B, S))
-        _expect(count, "count", torch.int32, (B,))
-        _need_cuda(is_sep, prefix, idx, count)
-    _need_cuda(is_sep)
-    dev = is_sep.device
     if out is None:
+        _need_cuda(is_sep)
+        dev = is_sep.device
         out = (torch.empty((B, S + 1), dtype=torch.int32, device=dev),
                torch.empty((B, S), dtype=torch.int32, device=dev),
                torch.empty((B,), dtype=torch.int32, device=dev))
     prefix, idx, count = out
+    _expect(prefix, "prefix", torch.int32, (B, S + 1))
+    _expect(idx, "idx", torch.int32, (B, S))
+    _expect(count, "count", torch.int32, (B,))
+    _need_cuda(is_sep, prefix, idx, count)
     _check("sep_build_index", _lib.sep_build_index(_ptr(is_sep), B, S, _ptr(prefix), _ptr(idx),
                                                    _ptr(count), _stream(stream)))
     return prefix, idx, count
@@ -215,21 +213,19 @@ def build_index_from_ids(ids: torch.Tensor, sep_ids, out=None, stream=None):
     (is_sep uint8 [B,S], prefix [B,S+1], idx [B,S], count [B]) on the device."""
     B, S = _dims(ids, "ids", 2)
     _expect(ids, "ids", torch.int32, (B, S))
-    if out is not None:
-        is_sep, prefix, idx, count = out
-        _expect(is_sep, "is_sep", torch.uint8, (B, S))
-        _expect(prefix, "prefix", torch.int32, (B, S + 1))
-        _expect(idx, "idx", torch.int32, (B, S))
-        _expect(count, "count", torch.int32, (B,))
-        _need_cuda(ids, is_sep, prefix, idx, count)
-    _need_cuda(ids)
-    dev = ids.device
     if out is None:
+        _need_cuda(ids)
+        dev = ids.device
         out = (torch.empty((B, S), dtype=torch.uint8, device=dev),
                torch.empty((B, S + 1), dtype=torch.int32, device=dev),
                torch.empty((B, S), dtype=torch.int32, device=dev),
                torch.empty((B,), dtype=torch.int32, device=dev))
     is_sep, prefix, idx, count = out
+    _expect(is_sep, "is_sep", torch.uint8, (B, S))
+    _expect(prefix, "prefix", torch.int32, (B, S + 1))
+    _expect(idx, "idx", torch.int32, (B, S))
+    _expect(count, "count", torch.int32, (B,))
+    _need_cuda(ids, is_sep, prefix, idx, count)
     arr = (ctypes.c_int32 * len(sep_ids))(*[int(x) for x in sep_ids])
     _check("sep_build_index_from_ids", _lib.sep_build_index_from_ids(
         _ptr(ids), B, S, ctypes.cast(arr, ctypes.c_void_p), len(sep_ids), _ptr(is_sep),
